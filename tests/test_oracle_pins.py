@@ -1,0 +1,384 @@
+"""Pins for the CPU oracle: each check ties an oracle function to something other
+than itself -- the pages' printed numbers, closed forms of the formats, library
+casts, exact-rational brute force, round trips and exact integer arithmetic.
+
+Citations name "MXCode: Vector Quantization for MX-Native Inference at Scale"
+(the method's paper) by table or caption.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import mxcode_oracle as O
+from vector_quantized_mx_b200 import synth
+
+
+def _load(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+def bf16_bits(vals):
+    return torch.tensor(vals, dtype=torch.float64).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+# ---------------------------------------------------------------------------
+# Formats (Table 1)
+# ---------------------------------------------------------------------------
+
+def test_e2m1_values_match_bitfield_closed_form():
+    # E2M1: sign s, exponent e (2 bits, bias 1), mantissa m (1 bit); e = 0 is subnormal.
+    for c in range(16):
+        s, e, m = c >> 3, (c >> 1) & 3, c & 1
+        ref = (0.5 * m) if e == 0 else (2.0 ** (e - 1)) * (1 + m / 2)
+        ref = -ref if s else ref
+        assert O.e2m1_value(c) == ref
+
+
+def test_e8m0_scale_range_table1(golden_dir):
+    t1 = _load(golden_dir, "table1_formats.json")["formats"]["E8M0-B32-FP4"]
+    assert O.e8m0_value(0) == 2.0 ** t1["min_positive_scale_log2"]
+    mx = float(O.e8m0_value(254))
+    assert float(f"{mx:.2e}") == t1["max_finite_scale"]
+    # library decode: torch's float8_e8m0fnu cast, every non-NaN byte
+    b = np.arange(255, dtype=np.uint8)
+    lib = torch.from_numpy(b).view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    assert np.array_equal(O.e8m0_value(b), lib)
+    with pytest.raises(ValueError):
+        O.e8m0_value(255)
+
+
+def test_e4m3_decode_vs_torch_and_table1(golden_dir):
+    t1 = _load(golden_dir, "table1_formats.json")["formats"]["E4M3-B16-FP4"]
+    b = np.array([x for x in range(256) if x not in (0x7F, 0xFF)], dtype=np.uint8)
+    lib = torch.from_numpy(b).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(O.e4m3_value(b), lib)
+    pos = O.e4m3_value(np.arange(1, 127))
+    assert pos.min() == 2.0 ** t1["min_positive_scale_log2"]
+    assert pos.max() == t1["max_finite_scale"]
+
+
+def test_e4m3_encode_vs_torch_cast():
+    rng = np.random.default_rng(7)
+    vals = list(rng.uniform(0, 448, 20000).astype(np.float32))
+    vals += list((rng.uniform(0, 2.0 ** -6, 5000)).astype(np.float32))  # subnormal range
+    grid = O.e4m3_value(np.arange(0, 127))
+    mids = ((grid[1:] + grid[:-1]) / 2).astype(np.float32)                # exact ties
+    assert np.array_equal(mids.astype(np.float64), (grid[1:] + grid[:-1]) / 2)
+    vals += list(mids) + list(grid.astype(np.float32))
+    v = np.array(vals, dtype=np.float32)
+    lib = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_encode_rne_satfinite(v.astype(np.float64)), lib)
+
+
+def test_e4m3_encode_saturates_at_table1_max():
+    big = np.array([448.0, 449.0, 464.0, 465.0, 1e6, np.inf])
+    assert np.all(O.e4m3_encode_rne_satfinite(big) == 0x7E)
+
+
+def test_bf16_decode_vs_torch():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    lib = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    ok = ~np.isnan(lib)
+    assert np.array_equal(O.bf16_value(bits)[ok], lib[ok])
+
+
+# ---------------------------------------------------------------------------
+# E2M1 round-to-nearest-even: exact rational brute force + worked examples
+# ---------------------------------------------------------------------------
+
+_E2M1_FR = [Fraction(0), Fraction(1, 2), Fraction(1), Fraction(3, 2), Fraction(2), Fraction(3), Fraction(4), Fraction(6)]
+
+
+def _rne_e2m1_fraction(q: Fraction) -> int:
+    """Nearest E2M1 magnitude by exact rational distance; a tie keeps the code whose mantissa bit is 0."""
+    q = abs(q)
+    best = None
+    for c, v in enumerate(_E2M1_FR):
+        d = abs(q - v)
+        if best is None or d < best[0] or (d == best[0] and (c & 1) == 0):
+            best = (d, c)
+    return best[1]
+
+
+def test_e2m1_rne_worked_examples(golden_dir):
+    for ex in _load(golden_dir, "act_quant_worked_examples.json")["e2m1_rne"]:
+        assert int(O.e2m1_encode_rne(ex["q"])) == ex["code"], ex
+
+
+def test_e2m1_rne_bruteforce_rational():
+    qs = [Fraction(i, 64) for i in range(0, 64 * 9)]
+    qs += [Fraction(v) for v in (1e-30, 5.999999, 6.000001, 1e9)]
+    got = O.e2m1_encode_rne(np.array([float(q) for q in qs]))
+    ref = [_rne_e2m1_fraction(q) for q in qs]
+    assert list(got) == ref
+
+
+# ---------------------------------------------------------------------------
+# Activation quantization
+# ---------------------------------------------------------------------------
+
+def test_e8m0_act_quant_worked_examples(golden_dir):
+    for ex in _load(golden_dir, "act_quant_worked_examples.json")["e8m0_blocks"]:
+        x = np.zeros((1, 32))
+        x[0, 0] = ex["block_amax_element"]
+        codes, sf = O.quantize_act_e8m0(bf16_bits(x))
+        assert int(sf[0, 0]) == ex["scale_byte"], ex
+        assert int(codes[0, 0]) == ex["code"], ex
+
+
+def test_e8m0_act_quant_every_bf16_amax():
+    """Every finite BF16 value v as a block's amax element (with a companion
+    element w = v * 0.37 rounded to BF16).  Independent characterisation of the
+    OCP MX shared scale: the exponent e is the unique integer with
+    |v| / 2^e in [4, 8), clamped to [-127, 127]; codes by exact rational RNE."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = O.bf16_value(bits)
+    keep = np.isfinite(vals) & (vals != 0)
+    bits, vals = bits[keep], vals[keep]
+    comp = bf16_bits(vals * 0.37)
+    x = np.zeros((len(bits), 32), dtype=np.uint16)
+    x[:, 0] = bits
+    x[:, 5] = comp
+    codes, sf = O.quantize_act_e8m0(x)
+    compv = O.bf16_value(comp)
+    for i in range(0, len(bits), 7):   # every 7th value keeps the loop at a few seconds
+        v = Fraction(float(vals[i]))
+        e = 0
+        while abs(v) / Fraction(2) ** e >= 8:
+            e += 1
+        while abs(v) / Fraction(2) ** e < 4:
+            e -= 1
+        e = max(-127, min(127, e))
+        assert int(sf[i, 0]) == e + 127
+        for col, val in ((0, v), (5, Fraction(float(compv[i])))):
+            mag = _rne_e2m1_fraction(val / Fraction(2) ** e)
+            sign = 8 if (val < 0 or (val == 0 and np.signbit(O.bf16_value(x[i, col])))) else 0
+            assert int(codes[i, col]) == (mag | sign), (i, col)
+
+
+def test_e8m0_all_zero_block_and_signed_zero():
+    x = bf16_bits(np.array([[0.0] * 16 + [-0.0] * 16]))
+    codes, sf = O.quantize_act_e8m0(x)
+    assert sf[0, 0] == 0
+    assert list(codes[0, :16]) == [0] * 16 and list(codes[0, 16:]) == [8] * 16
+
+
+def test_e4m3_act_quant_worked_examples(golden_dir):
+    for ex in _load(golden_dir, "act_quant_worked_examples.json")["e4m3_blocks"]:
+        x = np.zeros((1, 32))
+        x[0, 16] = ex["tensor_amax"]          # second block carries the tensor amax
+        x[0, :len(ex["block"])] = ex["block"]
+        codes, sf, s = O.quantize_act_e4m3(bf16_bits(x))
+        assert s == np.float32(ex["tensor_amax"]) / np.float32(2688)
+        assert int(sf[0, 0]) == ex["scale_byte"], ex
+        assert list(codes[0, :len(ex["block"])]) == ex["codes"], ex
+
+
+def test_e4m3_act_quant_fp32_recipe_and_exact_codes():
+    """Scale steps against torch's FP32 arithmetic; code decisions against exact rationals."""
+    w, _ = synth.config2(16)
+    x = synth.config2(16)[1]
+    codes, sf, s = O.quantize_act_e4m3(x)
+    xt = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).float()
+    amax_t = xt.abs().max()
+    assert s == (amax_t / 2688.0).item()
+    blocks = xt.reshape(16, -1, 16)
+    t = (blocks.abs().amax(dim=2) / 6.0) / torch.tensor(s, dtype=torch.float32)
+    sb_lib = t.clamp(max=448.0).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(sf, sb_lib)
+    denom = (torch.from_numpy(sf).view(torch.float8_e4m3fn).float() * torch.tensor(s, dtype=torch.float32)).numpy()
+    rng = np.random.default_rng(3)
+    xv = O.bf16_value(x)
+    for _ in range(3000):
+        m, kb, j = rng.integers(16), rng.integers(4096 // 16), rng.integers(16)
+        val = Fraction(float(xv[m, kb * 16 + j]))
+        d = Fraction(float(denom[m, kb]))
+        mag = 0 if d == 0 else _rne_e2m1_fraction(val / d)
+        assert int(codes[m, kb * 16 + j]) == (mag | (8 if np.signbit(xv[m, kb * 16 + j]) else 0))
+
+
+def test_e4m3_zero_scale_block_gives_zero_codes():
+    # tensor amax huge, one tiny block: amax_b/6/s underflows E4M3 -> scale byte 0 -> codes +-0
+    x = np.zeros((1, 32))
+    x[0, 16] = 3.0e38
+    x[0, 0], x[0, 1] = 1e-3, -1e-3
+    codes, sf, s = O.quantize_act_e4m3(bf16_bits(x))
+    assert sf[0, 0] == 0
+    assert codes[0, 0] == 0 and codes[0, 1] == 8
+
+
+def test_fp4_packing_low_nibble_first():
+    codes = np.array([[1, 2, 0xF, 0x8]], dtype=np.uint8)
+    p = O.pack_fp4(codes)
+    assert list(p[0]) == [0x21, 0x8F]
+    assert np.array_equal(O.unpack_fp4(p), codes)
+
+
+# ---------------------------------------------------------------------------
+# Weight reconstruction: round trips through an encoder written here
+# ---------------------------------------------------------------------------
+
+def _encode_vq(target_codes, qn, qk):
+    """Trivial exact VQ: per QBlock, the distinct 4-vectors become the codebook."""
+    N, K = target_codes.shape
+    idx = np.zeros((N, K // 4), dtype=np.uint8)
+    cb = np.zeros((N // qn, K // qk, 256), dtype=np.uint16)
+    for a in range(N // qn):
+        for b in range(K // qk):
+            blk = target_codes[a * qn:(a + 1) * qn, b * qk:(b + 1) * qk].reshape(qn, qk // 4, 4)
+            keys = [tuple(int(c) for c in v) for v in blk.reshape(-1, 4)]
+            table = sorted(set(keys))
+            assert len(table) <= 256
+            pos = {t: i for i, t in enumerate(table)}
+            for i, t in enumerate(table):
+                cb[a, b, i] = t[0] | (t[1] << 4) | (t[2] << 8) | (t[3] << 12)
+            idx[a * qn:(a + 1) * qn, b * qk // 4:(b + 1) * qk // 4] = \
+                np.array([pos[k] for k in keys], dtype=np.uint8).reshape(qn, qk // 4)
+    return idx, cb
+
+
+@pytest.mark.parametrize("qn,qk", [(8, 16), (16, 32), (32, 64)])
+def test_weight_codes_round_trip(qn, qk):
+    rng = np.random.default_rng(qn * 100 + qk)
+    N, K = 64, 128
+    target = np.zeros((N, K), dtype=np.uint8)
+    for a in range(N // qn):
+        for b in range(K // qk):
+            palette = rng.integers(0, 16, size=(200, 4), dtype=np.uint8)
+            pick = rng.integers(0, 200, size=(qn, qk // 4))
+            target[a * qn:(a + 1) * qn, b * qk:(b + 1) * qk] = palette[pick].reshape(qn, qk)
+    idx, cb = _encode_vq(target, qn, qk)
+    w = synth.VQWeight("e8m0_b32", "prescale", N, K, qn, qk, idx, cb,
+                       np.full((N, K // 32), 127, np.uint8), None, None, 1.0)
+    assert np.array_equal(O.weight_codes(w), target)
+
+
+@pytest.mark.parametrize("fmt", ["e8m0_b32", "e4m3_b16"])
+def test_scale_vq_round_trip(fmt):
+    rng = np.random.default_rng(11)
+    B = O.BLOCK[fmt]
+    N, K = 48, 8 * B * 6
+    palette = rng.integers(100, 140, size=(256, 8), dtype=np.uint8)
+    groups = rng.integers(0, 256, size=(N, K // (8 * B)))
+    target = palette[groups].reshape(N, K // B)
+    table, inv = np.unique(target.reshape(-1, 8), axis=0, return_inverse=True)
+    scb = np.zeros((256, 8), dtype=np.uint8)
+    scb[:len(table)] = table
+    sidx = inv.reshape(N, K // (8 * B)).astype(np.uint8)
+    w = synth.VQWeight(fmt, "prescale_plus", N, K, N, K, np.zeros((N, K // 4), np.uint8),
+                       np.zeros((1, 1, 256), np.uint16), None, sidx, scb, 1.0)
+    assert np.array_equal(O.weight_scale_bytes(w), target)
+
+
+# ---------------------------------------------------------------------------
+# GEMM: exact integer special case and exact rationals
+# ---------------------------------------------------------------------------
+
+def test_linear_integer_special_case():
+    """Block scales 2^-1 everywhere: 4*a and 4*w are integers (2 x E2M1 values),
+    so 16*Y must equal an exact int64 matmul."""
+    rng = np.random.default_rng(5)
+    M, N, K = 24, 40, 256
+    ca = rng.integers(0, 16, size=(M, K), dtype=np.uint8)
+    cw = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    a_hat = O.dequant_act(ca, np.full((M, K // 32), 126, np.uint8), "e8m0_b32", 1.0)
+    idx, cb = _encode_vq(cw, 8, 32)
+    w = synth.VQWeight("e8m0_b32", "prescale", N, K, 8, 32, idx, cb,
+                       np.full((N, K // 32), 126, np.uint8), None, None, 1.0)
+    w_hat = O.dequant_weight(w)
+    two = np.array([0, 1, 2, 3, 4, 6, 8, 12], dtype=np.int64)
+    ia = np.where(ca & 8, -two[ca & 7], two[ca & 7])
+    iw = np.where(cw & 8, -two[cw & 7], two[cw & 7])
+    exact = ia @ iw.T
+    assert np.array_equal((16 * O.linear(a_hat, w_hat)).astype(np.int64), exact)
+    assert np.all(16 * O.linear(a_hat, w_hat) == exact)
+
+
+def test_w4a4_linear_exact_rationals_tiny():
+    """A 4 x 8 x 64 E4M3 case summed with exact fractions."""
+    rng = np.random.default_rng(9)
+    x = bf16_bits(rng.normal(size=(4, 64)))
+    w = synth.make_weight(123, "e4m3_b16", "prescale", 8, 64, 0, 0)
+    y, sabs = O.w4a4_linear(x, w)
+    codes, sf, s = O.quantize_act_e4m3(x)
+    a = O.dequant_act(codes, sf, "e4m3_b16", s)
+    wh = O.dequant_weight(w)
+    for m in range(4):
+        for n in range(8):
+            exact = sum(Fraction(float(a[m, k])) * Fraction(float(wh[n, k])) for k in range(64))
+            assert abs(Fraction(float(y[m, n])) - exact) <= Fraction(2) ** -45 * max(1, abs(exact))
+
+
+def test_checksums_linearity():
+    rng = np.random.default_rng(2)
+    a = rng.normal(size=(33, 70))
+    w = rng.normal(size=(21, 70))
+    y = O.linear(a, w)
+    row, col, abs_row, abs_col = O.checksums(a, w)
+    assert np.allclose(row, y.sum(axis=1), rtol=0, atol=1e-10)
+    assert np.allclose(col, y.sum(axis=0), rtol=0, atol=1e-10)
+    assert np.allclose(abs_row, O.abs_linear(a, w).sum(axis=1))
+    assert np.allclose(abs_col, O.abs_linear(a, w).sum(axis=0))
+
+
+# ---------------------------------------------------------------------------
+# Storage accounting vs the pages' BPE numbers (Table 1, Table 2, Table 4 caption)
+# ---------------------------------------------------------------------------
+
+def test_bpe_native_table1_table2(golden_dir):
+    t1 = _load(golden_dir, "table1_formats.json")["formats"]
+    t2 = _load(golden_dir, "table2_bpe.json")["values"]
+    assert O.native_bits_per_weight("e8m0_b32") == t1["E8M0-B32-FP4"]["bpe"] == t2["E8M0-B32-FP4"]["native"]
+    assert O.native_bits_per_weight("e4m3_b16") == t1["E4M3-B16-FP4"]["bpe"] == t2["E4M3-B16-FP4"]["native"]
+
+
+def test_bpe_mxcode_table2(golden_dir):
+    g = _load(golden_dir, "table2_bpe.json")
+    N, K = g["readings"]["prescale_plus_tensor_shape"]
+    for name, fmt in (("E4M3-B16-FP4", "e4m3_b16"), ("E8M0-B32-FP4", "e8m0_b32")):
+        r = g["readings"][name]
+        for strat in ("postscale", "prescale", "prescale_plus"):
+            bpw = O.bits_per_weight(fmt, strat, N, K, r["qblock"], r["qblock"],
+                                    postscale_block_scales=r["postscale_block_scales"])
+            assert round(bpw, 2) == g["values"][name][strat], (name, strat, bpw)
+
+
+def test_index_bits_table4_caption(golden_dir):
+    g = _load(golden_dir, "table2_bpe.json")["index_bits_per_weight"]
+    # a full-tensor codebook on a large tensor leaves only the index bits (+ direct scales)
+    bpw = O.bits_per_weight("e8m0_b32", "postscale", 1 << 20, 1 << 20, 0, 0, postscale_block_scales=False)
+    assert abs(bpw - g["value"]) < 1e-6
+
+
+def test_storage_bytes_matches_bpe():
+    w = synth.make_weight(1, "e4m3_b16", "prescale", 512, 1024, 256, 256)
+    assert O.storage_bytes(w) * 8 / (512 * 1024) == pytest.approx(
+        O.bits_per_weight("e4m3_b16", "prescale", 512, 1024, 256, 256))
+
+
+# ---------------------------------------------------------------------------
+# Generator sanity (closed forms of the sampling distributions)
+# ---------------------------------------------------------------------------
+
+def test_zipf_routing_first_choice_matches_closed_form():
+    row_tok, off = synth.config4_routing()
+    assert off[-1] == synth.MOE_TOKENS * synth.MOE_TOPK and np.all(np.diff(off) >= 0)
+    # every token appears top_k times with distinct experts
+    exp_of_row = np.repeat(np.arange(synth.MOE_EXPERTS), np.diff(off))
+    pairs = set(zip(row_tok.tolist(), exp_of_row.tolist()))
+    assert len(pairs) == synth.MOE_TOKENS * synth.MOE_TOPK
+    # Gumbel-max: the arg-max choice follows p_i = i^-s / H exactly
+    rng = synth.stream(99, "route")
+    E, s, T = 128, 1.1, 200000
+    logp = -s * np.log(np.arange(1, E + 1))
+    first = np.argmax(logp[None, :] + rng.gumbel(size=(T, E)), axis=1)
+    H = sum(i ** -s for i in range(1, E + 1))
+    p1 = 1 / H
+    assert abs(H - 4.431) < 5e-3
+    assert abs(np.mean(first == 0) - p1) < 4 * math.sqrt(p1 * (1 - p1) / T)
