@@ -1,0 +1,387 @@
+"""Benchmark of the MXCode W4A4 hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--m 16]
+
+Workload: the decode GEMV shaped like a fused QKV projection -- PostScale,
+E4M3-B16-FP4, K_in = 4096, N_out = 9216, M = 16 tokens, one FP4 codebook per
+256 x 256 QBlock (synthetic, seeded; see vector_quantized_mx_b200/synth.py).
+One step = one pass of the whole path over one batch: activation tensor amax,
+BF16 -> FP4 activation quantization, and the split-K W4A4 linear layer that
+decodes the VQ weights on the fly.  Steps are captured in a CUDA graph and
+rotate over 12 copies of the packed weights (145 MB > 126 MB L2), so every
+step streams its weights from HBM.
+
+Metric: effective weight bandwidth -- compressed weight bytes consumed per
+second (GB/s), whole job over all ranks.  Extra keys report TFLOPS, the
+roofline of the dominant kernel, the same step with native FP4 weights
+(4.50 bits/weight) on the same decoded values, the oracle on the host cores,
+and the end-to-end number through the Python API with host buffers.
+
+--impl reference times the CPU oracle (oracle/) on a bounded sample of the
+same workload (a slice of the output channels per step).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "decode GEMV (fused-QKV shape): PostScale E4M3-B16-FP4, M=16, K=4096, N=9216, 256x256 QBlocks"
+N_COPIES = 12
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled while the timed region runs
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU legs (oracle)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(w, x, rows: slice):
+    """The oracle on a slice of output channels: (seconds, weight bytes consumed)."""
+    from oracle import mxcode_oracle as O
+    t0 = time.perf_counter()
+    sub = type(w)(w.fmt, w.strategy, rows.stop - rows.start, w.K, w.qn, w.qk, w.idx[rows],
+                  w.cb[rows.start // w.qn:rows.stop // w.qn], w.scales[rows], None, None, w.w_tscale)
+    O.w4a4_linear(x, sub)
+    dt = time.perf_counter() - t0
+    return dt, O.storage_bytes(sub)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, x, budget_s=12.0):
+    rows_per = 1152           # 1/8 of N_out per sample
+    t_tot, b_tot, n = 0.0, 0, 0
+    while t_tot < budget_s and n < 8:
+        r0 = (n * rows_per) % w.N
+        dt, b = oracle_sample(w, x, slice(r0, r0 + rows_per))
+        t_tot += dt
+        b_tot += b
+        n += 1
+    return {"value": b_tot / t_tot / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} oracle calls, each M=16 x K=4096 over {rows_per} of the 9216 output channels "
+                      f"(FP64 dequant + activation quant + FP64 GEMM), {t_tot:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    from vector_quantized_mx_b200 import synth
+    if rank != 0:
+        return
+    w, x = synth.config2(args.m)
+    rows_per = 1152
+    for i in range(args.warmup):
+        oracle_sample(w, x, slice((i * rows_per) % w.N, (i * rows_per) % w.N + rows_per))
+    t0 = time.perf_counter()
+    b = 0
+    for i in range(args.steps):
+        r0 = (i * rows_per) % w.N
+        _, bb = oracle_sample(w, x, slice(r0, r0 + rows_per))
+        b += bb
+    dt = time.perf_counter() - t0
+    v = b / dt / 1e9
+    out = {"impl": "reference", "metric": "MXCode W4A4 effective weight bandwidth (compressed bytes/s)",
+           "value": v, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": WORKLOAD, "M": args.m, "K": 4096, "N": 9216,
+                      "sample": f"{rows_per} of 9216 output channels per step"},
+           "cpu_baseline": {"value": v, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                            "sample": f"{rows_per} of 9216 output channels per step, M={args.m}"},
+           "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU leg
+# ---------------------------------------------------------------------------
+
+def run_gpu(args, rank, world, dist):
+    import torch
+    from vector_quantized_mx_b200 import build, mxc, synth
+
+    build.build()
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    M = args.m
+    w, x = synth.config2(M)
+    # weights: N_COPIES packed copies (identical values, distinct buffers)
+    pw0 = mxc.pack_weight(w, device=dev)
+    copies = [pw0] + [mxc.PackedWeight(pw0.fmt, pw0.strategy, pw0.N, pw0.K, pw0.qn, pw0.qk, pw0.idx.clone(),
+                                       pw0.cb.clone(), pw0.scales.clone(), None, None, pw0.w_tscale)
+                      for _ in range(N_COPIES - 1)]
+    wbytes = pw0.storage_bytes()
+    x_host = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    x_dev = x_host.to(dev)
+    act = mxc.empty_act(M, w.K, w.fmt, dev)
+    qws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    lws = mxc.linear_workspace(M, w.N, w.K, w.fmt, dev)
+    y = torch.empty((M, w.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i):
+        mxc.quantize_act(x_dev, w.fmt, out=act, ws=qws, stream=stream)
+        mxc.linear(act, copies[i % N_COPIES], y=y, ws=lws, stream=stream)
+
+    # correctness gate before timing: one step against the oracle on a slice
+    with torch.cuda.stream(stream):
+        step(0)
+    stream.synchronize()
+    assert mxc.get_device_error(stream) == 0
+    from oracle import mxcode_oracle as O
+    sub = slice(0, 256)
+    subw = type(w)(w.fmt, w.strategy, 256, w.K, w.qn, w.qk, w.idx[sub], w.cb[:1], w.scales[sub], None, None,
+                   w.w_tscale)
+    ref, sabs = O.w4a4_linear(x, subw)
+    got = y[:, :256].cpu().numpy()
+    if not np.all(np.abs(got - ref) <= 1e-4 * sabs):
+        raise SystemExit("bench: GPU result does not match the oracle")
+
+    def capture(n_steps, fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            fn(0)                                   # warm the launch path outside capture
+            stream.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n_steps):
+                    fn(i)
+        return g
+
+    def time_graph(g):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        g.replay()
+        end.record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        ms = start.elapsed_time(end)
+        if dist is not None:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = t.item()
+        return ms
+
+    steps, warmup = args.steps, args.warmup
+    g_warm = capture(max(warmup, 1), step)
+    g_main = capture(steps, step)
+    g_warm.replay()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    ms = time_graph(g_main)
+    clocks = sampler.stop()
+    ms_step = ms / steps
+    value = world * wbytes / (ms_step * 1e-3) / 1e9
+    flops = 2.0 * M * w.K * w.N
+    tflops = world * flops / (ms_step * 1e-3) / 1e12
+
+    # dominant kernel alone: the linear layer, back to back over the rotating copies
+    def lin_only(i):
+        mxc.linear(act, copies[i % N_COPIES], y=y, ws=lws, stream=stream)
+    g_lin = capture(steps, lin_only)
+    g_lin.replay()
+    ms_lin = time_graph(g_lin) / steps
+    a_bytes = M * w.K // 2 + M * w.K // 16
+    alg_bytes = wbytes + a_bytes + M * w.N * 4
+    hbm_peak, peak_kind = peaks()
+    achieved = alg_bytes / (ms_lin * 1e-3) / 1e9
+
+    # native FP4 on the same decoded values (4.50 bits/weight), same rotation
+    nat0 = mxc.decode_weight(pw0)
+    nats = [nat0] + [mxc.MXTensor(nat0.q.clone(), nat0.sf.clone(), nat0.tscale.clone(), nat0.rows, nat0.K, nat0.fmt)
+                     for _ in range(N_COPIES - 1)]
+    with torch.cuda.stream(stream):
+        yn = mxc.native_linear(act, nats[0], stream=stream)
+    stream.synchronize()
+    y_ref = torch.empty_like(y)
+    with torch.cuda.stream(stream):
+        mxc.linear(act, pw0, y=y_ref, ws=lws, stream=stream)
+    stream.synchronize()
+    same = bool(torch.equal(yn, y_ref))
+
+    def nat_step(i):
+        mxc.quantize_act(x_dev, w.fmt, out=act, ws=qws, stream=stream)
+        mxc.native_linear(act, nats[i % N_COPIES], y=y, ws=lws, stream=stream)
+    g_nat = capture(steps, nat_step)
+    g_nat.replay()
+    ms_nat = time_graph(g_nat) / steps
+    nat_bytes = w.N * w.K // 2 + w.N * w.K // 16
+
+    # end to end through the Python API with host buffers (pinned), no graph
+    y_host = torch.empty((M, w.N), dtype=torch.float32).pin_memory()
+
+    def e2e_step(i):
+        x_dev.copy_(x_host, non_blocking=True)
+        mxc.quantize_act(x_dev, w.fmt, out=act, ws=qws, stream=stream)
+        mxc.linear(act, copies[i % N_COPIES], y=y, ws=lws, stream=stream)
+        y_host.copy_(y, non_blocking=True)
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for i in range(steps):
+            e2e_step(i)
+        s1.record(stream)
+        torch.cuda.synchronize()
+    ms_e2e = s0.elapsed_time(s1) / steps
+    if dist is not None:
+        t = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = t.item()
+
+    if rank != 0:
+        return
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        try:
+            with open(prof) as f:
+                traffic = json.load(f).get("decode_gemv_m16_bytes_per_launch")
+        except Exception:
+            traffic = None
+    out = {
+        "metric": "MXCode W4A4 effective weight bandwidth (compressed bytes/s)",
+        "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e2m1 x e2m1 -> f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M, "K": w.K, "N": w.N, "bits_per_weight": wbytes * 8 / (w.N * w.K),
+                   "l2": f"rotating {N_COPIES} weight copies ({N_COPIES * wbytes / 1e6:.0f} MB > 126 MB L2)",
+                   "parallelism": f"replicas x{world}"},
+        "tflops": tflops,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": traffic, "peak_kind": peak_kind,
+                     "kernel": "gemm_kernel<E4M3, VQ direct, T=16> split-K decode",
+                     "ms_per_launch": ms_lin, "alg_bytes_per_launch": alg_bytes},
+        "native_fp4": {"ms_per_step": ms_nat, "weight_bytes": nat_bytes,
+                       "weight_GBps": world * nat_bytes / (ms_nat * 1e-3) / 1e9,
+                       "mxcode_speedup": ms_nat / ms_step, "bitwise_equal_outputs": same},
+        "e2e": {"value": world * wbytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": int(x_host.numel() * 2), "d2h_bytes_per_step": int(y_host.numel() * 4),
+                "ms_per_step": ms_e2e},
+        "gpu_launches": 3 * steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, x)
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="mxcode", choices=["mxcode", "reference"])
+    ap.add_argument("--m", type=int, default=16, choices=[1, 4, 16])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_gpu(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

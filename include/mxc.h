@@ -1,0 +1,256 @@
+/*
+ * mxc.h -- C ABI of the MXCode W4A4 linear-layer library for NVIDIA B200 (sm_100a).
+ *
+ * Method: "MXCode: Vector Quantization for MX-Native Inference at Scale".
+ * Weights are stored at about 2 bits each: a uint8 index per d=4 consecutive
+ * weights along the input-channel axis selects one of K=256 FP4 (E2M1)
+ * centroids of the weight's QBlock (abstract; Table 4 caption), and the
+ * centroid's codes are scaled by MX block scales (Table 1): E8M0 per 32
+ * weights, or E4M3 per 16 weights with an FP32 tensor scale.  PostScale and
+ * PreScale store the block scales directly; PreScale+ VQ-codes groups of 8
+ * scales with a 256-entry scale codebook (Table 4 caption).  The library
+ * decodes indices straight into MX-native FP4 operand tiles in shared memory
+ * and multiplies them with FP4-quantized activations on the tcgen05
+ * block-scaled tensor cores (W4A4, abstract and Table 2 caption); it never
+ * materialises BF16 weights.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Ownership: the caller allocates and owns every buffer and the stream.
+ *   The library keeps no allocation of its own apart from one 4-byte device
+ *   error word per device (a module global).  Pointers marked "device" must be
+ *   device memory of the current device; "host" pointers are host memory.
+ * - Asynchrony: GPU calls enqueue work on the given stream and return.  They
+ *   do not synchronize.  Argument, shape and alignment problems are reported
+ *   synchronously by the return value and nothing is enqueued.
+ * - Device-side problems (malformed MoE offsets, a pipeline wait that ran
+ *   out) set the device error word; read it with mxc_get_device_error().
+ * - No exception crosses this ABI; every entry point returns mxc_status.
+ * - Shapes: K (input channels) must be a multiple of 256, N (output channels)
+ *   a multiple of 128.  Buffers passed to the GPU must be 16-byte aligned.
+ *
+ * Layouts
+ * -------
+ * FP4 matrix  [R, K] as bytes [R, ld] (ld >= K/2, ld % 16 == 0): byte i of a
+ *             row holds elements 2i (low nibble) and 2i+1 (high nibble);
+ *             nibble = E2M1 code, bit 3 = sign.
+ * SF layout   block-scale bytes of an [R, K/B] scale matrix, grouped the way
+ *             the tcgen05 block-scaled MMA reads them: rows are padded to a
+ *             multiple of 128; byte (r, kb) sits at
+ *                 ((r/128) * (K/B/4) + kb/4) * 512
+ *               + (r%32) * 16 + ((r/32)%4) * 4 + (kb%4).
+ *             mxc_sf_bytes(R, K, fmt) gives the size.
+ * Packed VQ weight (mxc_pack_weight writes it; see mxc_weight below).
+ */
+#ifndef MXC_H_
+#define MXC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* mxc_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum mxc_status {
+  MXC_OK = 0,
+  MXC_ERR_INVALID_ARG = 1,    /* null pointer, bad enum, inconsistent shapes        */
+  MXC_ERR_UNSUPPORTED = 2,    /* e.g. the UE5M3 scale format, or M beyond limits    */
+  MXC_ERR_ALIGNMENT = 3,      /* K % 256, N % 128, QBlock sizes, 16-byte pointers   */
+  MXC_ERR_WORKSPACE = 4,      /* workspace missing or smaller than required         */
+  MXC_ERR_CUDA = 5,           /* a CUDA runtime/driver call failed                  */
+  MXC_ERR_DEVICE_INVALID = 6, /* device found malformed data (e.g. MoE offsets)     */
+  MXC_ERR_TIMEOUT = 7,        /* a bounded pipeline wait on the device expired      */
+  MXC_ERR_NO_DEVICE = 8       /* no sm_100 device is current                         */
+} mxc_status;
+
+/* Block-scaled FP4 formats (Table 1).  UE5M3-B16 has no native tensor-core
+ * path on this GPU and is rejected with MXC_ERR_UNSUPPORTED. */
+typedef enum mxc_format {
+  MXC_FMT_E8M0_B32 = 0, /* E8M0 scale per 32 elements, no tensor scale          */
+  MXC_FMT_E4M3_B16 = 1, /* E4M3 scale per 16 elements, FP32 tensor scale        */
+  MXC_FMT_UE5M3_B16 = 2 /* not supported                                        */
+} mxc_format;
+
+/* MXCode strategies (abstract).  PostScale and PreScale share one decode path
+ * (the pages' "shared Pre/PostScale FP4 projection backend", Figure 4 and
+ * Table 3 captions); the strategy only selects where block scales come from. */
+typedef enum mxc_strategy {
+  MXC_POSTSCALE = 0,     /* direct block scales                                */
+  MXC_PRESCALE = 1,      /* direct block scales                                */
+  MXC_PRESCALE_PLUS = 2  /* VQ-coded block scales (groups of 8, 256 entries)   */
+} mxc_strategy;
+
+typedef enum mxc_dtype { MXC_OUT_F32 = 0, MXC_OUT_BF16 = 1 } mxc_dtype;
+
+/* An MX-quantized matrix: FP4 codes + block scales (+ FP32 tensor scale).
+ * Activations are passed this way, and so are native-FP4 weights. */
+typedef struct mxc_mx_tensor {
+  const uint8_t* q;      /* device, FP4 matrix [rows, ldq bytes]                      */
+  const uint8_t* sf;     /* device, SF layout (see above) of the [rows, K/B] scales    */
+  const float* tscale;   /* device, one FP32 tensor scale; NULL means 1.0              */
+  int64_t rows;          /* M for activations, N for native weights                    */
+  int64_t K;             /* elements per row                                           */
+  int64_t ldq;           /* row stride of q in bytes                                   */
+  mxc_format fmt;
+} mxc_mx_tensor;
+
+/* A VQ-coded weight W[N, K] in the packed device layout.
+ *   idx     device, [N/128][K/256][128][64] bytes: for each 128-row x 256-column
+ *           tile, the tile's rows of uint8 indices (index j of row n covers
+ *           k = 4j..4j+3), 8 KB per tile, tiles in row-major tile order.
+ *   cb      device, [N/qn][K/qk][256] uint16 FP4 codebooks; centroid element t
+ *           (k mod 4) in bits 4t..4t+3.  512 bytes per QBlock.
+ *   scales  device (PostScale/PreScale), SF layout of the [N, K/B] scale bytes.
+ *   sidx    device (PreScale+), [N/128][K/256][128][256/(8B)] bytes: scale-codebook
+ *           index of each group of 8 consecutive scales along K.
+ *   scb     device (PreScale+), [256][8] scale bytes.
+ *   qn, qk  QBlock size; 0 means the whole dimension.  qn must be a multiple
+ *           of 128 (or N); qk must be 128 or a multiple of 256 (or K).
+ *   w_tscale  FP32 tensor scale (E4M3-B16); use 1.0 for E8M0-B32. */
+typedef struct mxc_weight {
+  mxc_strategy strategy;
+  mxc_format fmt;
+  int64_t N, K, qn, qk;
+  const uint8_t* idx;
+  const uint16_t* cb;
+  const uint8_t* scales;
+  const uint8_t* sidx;
+  const uint8_t* scb;
+  float w_tscale;
+} mxc_weight;
+
+/* The same weight in its logical host layout, as produced by a quantizer:
+ *   idx [N, K/4] uint8, cb [N/qn, K/qk, 256] uint16, scales [N, K/B] uint8
+ *   (direct) or sidx [N, K/(8B)] uint8 + scb [256, 8] uint8 (PreScale+). */
+typedef struct mxc_weight_host {
+  mxc_strategy strategy;
+  mxc_format fmt;
+  int64_t N, K, qn, qk;
+  const uint8_t* idx;
+  const uint16_t* cb;
+  const uint8_t* scales;
+  const uint8_t* sidx;
+  const uint8_t* scb;
+  float w_tscale;
+} mxc_weight_host;
+
+/* Byte sizes of the packed buffers (host-side arithmetic only). */
+typedef struct mxc_packed_sizes {
+  size_t idx, cb, scales, sidx, scb;
+} mxc_packed_sizes;
+
+/* ---- version / status ------------------------------------------------------------- */
+
+const char* mxc_status_string(mxc_status s);
+int mxc_version(void); /* 100 * major + minor */
+
+/* ---- host-side layout helpers (no GPU needed) ------------------------------------ */
+
+/* Bytes of an SF-layout buffer for an [rows, K/B] scale matrix (rows padded to 128). */
+size_t mxc_sf_bytes(int64_t rows, int64_t K, mxc_format fmt);
+
+/* Sizes of the packed buffers of a weight.  Returns MXC_ERR_* for bad shapes. */
+mxc_status mxc_packed_weight_sizes(const mxc_weight_host* w, mxc_packed_sizes* out);
+
+/* Reorders a logical host weight into the packed layout, host to host.
+ * idx_out, scales_out (direct) or sidx_out (PreScale+) must hold the sizes
+ * that mxc_packed_weight_sizes() reports; cb and scb are used as they are
+ * (their logical layout is already the packed one).  Unused outputs may be
+ * NULL.  Pure host code: safe without a GPU. */
+mxc_status mxc_pack_weight(const mxc_weight_host* w, uint8_t* idx_out, uint8_t* scales_out,
+                           uint8_t* sidx_out);
+
+/* Workspace bytes each GPU call needs (0 if none).  M = activation rows;
+ * for mxc_moe_linear M is the total number of (token, expert) rows. */
+size_t mxc_quantize_act_workspace_bytes(int64_t M, int64_t K, mxc_format fmt);
+size_t mxc_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, mxc_format fmt);
+size_t mxc_moe_workspace_bytes(int64_t M, int32_t E, int64_t N, int64_t K, mxc_format fmt);
+
+/* Rows of the SF layout that mxc_quantize_act_grouped writes:
+ * sum over groups of ceil(rows_g / 128) * 128, bounded by M + 128*E. */
+int64_t mxc_grouped_sf_rows_bound(int64_t M, int32_t E);
+
+/* ---- GPU calls ----------------------------------------------------------------------- */
+
+/* Activation MX quantization, BF16 -> FP4 codes + block scales (W4A4: abstract,
+ * Table 2 caption; formats: Table 1).  Rule (the pages give none; OCP MX):
+ *   E8M0-B32: per block of 32, e = floor(log2 amax) - 2 clamped to [-127,127]
+ *             (amax = 0 -> byte 0), codes = RNE_E2M1(x / 2^e) saturating at +-6.
+ *   E4M3-B16: s = amax_tensor / 2688 in FP32 (1 if amax = 0), unless
+ *             act_tscale_in gives it; per block of 16,
+ *             sb = E4M3_RNE_satfinite(fp32(fp32(amax/6) / s)),
+ *             codes = RNE_E2M1(x / fp32(sb * s)) decided exactly; sb = 0 -> +-0.
+ *   Signs are kept, so -0 becomes code 0x8.  NaN/Inf inputs are undefined.
+ * x_bf16        device, [M, ldx] BF16 elements (ldx >= K)
+ * act_tscale_in device FP32 or NULL (E4M3 only; ignored for E8M0)
+ * q_out         device, FP4 matrix [M, ldq] (ldq >= K/2, multiple of 16)
+ * sf_out        device, SF layout, mxc_sf_bytes(M, K, fmt) bytes; padding rows get 0
+ * act_tscale_out device FP32 (E4M3: receives s; may be NULL for E8M0)
+ * ws            device workspace of mxc_quantize_act_workspace_bytes() bytes */
+mxc_status mxc_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, mxc_format fmt,
+                            const float* act_tscale_in, uint8_t* q_out, int64_t ldq, uint8_t* sf_out,
+                            float* act_tscale_out, void* ws, size_t ws_bytes, mxc_stream_t stream);
+
+/* As mxc_quantize_act for rows sorted by group (MoE experts): row r belongs to
+ * group g when d_offsets[g] <= r < d_offsets[g+1].  q_out is dense [M, ldq];
+ * sf_out places each group's scale rows at the next multiple of 128 rows
+ * (mxc_grouped_sf_rows_bound(M, E) rows are enough), which is what
+ * mxc_moe_linear reads.  d_offsets is device int32 [E+1], offsets[0] = 0,
+ * non-decreasing, offsets[E] = M; violations set MXC_ERR_DEVICE_INVALID. */
+mxc_status mxc_quantize_act_grouped(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                                    mxc_format fmt, const int32_t* d_offsets, int32_t E,
+                                    const float* act_tscale_in, uint8_t* q_out, int64_t ldq,
+                                    uint8_t* sf_out, float* act_tscale_out, void* ws,
+                                    size_t ws_bytes, mxc_stream_t stream);
+
+/* MXCode W4A4 linear layer: y[M, N] = A[M, K] . W[N, K]^T, where A is the
+ * MX-quantized activation and W the VQ weight reconstructed on the fly
+ * (abstract: "reconstruct MX-native W4A4 operands without materializing
+ * intermediate high-precision weights").  Accumulation is FP32 on the tensor
+ * cores; y = acc * w_tscale * a_tscale, written as FP32 or BF16 (RNE).
+ * a         activation, a->fmt must equal w->fmt; a->rows = M; a->sf in SF layout
+ * w         packed VQ weight (device pointers inside)
+ * y         device, [M, ldy] elements of y_dtype (ldy >= N)
+ * ws        device workspace of mxc_linear_workspace_bytes() bytes
+ * M <= 16 takes the split-K decode path; larger M the tiled prefill path. */
+mxc_status mxc_linear(const mxc_mx_tensor* a, const mxc_weight* w, void* y, int64_t ldy,
+                      mxc_dtype y_dtype, void* ws, size_t ws_bytes, mxc_stream_t stream);
+
+/* Native block-scaled FP4 linear layer on the same pipeline, with the weight
+ * given as an MX tensor (w->rows = N): the "Native FP4" baseline of Table 2
+ * and Table 3.  Same output contract as mxc_linear. */
+mxc_status mxc_native_linear(const mxc_mx_tensor* a, const mxc_mx_tensor* w, void* y, int64_t ldy,
+                             mxc_dtype y_dtype, void* ws, size_t ws_bytes, mxc_stream_t stream);
+
+/* Grouped-expert (MoE) MXCode linear: rows of `a` are sorted by expert, expert e
+ * owning rows [d_offsets[e], d_offsets[e+1]); y[r, :] = A[r, :] . W_e^T.
+ * a         quantized with mxc_quantize_act_grouped (grouped SF layout)
+ * d_offsets device int32 [E+1] (validated on the device)
+ * experts   host array of E packed weights that share strategy, format, N, K,
+ *           qn, qk (their device pointers may differ); E <= 256
+ * y         device, [M, ldy]
+ * ws        device workspace of mxc_moe_workspace_bytes() bytes */
+mxc_status mxc_moe_linear(const mxc_mx_tensor* a, const int32_t* d_offsets, const mxc_weight* experts,
+                          int32_t E, void* y, int64_t ldy, mxc_dtype y_dtype, void* ws,
+                          size_t ws_bytes, mxc_stream_t stream);
+
+/* Runs the weight decode of mxc_linear (index -> codebook -> FP4 tile and
+ * scale decode, through shared memory) and writes the result out in plain
+ * layouts: q_out FP4 matrix [N, ldq], sf_out the SF layout of [N, K/B].
+ * Used to check the decode bit for bit and to build native-FP4 weights that
+ * hold exactly the same values. */
+mxc_status mxc_decode_weight(const mxc_weight* w, uint8_t* q_out, int64_t ldq, uint8_t* sf_out,
+                             mxc_stream_t stream);
+
+/* Waits for the stream, then reads and clears the device error word of the
+ * current device: MXC_OK, MXC_ERR_DEVICE_INVALID or MXC_ERR_TIMEOUT. */
+mxc_status mxc_get_device_error(mxc_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXC_H_ */

@@ -1,0 +1,156 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function that
+include/mxc.h declares, reports layout sizes, packs weights on the host, and
+rejects bad arguments synchronously (before touching any device)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from vector_quantized_mx_b200 import build, mxc, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return mxc.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "mxc.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mxc_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(mxc.EXPORTED)
+
+
+def test_status_strings(L):
+    for code in range(9):
+        assert L.mxc_status_string(code)
+    assert L.mxc_version() >= 100
+
+
+def test_sf_bytes(L):
+    assert L.mxc_sf_bytes(1, 512, 0) == 128 * 16
+    assert L.mxc_sf_bytes(129, 4096, 1) == 256 * 256
+    assert L.mxc_sf_bytes(0, 4096, 1) == 0
+    assert L.mxc_sf_bytes(10, 4096, 2) == 0      # UE5M3: unsupported
+
+
+def _pack(w):
+    return mxc.pack_weight_host(w)
+
+
+@pytest.mark.parametrize("fmt", ["e8m0_b32", "e4m3_b16"])
+@pytest.mark.parametrize("strategy", ["prescale", "prescale_plus"])
+def test_pack_layouts(L, fmt, strategy):
+    N, K = 256, 768
+    w = synth.make_weight(7, fmt, strategy, N, K, 128, 256)
+    h = _pack(w)
+    # index tiles: [N/128][K/256][128][64]
+    tiles = h["idx"].reshape(N // 128, K // 256, 128, 64)
+    for nt in range(N // 128):
+        for ks in range(K // 256):
+            assert np.array_equal(tiles[nt, ks], w.idx[nt * 128:(nt + 1) * 128, ks * 64:(ks + 1) * 64])
+    B = synth.BLOCK[fmt]
+    if strategy == "prescale_plus":
+        G = 256 // (8 * B)
+        st = h["sidx"].reshape(N // 128, K // 256, 128, G)
+        for nt in range(N // 128):
+            for ks in range(K // 256):
+                assert np.array_equal(st[nt, ks], w.sidx[nt * 128:(nt + 1) * 128, ks * G:(ks + 1) * G])
+        assert h["scales"] is None
+    else:
+        assert h["scales"].size == L.mxc_sf_bytes(N, K, mxc.FMT[fmt])
+        assert np.array_equal(mxc.sf_to_rows(h["scales"], N, K, fmt), w.scales)
+
+
+def test_sf_layout_word_holds_one_row(L):
+    """Each 32-bit word of the SF layout holds four consecutive scales of one row."""
+    N, K = 128, 512
+    w = synth.make_weight(3, "e4m3_b16", "prescale", N, K, 0, 0)
+    sf = _pack(w)["scales"].reshape(-1, 4)
+    KB = K // 16
+    for r in (0, 5, 31, 32, 77, 127):
+        for kb4 in range(KB // 4):
+            word = (kb4 * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4) // 4
+            assert np.array_equal(sf[word], w.scales[r, 4 * kb4:4 * kb4 + 4])
+
+
+def test_packed_sizes_rejects_bad_shapes(L):
+    w = synth.make_weight(1, "e8m0_b32", "prescale", 256, 512, 0, 0)
+    keep = []
+    hw = mxc._host_struct(w, keep)
+    sizes = mxc._PackedSizes()
+    assert L.mxc_packed_weight_sizes(ctypes.byref(hw), ctypes.byref(sizes)) == 0
+    assert sizes.idx == 256 * 128 and sizes.cb == 512
+    hw.K = 500
+    assert L.mxc_packed_weight_sizes(ctypes.byref(hw), ctypes.byref(sizes)) == 3   # alignment
+    hw.K = 512
+    hw.qk = 64
+    assert L.mxc_packed_weight_sizes(ctypes.byref(hw), ctypes.byref(sizes)) == 3
+    hw.qk = 0
+    hw.fmt = 2
+    assert L.mxc_packed_weight_sizes(ctypes.byref(hw), ctypes.byref(sizes)) == 2   # UE5M3 unsupported
+    hw.fmt = 7
+    assert L.mxc_packed_weight_sizes(ctypes.byref(hw), ctypes.byref(sizes)) == 1
+
+
+def test_workspace_sizes(L):
+    assert L.mxc_linear_workspace_bytes(4096, 9216, 4096, 1) == 0          # prefill: none
+    n = L.mxc_linear_workspace_bytes(16, 9216, 4096, 1)                     # decode: split-K partials
+    assert n >= 16 * 9216 * 4
+    assert L.mxc_moe_workspace_bytes(16384, 128, 3072, 4096, 1) >= 129 * 4
+    assert L.mxc_grouped_sf_rows_bound(16384, 128) == 16384 + 128 * 128
+
+
+def test_gpu_calls_reject_bad_arguments_synchronously(L):
+    """Argument errors come back before any device work (safe without a GPU)."""
+    a = mxc._MxTensor(16, 16, None, 4, 512, 256, 0)
+    w = mxc._Weight(1, 0, 256, 512, 0, 0, 16, 16, 16, None, None, 1.0)
+    y = 16
+    # null tensor / weight
+    assert L.mxc_linear(None, ctypes.byref(w), y, 256, 0, None, 0, None) == 1
+    # format mismatch
+    w.fmt = 1
+    assert L.mxc_linear(ctypes.byref(a), ctypes.byref(w), y, 256, 0, None, 0, None) == 1
+    w.fmt = 0
+    # K not a multiple of 256
+    a.K = 500
+    assert L.mxc_linear(ctypes.byref(a), ctypes.byref(w), y, 256, 0, None, 0, None) == 3
+    a.K = 512
+    # ldq too small
+    a.ldq = 128
+    assert L.mxc_linear(ctypes.byref(a), ctypes.byref(w), y, 256, 0, None, 0, None) == 3
+    a.ldq = 256
+    # misaligned pointer
+    w.idx = 17
+    assert L.mxc_linear(ctypes.byref(a), ctypes.byref(w), y, 256, 0, None, 0, None) == 3
+    w.idx = 16
+    # UE5M3
+    a.fmt = w.fmt = 2
+    assert L.mxc_linear(ctypes.byref(a), ctypes.byref(w), y, 256, 0, None, 0, None) == 2
+    a.fmt = w.fmt = 0
+    # PreScale+ without its scale codebook
+    w.strategy = 2
+    assert L.mxc_linear(ctypes.byref(a), ctypes.byref(w), y, 256, 0, None, 0, None) == 1
+    w.strategy = 1
+    # ldy < N
+    assert L.mxc_linear(ctypes.byref(a), ctypes.byref(w), y, 100, 0, None, 0, None) == 1
+    # MoE: too many experts, zero experts
+    table = (mxc._Weight * 1)(w)
+    assert L.mxc_moe_linear(ctypes.byref(a), 16, table, 0, y, 256, 0, None, 0, None) == 1
+    assert L.mxc_moe_linear(ctypes.byref(a), 16, table, 300, y, 256, 0, None, 0, None) == 2
+    # quantize: bad K
+    assert L.mxc_quantize_act(16, 4, 500, 512, 0, None, 16, 256, 16, None, 16, 256, None) == 3
+    # quantize: E4M3 needs a tensor-scale output
+    assert L.mxc_quantize_act(16, 4, 512, 512, 1, None, 16, 256, 16, None, 16, 256, None) == 1

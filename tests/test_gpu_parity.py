@@ -1,0 +1,279 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Bars (from the method's W4A4 contract and the oracle's definitions):
+* quantized activations (FP4 codes, scale bytes, tensor scale) and decoded
+  weights (FP4 codes, scale bytes): bit-exact;
+* linear outputs: |gpu - oracle| <= 1e-4 * sum_k |a_k w_k| per element (FP32
+  output); BF16 output additionally allows the BF16 rounding of the result;
+* MXCode and native FP4 on the same decoded weights: bit-identical outputs
+  (same operands, same tensor-core K order).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import mxcode_oracle as O
+from vector_quantized_mx_b200 import mxc, synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    mxc.lib()
+    assert torch.cuda.get_device_capability()[0] == 10
+
+
+def dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def assert_close(y, ref, sabs, tol=TOL, what=""):
+    y = np.asarray(y, dtype=np.float64)
+    err = np.abs(y - ref)
+    bound = tol * sabs
+    bad = err > bound
+    if bad.any():
+        i = np.argwhere(bad)[0]
+        raise AssertionError(f"{what}: {bad.sum()} of {bad.size} outside tolerance; first at {tuple(i)}: "
+                             f"gpu={y[tuple(i)]!r} ref={ref[tuple(i)]!r} bound={bound[tuple(i)]!r} "
+                             f"max err/bound={np.max(err / np.maximum(bound, 1e-300)):.3g}")
+
+
+def oracle_act(x_bits, fmt, tscale=None):
+    codes, sf, s = O.quantize_act(x_bits, fmt, tscale)
+    return O.pack_fp4(codes), sf, s
+
+
+def check_act(mx, x_bits, fmt, tscale=None):
+    M, K = x_bits.shape
+    q_ref, sf_ref, s_ref = oracle_act(x_bits, fmt, tscale)
+    q = mx.q.cpu().numpy()
+    assert np.array_equal(q, q_ref), f"FP4 codes differ at {np.argwhere(q != q_ref)[:5]}"
+    sf_all = mx.sf.cpu().numpy()
+    rows_pad = (M + 127) // 128 * 128
+    sf_rows = mxc.sf_to_rows(sf_all, rows_pad, K, fmt)
+    assert np.array_equal(sf_rows[:M], sf_ref), f"scales differ at {np.argwhere(sf_rows[:M] != sf_ref)[:5]}"
+    assert not sf_rows[M:].any(), "padding rows must have zero scales"
+    if fmt == "e4m3_b16":
+        assert mx.tscale.item() == np.float32(s_ref)
+
+
+# ---------------------------------------------------------------------------
+# Activation quantization: bit-exact
+# ---------------------------------------------------------------------------
+
+def special_activations(M, K, seed):
+    rng = np.random.default_rng(seed)
+    z = rng.normal(size=(M, K)) * np.exp(rng.uniform(-8, 8, size=(M, 1)))
+    x = torch.from_numpy(z).to(torch.bfloat16)
+    bits = x.view(torch.int16).numpy().view(np.uint16).copy()
+    # exact E2M1 midpoints after a power-of-two scale, zeros, negative zeros, subnormals, big values
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0, 7.0, -0.25, -2.5, -5.0])
+    for r in range(0, M, 3):
+        row = torch.from_numpy(mids * 2.0 ** rng.integers(-20, 20)).to(torch.bfloat16)
+        bits[r, 32:32 + len(mids)] = row.view(torch.int16).numpy().view(np.uint16)
+    specials = [(slice(0, 64), 0),           # +0 blocks
+                (slice(64, 96), 0x8000),     # -0 block
+                (slice(96, 128), 0x0001),    # smallest BF16 subnormal
+                (slice(128, 160), 0x7F7F),   # largest finite BF16
+                (slice(160, 176), 0x8080)]   # negative subnormal
+    for i, (cols, val) in enumerate(specials):
+        bits[(i + 1) % M, cols] = val
+    return bits
+
+
+ACT_CASES = {
+    "config1": lambda: synth.config1()[1],
+    "config2": lambda: synth.config2(16)[1],
+    "special_300x1024": lambda: special_activations(300, 1024, 1),
+    "one_row": lambda: special_activations(1, 512, 2),
+}
+
+
+@pytest.mark.parametrize("fmt", ["e8m0_b32", "e4m3_b16"])
+@pytest.mark.parametrize("case", list(ACT_CASES))
+def test_quantize_act_bitexact(fmt, case):
+    x = ACT_CASES[case]()
+    mx = mxc.quantize_act(dev_bf16(x), fmt)
+    torch.cuda.synchronize()
+    check_act(mx, x, fmt)
+
+
+def test_quantize_act_given_tensor_scale():
+    x = synth.config2(16)[1]
+    ts = torch.tensor([0.0123], dtype=torch.float32, device="cuda")
+    mx = mxc.quantize_act(dev_bf16(x), "e4m3_b16", tscale_in=ts)
+    check_act(mx, x, "e4m3_b16", tscale=np.float32(0.0123))
+
+
+# ---------------------------------------------------------------------------
+# Weight decode: bit-exact
+# ---------------------------------------------------------------------------
+
+def check_decode(w):
+    pw = mxc.pack_weight(w)
+    d = mxc.decode_weight(pw)
+    assert mxc.get_device_error() == 0
+    codes_ref = O.pack_fp4(O.weight_codes(w))
+    q = d.q.cpu().numpy()
+    assert np.array_equal(q, codes_ref), f"decoded FP4 differ at {np.argwhere(q != codes_ref)[:5]}"
+    sf = mxc.sf_to_rows(d.sf.cpu().numpy(), w.N, w.K, w.fmt)
+    assert np.array_equal(sf, O.weight_scale_bytes(w))
+    return pw, d
+
+
+DECODE_CASES = [
+    ("e8m0_b32", "prescale", 256, 1024, 0, 0),
+    ("e8m0_b32", "postscale", 512, 1024, 256, 256),
+    ("e8m0_b32", "prescale_plus", 384, 1536, 128, 128),
+    ("e4m3_b16", "prescale", 256, 1024, 128, 128),
+    ("e4m3_b16", "postscale", 256, 2048, 256, 1024),
+    ("e4m3_b16", "prescale_plus", 512, 1024, 256, 256),
+    ("e4m3_b16", "prescale_plus", 256, 768, 0, 0),
+]
+
+
+@pytest.mark.parametrize("case", DECODE_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_decode_weight_bitexact(case):
+    fmt, strat, N, K, qn, qk = case
+    check_decode(synth.make_weight(11, fmt, strat, N, K, qn, qk))
+
+
+def test_decode_config1_config2_full():
+    check_decode(synth.config1()[0])
+    check_decode(synth.config2(16)[0])
+
+
+# ---------------------------------------------------------------------------
+# Linear layers
+# ---------------------------------------------------------------------------
+
+def run_mxcode(w, x_bits, out_dtype=torch.float32):
+    pw = mxc.pack_weight(w)
+    a = mxc.quantize_act(dev_bf16(x_bits), w.fmt)
+    y = mxc.linear(a, pw, out_dtype)
+    assert mxc.get_device_error() == 0
+    return y, pw, a
+
+
+@pytest.mark.parametrize("fmt", ["e8m0_b32", "e4m3_b16"])
+@pytest.mark.parametrize("M", [1, 4, 16, 200])
+def test_native_linear(fmt, M):
+    w = synth.make_weight(21, fmt, "prescale", 256, 1024, 256, 256)
+    x = synth.make_activations(21, M, 1024, outliers=True)
+    pw = mxc.pack_weight(w)
+    wn = mxc.decode_weight(pw)
+    a = mxc.quantize_act(dev_bf16(x), fmt)
+    y = mxc.native_linear(a, wn).cpu().numpy()
+    assert mxc.get_device_error() == 0
+    ref, sabs = O.w4a4_linear(x, w)
+    assert_close(y, ref, sabs, what=f"native {fmt} M={M}")
+
+
+def test_config1_mxcode():
+    w, x = synth.config1()
+    y, _, _ = run_mxcode(w, x)
+    ref, sabs = O.w4a4_linear(x, w)
+    assert_close(y.cpu().numpy(), ref, sabs, what="config1")
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_config2_decode_gemv(M):
+    w, x = synth.config2(M)
+    y, _, _ = run_mxcode(w, x)
+    ref, sabs = O.w4a4_linear(x, w)
+    assert_close(y.cpu().numpy(), ref, sabs, what=f"config2 M={M}")
+
+
+SWEEP = [(f, s, qb) for f in ("e8m0_b32", "e4m3_b16") for s in ("postscale", "prescale", "prescale_plus")
+         for qb in (0, 256, 128)]
+
+
+@pytest.mark.parametrize("case", SWEEP, ids=lambda c: "-".join(map(str, c)))
+@pytest.mark.parametrize("M", [16, 130])
+def test_mxcode_linear_sweep(case, M):
+    fmt, strat, qb = case
+    w = synth.make_weight(31, fmt, strat, 512, 1024, qb, qb)
+    x = synth.make_activations(31, M, 1024, outliers=True)
+    y, _, _ = run_mxcode(w, x)
+    ref, sabs = O.w4a4_linear(x, w)
+    assert_close(y.cpu().numpy(), ref, sabs, what=f"{case} M={M}")
+
+
+@pytest.mark.parametrize("fmt", ["e8m0_b32", "e4m3_b16"])
+@pytest.mark.parametrize("M", [16, 300])
+def test_mxcode_equals_native_on_decoded_weights(fmt, M):
+    w = synth.make_weight(41, fmt, "prescale_plus", 384, 2048, 128, 256)
+    x = synth.make_activations(41, M, 2048, outliers=True)
+    y, pw, a = run_mxcode(w, x)
+    wn = mxc.decode_weight(pw)
+    yn = mxc.native_linear(a, wn)
+    assert torch.equal(y, yn)
+
+
+def test_bf16_output():
+    w = synth.make_weight(51, "e4m3_b16", "prescale", 256, 1024, 256, 256)
+    x = synth.make_activations(51, 40, 1024, outliers=True)
+    y, pw, a = run_mxcode(w, x, torch.bfloat16)
+    y32 = mxc.linear(a, pw, torch.float32)
+    ref_bf16 = y32.to(torch.bfloat16)               # RNE of the FP32 result
+    assert torch.equal(y, ref_bf16)
+    ref, sabs = O.w4a4_linear(x, w)
+    yy = y.float().cpu().numpy()
+    assert_close(yy, ref, sabs + np.abs(ref) * 2.0 ** -8 / TOL, what="bf16")
+
+
+# ---------------------------------------------------------------------------
+# Grouped experts (MoE)
+# ---------------------------------------------------------------------------
+
+def run_moe(fmt, strat, E, N, K, counts, seed):
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    M = int(offsets[-1])
+    ws = [synth.make_weight(seed, fmt, strat, N, K, 256, 256, sub=e) for e in range(E)]
+    x = synth.make_activations(seed, M, K, outliers=False)
+    off_d = torch.from_numpy(offsets.astype(np.int32)).cuda()
+    a = mxc.quantize_act_grouped(dev_bf16(x), fmt, off_d)
+    packed = [mxc.pack_weight(w) for w in ws]
+    y = mxc.moe_linear(a, off_d, packed).cpu().numpy()
+    assert mxc.get_device_error() == 0
+    # the activation tensor scale is shared by all rows
+    codes, sf, s = O.quantize_act(x, fmt)
+    a_hat = O.dequant_act(codes, sf, fmt, s)
+    # grouped quantization must equal the dense one, row for row
+    assert np.array_equal(a.q.cpu().numpy(), O.pack_fp4(codes))
+    for e in range(E):
+        r0, r1 = offsets[e], offsets[e + 1]
+        if r1 == r0:
+            continue
+        w_hat = O.dequant_weight(ws[e])
+        ref = O.linear(a_hat[r0:r1], w_hat)
+        sabs = O.abs_linear(a_hat[r0:r1], w_hat)
+        assert_close(y[r0:r1], ref, sabs, what=f"expert {e}")
+
+
+@pytest.mark.parametrize("fmt", ["e8m0_b32", "e4m3_b16"])
+@pytest.mark.parametrize("strat", ["prescale", "prescale_plus"])
+def test_moe_small(fmt, strat):
+    run_moe(fmt, strat, 6, 256, 512, [0, 5, 130, 1, 257, 0], seed=61)
+
+
+def test_moe_bad_offsets_sets_device_error():
+    E, N, K = 3, 128, 256
+    ws = [mxc.pack_weight(synth.make_weight(71, "e8m0_b32", "prescale", N, K, 0, 0, sub=e)) for e in range(E)]
+    x = synth.make_activations(71, 10, K, outliers=False)
+    good = torch.tensor([0, 4, 7, 10], dtype=torch.int32, device="cuda")
+    a = mxc.quantize_act_grouped(dev_bf16(x), "e8m0_b32", good)
+    assert mxc.get_device_error() == 0
+    bad = torch.tensor([0, 6, 3, 10], dtype=torch.int32, device="cuda")     # decreasing
+    y = torch.full((10, N), 7.0, device="cuda")
+    mxc.moe_linear(a, bad, ws, y=y)
+    assert mxc.get_device_error() == 6                                       # MXC_ERR_DEVICE_INVALID
+    assert torch.all(y == 7.0)                                               # nothing written
+    assert mxc.get_device_error() == 0                                       # cleared by the read

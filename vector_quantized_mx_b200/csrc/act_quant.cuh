@@ -1,0 +1,275 @@
+// act_quant.cu -- BF16 -> MX FP4 activation quantization (W4A4 activations).
+//
+// "MXCode: Vector Quantization for MX-Native Inference at Scale": W4A4 on native
+// block-scaled FP4 (abstract; Table 2 caption), formats E8M0-B32 and E4M3-B16
+// with an FP32 tensor scale (Table 1).  The pages give no activation recipe;
+// this follows the OCP MX rule (block scale from the block amax, E2M1 round to
+// nearest even, saturate at +-6) with the E4M3 tensor scale amax/(6*448).
+//
+// One thread quantizes one block (32 or 16 elements): vector loads of BF16,
+// block amax, scale byte, 32/16 E2M1 codes decided by the sign of an exact
+// fused multiply-add against each rounding midpoint, one vector store of FP4.
+// The work is HBM-bound (read 2 bytes/element, write ~0.53).
+#include <cstdint>
+
+#include "mxc_device.cuh"
+#include "mxc_internal.h"
+
+namespace mxc {
+
+// Byte offset of scale (r, kb) in the SF layout (see mxc.h).
+__device__ __forceinline__ size_t sf_offset(int64_t r, int kb, int kb_per_row) {
+  return (static_cast<size_t>(r >> 7) * (kb_per_row >> 2) + (kb >> 2)) * 512 + (r & 31) * 16 +
+         ((r >> 5) & 3) * 4 + (kb & 3);
+}
+
+// E4M3 (no infinities, max 448) of a non-negative float: round to nearest,
+// ties to even mantissa, saturating at 448.
+__device__ __forceinline__ uint32_t e4m3_encode_satfinite(float v) {
+  if (!(v < 448.0f)) return 0x7E;                        // >= 448 (and +inf)
+  if (v < 0.015625f) {                                   // below 2^-6: subnormal grid m * 2^-9
+    return static_cast<uint32_t>(__float2int_rn(v * 512.0f));   // exact scaling, RNE; 8 -> 0x08
+  }
+  const uint32_t u = __float_as_uint(v);
+  uint32_t x = u >> 20;                                  // exponent + top 3 mantissa bits
+  const uint32_t rem = u & 0xFFFFFu;
+  if (rem > 0x80000u || (rem == 0x80000u && (x & 1u))) x += 1;
+  const uint32_t b = x - ((127u - 7u) << 3);             // rebias 127 -> 7
+  return b > 0x7Eu ? 0x7Eu : b;
+}
+
+__device__ __forceinline__ float e4m3_decode(uint32_t b) {
+  const uint32_t e = (b >> 3) & 0xF, m = b & 7;
+  if (e == 0) return static_cast<float>(m) * 0.001953125f;  // m * 2^-9
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// 2^e for e in [-127, 127] as an exact float (2^-127 is subnormal).
+__device__ __forceinline__ float exp2_int(int e) {
+  return e >= -126 ? __uint_as_float(static_cast<uint32_t>(e + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// E2M1 code of x / d, round half to even, saturating at 6, sign of x kept.
+// Each midpoint test uses the sign of fma(mu, d, -|x|), which is the sign of
+// the exact value mu*d - |x| (one rounding never flips a sign).
+__device__ __forceinline__ uint32_t e2m1_code(float x, float d) {
+  const float a = fabsf(x);
+  uint32_t c = 0;
+  c += __fmaf_rn(0.25f, d, -a) < 0.0f;   // a >  0.25 d   (tie -> 0)
+  c += __fmaf_rn(0.75f, d, -a) <= 0.0f;  // a >= 0.75 d   (tie -> 1.0)
+  c += __fmaf_rn(1.25f, d, -a) < 0.0f;   // a >  1.25 d   (tie -> 1.0)
+  c += __fmaf_rn(1.75f, d, -a) <= 0.0f;  // a >= 1.75 d   (tie -> 2.0)
+  c += __fmaf_rn(2.50f, d, -a) < 0.0f;   // a >  2.5 d    (tie -> 2.0)
+  c += __fmaf_rn(3.50f, d, -a) <= 0.0f;  // a >= 3.5 d    (tie -> 4.0)
+  c += __fmaf_rn(5.00f, d, -a) < 0.0f;   // a >  5 d      (tie -> 4.0)
+  return c | ((__float_as_uint(x) >> 28) & 8u);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Quantizes one block of B = 32 or 16 BF16 values held as B/2 packed words.
+template <int B>
+__device__ __forceinline__ void quantize_block(const uint32_t (&w)[B / 2], bool e4m3, float s,
+                                               uint32_t (&q)[B / 8], uint32_t& sf_byte) {
+  uint32_t amax_bits = 0;
+#pragma unroll
+  for (int i = 0; i < B / 2; ++i) {
+    amax_bits = max(amax_bits, w[i] & 0x7FFFu);
+    amax_bits = max(amax_bits, (w[i] >> 16) & 0x7FFFu);
+  }
+  const float amax = __uint_as_float(amax_bits << 16);
+  float d = 0.0f;
+  if (!e4m3) {
+    if (amax_bits == 0) {
+      sf_byte = 0;
+    } else {
+      const uint32_t u = amax_bits << 16;
+      const uint32_t E = (u >> 23) & 0xFF;
+      const int flog = E ? static_cast<int>(E) - 127 : (31 - __clz(u & 0x7FFFFF)) - 149;
+      const int e = min(127, max(-127, flog - 2));
+      sf_byte = static_cast<uint32_t>(e + 127);
+      d = exp2_int(e);
+    }
+  } else {
+    const float t = __fdiv_rn(__fdiv_rn(amax, 6.0f), s);
+    sf_byte = e4m3_encode_satfinite(t);
+    d = sf_byte ? __fmul_rn(e4m3_decode(sf_byte), s) : 0.0f;
+  }
+#pragma unroll
+  for (int i = 0; i < B / 8; ++i) q[i] = 0;
+#pragma unroll
+  for (int i = 0; i < B / 2; ++i) {
+    const float x0 = bf16_lo(w[i]), x1 = bf16_hi(w[i]);
+    uint32_t c0, c1;
+    if (d == 0.0f) {  // all-zero block, or an E4M3 scale that rounded to 0: signed zeros
+      c0 = (w[i] >> 12) & 8u;
+      c1 = (w[i] >> 28) & 8u;
+    } else {
+      c0 = e2m1_code(x0, d);
+      c1 = e2m1_code(x1, d);
+    }
+    q[i / 4] |= (c0 | (c1 << 4)) << (8 * (i % 4));
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// Tensor amax (E4M3 path): max |x| over [M, K], as FP32 bits, via atomicMax on a
+// zero-initialised word (max is order independent, so the result is deterministic).
+// ------------------------------------------------------------------------------------
+__global__ void amax_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K, int64_t ldx,
+                            unsigned int* __restrict__ amax_out) {
+  const int64_t chunks_per_row = K / 8;
+  const int64_t total = M * chunks_per_row;
+  uint32_t m = 0;
+  for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < total;
+       c += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = c / chunks_per_row, k8 = c - r * chunks_per_row;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + r * ldx + k8 * 8));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      m = max(m, w[i] & 0x7FFFu);
+      m = max(m, (w[i] >> 16) & 0x7FFFu);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0 && m) atomicMax(amax_out, m << 16);
+}
+
+// ------------------------------------------------------------------------------------
+// Quantization.  One thread per (scale row, block).  Dense mode: scale row = data
+// row, rows in [M, round_up(M,128)) only get zero scales.  Grouped mode: scale
+// rows are padded per group to multiples of 128 (tile_prefix from the group
+// prologue) and mapped back to data rows.
+// ------------------------------------------------------------------------------------
+template <int B>
+__global__ void __launch_bounds__(256) quantize_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int64_t K, int64_t ldx, int e4m3,
+    const float* __restrict__ tscale_in, const unsigned int* __restrict__ amax_ws,
+    uint8_t* __restrict__ q, int64_t ldq, uint8_t* __restrict__ sf, float* __restrict__ tscale_out,
+    int64_t sf_rows, const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_prefix,
+    int32_t n_groups) {
+  const int kb_per_row = static_cast<int>(K / B);
+  float s = 1.0f;
+  if (e4m3) {
+    if (tscale_in) {
+      s = *tscale_in;
+    } else {
+      const float amax = __uint_as_float(*amax_ws);
+      s = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
+    }
+  }
+  if (tscale_out && blockIdx.x == 0 && threadIdx.x == 0) *tscale_out = s;
+  int64_t rows_total = sf_rows;
+  if (tile_prefix) rows_total = min(sf_rows, static_cast<int64_t>(tile_prefix[n_groups]) * 128);
+  const int64_t units = rows_total * kb_per_row;
+  for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < units;
+       u += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t pr = u / kb_per_row;          // scale row
+    const int kb = static_cast<int>(u - pr * kb_per_row);
+    int64_t r = pr;                             // data row, -1 = padding
+    if (tile_prefix) {
+      int lo = 0, hi = n_groups - 1;            // group g with tile_prefix[g]*128 <= pr
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (static_cast<int64_t>(tile_prefix[mid]) * 128 <= pr) lo = mid; else hi = mid - 1;
+      }
+      const int64_t local = pr - static_cast<int64_t>(tile_prefix[lo]) * 128;
+      r = local < offsets[lo + 1] - offsets[lo] ? offsets[lo] + local : -1;
+    } else if (pr >= M) {
+      r = -1;
+    }
+    uint32_t sfb = 0;
+    if (r >= 0) {
+      const uint16_t* src = x + r * ldx + static_cast<int64_t>(kb) * B;
+      uint32_t w[B / 2];
+#pragma unroll
+      for (int i = 0; i < B / 8; ++i) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
+        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+      }
+      uint32_t qw[B / 8];
+      quantize_block<B>(w, e4m3 != 0, s, qw, sfb);
+      uint8_t* dst = q + r * ldq + static_cast<int64_t>(kb) * (B / 2);
+      if (B == 32) {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(qw[0], qw[1], qw[2], qw[3]);
+      } else {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(qw[0], qw[1]);
+      }
+    }
+    sf[sf_offset(pr, kb, kb_per_row)] = static_cast<uint8_t>(sfb);
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// Group prologue: validates offsets and writes tile_prefix[g] = sum over g' < g of
+// ceil(rows_g' / 128), g = 0..E.  Malformed offsets set MXC_ERR_DEVICE_INVALID and
+// an all-zero prefix, so that the kernels that follow do no work.
+// ------------------------------------------------------------------------------------
+__global__ void group_prologue_kernel(const int32_t* __restrict__ offsets, int32_t E, int64_t M,
+                                      int32_t* __restrict__ tile_prefix) {
+  __shared__ int bad;
+  __shared__ int32_t tiles[kMaxGroups + 1];
+  if (threadIdx.x == 0) bad = (offsets[0] != 0 || offsets[E] != M);
+  __syncthreads();
+  for (int g = threadIdx.x; g < E; g += blockDim.x) {
+    const int32_t c = offsets[g + 1] - offsets[g];
+    if (c < 0) bad = 1;
+    tiles[g] = c > 0 ? (c + 127) / 128 : 0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t acc = 0;
+    for (int g = 0; g < E; ++g) {
+      tile_prefix[g] = bad ? 0 : acc;
+      acc += tiles[g];
+    }
+    tile_prefix[E] = bad ? 0 : acc;
+    if (bad) set_device_error(MXC_ERR_DEVICE_INVALID);
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// Host launchers
+// ------------------------------------------------------------------------------------
+cudaError_t launch_group_prologue(const int32_t* offsets, int32_t E, int64_t M, int32_t* tile_prefix,
+                                  cudaStream_t stream) {
+  group_prologue_kernel<<<1, 256, 0, stream>>>(offsets, E, M, tile_prefix);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
+  const bool e4m3 = a.fmt == MXC_FMT_E4M3_B16;
+  const int B = e4m3 ? 16 : 32;
+  unsigned int* amax_ws = reinterpret_cast<unsigned int*>(a.ws);
+  if (e4m3 && !a.tscale_in) {
+    cudaError_t err = cudaMemsetAsync(amax_ws, 0, sizeof(unsigned int), stream);
+    if (err != cudaSuccess) return err;
+    const int64_t chunks = a.M * (a.K / 8);
+    const int threads = 256;
+    const int64_t want = (chunks + threads - 1) / threads;
+    const int blocks = static_cast<int>(want < 148 * 8 ? (want > 0 ? want : 1) : 148 * 8);
+    amax_kernel<<<blocks, threads, 0, stream>>>(reinterpret_cast<const uint16_t*>(a.x), a.M, a.K, a.ldx,
+                                                amax_ws);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  const int64_t units = a.sf_rows * (a.K / B);
+  const int threads = 256;
+  const int64_t want = (units + threads - 1) / threads;
+  const int blocks = static_cast<int>(want < 148 * 16 ? (want > 0 ? want : 1) : 148 * 16);
+  if (e4m3) {
+    quantize_kernel<16><<<blocks, threads, 0, stream>>>(
+        reinterpret_cast<const uint16_t*>(a.x), a.M, a.K, a.ldx, 1, a.tscale_in, amax_ws, a.q, a.ldq,
+        a.sf, a.tscale_out, a.sf_rows, a.offsets, a.tile_prefix, a.n_groups);
+  } else {
+    quantize_kernel<32><<<blocks, threads, 0, stream>>>(
+        reinterpret_cast<const uint16_t*>(a.x), a.M, a.K, a.ldx, 0, nullptr, nullptr, a.q, a.ldq, a.sf,
+        a.tscale_out, a.sf_rows, a.offsets, a.tile_prefix, a.n_groups);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace mxc

@@ -1,0 +1,257 @@
+// linear.cuh -- host-side launch of the linear-layer kernels: tensor maps, tile and
+// split-K policy, workspace layout, template dispatch.
+#pragma once
+
+#include <cstring>
+
+#include "mma_kernel.cuh"
+
+namespace mxc {
+
+// ------------------------------------------------------------------------------------
+// Tensor maps (driver entry point fetched through the runtime, so the library does
+// not link libcuda directly).
+// ------------------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D map over an FP4 matrix [rows, K/2 bytes] (row stride ld bytes); box = 128
+// bytes (256 FP4 values) x box_rows rows, 128-byte swizzle, zero fill outside.
+inline bool make_fp4_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int64_t ld,
+                         int box_rows) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return false;
+  std::memset(map, 0, sizeof(*map));
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld)};
+  const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------------------------
+// Policy
+// ------------------------------------------------------------------------------------
+constexpr int kDecodeMaxM = 16;   // M <= 16: split-K decode path with a 16-token tile
+constexpr int kSMs = 148;
+
+inline int token_tile(int64_t M) { return M <= kDecodeMaxM ? 16 : 128; }
+
+// Split-K factor of the decode path: enough CTAs to cover the SMs twice, at
+// least two 256-channel stages per CTA, and no empty split.
+inline void decode_splits(int64_t N, int64_t K, int* splits, int* ks_per_split) {
+  const int n_tiles = static_cast<int>(N / kTileN);
+  const int KS = static_cast<int>(K / kStageK);
+  int s = (2 * kSMs + n_tiles - 1) / n_tiles;
+  s = s < 1 ? 1 : s;
+  const int smax = KS / 2 > 0 ? KS / 2 : 1;
+  s = s > smax ? smax : s;
+  const int per = (KS + s - 1) / s;
+  *ks_per_split = per;
+  *splits = (KS + per - 1) / per;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int /*fmt*/) {
+  if (M > kDecodeMaxM) return 0;
+  int splits, per;
+  decode_splits(N, K, &splits, &per);
+  if (splits <= 1) return 0;
+  return align_up(static_cast<size_t>(splits) * M * N * sizeof(float), 256) +
+         align_up(static_cast<size_t>(N / kTileN) * sizeof(int), 256);
+}
+
+size_t moe_workspace_bytes(int64_t /*M*/, int32_t E, int64_t /*N*/, int64_t /*K*/, int /*fmt*/) {
+  return align_up(static_cast<size_t>(E + 1) * sizeof(int32_t), 256);
+}
+
+// ------------------------------------------------------------------------------------
+// Launch
+// ------------------------------------------------------------------------------------
+template <int FMT, int WSRC, int T, bool MOE>
+cudaError_t launch_gemm(const CUtensorMap& tx, const CUtensorMap& tw,
+                        const GemmParams<MOE ? kMaxGroups : 1>& p, dim3 grid, cudaStream_t stream) {
+  using L = StageLayout<FMT, WSRC, T>;
+  auto kern = gemm_kernel<FMT, WSRC, T, MOE>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+  if (err != cudaSuccess) return err;
+  kern<<<grid, kThreads, L::SMEM, stream>>>(tx, tw, p);
+  return cudaGetLastError();
+}
+
+template <int FMT, int WSRC, int T>
+cudaError_t dispatch_dense(const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams<1>& p, dim3 grid,
+                           cudaStream_t stream) {
+  return launch_gemm<FMT, WSRC, T, false>(tx, tw, p, grid, stream);
+}
+
+template <int FMT, int WSRC>
+cudaError_t dispatch_tile(int T, const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams<1>& p, dim3 grid,
+                          cudaStream_t stream) {
+  if (T == 16) return dispatch_dense<FMT, WSRC, 16>(tx, tw, p, grid, stream);
+  return dispatch_dense<FMT, WSRC, 128>(tx, tw, p, grid, stream);
+}
+
+inline ExpertPtrs expert_ptrs(const LinearArgs& a) {
+  ExpertPtrs e{};
+  e.idx = a.w_idx;
+  e.cb = a.w_cb;
+  e.sf = a.w_sf;
+  e.sidx = a.w_sidx;
+  e.scb = a.w_scb;
+  e.w_tscale = a.w_tscale;
+  return e;
+}
+
+mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
+  const int T = token_tile(a.M);
+  CUtensorMap tx, tw;
+  if (!make_fp4_map(&tx, a.a_q, a.M, a.K, a.ldq, T)) return MXC_ERR_CUDA;
+  if (a.wsrc == WSRC_NATIVE) {
+    if (!make_fp4_map(&tw, a.w_q, a.N, a.K, a.w_ldq, 128)) return MXC_ERR_CUDA;
+  } else {
+    tw = tx;  // unused
+  }
+  GemmParams<1> p{};
+  p.M = static_cast<int>(a.M);
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.qn = static_cast<int>(a.qn);
+  p.qk = static_cast<int>(a.qk);
+  p.a_sf = a.a_sf;
+  p.a_tscale = a.a_tscale;
+  p.w_tscale_dev = a.w_tscale_dev;
+  p.y = a.y;
+  p.ldy = a.ldy;
+  p.out_bf16 = a.out_bf16;
+  p.splits = 1;
+  p.ks_per_split = static_cast<int>(a.K / kStageK);
+  p.w[0] = expert_ptrs(a);
+  if (a.wsrc == WSRC_NATIVE) p.w[0].sf = a.w_sf;
+  const int n_tiles = static_cast<int>(a.N / kTileN);
+  const int m_tiles = static_cast<int>((a.M + T - 1) / T);
+  if (T == 16) {
+    int splits, per;
+    decode_splits(a.N, a.K, &splits, &per);
+    if (splits > 1) {
+      const size_t need = linear_workspace_bytes(a.M, a.N, a.K, a.fmt);
+      if (!a.ws || a.ws_bytes < need) return MXC_ERR_WORKSPACE;
+      p.splits = splits;
+      p.ks_per_split = per;
+      p.partials = reinterpret_cast<float*>(a.ws);
+      p.counters = reinterpret_cast<int*>(reinterpret_cast<char*>(a.ws) +
+                                          align_up(static_cast<size_t>(splits) * a.M * a.N * sizeof(float), 256));
+      if (cudaMemsetAsync(p.counters, 0, static_cast<size_t>(n_tiles) * m_tiles * sizeof(int), stream) !=
+          cudaSuccess)
+        return MXC_ERR_CUDA;
+    }
+  }
+  const dim3 grid(n_tiles, m_tiles, p.splits);
+  cudaError_t err;
+  if (a.fmt == FMT_E8M0) {
+    if (a.wsrc == WSRC_VQ_DIRECT) err = dispatch_tile<FMT_E8M0, WSRC_VQ_DIRECT>(T, tx, tw, p, grid, stream);
+    else if (a.wsrc == WSRC_VQ_SVQ) err = dispatch_tile<FMT_E8M0, WSRC_VQ_SVQ>(T, tx, tw, p, grid, stream);
+    else err = dispatch_tile<FMT_E8M0, WSRC_NATIVE>(T, tx, tw, p, grid, stream);
+  } else {
+    if (a.wsrc == WSRC_VQ_DIRECT) err = dispatch_tile<FMT_E4M3, WSRC_VQ_DIRECT>(T, tx, tw, p, grid, stream);
+    else if (a.wsrc == WSRC_VQ_SVQ) err = dispatch_tile<FMT_E4M3, WSRC_VQ_SVQ>(T, tx, tw, p, grid, stream);
+    else err = dispatch_tile<FMT_E4M3, WSRC_NATIVE>(T, tx, tw, p, grid, stream);
+  }
+  return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
+}
+
+mxc_status run_moe_linear(const MoeArgs& m, cudaStream_t stream) {
+  const LinearArgs& a = m.base;
+  const size_t need = moe_workspace_bytes(a.M, m.E, a.N, a.K, a.fmt);
+  if (!a.ws || a.ws_bytes < need) return MXC_ERR_WORKSPACE;
+  int32_t* tile_prefix = reinterpret_cast<int32_t*>(a.ws);
+  if (launch_group_prologue(m.offsets, m.E, a.M, tile_prefix, stream) != cudaSuccess) return MXC_ERR_CUDA;
+  CUtensorMap tx;
+  if (!make_fp4_map(&tx, a.a_q, a.M, a.K, a.ldq, 128)) return MXC_ERR_CUDA;
+  // GemmParams with the expert table (about 12 KB of kernel parameters).
+  static thread_local GemmParams<kMaxGroups> p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = static_cast<int>(a.M);
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.qn = static_cast<int>(a.qn);
+  p.qk = static_cast<int>(a.qk);
+  p.a_sf = a.a_sf;
+  p.a_tscale = a.a_tscale;
+  p.y = a.y;
+  p.ldy = a.ldy;
+  p.out_bf16 = a.out_bf16;
+  p.splits = 1;
+  p.ks_per_split = static_cast<int>(a.K / kStageK);
+  p.E = m.E;
+  p.offsets = m.offsets;
+  p.tile_prefix = tile_prefix;
+  for (int e = 0; e < m.E; ++e) {
+    const mxc_weight& w = m.experts[e];
+    p.w[e].idx = w.idx;
+    p.w[e].cb = w.cb;
+    p.w[e].sf = w.scales;
+    p.w[e].sidx = w.sidx;
+    p.w[e].scb = w.scb;
+    p.w[e].w_tscale = w.w_tscale;
+  }
+  const dim3 grid(static_cast<unsigned>(a.N / kTileN), static_cast<unsigned>((a.M + 127) / 128 + m.E), 1);
+  cudaError_t err;
+  if (a.fmt == FMT_E8M0) {
+    if (a.wsrc == WSRC_VQ_DIRECT) err = launch_gemm<FMT_E8M0, WSRC_VQ_DIRECT, 128, true>(tx, tx, p, grid, stream);
+    else err = launch_gemm<FMT_E8M0, WSRC_VQ_SVQ, 128, true>(tx, tx, p, grid, stream);
+  } else {
+    if (a.wsrc == WSRC_VQ_DIRECT) err = launch_gemm<FMT_E4M3, WSRC_VQ_DIRECT, 128, true>(tx, tx, p, grid, stream);
+    else err = launch_gemm<FMT_E4M3, WSRC_VQ_SVQ, 128, true>(tx, tx, p, grid, stream);
+  }
+  return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
+}
+
+template <int FMT, int WSRC>
+cudaError_t launch_decode_dump(const DecodeArgs& a, cudaStream_t stream) {
+  using L = StageLayout<FMT, WSRC, 16>;
+  constexpr int smem = 1024 + L::CTRL + L::BYTES;
+  auto kern = decode_dump_kernel<FMT, WSRC>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  ExpertPtrs w{};
+  w.idx = a.w_idx;
+  w.cb = a.w_cb;
+  w.sf = a.w_sf;
+  w.sidx = a.w_sidx;
+  w.scb = a.w_scb;
+  const dim3 grid(static_cast<unsigned>(a.N / kTileN), static_cast<unsigned>(a.K / kStageK));
+  kern<<<grid, 160, smem, stream>>>(w, static_cast<int>(a.N), static_cast<int>(a.K), static_cast<int>(a.qn),
+                                    static_cast<int>(a.qk), a.q_out, a.ldq, a.sf_out);
+  return cudaGetLastError();
+}
+
+mxc_status run_decode_weight(const DecodeArgs& a, cudaStream_t stream) {
+  cudaError_t err;
+  if (a.fmt == FMT_E8M0) {
+    err = a.wsrc == WSRC_VQ_SVQ ? launch_decode_dump<FMT_E8M0, WSRC_VQ_SVQ>(a, stream)
+                                : launch_decode_dump<FMT_E8M0, WSRC_VQ_DIRECT>(a, stream);
+  } else {
+    err = a.wsrc == WSRC_VQ_SVQ ? launch_decode_dump<FMT_E4M3, WSRC_VQ_SVQ>(a, stream)
+                                : launch_decode_dump<FMT_E4M3, WSRC_VQ_DIRECT>(a, stream);
+  }
+  return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
+}
+
+}  // namespace mxc
