@@ -107,8 +107,7 @@ def test_packed_sizes_rejects_bad_shapes(L):
 
 def test_workspace_sizes(L):
     assert L.mxc_linear_workspace_bytes(4096, 9216, 4096, 1) == 0          # prefill: none
-    n = L.mxc_linear_workspace_bytes(16, 9216, 4096, 1)                     # decode: split-K partials
-    assert n >= 16 * 9216 * 4
+    assert L.mxc_linear_workspace_bytes(16, 9216, 4096, 1) == 0            # decode: split-K in cluster SMEM
     assert L.mxc_moe_workspace_bytes(16384, 128, 3072, 4096, 1) >= 129 * 4
     assert L.mxc_grouped_sf_rows_bound(16384, 128) == 16384 + 128 * 128
 

@@ -119,12 +119,11 @@ __device__ __forceinline__ void quantize_block(const uint32_t (&w)[B / 2], bool 
 // ------------------------------------------------------------------------------------
 __global__ void amax_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K, int64_t ldx,
                             unsigned int* __restrict__ amax_out) {
-  const int64_t chunks_per_row = K / 8;
-  const int64_t total = M * chunks_per_row;
+  const uint32_t chunks_per_row = static_cast<uint32_t>(K / 8);
+  const uint32_t total = static_cast<uint32_t>(M) * chunks_per_row;
   uint32_t m = 0;
-  for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < total;
-       c += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = c / chunks_per_row, k8 = c - r * chunks_per_row;
+  for (uint32_t c = blockIdx.x * blockDim.x + threadIdx.x; c < total; c += gridDim.x * blockDim.x) {
+    const uint32_t r = c / chunks_per_row, k8 = c - r * chunks_per_row;
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + r * ldx + k8 * 8));
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -136,6 +135,50 @@ __global__ void amax_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   if ((threadIdx.x & 31) == 0 && m) atomicMax(amax_out, m << 16);
+}
+
+// One (scale row, block) unit: dense mode maps scale row = data row (rows past M
+// only get zero scales); grouped mode maps padded scale rows back to data rows.
+template <int B>
+__device__ __forceinline__ void quantize_unit(const uint16_t* __restrict__ x, int64_t M, int64_t K, int64_t ldx,
+                                              int e4m3, float s, uint8_t* __restrict__ q, int64_t ldq,
+                                              uint8_t* __restrict__ sf, uint32_t u, int kb_per_row,
+                                              const int32_t* __restrict__ offsets,
+                                              const int32_t* __restrict__ tile_prefix, int32_t n_groups) {
+  const uint32_t pr32 = u / static_cast<uint32_t>(kb_per_row);
+  const int64_t pr = pr32;                    // scale row
+  const int kb = static_cast<int>(u - pr32 * static_cast<uint32_t>(kb_per_row));
+  int64_t r = pr;                             // data row, -1 = padding
+  if (tile_prefix) {
+    int lo = 0, hi = n_groups - 1;            // group g with tile_prefix[g]*128 <= pr
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (static_cast<int64_t>(tile_prefix[mid]) * 128 <= pr) lo = mid; else hi = mid - 1;
+    }
+    const int64_t local = pr - static_cast<int64_t>(tile_prefix[lo]) * 128;
+    r = local < offsets[lo + 1] - offsets[lo] ? offsets[lo] + local : -1;
+  } else if (pr >= M) {
+    r = -1;
+  }
+  uint32_t sfb = 0;
+  if (r >= 0) {
+    const uint16_t* src = x + r * ldx + static_cast<int64_t>(kb) * B;
+    uint32_t w[B / 2];
+#pragma unroll
+    for (int i = 0; i < B / 8; ++i) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
+      w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+    }
+    uint32_t qw[B / 8];
+    quantize_block<B>(w, e4m3 != 0, s, qw, sfb);
+    uint8_t* dst = q + r * ldq + static_cast<int64_t>(kb) * (B / 2);
+    if (B == 32) {
+      *reinterpret_cast<uint4*>(dst) = make_uint4(qw[0], qw[1], qw[2], qw[3]);
+    } else {
+      *reinterpret_cast<uint2*>(dst) = make_uint2(qw[0], qw[1]);
+    }
+  }
+  sf[sf_offset(pr, kb, kb_per_row)] = static_cast<uint8_t>(sfb);
 }
 
 // ------------------------------------------------------------------------------------
@@ -164,42 +207,70 @@ __global__ void __launch_bounds__(256) quantize_kernel(
   if (tscale_out && blockIdx.x == 0 && threadIdx.x == 0) *tscale_out = s;
   int64_t rows_total = sf_rows;
   if (tile_prefix) rows_total = min(sf_rows, static_cast<int64_t>(tile_prefix[n_groups]) * 128);
-  const int64_t units = rows_total * kb_per_row;
-  for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < units;
-       u += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t pr = u / kb_per_row;          // scale row
-    const int kb = static_cast<int>(u - pr * kb_per_row);
-    int64_t r = pr;                             // data row, -1 = padding
-    if (tile_prefix) {
-      int lo = 0, hi = n_groups - 1;            // group g with tile_prefix[g]*128 <= pr
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (static_cast<int64_t>(tile_prefix[mid]) * 128 <= pr) lo = mid; else hi = mid - 1;
-      }
-      const int64_t local = pr - static_cast<int64_t>(tile_prefix[lo]) * 128;
-      r = local < offsets[lo + 1] - offsets[lo] ? offsets[lo] + local : -1;
-    } else if (pr >= M) {
-      r = -1;
-    }
-    uint32_t sfb = 0;
-    if (r >= 0) {
-      const uint16_t* src = x + r * ldx + static_cast<int64_t>(kb) * B;
-      uint32_t w[B / 2];
+  const uint32_t units = static_cast<uint32_t>(rows_total * kb_per_row);
+  for (uint32_t u = blockIdx.x * blockDim.x + threadIdx.x; u < units; u += gridDim.x * blockDim.x)
+    quantize_unit<B>(x, M, K, ldx, e4m3, s, q, ldq, sf, u, kb_per_row, offsets, tile_prefix, n_groups);
+}
+
+// Small activations (decode batches): one launch, grid (KB/256 blocks, rows).
+// Every CTA computes the tensor amax itself (the tensor is at most a few hundred
+// KB and sits in L2) and then quantizes blocks of its row; the CTAs of row 0 also
+// clear the padding scale rows [M, round_up(M,128)) a 32-bit word at a time.
+template <int B>
+__global__ void __launch_bounds__(256) quantize_small_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int64_t K, int64_t ldx, int e4m3,
+    const float* __restrict__ tscale_in, uint8_t* __restrict__ q, int64_t ldq, uint8_t* __restrict__ sf,
+    float* __restrict__ tscale_out, int64_t sf_rows) {
+  __shared__ uint32_t red[8];
+  const int kb_per_row = static_cast<int>(K / B);
+  const int rows = static_cast<int>(M), k8s = static_cast<int>(K / 8);
+  float s = 1.0f;
+  if (e4m3) {
+    if (tscale_in) {
+      s = *tscale_in;
+    } else {
+      // 8 independent 16-byte loads in flight per thread (a small grid cannot hide
+      // L2 latency with other warps)
+      uint32_t m = 0;
+      const int total = rows * k8s;
+      for (int c0 = threadIdx.x; c0 < total; c0 += 8 * 256) {
+        uint4 v[8];
 #pragma unroll
-      for (int i = 0; i < B / 8; ++i) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
-        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        for (int j = 0; j < 8; ++j) {
+          const int c = c0 + j * 256;
+          v[j] = c < total ? __ldg(reinterpret_cast<const uint4*>(x + (c / k8s) * ldx) + (c % k8s))
+                           : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          m = max(m, max(max(v[j].x & 0x7FFFu, (v[j].x >> 16) & 0x7FFFu), max(v[j].y & 0x7FFFu, (v[j].y >> 16) & 0x7FFFu)));
+          m = max(m, max(max(v[j].z & 0x7FFFu, (v[j].z >> 16) & 0x7FFFu), max(v[j].w & 0x7FFFu, (v[j].w >> 16) & 0x7FFFu)));
+        }
       }
-      uint32_t qw[B / 8];
-      quantize_block<B>(w, e4m3 != 0, s, qw, sfb);
-      uint8_t* dst = q + r * ldq + static_cast<int64_t>(kb) * (B / 2);
-      if (B == 32) {
-        *reinterpret_cast<uint4*>(dst) = make_uint4(qw[0], qw[1], qw[2], qw[3]);
-      } else {
-        *reinterpret_cast<uint2*>(dst) = make_uint2(qw[0], qw[1]);
-      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+      __syncthreads();
+      m = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = max(m, red[i]);
+      const float amax = __uint_as_float(m << 16);
+      s = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
     }
-    sf[sf_offset(pr, kb, kb_per_row)] = static_cast<uint8_t>(sfb);
+  }
+  if (tscale_out && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *tscale_out = s;
+  const int r = blockIdx.y;
+  const int kb = blockIdx.x * blockDim.x + threadIdx.x;
+  if (kb < kb_per_row)
+    quantize_unit<B>(x, M, K, ldx, e4m3, s, q, ldq, sf, static_cast<uint32_t>(r) * kb_per_row + kb, kb_per_row,
+                     nullptr, nullptr, 0);
+  if (r == 0) {
+    const int kb4 = kb_per_row / 4;
+    const int pad_words = static_cast<int>(sf_rows - M) * kb4;
+    for (int u = blockIdx.x * blockDim.x + threadIdx.x; u < pad_words; u += gridDim.x * blockDim.x) {
+      const int64_t pr = M + u / kb4;
+      *reinterpret_cast<uint32_t*>(sf + sf_offset(pr, (u % kb4) * 4, kb_per_row)) = 0u;
+    }
   }
 }
 
@@ -240,10 +311,24 @@ cudaError_t launch_group_prologue(const int32_t* offsets, int32_t E, int64_t M, 
   return cudaGetLastError();
 }
 
+// Activations up to this many elements (e.g. 16 x 8192) take the one-CTA path.
+constexpr int64_t kSmallQuantElems = 16 * 8192;
+
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
   const bool e4m3 = a.fmt == MXC_FMT_E4M3_B16;
   const int B = e4m3 ? 16 : 32;
   unsigned int* amax_ws = reinterpret_cast<unsigned int*>(a.ws);
+  if (!a.tile_prefix && a.M * a.K <= kSmallQuantElems) {
+    const dim3 blocks(static_cast<unsigned>((a.K / B + 255) / 256), static_cast<unsigned>(a.M));
+    if (e4m3) {
+      quantize_small_kernel<16><<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint16_t*>(a.x), a.M, a.K, a.ldx, 1,
+                                                            a.tscale_in, a.q, a.ldq, a.sf, a.tscale_out, a.sf_rows);
+    } else {
+      quantize_small_kernel<32><<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint16_t*>(a.x), a.M, a.K, a.ldx, 0,
+                                                            nullptr, a.q, a.ldq, a.sf, a.tscale_out, a.sf_rows);
+    }
+    return cudaGetLastError();
+  }
   if (e4m3 && !a.tscale_in) {
     cudaError_t err = cudaMemsetAsync(amax_ws, 0, sizeof(unsigned int), stream);
     if (err != cudaSuccess) return err;

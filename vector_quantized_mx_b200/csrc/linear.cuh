@@ -52,15 +52,15 @@ constexpr int kSMs = 148;
 
 inline int token_tile(int64_t M) { return M <= kDecodeMaxM ? 16 : 128; }
 
-// Split-K factor of the decode path: enough CTAs to cover the SMs twice, at
-// least two 256-channel stages per CTA, and no empty split.
+// Split-K factor of the decode path: the CTAs of one 128-row output tile form a
+// cluster of `splits`; choose the largest factor (<= kMaxSplits) that keeps all
+// CTAs in one wave, with at least one 256-channel stage per CTA.
 inline void decode_splits(int64_t N, int64_t K, int* splits, int* ks_per_split) {
   const int n_tiles = static_cast<int>(N / kTileN);
   const int KS = static_cast<int>(K / kStageK);
-  int s = (2 * kSMs + n_tiles - 1) / n_tiles;
-  s = s < 1 ? 1 : s;
-  const int smax = KS / 2 > 0 ? KS / 2 : 1;
-  s = s > smax ? smax : s;
+  int s = kSMs / (n_tiles > 0 ? n_tiles : 1);
+  s = s < 1 ? 1 : (s > kMaxSplits ? kMaxSplits : s);
+  s = s > KS ? KS : s;
   const int per = (KS + s - 1) / s;
   *ks_per_split = per;
   *splits = (KS + per - 1) / per;
@@ -68,14 +68,9 @@ inline void decode_splits(int64_t N, int64_t K, int* splits, int* ks_per_split) 
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-size_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int /*fmt*/) {
-  if (M > kDecodeMaxM) return 0;
-  int splits, per;
-  decode_splits(N, K, &splits, &per);
-  if (splits <= 1) return 0;
-  return align_up(static_cast<size_t>(splits) * M * N * sizeof(float), 256) +
-         align_up(static_cast<size_t>(N / kTileN) * sizeof(int), 256);
-}
+// The linear layer keeps its split-K partial sums in cluster shared memory and
+// needs no workspace.
+size_t linear_workspace_bytes(int64_t /*M*/, int64_t /*N*/, int64_t /*K*/, int /*fmt*/) { return 0; }
 
 size_t moe_workspace_bytes(int64_t /*M*/, int32_t E, int64_t /*N*/, int64_t /*K*/, int /*fmt*/) {
   return align_up(static_cast<size_t>(E + 1) * sizeof(int32_t), 256);
@@ -91,7 +86,22 @@ cudaError_t launch_gemm(const CUtensorMap& tx, const CUtensorMap& tw,
   auto kern = gemm_kernel<FMT, WSRC, T, MOE>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (err != cudaSuccess) return err;
-  kern<<<grid, kThreads, L::SMEM, stream>>>(tx, tw, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = L::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  if (p.splits > 1) {                       // the split CTAs of a tile are one cluster
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = static_cast<unsigned>(p.splits);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  err = cudaLaunchKernelEx(&cfg, kern, tx, tw, p);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
@@ -149,18 +159,8 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
   if (T == 16) {
     int splits, per;
     decode_splits(a.N, a.K, &splits, &per);
-    if (splits > 1) {
-      const size_t need = linear_workspace_bytes(a.M, a.N, a.K, a.fmt);
-      if (!a.ws || a.ws_bytes < need) return MXC_ERR_WORKSPACE;
-      p.splits = splits;
-      p.ks_per_split = per;
-      p.partials = reinterpret_cast<float*>(a.ws);
-      p.counters = reinterpret_cast<int*>(reinterpret_cast<char*>(a.ws) +
-                                          align_up(static_cast<size_t>(splits) * a.M * a.N * sizeof(float), 256));
-      if (cudaMemsetAsync(p.counters, 0, static_cast<size_t>(n_tiles) * m_tiles * sizeof(int), stream) !=
-          cudaSuccess)
-        return MXC_ERR_CUDA;
-    }
+    p.splits = splits;
+    p.ks_per_split = per;
   }
   const dim3 grid(n_tiles, m_tiles, p.splits);
   cudaError_t err;
@@ -225,8 +225,7 @@ mxc_status run_moe_linear(const MoeArgs& m, cudaStream_t stream) {
 
 template <int FMT, int WSRC>
 cudaError_t launch_decode_dump(const DecodeArgs& a, cudaStream_t stream) {
-  using L = StageLayout<FMT, WSRC, 16>;
-  constexpr int smem = 1024 + L::CTRL + L::BYTES;
+  constexpr int smem = DumpLayout<FMT, WSRC>::SMEM;
   auto kern = decode_dump_kernel<FMT, WSRC>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;

@@ -10,21 +10,25 @@
 //               copies of its scale atoms, the stage's packed index tile (8 KB),
 //               its QBlock codebook(s) (512 B each) and the weight scales (direct
 //               atoms, or scale-VQ indices).  Native FP4 weights come by TMA.
-//   warps 2..5  decoders: index -> 16-bit codebook entry (4 E2M1 codes) -> 16-byte
-//               chunks of FP4 written straight into the swizzled K-major operand
-//               tile the tensor core reads; PreScale+ scale indices -> scale
+//   warps 2..5  decoders: the stage's codebook is replicated once per lane (so
+//               the random gathers are free of bank conflicts), then every index
+//               becomes a 16-bit codebook entry (4 E2M1 codes) and 16-byte chunks
+//               of FP4 are written straight into the swizzled K-major operand
+//               tile the tensor core reads.  PreScale+ scale indices become scale
 //               bytes in the tcgen05 scale-factor atom layout.  Then epilogue.
 //   warp 1      one thread issues tcgen05.cp (scale atoms -> TMEM) and four
 //               tcgen05.mma block-scaled FP4 MMAs (K = 64 each) per stage into a
 //               128 x T FP32 accumulator in TMEM, and frees the stage with
 //               tcgen05.commit.
 //   epilogue    warps 2..5 read the accumulator with tcgen05.ld, apply the FP32
-//               tensor scales and store FP32/BF16 rows of Y (or split-K partials,
-//               reduced in a fixed order by the last CTA of the tile).
+//               tensor scales and store FP32/BF16 rows of Y.  For split-K (decode)
+//               the CTAs of one output tile form a thread-block cluster: ranks
+//               1.. write their partial tiles into rank 0's shared memory and
+//               rank 0 adds them in rank order (deterministic, no workspace).
 //
 // The weight tile is the MMA's A operand (M = 128 rows of W), the token tile is
 // the B operand (N = T tokens), so one kernel serves decode (T = 16) and
-// prefill (T = 128/256) without a transpose.
+// prefill (T = 128) without a transpose.
 #pragma once
 
 #include "mxc_device.cuh"
@@ -34,6 +38,8 @@ namespace mxc {
 
 enum : int { WSRC_VQ_DIRECT = 0, WSRC_VQ_SVQ = 1, WSRC_NATIVE = 2 };
 enum : int { FMT_E8M0 = 0, FMT_E4M3 = 1 };
+
+constexpr int kMaxSplits = 4;      // cluster split-K factor of the decode path
 
 struct ExpertPtrs {
   const uint8_t* idx;
@@ -55,16 +61,14 @@ struct GemmParams {
   void* y;
   int64_t ldy;
   int out_bf16;
-  int splits, ks_per_split;  // split-K (1 = off)
-  float* partials;           // [splits][M][N] FP32
-  int* counters;             // one per output tile, zero on entry
+  int splits, ks_per_split;  // split-K over a cluster of `splits` CTAs (1 = off)
   int E;                     // MoE
   const int32_t* offsets;
   const int32_t* tile_prefix;
   ExpertPtrs w[NEXP];
 };
 
-// Shared-memory layout of one pipeline stage.
+// Shared-memory layout of one pipeline stage and of the whole CTA.
 template <int FMT, int WSRC, int T>
 struct StageLayout {
   static constexpr bool kVQ = WSRC != WSRC_NATIVE;
@@ -83,9 +87,13 @@ struct StageLayout {
   static constexpr int END = SIDX_OFF + (kSVQ ? 128 * kG : 0);
   static constexpr int BYTES = (END + 1023) / 1024 * 1024;
   static constexpr int CTRL = 4096;                   // barriers, TMEM slot, scale codebook
-  static constexpr int BUDGET = 227 * 1024 - 1024 - CTRL;
+  static constexpr int LUT = kVQ ? 2 * 128 * 32 * 4 : 0;             // two per-lane codebook copies
+  static constexpr int RED = T <= 32 ? (kMaxSplits - 1) * T * 128 * 4 : 0;  // split-K receive slots
+  static constexpr int BUDGET = 227 * 1024 - 1024 - CTRL - LUT - RED;
   static constexpr int STAGES = (BUDGET / BYTES) > 8 ? 8 : (BUDGET / BYTES);
-  static constexpr int SMEM = 1024 + CTRL + STAGES * BYTES;
+  static constexpr int LUT_OFF = CTRL + STAGES * BYTES;
+  static constexpr int RED_OFF = LUT_OFF + LUT;
+  static constexpr int SMEM = 1024 + RED_OFF + RED;
   // TMEM columns: accumulator [0,T), weight scales [T,T+16), token scales after.
   static constexpr int COL_SFW = T;
   static constexpr int COL_SFX = T + 16;
@@ -94,45 +102,67 @@ struct StageLayout {
                                    : COLS_USED <= 256 ? 256 : 512;
   static_assert(STAGES >= 2, "stage does not fit");
   static_assert(T % 16 == 0 && T >= 16 && T <= 256, "token tile");
+  static_assert(SMEM <= 232448, "shared memory");
 };
 
-constexpr int kThreads = 192;   // 6 warps
+constexpr int kDecWarps = 8;                       // decoder / epilogue warps (2 per SM sub-partition)
+constexpr int kDecThreads = 32 * kDecWarps;
+constexpr int kThreads = 64 + kDecThreads;         // + loader warp + MMA warp
 
 // ------------------------------------------------------------------------------------
-// Decoders (shared with the decode-dump kernel)
+// Decoders (shared with the decode-dump kernel).  dt = decoder thread 0..NT-1.
 // ------------------------------------------------------------------------------------
-// One 128 x 256 weight tile: idx [128][64] bytes, codebook(s) of 256 uint16
-// entries (two when the QBlock is 128 wide along K: chunks 0..3 use the first),
-// output FP4 [128][128] bytes in the 128-byte swizzle (16-byte chunk j of row r
-// stored at chunk j ^ (r % 8)).  dt = 0..127.
-__device__ __forceinline__ void decode_w_tile(const uint8_t* __restrict__ idx,
-                                              const uint16_t* __restrict__ cb, bool cb_split,
-                                              uint8_t* __restrict__ wt, int dt) {
-#pragma unroll 2
-  for (int it = 0; it < 8; ++it) {
-    const int c = it * 128 + dt;
+// Per-lane codebook copies: word (w*32 + lane) holds centroids 2w and 2w+1, so the
+// 32 lanes of a warp always read 32 different banks.  `ncb` = 1 or 2 codebooks
+// (two when the QBlock is 128 wide along K).  Stores are 16 B per thread over
+// consecutive addresses (bank-conflict free); the source word is a broadcast.
+template <int NT>
+__device__ __forceinline__ void build_lut(const uint32_t* __restrict__ cbw, int ncb, uint32_t* __restrict__ lut,
+                                          int dt) {
+  for (int u = dt; u < 1024 * ncb; u += NT) {  // uint4 u: words 4u..4u+3 = entry word u/8, lanes 4(u%8)..
+    const uint32_t v = cbw[u >> 3];
+    reinterpret_cast<uint4*>(lut)[u] = make_uint4(v, v, v, v);
+  }
+}
+
+// One 128 x 256 weight tile: idx [128][64] bytes -> FP4 [128][128] bytes in the
+// 128-byte swizzle (16-byte chunk j of row r stored at chunk j ^ (r % 8)).
+// Chunks 0..3 of a row use codebook 0, chunks 4..7 codebook `cb_split`.
+template <int NT>
+__device__ __forceinline__ void decode_w_tile(const uint8_t* __restrict__ idx, const uint32_t* __restrict__ lut,
+                                              int cb_split, uint8_t* __restrict__ wt, int dt) {
+  const int lane = dt & 31;
+  const uint16_t* l16 = reinterpret_cast<const uint16_t*>(lut) + 2 * lane;
+#pragma unroll
+  for (int it = 0; it < 1024 / NT; ++it) {
+    const int c = it * NT + dt;
     const int r = c >> 3, j = c & 7;
     const uint2 iv = *reinterpret_cast<const uint2*>(idx + r * 64 + j * 8);
-    const uint16_t* t = cb + ((cb_split && j >= 4) ? 256 : 0);
-    const uint32_t w0 = t[iv.x & 0xFF] | (static_cast<uint32_t>(t[(iv.x >> 8) & 0xFF]) << 16);
-    const uint32_t w1 = t[(iv.x >> 16) & 0xFF] | (static_cast<uint32_t>(t[iv.x >> 24]) << 16);
-    const uint32_t w2 = t[iv.y & 0xFF] | (static_cast<uint32_t>(t[(iv.y >> 8) & 0xFF]) << 16);
-    const uint32_t w3 = t[(iv.y >> 16) & 0xFF] | (static_cast<uint32_t>(t[iv.y >> 24]) << 16);
+    const uint16_t* t = l16 + ((cb_split && j >= 4) ? 128 * 32 * 2 : 0);
+    // entry e: word (e >> 1) * 32 + lane, half e & 1  ->  16-bit index ((e>>1)*32)*2 + (e&1) from l16
+#define MXC_LUT(e) t[(((e) >> 1) << 6) | ((e) & 1)]
+    const uint32_t b0 = iv.x & 0xFF, b1 = (iv.x >> 8) & 0xFF, b2 = (iv.x >> 16) & 0xFF, b3 = iv.x >> 24;
+    const uint32_t b4 = iv.y & 0xFF, b5 = (iv.y >> 8) & 0xFF, b6 = (iv.y >> 16) & 0xFF, b7 = iv.y >> 24;
+    const uint32_t w0 = MXC_LUT(b0) | (static_cast<uint32_t>(MXC_LUT(b1)) << 16);
+    const uint32_t w1 = MXC_LUT(b2) | (static_cast<uint32_t>(MXC_LUT(b3)) << 16);
+    const uint32_t w2 = MXC_LUT(b4) | (static_cast<uint32_t>(MXC_LUT(b5)) << 16);
+    const uint32_t w3 = MXC_LUT(b6) | (static_cast<uint32_t>(MXC_LUT(b7)) << 16);
+#undef MXC_LUT
     *reinterpret_cast<uint4*>(wt + r * 128 + ((j ^ (r & 7)) << 4)) = make_uint4(w0, w1, w2, w3);
   }
 }
 
-// PreScale+ (Table 4 caption: Ks = 256, ds = 8): the G scale-codebook indices of
-// row dt select 8 scale bytes each, i.e. two 32-bit words of the scale-factor
-// atoms (kb 8g..8g+3 -> atom 2g, kb 8g+4..8g+7 -> atom 2g+1).
-template <int G>
+// PreScale+ (Table 4 caption: Ks = 256, ds = 8): each scale-codebook index
+// selects 8 scale bytes, i.e. two 32-bit words of the scale-factor atoms (kb
+// 8g..8g+3 -> atom 2g, kb 8g+4..8g+7 -> atom 2g+1).  128 rows x G groups.
+template <int G, int NT>
 __device__ __forceinline__ void decode_sf_tile(const uint8_t* __restrict__ sidx,
                                                const uint8_t* __restrict__ scb, uint8_t* __restrict__ sfw,
                                                int dt) {
-  const int word = (dt & 31) * 4 + ((dt >> 5) & 3);
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const uint32_t si = sidx[dt * G + g];
+  for (int u = dt; u < 128 * G; u += NT) {
+    const int r = u & 127, g = u >> 7;
+    const int word = (r & 31) * 4 + ((r >> 5) & 3);
+    const uint32_t si = sidx[r * G + g];
     const uint2 s8 = *reinterpret_cast<const uint2*>(scb + si * 8);
     reinterpret_cast<uint32_t*>(sfw + (2 * g) * 512)[word] = s8.x;
     reinterpret_cast<uint32_t*>(sfw + (2 * g + 1) * 512)[word] = s8.y;
@@ -141,6 +171,29 @@ __device__ __forceinline__ void decode_sf_tile(const uint8_t* __restrict__ sidx,
 
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier that also ANDs a predicate over the participating threads, so a
+// group can take one uniform decision (e.g. all stop after any of them timed out).
+__device__ __forceinline__ bool named_bar_and(int id, int count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pin, pout;\n\t"
+      "setp.ne.u32 pin, %1, 0;\n\t"
+      "bar.red.and.pred pout, %2, %3, pin;\n\t"
+      "selp.u32 %0, 1, 0, pout;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void store_out(void* y, int64_t ldy, int out_bf16, int64_t m, int64_t n, float v) {
+  if (out_bf16) {
+    reinterpret_cast<uint16_t*>(y)[m * ldy + n] = f32_to_bf16_rne(v);
+  } else {
+    reinterpret_cast<float*>(y)[m * ldy + n] = v;
+  }
 }
 
 // ------------------------------------------------------------------------------------
@@ -154,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int STAGES = L::STAGES;
   constexpr int A = L::kAtoms;
   constexpr int XG = L::kXG;
+  constexpr int TCOL = T / 2;                        // accumulator columns per epilogue warp
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -162,13 +216,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = dec + STAGES;
   uint64_t* accum = empty + STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
-  int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);
   uint8_t* scb_smem = smem + 2048;
   uint8_t* stages = smem + L::CTRL;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int KS = p.K / kStageK;
-  const int KB4 = p.K / L::kB / 4;      // scale atoms per 128 rows over all of K
+  const int K = p.K;
+  const int KS = K / kStageK;
+  const int KB4 = K / L::kB / 4;      // scale atoms per 128 rows over all of K
+  const int splits = p.splits;
 
   // ---- which tile this CTA owns ----
   const int n_tile = blockIdx.x;
@@ -196,12 +251,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     ks_end = min(KS, ks_begin + p.ks_per_split);
   }
   const int nks = ks_end - ks_begin;
+  // Loop invariants in registers (the asm statements below clobber "memory").
+  const uint8_t* const w_idx = wp->idx;
+  const uint16_t* const w_cb = wp->cb;
+  const uint8_t* const w_sf = wp->sf;
+  const uint8_t* const w_sidx = wp->sidx;
+  const uint8_t* const w_scb = wp->scb;
+  const float w_tscale0 = wp->w_tscale;
+  const uint8_t* const a_sf = p.a_sf;
+  const int qn = p.qn, qk = p.qk;
 
   // ---- setup ----
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&dec[s], 128);
+      mbar_init(&dec[s], kDecThreads);
       mbar_init(&empty[s], 1);
     }
     mbar_init(accum, 1);
@@ -215,81 +279,107 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if constexpr (L::kSVQ) {
     for (int i = threadIdx.x; i < 512; i += kThreads)
-      reinterpret_cast<uint32_t*>(scb_smem)[i] = __ldg(reinterpret_cast<const uint32_t*>(wp->scb) + i);
+      reinterpret_cast<uint32_t*>(scb_smem)[i] = __ldg(reinterpret_cast<const uint32_t*>(w_scb) + i);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // epilogue state (warps 2..9), kept in registers across the cluster barrier
+  uint32_t acc_regs[T <= 32 ? TCOL : 1];
+  bool ep_ok = false;
+  const int qd = warp & 3;                           // TMEM lane quadrant this warp may read
+  const int chalf = (warp - 2) >> 2;                 // which half of the accumulator columns
+  const int row = qd * 32 + lane;
+  const int64_t n = static_cast<int64_t>(n_tile) * 128 + row;
+  const int64_t mbase = m0 + chalf * TCOL;           // first token of this warp's columns
+  float scale = 1.0f;
+
   if (warp == 0) {
     // =============================== loader ===============================
-    if (lane == 0) {
-      const int qbn = static_cast<int>((static_cast<int64_t>(n_tile) * 128) / p.qn);
-      const int cb_per_row = p.K / p.qk;
-      const bool cb_split = p.qk == 128;
-      uint32_t tx = T * 128 + XG * A * 512;
-      if constexpr (WSRC == WSRC_NATIVE) tx += 16384 + A * 512;
-      if constexpr (WSRC == WSRC_VQ_DIRECT) tx += 8192 + (cb_split ? 1024 : 512) + A * 512;
-      if constexpr (WSRC == WSRC_VQ_SVQ) tx += 8192 + (cb_split ? 1024 : 512) + 128 * L::kG;
-      int issued = 0;
-      for (int i = 0; i < nks; ++i) {
-        const int s = i % STAGES;
-        const uint32_t ph = (i / STAGES) & 1;
-        if (i >= STAGES && !mbar_wait(&empty[s], ph ^ 1)) break;
+    const int qbn = static_cast<int>((static_cast<int64_t>(n_tile) * 128) / qn);
+    const int cb_per_row = K / qk;
+    const bool cb_split = qk == 128;
+    uint32_t tx = T * 128 + XG * A * 512;
+    if constexpr (WSRC == WSRC_NATIVE) tx += 16384 + A * 512;
+    if constexpr (WSRC == WSRC_VQ_DIRECT) tx += 8192 + (cb_split ? 1024 : 512) + A * 512;
+    if constexpr (WSRC == WSRC_VQ_SVQ) tx += 8192 + (cb_split ? 1024 : 512) + 128 * L::kG;
+    const uint8_t* sfx_src = a_sf + static_cast<size_t>(sf_group0) * KB4 * 512;
+    const uint8_t* sfw_src = w_sf + static_cast<size_t>(n_tile) * KB4 * 512;
+    const uint8_t* idx_src = w_idx + static_cast<size_t>(n_tile) * KS * 8192;
+    const uint8_t* sidx_src = w_sidx + static_cast<size_t>(n_tile) * KS * (128 * L::kG);
+    const uint16_t* cb_src = w_cb + static_cast<size_t>(qbn) * cb_per_row * 256;
+    const int y0 = static_cast<int>(m0);
+    int issued = 0;
+    for (int i = 0; i < nks; ++i) {
+      const int s = i % STAGES;
+      const uint32_t ph = (i / STAGES) & 1;
+      if (i >= STAGES && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1))) break;
+      if (elect_one()) {
         const int ks = ks_begin + i;
         uint8_t* st = stages + s * L::BYTES;
         mbar_arrive_expect_tx(&full[s], tx);
-        tma_load_2d(st + L::X_OFF, &tmap_x, ks * 128, static_cast<int>(m0), &full[s]);
+        tma_load_2d(st + L::X_OFF, &tmap_x, ks * 128, y0, &full[s]);
 #pragma unroll
         for (int g = 0; g < XG; ++g)
-          bulk_load(st + L::SFX_OFF + g * A * 512,
-                    p.a_sf + (static_cast<size_t>(sf_group0 + g) * KB4 + static_cast<size_t>(ks) * A) * 512,
+          bulk_load(st + L::SFX_OFF + g * A * 512, sfx_src + (static_cast<size_t>(g) * KB4 + ks * A) * 512,
                     A * 512, &full[s]);
-        const size_t wsf = (static_cast<size_t>(n_tile) * KB4 + static_cast<size_t>(ks) * A) * 512;
         if constexpr (WSRC == WSRC_NATIVE) {
           tma_load_2d(st + L::W_OFF, &tmap_wq, ks * 128, n_tile * 128, &full[s]);
-          bulk_load(st + L::SFW_OFF, wp->sf + wsf, A * 512, &full[s]);
+          bulk_load(st + L::SFW_OFF, sfw_src + static_cast<size_t>(ks) * A * 512, A * 512, &full[s]);
         } else {
-          const size_t tile_id = static_cast<size_t>(n_tile) * KS + ks;
-          bulk_load(st + L::IDX_OFF, wp->idx + tile_id * 8192, 8192, &full[s]);
-          const int qbk = cb_split ? 2 * ks : (ks * kStageK) / p.qk;
-          bulk_load(st + L::CB_OFF, wp->cb + (static_cast<size_t>(qbn) * cb_per_row + qbk) * 256,
-                    cb_split ? 1024 : 512, &full[s]);
+          bulk_load(st + L::IDX_OFF, idx_src + static_cast<size_t>(ks) * 8192, 8192, &full[s]);
+          const int qbk = cb_split ? 2 * ks : (ks * kStageK) / qk;
+          bulk_load(st + L::CB_OFF, cb_src + static_cast<size_t>(qbk) * 256, cb_split ? 1024 : 512, &full[s]);
           if constexpr (WSRC == WSRC_VQ_DIRECT) {
-            bulk_load(st + L::SFW_OFF, wp->sf + wsf, A * 512, &full[s]);
+            bulk_load(st + L::SFW_OFF, sfw_src + static_cast<size_t>(ks) * A * 512, A * 512, &full[s]);
           } else {
-            bulk_load(st + L::SIDX_OFF, wp->sidx + tile_id * (128 * L::kG), 128 * L::kG, &full[s]);
+            bulk_load(st + L::SIDX_OFF, sidx_src + static_cast<size_t>(ks) * (128 * L::kG), 128 * L::kG,
+                      &full[s]);
           }
         }
-        ++issued;
       }
-      // Let every copy this warp started land before the CTA can retire.
-      for (int i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
-        mbar_wait(&full[i % STAGES], (i / STAGES) & 1);
+      __syncwarp();
+      ++issued;
     }
+    // Let every copy this warp started land before the CTA can retire.
+    for (int i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
+      mbar_wait(&full[i % STAGES], (i / STAGES) & 1);
   } else if (warp == 1) {
     // ============================ MMA issuer ==============================
-    if (lane == 0) {
-      for (int i = 0; i < nks; ++i) {
-        const int s = i % STAGES;
-        const uint32_t ph = (i / STAGES) & 1;
-        if (!mbar_wait(&full[s], ph)) break;
-        if constexpr (L::kVQ) {
-          if (!mbar_wait(&dec[s], ph)) break;
-        }
-        fence_proxy_async_smem();
-        tc_fence_after();
-        const uint8_t* st = stages + s * L::BYTES;
-        const uint32_t sfw_s = smem_u32(st + L::SFW_OFF), sfx_s = smem_u32(st + L::SFX_OFF);
-#pragma unroll
-        for (int a = 0; a < A; ++a) tc_cp_32x128b_warpx4(tmem + L::COL_SFW + 4 * a, sdesc_sf_atom(sfw_s + a * 512));
+    for (int i = 0; i < nks; ++i) {
+      const int s = i % STAGES;
+      const uint32_t ph = (i / STAGES) & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) break;
+      tc_fence_after();
+      const uint8_t* st = stages + s * L::BYTES;
+      const uint32_t sfw_s = smem_u32(st + L::SFW_OFF), sfx_s = smem_u32(st + L::SFX_OFF);
+      // Scale atoms that arrived by copy go to TMEM while the decoders work.
+      if (elect_one()) {
 #pragma unroll
         for (int g = 0; g < XG; ++g)
 #pragma unroll
           for (int a = 0; a < A; ++a)
             tc_cp_32x128b_warpx4(tmem + L::COL_SFX + (XG == 2 ? 8 * a + 4 * g : 4 * a),
                                  sdesc_sf_atom(sfx_s + (g * A + a) * 512));
+        if constexpr (!L::kSVQ) {
+#pragma unroll
+          for (int a = 0; a < A; ++a)
+            tc_cp_32x128b_warpx4(tmem + L::COL_SFW + 4 * a, sdesc_sf_atom(sfw_s + a * 512));
+        }
+      }
+      __syncwarp();
+      if constexpr (L::kVQ) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&dec[s], ph))) break;
+        tc_fence_after();
+      }
+      if (elect_one()) {
+        if constexpr (L::kSVQ) {
+#pragma unroll
+          for (int a = 0; a < A; ++a)
+            tc_cp_32x128b_warpx4(tmem + L::COL_SFW + 4 * a, sdesc_sf_atom(sfw_s + a * 512));
+        }
         const uint32_t w_s = smem_u32(st + L::W_OFF), x_s = smem_u32(st + L::X_OFF);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -310,80 +400,77 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit(&empty[s]);
       }
-      tc_commit(accum);
-      mbar_wait(accum, 0);      // our own MMAs must finish before the CTA retires
+      __syncwarp();
     }
+    if (elect_one()) tc_commit(accum);
+    __syncwarp();
+    mbar_wait(accum, 0);      // our own MMAs must finish before the CTA retires
   } else {
     // ======================= decoders, then epilogue ======================
     const int dt = threadIdx.x - 64;
     if constexpr (L::kVQ) {
-      const bool cb_split = p.qk == 128;
+      const int cb_split = qk == 128;
+      uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L::LUT_OFF);
       for (int i = 0; i < nks; ++i) {
         const int s = i % STAGES;
         const uint32_t ph = (i / STAGES) & 1;
-        if (!mbar_wait(&full[s], ph)) break;
+        // one decision for all decoders; also orders the previous stage's lookups
+        // before the codebook copies are rebuilt
+        if (!named_bar_and(2, kDecThreads, mbar_wait(&full[s], ph))) break;
         uint8_t* st = stages + s * L::BYTES;
-        decode_w_tile(st + L::IDX_OFF, reinterpret_cast<const uint16_t*>(st + L::CB_OFF), cb_split,
-                      st + L::W_OFF, dt);
-        if constexpr (L::kSVQ) decode_sf_tile<L::kG>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, dt);
+        build_lut<kDecThreads>(reinterpret_cast<const uint32_t*>(st + L::CB_OFF), 1 + cb_split, lut, dt);
+        named_bar_sync(2, kDecThreads);              // copies visible to all decoders
+        decode_w_tile<kDecThreads>(st + L::IDX_OFF, lut, cb_split, st + L::W_OFF, dt);
+        if constexpr (L::kSVQ) decode_sf_tile<L::kG, kDecThreads>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, dt);
         fence_proxy_async_smem();
         mbar_arrive(&dec[s]);
       }
     }
-    const bool ok = mbar_wait(accum, 0);
+    ep_ok = mbar_wait(accum, 0);
     tc_fence_after();
-    const int qd = warp & 3;                         // TMEM lane quadrant this warp may read
-    const int row = qd * 32 + lane;
-    const int64_t n = static_cast<int64_t>(n_tile) * 128 + row;
-    float wts = wp->w_tscale;
+    float wts = w_tscale0;
     if constexpr (WSRC == WSRC_NATIVE) {
       if (p.w_tscale_dev) wts = *p.w_tscale_dev;
     }
-    const float scale = wts * (p.a_tscale ? *p.a_tscale : 1.0f);
-    const bool partial = p.splits > 1;
-#pragma unroll 1
-    for (int c0 = 0; c0 < T; c0 += 16) {
-      uint32_t v[16];
-      tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(qd * 32) << 16) + c0, v);
+    scale = wts * (p.a_tscale ? *p.a_tscale : 1.0f);
+    void* const y = p.y;
+    const int64_t ldy = p.ldy;
+    const int out_bf16 = p.out_bf16;
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(qd * 32) << 16) + chalf * TCOL;
+    if constexpr (T <= 32) {
+      // this warp's accumulator columns in registers: one TMEM round trip
+      if constexpr (TCOL == 8) tmem_ld_32x32b_x8(taddr, acc_regs);
+      else tmem_ld_32x32b_x16(taddr, acc_regs);
       tmem_ld_wait();
-      if (!ok) continue;
+      if (ep_ok) {
+        if (splits > 1) {
+          const uint32_t rank = cluster_ctarank();
+          if (rank != 0) {
+            // partial tile -> rank 0's receive slot (rank-1), [T][128] floats
+            const uint32_t slot = smem_u32(smem + L::RED_OFF) + (((rank - 1) * T + chalf * TCOL) * 128 + row) * 4;
+            const uint32_t remote = mapa_shared(slot, 0);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const int64_t m = m0 + c0 + c;
-        if (m >= m_end) break;
-        const float acc = __uint_as_float(v[c]);
-        if (partial) {
-          p.partials[(static_cast<size_t>(split) * p.M + m) * p.N + n] = acc;
-        } else if (p.out_bf16) {
-          reinterpret_cast<uint16_t*>(p.y)[m * p.ldy + n] = f32_to_bf16_rne(acc * scale);
-        } else {
-          reinterpret_cast<float*>(p.y)[m * p.ldy + n] = acc * scale;
-        }
-      }
-    }
-    if (partial && ok) {
-      // Split-K: the last CTA of this output tile sums the partials in split order.
-      __threadfence();
-      named_bar_sync(1, 128);
-      if (dt == 0) {
-        const int tile_id = blockIdx.y * gridDim.x + blockIdx.x;
-        *last_flag = atomicAdd(&p.counters[tile_id], 1) == p.splits - 1;
-      }
-      named_bar_sync(1, 128);
-      if (*last_flag) {
-        __threadfence();
-        for (int c = 0; c < T; ++c) {
-          const int64_t m = m0 + c;
-          if (m >= m_end) break;
-          float sum = 0.0f;
-          for (int s2 = 0; s2 < p.splits; ++s2)
-            sum += __ldcg(&p.partials[(static_cast<size_t>(s2) * p.M + m) * p.N + n]);
-          if (p.out_bf16) {
-            reinterpret_cast<uint16_t*>(p.y)[m * p.ldy + n] = f32_to_bf16_rne(sum * scale);
-          } else {
-            reinterpret_cast<float*>(p.y)[m * p.ldy + n] = sum * scale;
+            for (int c = 0; c < TCOL; ++c) st_cluster_f32(remote + c * 128 * 4, __uint_as_float(acc_regs[c]));
           }
+        } else {
+#pragma unroll
+          for (int c = 0; c < TCOL; ++c)
+            if (mbase + c < m_end) store_out(y, ldy, out_bf16, mbase + c, n, __uint_as_float(acc_regs[c]) * scale);
         }
+      }
+    } else {
+#pragma unroll 1
+      for (int c0 = 0; c0 < TCOL; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + c0, v);
+        tmem_ld_wait();
+        if (!ep_ok) continue;
+        const int64_t rem = m_end - (mbase + c0);
+        if (rem <= 0) continue;
+        const int cmax = rem < 32 ? static_cast<int>(rem) : 32;
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (c < cmax) store_out(y, ldy, out_bf16, mbase + c0 + c, n, __uint_as_float(v[c]) * scale);
       }
     }
   }
@@ -395,12 +482,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);
   }
+  if constexpr (T <= 32 && !MOE) {
+    if (splits > 1) {
+      // All partial tiles have landed in rank 0's shared memory after this barrier.
+      __syncwarp();
+      cluster_sync_all();
+      if (warp >= 2 && ep_ok && cluster_ctarank() == 0) {
+        const float* red = reinterpret_cast<const float*>(smem + L::RED_OFF);
+#pragma unroll
+        for (int c = 0; c < TCOL; ++c) {
+          float sum = __uint_as_float(acc_regs[c]);
+          for (int r = 1; r < splits; ++r) sum += red[((r - 1) * T + chalf * TCOL + c) * 128 + row];
+          if (mbase + c < m_end) store_out(p.y, p.ldy, p.out_bf16, mbase + c, n, sum * scale);
+        }
+      }
+    }
+  }
 }
 
 // ------------------------------------------------------------------------------------
 // Decode dump: the decoders of gemm_kernel, with the stage written back to global
 // memory in plain layouts (FP4 matrix, SF layout).  Grid (N/128, K/256), 160 threads.
 // ------------------------------------------------------------------------------------
+template <int FMT, int WSRC>
+struct DumpLayout {
+  using L = StageLayout<FMT, WSRC, 16>;
+  static constexpr int LUT_OFF = L::CTRL + L::BYTES;
+  static constexpr int SMEM = 1024 + LUT_OFF + 2 * 128 * 32 * 4;
+};
+
 template <int FMT, int WSRC>
 __global__ void __launch_bounds__(160)
     decode_dump_kernel(const ExpertPtrs w, int N, int K, int qn, int qk, uint8_t* __restrict__ q_out,
@@ -412,9 +522,10 @@ __global__ void __launch_bounds__(160)
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
   uint8_t* scb_smem = smem + 2048;
   uint8_t* st = smem + L::CTRL;
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + DumpLayout<FMT, WSRC>::LUT_OFF);
   const int n_tile = blockIdx.x, ks = blockIdx.y;
   const int KS = K / kStageK, KB4 = K / L::kB / 4;
-  const bool cb_split = qk == 128;
+  const int cb_split = qk == 128;
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
@@ -441,14 +552,15 @@ __global__ void __launch_bounds__(160)
     }
   }
   const bool ok = mbar_wait(bar, 0);
+  const int dt = threadIdx.x - 32;
+  if (threadIdx.x >= 32 && ok) build_lut<128>(reinterpret_cast<const uint32_t*>(st + L::CB_OFF), 1 + cb_split, lut, dt);
+  __syncthreads();
   if (threadIdx.x >= 32 && ok) {
-    const int dt = threadIdx.x - 32;
-    decode_w_tile(st + L::IDX_OFF, reinterpret_cast<const uint16_t*>(st + L::CB_OFF), cb_split, st + L::W_OFF, dt);
-    if constexpr (L::kSVQ) decode_sf_tile<L::kG>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, dt);
+    decode_w_tile<128>(st + L::IDX_OFF, lut, cb_split, st + L::W_OFF, dt);
+    if constexpr (L::kSVQ) decode_sf_tile<L::kG, 128>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, dt);
   }
   __syncthreads();
   if (threadIdx.x >= 32 && ok) {
-    const int dt = threadIdx.x - 32;
     for (int it = 0; it < 8; ++it) {
       const int c = it * 128 + dt;
       const int r = c >> 3, j = c & 7;
