@@ -237,6 +237,26 @@ mxc_status mxc_moe_linear(const mxc_mx_tensor* a, const int32_t* d_offsets, cons
                           int32_t E, void* y, int64_t ldy, mxc_dtype y_dtype, void* ws,
                           size_t ws_bytes, mxc_stream_t stream);
 
+/* mxc_moe_linear for callers that cannot allocate device memory: code that
+ * runs inside a CUDA stream capture, plugin hosts and real-time serving loops
+ * that forbid allocator calls, or C callers with no device allocator at hand.
+ * The paper has no counterpart to this entry point; it exists for the calling
+ * environment only.  It takes the same arguments as mxc_moe_linear minus the
+ * workspace, and runs the same kernels.
+ * Scratch: the per-call expert tile table lives in a fixed module-global array
+ * in device memory, held by every GPU that loads the library until the process
+ * exits.  Limit: E <= 256 experts; larger E returns MXC_ERR_UNSUPPORTED and
+ * enqueues nothing.
+ * The first call on each device looks up that array's device address (no
+ * allocation); make the first call on a device before any stream capture that
+ * includes this entry point.  Every call rewrites the table before reading it,
+ * so nothing needs clearing between calls, but all calls on a device share the
+ * array: calls whose executions overlap on the GPU (e.g. on two streams without
+ * ordering between them) race.  The function calls no cudaMalloc, cudaFree or
+ * other allocating routine. */
+mxc_status mxc_moe_linear_noalloc(const mxc_mx_tensor* a, const int32_t* d_offsets, const mxc_weight* experts,
+                                  int32_t E, void* y, int64_t ldy, mxc_dtype y_dtype, mxc_stream_t stream);
+
 /* Runs the weight decode of mxc_linear (index -> codebook -> FP4 tile and
  * scale decode, through shared memory) and writes the result out in plain
  * layouts: q_out FP4 matrix [N, ldq], sf_out the SF layout of [N, K/B].

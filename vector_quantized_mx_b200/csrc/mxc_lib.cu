@@ -3,6 +3,7 @@
 // The whole library is one translation unit (this file includes the kernels), so
 // the per-device error word is an ordinary module global.  Entry points validate
 // their arguments on the host, then enqueue kernels on the caller's stream.
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
@@ -361,6 +362,52 @@ mxc_status mxc_moe_linear(const mxc_mx_tensor* a, const int32_t* d_offsets, cons
   m.E = E;
   m.experts = experts;
   return run_moe_linear(m, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------------------
+// Allocation-free MoE entry point: the expert tile table (E+1 int32) lives in a
+// fixed module-global array instead of a caller workspace.
+// ------------------------------------------------------------------------------------
+namespace {
+
+constexpr int kNoallocScratchInts = kMaxGroups + 1;   // largest table: 256 experts
+static __device__ __align__(256) int32_t g_moe_noalloc_scratch[kNoallocScratchInts];
+
+constexpr int kMaxDevices = 64;
+std::atomic<int32_t*> g_noalloc_ptr[kMaxDevices];
+
+// Device address of g_moe_noalloc_scratch on the current device (looked up once
+// per device; a host-side name of a __device__ array is not a device address).
+mxc_status noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MXC_ERR_NO_DEVICE;
+  int32_t* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_moe_noalloc_scratch) != cudaSuccess || !addr) return MXC_ERR_CUDA;
+    p = static_cast<int32_t*>(addr);
+    g_noalloc_ptr[dev].store(p, std::memory_order_release);
+  }
+  *out = p;
+  return MXC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mxc_status mxc_moe_linear_noalloc(const mxc_mx_tensor* a, const int32_t* d_offsets, const mxc_weight* experts,
+                                  int32_t E, void* y, int64_t ldy, mxc_dtype y_dtype, mxc_stream_t stream) {
+  if (E > kNoallocScratchInts - 1) return MXC_ERR_UNSUPPORTED;
+  if (!a || !d_offsets || !experts || E <= 0) return MXC_ERR_INVALID_ARG;
+  mxc_status s = check_device();
+  if (s != MXC_OK) return s;
+  int32_t* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != MXC_OK) return s;
+  return mxc_moe_linear(a, d_offsets, experts, E, y, ldy, y_dtype, scratch,
+                        sizeof(int32_t) * kNoallocScratchInts, stream);
 }
 
 mxc_status mxc_decode_weight(const mxc_weight* w, uint8_t* q_out, int64_t ldq, uint8_t* sf_out, mxc_stream_t stream) {

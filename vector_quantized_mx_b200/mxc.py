@@ -30,7 +30,7 @@ EXPORTED = (
     "mxc_status_string", "mxc_version", "mxc_sf_bytes", "mxc_packed_weight_sizes", "mxc_pack_weight",
     "mxc_quantize_act_workspace_bytes", "mxc_linear_workspace_bytes", "mxc_moe_workspace_bytes",
     "mxc_grouped_sf_rows_bound", "mxc_quantize_act", "mxc_quantize_act_grouped", "mxc_linear",
-    "mxc_native_linear", "mxc_moe_linear", "mxc_decode_weight", "mxc_get_device_error",
+    "mxc_native_linear", "mxc_moe_linear", "mxc_moe_linear_noalloc", "mxc_decode_weight", "mxc_get_device_error",
 )
 
 
@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
                                                  ctypes.c_int, vp, sz, vp]),
             "mxc_moe_linear": (ctypes.c_int, [ctypes.POINTER(_MxTensor), vp, ctypes.POINTER(_Weight), i32, vp, i64,
                                               ctypes.c_int, vp, sz, vp]),
+            "mxc_moe_linear_noalloc": (ctypes.c_int, [ctypes.POINTER(_MxTensor), vp, ctypes.POINTER(_Weight), i32,
+                                                      vp, i64, ctypes.c_int, vp]),
             "mxc_decode_weight": (ctypes.c_int, [ctypes.POINTER(_Weight), vp, i64, vp, vp]),
             "mxc_get_device_error": (ctypes.c_int, [vp]),
         }
@@ -306,6 +308,19 @@ def moe_linear(a: MXTensor, offsets: torch.Tensor, experts: Sequence[PackedWeigh
     at = a._c()
     _check(lib().mxc_moe_linear(ctypes.byref(at), offsets.data_ptr(), table, E, y.data_ptr(), y.stride(0),
                                 OUT[y.dtype], ws.data_ptr(), ws.numel(), _stream(stream)), "mxc_moe_linear")
+    return y
+
+
+def moe_linear_noalloc(a: MXTensor, offsets: torch.Tensor, experts: Sequence[PackedWeight],
+                       out_dtype=torch.float32, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """mxc_moe_linear_noalloc: mxc_moe_linear without a caller workspace (for callers that
+    cannot allocate device memory); the library uses a fixed device array instead."""
+    E = len(experts)
+    y = _out(a.rows, experts[0].N, out_dtype, a.q.device) if y is None else y
+    table = (_Weight * E)(*[w._c() for w in experts])
+    at = a._c()
+    _check(lib().mxc_moe_linear_noalloc(ctypes.byref(at), offsets.data_ptr(), table, E, y.data_ptr(), y.stride(0),
+                                        OUT[y.dtype], _stream(stream)), "mxc_moe_linear_noalloc")
     return y
 
 
