@@ -324,13 +324,12 @@ def run_gpu(args, rank, world, dist):
     if rank != 0:
         return
     traffic = None
-    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    prof = os.path.join(ROOT, "profiles", "traffic.txt")   # ncu dram read+write of one launch
     if os.path.exists(prof):
-        try:
-            with open(prof) as f:
-                traffic = json.load(f).get("decode_gemv_m16_bytes_per_launch")
-        except Exception:
-            traffic = None
+        for line in open(prof):
+            parts = line.split()
+            if len(parts) == 2 and parts[0] == "decode_gemv_m16_bytes_per_launch":
+                traffic = int(parts[1])
     out = {
         "metric": "MXCode W4A4 effective weight bandwidth (compressed bytes/s)",
         "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": warmup,
