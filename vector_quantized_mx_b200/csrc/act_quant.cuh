@@ -212,65 +212,75 @@ __global__ void __launch_bounds__(256) quantize_kernel(
     quantize_unit<B>(x, M, K, ldx, e4m3, s, q, ldq, sf, u, kb_per_row, offsets, tile_prefix, n_groups);
 }
 
-// Small activations (decode batches): one launch, grid (KB/256 blocks, rows).
-// Every CTA computes the tensor amax itself (the tensor is at most a few hundred
-// KB and sits in L2) and then quantizes blocks of its row; the CTAs of row 0 also
-// clear the padding scale rows [M, round_up(M,128)) a 32-bit word at a time.
+// Small activations (decode batches): one launch of one 8-CTA cluster.  Each CTA
+// reduces 1/8 of the tensor to a partial amax, the partials are exchanged through
+// distributed shared memory (so each CTA reads only its share, and the loads of
+// one thread are all in flight together), then the CTAs quantize interleaved
+// blocks and clear the padding scale rows [M, round_up(M,128)) word by word.
+constexpr int kSmallQuantCtas = 8;
+constexpr int kSmallQuantThreads = 512;
+
 template <int B>
-__global__ void __launch_bounds__(256) quantize_small_kernel(
+__global__ void __launch_bounds__(kSmallQuantThreads) quantize_small_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t K, int64_t ldx, int e4m3,
     const float* __restrict__ tscale_in, uint8_t* __restrict__ q, int64_t ldq, uint8_t* __restrict__ sf,
     float* __restrict__ tscale_out, int64_t sf_rows) {
-  __shared__ uint32_t red[8];
+  __shared__ uint32_t red[kSmallQuantThreads / 32];
+  __shared__ uint32_t partial;
   const int kb_per_row = static_cast<int>(K / B);
-  const int rows = static_cast<int>(M), k8s = static_cast<int>(K / 8);
+  const int k8s = static_cast<int>(K / 8);
+  const uint32_t rank = cluster_ctarank();
+  const bool need_amax = e4m3 && !tscale_in;
   float s = 1.0f;
-  if (e4m3) {
-    if (tscale_in) {
-      s = *tscale_in;
-    } else {
-      // 8 independent 16-byte loads in flight per thread (a small grid cannot hide
-      // L2 latency with other warps)
-      uint32_t m = 0;
-      const int total = rows * k8s;
-      for (int c0 = threadIdx.x; c0 < total; c0 += 8 * 256) {
-        uint4 v[8];
+  if (e4m3 && tscale_in) s = *tscale_in;
+  if (need_amax) {
+    const int total = static_cast<int>(M) * k8s;
+    const int per = (total + kSmallQuantCtas - 1) / kSmallQuantCtas;
+    const int c_begin = static_cast<int>(rank) * per, c_end = min(total, c_begin + per);
+    uint32_t m = 0;
+    for (int c0 = c_begin + threadIdx.x; c0 < c_end; c0 += 4 * kSmallQuantThreads) {
+      uint4 v[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int c = c0 + j * 256;
-          v[j] = c < total ? __ldg(reinterpret_cast<const uint4*>(x + (c / k8s) * ldx) + (c % k8s))
-                           : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          m = max(m, max(max(v[j].x & 0x7FFFu, (v[j].x >> 16) & 0x7FFFu), max(v[j].y & 0x7FFFu, (v[j].y >> 16) & 0x7FFFu)));
-          m = max(m, max(max(v[j].z & 0x7FFFu, (v[j].z >> 16) & 0x7FFFu), max(v[j].w & 0x7FFFu, (v[j].w >> 16) & 0x7FFFu)));
-        }
+      for (int j = 0; j < 4; ++j) {
+        const int c = c0 + j * kSmallQuantThreads;
+        v[j] = c < c_end ? __ldg(reinterpret_cast<const uint4*>(x + (c / k8s) * ldx) + (c % k8s))
+                         : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-      if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-      __syncthreads();
-      m = 0;
+      for (int j = 0; j < 4; ++j) {
+        m = max(m, max(max(v[j].x & 0x7FFFu, (v[j].x >> 16) & 0x7FFFu), max(v[j].y & 0x7FFFu, (v[j].y >> 16) & 0x7FFFu)));
+        m = max(m, max(max(v[j].z & 0x7FFFu, (v[j].z >> 16) & 0x7FFFu), max(v[j].w & 0x7FFFu, (v[j].w >> 16) & 0x7FFFu)));
+      }
+    }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m = max(m, red[i]);
-      const float amax = __uint_as_float(m << 16);
-      s = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint32_t mm = 0;
+#pragma unroll
+      for (int i = 0; i < kSmallQuantThreads / 32; ++i) mm = max(mm, red[i]);
+      partial = mm;
     }
+    cluster_sync_all();                      // every CTA's partial is in its shared memory
+    uint32_t mm = 0;
+    const uint32_t local = smem_u32(&partial);
+#pragma unroll
+    for (int r = 0; r < kSmallQuantCtas; ++r) mm = max(mm, ld_cluster_u32(mapa_shared(local, r)));
+    cluster_sync_all();                      // no CTA leaves while others still read it
+    const float amax = __uint_as_float(mm << 16);
+    s = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
   }
-  if (tscale_out && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *tscale_out = s;
-  const int r = blockIdx.y;
-  const int kb = blockIdx.x * blockDim.x + threadIdx.x;
-  if (kb < kb_per_row)
-    quantize_unit<B>(x, M, K, ldx, e4m3, s, q, ldq, sf, static_cast<uint32_t>(r) * kb_per_row + kb, kb_per_row,
-                     nullptr, nullptr, 0);
-  if (r == 0) {
-    const int kb4 = kb_per_row / 4;
-    const int pad_words = static_cast<int>(sf_rows - M) * kb4;
-    for (int u = blockIdx.x * blockDim.x + threadIdx.x; u < pad_words; u += gridDim.x * blockDim.x) {
-      const int64_t pr = M + u / kb4;
-      *reinterpret_cast<uint32_t*>(sf + sf_offset(pr, (u % kb4) * 4, kb_per_row)) = 0u;
-    }
+  if (tscale_out && rank == 0 && threadIdx.x == 0) *tscale_out = s;
+  const uint32_t stride = kSmallQuantCtas * kSmallQuantThreads;
+  const uint32_t data_units = static_cast<uint32_t>(M) * kb_per_row;
+  for (uint32_t u = rank * kSmallQuantThreads + threadIdx.x; u < data_units; u += stride)
+    quantize_unit<B>(x, M, K, ldx, e4m3, s, q, ldq, sf, u, kb_per_row, nullptr, nullptr, 0);
+  const int kb4 = kb_per_row / 4;
+  const uint32_t pad_words = static_cast<uint32_t>(sf_rows - M) * kb4;
+  for (uint32_t u = rank * kSmallQuantThreads + threadIdx.x; u < pad_words; u += stride) {
+    const int64_t pr = M + u / kb4;
+    *reinterpret_cast<uint32_t*>(sf + sf_offset(pr, static_cast<int>(u % kb4) * 4, kb_per_row)) = 0u;
   }
 }
 
@@ -319,14 +329,27 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
   const int B = e4m3 ? 16 : 32;
   unsigned int* amax_ws = reinterpret_cast<unsigned int*>(a.ws);
   if (!a.tile_prefix && a.M * a.K <= kSmallQuantElems) {
-    const dim3 blocks(static_cast<unsigned>((a.K / B + 255) / 256), static_cast<unsigned>(a.M));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kSmallQuantCtas);
+    cfg.blockDim = dim3(kSmallQuantThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kSmallQuantCtas;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const uint16_t* xp = reinterpret_cast<const uint16_t*>(a.x);
+    cudaError_t err;
     if (e4m3) {
-      quantize_small_kernel<16><<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint16_t*>(a.x), a.M, a.K, a.ldx, 1,
-                                                            a.tscale_in, a.q, a.ldq, a.sf, a.tscale_out, a.sf_rows);
+      err = cudaLaunchKernelEx(&cfg, quantize_small_kernel<16>, xp, a.M, a.K, a.ldx, 1, a.tscale_in, a.q, a.ldq,
+                               a.sf, a.tscale_out, a.sf_rows);
     } else {
-      quantize_small_kernel<32><<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint16_t*>(a.x), a.M, a.K, a.ldx, 0,
-                                                            nullptr, a.q, a.ldq, a.sf, a.tscale_out, a.sf_rows);
+      err = cudaLaunchKernelEx(&cfg, quantize_small_kernel<32>, xp, a.M, a.K, a.ldx, 0,
+                               static_cast<const float*>(nullptr), a.q, a.ldq, a.sf, a.tscale_out, a.sf_rows);
     }
+    if (err != cudaSuccess) return err;
     return cudaGetLastError();
   }
   if (e4m3 && !a.tscale_in) {

@@ -79,11 +79,11 @@ size_t moe_workspace_bytes(int64_t /*M*/, int32_t E, int64_t /*N*/, int64_t /*K*
 // ------------------------------------------------------------------------------------
 // Launch
 // ------------------------------------------------------------------------------------
-template <int FMT, int WSRC, int T, bool MOE>
-cudaError_t launch_gemm(const CUtensorMap& tx, const CUtensorMap& tw,
-                        const GemmParams<MOE ? kMaxGroups : 1>& p, dim3 grid, cudaStream_t stream) {
-  using L = StageLayout<FMT, WSRC, T>;
-  auto kern = gemm_kernel<FMT, WSRC, T, MOE>;
+template <int FMT, int WSRC, int T, bool MOE, int NCB>
+cudaError_t launch_gemm_ncb(const CUtensorMap& tx, const CUtensorMap& tw,
+                            const GemmParams<MOE ? kMaxGroups : 1>& p, dim3 grid, cudaStream_t stream) {
+  using L = StageLayout<FMT, WSRC, T, NCB>;
+  auto kern = gemm_kernel<FMT, WSRC, T, MOE, NCB>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -103,6 +103,16 @@ cudaError_t launch_gemm(const CUtensorMap& tx, const CUtensorMap& tw,
   err = cudaLaunchKernelEx(&cfg, kern, tx, tw, p);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
+}
+
+// Two codebooks per stage only for VQ weights whose QBlock is 128 wide along K.
+template <int FMT, int WSRC, int T, bool MOE>
+cudaError_t launch_gemm(const CUtensorMap& tx, const CUtensorMap& tw,
+                        const GemmParams<MOE ? kMaxGroups : 1>& p, dim3 grid, cudaStream_t stream) {
+  if constexpr (WSRC != WSRC_NATIVE) {
+    if (p.qk == 128) return launch_gemm_ncb<FMT, WSRC, T, MOE, 2>(tx, tw, p, grid, stream);
+  }
+  return launch_gemm_ncb<FMT, WSRC, T, MOE, 1>(tx, tw, p, grid, stream);
 }
 
 template <int FMT, int WSRC, int T>

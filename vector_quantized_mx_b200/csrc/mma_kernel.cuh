@@ -68,8 +68,9 @@ struct GemmParams {
   ExpertPtrs w[NEXP];
 };
 
-// Shared-memory layout of one pipeline stage and of the whole CTA.
-template <int FMT, int WSRC, int T>
+// Shared-memory layout of one pipeline stage and of the whole CTA.  NCB = codebooks
+// per 256-channel stage: 2 when the QBlock is 128 wide along K, else 1.
+template <int FMT, int WSRC, int T, int NCB = 1>
 struct StageLayout {
   static constexpr bool kVQ = WSRC != WSRC_NATIVE;
   static constexpr bool kSVQ = WSRC == WSRC_VQ_SVQ;
@@ -87,7 +88,7 @@ struct StageLayout {
   static constexpr int END = SIDX_OFF + (kSVQ ? 128 * kG : 0);
   static constexpr int BYTES = (END + 1023) / 1024 * 1024;
   static constexpr int CTRL = 4096;                   // barriers, TMEM slot, scale codebook
-  static constexpr int LUT = kVQ ? 2 * 128 * 32 * 4 : 0;             // two per-lane codebook copies
+  static constexpr int LUT = kVQ ? NCB * 256 * 32 * 4 : 0;           // per-lane codebook copies (32 KB each)
   static constexpr int RED = T <= 32 ? (kMaxSplits - 1) * T * 128 * 4 : 0;  // split-K receive slots
   static constexpr int BUDGET = 227 * 1024 - 1024 - CTRL - LUT - RED;
   static constexpr int STAGES = (BUDGET / BYTES) > 8 ? 8 : (BUDGET / BYTES);
@@ -105,50 +106,71 @@ struct StageLayout {
   static_assert(SMEM <= 232448, "shared memory");
 };
 
-constexpr int kDecWarps = 8;                       // decoder / epilogue warps (2 per SM sub-partition)
+#ifndef MXC_DEC_WARPS
+#define MXC_DEC_WARPS 16
+#endif
+constexpr int kDecWarps = MXC_DEC_WARPS;           // decoder / epilogue warps (4 per SM sub-partition)
+constexpr int kColGroups = kDecWarps / 4;          // epilogue warps per TMEM lane quadrant
 constexpr int kDecThreads = 32 * kDecWarps;
 constexpr int kThreads = 64 + kDecThreads;         // + loader warp + MMA warp
 
 // ------------------------------------------------------------------------------------
 // Decoders (shared with the decode-dump kernel).  dt = decoder thread 0..NT-1.
 // ------------------------------------------------------------------------------------
-// Per-lane codebook copies: word (w*32 + lane) holds centroids 2w and 2w+1, so the
-// 32 lanes of a warp always read 32 different banks.  `ncb` = 1 or 2 codebooks
-// (two when the QBlock is 128 wide along K).  Stores are 16 B per thread over
-// consecutive addresses (bank-conflict free); the source word is a broadcast.
+// Per-lane codebook copies: 32-bit word (e*32 + lane) holds centroid e (its 16-bit
+// entry, zero-extended), so the 32 lanes of a warp always read 32 different banks
+// and a lookup is one byte extract, one shift-add and one shared load.  `ncb` = 1
+// or 2 codebooks (two when the QBlock is 128 wide along K), 32 KB each.  Stores
+// are 16 B per thread over consecutive addresses (bank-conflict free).
 template <int NT>
-__device__ __forceinline__ void build_lut(const uint32_t* __restrict__ cbw, int ncb, uint32_t* __restrict__ lut,
+__device__ __forceinline__ void build_lut(const uint16_t* __restrict__ cb, int ncb, uint32_t* __restrict__ lut,
                                           int dt) {
-  for (int u = dt; u < 1024 * ncb; u += NT) {  // uint4 u: words 4u..4u+3 = entry word u/8, lanes 4(u%8)..
-    const uint32_t v = cbw[u >> 3];
+  for (int u = dt; u < 2048 * ncb; u += NT) {   // uint4 u: words 4u..4u+3 = entry u/8, lanes 4(u%8)..
+    const uint32_t v = cb[u >> 3];
     reinterpret_cast<uint4*>(lut)[u] = make_uint4(v, v, v, v);
   }
 }
 
+// Byte k of w, zero-extended.
+__device__ __forceinline__ uint32_t byte_of(uint32_t w, int k) { return __byte_perm(w, 0u, 0x4440 | k); }
+
 // One 128 x 256 weight tile: idx [128][64] bytes -> FP4 [128][128] bytes in the
 // 128-byte swizzle (16-byte chunk j of row r stored at chunk j ^ (r % 8)).
-// Chunks 0..3 of a row use codebook 0, chunks 4..7 codebook `cb_split`.
+// Thread dt owns chunks it*NT + dt; their shared-memory offsets are fixed per
+// thread and computed once (ChunkMap).  Chunks 0..3 of a row use codebook 0,
+// chunks 4..7 codebook 1 when the QBlock is 128 wide along K.
 template <int NT>
-__device__ __forceinline__ void decode_w_tile(const uint8_t* __restrict__ idx, const uint32_t* __restrict__ lut,
-                                              int cb_split, uint8_t* __restrict__ wt, int dt) {
-  const int lane = dt & 31;
-  const uint16_t* l16 = reinterpret_cast<const uint16_t*>(lut) + 2 * lane;
+struct ChunkMap {
+  static constexpr int kN = 1024 / NT;
+  uint32_t idx_off[kN];   // byte offset into the index tile
+  uint32_t w_off[kN];     // byte offset into the swizzled FP4 tile
+  uint32_t lut_off[kN];   // byte offset of this lane's codebook copy (codebook 0 or 1)
+  __device__ __forceinline__ void init(int dt, int cb_split) {
 #pragma unroll
-  for (int it = 0; it < 1024 / NT; ++it) {
-    const int c = it * NT + dt;
-    const int r = c >> 3, j = c & 7;
-    const uint2 iv = *reinterpret_cast<const uint2*>(idx + r * 64 + j * 8);
-    const uint16_t* t = l16 + ((cb_split && j >= 4) ? 128 * 32 * 2 : 0);
-    // entry e: word (e >> 1) * 32 + lane, half e & 1  ->  16-bit index ((e>>1)*32)*2 + (e&1) from l16
-#define MXC_LUT(e) t[(((e) >> 1) << 6) | ((e) & 1)]
-    const uint32_t b0 = iv.x & 0xFF, b1 = (iv.x >> 8) & 0xFF, b2 = (iv.x >> 16) & 0xFF, b3 = iv.x >> 24;
-    const uint32_t b4 = iv.y & 0xFF, b5 = (iv.y >> 8) & 0xFF, b6 = (iv.y >> 16) & 0xFF, b7 = iv.y >> 24;
-    const uint32_t w0 = MXC_LUT(b0) | (static_cast<uint32_t>(MXC_LUT(b1)) << 16);
-    const uint32_t w1 = MXC_LUT(b2) | (static_cast<uint32_t>(MXC_LUT(b3)) << 16);
-    const uint32_t w2 = MXC_LUT(b4) | (static_cast<uint32_t>(MXC_LUT(b5)) << 16);
-    const uint32_t w3 = MXC_LUT(b6) | (static_cast<uint32_t>(MXC_LUT(b7)) << 16);
+    for (int it = 0; it < kN; ++it) {
+      const int c = it * NT + dt;
+      const int r = c >> 3, j = c & 7;
+      idx_off[it] = r * 64 + j * 8;
+      w_off[it] = r * 128 + ((j ^ (r & 7)) << 4);
+      lut_off[it] = ((cb_split && j >= 4) ? 256 * 32 * 4 : 0) + (dt & 31) * 4;
+    }
+  }
+};
+
+template <int NT>
+__device__ __forceinline__ void decode_w_tile(const uint8_t* __restrict__ idx, uint32_t lut_s,
+                                              uint8_t* __restrict__ wt, const ChunkMap<NT>& cm) {
+#pragma unroll
+  for (int it = 0; it < ChunkMap<NT>::kN; ++it) {
+    const uint2 iv = *reinterpret_cast<const uint2*>(idx + cm.idx_off[it]);
+    const uint32_t base = lut_s + cm.lut_off[it];
+#define MXC_LUT(w, k) lds_u32(base + (byte_of(w, k) << 7))
+    const uint32_t e0 = MXC_LUT(iv.x, 0), e1 = MXC_LUT(iv.x, 1), e2 = MXC_LUT(iv.x, 2), e3 = MXC_LUT(iv.x, 3);
+    const uint32_t e4 = MXC_LUT(iv.y, 0), e5 = MXC_LUT(iv.y, 1), e6 = MXC_LUT(iv.y, 2), e7 = MXC_LUT(iv.y, 3);
 #undef MXC_LUT
-    *reinterpret_cast<uint4*>(wt + r * 128 + ((j ^ (r & 7)) << 4)) = make_uint4(w0, w1, w2, w3);
+    *reinterpret_cast<uint4*>(wt + cm.w_off[it]) =
+        make_uint4(__byte_perm(e0, e1, 0x5410), __byte_perm(e2, e3, 0x5410), __byte_perm(e4, e5, 0x5410),
+                   __byte_perm(e6, e7, 0x5410));
   }
 }
 
@@ -199,15 +221,15 @@ __device__ __forceinline__ void store_out(void* y, int64_t ldy, int out_bf16, in
 // ------------------------------------------------------------------------------------
 // The kernel
 // ------------------------------------------------------------------------------------
-template <int FMT, int WSRC, int T, bool MOE>
+template <int FMT, int WSRC, int T, bool MOE, int NCB>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_wq,
                 const __grid_constant__ GemmParams<MOE ? kMaxGroups : 1> p) {
-  using L = StageLayout<FMT, WSRC, T>;
+  using L = StageLayout<FMT, WSRC, T, NCB>;
   constexpr int STAGES = L::STAGES;
   constexpr int A = L::kAtoms;
   constexpr int XG = L::kXG;
-  constexpr int TCOL = T / 2;                        // accumulator columns per epilogue warp
+  constexpr int TCOL = T / kColGroups;               // accumulator columns per epilogue warp
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -265,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&dec[s], kDecThreads);
+      mbar_init(&dec[s], kDecWarps);
       mbar_init(&empty[s], 1);
     }
     mbar_init(accum, 1);
@@ -290,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t acc_regs[T <= 32 ? TCOL : 1];
   bool ep_ok = false;
   const int qd = warp & 3;                           // TMEM lane quadrant this warp may read
-  const int chalf = (warp - 2) >> 2;                 // which half of the accumulator columns
+  const int chalf = (warp - 2) >> 2;                 // which column group of the accumulator
   const int row = qd * 32 + lane;
   const int64_t n = static_cast<int64_t>(n_tile) * 128 + row;
   const int64_t mbase = m0 + chalf * TCOL;           // first token of this warp's columns
@@ -300,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // =============================== loader ===============================
     const int qbn = static_cast<int>((static_cast<int64_t>(n_tile) * 128) / qn);
     const int cb_per_row = K / qk;
-    const bool cb_split = qk == 128;
+    constexpr bool cb_split = NCB == 2;
     uint32_t tx = T * 128 + XG * A * 512;
     if constexpr (WSRC == WSRC_NATIVE) tx += 16384 + A * 512;
     if constexpr (WSRC == WSRC_VQ_DIRECT) tx += 8192 + (cb_split ? 1024 : 512) + A * 512;
@@ -409,8 +431,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ======================= decoders, then epilogue ======================
     const int dt = threadIdx.x - 64;
     if constexpr (L::kVQ) {
-      const int cb_split = qk == 128;
+      constexpr int cb_split = NCB == 2;
       uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L::LUT_OFF);
+      const uint32_t lut_s = smem_u32(lut);
+      ChunkMap<kDecThreads> cm;
+      cm.init(dt, cb_split);
       for (int i = 0; i < nks; ++i) {
         const int s = i % STAGES;
         const uint32_t ph = (i / STAGES) & 1;
@@ -418,12 +443,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // before the codebook copies are rebuilt
         if (!named_bar_and(2, kDecThreads, mbar_wait(&full[s], ph))) break;
         uint8_t* st = stages + s * L::BYTES;
-        build_lut<kDecThreads>(reinterpret_cast<const uint32_t*>(st + L::CB_OFF), 1 + cb_split, lut, dt);
+        build_lut<kDecThreads>(reinterpret_cast<const uint16_t*>(st + L::CB_OFF), 1 + cb_split, lut, dt);
         named_bar_sync(2, kDecThreads);              // copies visible to all decoders
-        decode_w_tile<kDecThreads>(st + L::IDX_OFF, lut, cb_split, st + L::W_OFF, dt);
+        decode_w_tile<kDecThreads>(st + L::IDX_OFF, lut_s, st + L::W_OFF, cm);
         if constexpr (L::kSVQ) decode_sf_tile<L::kG, kDecThreads>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, dt);
-        fence_proxy_async_smem();
-        mbar_arrive(&dec[s]);
+        fence_proxy_async_smem();                    // each thread's tile writes -> async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dec[s]);         // one arrival per decoder warp
       }
     }
     ep_ok = mbar_wait(accum, 0);
@@ -439,7 +465,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t taddr = tmem + (static_cast<uint32_t>(qd * 32) << 16) + chalf * TCOL;
     if constexpr (T <= 32) {
       // this warp's accumulator columns in registers: one TMEM round trip
-      if constexpr (TCOL == 8) tmem_ld_32x32b_x8(taddr, acc_regs);
+      if constexpr (TCOL == 4) tmem_ld_32x32b_x4(taddr, acc_regs);
+      else if constexpr (TCOL == 8) tmem_ld_32x32b_x8(taddr, acc_regs);
       else tmem_ld_32x32b_x16(taddr, acc_regs);
       tmem_ld_wait();
       if (ep_ok) {
@@ -508,7 +535,7 @@ template <int FMT, int WSRC>
 struct DumpLayout {
   using L = StageLayout<FMT, WSRC, 16>;
   static constexpr int LUT_OFF = L::CTRL + L::BYTES;
-  static constexpr int SMEM = 1024 + LUT_OFF + 2 * 128 * 32 * 4;
+  static constexpr int SMEM = 1024 + LUT_OFF + 2 * 256 * 32 * 4;
 };
 
 template <int FMT, int WSRC>
@@ -553,10 +580,12 @@ __global__ void __launch_bounds__(160)
   }
   const bool ok = mbar_wait(bar, 0);
   const int dt = threadIdx.x - 32;
-  if (threadIdx.x >= 32 && ok) build_lut<128>(reinterpret_cast<const uint32_t*>(st + L::CB_OFF), 1 + cb_split, lut, dt);
+  if (threadIdx.x >= 32 && ok) build_lut<128>(reinterpret_cast<const uint16_t*>(st + L::CB_OFF), 1 + cb_split, lut, dt);
   __syncthreads();
   if (threadIdx.x >= 32 && ok) {
-    decode_w_tile<128>(st + L::IDX_OFF, lut, cb_split, st + L::W_OFF, dt);
+    ChunkMap<128> cm;
+    cm.init(dt, cb_split);
+    decode_w_tile<128>(st + L::IDX_OFF, smem_u32(lut), st + L::W_OFF, cm);
     if constexpr (L::kSVQ) decode_sf_tile<L::kG, 128>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, dt);
   }
   __syncthreads();
