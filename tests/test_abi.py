@@ -56,11 +56,13 @@ def test_pack_layouts(L, fmt, strategy):
     N, K = 256, 768
     w = synth.make_weight(7, fmt, strategy, N, K, 128, 256)
     h = _pack(w)
-    # index tiles: [N/128][K/256][128][64]
-    tiles = h["idx"].reshape(N // 128, K // 256, 128, 64)
+    # index slabs: [N/128][4 K-quarters][K/256][128 rows][16 bytes]
+    tiles = h["idx"].reshape(N // 128, 4, K // 256, 128, 16)
     for nt in range(N // 128):
         for ks in range(K // 256):
-            assert np.array_equal(tiles[nt, ks], w.idx[nt * 128:(nt + 1) * 128, ks * 64:(ks + 1) * 64])
+            for c in range(4):
+                assert np.array_equal(tiles[nt, c, ks],
+                                      w.idx[nt * 128:(nt + 1) * 128, ks * 64 + c * 16:ks * 64 + (c + 1) * 16])
     B = synth.BLOCK[fmt]
     if strategy == "prescale_plus":
         G = 256 // (8 * B)

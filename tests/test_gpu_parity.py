@@ -277,3 +277,32 @@ def test_moe_bad_offsets_sets_device_error():
     assert mxc.get_device_error() == 6                                       # MXC_ERR_DEVICE_INVALID
     assert torch.all(y == 7.0)                                               # nothing written
     assert mxc.get_device_error() == 0                                       # cleared by the read
+
+
+# ---------------------------------------------------------------------------
+# Decode GEMV (M <= 16): stage counts 1..8 per CTA, ragged last split, both
+# codebook widths along K, cluster sizes 1..4, and the long-K fallback
+# ---------------------------------------------------------------------------
+
+GEMV_CASES = [
+    (1024, 2048, 128, "e8m0_b32", "prescale_plus", 16),   # 2 stages per CTA, two codebooks per stage
+    (256, 3072, 128, "e4m3_b16", "prescale", 7),          # 3 stages per CTA
+    (2048, 5120, 256, "e8m0_b32", "prescale", 3),         # 5 stages per CTA
+    (128, 7936, 0, "e4m3_b16", "postscale", 16),          # one tensor codebook, splits 8/8/8/7
+    (9216, 4096, 128, "e4m3_b16", "postscale", 16),       # 8 stages, two codebooks per stage
+    (18944, 1024, 256, "e4m3_b16", "prescale_plus", 2),   # 148 tiles: no split (cluster of 1)
+    (256, 12288, 256, "e8m0_b32", "postscale", 5),        # 12 stages per CTA: pipelined kernel
+]
+
+
+@pytest.mark.parametrize("case", GEMV_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_decode_gemv_shapes(case):
+    N, K, qb, fmt, strat, M = case
+    w = synth.make_weight(61, fmt, strat, N, K, qb, qb)
+    x = synth.make_activations(61, M, K, outliers=True)
+    y, pw, a = run_mxcode(w, x)
+    assert mxc.get_device_error() == 0
+    ref, sabs = O.w4a4_linear(x, w)
+    assert_close(y.cpu().numpy(), ref, sabs, what=f"{case}")
+    yn = mxc.native_linear(a, mxc.decode_weight(pw))
+    assert torch.equal(y, yn)

@@ -212,75 +212,101 @@ __global__ void __launch_bounds__(256) quantize_kernel(
     quantize_unit<B>(x, M, K, ldx, e4m3, s, q, ldq, sf, u, kb_per_row, offsets, tile_prefix, n_groups);
 }
 
-// Small activations (decode batches): one launch of one 8-CTA cluster.  Each CTA
-// reduces 1/8 of the tensor to a partial amax, the partials are exchanged through
-// distributed shared memory (so each CTA reads only its share, and the loads of
-// one thread are all in flight together), then the CTAs quantize interleaved
-// blocks and clear the padding scale rows [M, round_up(M,128)) word by word.
+// Small activations (decode batches): one launch of one 8-CTA cluster, one pass.
+// Each thread loads its (at most two) blocks into registers once; for E4M3 the CTA
+// maxima are pushed into every CTA's shared memory (distributed shared memory,
+// one cluster barrier), so each thread then has the tensor amax locally and
+// quantizes its blocks from registers (a relaxed cluster arrive at the start and
+// its wait before the pushes make sure every CTA runs before it is written to).
+// Padding scale rows [M, round_up(M,128))
+// are cleared word by word.
 constexpr int kSmallQuantCtas = 8;
 constexpr int kSmallQuantThreads = 512;
+constexpr int kSmallQuantElems = 16 * 8192;       // M*K up to this takes the one-cluster path
+
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 
 template <int B>
 __global__ void __launch_bounds__(kSmallQuantThreads) quantize_small_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t K, int64_t ldx, int e4m3,
     const float* __restrict__ tscale_in, uint8_t* __restrict__ q, int64_t ldq, uint8_t* __restrict__ sf,
     float* __restrict__ tscale_out, int64_t sf_rows) {
+  constexpr int kThreadsAll = kSmallQuantCtas * kSmallQuantThreads;
+  constexpr int kUPT = (kSmallQuantElems / B + kThreadsAll - 1) / kThreadsAll;   // blocks per thread
   __shared__ uint32_t red[kSmallQuantThreads / 32];
-  __shared__ uint32_t partial;
-  const int kb_per_row = static_cast<int>(K / B);
-  const int k8s = static_cast<int>(K / 8);
-  const uint32_t rank = cluster_ctarank();
+  __shared__ uint32_t cta_max[kSmallQuantCtas];
   const bool need_amax = e4m3 && !tscale_in;
+  if (need_amax) cluster_arrive_relaxed();  // "started": no remote store before every CTA runs
+  griddep_launch_dependents();              // the next kernel may set up meanwhile
+  griddep_wait();                           // x may come from the previous kernel
+  const uint32_t rank = cluster_ctarank();
+  const int kb_per_row = static_cast<int>(K / B);
+  const uint32_t g = rank * kSmallQuantThreads + threadIdx.x;
+  const uint32_t units = static_cast<uint32_t>(M) * kb_per_row;
+  // this thread's blocks, in registers
+  uint32_t w[kUPT][B / 2];
+  uint32_t m = 0;
+#pragma unroll
+  for (int t = 0; t < kUPT; ++t) {
+    const uint32_t u = g + t * kThreadsAll;
+    if (u < units) {
+      const uint32_t r = u / kb_per_row, kb = u - r * kb_per_row;
+      const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx + static_cast<int64_t>(kb) * B);
+#pragma unroll
+      for (int i = 0; i < B / 8; ++i) {
+        const uint4 v = __ldg(src + i);
+        w[t][4 * i] = v.x; w[t][4 * i + 1] = v.y; w[t][4 * i + 2] = v.z; w[t][4 * i + 3] = v.w;
+      }
+#pragma unroll
+      for (int i = 0; i < B / 2; ++i) m = max(m, max(w[t][i] & 0x7FFFu, (w[t][i] >> 16) & 0x7FFFu));
+    }
+  }
+  // padding scale rows: zero
+  const int kb4 = kb_per_row / 4;
+  const uint32_t pad_words = static_cast<uint32_t>(sf_rows - M) * kb4;
+  for (uint32_t v = g; v < pad_words; v += kThreadsAll) {
+    const int64_t pr = M + v / kb4;
+    *reinterpret_cast<uint32_t*>(sf + sf_offset(pr, static_cast<int>(v % kb4) * 4, kb_per_row)) = 0u;
+  }
   float s = 1.0f;
   if (e4m3 && tscale_in) s = *tscale_in;
   if (need_amax) {
-    const int total = static_cast<int>(M) * k8s;
-    const int per = (total + kSmallQuantCtas - 1) / kSmallQuantCtas;
-    const int c_begin = static_cast<int>(rank) * per, c_end = min(total, c_begin + per);
-    uint32_t m = 0;
-    for (int c0 = c_begin + threadIdx.x; c0 < c_end; c0 += 4 * kSmallQuantThreads) {
-      uint4 v[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c = c0 + j * kSmallQuantThreads;
-        v[j] = c < c_end ? __ldg(reinterpret_cast<const uint4*>(x + (c / k8s) * ldx) + (c % k8s))
-                         : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        m = max(m, max(max(v[j].x & 0x7FFFu, (v[j].x >> 16) & 0x7FFFu), max(v[j].y & 0x7FFFu, (v[j].y >> 16) & 0x7FFFu)));
-        m = max(m, max(max(v[j].z & 0x7FFFu, (v[j].z >> 16) & 0x7FFFu), max(v[j].w & 0x7FFFu, (v[j].w >> 16) & 0x7FFFu)));
-      }
-    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    cluster_wait_acquire();                  // every CTA of the cluster is running
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x < kSmallQuantCtas) {     // push this CTA's maximum into CTA threadIdx.x
       uint32_t mm = 0;
 #pragma unroll
       for (int i = 0; i < kSmallQuantThreads / 32; ++i) mm = max(mm, red[i]);
-      partial = mm;
+      st_cluster_u32(mapa_shared(smem_u32(&cta_max[rank]), threadIdx.x), mm);
     }
-    cluster_sync_all();                      // every CTA's partial is in its shared memory
+    cluster_sync_all();                      // all maxima everywhere; nothing remote after this
     uint32_t mm = 0;
-    const uint32_t local = smem_u32(&partial);
 #pragma unroll
-    for (int r = 0; r < kSmallQuantCtas; ++r) mm = max(mm, ld_cluster_u32(mapa_shared(local, r)));
-    cluster_sync_all();                      // no CTA leaves while others still read it
+    for (int i = 0; i < kSmallQuantCtas; ++i) mm = max(mm, cta_max[i]);
     const float amax = __uint_as_float(mm << 16);
     s = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
   }
   if (tscale_out && rank == 0 && threadIdx.x == 0) *tscale_out = s;
-  const uint32_t stride = kSmallQuantCtas * kSmallQuantThreads;
-  const uint32_t data_units = static_cast<uint32_t>(M) * kb_per_row;
-  for (uint32_t u = rank * kSmallQuantThreads + threadIdx.x; u < data_units; u += stride)
-    quantize_unit<B>(x, M, K, ldx, e4m3, s, q, ldq, sf, u, kb_per_row, nullptr, nullptr, 0);
-  const int kb4 = kb_per_row / 4;
-  const uint32_t pad_words = static_cast<uint32_t>(sf_rows - M) * kb4;
-  for (uint32_t u = rank * kSmallQuantThreads + threadIdx.x; u < pad_words; u += stride) {
-    const int64_t pr = M + u / kb4;
-    *reinterpret_cast<uint32_t*>(sf + sf_offset(pr, static_cast<int>(u % kb4) * 4, kb_per_row)) = 0u;
+#pragma unroll
+  for (int t = 0; t < kUPT; ++t) {
+    const uint32_t u = g + t * kThreadsAll;
+    if (u < units) {
+      const uint32_t r = u / kb_per_row, kb = u - r * kb_per_row;
+      uint32_t qw[B / 8], sfb;
+      quantize_block<B>(w[t], e4m3 != 0, s, qw, sfb);
+      uint8_t* dst = q + static_cast<int64_t>(r) * ldq + static_cast<int64_t>(kb) * (B / 2);
+      if (B == 32) {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(qw[0], qw[1], qw[2], qw[3]);
+      } else {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(qw[0], qw[1]);
+      }
+      sf[sf_offset(r, static_cast<int>(kb), kb_per_row)] = static_cast<uint8_t>(sfb);
+    }
   }
 }
 
@@ -321,9 +347,6 @@ cudaError_t launch_group_prologue(const int32_t* offsets, int32_t E, int64_t M, 
   return cudaGetLastError();
 }
 
-// Activations up to this many elements (e.g. 16 x 8192) take the one-CTA path.
-constexpr int64_t kSmallQuantElems = 16 * 8192;
-
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
   const bool e4m3 = a.fmt == MXC_FMT_E4M3_B16;
   const int B = e4m3 ? 16 : 32;
@@ -333,13 +356,15 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
     cfg.gridDim = dim3(kSmallQuantCtas);
     cfg.blockDim = dim3(kSmallQuantThreads);
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = kSmallQuantCtas;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     const uint16_t* xp = reinterpret_cast<const uint16_t*>(a.x);
     cudaError_t err;
     if (e4m3) {

@@ -1,0 +1,461 @@
+// gemv_kernel.cuh -- the decode-shaped MXCode W4A4 linear layer (M <= 16 tokens).
+//
+// "MXCode: Vector Quantization for MX-Native Inference at Scale", Sec. 5 (decode
+// TPOT): at decode batch sizes the layer streams its weights once, so the time goes
+// to bringing the compressed weights in and turning them into tensor-core operands.
+// Each CTA owns 128 output channels x a slice of at most 8 stages of 256 input
+// channels (split-K over the CTAs of a thread-block cluster) and keeps the slice on
+// chip:
+//
+//   * the loader copies the slice's index bytes with one bulk copy per K-quarter
+//     (the packed layout keeps, per 128-row band, quarter c of all stages
+//     contiguous), quarter 0 first, and all token tiles with one 3-D tensor copy;
+//   * decoder lane l decodes stage l mod 8, so the 32 per-lane codebook copies in
+//     shared memory hold, in bank l, the codebook of lane l's stage: the codebooks
+//     of the whole slice are laid out once (16-bit entries, 16 KB) and no lookup
+//     meets a bank conflict;
+//   * the decoders finish K-quarter j of every stage before quarter j+1; the MMA
+//     warp issues the block-scaled MMAs of quarter j of all stages while quarter
+//     j+1 is decoded.  Native FP4 weights use the same quarter-major MMA order, so
+//     both give bit-identical results on the same operands;
+//   * the index slabs pass through a ring of three quarter buffers (quarter 3
+//     reuses quarter 0's buffer once it is decoded), which leaves room to bring
+//     the weight scale atoms in by one bulk copy for tcgen05.cp from the MMA warp;
+//     the token scale atoms (16 rows) go from registers to TMEM with tcgen05.st,
+//     in the layout the tcgen05.cp 32x128b.warpx4 copy gives;
+//   * split-K partial tiles go to the cluster's rank 0 by st.async with completion
+//     on an mbarrier there; rank 0 adds them in rank order (deterministic).
+//
+// Programmatic dependent launch: the CTA sets up and prefetches its weight stream
+// into L2 before griddepcontrol.wait, overlapping the previous kernel (typically
+// the activation quantizer); nothing that kernel writes is read before the wait.
+#pragma once
+
+#include "mma_kernel.cuh"
+
+namespace mxc {
+
+constexpr int kGemvT = 16;          // token tile = MMA N
+constexpr int kGemvMaxStages = 8;   // 256-channel stages per CTA, all resident
+constexpr int kGemvMaxSplits = 4;   // cluster size
+
+struct GemvParams {
+  int M, N, K;
+  int qn, qk;                 // resolved QBlock
+  const uint8_t* a_sf;        // activation scales, SF layout
+  const float* a_tscale;      // device or null
+  const float* w_tscale_dev;  // native weights: device tensor scale or null
+  void* y;
+  int64_t ldy;
+  int out_bf16;
+  int splits, ks_per_split;
+  ExpertPtrs w;
+};
+
+template <int FMT, int WSRC>
+struct GemvLayout {
+  static constexpr bool kVQ = WSRC != WSRC_NATIVE;
+  static constexpr bool kSVQ = WSRC == WSRC_VQ_SVQ;
+  static constexpr int kB = FMT == FMT_E8M0 ? 32 : 16;
+  static constexpr int kAtoms = kStageK / kB / 4;      // scale atoms per 128 rows per stage
+  static constexpr int kG = kStageK / (8 * kB);        // PreScale+ scale groups per row per stage
+  static constexpr int S = kGemvMaxStages;
+  static constexpr int W_OFF = 0;                      // S x [128][128 B] FP4, 128-byte swizzle
+  static constexpr int X_OFF = W_OFF + S * 16384;      // S x [16][128 B] FP4 token tiles
+  // index slabs, 3 buffers x [S stages][128][16 B] (quarter j in buffer j mod 3,
+  // quarter 3 in buffer 0); afterwards rank 0's receive area for the other ranks'
+  // partial tiles, [rank-1][128][16] FP32
+  static constexpr int IDX_OFF = X_OFF + S * kGemvT * 128;
+  static constexpr int IDX_BUF = S * 2048;
+  static constexpr int SFW_OFF = IDX_OFF + 3 * IDX_BUF;           // weight scale atoms (direct, native)
+  static constexpr int LUT_OFF = SFW_OFF + (kSVQ ? 0 : S * kAtoms * 512);   // 128 words x 32 lanes
+  static constexpr int CTRL_OFF = LUT_OFF + (kVQ ? 16384 : 0);
+  // The slice's codebooks (at most 16 x 512 B) land in the second half of the last
+  // stage's FP4 tile, which is not written before the codebook copies are laid out.
+  static constexpr int CB_OFF = W_OFF + (S - 1) * 16384 + 8192;
+  static constexpr int SMEM = 1024 + CTRL_OFF + 256;
+  static constexpr int RED = (kGemvMaxSplits - 1) * 128 * kGemvT * 4;
+  // TMEM: accumulator [0,16); the scale atoms of all stages, 4 columns each:
+  // weight scales from column 32, token scales after them.
+  static constexpr int COL_SFW = 32;
+  static constexpr int COL_SFX = COL_SFW + S * kAtoms * 4;
+  static constexpr int TMEM_COLS = COL_SFX + S * kAtoms * 4 <= 256 ? 256 : 512;
+  static_assert(RED <= 3 * IDX_BUF, "receive area");
+  static_assert(SMEM <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint4 v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Two index bytes (k, k+1 of word x) -> 8 FP4 values (32 bits) through this lane's
+// codebook copy: 16-bit entries, two per word, word (e/2)*32 + lane.  The two
+// lookups are merged with one byte permute whose selector picks each entry's half.
+__device__ __forceinline__ uint32_t lut16_pair(uint32_t lut_lane, uint32_t x, int k) {
+  const uint32_t wa = lds_u32(lut_lane + (((x >> (8 * k + 1)) & 0x7Fu) << 7));
+  const uint32_t wb = lds_u32(lut_lane + (((x >> (8 * k + 9)) & 0x7Fu) << 7));
+  return __byte_perm(wa, wb, 0x5410u + ((x >> (8 * k)) & 0x101u) * 0x22u);
+}
+
+template <int FMT, int WSRC>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemv_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_wq,
+                const __grid_constant__ GemvParams p) {
+  using L = GemvLayout<FMT, WSRC>;
+  constexpr int A = L::kAtoms;
+  static_assert(kDecWarps == 16, "decode map assumes 16 decoder warps");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::CTRL_OFF);
+  uint64_t* full = bars;            // [8] VQ: K-quarter j of all index slabs (j < 4); native: stage tiles
+  uint64_t* bar_x = bars + 8;       // token tiles
+  uint64_t* dec_ph = bars + 9;      // [4] K-quarter j decoded (one arrival per decoder warp)
+  uint64_t* sf_ready = bars + 13;   // scale atoms in TMEM (one arrival per decoder warp)
+  uint64_t* accum = bars + 14;
+  uint64_t* red_full = bars + 15;   // rank 0: partial tiles received
+  uint64_t* red_ready = bars + 16;  // rank > 0: rank 0 may receive
+  uint64_t* bar_sfw = bars + 17;    // weight scale atoms (bulk copy)
+  uint64_t* bar_cb = bars + 18;     // codebooks of the slice (bulk copy)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int K = p.K, KS = K / kStageK, KB4 = K / L::kB / 4;
+  const int n_tile = blockIdx.x;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kGemvT;
+  const int sf_group0 = static_cast<int>(m0 / 128);
+  const int splits = p.splits;
+  const int ks_begin = blockIdx.z * p.ks_per_split;
+  const int ks_end = min(KS, ks_begin + p.ks_per_split);
+  const int nks = ks_end - ks_begin;
+  const uint32_t rank = splits > 1 ? cluster_ctarank() : 0u;
+  const int H = (L::kVQ && p.qk == 128) ? 2 : 1;     // codebooks per stage along K
+  const int qbn = L::kVQ ? static_cast<int>((static_cast<int64_t>(n_tile) * 128) / p.qn) : 0;
+  const int cb_per_row = L::kVQ ? K / p.qk : 0;
+  // quarter j of this slice: w_idx + j * KS * 2048, nks slabs of 2 KB
+  const uint8_t* const w_idx = p.w.idx + (static_cast<size_t>(n_tile) * 4 * KS + ks_begin) * 2048;
+  const uint16_t* const w_cb = p.w.cb + static_cast<size_t>(qbn) * cb_per_row * 256;
+  const uint8_t* const w_sf = p.w.sf + (static_cast<size_t>(n_tile) * KB4 + static_cast<size_t>(ks_begin) * A) * 512;
+  const uint8_t* const w_sidx = p.w.sidx + (static_cast<size_t>(n_tile) * KS + ks_begin) * (128 * L::kG);
+  const uint8_t* const a_sf =
+      p.a_sf + (static_cast<size_t>(sf_group0) * KB4 + static_cast<size_t>(ks_begin) * A) * 512;
+  // codebooks used by the slice: a contiguous range [qb0, qb1] of the band's row
+  const int qb0 = !L::kVQ ? 0 : H == 2 ? 2 * ks_begin : (ks_begin * kStageK) / p.qk;
+  const int qb1 = !L::kVQ ? 0 : H == 2 ? 2 * ks_end - 1 : ((ks_end - 1) * kStageK) / p.qk;
+
+  // ---- setup (nothing here depends on earlier kernels) ----
+  if (warp == 0) {
+    // full[0..7], bar_x, dec_ph[0..3], sf_ready, accum, red_full, red_ready, bar_sfw, bar_cb
+    if (lane < 19) mbar_init(bars + lane, (lane >= 9 && lane < 14) ? kDecWarps : 1);
+    __syncwarp();
+  }
+  if (warp == 0 && lane == 0) {
+    // rank 0 expects every other rank's partial tile; armed before it lets them send
+    if (splits > 1 && rank == 0) mbar_arrive_expect_tx(red_full, (splits - 1) * 128 * kGemvT * 4);
+    fence_mbar_init();
+    prefetch_tensormap(&tmap_x);
+    if constexpr (WSRC == WSRC_NATIVE) prefetch_tensormap(&tmap_wq);
+    // this CTA's weight stream into L2: codebooks and scales first, then the bulk
+    if constexpr (L::kVQ) {
+      l2_prefetch_bulk(w_cb + static_cast<size_t>(qb0) * 256, static_cast<uint32_t>(qb1 - qb0 + 1) * 512);
+    }
+    if constexpr (L::kSVQ) {
+      l2_prefetch_bulk(w_sidx, static_cast<uint32_t>(nks) * 128 * L::kG);
+    } else {
+      l2_prefetch_bulk(w_sf, static_cast<uint32_t>(nks) * A * 512);
+    }
+    if constexpr (L::kVQ) {
+      for (int j = 0; j < 4; ++j)
+        l2_prefetch_bulk(w_idx + static_cast<size_t>(j) * KS * 2048, static_cast<uint32_t>(nks) * 2048);
+    } else {
+      for (int s = 0; s < nks; ++s) l2_prefetch_tile_2d(&tmap_wq, (ks_begin + s) * 128, n_tile * 128);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (splits > 1) cluster_arrive_relaxed();          // barriers above are initialised (fenced)
+  griddep_launch_dependents();
+  griddep_wait();                                    // earlier kernels' results are visible
+  if (splits > 1) cluster_wait_acquire();            // every CTA of the cluster is set up
+  // output scale: read now, used at the very end
+  float out_scale = p.w.w_tscale;
+  if (warp >= 2) {
+    if constexpr (WSRC == WSRC_NATIVE) {
+      if (p.w_tscale_dev) out_scale = __ldg(p.w_tscale_dev);
+    }
+    if (p.a_tscale) out_scale *= __ldg(p.a_tscale);
+  }
+
+  // epilogue coordinates (decoder warps)
+  const int qd = warp & 3;                           // TMEM lane quadrant this warp may access
+  const int cg = (warp - 2) >> 2;                    // 4-column group of the accumulator
+  const int row = qd * 32 + lane;
+  const int64_t n = static_cast<int64_t>(n_tile) * 128 + row;
+  const int64_t mbase = m0 + cg * 4;
+
+  if (warp == 0) {
+    // =============================== loader ===============================
+    if (elect_one()) {
+      // in the order they are needed: codebooks, index quarter 0, scales, tokens, quarters 1..3
+      if constexpr (L::kVQ) {
+        const uint32_t cb_bytes = static_cast<uint32_t>(qb1 - qb0 + 1) * 512;
+        mbar_arrive_expect_tx(bar_cb, cb_bytes);
+        bulk_load(smem + L::CB_OFF, w_cb + static_cast<size_t>(qb0) * 256, cb_bytes, bar_cb);
+#ifdef MXC_GEMV_CB_ALONE
+        mbar_wait(bar_cb, 0);                        // the codebooks land alone, first
+#endif
+        mbar_arrive_expect_tx(&full[0], nks * 2048);
+        bulk_load(smem + L::IDX_OFF, w_idx, nks * 2048, &full[0]);
+      }
+      if constexpr (!L::kSVQ) {
+        mbar_arrive_expect_tx(bar_sfw, nks * A * 512);
+        bulk_load(smem + L::SFW_OFF, w_sf, nks * A * 512, bar_sfw);
+      }
+      // token tiles of all stages: box {128 B, 16 rows, ks_per_split stages}; stages
+      // past K (last split) arrive zero-filled and are not used
+      mbar_arrive_expect_tx(bar_x, p.ks_per_split * kGemvT * 128);
+      tma_load_3d(smem + L::X_OFF, &tmap_x, 0, static_cast<int>(m0), ks_begin, bar_x);
+      if constexpr (L::kVQ) {
+        for (int j = 1; j < 4; ++j) {                // K-quarter j of every stage
+          if (j == 3 && !mbar_wait(&dec_ph[0], 0)) break;   // buffer 0 is free again
+          mbar_arrive_expect_tx(&full[j], nks * 2048);
+          bulk_load(smem + L::IDX_OFF + (j % 3) * L::IDX_BUF, w_idx + static_cast<size_t>(j) * KS * 2048, nks * 2048,
+                    &full[j]);
+        }
+      } else {
+        for (int s = 0; s < nks; ++s) {
+          mbar_arrive_expect_tx(&full[s], 16384);
+          tma_load_2d(smem + L::W_OFF + s * 16384, &tmap_wq, (ks_begin + s) * 128, n_tile * 128, &full[s]);
+        }
+      }
+    }
+    __syncwarp();
+    if (splits > 1 && rank == 0) {
+      // The index buffers are rank 0's receive area once its decoders are done with
+      // them: then let the other ranks send their partials (even after a failed
+      // wait, so that no rank waits for the signal in vain).
+      if constexpr (L::kVQ) mbar_wait(&dec_ph[3], 0);
+      if (lane > 0 && lane < splits) mbar_remote_arrive(mapa_shared(smem_u32(red_ready), lane));
+    }
+  } else if (warp == 1) {
+    // ============================ MMA issuer ==============================
+    const uint32_t w_s0 = smem_u32(smem + L::W_OFF), x_s0 = smem_u32(smem + L::X_OFF);
+    bool ok = true;
+    if constexpr (!L::kSVQ) {
+      // weight scale atoms -> TMEM; copies and MMAs issue in order from this thread
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_sfw, 0));
+      if (ok && elect_one()) {
+        const uint32_t sfw_s0 = smem_u32(smem + L::SFW_OFF);
+        for (int i = 0; i < nks * A; ++i)
+          tc_cp_32x128b_warpx4(tmem + L::COL_SFW + 4 * i, sdesc_sf_atom(sfw_s0 + i * 512));
+      }
+      __syncwarp();
+    }
+    ok = __all_sync(0xffffffffu, mbar_wait(bar_x, 0)) && ok;
+    ok = __all_sync(0xffffffffu, mbar_wait(sf_ready, 0)) && ok;
+    if constexpr (!L::kVQ) {
+      for (int s = 0; s < nks && ok; ++s) ok = __all_sync(0xffffffffu, mbar_wait(&full[s], 0));
+    }
+    tc_fence_after();
+    for (int j = 0; j < 4 && ok; ++j) {
+      if constexpr (L::kVQ) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&dec_ph[j], 0))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      if (elect_one()) {
+        for (int s = 0; s < nks; ++s) {
+          const uint64_t adesc = sdesc_kmajor_sw128(w_s0 + s * 16384 + 32 * j);
+          const uint64_t bdesc = sdesc_kmajor_sw128(x_s0 + s * kGemvT * 128 + 32 * j);
+          const uint32_t acc = (s > 0 || j > 0) ? 1u : 0u;
+          const uint32_t sfw_t = tmem + L::COL_SFW + 4 * s * A, sfx_t = tmem + L::COL_SFX + 4 * s * A;
+          if constexpr (FMT == FMT_E4M3) {
+            constexpr uint32_t idesc = idesc_mxf4(kGemvT, 0, 0, 0);
+            tc_mma_mxf4nvf4_block16(tmem, adesc, bdesc, idesc, sfw_t + 4 * j, sfx_t + 4 * j, acc);
+          } else {
+            const int a = j >> 1;
+            const uint32_t id = static_cast<uint32_t>(j & 1) * 2;
+            const uint32_t idesc = idesc_mxf4(kGemvT, 1, static_cast<int>(id), static_cast<int>(id));
+            tc_mma_mxf4_block32(tmem, adesc, bdesc, idesc, (sfw_t + 4 * a) | (id << 30), (sfx_t + 4 * a) | (id << 30),
+                                acc);
+          }
+        }
+      }
+      __syncwarp();
+    }
+    if (elect_one()) tc_commit(accum);
+    __syncwarp();
+    mbar_wait(accum, 0);      // our own MMAs finish before the CTA retires
+  } else {
+    // ======================= decoders, then epilogue ======================
+    const int dw = warp - 2;
+    // --- the stage codebook words this lane lays out (loads issued first) ---
+    const int s_l = lane & 7;                        // this lane's stage
+    const int q = dw * 4 + (lane >> 3);              // 64 threads per stage
+    const bool active = L::kVQ && s_l < nks;
+    // words [8 dw, 8 dw + 8) of the codebook of this lane's stage, for the first or
+    // (QBlock 128 wide along K) the second half of the stage
+    auto cb_words = [&](int epoch, uint4* c0, uint4* c1) {
+      const int ks = ks_begin + s_l;
+      const int qbk = H == 2 ? 2 * ks + epoch : (ks * kStageK) / p.qk;
+      const uint4* cp = reinterpret_cast<const uint4*>(smem + L::CB_OFF + (qbk - qb0) * 512 + 32 * dw);
+      *c0 = cp[0];
+      *c1 = cp[1];
+    };
+
+    // --- token scale atoms (and PreScale+ weight scales) -> TMEM lanes of this
+    //     warp's quadrant; atoms i = cg mod 4.  Loads now, stores after phase 0. ---
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    const int natoms = nks * A;
+    constexpr int kPer = L::S * A / 4;               // atoms per warp, at most
+    uint4 sx[kPer];
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {                 // rows 0..15 of the atom are the 16 tokens
+      const int i = cg + 4 * t;
+      sx[t] = (i < natoms && lane < kGemvT) ? ldg_nc_v4(a_sf + static_cast<size_t>(i) * 512 + lane * 16)
+                                            : make_uint4(0, 0, 0, 0);
+    }
+    auto scales_to_tmem = [&]() {
+#pragma unroll
+      for (int t = 0; t < kPer; ++t) {
+        const int i = cg + 4 * t;
+        if (i < natoms) tmem_st_32x32b_x4(lane_base + L::COL_SFX + 4 * i, sx[t]);
+      }
+      if constexpr (L::kSVQ) {
+        // PreScale+ (Table 4 caption: Ks = 256, ds = 8): row `lane` of atom (s, a)
+        // holds, for rows 32 g + lane (g = 0..3), scales 4a..4a+3 of stage s, i.e.
+        // word a mod 2 of the 8-byte scale-codebook entry of scale group a/2.
+        const uint32_t* scb32 = reinterpret_cast<const uint32_t*>(p.w.scb);
+        for (int i = cg; i < natoms; i += 4) {
+          const int s = i / A, a = i % A;
+          const uint8_t* si = w_sidx + static_cast<size_t>(s) * 128 * L::kG + (a >> 1);
+          uint4 v;
+          v.x = __ldg(scb32 + 2 * __ldg(si + (0 * 32 + lane) * L::kG) + (a & 1));
+          v.y = __ldg(scb32 + 2 * __ldg(si + (1 * 32 + lane) * L::kG) + (a & 1));
+          v.z = __ldg(scb32 + 2 * __ldg(si + (2 * 32 + lane) * L::kG) + (a & 1));
+          v.w = __ldg(scb32 + 2 * __ldg(si + (3 * 32 + lane) * L::kG) + (a & 1));
+          tmem_st_32x32b_x4(lane_base + L::COL_SFW + 4 * i, v);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sf_ready);
+    };
+    if constexpr (!L::kVQ) scales_to_tmem();
+
+    if constexpr (L::kVQ) {
+      // both codebooks into registers now: the staging area is overwritten by the
+      // decoded tiles of the last stage
+      uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0, d0 = c0, d1 = c0;
+      const bool cb_ok = mbar_wait(bar_cb, 0);
+      if (active && cb_ok) {
+        cb_words(0, &c0, &c1);
+        if (H == 2) cb_words(1, &d0, &d1);
+      }
+      // --- codebook copies: lane l's copy (bank l) = codebook of stage l mod 8 ---
+      uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L::LUT_OFF) + (8 * dw) * 32 + lane;
+      auto lay_out = [&](const uint4& a, const uint4& b) {
+        if (!active) return;
+        lut[0 * 32] = a.x;
+        lut[1 * 32] = a.y;
+        lut[2 * 32] = a.z;
+        lut[3 * 32] = a.w;
+        lut[4 * 32] = b.x;
+        lut[5 * 32] = b.y;
+        lut[6 * 32] = b.z;
+        lut[7 * 32] = b.w;
+      };
+      lay_out(c0, c1);
+      named_bar_sync(2, kDecThreads);                // all copies written
+      const uint32_t lut_lane = smem_u32(smem + L::LUT_OFF) + lane * 4;
+      const uint8_t* idx_l = smem + L::IDX_OFF + s_l * 2048;
+      uint8_t* wt = smem + L::W_OFF + s_l * 16384;
+      for (int j = 0; j < 4; ++j) {
+        if (H == 2 && j == 2) {                      // second half of each stage: its own codebook
+          named_bar_sync(2, kDecThreads);            // everyone is done with the first codebooks
+          lay_out(d0, d1);
+          named_bar_sync(2, kDecThreads);
+        }
+        const bool landed = mbar_wait(&full[j], 0);
+        if (active && landed) {
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int r = (q + 64 * i + s_l) & 127;  // offset by the stage: conflict-free stores
+            const uint4 iv = *reinterpret_cast<const uint4*>(idx_l + (j % 3) * L::IDX_BUF + r * 16);
+            const uint4 o0 = make_uint4(lut16_pair(lut_lane, iv.x, 0), lut16_pair(lut_lane, iv.x, 2),
+                                        lut16_pair(lut_lane, iv.y, 0), lut16_pair(lut_lane, iv.y, 2));
+            const uint4 o1 = make_uint4(lut16_pair(lut_lane, iv.z, 0), lut16_pair(lut_lane, iv.z, 2),
+                                        lut16_pair(lut_lane, iv.w, 0), lut16_pair(lut_lane, iv.w, 2));
+            *reinterpret_cast<uint4*>(wt + r * 128 + (((2 * j) ^ (r & 7)) << 4)) = o0;
+            *reinterpret_cast<uint4*>(wt + r * 128 + (((2 * j + 1) ^ (r & 7)) << 4)) = o1;
+          }
+        }
+        fence_proxy_async_smem();                    // tile writes -> tensor-core operand reads
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dec_ph[j]);
+        if (j == 0) scales_to_tmem();                // needed with quarter 0's MMAs
+      }
+    }
+    // ------------------------------ epilogue ------------------------------
+    const bool ep_ok = mbar_wait(accum, 0);
+    tc_fence_after();
+    const float scale = out_scale;
+    uint32_t acc[4];
+    tmem_ld_32x32b_x4(tmem + (static_cast<uint32_t>(qd * 32) << 16) + cg * 4, acc);
+    tmem_ld_wait();
+    float v[4] = {__uint_as_float(acc[0]), __uint_as_float(acc[1]), __uint_as_float(acc[2]), __uint_as_float(acc[3])};
+    const uint32_t red_slot = smem_u32(smem + L::IDX_OFF) + (row * kGemvT + cg * 4) * 4;
+    bool store = ep_ok;
+    if (splits > 1) {
+      if (rank != 0) {
+        store = false;
+        if (mbar_wait(red_ready, 0)) {              // sent even when ep_ok is false: rank 0 waits for it
+          st_async_v4_f32(mapa_shared(red_slot + (rank - 1) * 128 * kGemvT * 4, 0), v[0], v[1], v[2], v[3],
+                          mapa_shared(smem_u32(red_full), 0));
+        }
+      } else {
+        const bool got = mbar_wait(red_full, 0);    // all partials landed: none in flight at exit
+        store = store && got;
+        if (store) {
+          for (int r = 1; r < splits; ++r) {
+            const float4 o = *reinterpret_cast<const float4*>(smem + L::IDX_OFF + ((r - 1) * 128 * kGemvT +
+                                                                                  row * kGemvT + cg * 4) * 4);
+            v[0] += o.x;
+            v[1] += o.y;
+            v[2] += o.z;
+            v[3] += o.w;
+          }
+        }
+      }
+    }
+    if (store) {
+      void* const y = p.y;
+      const int64_t ldy = p.ldy;
+      const int out_bf16 = p.out_bf16;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (mbase + c < p.M) store_out(y, ldy, out_bf16, mbase + c, n, v[c] * scale);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+}  // namespace mxc

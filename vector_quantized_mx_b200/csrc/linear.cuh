@@ -4,7 +4,7 @@
 
 #include <cstring>
 
-#include "mma_kernel.cuh"
+#include "gemv_kernel.cuh"
 
 namespace mxc {
 
@@ -40,6 +40,23 @@ inline bool make_fp4_map(CUtensorMap* map, const void* base, int64_t rows, int64
   const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over the same FP4 matrix seen as [K/256 stages][rows][128 bytes] (stage
+// stride 128 bytes): one box = box_rows rows x box_stages consecutive 256-column
+// stages, each stage a [box_rows][128 B] tile in the 128-byte swizzle.
+inline bool make_fp4_stage_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int64_t ld,
+                               int box_rows, int box_stages) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return false;
+  std::memset(map, 0, sizeof(*map));
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(K / 256)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld), 128};
+  const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(box_stages)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -128,6 +145,48 @@ cudaError_t dispatch_tile(int T, const CUtensorMap& tx, const CUtensorMap& tw, c
   return dispatch_dense<FMT, WSRC, 128>(tx, tw, p, grid, stream);
 }
 
+// Decode GEMV: a cluster of `splits` CTAs per 128-row output tile, launched with
+// programmatic stream serialization (the kernel waits for the previous kernel's
+// results itself, after its setup and weight prefetch).
+template <int FMT, int WSRC>
+cudaError_t launch_gemv(const CUtensorMap& tx, const CUtensorMap& tw, const GemvParams& p, dim3 grid,
+                        cudaStream_t stream) {
+  using L = GemvLayout<FMT, WSRC>;
+  auto kern = gemv_kernel<FMT, WSRC>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = L::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (p.splits > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = static_cast<unsigned>(p.splits);
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  err = cudaLaunchKernelEx(&cfg, kern, tx, tw, p);
+  if (err != cudaSuccess) return err;
+  return cudaGetLastError();
+}
+
+template <int FMT>
+cudaError_t dispatch_gemv(int wsrc, const CUtensorMap& tx, const CUtensorMap& tw, const GemvParams& p, dim3 grid,
+                          cudaStream_t stream) {
+  if (wsrc == WSRC_VQ_DIRECT) return launch_gemv<FMT, WSRC_VQ_DIRECT>(tx, tw, p, grid, stream);
+  if (wsrc == WSRC_VQ_SVQ) return launch_gemv<FMT, WSRC_VQ_SVQ>(tx, tw, p, grid, stream);
+  return launch_gemv<FMT, WSRC_NATIVE>(tx, tw, p, grid, stream);
+}
+
 inline ExpertPtrs expert_ptrs(const LinearArgs& a) {
   ExpertPtrs e{};
   e.idx = a.w_idx;
@@ -171,6 +230,29 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
     decode_splits(a.N, a.K, &splits, &per);
     p.splits = splits;
     p.ks_per_split = per;
+    if (per <= kGemvMaxStages && splits <= kGemvMaxSplits) {
+      CUtensorMap tx3;
+      if (!make_fp4_stage_map(&tx3, a.a_q, a.M, a.K, a.ldq, kGemvT, per)) return MXC_ERR_CUDA;
+      GemvParams g{};
+      g.M = p.M;
+      g.N = p.N;
+      g.K = p.K;
+      g.qn = p.qn;
+      g.qk = p.qk;
+      g.a_sf = p.a_sf;
+      g.a_tscale = p.a_tscale;
+      g.w_tscale_dev = p.w_tscale_dev;
+      g.y = p.y;
+      g.ldy = p.ldy;
+      g.out_bf16 = p.out_bf16;
+      g.splits = splits;
+      g.ks_per_split = per;
+      g.w = p.w[0];
+      const dim3 grid(n_tiles, m_tiles, splits);
+      const cudaError_t err = a.fmt == FMT_E8M0 ? dispatch_gemv<FMT_E8M0>(a.wsrc, tx3, tw, g, grid, stream)
+                                                : dispatch_gemv<FMT_E4M3>(a.wsrc, tx3, tw, g, grid, stream);
+      return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
+    }
   }
   const dim3 grid(n_tiles, m_tiles, p.splits);
   cudaError_t err;

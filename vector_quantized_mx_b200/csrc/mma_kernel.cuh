@@ -134,8 +134,8 @@ __device__ __forceinline__ void build_lut(const uint16_t* __restrict__ cb, int n
 // Byte k of w, zero-extended.
 __device__ __forceinline__ uint32_t byte_of(uint32_t w, int k) { return __byte_perm(w, 0u, 0x4440 | k); }
 
-// One 128 x 256 weight tile: idx [128][64] bytes -> FP4 [128][128] bytes in the
-// 128-byte swizzle (16-byte chunk j of row r stored at chunk j ^ (r % 8)).
+// One 128 x 256 weight tile: idx (four K-quarter slabs [128][16] bytes) -> FP4
+// [128][128] bytes in the 128-byte swizzle (16-byte chunk j of row r stored at chunk j ^ (r % 8)).
 // Thread dt owns chunks it*NT + dt; their shared-memory offsets are fixed per
 // thread and computed once (ChunkMap).  Chunks 0..3 of a row use codebook 0,
 // chunks 4..7 codebook 1 when the QBlock is 128 wide along K.
@@ -150,7 +150,7 @@ struct ChunkMap {
     for (int it = 0; it < kN; ++it) {
       const int c = it * NT + dt;
       const int r = c >> 3, j = c & 7;
-      idx_off[it] = r * 64 + j * 8;
+      idx_off[it] = (j >> 1) * 2048 + r * 16 + (j & 1) * 8;   // K-quarter slab j/2
       w_off[it] = r * 128 + ((j ^ (r & 7)) << 4);
       lut_off[it] = ((cb_split && j >= 4) ? 256 * 32 * 4 : 0) + (dt & 31) * 4;
     }
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (WSRC == WSRC_VQ_SVQ) tx += 8192 + (cb_split ? 1024 : 512) + 128 * L::kG;
     const uint8_t* sfx_src = a_sf + static_cast<size_t>(sf_group0) * KB4 * 512;
     const uint8_t* sfw_src = w_sf + static_cast<size_t>(n_tile) * KB4 * 512;
-    const uint8_t* idx_src = w_idx + static_cast<size_t>(n_tile) * KS * 8192;
+    const uint8_t* idx_src = w_idx + static_cast<size_t>(n_tile) * 4 * KS * 2048;   // band: [4][KS][128][16]
     const uint8_t* sidx_src = w_sidx + static_cast<size_t>(n_tile) * KS * (128 * L::kG);
     const uint16_t* cb_src = w_cb + static_cast<size_t>(qbn) * cb_per_row * 256;
     const int y0 = static_cast<int>(m0);
@@ -351,7 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(st + L::W_OFF, &tmap_wq, ks * 128, n_tile * 128, &full[s]);
           bulk_load(st + L::SFW_OFF, sfw_src + static_cast<size_t>(ks) * A * 512, A * 512, &full[s]);
         } else {
-          bulk_load(st + L::IDX_OFF, idx_src + static_cast<size_t>(ks) * 8192, 8192, &full[s]);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)                // the stage's four K-quarter slabs
+            bulk_load(st + L::IDX_OFF + c * 2048, idx_src + (static_cast<size_t>(c) * KS + ks) * 2048, 2048, &full[s]);
           const int qbk = cb_split ? 2 * ks : (ks * kStageK) / qk;
           bulk_load(st + L::CB_OFF, cb_src + static_cast<size_t>(qbk) * 256, cb_split ? 1024 : 512, &full[s]);
           if constexpr (WSRC == WSRC_VQ_DIRECT) {
@@ -567,7 +569,9 @@ __global__ void __launch_bounds__(160)
   if (threadIdx.x == 0) {
     const uint32_t tx = 8192 + (cb_split ? 1024 : 512) + (L::kSVQ ? 128 * L::kG : A * 512);
     mbar_arrive_expect_tx(bar, tx);
-    bulk_load(st + L::IDX_OFF, w.idx + tile_id * 8192, 8192, bar);
+    for (int c = 0; c < 4; ++c)
+      bulk_load(st + L::IDX_OFF + c * 2048, w.idx + ((static_cast<size_t>(n_tile) * 4 + c) * KS + ks) * 2048, 2048,
+                bar);
     const int qbn = static_cast<int>((static_cast<int64_t>(n_tile) * 128) / qn);
     const int qbk = cb_split ? 2 * ks : (ks * kStageK) / qk;
     bulk_load(st + L::CB_OFF, w.cb + (static_cast<size_t>(qbn) * (K / qk) + qbk) * 256, cb_split ? 1024 : 512,

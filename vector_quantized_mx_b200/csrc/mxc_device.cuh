@@ -107,6 +107,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -205,6 +214,63 @@ __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
 // Full cluster barrier (release on arrive, acquire on wait); all threads, warp-converged.
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+
+// Split cluster barrier (non-aligned forms: threads may arrive and wait at
+// different points of the program).
+// Relaxed arrive: orders nothing by itself (a release arrive would also wait for
+// this thread's outstanding memory traffic); mbarrier initialisation is published
+// by fence.mbarrier_init before it.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+// 16-byte store into another CTA's shared memory whose completion counts 16 bytes
+// on that CTA's mbarrier (both addresses from mapa_shared).
+__device__ __forceinline__ void st_async_v4_f32(uint32_t remote_addr, float a, float b, float c, float d,
+                                                uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   remote_addr),
+               "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
+               : "memory");
+}
+// Arrive on an mbarrier of another CTA of the cluster (release at cluster scope).
+__device__ __forceinline__ void mbar_remote_arrive(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+
+// ------------------------------------------------------------------------------------
+// Programmatic dependent launch and L2 prefetch
+// ------------------------------------------------------------------------------------
+// Without the launch attribute both are no-ops.  A kernel reads nothing that the
+// previous kernel of the stream may have written, and writes nothing, before
+// griddep_wait() returns in the thread doing it.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Fetch [src, src + bytes) into L2 (no completion, no data returned).  src 16-byte
+// aligned, bytes a multiple of 16.  Reads through L2 stay coherent with later writes,
+// so a prefetch is safe before griddep_wait().
+__device__ __forceinline__ void l2_prefetch_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void l2_prefetch_tile_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+// 16-byte read-only global load (non-coherent path; L1 may serve the other half of
+// a 32-byte sector fetched for a neighbouring load).
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
 }
 
 // TMEM -> registers: this warp's 32 lanes x 32 consecutive 32-bit columns.
