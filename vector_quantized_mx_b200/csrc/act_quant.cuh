@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(
     quantize_unit<B>(x, M, K, ldx, e4m3, s, q, ldq, sf, u, kb_per_row, offsets, tile_prefix, n_groups);
 }
 
-// Small activations (decode batches): one launch of one 8-CTA cluster, one pass.
+// Small activations (decode batches): one launch of one 16-CTA (else 8-CTA) cluster, one pass.
 // Each thread loads its (at most two) blocks into registers once; for E4M3 the CTA
 // maxima are pushed into every CTA's shared memory (distributed shared memory,
 // one cluster barrier), so each thread then has the tensor amax locally and
@@ -220,30 +220,30 @@ __global__ void __launch_bounds__(256) quantize_kernel(
 // its wait before the pushes make sure every CTA runs before it is written to).
 // Padding scale rows [M, round_up(M,128))
 // are cleared word by word.
-constexpr int kSmallQuantCtas = 8;
-constexpr int kSmallQuantThreads = 512;
+constexpr int kSmallQuantThreadsAll = 4096;       // threads of the cluster
 constexpr int kSmallQuantElems = 16 * 8192;       // M*K up to this takes the one-cluster path
 
 __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-template <int B>
-__global__ void __launch_bounds__(kSmallQuantThreads) quantize_small_kernel(
+template <int B, int CTAS>
+__global__ void __launch_bounds__(kSmallQuantThreadsAll / CTAS) quantize_small_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t K, int64_t ldx, int e4m3,
     const float* __restrict__ tscale_in, uint8_t* __restrict__ q, int64_t ldq, uint8_t* __restrict__ sf,
     float* __restrict__ tscale_out, int64_t sf_rows) {
-  constexpr int kThreadsAll = kSmallQuantCtas * kSmallQuantThreads;
+  constexpr int kThreadsAll = kSmallQuantThreadsAll;
+  constexpr int kThreads = kThreadsAll / CTAS;
   constexpr int kUPT = (kSmallQuantElems / B + kThreadsAll - 1) / kThreadsAll;   // blocks per thread
-  __shared__ uint32_t red[kSmallQuantThreads / 32];
-  __shared__ uint32_t cta_max[kSmallQuantCtas];
+  __shared__ uint32_t red[kThreads / 32];
+  __shared__ uint32_t cta_max[CTAS];
   const bool need_amax = e4m3 && !tscale_in;
   if (need_amax) cluster_arrive_relaxed();  // "started": no remote store before every CTA runs
   griddep_launch_dependents();              // the next kernel may set up meanwhile
   griddep_wait();                           // x may come from the previous kernel
   const uint32_t rank = cluster_ctarank();
   const int kb_per_row = static_cast<int>(K / B);
-  const uint32_t g = rank * kSmallQuantThreads + threadIdx.x;
+  const uint32_t g = rank * kThreads + threadIdx.x;
   const uint32_t units = static_cast<uint32_t>(M) * kb_per_row;
   // this thread's blocks, in registers
   uint32_t w[kUPT][B / 2];
@@ -278,16 +278,17 @@ __global__ void __launch_bounds__(kSmallQuantThreads) quantize_small_kernel(
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
     cluster_wait_acquire();                  // every CTA of the cluster is running
     __syncthreads();
-    if (threadIdx.x < kSmallQuantCtas) {     // push this CTA's maximum into CTA threadIdx.x
+    if (threadIdx.x < CTAS) {                // push this CTA's maximum into CTA threadIdx.x
       uint32_t mm = 0;
 #pragma unroll
-      for (int i = 0; i < kSmallQuantThreads / 32; ++i) mm = max(mm, red[i]);
+      for (int i = 0; i < kThreads / 32; ++i) mm = max(mm, red[i]);
       st_cluster_u32(mapa_shared(smem_u32(&cta_max[rank]), threadIdx.x), mm);
     }
+    __syncwarp();                            // the cluster barrier is warp-aligned
     cluster_sync_all();                      // all maxima everywhere; nothing remote after this
     uint32_t mm = 0;
 #pragma unroll
-    for (int i = 0; i < kSmallQuantCtas; ++i) mm = max(mm, cta_max[i]);
+    for (int i = 0; i < CTAS; ++i) mm = max(mm, cta_max[i]);
     const float amax = __uint_as_float(mm << 16);
     s = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
   }
@@ -347,35 +348,63 @@ cudaError_t launch_group_prologue(const int32_t* offsets, int32_t E, int64_t M, 
   return cudaGetLastError();
 }
 
+template <int B, int CTAS>
+cudaError_t launch_quantize_small_ctas(const QuantizeArgs& a, const uint16_t* xp, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CTAS);
+  cfg.blockDim = dim3(kSmallQuantThreadsAll / CTAS);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CTAS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const int e4m3 = B == 16;
+  const float* tin = e4m3 ? a.tscale_in : nullptr;
+  cudaError_t err = cudaLaunchKernelEx(&cfg, quantize_small_kernel<B, CTAS>, xp, a.M, a.K, a.ldx, e4m3, tin, a.q,
+                                       a.ldq, a.sf, a.tscale_out, a.sf_rows);
+  if (err != cudaSuccess) return err;
+  return cudaGetLastError();
+}
+
+// A cluster of 16 CTAs (non-portable size) where the device schedules one, else 8.
+template <int B>
+cudaError_t launch_quantize_small(const QuantizeArgs& a, const uint16_t* xp, cudaStream_t stream) {
+  static int use16 = -1;                     // decided once per process
+  if (use16 < 0) {
+    auto k = quantize_small_kernel<B, 16>;
+    int n = 0;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(16);
+      cfg.blockDim = dim3(kSmallQuantThreadsAll / 16);
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 16;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();                      // clear a refusal of the query
+    use16 = n > 0 ? 1 : 0;
+  }
+  return use16 ? launch_quantize_small_ctas<B, 16>(a, xp, stream) : launch_quantize_small_ctas<B, 8>(a, xp, stream);
+}
+
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
   const bool e4m3 = a.fmt == MXC_FMT_E4M3_B16;
   const int B = e4m3 ? 16 : 32;
   unsigned int* amax_ws = reinterpret_cast<unsigned int*>(a.ws);
   if (!a.tile_prefix && a.M * a.K <= kSmallQuantElems) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kSmallQuantCtas);
-    cfg.blockDim = dim3(kSmallQuantThreads);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kSmallQuantCtas;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
     const uint16_t* xp = reinterpret_cast<const uint16_t*>(a.x);
-    cudaError_t err;
-    if (e4m3) {
-      err = cudaLaunchKernelEx(&cfg, quantize_small_kernel<16>, xp, a.M, a.K, a.ldx, 1, a.tscale_in, a.q, a.ldq,
-                               a.sf, a.tscale_out, a.sf_rows);
-    } else {
-      err = cudaLaunchKernelEx(&cfg, quantize_small_kernel<32>, xp, a.M, a.K, a.ldx, 0,
-                               static_cast<const float*>(nullptr), a.q, a.ldq, a.sf, a.tscale_out, a.sf_rows);
-    }
-    if (err != cudaSuccess) return err;
-    return cudaGetLastError();
+    if (e4m3) return launch_quantize_small<16>(a, xp, stream);
+    return launch_quantize_small<32>(a, xp, stream);
   }
   if (e4m3 && !a.tscale_in) {
     cudaError_t err = cudaMemsetAsync(amax_ws, 0, sizeof(unsigned int), stream);

@@ -18,11 +18,10 @@
 //     warp issues the block-scaled MMAs of quarter j of all stages while quarter
 //     j+1 is decoded.  Native FP4 weights use the same quarter-major MMA order, so
 //     both give bit-identical results on the same operands;
-//   * the index slabs pass through a ring of three quarter buffers (quarter 3
-//     reuses quarter 0's buffer once it is decoded), which leaves room to bring
-//     the weight scale atoms in by one bulk copy for tcgen05.cp from the MMA warp;
-//     the token scale atoms (16 rows) go from registers to TMEM with tcgen05.st,
-//     in the layout the tcgen05.cp 32x128b.warpx4 copy gives;
+//   * the index slabs pass through two quarter buffers (quarters 2 and 3 reuse
+//     the buffers of quarters 0 and 1 once those are decoded), which leaves room
+//     to bring the weight and token scale atoms in by bulk copies; the MMA warp
+//     moves both to TMEM with tcgen05.cp;
 //   * split-K partial tiles go to the cluster's rank 0 by st.async with completion
 //     on an mbarrier there; rank 0 adds them in rank order (deterministic).
 //
@@ -62,11 +61,14 @@ struct GemvLayout {
   static constexpr int S = kGemvMaxStages;
   static constexpr int W_OFF = 0;                      // S x [128][128 B] FP4, 128-byte swizzle
   static constexpr int X_OFF = W_OFF + S * 16384;      // S x [16][128 B] FP4 token tiles
-  // index slabs, 3 buffers x [S stages][128][16 B] (quarter j in buffer j mod 3,
-  // quarter 3 in buffer 0); afterwards rank 0's receive area for the other ranks'
-  // partial tiles, [rank-1][128][16] FP32
+  // index slabs, 2 buffers x [S stages][128][16 B] (quarter j in buffer j mod 2),
+  // then the token scale atoms (one buffer).  Rank 0 receives the other ranks'
+  // partial tiles, [rank-1][128][16] FP32, in the token-scale buffer (2 ranks,
+  // free once the scales are in TMEM) or from the start of the index buffers
+  // (more ranks, free once rank 0 has decoded).
   static constexpr int IDX_OFF = X_OFF + S * kGemvT * 128;
   static constexpr int IDX_BUF = S * 2048;
+  static constexpr int SFX_OFF = IDX_OFF + 2 * IDX_BUF;
   static constexpr int SFW_OFF = IDX_OFF + 3 * IDX_BUF;           // weight scale atoms (direct, native)
   static constexpr int LUT_OFF = SFW_OFF + (kSVQ ? 0 : S * kAtoms * 512);   // 128 words x 32 lanes
   static constexpr int CTRL_OFF = LUT_OFF + (kVQ ? 16384 : 0);
@@ -80,7 +82,7 @@ struct GemvLayout {
   static constexpr int COL_SFW = 32;
   static constexpr int COL_SFX = COL_SFW + S * kAtoms * 4;
   static constexpr int TMEM_COLS = COL_SFX + S * kAtoms * 4 <= 256 ? 256 : 512;
-  static_assert(RED <= 3 * IDX_BUF, "receive area");
+  static_assert(RED <= 2 * IDX_BUF && 128 * kGemvT * 4 <= IDX_BUF, "receive areas");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
@@ -120,7 +122,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* red_ready = bars + 16;  // rank > 0: rank 0 may receive
   uint64_t* bar_sfw = bars + 17;    // weight scale atoms (bulk copy)
   uint64_t* bar_cb = bars + 18;     // codebooks of the slice (bulk copy)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  uint64_t* bar_sfx = bars + 20;    // token scale atoms (bulk copy)
+  uint64_t* sfx_free = bars + 21;   // their tcgen05.cp copies are done: the buffer is free
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = p.K, KS = K / kStageK, KB4 = K / L::kB / 4;
@@ -142,14 +146,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint8_t* const w_sidx = p.w.sidx + (static_cast<size_t>(n_tile) * KS + ks_begin) * (128 * L::kG);
   const uint8_t* const a_sf =
       p.a_sf + (static_cast<size_t>(sf_group0) * KB4 + static_cast<size_t>(ks_begin) * A) * 512;
+  const int red_off = splits == 2 ? L::SFX_OFF : L::IDX_OFF;   // rank 0's receive area
   // codebooks used by the slice: a contiguous range [qb0, qb1] of the band's row
   const int qb0 = !L::kVQ ? 0 : H == 2 ? 2 * ks_begin : (ks_begin * kStageK) / p.qk;
   const int qb1 = !L::kVQ ? 0 : H == 2 ? 2 * ks_end - 1 : ((ks_end - 1) * kStageK) / p.qk;
 
   // ---- setup (nothing here depends on earlier kernels) ----
   if (warp == 0) {
-    // full[0..7], bar_x, dec_ph[0..3], sf_ready, accum, red_full, red_ready, bar_sfw, bar_cb
-    if (lane < 19) mbar_init(bars + lane, (lane >= 9 && lane < 14) ? kDecWarps : 1);
+    // full[0..7], bar_x, dec_ph[0..3], sf_ready, accum, red_full, red_ready, bar_sfw, bar_cb,
+    // (unused), bar_sfx, sfx_free
+    if (lane < 22) mbar_init(bars + lane, (lane >= 9 && lane < 14) ? kDecWarps : 1);
     __syncwarp();
   }
   if (warp == 0 && lane == 0) {
@@ -175,6 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if (warp == 1) {
+    __syncwarp();                                    // tcgen05.alloc is warp-aligned
     tmem_alloc(tmem_slot, L::TMEM_COLS);
     tmem_relinquish();
   }
@@ -204,18 +211,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // =============================== loader ===============================
+    __syncwarp();
     if (elect_one()) {
       // in the order they are needed: codebooks, index quarter 0, scales, tokens, quarters 1..3
       if constexpr (L::kVQ) {
         const uint32_t cb_bytes = static_cast<uint32_t>(qb1 - qb0 + 1) * 512;
         mbar_arrive_expect_tx(bar_cb, cb_bytes);
         bulk_load(smem + L::CB_OFF, w_cb + static_cast<size_t>(qb0) * 256, cb_bytes, bar_cb);
-#ifdef MXC_GEMV_CB_ALONE
-        mbar_wait(bar_cb, 0);                        // the codebooks land alone, first
-#endif
         mbar_arrive_expect_tx(&full[0], nks * 2048);
         bulk_load(smem + L::IDX_OFF, w_idx, nks * 2048, &full[0]);
       }
+      mbar_arrive_expect_tx(bar_sfx, nks * A * 512);
+      bulk_load(smem + L::SFX_OFF, a_sf, nks * A * 512, bar_sfx);
       if constexpr (!L::kSVQ) {
         mbar_arrive_expect_tx(bar_sfw, nks * A * 512);
         bulk_load(smem + L::SFW_OFF, w_sf, nks * A * 512, bar_sfw);
@@ -226,9 +233,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(smem + L::X_OFF, &tmap_x, 0, static_cast<int>(m0), ks_begin, bar_x);
       if constexpr (L::kVQ) {
         for (int j = 1; j < 4; ++j) {                // K-quarter j of every stage
-          if (j == 3 && !mbar_wait(&dec_ph[0], 0)) break;   // buffer 0 is free again
+          if (j >= 2 && !mbar_wait(&dec_ph[j - 2], 0)) break;   // its buffer has been decoded
           mbar_arrive_expect_tx(&full[j], nks * 2048);
-          bulk_load(smem + L::IDX_OFF + (j % 3) * L::IDX_BUF, w_idx + static_cast<size_t>(j) * KS * 2048, nks * 2048,
+          bulk_load(smem + L::IDX_OFF + (j % 2) * L::IDX_BUF, w_idx + static_cast<size_t>(j) * KS * 2048, nks * 2048,
                     &full[j]);
         }
       } else {
@@ -240,10 +247,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
     if (splits > 1 && rank == 0) {
-      // The index buffers are rank 0's receive area once its decoders are done with
-      // them: then let the other ranks send their partials (even after a failed
-      // wait, so that no rank waits for the signal in vain).
-      if constexpr (L::kVQ) mbar_wait(&dec_ph[3], 0);
+      // Let the other ranks send their partials once the receive area is free:
+      // the token-scale buffer after its tcgen05.cp copies (2 ranks), the index
+      // buffers after the last decode phase (more ranks).  Sent even after a
+      // failed wait, so that no rank waits for the signal in vain.
+      if (splits == 2) {
+        mbar_wait(sfx_free, 0);
+      } else if constexpr (L::kVQ) {
+        mbar_wait(&dec_ph[3], 0);
+      }
       if (lane > 0 && lane < splits) mbar_remote_arrive(mapa_shared(smem_u32(red_ready), lane));
     }
   } else if (warp == 1) {
@@ -260,8 +272,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     }
+    {
+      // token scale atoms -> TMEM, then free their buffer for index quarter 2
+      const bool got = __all_sync(0xffffffffu, mbar_wait(bar_sfx, 0));
+      if (got && elect_one()) {
+        const uint32_t sfx_s0 = smem_u32(smem + L::SFX_OFF);
+        for (int i = 0; i < nks * A; ++i)
+          tc_cp_32x128b_warpx4(tmem + L::COL_SFX + 4 * i, sdesc_sf_atom(sfx_s0 + i * 512));
+      }
+      __syncwarp();
+      if (elect_one()) tc_commit(sfx_free);          // arrives when the copies have read it (also on failure)
+      __syncwarp();
+      ok = got && ok;
+    }
     ok = __all_sync(0xffffffffu, mbar_wait(bar_x, 0)) && ok;
-    ok = __all_sync(0xffffffffu, mbar_wait(sf_ready, 0)) && ok;
+    if constexpr (L::kSVQ) ok = __all_sync(0xffffffffu, mbar_wait(sf_ready, 0)) && ok;
     if constexpr (!L::kVQ) {
       for (int s = 0; s < nks && ok; ++s) ok = __all_sync(0xffffffffu, mbar_wait(&full[s], 0));
     }
@@ -314,30 +339,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       *c1 = cp[1];
     };
 
-    // --- token scale atoms (and PreScale+ weight scales) -> TMEM lanes of this
-    //     warp's quadrant; atoms i = cg mod 4.  Loads now, stores after phase 0. ---
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(qd * 32) << 16);
-    const int natoms = nks * A;
-    constexpr int kPer = L::S * A / 4;               // atoms per warp, at most
-    uint4 sx[kPer];
-#pragma unroll
-    for (int t = 0; t < kPer; ++t) {                 // rows 0..15 of the atom are the 16 tokens
-      const int i = cg + 4 * t;
-      sx[t] = (i < natoms && lane < kGemvT) ? ldg_nc_v4(a_sf + static_cast<size_t>(i) * 512 + lane * 16)
-                                            : make_uint4(0, 0, 0, 0);
-    }
-    auto scales_to_tmem = [&]() {
-#pragma unroll
-      for (int t = 0; t < kPer; ++t) {
-        const int i = cg + 4 * t;
-        if (i < natoms) tmem_st_32x32b_x4(lane_base + L::COL_SFX + 4 * i, sx[t]);
-      }
+    // --- PreScale+ weight scale atoms -> TMEM lanes of this warp's quadrant
+    //     (atoms i = cg mod 4), after decode phase 0 ---
+    auto svq_scales_to_tmem = [&]() {
       if constexpr (L::kSVQ) {
+        __syncwarp();                                // tcgen05.st is warp-aligned
         // PreScale+ (Table 4 caption: Ks = 256, ds = 8): row `lane` of atom (s, a)
         // holds, for rows 32 g + lane (g = 0..3), scales 4a..4a+3 of stage s, i.e.
         // word a mod 2 of the 8-byte scale-codebook entry of scale group a/2.
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(qd * 32) << 16);
         const uint32_t* scb32 = reinterpret_cast<const uint32_t*>(p.w.scb);
-        for (int i = cg; i < natoms; i += 4) {
+        for (int i = cg; i < nks * A; i += 4) {
           const int s = i / A, a = i % A;
           const uint8_t* si = w_sidx + static_cast<size_t>(s) * 128 * L::kG + (a >> 1);
           uint4 v;
@@ -347,13 +359,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           v.w = __ldg(scb32 + 2 * __ldg(si + (3 * 32 + lane) * L::kG) + (a & 1));
           tmem_st_32x32b_x4(lane_base + L::COL_SFW + 4 * i, v);
         }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sf_ready);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sf_ready);
     };
-    if constexpr (!L::kVQ) scales_to_tmem();
 
     if constexpr (L::kVQ) {
       // both codebooks into registers now: the staging area is overwritten by the
@@ -393,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             const int r = (q + 64 * i + s_l) & 127;  // offset by the stage: conflict-free stores
-            const uint4 iv = *reinterpret_cast<const uint4*>(idx_l + (j % 3) * L::IDX_BUF + r * 16);
+            const uint4 iv = *reinterpret_cast<const uint4*>(idx_l + (j % 2) * L::IDX_BUF + r * 16);
             const uint4 o0 = make_uint4(lut16_pair(lut_lane, iv.x, 0), lut16_pair(lut_lane, iv.x, 2),
                                         lut16_pair(lut_lane, iv.y, 0), lut16_pair(lut_lane, iv.y, 2));
             const uint4 o1 = make_uint4(lut16_pair(lut_lane, iv.z, 0), lut16_pair(lut_lane, iv.z, 2),
@@ -405,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();                    // tile writes -> tensor-core operand reads
         __syncwarp();
         if (lane == 0) mbar_arrive(&dec_ph[j]);
-        if (j == 0) scales_to_tmem();                // needed with quarter 0's MMAs
+        if (j == 0) svq_scales_to_tmem();            // needed with quarter 0's MMAs
       }
     }
     // ------------------------------ epilogue ------------------------------
@@ -413,10 +424,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const float scale = out_scale;
     uint32_t acc[4];
+    __syncwarp();                                    // tcgen05.ld is warp-aligned: converge after the waits
     tmem_ld_32x32b_x4(tmem + (static_cast<uint32_t>(qd * 32) << 16) + cg * 4, acc);
     tmem_ld_wait();
     float v[4] = {__uint_as_float(acc[0]), __uint_as_float(acc[1]), __uint_as_float(acc[2]), __uint_as_float(acc[3])};
-    const uint32_t red_slot = smem_u32(smem + L::IDX_OFF) + (row * kGemvT + cg * 4) * 4;
+    const uint32_t red_slot = smem_u32(smem + red_off) + (row * kGemvT + cg * 4) * 4;
     bool store = ep_ok;
     if (splits > 1) {
       if (rank != 0) {
@@ -430,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         store = store && got;
         if (store) {
           for (int r = 1; r < splits; ++r) {
-            const float4 o = *reinterpret_cast<const float4*>(smem + L::IDX_OFF + ((r - 1) * 128 * kGemvT +
+            const float4 o = *reinterpret_cast<const float4*>(smem + red_off + ((r - 1) * 128 * kGemvT +
                                                                                   row * kGemvT + cg * 4) * 4);
             v[0] += o.x;
             v[1] += o.y;
@@ -449,6 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (mbase + c < p.M) store_out(y, ldy, out_bf16, mbase + c, n, v[c] * scale);
     }
   }
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

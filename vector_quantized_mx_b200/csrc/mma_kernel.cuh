@@ -191,8 +191,10 @@ __device__ __forceinline__ void decode_sf_tile(const uint8_t* __restrict__ sidx,
   }
 }
 
+// Named barriers in their non-aligned form: threads of a warp may reach them from
+// divergent paths.
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Named barrier that also ANDs a predicate over the participating threads, so a
@@ -202,7 +204,7 @@ __device__ __forceinline__ bool named_bar_and(int id, int count, bool v) {
   asm volatile(
       "{\n\t.reg .pred pin, pout;\n\t"
       "setp.ne.u32 pin, %1, 0;\n\t"
-      "bar.red.and.pred pout, %2, %3, pin;\n\t"
+      "barrier.red.and.pred pout, %2, %3, pin;\n\t"
       "selp.u32 %0, 1, 0, pout;\n\t}"
       : "=r"(r)
       : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(count)
@@ -296,6 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (WSRC == WSRC_NATIVE) prefetch_tensormap(&tmap_wq);
   }
   if (warp == 1) {
+    __syncwarp();                                  // tcgen05.alloc is warp-aligned
     tmem_alloc(tmem_slot, L::TMEM_COLS);
     tmem_relinquish();
   }
@@ -467,6 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t taddr = tmem + (static_cast<uint32_t>(qd * 32) << 16) + chalf * TCOL;
     if constexpr (T <= 32) {
       // this warp's accumulator columns in registers: one TMEM round trip
+      __syncwarp();                                  // tcgen05.ld is warp-aligned: converge after the waits
       if constexpr (TCOL == 4) tmem_ld_32x32b_x4(taddr, acc_regs);
       else if constexpr (TCOL == 8) tmem_ld_32x32b_x8(taddr, acc_regs);
       else tmem_ld_32x32b_x16(taddr, acc_regs);
@@ -491,6 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int c0 = 0; c0 < TCOL; c0 += 32) {
         uint32_t v[32];
+        __syncwarp();                                // tcgen05.ld is warp-aligned
         tmem_ld_32x32b_x32(taddr + c0, v);
         tmem_ld_wait();
         if (!ep_ok) continue;
@@ -504,6 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
