@@ -130,7 +130,7 @@ def blas_threads():
 def cpu_baseline(w, x, budget_s=12.0):
     rows_per = 1024           # 1/9 of N_out per sample (whole 256-row QBlocks)
     t_tot, b_tot, n = 0.0, 0, 0
-    while t_tot < budget_s and n < 8:
+    while t_tot < budget_s and n < 200:
         r0 = (n * rows_per) % w.N
         dt, b = oracle_sample(w, x, slice(r0, r0 + rows_per))
         t_tot += dt
