@@ -67,7 +67,9 @@ inline bool make_fp4_stage_map(CUtensorMap* map, const void* base, int64_t rows,
 constexpr int kDecodeMaxM = 16;   // M <= 16: split-K decode path with a 16-token tile
 constexpr int kSMs = 148;
 
-inline int token_tile(int64_t M) { return M <= kDecodeMaxM ? 16 : 128; }
+// Token tile (the MMA's N): 16 for decode, 256 for prefill (each decoded or loaded
+// 128-row weight tile then feeds twice the tensor-core work), 128 in between.
+inline int token_tile(int64_t M) { return M <= kDecodeMaxM ? 16 : M <= 128 ? 128 : 256; }
 
 // Split-K factor of the decode path: the CTAs of one 128-row output tile form a
 // cluster of `splits`; choose the largest factor (<= kMaxSplits) that keeps all
@@ -142,6 +144,7 @@ template <int FMT, int WSRC>
 cudaError_t dispatch_tile(int T, const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams<1>& p, dim3 grid,
                           cudaStream_t stream) {
   if (T == 16) return dispatch_dense<FMT, WSRC, 16>(tx, tw, p, grid, stream);
+  if (T == 256) return dispatch_dense<FMT, WSRC, 256>(tx, tw, p, grid, stream);
   return dispatch_dense<FMT, WSRC, 128>(tx, tw, p, grid, stream);
 }
 

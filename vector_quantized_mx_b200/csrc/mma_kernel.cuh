@@ -326,7 +326,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qbn = static_cast<int>((static_cast<int64_t>(n_tile) * 128) / qn);
     const int cb_per_row = K / qk;
     constexpr bool cb_split = NCB == 2;
-    uint32_t tx = T * 128 + XG * A * 512;
+    // Token scale groups that exist: the SF buffer holds ceil(M/128) groups of 128
+    // rows (dense) -- a 256-token tile at the end of M may cover only one.
+    int xg_valid = XG;
+    if constexpr (!MOE) {
+      const int groups = static_cast<int>((static_cast<int64_t>(p.M) + 127) / 128);
+      xg_valid = groups - sf_group0 < XG ? groups - sf_group0 : XG;
+    }
+    uint32_t tx = T * 128 + xg_valid * A * 512;
     if constexpr (WSRC == WSRC_NATIVE) tx += 16384 + A * 512;
     if constexpr (WSRC == WSRC_VQ_DIRECT) tx += 8192 + (cb_split ? 1024 : 512) + A * 512;
     if constexpr (WSRC == WSRC_VQ_SVQ) tx += 8192 + (cb_split ? 1024 : 512) + 128 * L::kG;
@@ -348,8 +355,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(st + L::X_OFF, &tmap_x, ks * 128, y0, &full[s]);
 #pragma unroll
         for (int g = 0; g < XG; ++g)
-          bulk_load(st + L::SFX_OFF + g * A * 512, sfx_src + (static_cast<size_t>(g) * KB4 + ks * A) * 512,
-                    A * 512, &full[s]);
+          if (g < xg_valid)                          // a missing group's rows are past M: never stored
+            bulk_load(st + L::SFX_OFF + g * A * 512, sfx_src + (static_cast<size_t>(g) * KB4 + ks * A) * 512,
+                      A * 512, &full[s]);
         if constexpr (WSRC == WSRC_NATIVE) {
           tma_load_2d(st + L::W_OFF, &tmap_wq, ks * 128, n_tile * 128, &full[s]);
           bulk_load(st + L::SFW_OFF, sfw_src + static_cast<size_t>(ks) * A * 512, A * 512, &full[s]);
