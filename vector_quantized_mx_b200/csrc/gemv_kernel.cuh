@@ -93,15 +93,6 @@ __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint4 v) {
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Two index bytes (k, k+1 of word x) -> 8 FP4 values (32 bits) through this lane's
-// codebook copy: 16-bit entries, two per word, word (e/2)*32 + lane.  The two
-// lookups are merged with one byte permute whose selector picks each entry's half.
-__device__ __forceinline__ uint32_t lut16_pair(uint32_t lut_lane, uint32_t x, int k) {
-  const uint32_t wa = lds_u32(lut_lane + (((x >> (8 * k + 1)) & 0x7Fu) << 7));
-  const uint32_t wb = lds_u32(lut_lane + (((x >> (8 * k + 9)) & 0x7Fu) << 7));
-  return __byte_perm(wa, wb, 0x5410u + ((x >> (8 * k)) & 0x101u) * 0x22u);
-}
-
 template <int FMT, int WSRC>
 __global__ void __launch_bounds__(kThreads, 1)
     gemv_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_wq,

@@ -88,7 +88,7 @@ struct StageLayout {
   static constexpr int END = SIDX_OFF + (kSVQ ? 128 * kG : 0);
   static constexpr int BYTES = (END + 1023) / 1024 * 1024;
   static constexpr int CTRL = 4096;                   // barriers, TMEM slot, scale codebook
-  static constexpr int LUT = kVQ ? NCB * 256 * 32 * 4 : 0;           // per-lane codebook copies (32 KB each)
+  static constexpr int LUT = kVQ ? 2 * NCB * 128 * 32 * 4 : 0;       // 2 buffers of per-lane codebook copies
   static constexpr int RED = T <= 32 ? (kMaxSplits - 1) * T * 128 * 4 : 0;  // split-K receive slots
   static constexpr int BUDGET = 227 * 1024 - 1024 - CTRL - LUT - RED;
   static constexpr int STAGES = (BUDGET / BYTES) > 8 ? 8 : (BUDGET / BYTES);
@@ -117,22 +117,31 @@ constexpr int kThreads = 64 + kDecThreads;         // + loader warp + MMA warp
 // ------------------------------------------------------------------------------------
 // Decoders (shared with the decode-dump kernel).  dt = decoder thread 0..NT-1.
 // ------------------------------------------------------------------------------------
-// Per-lane codebook copies: 32-bit word (e*32 + lane) holds centroid e (its 16-bit
-// entry, zero-extended), so the 32 lanes of a warp always read 32 different banks
-// and a lookup is one byte extract, one shift-add and one shared load.  `ncb` = 1
-// or 2 codebooks (two when the QBlock is 128 wide along K), 32 KB each.  Stores
-// are 16 B per thread over consecutive addresses (bank-conflict free).
+// Per-lane codebook copies with 16-bit entries: word (j*32 + lane) holds centroids
+// 2j (low half) and 2j+1 (high half), so the 32 lanes of a warp always read 32
+// different banks.  `ncb` = 1 or 2 codebooks (two when the QBlock is 128 wide along
+// K), 16 KB each.  Stores are 16 B per thread over consecutive addresses (bank-
+// conflict free).
+constexpr int kLutBytes = 128 * 32 * 4;
 template <int NT>
 __device__ __forceinline__ void build_lut(const uint16_t* __restrict__ cb, int ncb, uint32_t* __restrict__ lut,
                                           int dt) {
-  for (int u = dt; u < 2048 * ncb; u += NT) {   // uint4 u: words 4u..4u+3 = entry u/8, lanes 4(u%8)..
-    const uint32_t v = cb[u >> 3];
+  const uint32_t* cb32 = reinterpret_cast<const uint32_t*>(cb);
+  for (int u = dt; u < 1024 * ncb; u += NT) {   // uint4 u: words 4u..4u+3 = entry word u/8, lanes 4(u%8)..
+    const uint32_t v = cb32[u >> 3];
     reinterpret_cast<uint4*>(lut)[u] = make_uint4(v, v, v, v);
   }
 }
 
-// Byte k of w, zero-extended.
-__device__ __forceinline__ uint32_t byte_of(uint32_t w, int k) { return __byte_perm(w, 0u, 0x4440 | k); }
+// Two index bytes (k, k+1 of word x) -> 8 FP4 values (32 bits) through this lane's
+// codebook copy (lut_lane = copy base + lane*4): the word (e/2)*32 + lane holds
+// entry e in half e%2; one byte permute merges both lookups, its selector picking
+// each entry's half.
+__device__ __forceinline__ uint32_t lut16_pair(uint32_t lut_lane, uint32_t x, int k) {
+  const uint32_t wa = lds_u32(lut_lane + (((x >> (8 * k + 1)) & 0x7Fu) << 7));
+  const uint32_t wb = lds_u32(lut_lane + (((x >> (8 * k + 9)) & 0x7Fu) << 7));
+  return __byte_perm(wa, wb, 0x5410u + ((x >> (8 * k)) & 0x101u) * 0x22u);
+}
 
 // One 128 x 256 weight tile: idx (four K-quarter slabs [128][16] bytes) -> FP4
 // [128][128] bytes in the 128-byte swizzle (16-byte chunk j of row r stored at chunk j ^ (r % 8)).
@@ -152,7 +161,7 @@ struct ChunkMap {
       const int r = c >> 3, j = c & 7;
       idx_off[it] = (j >> 1) * 2048 + r * 16 + (j & 1) * 8;   // K-quarter slab j/2
       w_off[it] = r * 128 + ((j ^ (r & 7)) << 4);
-      lut_off[it] = ((cb_split && j >= 4) ? 256 * 32 * 4 : 0) + (dt & 31) * 4;
+      lut_off[it] = ((cb_split && j >= 4) ? kLutBytes : 0) + (dt & 31) * 4;
     }
   }
 };
@@ -164,13 +173,9 @@ __device__ __forceinline__ void decode_w_tile(const uint8_t* __restrict__ idx, u
   for (int it = 0; it < ChunkMap<NT>::kN; ++it) {
     const uint2 iv = *reinterpret_cast<const uint2*>(idx + cm.idx_off[it]);
     const uint32_t base = lut_s + cm.lut_off[it];
-#define MXC_LUT(w, k) lds_u32(base + (byte_of(w, k) << 7))
-    const uint32_t e0 = MXC_LUT(iv.x, 0), e1 = MXC_LUT(iv.x, 1), e2 = MXC_LUT(iv.x, 2), e3 = MXC_LUT(iv.x, 3);
-    const uint32_t e4 = MXC_LUT(iv.y, 0), e5 = MXC_LUT(iv.y, 1), e6 = MXC_LUT(iv.y, 2), e7 = MXC_LUT(iv.y, 3);
-#undef MXC_LUT
     *reinterpret_cast<uint4*>(wt + cm.w_off[it]) =
-        make_uint4(__byte_perm(e0, e1, 0x5410), __byte_perm(e2, e3, 0x5410), __byte_perm(e4, e5, 0x5410),
-                   __byte_perm(e6, e7, 0x5410));
+        make_uint4(lut16_pair(base, iv.x, 0), lut16_pair(base, iv.x, 2), lut16_pair(base, iv.y, 0),
+                   lut16_pair(base, iv.y, 2));
   }
 }
 
@@ -444,25 +449,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ======================= decoders, then epilogue ======================
     const int dt = threadIdx.x - 64;
     if constexpr (L::kVQ) {
+      // Codebook copies double-buffered: stage i decodes through buffer i%2 while the
+      // copies of stage i+1 go into the other buffer; one decoder barrier per stage
+      // (it also orders stage i's lookups before buffer i%2 is rebuilt).
       constexpr int cb_split = NCB == 2;
-      uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L::LUT_OFF);
+      constexpr int kBuf = NCB * kLutBytes;
+      uint8_t* lut = smem + L::LUT_OFF;
       const uint32_t lut_s = smem_u32(lut);
       ChunkMap<kDecThreads> cm;
       cm.init(dt, cb_split);
-      for (int i = 0; i < nks; ++i) {
+      bool ok = true;
+      if (nks > 0) {
+        const bool got = mbar_wait(&full[0], 0);
+        if (got)
+          build_lut<kDecThreads>(reinterpret_cast<const uint16_t*>(stages + L::CB_OFF), 1 + cb_split,
+                                 reinterpret_cast<uint32_t*>(lut), dt);
+        ok = named_bar_and(2, kDecThreads, got);     // one decision for all decoders
+      }
+      for (int i = 0; i < nks && ok; ++i) {
         const int s = i % STAGES;
-        const uint32_t ph = (i / STAGES) & 1;
-        // one decision for all decoders; also orders the previous stage's lookups
-        // before the codebook copies are rebuilt
-        if (!named_bar_and(2, kDecThreads, mbar_wait(&full[s], ph))) break;
         uint8_t* st = stages + s * L::BYTES;
-        build_lut<kDecThreads>(reinterpret_cast<const uint16_t*>(st + L::CB_OFF), 1 + cb_split, lut, dt);
-        named_bar_sync(2, kDecThreads);              // copies visible to all decoders
-        decode_w_tile<kDecThreads>(st + L::IDX_OFF, lut_s, st + L::W_OFF, cm);
+        decode_w_tile<kDecThreads>(st + L::IDX_OFF, lut_s + (i & 1) * kBuf, st + L::W_OFF, cm);
         if constexpr (L::kSVQ) decode_sf_tile<L::kG, kDecThreads>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, dt);
         fence_proxy_async_smem();                    // each thread's tile writes -> async proxy
         __syncwarp();
         if (lane == 0) mbar_arrive(&dec[s]);         // one arrival per decoder warp
+        if (i + 1 < nks) {                           // the next stage's copies, other buffer
+          const int s1 = (i + 1) % STAGES;
+          const bool got = mbar_wait(&full[s1], ((i + 1) / STAGES) & 1);
+          if (got)
+            build_lut<kDecThreads>(reinterpret_cast<const uint16_t*>(stages + s1 * L::BYTES + L::CB_OFF),
+                                   1 + cb_split, reinterpret_cast<uint32_t*>(lut + ((i + 1) & 1) * kBuf), dt);
+          ok = named_bar_and(2, kDecThreads, got);
+        }
       }
     }
     ep_ok = mbar_wait(accum, 0);
@@ -551,7 +570,7 @@ template <int FMT, int WSRC>
 struct DumpLayout {
   using L = StageLayout<FMT, WSRC, 16>;
   static constexpr int LUT_OFF = L::CTRL + L::BYTES;
-  static constexpr int SMEM = 1024 + LUT_OFF + 2 * 256 * 32 * 4;
+  static constexpr int SMEM = 1024 + LUT_OFF + 2 * kLutBytes;
 };
 
 template <int FMT, int WSRC>
