@@ -98,12 +98,10 @@ typedef struct mxc_mx_tensor {
 } mxc_mx_tensor;
 
 /* A VQ-coded weight W[N, K] in the packed device layout.
- *   idx     device, [N/128][4][K/256][128][16] bytes: for each 128-row band of
- *           output channels and each K-quarter c (64 input channels of every
- *           256-channel stage), the stages' slabs of 128 rows x 16 uint8 indices,
- *           2 KB each (index j of row n in slab (c, ks) covers
- *           k = 256 ks + 64 c + 4j .. + 3).  A band's quarter c is contiguous over
- *           the stages.
+ *   idx     device, [N/128][K/256][4][128][16] bytes: each 128-row x 256-column
+ *           tile (8 KB, tiles in row-major tile order) holds four K-quarter slabs
+ *           of 64 input channels; slab c holds, for each of the 128 rows, its 16
+ *           uint8 indices (index j covers k = 256 ks + 64 c + 4j .. + 3).
  *   cb      device, [N/qn][K/qk][256] uint16 FP4 codebooks; centroid element t
  *           (k mod 4) in bits 4t..4t+3.  512 bytes per QBlock.
  *   scales  device (PostScale/PreScale), SF layout of the [N, K/B] scale bytes.

@@ -56,12 +56,12 @@ def test_pack_layouts(L, fmt, strategy):
     N, K = 256, 768
     w = synth.make_weight(7, fmt, strategy, N, K, 128, 256)
     h = _pack(w)
-    # index slabs: [N/128][4 K-quarters][K/256][128 rows][16 bytes]
-    tiles = h["idx"].reshape(N // 128, 4, K // 256, 128, 16)
+    # index tiles: [N/128][K/256][4 K-quarter slabs][128 rows][16 bytes]
+    tiles = h["idx"].reshape(N // 128, K // 256, 4, 128, 16)
     for nt in range(N // 128):
         for ks in range(K // 256):
             for c in range(4):
-                assert np.array_equal(tiles[nt, c, ks],
+                assert np.array_equal(tiles[nt, ks, c],
                                       w.idx[nt * 128:(nt + 1) * 128, ks * 64 + c * 16:ks * 64 + (c + 1) * 16])
     B = synth.BLOCK[fmt]
     if strategy == "prescale_plus":

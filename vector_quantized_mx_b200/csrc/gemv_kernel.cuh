@@ -7,9 +7,10 @@
 // channels (split-K over the CTAs of a thread-block cluster) and keeps the slice on
 // chip:
 //
-//   * the loader copies the slice's index bytes with one bulk copy per K-quarter
-//     (the packed layout keeps, per 128-row band, quarter c of all stages
-//     contiguous), quarter 0 first, and all token tiles with one 3-D tensor copy;
+//   * the loader copies the slice's index bytes with one 4-D tensor copy per
+//     K-quarter (quarter c of every stage: the packed layout stores each 128 x 256
+//     tile as four slabs of 64 input channels), quarter 0 first, and all token
+//     tiles with one 3-D tensor copy;
 //   * decoder lane l decodes stage l mod 8, so the 32 per-lane codebook copies in
 //     shared memory hold, in bank l, the codebook of lane l's stage: the codebooks
 //     of the whole slice are laid out once (16-bit entries, 16 KB) and no lookup
@@ -96,7 +97,7 @@ __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.
 template <int FMT, int WSRC>
 __global__ void __launch_bounds__(kThreads, 1)
     gemv_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_wq,
-                const __grid_constant__ GemvParams p) {
+                const __grid_constant__ CUtensorMap tmap_idx, const __grid_constant__ GemvParams p) {
   using L = GemvLayout<FMT, WSRC>;
   constexpr int A = L::kAtoms;
   static_assert(kDecWarps == 16, "decode map assumes 16 decoder warps");
@@ -130,8 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int H = (L::kVQ && p.qk == 128) ? 2 : 1;     // codebooks per stage along K
   const int qbn = L::kVQ ? static_cast<int>((static_cast<int64_t>(n_tile) * 128) / p.qn) : 0;
   const int cb_per_row = L::kVQ ? K / p.qk : 0;
-  // quarter j of this slice: w_idx + j * KS * 2048, nks slabs of 2 KB
-  const uint8_t* const w_idx = p.w.idx + (static_cast<size_t>(n_tile) * 4 * KS + ks_begin) * 2048;
+  // this slice's index tiles: nks contiguous 8 KB tiles, quarter j at +2048 j in each
+  const uint8_t* const w_idx = p.w.idx + (static_cast<size_t>(n_tile) * KS + ks_begin) * 8192;
   const uint16_t* const w_cb = p.w.cb + static_cast<size_t>(qbn) * cb_per_row * 256;
   const uint8_t* const w_sf = p.w.sf + (static_cast<size_t>(n_tile) * KB4 + static_cast<size_t>(ks_begin) * A) * 512;
   const uint8_t* const w_sidx = p.w.sidx + (static_cast<size_t>(n_tile) * KS + ks_begin) * (128 * L::kG);
@@ -155,6 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     prefetch_tensormap(&tmap_x);
     if constexpr (WSRC == WSRC_NATIVE) prefetch_tensormap(&tmap_wq);
+    if constexpr (L::kVQ) prefetch_tensormap(&tmap_idx);
     // this CTA's weight stream into L2: codebooks and scales first, then the bulk
     if constexpr (L::kVQ) {
       l2_prefetch_bulk(w_cb + static_cast<size_t>(qb0) * 256, static_cast<uint32_t>(qb1 - qb0 + 1) * 512);
@@ -165,8 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       l2_prefetch_bulk(w_sf, static_cast<uint32_t>(nks) * A * 512);
     }
     if constexpr (L::kVQ) {
-      for (int j = 0; j < 4; ++j)
-        l2_prefetch_bulk(w_idx + static_cast<size_t>(j) * KS * 2048, static_cast<uint32_t>(nks) * 2048);
+      l2_prefetch_bulk(w_idx, static_cast<uint32_t>(nks) * 8192);
     } else {
       for (int s = 0; s < nks; ++s) l2_prefetch_tile_2d(&tmap_wq, (ks_begin + s) * 128, n_tile * 128);
     }
@@ -209,8 +210,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t cb_bytes = static_cast<uint32_t>(qb1 - qb0 + 1) * 512;
         mbar_arrive_expect_tx(bar_cb, cb_bytes);
         bulk_load(smem + L::CB_OFF, w_cb + static_cast<size_t>(qb0) * 256, cb_bytes, bar_cb);
-        mbar_arrive_expect_tx(&full[0], nks * 2048);
-        bulk_load(smem + L::IDX_OFF, w_idx, nks * 2048, &full[0]);
+        // quarter j of stages [ks_begin, ks_begin + ks_per_split): box {2048 B, 1, stages, 1};
+        // stages past K (last split) arrive zero-filled and are not used
+        mbar_arrive_expect_tx(&full[0], p.ks_per_split * 2048);
+        tma_load_4d(smem + L::IDX_OFF, &tmap_idx, 0, 0, ks_begin, n_tile, &full[0]);
       }
       mbar_arrive_expect_tx(bar_sfx, nks * A * 512);
       bulk_load(smem + L::SFX_OFF, a_sf, nks * A * 512, bar_sfx);
@@ -225,9 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (L::kVQ) {
         for (int j = 1; j < 4; ++j) {                // K-quarter j of every stage
           if (j >= 2 && !mbar_wait(&dec_ph[j - 2], 0)) break;   // its buffer has been decoded
-          mbar_arrive_expect_tx(&full[j], nks * 2048);
-          bulk_load(smem + L::IDX_OFF + (j % 2) * L::IDX_BUF, w_idx + static_cast<size_t>(j) * KS * 2048, nks * 2048,
-                    &full[j]);
+          mbar_arrive_expect_tx(&full[j], p.ks_per_split * 2048);
+          tma_load_4d(smem + L::IDX_OFF + (j % 2) * L::IDX_BUF, &tmap_idx, 0, j, ks_begin, n_tile, &full[j]);
         }
       } else {
         for (int s = 0; s < nks; ++s) {

@@ -61,6 +61,23 @@ inline bool make_fp4_stage_map(CUtensorMap* map, const void* base, int64_t rows,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D map over packed weight indices [N/128][K/256][4][128][16] seen as 8-byte
+// elements: dims {256 (one 2 KB K-quarter slab), 4 quarters, K/256 stages, N/128
+// bands}; one box = quarter q of box_stages consecutive stages of one band.
+inline bool make_idx_map(CUtensorMap* map, const void* base, int64_t N, int64_t K, int box_stages) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return false;
+  std::memset(map, 0, sizeof(*map));
+  const cuuint64_t KS = static_cast<cuuint64_t>(K / 256);
+  const cuuint64_t dims[4] = {256, 4, KS, static_cast<cuuint64_t>(N / 128)};
+  const cuuint64_t strides[3] = {2048, 8192, KS * 8192};
+  const cuuint32_t box[4] = {256, 1, static_cast<cuuint32_t>(box_stages), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------------------------
 // Policy
 // ------------------------------------------------------------------------------------
@@ -152,8 +169,8 @@ cudaError_t dispatch_tile(int T, const CUtensorMap& tx, const CUtensorMap& tw, c
 // programmatic stream serialization (the kernel waits for the previous kernel's
 // results itself, after its setup and weight prefetch).
 template <int FMT, int WSRC>
-cudaError_t launch_gemv(const CUtensorMap& tx, const CUtensorMap& tw, const GemvParams& p, dim3 grid,
-                        cudaStream_t stream) {
+cudaError_t launch_gemv(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ti, const GemvParams& p,
+                        dim3 grid, cudaStream_t stream) {
   using L = GemvLayout<FMT, WSRC>;
   auto kern = gemv_kernel<FMT, WSRC>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
@@ -177,17 +194,17 @@ cudaError_t launch_gemv(const CUtensorMap& tx, const CUtensorMap& tw, const Gemv
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  err = cudaLaunchKernelEx(&cfg, kern, tx, tw, p);
+  err = cudaLaunchKernelEx(&cfg, kern, tx, tw, ti, p);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
 template <int FMT>
-cudaError_t dispatch_gemv(int wsrc, const CUtensorMap& tx, const CUtensorMap& tw, const GemvParams& p, dim3 grid,
-                          cudaStream_t stream) {
-  if (wsrc == WSRC_VQ_DIRECT) return launch_gemv<FMT, WSRC_VQ_DIRECT>(tx, tw, p, grid, stream);
-  if (wsrc == WSRC_VQ_SVQ) return launch_gemv<FMT, WSRC_VQ_SVQ>(tx, tw, p, grid, stream);
-  return launch_gemv<FMT, WSRC_NATIVE>(tx, tw, p, grid, stream);
+cudaError_t dispatch_gemv(int wsrc, const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ti,
+                          const GemvParams& p, dim3 grid, cudaStream_t stream) {
+  if (wsrc == WSRC_VQ_DIRECT) return launch_gemv<FMT, WSRC_VQ_DIRECT>(tx, tw, ti, p, grid, stream);
+  if (wsrc == WSRC_VQ_SVQ) return launch_gemv<FMT, WSRC_VQ_SVQ>(tx, tw, ti, p, grid, stream);
+  return launch_gemv<FMT, WSRC_NATIVE>(tx, tw, ti, p, grid, stream);
 }
 
 inline ExpertPtrs expert_ptrs(const LinearArgs& a) {
@@ -234,8 +251,9 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
     p.splits = splits;
     p.ks_per_split = per;
     if (per <= kGemvMaxStages && splits <= kGemvMaxSplits) {
-      CUtensorMap tx3;
+      CUtensorMap tx3, ti = tw;
       if (!make_fp4_stage_map(&tx3, a.a_q, a.M, a.K, a.ldq, kGemvT, per)) return MXC_ERR_CUDA;
+      if (a.wsrc != WSRC_NATIVE && !make_idx_map(&ti, a.w_idx, a.N, a.K, per)) return MXC_ERR_CUDA;
       GemvParams g{};
       g.M = p.M;
       g.N = p.N;
@@ -252,8 +270,8 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
       g.ks_per_split = per;
       g.w = p.w[0];
       const dim3 grid(n_tiles, m_tiles, splits);
-      const cudaError_t err = a.fmt == FMT_E8M0 ? dispatch_gemv<FMT_E8M0>(a.wsrc, tx3, tw, g, grid, stream)
-                                                : dispatch_gemv<FMT_E4M3>(a.wsrc, tx3, tw, g, grid, stream);
+      const cudaError_t err = a.fmt == FMT_E8M0 ? dispatch_gemv<FMT_E8M0>(a.wsrc, tx3, tw, ti, g, grid, stream)
+                                                : dispatch_gemv<FMT_E4M3>(a.wsrc, tx3, tw, ti, g, grid, stream);
       return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
     }
   }

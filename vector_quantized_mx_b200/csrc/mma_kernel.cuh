@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (WSRC == WSRC_VQ_SVQ) tx += 8192 + (cb_split ? 1024 : 512) + 128 * L::kG;
     const uint8_t* sfx_src = a_sf + static_cast<size_t>(sf_group0) * KB4 * 512;
     const uint8_t* sfw_src = w_sf + static_cast<size_t>(n_tile) * KB4 * 512;
-    const uint8_t* idx_src = w_idx + static_cast<size_t>(n_tile) * 4 * KS * 2048;   // band: [4][KS][128][16]
+    const uint8_t* idx_src = w_idx + static_cast<size_t>(n_tile) * KS * 8192;
     const uint8_t* sidx_src = w_sidx + static_cast<size_t>(n_tile) * KS * (128 * L::kG);
     const uint16_t* cb_src = w_cb + static_cast<size_t>(qbn) * cb_per_row * 256;
     const int y0 = static_cast<int>(m0);
@@ -367,9 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(st + L::W_OFF, &tmap_wq, ks * 128, n_tile * 128, &full[s]);
           bulk_load(st + L::SFW_OFF, sfw_src + static_cast<size_t>(ks) * A * 512, A * 512, &full[s]);
         } else {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)                // the stage's four K-quarter slabs
-            bulk_load(st + L::IDX_OFF + c * 2048, idx_src + (static_cast<size_t>(c) * KS + ks) * 2048, 2048, &full[s]);
+          bulk_load(st + L::IDX_OFF, idx_src + static_cast<size_t>(ks) * 8192, 8192, &full[s]);
           const int qbk = cb_split ? 2 * ks : (ks * kStageK) / qk;
           bulk_load(st + L::CB_OFF, cb_src + static_cast<size_t>(qbk) * 256, cb_split ? 1024 : 512, &full[s]);
           if constexpr (WSRC == WSRC_VQ_DIRECT) {
@@ -602,9 +600,7 @@ __global__ void __launch_bounds__(160)
   if (threadIdx.x == 0) {
     const uint32_t tx = 8192 + (cb_split ? 1024 : 512) + (L::kSVQ ? 128 * L::kG : A * 512);
     mbar_arrive_expect_tx(bar, tx);
-    for (int c = 0; c < 4; ++c)
-      bulk_load(st + L::IDX_OFF + c * 2048, w.idx + ((static_cast<size_t>(n_tile) * 4 + c) * KS + ks) * 2048, 2048,
-                bar);
+    bulk_load(st + L::IDX_OFF, w.idx + tile_id * 8192, 8192, bar);
     const int qbn = static_cast<int>((static_cast<int64_t>(n_tile) * 128) / qn);
     const int qbk = cb_split ? 2 * ks : (ks * kStageK) / qk;
     bulk_load(st + L::CB_OFF, w.cb + (static_cast<size_t>(qbn) * (K / qk) + qbk) * 256, cb_split ? 1024 : 512,

@@ -161,7 +161,7 @@ mxc_status mxc_pack_weight(const mxc_weight_host* w, uint8_t* idx_out, uint8_t* 
       for (int64_t ks = 0; ks < KS; ++ks)
         for (int64_t c = 0; c < 4; ++c)         // K-quarter slabs of 16 index bytes per row
           for (int64_t r = 0; r < kTileN; ++r)
-            std::memcpy(idx_out + ((nt * 4 + c) * KS + ks) * 2048 + r * 16,
+            std::memcpy(idx_out + ((nt * KS + ks) * 4 + c) * 2048 + r * 16,
                         w->idx + (nt * kTileN + r) * (K / 4) + ks * 64 + c * 16, 16);
   }
   if (w->strategy == MXC_PRESCALE_PLUS) {
