@@ -296,7 +296,7 @@ mxc_status run_moe_linear(const MoeArgs& m, cudaStream_t stream) {
   int32_t* tile_prefix = reinterpret_cast<int32_t*>(a.ws);
   if (launch_group_prologue(m.offsets, m.E, a.M, tile_prefix, stream) != cudaSuccess) return MXC_ERR_CUDA;
   CUtensorMap tx;
-  if (!make_fp4_map(&tx, a.a_q, a.M, a.K, a.ldq, 128)) return MXC_ERR_CUDA;
+  if (!make_fp4_map(&tx, a.a_q, a.M, a.K, a.ldq, kMoeXBox)) return MXC_ERR_CUDA;   // 32-row boxes
   // GemmParams with the expert table (about 12 KB of kernel parameters).
   static thread_local GemmParams<kMaxGroups> p;
   std::memset(&p, 0, sizeof(p));

@@ -40,6 +40,7 @@ enum : int { WSRC_VQ_DIRECT = 0, WSRC_VQ_SVQ = 1, WSRC_NATIVE = 2 };
 enum : int { FMT_E8M0 = 0, FMT_E4M3 = 1 };
 
 constexpr int kMaxSplits = 4;      // cluster split-K factor of the decode path
+constexpr int kMoeXBox = 32;       // rows per token-tile copy of an expert tile
 
 struct ExpertPtrs {
   const uint8_t* idx;
@@ -114,6 +115,13 @@ constexpr int kColGroups = kDecWarps / 4;          // epilogue warps per TMEM la
 constexpr int kDecThreads = 32 * kDecWarps;
 constexpr int kThreads = 64 + kDecThreads;         // + loader warp + MMA warp
 
+// Decoder groups: with token tiles of up to 128 the tensor-core work per stage is
+// short, so two groups of 8 warps decode alternate stages at the same time (each
+// with its own codebook copies and named barrier); with 256 one group decodes
+// every stage with double-buffered copies.
+template <int T>
+__host__ __device__ constexpr int dec_groups() { return T <= 128 ? 2 : 1; }
+
 // ------------------------------------------------------------------------------------
 // Decoders (shared with the decode-dump kernel).  dt = decoder thread 0..NT-1.
 // ------------------------------------------------------------------------------------
@@ -144,38 +152,46 @@ __device__ __forceinline__ uint32_t lut16_pair(uint32_t lut_lane, uint32_t x, in
 }
 
 // One 128 x 256 weight tile: idx (four K-quarter slabs [128][16] bytes) -> FP4
-// [128][128] bytes in the 128-byte swizzle (16-byte chunk j of row r stored at chunk j ^ (r % 8)).
-// Thread dt owns chunks it*NT + dt; their shared-memory offsets are fixed per
-// thread and computed once (ChunkMap).  Chunks 0..3 of a row use codebook 0,
-// chunks 4..7 codebook 1 when the QBlock is 128 wide along K.
+// [128][128] bytes in the 128-byte swizzle (16-byte chunk j of row r stored at
+// chunk j ^ (r % 8)).  Item (r, q) = the 16 indices of row r in quarter q -> FP4
+// chunks 2q, 2q+1 of row r.  Thread dt owns items it*NT + dt, r = item % 128, so
+// the lanes of a warp read consecutive rows of one slab (16-byte loads, no bank
+// conflict) and store to 8 different bank groups per quarter warp.  Offsets are
+// fixed per thread and computed once (ItemMap).  Quarters 2, 3 use codebook 1 when
+// the QBlock is 128 wide along K.
 template <int NT>
-struct ChunkMap {
-  static constexpr int kN = 1024 / NT;
+struct ItemMap {
+  static constexpr int kN = 512 / NT;
   uint32_t idx_off[kN];   // byte offset into the index tile
-  uint32_t w_off[kN];     // byte offset into the swizzled FP4 tile
+  uint32_t w_off[kN];     // byte offset of row r in the FP4 tile
+  uint32_t sw[kN];        // (2q) ^ (r % 8): swizzled position of the first chunk
   uint32_t lut_off[kN];   // byte offset of this lane's codebook copy (codebook 0 or 1)
   __device__ __forceinline__ void init(int dt, int cb_split) {
 #pragma unroll
     for (int it = 0; it < kN; ++it) {
-      const int c = it * NT + dt;
-      const int r = c >> 3, j = c & 7;
-      idx_off[it] = (j >> 1) * 2048 + r * 16 + (j & 1) * 8;   // K-quarter slab j/2
-      w_off[it] = r * 128 + ((j ^ (r & 7)) << 4);
-      lut_off[it] = ((cb_split && j >= 4) ? kLutBytes : 0) + (dt & 31) * 4;
+      const int item = it * NT + dt;
+      const int r = item & 127, q = item >> 7;
+      idx_off[it] = q * 2048 + r * 16;
+      w_off[it] = r * 128;
+      sw[it] = static_cast<uint32_t>((2 * q) ^ (r & 7));
+      lut_off[it] = ((cb_split && q >= 2) ? kLutBytes : 0) + (dt & 31) * 4;
     }
   }
 };
 
 template <int NT>
 __device__ __forceinline__ void decode_w_tile(const uint8_t* __restrict__ idx, uint32_t lut_s,
-                                              uint8_t* __restrict__ wt, const ChunkMap<NT>& cm) {
+                                              uint8_t* __restrict__ wt, const ItemMap<NT>& im) {
 #pragma unroll
-  for (int it = 0; it < ChunkMap<NT>::kN; ++it) {
-    const uint2 iv = *reinterpret_cast<const uint2*>(idx + cm.idx_off[it]);
-    const uint32_t base = lut_s + cm.lut_off[it];
-    *reinterpret_cast<uint4*>(wt + cm.w_off[it]) =
-        make_uint4(lut16_pair(base, iv.x, 0), lut16_pair(base, iv.x, 2), lut16_pair(base, iv.y, 0),
-                   lut16_pair(base, iv.y, 2));
+  for (int it = 0; it < ItemMap<NT>::kN; ++it) {
+    const uint4 iv = *reinterpret_cast<const uint4*>(idx + im.idx_off[it]);
+    const uint32_t base = lut_s + im.lut_off[it];
+    const uint4 o0 = make_uint4(lut16_pair(base, iv.x, 0), lut16_pair(base, iv.x, 2), lut16_pair(base, iv.y, 0),
+                                lut16_pair(base, iv.y, 2));
+    const uint4 o1 = make_uint4(lut16_pair(base, iv.z, 0), lut16_pair(base, iv.z, 2), lut16_pair(base, iv.w, 0),
+                                lut16_pair(base, iv.w, 2));
+    *reinterpret_cast<uint4*>(wt + im.w_off[it] + (im.sw[it] << 4)) = o0;
+    *reinterpret_cast<uint4*>(wt + im.w_off[it] + ((im.sw[it] ^ 1u) << 4)) = o1;
   }
 }
 
@@ -186,9 +202,9 @@ template <int G, int NT>
 __device__ __forceinline__ void decode_sf_tile(const uint8_t* __restrict__ sidx,
                                                const uint8_t* __restrict__ scb, uint8_t* __restrict__ sfw,
                                                int dt) {
-  for (int u = dt; u < 128 * G; u += NT) {
-    const int r = u & 127, g = u >> 7;
-    const int word = (r & 31) * 4 + ((r >> 5) & 3);
+  for (int u = dt; u < 128 * G; u += NT) {   // consecutive threads: consecutive atom words
+    const int word = u & 127, g = u >> 7;
+    const int r = (word >> 2) + 32 * (word & 3);
     const uint32_t si = sidx[r * G + g];
     const uint2 s8 = *reinterpret_cast<const uint2*>(scb + si * 8);
     reinterpret_cast<uint32_t*>(sfw + (2 * g) * 512)[word] = s8.x;
@@ -294,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&dec[s], kDecWarps);
+      mbar_init(&dec[s], kDecWarps / dec_groups<T>());
       mbar_init(&empty[s], 1);
     }
     mbar_init(accum, 1);
@@ -338,7 +354,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int groups = static_cast<int>((static_cast<int64_t>(p.M) + 127) / 128);
       xg_valid = groups - sf_group0 < XG ? groups - sf_group0 : XG;
     }
-    uint32_t tx = T * 128 + xg_valid * A * 512;
+    // Expert tiles load only the 32-row boxes that hold the expert's rows (most
+    // experts own far fewer than 128): the rows of the neighbouring experts would
+    // be wasted ingest.  Columns past the expert's rows are computed on stale
+    // (finite: E2M1 has no NaN) shared memory and never stored.
+    int x_boxes = 1, x_box_bytes = T * 128;
+    if constexpr (MOE) {
+      const int64_t rows = m_end - m0 < T ? m_end - m0 : T;
+      x_boxes = static_cast<int>((rows + kMoeXBox - 1) / kMoeXBox);
+      x_box_bytes = kMoeXBox * 128;
+    }
+    uint32_t tx = x_boxes * x_box_bytes + xg_valid * A * 512;
     if constexpr (WSRC == WSRC_NATIVE) tx += 16384 + A * 512;
     if constexpr (WSRC == WSRC_VQ_DIRECT) tx += 8192 + (cb_split ? 1024 : 512) + A * 512;
     if constexpr (WSRC == WSRC_VQ_SVQ) tx += 8192 + (cb_split ? 1024 : 512) + 128 * L::kG;
@@ -357,7 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ks = ks_begin + i;
         uint8_t* st = stages + s * L::BYTES;
         mbar_arrive_expect_tx(&full[s], tx);
-        tma_load_2d(st + L::X_OFF, &tmap_x, ks * 128, y0, &full[s]);
+        for (int q = 0; q < x_boxes; ++q)
+          tma_load_2d(st + L::X_OFF + q * x_box_bytes, &tmap_x, ks * 128, y0 + q * kMoeXBox, &full[s]);
 #pragma unroll
         for (int g = 0; g < XG; ++g)
           if (g < xg_valid)                          // a missing group's rows are past M: never stored
@@ -447,38 +474,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ======================= decoders, then epilogue ======================
     const int dt = threadIdx.x - 64;
     if constexpr (L::kVQ) {
-      // Codebook copies double-buffered: stage i decodes through buffer i%2 while the
-      // copies of stage i+1 go into the other buffer; one decoder barrier per stage
-      // (it also orders stage i's lookups before buffer i%2 is rebuilt).
+      // Group g decodes stages g, g + G, ...  One group: codebook copies double-
+      // buffered -- stage i decodes through buffer i%2 while the copies of stage
+      // i+1 go into the other; one barrier per stage (it also orders stage i's
+      // lookups before buffer i%2 is rebuilt).  Two groups: one buffer each, a
+      // barrier before and after each rebuild.
+      constexpr int G = dec_groups<T>();
+      constexpr int GT = kDecThreads / G;            // threads per group
       constexpr int cb_split = NCB == 2;
       constexpr int kBuf = NCB * kLutBytes;
-      uint8_t* lut = smem + L::LUT_OFF;
+      constexpr int kBufs = 2 / G;                   // copy buffers per group
+      const int grp = dt / GT, gt = dt - grp * GT;
+      const int bar_id = 2 + grp;
+      uint8_t* lut = smem + L::LUT_OFF + grp * kBufs * kBuf;
       const uint32_t lut_s = smem_u32(lut);
-      ChunkMap<kDecThreads> cm;
-      cm.init(dt, cb_split);
+      ItemMap<GT> cm;
+      cm.init(gt, cb_split);
+      auto stage_cb = [&](int i) {
+        return reinterpret_cast<const uint16_t*>(stages + (i % STAGES) * L::BYTES + L::CB_OFF);
+      };
       bool ok = true;
-      if (nks > 0) {
-        const bool got = mbar_wait(&full[0], 0);
-        if (got)
-          build_lut<kDecThreads>(reinterpret_cast<const uint16_t*>(stages + L::CB_OFF), 1 + cb_split,
-                                 reinterpret_cast<uint32_t*>(lut), dt);
-        ok = named_bar_and(2, kDecThreads, got);     // one decision for all decoders
+      int b = 0;
+      if (grp < nks) {
+        const bool got = mbar_wait(&full[grp % STAGES], (grp / STAGES) & 1);
+        if (got) build_lut<GT>(stage_cb(grp), 1 + cb_split, reinterpret_cast<uint32_t*>(lut), gt);
+        ok = named_bar_and(bar_id, GT, got);         // one decision for the group
       }
-      for (int i = 0; i < nks && ok; ++i) {
+      for (int i = grp; i < nks && ok; i += G) {
         const int s = i % STAGES;
         uint8_t* st = stages + s * L::BYTES;
-        decode_w_tile<kDecThreads>(st + L::IDX_OFF, lut_s + (i & 1) * kBuf, st + L::W_OFF, cm);
-        if constexpr (L::kSVQ) decode_sf_tile<L::kG, kDecThreads>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, dt);
+        decode_w_tile<GT>(st + L::IDX_OFF, lut_s + b * kBuf, st + L::W_OFF, cm);
+        if constexpr (L::kSVQ) decode_sf_tile<L::kG, GT>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, gt);
         fence_proxy_async_smem();                    // each thread's tile writes -> async proxy
         __syncwarp();
-        if (lane == 0) mbar_arrive(&dec[s]);         // one arrival per decoder warp
-        if (i + 1 < nks) {                           // the next stage's copies, other buffer
-          const int s1 = (i + 1) % STAGES;
-          const bool got = mbar_wait(&full[s1], ((i + 1) / STAGES) & 1);
-          if (got)
-            build_lut<kDecThreads>(reinterpret_cast<const uint16_t*>(stages + s1 * L::BYTES + L::CB_OFF),
-                                   1 + cb_split, reinterpret_cast<uint32_t*>(lut + ((i + 1) & 1) * kBuf), dt);
-          ok = named_bar_and(2, kDecThreads, got);
+        if (lane == 0) mbar_arrive(&dec[s]);         // one arrival per decoder warp of the group
+        const int in = i + G;
+        if (in < nks) {                              // this group's next stage
+          if (kBufs == 1) named_bar_sync(bar_id, GT);   // lookups of stage i done before the rebuild
+          const int nb = kBufs == 2 ? (b ^ 1) : 0;
+          const bool got = mbar_wait(&full[in % STAGES], (in / STAGES) & 1);
+          if (got) build_lut<GT>(stage_cb(in), 1 + cb_split, reinterpret_cast<uint32_t*>(lut + nb * kBuf), gt);
+          ok = named_bar_and(bar_id, GT, got);
+          b = nb;
         }
       }
     }
@@ -616,7 +653,7 @@ __global__ void __launch_bounds__(160)
   if (threadIdx.x >= 32 && ok) build_lut<128>(reinterpret_cast<const uint16_t*>(st + L::CB_OFF), 1 + cb_split, lut, dt);
   __syncthreads();
   if (threadIdx.x >= 32 && ok) {
-    ChunkMap<128> cm;
+    ItemMap<128> cm;
     cm.init(dt, cb_split);
     decode_w_tile<128>(st + L::IDX_OFF, smem_u32(lut), st + L::W_OFF, cm);
     if constexpr (L::kSVQ) decode_sf_tile<L::kG, 128>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, dt);
