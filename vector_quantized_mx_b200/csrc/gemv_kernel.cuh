@@ -23,8 +23,12 @@
 //     the buffers of quarters 0 and 1 once those are decoded), which leaves room
 //     to bring the weight and token scale atoms in by bulk copies; the MMA warp
 //     moves both to TMEM with tcgen05.cp;
-//   * split-K partial tiles go to the cluster's rank 0 by st.async with completion
-//     on an mbarrier there; rank 0 adds them in rank order (deterministic).
+//   * split-K, two ranks, FP32 output: rank 0 zeroes its output tile after the
+//     dependency wait and both ranks add their scaled partials with red.global.add
+//     (two addends onto zero: the result does not depend on their order); more
+//     ranks or BF16 output: the partial tiles go to rank 0 as one 8 KB bulk copy
+//     between shared memories (completion on an mbarrier there, an acknowledgement
+//     back before the sender may exit) and rank 0 adds them in rank order.
 //
 // Programmatic dependent launch: the CTA sets up and prefetches its weight stream
 // into L2 before griddepcontrol.wait, overlapping the previous kernel (typically
@@ -116,7 +120,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_cb = bars + 18;     // codebooks of the slice (bulk copy)
   uint64_t* bar_sfx = bars + 20;    // token scale atoms (bulk copy)
   uint64_t* sfx_free = bars + 21;   // their tcgen05.cp copies are done: the buffer is free
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
+  uint64_t* red_ack = bars + 22;    // rank > 0: rank 0 has received this rank's partial tile
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = p.K, KS = K / kStageK, KB4 = K / L::kB / 4;
@@ -139,6 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint8_t* const a_sf =
       p.a_sf + (static_cast<size_t>(sf_group0) * KB4 + static_cast<size_t>(ks_begin) * A) * 512;
   const int red_off = splits == 2 ? L::SFX_OFF : L::IDX_OFF;   // rank 0's receive area
+  const bool red_atomic = splits == 2 && !p.out_bf16;           // split-K by global reductions
   // codebooks used by the slice: a contiguous range [qb0, qb1] of the band's row
   const int qb0 = !L::kVQ ? 0 : H == 2 ? 2 * ks_begin : (ks_begin * kStageK) / p.qk;
   const int qb1 = !L::kVQ ? 0 : H == 2 ? 2 * ks_end - 1 : ((ks_end - 1) * kStageK) / p.qk;
@@ -146,8 +152,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- setup (nothing here depends on earlier kernels) ----
   if (warp == 0) {
     // full[0..7], bar_x, dec_ph[0..3], sf_ready, accum, red_full, red_ready, bar_sfw, bar_cb,
-    // (unused), bar_sfx, sfx_free
-    if (lane < 22) mbar_init(bars + lane, (lane >= 9 && lane < 14) ? kDecWarps : 1);
+    // (unused), bar_sfx, sfx_free, red_ack
+    if (lane < 23) mbar_init(bars + lane, (lane >= 9 && lane < 14) ? kDecWarps : 1);
     __syncwarp();
   }
   if (warp == 0 && lane == 0) {
@@ -185,6 +191,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   griddep_launch_dependents();
   griddep_wait();                                    // earlier kernels' results are visible
   if (splits > 1) cluster_wait_acquire();            // every CTA of the cluster is set up
+  // Two ranks, FP32 output: rank 0's decoder warps zero this tile of Y (rows < M) now
+  // and publish the stores with a release arrive on the second cluster-barrier phase
+  // once the codebook copies are laid out (the stores are complete by then, so the
+  // release does not stall); both ranks then only add to the tile.  All other warps
+  // arrive relaxed (a release would wait for their prefetches).  Every cluster-barrier
+  // arrive and wait is made by whole, converged warps.
+  if (red_atomic && warp < 2) {
+    __syncwarp();
+    cluster_arrive_relaxed();
+  }
+  if (red_atomic && rank == 0 && warp >= 2) {
+    const int dt = threadIdx.x - 64;
+    const int64_t m = m0 + (dt >> 5);
+    if (m < p.M) {
+      float* yrow = reinterpret_cast<float*>(p.y) + m * p.ldy + static_cast<int64_t>(n_tile) * 128 + (dt & 31) * 4;
+      yrow[0] = 0.0f;
+      yrow[1] = 0.0f;
+      yrow[2] = 0.0f;
+      yrow[3] = 0.0f;
+    }
+  }
+  auto publish_zeroing = [&]() {                     // decoder warps, converged
+    if (red_atomic) {
+      __syncwarp();
+      if (rank == 0) cluster_arrive_release(); else cluster_arrive_relaxed();
+    }
+  };
   // output scale: read now, used at the very end
   float out_scale = p.w.w_tscale;
   if (warp >= 2) {
@@ -239,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-    if (splits > 1 && rank == 0) {
+    if (splits > 1 && rank == 0 && !red_atomic) {
       // Let the other ranks send their partials once the receive area is free:
       // the token-scale buffer after its tcgen05.cp copies (2 ranks), the index
       // buffers after the last decode phase (more ranks).  Sent even after a
@@ -322,14 +355,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int s_l = lane & 7;                        // this lane's stage
     const int q = dw * 4 + (lane >> 3);              // 64 threads per stage
     const bool active = L::kVQ && s_l < nks;
-    // words [8 dw, 8 dw + 8) of the codebook of this lane's stage, for the first or
-    // (QBlock 128 wide along K) the second half of the stage
+    // Words [8 kb, 8 kb + 8) of the codebook of this lane's stage (first or, QBlock
+    // 128 wide along K, second half of the stage), kb = (dw + s_l/2) mod 16: over the
+    // 16 warps each lane still covers all 128 words, and the 8 lanes of a quarter
+    // warp (8 stages, codebooks 512 B apart) read 8 different bank groups -- the
+    // two 16-byte halves are read in an order that alternates with the stage.
+    const int kb = (dw + (s_l >> 1)) & 15;
+    const int h0 = s_l & 1;
     auto cb_words = [&](int epoch, uint4* c0, uint4* c1) {
       const int ks = ks_begin + s_l;
       const int qbk = H == 2 ? 2 * ks + epoch : (ks * kStageK) / p.qk;
-      const uint4* cp = reinterpret_cast<const uint4*>(smem + L::CB_OFF + (qbk - qb0) * 512 + 32 * dw);
-      *c0 = cp[0];
-      *c1 = cp[1];
+      const uint8_t* cp = smem + L::CB_OFF + (qbk - qb0) * 512 + 32 * kb;
+      const uint4 first = *reinterpret_cast<const uint4*>(cp + 16 * h0);
+      const uint4 second = *reinterpret_cast<const uint4*>(cp + 16 * (1 - h0));
+      *c0 = h0 ? second : first;                      // words 8 kb .. 8 kb + 3
+      *c1 = h0 ? first : second;                      // words 8 kb + 4 .. 8 kb + 7
     };
 
     // --- PreScale+ weight scale atoms -> TMEM lanes of this warp's quadrant
@@ -359,6 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
 
+    if constexpr (!L::kVQ) publish_zeroing();
     if constexpr (L::kVQ) {
       // both codebooks into registers now: the staging area is overwritten by the
       // decoded tiles of the last stage
@@ -369,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (H == 2) cb_words(1, &d0, &d1);
       }
       // --- codebook copies: lane l's copy (bank l) = codebook of stage l mod 8 ---
-      uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L::LUT_OFF) + (8 * dw) * 32 + lane;
+      uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L::LUT_OFF) + (8 * kb) * 32 + lane;
       auto lay_out = [&](const uint4& a, const uint4& b) {
         if (!active) return;
         lut[0 * 32] = a.x;
@@ -383,6 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       lay_out(c0, c1);
       named_bar_sync(2, kDecThreads);                // all copies written
+      publish_zeroing();
       const uint32_t lut_lane = smem_u32(smem + L::LUT_OFF) + lane * 4;
       const uint8_t* idx_l = smem + L::IDX_OFF + s_l * 2048;
       uint8_t* wt = smem + L::W_OFF + s_l * 16384;
@@ -421,17 +463,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_ld_32x32b_x4(tmem + (static_cast<uint32_t>(qd * 32) << 16) + cg * 4, acc);
     tmem_ld_wait();
     float v[4] = {__uint_as_float(acc[0]), __uint_as_float(acc[1]), __uint_as_float(acc[2]), __uint_as_float(acc[3])};
-    const uint32_t red_slot = smem_u32(smem + red_off) + (row * kGemvT + cg * 4) * 4;
     bool store = ep_ok;
-    if (splits > 1) {
+    if (red_atomic) {
+      store = false;
+      __syncwarp();
+      cluster_wait_acquire();                        // rank 0's zeroing is visible
+      if (ep_ok) {
+        float* const y = reinterpret_cast<float*>(p.y);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (mbase + c < p.M) atomicAdd(y + (mbase + c) * p.ldy + n, v[c] * scale);
+      }
+    } else if (splits > 1) {
       if (rank != 0) {
+        // the partial tile [128][16] FP32 into this CTA's receive-area offset, then one
+        // bulk copy to rank 0's slot rank-1 (sent even when ep_ok is false: rank 0 waits)
         store = false;
-        if (mbar_wait(red_ready, 0)) {              // sent even when ep_ok is false: rank 0 waits for it
-          st_async_v4_f32(mapa_shared(red_slot + (rank - 1) * 128 * kGemvT * 4, 0), v[0], v[1], v[2], v[3],
-                          mapa_shared(smem_u32(red_full), 0));
+        *reinterpret_cast<float4*>(smem + red_off + (row * kGemvT + cg * 4) * 4) = make_float4(v[0], v[1], v[2], v[3]);
+        fence_proxy_async_smem();                    // generic writes -> the bulk copy's reads
+        named_bar_sync(2, kDecThreads);
+        if (threadIdx.x == 64) {
+          if (mbar_wait(red_ready, 0)) {
+            constexpr uint32_t kTile = 128 * kGemvT * 4;
+            bulk_copy_to_cluster(mapa_shared(smem_u32(smem + red_off) + (rank - 1) * kTile, 0),
+                                 smem_u32(smem + red_off), kTile, mapa_shared(smem_u32(red_full), 0));
+          }
+          // rank 0 has it (or gave up waiting): the source may go.  Rank 0 always sends
+          // this acknowledgement, so no rank exits while rank 0 still signals it.
+          mbar_wait(red_ack, 0);
         }
       } else {
         const bool got = mbar_wait(red_full, 0);    // all partials landed: none in flight at exit
+        if (threadIdx.x == 64) {                     // let the senders go
+          for (uint32_t r = 1; r < static_cast<uint32_t>(splits); ++r)
+            mbar_remote_arrive(mapa_shared(smem_u32(red_ack), r));
+        }
         store = store && got;
         if (store) {
           for (int r = 1; r < splits; ++r) {
@@ -453,6 +519,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 4; ++c)
         if (mbase + c < p.M) store_out(y, ldy, out_bf16, mbase + c, n, v[c] * scale);
     }
+  }
+  if (red_atomic && warp < 2) {                      // every thread completes the barrier phase
+    __syncwarp();
+    cluster_wait_acquire();
   }
   __syncwarp();
   tc_fence_before();

@@ -74,10 +74,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity to complete.  Returns false
 // (and records MXC_ERR_TIMEOUT) if it does not complete within kWaitLimitCycles.
+// Between polls the thread backs off briefly, so that many waiting threads do not
+// keep the shared-memory pipe busy with barrier polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
+    __nanosleep(32);
     if (mbar_try_wait(bar, parity)) return true;
     if (clock64() - t0 > kWaitLimitCycles) {
       set_device_error(MXC_ERR_TIMEOUT);
@@ -233,6 +236,9 @@ __device__ __forceinline__ void cluster_sync_all() {
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
 }
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_wait_acquire() {
   asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
 }
@@ -243,6 +249,15 @@ __device__ __forceinline__ void st_async_v4_f32(uint32_t remote_addr, float a, f
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
                    remote_addr),
                "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
+               : "memory");
+}
+// Bulk copy from this CTA's shared memory into another CTA's (both addresses in the
+// shared::cluster window, 16-byte aligned, bytes a multiple of 16); completion
+// counts the bytes on the destination CTA's mbarrier.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t dst_bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst),
+               "r"(src), "r"(bytes), "r"(dst_bar)
                : "memory");
 }
 // Arrive on an mbarrier of another CTA of the cluster (release at cluster scope).
