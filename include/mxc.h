@@ -23,6 +23,15 @@
  * - Asynchrony: GPU calls enqueue work on the given stream and return.  They
  *   do not synchronize.  Argument, shape and alignment problems are reported
  *   synchronously by the return value and nothing is enqueued.
+ * - Programmatic dependent launch: mxc_quantize_act (M*K <= 16*8192) and the
+ *   M <= 16 path of mxc_linear / mxc_native_linear let the next kernel of the
+ *   stream start early, and the decode path loads and decodes its weight
+ *   buffers before waiting for the previous kernel.  Weight buffers are
+ *   therefore constants of the stream: they must not be written by a kernel
+ *   that itself launches with programmatic dependent launch right before the
+ *   call (host copies, ordinary kernels, this library's packing and decode
+ *   calls are fine).  Activation, scale and output buffers follow plain stream
+ *   order.
  * - Device-side problems (malformed MoE offsets, a pipeline wait that ran
  *   out) set the device error word; read it with mxc_get_device_error().
  * - No exception crosses this ABI; every entry point returns mxc_status.

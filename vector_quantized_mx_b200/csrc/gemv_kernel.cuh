@@ -30,9 +30,14 @@
 //     between shared memories (completion on an mbarrier there, an acknowledgement
 //     back before the sender may exit) and rank 0 adds them in rank order.
 //
-// Programmatic dependent launch: the CTA sets up and prefetches its weight stream
-// into L2 before griddepcontrol.wait, overlapping the previous kernel (typically
-// the activation quantizer); nothing that kernel writes is read before the wait.
+// Programmatic dependent launch: only the token tiles, the token scales and the
+// activation tensor scale come from the previous kernel (typically the activation
+// quantizer), and the output tile is written.  Everything else -- loading and
+// decoding the whole weight slice, the weight scales into TMEM -- runs before
+// griddepcontrol.wait and overlaps that kernel; the MMA warp waits, then fetches
+// the token operands, and the decoder warps wait before they touch the output.
+// The weight buffers are therefore read while the previous kernel may still run:
+// they must not be written by a kernel of the same programmatic-launch chain.
 #pragma once
 
 #include "mma_kernel.cuh"
@@ -187,44 +192,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (splits > 1) cluster_arrive_relaxed();          // barriers above are initialised (fenced)
+  if (splits > 1) {
+    __syncwarp();
+    cluster_arrive_relaxed();                        // barriers above are initialised (fenced)
+  }
   griddep_launch_dependents();
-  griddep_wait();                                    // earlier kernels' results are visible
-  if (splits > 1) cluster_wait_acquire();            // every CTA of the cluster is set up
-  // Two ranks, FP32 output: rank 0's decoder warps zero this tile of Y (rows < M) now
-  // and publish the stores with a release arrive on the second cluster-barrier phase
-  // once the codebook copies are laid out (the stores are complete by then, so the
-  // release does not stall); both ranks then only add to the tile.  All other warps
-  // arrive relaxed (a release would wait for their prefetches).  Every cluster-barrier
-  // arrive and wait is made by whole, converged warps.
+  if (splits > 1) {
+    __syncwarp();
+    cluster_wait_acquire();                          // every CTA of the cluster is set up
+  }
+  // Two ranks, FP32 output: after the dependency wait (and their decode phases) rank
+  // 0's decoder warps zero this tile of Y (rows < M) and publish the stores with a
+  // release arrive on the second cluster-barrier phase; both ranks then only add to
+  // the tile.  All other warps arrive relaxed (a release would wait for their
+  // prefetches).  Every cluster-barrier arrive and wait is made by whole, converged
+  // warps.
   if (red_atomic && warp < 2) {
     __syncwarp();
     cluster_arrive_relaxed();
-  }
-  if (red_atomic && rank == 0 && warp >= 2) {
-    const int dt = threadIdx.x - 64;
-    const int64_t m = m0 + (dt >> 5);
-    if (m < p.M) {
-      float* yrow = reinterpret_cast<float*>(p.y) + m * p.ldy + static_cast<int64_t>(n_tile) * 128 + (dt & 31) * 4;
-      yrow[0] = 0.0f;
-      yrow[1] = 0.0f;
-      yrow[2] = 0.0f;
-      yrow[3] = 0.0f;
-    }
-  }
-  auto publish_zeroing = [&]() {                     // decoder warps, converged
-    if (red_atomic) {
-      __syncwarp();
-      if (rank == 0) cluster_arrive_release(); else cluster_arrive_relaxed();
-    }
-  };
-  // output scale: read now, used at the very end
-  float out_scale = p.w.w_tscale;
-  if (warp >= 2) {
-    if constexpr (WSRC == WSRC_NATIVE) {
-      if (p.w_tscale_dev) out_scale = __ldg(p.w_tscale_dev);
-    }
-    if (p.a_tscale) out_scale *= __ldg(p.a_tscale);
   }
 
   // epilogue coordinates (decoder warps)
@@ -238,7 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // =============================== loader ===============================
     __syncwarp();
     if (elect_one()) {
-      // in the order they are needed: codebooks, index quarter 0, scales, tokens, quarters 1..3
+      // weights only, in the order they are needed: codebooks, index quarter 0, weight
+      // scales, quarters 1..3 (the MMA warp fetches the token operands after the wait)
       if constexpr (L::kVQ) {
         const uint32_t cb_bytes = static_cast<uint32_t>(qb1 - qb0 + 1) * 512;
         mbar_arrive_expect_tx(bar_cb, cb_bytes);
@@ -248,16 +234,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&full[0], p.ks_per_split * 2048);
         tma_load_4d(smem + L::IDX_OFF, &tmap_idx, 0, 0, ks_begin, n_tile, &full[0]);
       }
-      mbar_arrive_expect_tx(bar_sfx, nks * A * 512);
-      bulk_load(smem + L::SFX_OFF, a_sf, nks * A * 512, bar_sfx);
       if constexpr (!L::kSVQ) {
         mbar_arrive_expect_tx(bar_sfw, nks * A * 512);
         bulk_load(smem + L::SFW_OFF, w_sf, nks * A * 512, bar_sfw);
       }
-      // token tiles of all stages: box {128 B, 16 rows, ks_per_split stages}; stages
-      // past K (last split) arrive zero-filled and are not used
-      mbar_arrive_expect_tx(bar_x, p.ks_per_split * kGemvT * 128);
-      tma_load_3d(smem + L::X_OFF, &tmap_x, 0, static_cast<int>(m0), ks_begin, bar_x);
       if constexpr (L::kVQ) {
         for (int j = 1; j < 4; ++j) {                // K-quarter j of every stage
           if (j >= 2 && !mbar_wait(&dec_ph[j - 2], 0)) break;   // its buffer has been decoded
@@ -298,8 +278,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     }
+    griddep_wait();                                  // the token operands are written
+    __syncwarp();
+    if (elect_one()) {
+      mbar_arrive_expect_tx(bar_sfx, nks * A * 512);
+      bulk_load(smem + L::SFX_OFF, a_sf, nks * A * 512, bar_sfx);
+      // token tiles of all stages: box {128 B, 16 rows, ks_per_split stages}; stages
+      // past K (last split) arrive zero-filled and are not used
+      mbar_arrive_expect_tx(bar_x, p.ks_per_split * kGemvT * 128);
+      tma_load_3d(smem + L::X_OFF, &tmap_x, 0, static_cast<int>(m0), ks_begin, bar_x);
+    }
+    __syncwarp();
     {
-      // token scale atoms -> TMEM, then free their buffer for index quarter 2
+      // token scale atoms -> TMEM (their buffer then receives rank 1's partial tile)
       const bool got = __all_sync(0xffffffffu, mbar_wait(bar_sfx, 0));
       if (got && elect_one()) {
         const uint32_t sfx_s0 = smem_u32(smem + L::SFX_OFF);
@@ -399,7 +390,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
 
-    if constexpr (!L::kVQ) publish_zeroing();
     if constexpr (L::kVQ) {
       // both codebooks into registers now: the staging area is overwritten by the
       // decoded tiles of the last stage
@@ -424,7 +414,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       lay_out(c0, c1);
       named_bar_sync(2, kDecThreads);                // all copies written
-      publish_zeroing();
       const uint32_t lut_lane = smem_u32(smem + L::LUT_OFF) + lane * 4;
       const uint8_t* idx_l = smem + L::IDX_OFF + s_l * 2048;
       uint8_t* wt = smem + L::W_OFF + s_l * 16384;
@@ -455,6 +444,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     // ------------------------------ epilogue ------------------------------
+    __syncwarp();
+    griddep_wait();                                  // the output and the token scale may be touched
+    if (red_atomic) {
+      if (rank == 0) {
+        const int dt = threadIdx.x - 64;
+        const int64_t m = m0 + (dt >> 5);
+        if (m < p.M) {
+          float* yrow = reinterpret_cast<float*>(p.y) + m * p.ldy + static_cast<int64_t>(n_tile) * 128 + (dt & 31) * 4;
+          yrow[0] = 0.0f;
+          yrow[1] = 0.0f;
+          yrow[2] = 0.0f;
+          yrow[3] = 0.0f;
+        }
+      }
+      __syncwarp();
+      if (rank == 0) cluster_arrive_release(); else cluster_arrive_relaxed();
+    }
+    float out_scale = p.w.w_tscale;
+    if constexpr (WSRC == WSRC_NATIVE) {
+      if (p.w_tscale_dev) out_scale = __ldg(p.w_tscale_dev);
+    }
+    if (p.a_tscale) out_scale *= __ldg(p.a_tscale);
     const bool ep_ok = mbar_wait(accum, 0);
     tc_fence_after();
     const float scale = out_scale;
