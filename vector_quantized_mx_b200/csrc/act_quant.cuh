@@ -51,17 +51,18 @@ __device__ __forceinline__ float exp2_int(int e) {
 
 // E2M1 code of x / d, round half to even, saturating at 6, sign of x kept.
 // Each midpoint test uses the sign of fma(mu, d, -|x|), which is the sign of
-// the exact value mu*d - |x| (one rounding never flips a sign).
+// the exact value mu*d - |x| (one rounding never flips a sign).  The code is
+// the number of midpoints |x|/d lies above, found by a three-level binary
+// search: 1.75 first (tie -> 2.0, code 4), then 3.5 or 0.75 (ties -> 4.0 /
+// 1.0, the even codes above), then 5, 2.5, 1.25 or 0.25 (ties -> 4.0, 2.0, 1.0,
+// 0: the even codes below).
 __device__ __forceinline__ uint32_t e2m1_code(float x, float d) {
   const float a = fabsf(x);
-  uint32_t c = 0;
-  c += __fmaf_rn(0.25f, d, -a) < 0.0f;   // a >  0.25 d   (tie -> 0)
-  c += __fmaf_rn(0.75f, d, -a) <= 0.0f;  // a >= 0.75 d   (tie -> 1.0)
-  c += __fmaf_rn(1.25f, d, -a) < 0.0f;   // a >  1.25 d   (tie -> 1.0)
-  c += __fmaf_rn(1.75f, d, -a) <= 0.0f;  // a >= 1.75 d   (tie -> 2.0)
-  c += __fmaf_rn(2.50f, d, -a) < 0.0f;   // a >  2.5 d    (tie -> 2.0)
-  c += __fmaf_rn(3.50f, d, -a) <= 0.0f;  // a >= 3.5 d    (tie -> 4.0)
-  c += __fmaf_rn(5.00f, d, -a) < 0.0f;   // a >  5 d      (tie -> 4.0)
+  const bool hi = __fmaf_rn(1.75f, d, -a) <= 0.0f;                // a >= 1.75 d
+  const bool mid = __fmaf_rn(hi ? 3.5f : 0.75f, d, -a) <= 0.0f;   // a >= 3.5 d / 0.75 d
+  const float mu = hi ? (mid ? 5.0f : 2.5f) : (mid ? 1.25f : 0.25f);
+  const bool lo = __fmaf_rn(mu, d, -a) < 0.0f;                     // a > mu d
+  const uint32_t c = (hi ? 4u : 0u) + (mid ? 2u : 0u) + (lo ? 1u : 0u);
   return c | ((__float_as_uint(x) >> 28) & 8u);
 }
 

@@ -13,18 +13,25 @@
 //     tiles with one 3-D tensor copy;
 //   * decoder lane l decodes stage l mod 8, so the 32 per-lane codebook copies in
 //     shared memory hold, in bank l, the codebook of lane l's stage: the codebooks
-//     of the whole slice are laid out once (16-bit entries, 16 KB) and no lookup
-//     meets a bank conflict;
+//     of the whole slice are laid out once (one entry per 32-bit word, 32 KB) and
+//     no lookup meets a bank conflict; two lookups merge with one fixed byte
+//     permute;
 //   * the decoders finish K-quarter j of every stage before quarter j+1; the MMA
 //     warp issues the block-scaled MMAs of quarter j of all stages while quarter
 //     j+1 is decoded.  Native FP4 weights use the same quarter-major MMA order, so
 //     both give bit-identical results on the same operands;
 //   * the index slabs pass through two quarter buffers (quarters 2 and 3 reuse
-//     the buffers of quarters 0 and 1 once those are decoded), which leaves room
-//     to bring the weight and token scale atoms in by bulk copies; the MMA warp
-//     moves both to TMEM with tcgen05.cp;
+//     the buffers of quarters 0 and 1 once those are decoded); the weight scale
+//     atoms come in by one bulk copy and the MMA warp moves them to TMEM with
+//     tcgen05.cp;
+//   * token scales: with at most 16 tokens only the first 16 of the 128 rows of
+//     an activation scale atom carry scales (the rest is zero padding), so four
+//     extra warps, one per TMEM lane quadrant, load those 16 words per atom and
+//     write the atoms' TMEM image with tcgen05.st -- the image tcgen05.cp would
+//     make of the whole atom -- instead of 144 CTAs copying 16 KB each;
 //   * split-K, two ranks, FP32 output: rank 0 zeroes its output tile after the
-//     dependency wait and both ranks add their scaled partials with red.global.add
+//     dependency wait (token-scale warps) and both ranks add their scaled partials
+//     with red.global.add
 //     (two addends onto zero: the result does not depend on their order); more
 //     ranks or BF16 output: the partial tiles go to rank 0 as one 8 KB bulk copy
 //     between shared memories (completion on an mbarrier there, an acknowledgement
@@ -47,6 +54,9 @@ namespace mxc {
 constexpr int kGemvT = 16;          // token tile = MMA N
 constexpr int kGemvMaxStages = 8;   // 256-channel stages per CTA, all resident
 constexpr int kGemvMaxSplits = 4;   // cluster size
+constexpr int kGemvSfxWarps = 4;    // token-scale warps, one per TMEM lane quadrant
+constexpr int kGemvThreads = kThreads + 32 * kGemvSfxWarps;
+constexpr int kGemvLutBytes = 256 * 32 * 4;   // 32 per-lane copies, one entry per word
 
 struct GemvParams {
   int M, N, K;
@@ -71,17 +81,15 @@ struct GemvLayout {
   static constexpr int S = kGemvMaxStages;
   static constexpr int W_OFF = 0;                      // S x [128][128 B] FP4, 128-byte swizzle
   static constexpr int X_OFF = W_OFF + S * 16384;      // S x [16][128 B] FP4 token tiles
-  // index slabs, 2 buffers x [S stages][128][16 B] (quarter j in buffer j mod 2),
-  // then the token scale atoms (one buffer).  Rank 0 receives the other ranks'
-  // partial tiles, [rank-1][128][16] FP32, in the token-scale buffer (2 ranks,
-  // free once the scales are in TMEM) or from the start of the index buffers
-  // (more ranks, free once rank 0 has decoded).
+  // index slabs, 2 buffers x [S stages][128][16 B] (quarter j in buffer j mod 2).
+  // Without the FP32 reduction in global memory, rank 0 receives the other ranks'
+  // partial tiles, [rank-1][128][16] FP32, at the start of the index buffers (free
+  // once rank 0 has decoded; never used by native weights).
   static constexpr int IDX_OFF = X_OFF + S * kGemvT * 128;
   static constexpr int IDX_BUF = S * 2048;
-  static constexpr int SFX_OFF = IDX_OFF + 2 * IDX_BUF;
-  static constexpr int SFW_OFF = IDX_OFF + 3 * IDX_BUF;           // weight scale atoms (direct, native)
-  static constexpr int LUT_OFF = SFW_OFF + (kSVQ ? 0 : S * kAtoms * 512);   // 128 words x 32 lanes
-  static constexpr int CTRL_OFF = LUT_OFF + (kVQ ? 16384 : 0);
+  static constexpr int SFW_OFF = IDX_OFF + 2 * IDX_BUF;           // weight scale atoms (direct, native)
+  static constexpr int LUT_OFF = SFW_OFF + (kSVQ ? 0 : S * kAtoms * 512);   // 256 words x 32 lanes
+  static constexpr int CTRL_OFF = LUT_OFF + (kVQ ? kGemvLutBytes : 0);
   // The slice's codebooks (at most 16 x 512 B) land in the second half of the last
   // stage's FP4 tile, which is not written before the codebook copies are laid out.
   static constexpr int CB_OFF = W_OFF + (S - 1) * 16384 + 8192;
@@ -102,9 +110,29 @@ __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint4 v) {
                : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// Writes 8 scale atoms' worth of TMEM columns for this warp's lane quadrant: column 4a
+// gets v[a], columns 4a+1..4a+3 get zero (rows 32.. of the atom are padding here).
+__device__ __forceinline__ void tmem_st_sfx8(uint32_t taddr, const uint32_t* v) {
+  const uint32_t z = 0;
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %9, %9, %9, %2, %9, %9, %9, %3, %9, %9, %9, %4, %9, %9, %9, "
+      "%5, %9, %9, %9, %6, %9, %9, %9, %7, %9, %9, %9, %8, %9, %9, %9};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(z)
+      : "memory");
+}
+// Two index bytes (k, k+1 of word x) -> 8 FP4 values through this lane's codebook
+// copy (lut_lane = copy base + lane*4; entry e in the low half of word e*32 + lane).
+__device__ __forceinline__ uint32_t lut32_pair(uint32_t lut_lane, uint32_t x, int k) {
+  const uint32_t wa = lds_u32(lut_lane + (((x >> (8 * k)) & 0xFFu) << 7));
+  const uint32_t wb = lds_u32(lut_lane + (((x >> (8 * k + 8)) & 0xFFu) << 7));
+  return __byte_perm(wa, wb, 0x5410u);
+}
 
+// At most 64 registers a thread (704 x 64 = 45,056 of the SM's 65,536), so that the
+// kernel launched next to it (the activation quantizer of the next layer, a
+// 16-CTA cluster of 256-thread CTAs) still finds room on the same SMs.
 template <int FMT, int WSRC>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(64)
     gemv_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_wq,
                 const __grid_constant__ CUtensorMap tmap_idx, const __grid_constant__ GemvParams p) {
   using L = GemvLayout<FMT, WSRC>;
@@ -123,8 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* red_ready = bars + 16;  // rank > 0: rank 0 may receive
   uint64_t* bar_sfw = bars + 17;    // weight scale atoms (bulk copy)
   uint64_t* bar_cb = bars + 18;     // codebooks of the slice (bulk copy)
-  uint64_t* bar_sfx = bars + 20;    // token scale atoms (bulk copy)
-  uint64_t* sfx_free = bars + 21;   // their tcgen05.cp copies are done: the buffer is free
+  uint64_t* sfx_ready = bars + 20; // token scale atoms in TMEM (one arrival per token-scale warp)
   uint64_t* red_ack = bars + 22;    // rank > 0: rank 0 has received this rank's partial tile
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
 
@@ -148,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint8_t* const w_sidx = p.w.sidx + (static_cast<size_t>(n_tile) * KS + ks_begin) * (128 * L::kG);
   const uint8_t* const a_sf =
       p.a_sf + (static_cast<size_t>(sf_group0) * KB4 + static_cast<size_t>(ks_begin) * A) * 512;
-  const int red_off = splits == 2 ? L::SFX_OFF : L::IDX_OFF;   // rank 0's receive area
+  const int red_off = L::IDX_OFF;                               // rank 0's receive area
   const bool red_atomic = splits == 2 && !p.out_bf16;           // split-K by global reductions
   // codebooks used by the slice: a contiguous range [qb0, qb1] of the band's row
   const int qb0 = !L::kVQ ? 0 : H == 2 ? 2 * ks_begin : (ks_begin * kStageK) / p.qk;
@@ -157,8 +184,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- setup (nothing here depends on earlier kernels) ----
   if (warp == 0) {
     // full[0..7], bar_x, dec_ph[0..3], sf_ready, accum, red_full, red_ready, bar_sfw, bar_cb,
-    // (unused), bar_sfx, sfx_free, red_ack
-    if (lane < 23) mbar_init(bars + lane, (lane >= 9 && lane < 14) ? kDecWarps : 1);
+    // (unused), sfx_ready, (unused), red_ack
+    if (lane < 23) mbar_init(bars + lane, (lane >= 9 && lane < 14) ? kDecWarps : lane == 20 ? kGemvSfxWarps : 1);
     __syncwarp();
   }
   if (warp == 0 && lane == 0) {
@@ -201,12 +228,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     cluster_wait_acquire();                          // every CTA of the cluster is set up
   }
-  // Two ranks, FP32 output: after the dependency wait (and their decode phases) rank
-  // 0's decoder warps zero this tile of Y (rows < M) and publish the stores with a
-  // release arrive on the second cluster-barrier phase; both ranks then only add to
-  // the tile.  All other warps arrive relaxed (a release would wait for their
-  // prefetches).  Every cluster-barrier arrive and wait is made by whole, converged
-  // warps.
+  // Two ranks, FP32 output: after the dependency wait rank 0's token-scale warps zero
+  // this tile of Y (rows < M) and publish the stores with a release arrive on the
+  // second cluster-barrier phase; both ranks then only add to the tile.  All other
+  // warps arrive relaxed (a release would wait for their prefetches).  Every
+  // cluster-barrier arrive and wait is made by whole, converged warps.
+  const bool sfx_warp = warp >= 2 + kDecWarps;
   if (red_atomic && warp < 2) {
     __syncwarp();
     cluster_arrive_relaxed();
@@ -253,15 +280,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
     if (splits > 1 && rank == 0 && !red_atomic) {
-      // Let the other ranks send their partials once the receive area is free:
-      // the token-scale buffer after its tcgen05.cp copies (2 ranks), the index
-      // buffers after the last decode phase (more ranks).  Sent even after a
-      // failed wait, so that no rank waits for the signal in vain.
-      if (splits == 2) {
-        mbar_wait(sfx_free, 0);
-      } else if constexpr (L::kVQ) {
-        mbar_wait(&dec_ph[3], 0);
-      }
+      // Let the other ranks send their partials once the receive area (the index
+      // buffers) is free: after the last decode phase.  Sent even after a failed
+      // wait, so that no rank waits for the signal in vain.
+      if constexpr (L::kVQ) mbar_wait(&dec_ph[3], 0);
       if (lane > 0 && lane < splits) mbar_remote_arrive(mapa_shared(smem_u32(red_ready), lane));
     }
   } else if (warp == 1) {
@@ -281,27 +303,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     griddep_wait();                                  // the token operands are written
     __syncwarp();
     if (elect_one()) {
-      mbar_arrive_expect_tx(bar_sfx, nks * A * 512);
-      bulk_load(smem + L::SFX_OFF, a_sf, nks * A * 512, bar_sfx);
       // token tiles of all stages: box {128 B, 16 rows, ks_per_split stages}; stages
       // past K (last split) arrive zero-filled and are not used
       mbar_arrive_expect_tx(bar_x, p.ks_per_split * kGemvT * 128);
       tma_load_3d(smem + L::X_OFF, &tmap_x, 0, static_cast<int>(m0), ks_begin, bar_x);
     }
     __syncwarp();
-    {
-      // token scale atoms -> TMEM (their buffer then receives rank 1's partial tile)
-      const bool got = __all_sync(0xffffffffu, mbar_wait(bar_sfx, 0));
-      if (got && elect_one()) {
-        const uint32_t sfx_s0 = smem_u32(smem + L::SFX_OFF);
-        for (int i = 0; i < nks * A; ++i)
-          tc_cp_32x128b_warpx4(tmem + L::COL_SFX + 4 * i, sdesc_sf_atom(sfx_s0 + i * 512));
-      }
-      __syncwarp();
-      if (elect_one()) tc_commit(sfx_free);          // arrives when the copies have read it (also on failure)
-      __syncwarp();
-      ok = got && ok;
-    }
+    ok = __all_sync(0xffffffffu, mbar_wait(sfx_ready, 0)) && ok;
     ok = __all_sync(0xffffffffu, mbar_wait(bar_x, 0)) && ok;
     if constexpr (L::kSVQ) ok = __all_sync(0xffffffffu, mbar_wait(sf_ready, 0)) && ok;
     if constexpr (!L::kVQ) {
@@ -339,6 +347,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (elect_one()) tc_commit(accum);
     __syncwarp();
     mbar_wait(accum, 0);      // our own MMAs finish before the CTA retires
+  } else if (sfx_warp) {
+    // ========================= token scales -> TMEM =========================
+    // Row r < 16 of atom i is word r of the atom's first 16 lines (line r, bytes
+    // 0..3 of 16); tcgen05.cp of the whole atom would put line l into lane l of
+    // every lane quadrant, columns 4i..4i+3.  Rows 16..127 are zero padding.
+    griddep_wait();                                  // the activation scales are written
+    // Lane l < 16 loads row l of atoms 0..15, lane l + 16 row l of atoms 16..31 (all
+    // loads in flight at once); the upper half reaches lanes 0..15 by a shuffle.
+    const uint32_t taddr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + L::COL_SFX;
+    const int r16 = lane & 15, half = lane >> 4;
+    uint32_t v[16];
+#pragma unroll
+    for (int a = 0; a < 16; ++a) {
+      const int atom = 16 * half + a;
+      v[a] = atom < nks * A
+                 ? __ldg(reinterpret_cast<const uint32_t*>(a_sf + static_cast<size_t>(atom) * 512 + r16 * 16))
+                 : 0u;
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {                    // 8 atoms = 32 columns per store
+      if (8 * c >= nks * A) break;                   // uniform over the warp
+      uint32_t w[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) {
+        const uint32_t x = c < 2 ? v[8 * c + a] : __shfl_down_sync(0xffffffffu, v[8 * (c - 2) + a], 16);
+        w[a] = half == 0 ? x : 0u;                   // lanes 16..31: padding rows
+      }
+      __syncwarp();                                  // tcgen05.st is warp-aligned
+      tmem_st_sfx8(taddr + 32 * c, w);
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sfx_ready);
+    if (red_atomic) {
+      if (rank == 0) {                               // zero this tile of Y, rows < M
+        const int st = threadIdx.x - (2 + kDecWarps) * 32;
+        for (int e = st; e < kGemvT * 128; e += 32 * kGemvSfxWarps) {
+          const int64_t m = m0 + e / 128;
+          if (m < p.M) reinterpret_cast<float*>(p.y)[m * p.ldy + static_cast<int64_t>(n_tile) * 128 + (e & 127)] = 0.0f;
+        }
+      }
+      __syncwarp();
+      if (rank == 0) cluster_arrive_release(); else cluster_arrive_relaxed();
+    }
   } else {
     // ======================= decoders, then epilogue ======================
     const int dw = warp - 2;
@@ -346,11 +399,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int s_l = lane & 7;                        // this lane's stage
     const int q = dw * 4 + (lane >> 3);              // 64 threads per stage
     const bool active = L::kVQ && s_l < nks;
-    // Words [8 kb, 8 kb + 8) of the codebook of this lane's stage (first or, QBlock
-    // 128 wide along K, second half of the stage), kb = (dw + s_l/2) mod 16: over the
-    // 16 warps each lane still covers all 128 words, and the 8 lanes of a quarter
-    // warp (8 stages, codebooks 512 B apart) read 8 different bank groups -- the
-    // two 16-byte halves are read in an order that alternates with the stage.
+    // Entries [16 kb, 16 kb + 16) of the codebook of this lane's stage (first or,
+    // QBlock 128 wide along K, second half of the stage), kb = (dw + s_l/2) mod 16:
+    // over the 16 warps each lane still covers all 256 entries, and the 8 lanes of a
+    // quarter warp (8 stages, codebooks 512 B apart) read 8 different bank groups --
+    // the two 16-byte halves are read in an order that alternates with the stage.
     const int kb = (dw + (s_l >> 1)) & 15;
     const int h0 = s_l & 1;
     auto cb_words = [&](int epoch, uint4* c0, uint4* c1) {
@@ -359,8 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint8_t* cp = smem + L::CB_OFF + (qbk - qb0) * 512 + 32 * kb;
       const uint4 first = *reinterpret_cast<const uint4*>(cp + 16 * h0);
       const uint4 second = *reinterpret_cast<const uint4*>(cp + 16 * (1 - h0));
-      *c0 = h0 ? second : first;                      // words 8 kb .. 8 kb + 3
-      *c1 = h0 ? first : second;                      // words 8 kb + 4 .. 8 kb + 7
+      *c0 = h0 ? second : first;                      // entries 16 kb .. 16 kb + 7
+      *c1 = h0 ? first : second;                      // entries 16 kb + 8 .. 16 kb + 15
     };
 
     // --- PreScale+ weight scale atoms -> TMEM lanes of this warp's quadrant
@@ -399,18 +452,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         cb_words(0, &c0, &c1);
         if (H == 2) cb_words(1, &d0, &d1);
       }
-      // --- codebook copies: lane l's copy (bank l) = codebook of stage l mod 8 ---
-      uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L::LUT_OFF) + (8 * kb) * 32 + lane;
+      // --- codebook copies: lane l's copy (bank l) = codebook of stage l mod 8,
+      //     entry e in the low half of word e*32 + l ---
+      uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L::LUT_OFF) + (16 * kb) * 32 + lane;
       auto lay_out = [&](const uint4& a, const uint4& b) {
         if (!active) return;
-        lut[0 * 32] = a.x;
-        lut[1 * 32] = a.y;
-        lut[2 * 32] = a.z;
-        lut[3 * 32] = a.w;
-        lut[4 * 32] = b.x;
-        lut[5 * 32] = b.y;
-        lut[6 * 32] = b.z;
-        lut[7 * 32] = b.w;
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          lut[(2 * i) * 32] = w[i] & 0xFFFFu;
+          lut[(2 * i + 1) * 32] = w[i] >> 16;
+        }
       };
       lay_out(c0, c1);
       named_bar_sync(2, kDecThreads);                // all copies written
@@ -429,10 +481,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 2; ++i) {
             const int r = (q + 64 * i + s_l) & 127;  // offset by the stage: conflict-free stores
             const uint4 iv = *reinterpret_cast<const uint4*>(idx_l + (j % 2) * L::IDX_BUF + r * 16);
-            const uint4 o0 = make_uint4(lut16_pair(lut_lane, iv.x, 0), lut16_pair(lut_lane, iv.x, 2),
-                                        lut16_pair(lut_lane, iv.y, 0), lut16_pair(lut_lane, iv.y, 2));
-            const uint4 o1 = make_uint4(lut16_pair(lut_lane, iv.z, 0), lut16_pair(lut_lane, iv.z, 2),
-                                        lut16_pair(lut_lane, iv.w, 0), lut16_pair(lut_lane, iv.w, 2));
+            const uint4 o0 = make_uint4(lut32_pair(lut_lane, iv.x, 0), lut32_pair(lut_lane, iv.x, 2),
+                                        lut32_pair(lut_lane, iv.y, 0), lut32_pair(lut_lane, iv.y, 2));
+            const uint4 o1 = make_uint4(lut32_pair(lut_lane, iv.z, 0), lut32_pair(lut_lane, iv.z, 2),
+                                        lut32_pair(lut_lane, iv.w, 0), lut32_pair(lut_lane, iv.w, 2));
             *reinterpret_cast<uint4*>(wt + r * 128 + (((2 * j) ^ (r & 7)) << 4)) = o0;
             *reinterpret_cast<uint4*>(wt + r * 128 + (((2 * j + 1) ^ (r & 7)) << 4)) = o1;
           }
@@ -447,19 +499,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     griddep_wait();                                  // the output and the token scale may be touched
     if (red_atomic) {
-      if (rank == 0) {
-        const int dt = threadIdx.x - 64;
-        const int64_t m = m0 + (dt >> 5);
-        if (m < p.M) {
-          float* yrow = reinterpret_cast<float*>(p.y) + m * p.ldy + static_cast<int64_t>(n_tile) * 128 + (dt & 31) * 4;
-          yrow[0] = 0.0f;
-          yrow[1] = 0.0f;
-          yrow[2] = 0.0f;
-          yrow[3] = 0.0f;
-        }
-      }
       __syncwarp();
-      if (rank == 0) cluster_arrive_release(); else cluster_arrive_relaxed();
+      cluster_arrive_relaxed();
     }
     float out_scale = p.w.w_tscale;
     if constexpr (WSRC == WSRC_NATIVE) {
@@ -531,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (mbase + c < p.M) store_out(y, ldy, out_bf16, mbase + c, n, v[c] * scale);
     }
   }
-  if (red_atomic && warp < 2) {                      // every thread completes the barrier phase
+  if (red_atomic && (warp < 2 || sfx_warp)) {        // every thread completes the barrier phase
     __syncwarp();
     cluster_wait_acquire();
   }

@@ -177,7 +177,7 @@ cudaError_t launch_gemv(const CUtensorMap& tx, const CUtensorMap& tw, const CUte
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kGemvThreads);
   cfg.dynamicSmemBytes = L::SMEM;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
