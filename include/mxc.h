@@ -174,7 +174,11 @@ mxc_status mxc_pack_weight(const mxc_weight_host* w, uint8_t* idx_out, uint8_t* 
                            uint8_t* sidx_out);
 
 /* Workspace bytes each GPU call needs (0 if none).  M = activation rows;
- * for mxc_moe_linear M is the total number of (token, expert) rows. */
+ * for mxc_moe_linear M is the total number of (token, expert) rows.
+ * mxc_linear: 0 below 1024 rows; from 1024 rows the room for the weight decoded
+ * once per call (N*K/2 bytes of FP4 codes rounded up to 1 KiB, then N*K/B bytes
+ * of SF-layout scales).  A smaller workspace is not an error there: the call
+ * then runs the fused decode-in-GEMM kernel, which is slower at that size. */
 size_t mxc_quantize_act_workspace_bytes(int64_t M, int64_t K, mxc_format fmt);
 size_t mxc_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, mxc_format fmt);
 size_t mxc_moe_workspace_bytes(int64_t M, int32_t E, int64_t N, int64_t K, mxc_format fmt);
@@ -224,8 +228,12 @@ mxc_status mxc_quantize_act_grouped(const void* x_bf16, int64_t M, int64_t K, in
  * a         activation, a->fmt must equal w->fmt; a->rows = M; a->sf in SF layout
  * w         packed VQ weight (device pointers inside)
  * y         device, [M, ldy] elements of y_dtype (ldy >= N)
- * ws        device workspace of mxc_linear_workspace_bytes() bytes
- * M <= 16 takes the split-K decode path; larger M the tiled prefill path. */
+ * ws        device workspace of mxc_linear_workspace_bytes() bytes (16-byte aligned)
+ * M <= 16 takes the split-K decode path; larger M the tiled prefill path, which
+ * decodes each weight tile inside the GEMM.  From 1024 rows, with the workspace
+ * given, the call instead decodes the weight once into it (MX-native FP4 codes
+ * and scales, the output of mxc_decode_weight) and runs the native block-scaled
+ * GEMM on that: the same operands in the same K order, so the same result bits. */
 mxc_status mxc_linear(const mxc_mx_tensor* a, const mxc_weight* w, void* y, int64_t ldy,
                       mxc_dtype y_dtype, void* ws, size_t ws_bytes, mxc_stream_t stream);
 

@@ -108,7 +108,10 @@ def test_packed_sizes_rejects_bad_shapes(L):
 
 
 def test_workspace_sizes(L):
-    assert L.mxc_linear_workspace_bytes(4096, 9216, 4096, 1) == 0          # prefill: none
+    # from 1024 tokens: the decoded weight (FP4 codes, then the SF-layout scales)
+    assert L.mxc_linear_workspace_bytes(4096, 9216, 4096, 1) == 9216 * 4096 // 2 + 9216 * 4096 // 16
+    assert L.mxc_linear_workspace_bytes(1024, 9216, 4096, 0) == 9216 * 4096 // 2 + 9216 * 4096 // 32
+    assert L.mxc_linear_workspace_bytes(1023, 9216, 4096, 1) == 0          # fused tiles: none
     assert L.mxc_linear_workspace_bytes(16, 9216, 4096, 1) == 0            # decode: split-K in cluster SMEM
     assert L.mxc_moe_workspace_bytes(16384, 128, 3072, 4096, 1) >= 129 * 4
     assert L.mxc_grouped_sf_rows_bound(16384, 128) == 16384 + 128 * 128

@@ -306,3 +306,83 @@ def test_decode_gemv_shapes(case):
     assert_close(y.cpu().numpy(), ref, sabs, what=f"{case}")
     yn = mxc.native_linear(a, mxc.decode_weight(pw))
     assert torch.equal(y, yn)
+
+
+# ---------------------------------------------------------------------------
+# Full-size workloads: sampled outputs and checksums (linearity) against the oracle
+# ---------------------------------------------------------------------------
+
+def _tile_and_checksums(y, a_hat, w_hat, rows, cols, what):
+    yc = y.cpu().numpy().astype(np.float64)
+    assert_close(yc[rows][:, cols], O.linear(a_hat[rows], w_hat[cols]), O.abs_linear(a_hat[rows], w_hat[cols]),
+                 what=f"{what} tile")
+    row, col, abs_row, abs_col = O.checksums(a_hat, w_hat)
+    assert_close(yc.sum(axis=1), row, abs_row, what=f"{what} row sums")
+    assert_close(yc.sum(axis=0), col, abs_col, what=f"{what} column sums")
+
+
+def test_config3_full_size_prefill():
+    """M=8192, K=4096, N=9216 (PreScale E8M0-B32): the decode-once path (workspace
+    given) and the fused path (no workspace) are bit-identical; a seeded 256 x 256
+    output tile and all row and column sums match the oracle."""
+    w, x = synth.config3()
+    pw = mxc.pack_weight(w)
+    a = mxc.quantize_act(dev_bf16(x), w.fmt)
+    y = mxc.linear(a, pw)
+    y_fused = mxc.linear(a, pw, ws=torch.empty((16,), dtype=torch.uint8, device="cuda"))
+    assert mxc.get_device_error() == 0
+    assert torch.equal(y, y_fused)
+    codes, sf, s = O.quantize_act(x, w.fmt)
+    a_hat = O.dequant_act(codes, sf, w.fmt, s)
+    w_hat = O.dequant_weight(w)
+    rng = np.random.default_rng(3)
+    r0, c0 = int(rng.integers(0, 8192 - 256)), int(rng.integers(0, 9216 - 256))
+    _tile_and_checksums(y, a_hat, w_hat, np.arange(r0, r0 + 256), np.arange(c0, c0 + 256), "config 3")
+
+
+@pytest.mark.parametrize("M", [16, 1024])
+def test_config5_full_size_point(M):
+    """K = N = 8192, PreScale E4M3-B16 with 256 x 256 QBlocks: M=16 (decode, pipelined
+    fallback: 16 stages per split) and M=1024 (decode-once); oracle tile + checksums,
+    and equality with native FP4 on the decoded weight."""
+    w = synth.config5_weight(256, "prescale", "e4m3_b16")
+    x = synth.config5_activations(M)
+    pw = mxc.pack_weight(w)
+    a = mxc.quantize_act(dev_bf16(x), w.fmt)
+    y = mxc.linear(a, pw)
+    yn = mxc.native_linear(a, mxc.decode_weight(pw))
+    assert mxc.get_device_error() == 0
+    assert torch.equal(y, yn)
+    codes, sf, s = O.quantize_act(x, w.fmt)
+    a_hat = O.dequant_act(codes, sf, w.fmt, s)
+    w_hat = O.dequant_weight(w)
+    rows = np.arange(M) if M <= 256 else np.random.default_rng(5).choice(M, 256, replace=False)
+    _tile_and_checksums(y, a_hat, w_hat, rows, np.arange(8192 - 256, 8192), f"config 5 M={M}")
+
+
+def test_config4_full_size_moe():
+    """MoE gate/up at full size: 2048 tokens routed top-8 (Zipf 1.1) over 128 experts of
+    [3072, 4096] (PreScale+ E4M3-B16) = 16384 expert-sorted rows.  The tensor scale is
+    the oracle's; for the largest, the smallest and two fixed experts, up to 64 of
+    their rows x 256 columns densely and the expert's row and column sums."""
+    row_tok, off = synth.config4_routing()
+    xg = synth.config4_activations("gate_up", row_tok)
+    experts = [synth.config4_expert(e, "gate_up") for e in range(synth.MOE_EXPERTS)]
+    packed = [mxc.pack_weight(w) for w in experts]
+    offd = torch.from_numpy(off.astype(np.int32)).cuda()
+    a = mxc.quantize_act_grouped(dev_bf16(xg), "e4m3_b16", offd)
+    y = mxc.moe_linear(a, offd, packed)
+    assert mxc.get_device_error() == 0
+    s = O.tensor_scale_e4m3(xg)
+    assert a.tscale.item() == np.float32(s)
+    counts = np.diff(off)
+    nonempty = np.flatnonzero(counts)
+    for e in sorted({int(counts.argmax()), int(nonempty[counts[nonempty].argmin()]), 0, 127}):
+        r0, r1 = int(off[e]), int(off[e + 1])
+        if r1 == r0:
+            continue
+        codes, sf, _ = O.quantize_act(xg[r0:r1], "e4m3_b16", s)
+        a_hat = O.dequant_act(codes, sf, "e4m3_b16", s)
+        w_hat = O.dequant_weight(experts[e])
+        rows = np.arange(min(64, r1 - r0))
+        _tile_and_checksums(y[r0:r1], a_hat, w_hat, rows, np.arange(1024, 1280), f"expert {e}")
