@@ -16,6 +16,10 @@ What it computes, and where the method defines it
   centroids of the weight's QBlock; the centroid's E2M1 codes are scaled by the
   MX block scale.  PostScale/PreScale store block scales directly; PreScale+
   VQ-codes groups of ds=8 scales with a Ks=256-entry scale codebook.
+  PostScale-QB ("postscale_qb"): PostScale as Table 2's bits per weight imply
+  (2.06 for E4M3-B16 at 256 x 256 QBlocks, 2.25 for E8M0-B32 at 128 x 128): the
+  MXFP4-quantized codebook carries one scale, shared by every block of its
+  QBlock, so no per-block weight scales are stored.
 * W4A4 (abstract; Table 2 caption): activations are MX-quantized to FP4 too.
   The pages give no activation recipe; the oracle follows the OCP MX rule
   (shared scale from the block's amax, E2M1 round-to-nearest-even, saturate at
@@ -237,7 +241,13 @@ def weight_codes(w) -> np.ndarray:
 
 
 def weight_scale_bytes(w) -> np.ndarray:
-    """Block-scale bytes [N, K/B]: stored directly, or scb[sidx[n, kb//8], kb % 8] (PreScale+)."""
+    """Block-scale bytes [N, K/B]: stored directly, scb[sidx[n, kb//8], kb % 8] (PreScale+),
+    or the QBlock's scale scales[n//qn, (kb*B)//qk] (PostScale-QB)."""
+    if w.strategy == "postscale_qb":
+        B = BLOCK[w.fmt]
+        n = np.arange(w.N)[:, None]
+        kb = np.arange(w.K // B)[None, :]
+        return np.asarray(w.scales, dtype=np.uint8)[n // w.qn, (kb * B) // w.qk]
     if w.strategy == "prescale_plus":
         KB = w.K // BLOCK[w.fmt]
         kb = np.arange(KB)[None, :]
@@ -310,6 +320,7 @@ def bits_per_weight(fmt: str, strategy: str, N: int, K: int, qn: int, qk: int,
     direct scales  8 bits per block of B
     PreScale+      log2(Ks) bits per group of ds scales, plus the Ks x ds byte scale
                    codebook of the tensor
+    PostScale-QB   8 bits per QBlock
     The FP32 tensor scale is excluded (Table 1 caption).  postscale_block_scales=False
     is the PostScale reading in which no per-block weight scales are stored.
     """
@@ -321,6 +332,8 @@ def bits_per_weight(fmt: str, strategy: str, N: int, K: int, qn: int, qk: int,
     if strategy == "prescale_plus":
         bits += math.log2(scale_codebook) / (scale_group * B)
         bits += scale_codebook * scale_group * 8.0 / (N * K)
+    elif strategy == "postscale_qb":
+        bits += 8.0 / (qn * qk)
     elif strategy == "prescale" or postscale_block_scales:
         bits += 8.0 / B
     return bits

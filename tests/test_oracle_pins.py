@@ -349,6 +349,35 @@ def test_bpe_mxcode_table2(golden_dir):
             assert round(bpw, 2) == g["values"][name][strat], (name, strat, bpw)
 
 
+def test_bpe_postscale_qb_table2(golden_dir):
+    """PostScale-QB (one scale per QBlock) gives Table 2's PostScale column."""
+    g = _load(golden_dir, "table2_bpe.json")
+    for name, fmt in (("E4M3-B16-FP4", "e4m3_b16"), ("E8M0-B32-FP4", "e8m0_b32")):
+        qb = g["readings"][name]["qblock"]
+        bpw = O.bits_per_weight(fmt, "postscale_qb", 9216, 4096, qb, qb)
+        assert round(bpw, 2) == g["values"][name]["postscale"], (name, bpw)
+
+
+@pytest.mark.parametrize("fmt,qn,qk", [("e4m3_b16", 128, 256), ("e8m0_b32", 256, 128), ("e8m0_b32", 128, 512)])
+def test_postscale_qb_dequant_expands_the_qblock_scale(fmt, qn, qk):
+    """Dequantizing a PostScale-QB weight equals dequantizing the same weight with
+    per-block scales copied, block by block, from the QBlock that holds the block
+    (expanded here with explicit loops over rows and K ranges)."""
+    w = synth.make_weight(9, fmt, "postscale_qb", 256, 1024, qn, qk)
+    assert w.scales.shape == (256 // qn, 1024 // qk)
+    B = O.BLOCK[fmt]
+    per_block = np.zeros((256, 1024 // B), dtype=np.uint8)
+    for n in range(256):
+        for kb in range(1024 // B):
+            k0 = kb * B                              # first input channel of the block
+            per_block[n, kb] = w.scales[n // qn][k0 // qk]
+    direct = type(w)(fmt, "postscale", 256, 1024, qn, qk, w.idx, w.cb, per_block, None, None, w.w_tscale)
+    assert np.array_equal(O.weight_scale_bytes(w), per_block)
+    assert np.array_equal(O.dequant_weight(w), O.dequant_weight(direct))
+    assert O.storage_bytes(w) * 8 / (256 * 1024) == pytest.approx(
+        O.bits_per_weight(fmt, "postscale_qb", 256, 1024, qn, qk))
+
+
 def test_index_bits_table4_caption(golden_dir):
     g = _load(golden_dir, "table2_bpe.json")["index_bits_per_weight"]
     # a full-tensor codebook on a large tensor leaves only the index bits (+ direct scales)

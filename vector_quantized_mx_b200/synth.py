@@ -30,6 +30,7 @@ FORMATS = (FMT_E8M0_B32, FMT_E4M3_B16)
 POSTSCALE = "postscale"
 PRESCALE = "prescale"
 PRESCALE_PLUS = "prescale_plus"
+POSTSCALE_QB = "postscale_qb"     # PostScale with one scale per QBlock (Table 2's 2.06 / 2.25 BPE)
 STRATEGIES = (POSTSCALE, PRESCALE, PRESCALE_PLUS)
 
 BLOCK = {FMT_E8M0_B32: 32, FMT_E4M3_B16: 16}
@@ -168,10 +169,11 @@ def make_weight(seed: int, fmt: str, strategy: str, N: int, K: int, qn: int, qk:
         else:
             scb = draw_e4m3_bytes(stream(seed, "scb", sub), (256, 8))
     else:
+        shape = (N // qn, K // qk) if strategy == POSTSCALE_QB else (N, K // B)   # per QBlock or per block
         if fmt == FMT_E8M0_B32:
-            scales = draw_e8m0_bytes(stream(seed, "scale", sub), (N, K // B), *e8m0_exp)
+            scales = draw_e8m0_bytes(stream(seed, "scale", sub), shape, *e8m0_exp)
         else:
-            scales = draw_e4m3_bytes(stream(seed, "scale", sub), (N, K // B))
+            scales = draw_e4m3_bytes(stream(seed, "scale", sub), shape)
     w_tscale = 1.0 if fmt == FMT_E8M0_B32 else TSCALE_E4M3
     return VQWeight(fmt, strategy, N, K, qn, qk, idx, cb, scales, sidx, scb, w_tscale)
 
