@@ -89,7 +89,10 @@ typedef enum mxc_format {
 typedef enum mxc_strategy {
   MXC_POSTSCALE = 0,     /* direct block scales                                */
   MXC_PRESCALE = 1,      /* direct block scales                                */
-  MXC_PRESCALE_PLUS = 2  /* VQ-coded block scales (groups of 8, 256 entries)   */
+  MXC_PRESCALE_PLUS = 2, /* VQ-coded block scales (groups of 8, 256 entries)   */
+  MXC_POSTSCALE_QB = 3   /* PostScale with one scale per QBlock: the codebook's
+                            own MX scale, shared by every block of the QBlock
+                            (the 2.06 / 2.25 bits per weight of Table 2)       */
 } mxc_strategy;
 
 typedef enum mxc_dtype { MXC_OUT_F32 = 0, MXC_OUT_BF16 = 1 } mxc_dtype;
@@ -113,7 +116,8 @@ typedef struct mxc_mx_tensor {
  *           uint8 indices (index j covers k = 256 ks + 64 c + 4j .. + 3).
  *   cb      device, [N/qn][K/qk][256] uint16 FP4 codebooks; centroid element t
  *           (k mod 4) in bits 4t..4t+3.  512 bytes per QBlock.
- *   scales  device (PostScale/PreScale), SF layout of the [N, K/B] scale bytes.
+ *   scales  device (PostScale/PreScale), SF layout of the [N, K/B] scale bytes;
+ *           (MXC_POSTSCALE_QB) [N/qn][K/qk] bytes, one scale per QBlock.
  *   sidx    device (PreScale+), [N/128][K/256][128][256/(8B)] bytes: scale-codebook
  *           index of each group of 8 consecutive scales along K.
  *   scb     device (PreScale+), [256][8] scale bytes.
@@ -134,7 +138,8 @@ typedef struct mxc_weight {
 
 /* The same weight in its logical host layout, as produced by a quantizer:
  *   idx [N, K/4] uint8, cb [N/qn, K/qk, 256] uint16, scales [N, K/B] uint8
- *   (direct) or sidx [N, K/(8B)] uint8 + scb [256, 8] uint8 (PreScale+). */
+ *   (direct), [N/qn, K/qk] uint8 (PostScale-QB), or sidx [N, K/(8B)] uint8 +
+ *   scb [256, 8] uint8 (PreScale+). */
 typedef struct mxc_weight_host {
   mxc_strategy strategy;
   mxc_format fmt;

@@ -51,7 +51,7 @@ def _pack(w):
 
 
 @pytest.mark.parametrize("fmt", ["e8m0_b32", "e4m3_b16"])
-@pytest.mark.parametrize("strategy", ["prescale", "prescale_plus"])
+@pytest.mark.parametrize("strategy", ["prescale", "prescale_plus", "postscale_qb"])
 def test_pack_layouts(L, fmt, strategy):
     N, K = 256, 768
     w = synth.make_weight(7, fmt, strategy, N, K, 128, 256)
@@ -71,6 +71,9 @@ def test_pack_layouts(L, fmt, strategy):
             for ks in range(K // 256):
                 assert np.array_equal(st[nt, ks], w.sidx[nt * 128:(nt + 1) * 128, ks * G:(ks + 1) * G])
         assert h["scales"] is None
+    elif strategy == "postscale_qb":                # one scale per QBlock, kept as [N/qn][K/qk]
+        assert h["scales"].size == (N // 128) * (K // 256) and h["sidx"] is None
+        assert np.array_equal(h["scales"].reshape(N // 128, K // 256), w.scales)
     else:
         assert h["scales"].size == L.mxc_sf_bytes(N, K, mxc.FMT[fmt])
         assert np.array_equal(mxc.sf_to_rows(h["scales"], N, K, fmt), w.scales)

@@ -135,6 +135,10 @@ DECODE_CASES = [
     ("e4m3_b16", "postscale", 256, 2048, 256, 1024),
     ("e4m3_b16", "prescale_plus", 512, 1024, 256, 256),
     ("e4m3_b16", "prescale_plus", 256, 768, 0, 0),
+    ("e4m3_b16", "postscale_qb", 512, 1024, 256, 256),
+    ("e8m0_b32", "postscale_qb", 256, 1024, 128, 128),
+    ("e8m0_b32", "postscale_qb", 256, 1536, 128, 512),
+    ("e4m3_b16", "postscale_qb", 384, 768, 0, 0),
 ]
 
 
@@ -190,8 +194,8 @@ def test_config2_decode_gemv(M):
     assert_close(y.cpu().numpy(), ref, sabs, what=f"config2 M={M}")
 
 
-SWEEP = [(f, s, qb) for f in ("e8m0_b32", "e4m3_b16") for s in ("postscale", "prescale", "prescale_plus")
-         for qb in (0, 256, 128)]
+SWEEP = [(f, s, qb) for f in ("e8m0_b32", "e4m3_b16")
+         for s in ("postscale", "prescale", "prescale_plus", "postscale_qb") for qb in (0, 256, 128)]
 
 
 @pytest.mark.parametrize("case", SWEEP, ids=lambda c: "-".join(map(str, c)))
@@ -207,8 +211,9 @@ def test_mxcode_linear_sweep(case, M):
 
 @pytest.mark.parametrize("fmt", ["e8m0_b32", "e4m3_b16"])
 @pytest.mark.parametrize("M", [16, 300])
-def test_mxcode_equals_native_on_decoded_weights(fmt, M):
-    w = synth.make_weight(41, fmt, "prescale_plus", 384, 2048, 128, 256)
+@pytest.mark.parametrize("strat", ["prescale_plus", "postscale_qb"])
+def test_mxcode_equals_native_on_decoded_weights(fmt, M, strat):
+    w = synth.make_weight(41, fmt, strat, 384, 2048, 128, 256)
     x = synth.make_activations(41, M, 2048, outliers=True)
     y, pw, a = run_mxcode(w, x)
     wn = mxc.decode_weight(pw)
@@ -259,7 +264,7 @@ def run_moe(fmt, strat, E, N, K, counts, seed):
 
 
 @pytest.mark.parametrize("fmt", ["e8m0_b32", "e4m3_b16"])
-@pytest.mark.parametrize("strat", ["prescale", "prescale_plus"])
+@pytest.mark.parametrize("strat", ["prescale", "prescale_plus", "postscale_qb"])
 def test_moe_small(fmt, strat):
     run_moe(fmt, strat, 6, 256, 512, [0, 5, 130, 1, 257, 0], seed=61)
 
@@ -292,6 +297,8 @@ GEMV_CASES = [
     (9216, 4096, 128, "e4m3_b16", "postscale", 16),       # 8 stages, two codebooks per stage
     (18944, 1024, 256, "e4m3_b16", "prescale_plus", 2),   # 148 tiles: no split (cluster of 1)
     (256, 12288, 256, "e8m0_b32", "postscale", 5),        # 12 stages per CTA: pipelined kernel
+    (9216, 4096, 256, "e4m3_b16", "postscale_qb", 16),    # PostScale-QB on the fused-QKV shape
+    (1024, 2048, 128, "e8m0_b32", "postscale_qb", 1),     # PostScale-QB, two QBlocks per stage
 ]
 
 
@@ -386,3 +393,21 @@ def test_config4_full_size_moe():
         w_hat = O.dequant_weight(experts[e])
         rows = np.arange(min(64, r1 - r0))
         _tile_and_checksums(y[r0:r1], a_hat, w_hat, rows, np.arange(1024, 1280), f"expert {e}")
+
+
+@pytest.mark.parametrize("M", [5, 16])
+def test_decode_gemv_bf16_output(M):
+    """Decode shape (N=9216, K=4096: two split-K ranks) with BF16 output, where the
+    ranks hand their partial tiles over through distributed shared memory: equal to
+    the RNE of the FP32 path (which adds the same two scaled partials in global
+    memory), to native FP4, and within the oracle's bound plus BF16 rounding."""
+    w = synth.make_weight(71, "e4m3_b16", "postscale", 9216, 4096, 256, 256)
+    x = synth.make_activations(71, M, 4096, outliers=True)
+    y16, pw, a = run_mxcode(w, x, torch.bfloat16)
+    y32 = mxc.linear(a, pw, torch.float32)
+    yn = mxc.native_linear(a, mxc.decode_weight(pw), torch.bfloat16)
+    assert mxc.get_device_error() == 0
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+    assert torch.equal(y16, yn)
+    ref, sabs = O.w4a4_linear(x, w)
+    assert_close(y16.float().cpu().numpy(), ref, sabs + np.abs(ref) * 2.0 ** -8 / TOL, what=f"bf16 M={M}")

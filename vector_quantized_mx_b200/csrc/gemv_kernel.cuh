@@ -75,6 +75,7 @@ template <int FMT, int WSRC>
 struct GemvLayout {
   static constexpr bool kVQ = WSRC != WSRC_NATIVE;
   static constexpr bool kSVQ = WSRC == WSRC_VQ_SVQ;
+  static constexpr bool kQBS = WSRC == WSRC_VQ_QBS;   // atoms built from one byte per QBlock
   static constexpr int kB = FMT == FMT_E8M0 ? 32 : 16;
   static constexpr int kAtoms = kStageK / kB / 4;      // scale atoms per 128 rows per stage
   static constexpr int kG = kStageK / (8 * kB);        // PreScale+ scale groups per row per stage
@@ -171,6 +172,7 @@ __global__ void __maxnreg__(64)
   // this slice's index tiles: nks contiguous 8 KB tiles, quarter j at +2048 j in each
   const uint8_t* const w_idx = p.w.idx + (static_cast<size_t>(n_tile) * KS + ks_begin) * 8192;
   const uint16_t* const w_cb = p.w.cb + static_cast<size_t>(qbn) * cb_per_row * 256;
+  // direct scales: this slice's atoms in the SF layout (PostScale-QB indexes p.w.sf by QBlock)
   const uint8_t* const w_sf = p.w.sf + (static_cast<size_t>(n_tile) * KB4 + static_cast<size_t>(ks_begin) * A) * 512;
   const uint8_t* const w_sidx = p.w.sidx + (static_cast<size_t>(n_tile) * KS + ks_begin) * (128 * L::kG);
   const uint8_t* const a_sf =
@@ -201,7 +203,7 @@ __global__ void __maxnreg__(64)
     }
     if constexpr (L::kSVQ) {
       l2_prefetch_bulk(w_sidx, static_cast<uint32_t>(nks) * 128 * L::kG);
-    } else {
+    } else if constexpr (!L::kQBS) {
       l2_prefetch_bulk(w_sf, static_cast<uint32_t>(nks) * A * 512);
     }
     if constexpr (L::kVQ) {
@@ -261,13 +263,35 @@ __global__ void __maxnreg__(64)
         mbar_arrive_expect_tx(&full[0], p.ks_per_split * 2048);
         tma_load_4d(smem + L::IDX_OFF, &tmap_idx, 0, 0, ks_begin, n_tile, &full[0]);
       }
-      if constexpr (!L::kSVQ) {
+      if constexpr (!L::kSVQ && !L::kQBS) {
         mbar_arrive_expect_tx(bar_sfw, nks * A * 512);
         bulk_load(smem + L::SFW_OFF, w_sf, nks * A * 512, bar_sfw);
       }
+      if constexpr (L::kVQ) {                        // K-quarter 1 of every stage
+        mbar_arrive_expect_tx(&full[1], p.ks_per_split * 2048);
+        tma_load_4d(smem + L::IDX_OFF + L::IDX_BUF, &tmap_idx, 0, 1, ks_begin, n_tile, &full[1]);
+      }
+    }
+    __syncwarp();
+    if constexpr (L::kQBS) {
+      // PostScale-QB: the weight scale atoms of the slice, each 512 bytes of its
+      // QBlock's scale (atoms in the second half of a stage use the second QBlock
+      // when the QBlock is 128 wide along K); then the MMA warp copies them to TMEM.
+      const uint8_t* qb = p.w.sf + static_cast<size_t>((static_cast<int64_t>(n_tile) * 128) / p.qn) * (K / p.qk);
+      for (int i = 0; i < nks * A; ++i) {
+        const int ks = ks_begin + i / A, a = i % A;
+        const int qbk = H == 2 ? 2 * ks + (a >= A / 2 ? 1 : 0) : (ks * kStageK) / p.qk;
+        const uint32_t v = static_cast<uint32_t>(__ldg(qb + qbk)) * 0x01010101u;
+        reinterpret_cast<uint4*>(smem + L::SFW_OFF + i * 512)[lane] = make_uint4(v, v, v, v);
+      }
+      fence_proxy_async_smem();                      // generic writes -> tcgen05.cp reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_sfw);
+    }
+    if (elect_one()) {
       if constexpr (L::kVQ) {
-        for (int j = 1; j < 4; ++j) {                // K-quarter j of every stage
-          if (j >= 2 && !mbar_wait(&dec_ph[j - 2], 0)) break;   // its buffer has been decoded
+        for (int j = 2; j < 4; ++j) {                // K-quarter j of every stage
+          if (!mbar_wait(&dec_ph[j - 2], 0)) break;  // its buffer has been decoded
           mbar_arrive_expect_tx(&full[j], p.ks_per_split * 2048);
           tma_load_4d(smem + L::IDX_OFF + (j % 2) * L::IDX_BUF, &tmap_idx, 0, j, ks_begin, n_tile, &full[j]);
         }
@@ -524,7 +548,7 @@ __global__ void __maxnreg__(64)
         float* const y = reinterpret_cast<float*>(p.y);
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-          if (mbase + c < p.M) atomicAdd(y + (mbase + c) * p.ldy + n, v[c] * scale);
+          if (mbase + c < p.M) atomicAdd(y + (mbase + c) * p.ldy + n, __fmul_rn(v[c], scale));
       }
     } else if (splits > 1) {
       if (rank != 0) {
@@ -552,16 +576,25 @@ __global__ void __maxnreg__(64)
         }
         store = store && got;
         if (store) {
+          // scaled partials summed in rank order: with two ranks the same FP32 value
+          // as the reduction in global memory (+0 + s*v0 + s*v1), so a BF16 output is
+          // exactly the rounding of the FP32 one
+          // (separately rounded products and sums: no contraction into an FMA)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) v[c] = __fmul_rn(v[c], scale);
           for (int r = 1; r < splits; ++r) {
             const float4 o = *reinterpret_cast<const float4*>(smem + red_off + ((r - 1) * 128 * kGemvT +
                                                                                   row * kGemvT + cg * 4) * 4);
-            v[0] += o.x;
-            v[1] += o.y;
-            v[2] += o.z;
-            v[3] += o.w;
+            v[0] = __fadd_rn(v[0], __fmul_rn(o.x, scale));
+            v[1] = __fadd_rn(v[1], __fmul_rn(o.y, scale));
+            v[2] = __fadd_rn(v[2], __fmul_rn(o.z, scale));
+            v[3] = __fadd_rn(v[3], __fmul_rn(o.w, scale));
           }
         }
       }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) v[c] = __fmul_rn(v[c], scale);   // no split: scale the whole sum
     }
     if (store) {
       void* const y = p.y;
@@ -569,7 +602,7 @@ __global__ void __maxnreg__(64)
       const int out_bf16 = p.out_bf16;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        if (mbase + c < p.M) store_out(y, ldy, out_bf16, mbase + c, n, v[c] * scale);
+        if (mbase + c < p.M) store_out(y, ldy, out_bf16, mbase + c, n, v[c]);
     }
   }
   if (red_atomic && (warp < 2 || sfx_warp)) {        // every thread completes the barrier phase

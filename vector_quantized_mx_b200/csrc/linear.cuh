@@ -220,6 +220,7 @@ cudaError_t dispatch_gemv(int wsrc, const CUtensorMap& tx, const CUtensorMap& tw
                           const GemvParams& p, dim3 grid, cudaStream_t stream) {
   if (wsrc == WSRC_VQ_DIRECT) return launch_gemv<FMT, WSRC_VQ_DIRECT>(tx, tw, ti, p, grid, stream);
   if (wsrc == WSRC_VQ_SVQ) return launch_gemv<FMT, WSRC_VQ_SVQ>(tx, tw, ti, p, grid, stream);
+  if (wsrc == WSRC_VQ_QBS) return launch_gemv<FMT, WSRC_VQ_QBS>(tx, tw, ti, p, grid, stream);
   return launch_gemv<FMT, WSRC_NATIVE>(tx, tw, ti, p, grid, stream);
 }
 
@@ -328,10 +329,12 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
   if (a.fmt == FMT_E8M0) {
     if (a.wsrc == WSRC_VQ_DIRECT) err = dispatch_tile<FMT_E8M0, WSRC_VQ_DIRECT>(T, tx, tw, p, grid, stream);
     else if (a.wsrc == WSRC_VQ_SVQ) err = dispatch_tile<FMT_E8M0, WSRC_VQ_SVQ>(T, tx, tw, p, grid, stream);
+    else if (a.wsrc == WSRC_VQ_QBS) err = dispatch_tile<FMT_E8M0, WSRC_VQ_QBS>(T, tx, tw, p, grid, stream);
     else err = dispatch_tile<FMT_E8M0, WSRC_NATIVE>(T, tx, tw, p, grid, stream);
   } else {
     if (a.wsrc == WSRC_VQ_DIRECT) err = dispatch_tile<FMT_E4M3, WSRC_VQ_DIRECT>(T, tx, tw, p, grid, stream);
     else if (a.wsrc == WSRC_VQ_SVQ) err = dispatch_tile<FMT_E4M3, WSRC_VQ_SVQ>(T, tx, tw, p, grid, stream);
+    else if (a.wsrc == WSRC_VQ_QBS) err = dispatch_tile<FMT_E4M3, WSRC_VQ_QBS>(T, tx, tw, p, grid, stream);
     else err = dispatch_tile<FMT_E4M3, WSRC_NATIVE>(T, tx, tw, p, grid, stream);
   }
   return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
@@ -376,10 +379,12 @@ mxc_status run_moe_linear(const MoeArgs& m, cudaStream_t stream) {
   cudaError_t err;
   if (a.fmt == FMT_E8M0) {
     if (a.wsrc == WSRC_VQ_DIRECT) err = launch_gemm<FMT_E8M0, WSRC_VQ_DIRECT, 128, true>(tx, tx, p, grid, stream);
-    else err = launch_gemm<FMT_E8M0, WSRC_VQ_SVQ, 128, true>(tx, tx, p, grid, stream);
+    else if (a.wsrc == WSRC_VQ_SVQ) err = launch_gemm<FMT_E8M0, WSRC_VQ_SVQ, 128, true>(tx, tx, p, grid, stream);
+    else err = launch_gemm<FMT_E8M0, WSRC_VQ_QBS, 128, true>(tx, tx, p, grid, stream);
   } else {
     if (a.wsrc == WSRC_VQ_DIRECT) err = launch_gemm<FMT_E4M3, WSRC_VQ_DIRECT, 128, true>(tx, tx, p, grid, stream);
-    else err = launch_gemm<FMT_E4M3, WSRC_VQ_SVQ, 128, true>(tx, tx, p, grid, stream);
+    else if (a.wsrc == WSRC_VQ_SVQ) err = launch_gemm<FMT_E4M3, WSRC_VQ_SVQ, 128, true>(tx, tx, p, grid, stream);
+    else err = launch_gemm<FMT_E4M3, WSRC_VQ_QBS, 128, true>(tx, tx, p, grid, stream);
   }
   return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
 }
@@ -405,11 +410,13 @@ cudaError_t launch_decode_dump(const DecodeArgs& a, cudaStream_t stream) {
 mxc_status run_decode_weight(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t err;
   if (a.fmt == FMT_E8M0) {
-    err = a.wsrc == WSRC_VQ_SVQ ? launch_decode_dump<FMT_E8M0, WSRC_VQ_SVQ>(a, stream)
-                                : launch_decode_dump<FMT_E8M0, WSRC_VQ_DIRECT>(a, stream);
+    err = a.wsrc == WSRC_VQ_SVQ   ? launch_decode_dump<FMT_E8M0, WSRC_VQ_SVQ>(a, stream)
+          : a.wsrc == WSRC_VQ_QBS ? launch_decode_dump<FMT_E8M0, WSRC_VQ_QBS>(a, stream)
+                                  : launch_decode_dump<FMT_E8M0, WSRC_VQ_DIRECT>(a, stream);
   } else {
-    err = a.wsrc == WSRC_VQ_SVQ ? launch_decode_dump<FMT_E4M3, WSRC_VQ_SVQ>(a, stream)
-                                : launch_decode_dump<FMT_E4M3, WSRC_VQ_DIRECT>(a, stream);
+    err = a.wsrc == WSRC_VQ_SVQ   ? launch_decode_dump<FMT_E4M3, WSRC_VQ_SVQ>(a, stream)
+          : a.wsrc == WSRC_VQ_QBS ? launch_decode_dump<FMT_E4M3, WSRC_VQ_QBS>(a, stream)
+                                  : launch_decode_dump<FMT_E4M3, WSRC_VQ_DIRECT>(a, stream);
   }
   return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
 }

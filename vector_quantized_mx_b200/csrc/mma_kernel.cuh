@@ -36,7 +36,9 @@
 
 namespace mxc {
 
-enum : int { WSRC_VQ_DIRECT = 0, WSRC_VQ_SVQ = 1, WSRC_NATIVE = 2 };
+// Weight sources: VQ with block scales stored directly, VQ with VQ-coded block
+// scales (PreScale+), native FP4, VQ with one scale per QBlock (PostScale-QB).
+enum : int { WSRC_VQ_DIRECT = 0, WSRC_VQ_SVQ = 1, WSRC_NATIVE = 2, WSRC_VQ_QBS = 3 };
 enum : int { FMT_E8M0 = 0, FMT_E4M3 = 1 };
 
 constexpr int kMaxSplits = 4;      // cluster split-K factor of the decode path
@@ -75,6 +77,8 @@ template <int FMT, int WSRC, int T, int NCB = 1>
 struct StageLayout {
   static constexpr bool kVQ = WSRC != WSRC_NATIVE;
   static constexpr bool kSVQ = WSRC == WSRC_VQ_SVQ;
+  static constexpr bool kQBS = WSRC == WSRC_VQ_QBS;
+  static constexpr bool kSfwDec = kSVQ || kQBS;       // weight scale atoms written by the decoders
   static constexpr int kB = FMT == FMT_E8M0 ? 32 : 16;
   static constexpr int kAtoms = kStageK / kB / 4;     // scale atoms per 128 rows per stage
   static constexpr int kXG = (T + 127) / 128;         // 128-row scale groups in the token tile
@@ -209,6 +213,18 @@ __device__ __forceinline__ void decode_sf_tile(const uint8_t* __restrict__ sidx,
     const uint2 s8 = *reinterpret_cast<const uint2*>(scb + si * 8);
     reinterpret_cast<uint32_t*>(sfw + (2 * g) * 512)[word] = s8.x;
     reinterpret_cast<uint32_t*>(sfw + (2 * g + 1) * 512)[word] = s8.y;
+  }
+}
+
+// PostScale-QB: every block of a QBlock has the QBlock's scale, so the stage's A
+// scale atoms are that byte everywhere -- b0 for all of them, or b0 for the first
+// half of the stage and b1 for the second when the QBlock is 128 wide along K.
+template <int A, int NT>
+__device__ __forceinline__ void fill_sf_qbs(uint8_t* __restrict__ sfw, uint32_t b0, uint32_t b1, int dt) {
+  const uint32_t w0 = b0 * 0x01010101u, w1 = b1 * 0x01010101u;
+  for (int u = dt; u < A * 32; u += NT) {             // 16 bytes a thread, atom u / 32
+    const uint32_t v = (u / 32) < A / 2 ? w0 : w1;
+    reinterpret_cast<uint4*>(sfw)[u] = make_uint4(v, v, v, v);
   }
 }
 
@@ -368,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (WSRC == WSRC_NATIVE) tx += 16384 + A * 512;
     if constexpr (WSRC == WSRC_VQ_DIRECT) tx += 8192 + (cb_split ? 1024 : 512) + A * 512;
     if constexpr (WSRC == WSRC_VQ_SVQ) tx += 8192 + (cb_split ? 1024 : 512) + 128 * L::kG;
+    if constexpr (WSRC == WSRC_VQ_QBS) tx += 8192 + (cb_split ? 1024 : 512);
     const uint8_t* sfx_src = a_sf + static_cast<size_t>(sf_group0) * KB4 * 512;
     const uint8_t* sfw_src = w_sf + static_cast<size_t>(n_tile) * KB4 * 512;
     const uint8_t* idx_src = w_idx + static_cast<size_t>(n_tile) * KS * 8192;
@@ -399,10 +416,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_load(st + L::CB_OFF, cb_src + static_cast<size_t>(qbk) * 256, cb_split ? 1024 : 512, &full[s]);
           if constexpr (WSRC == WSRC_VQ_DIRECT) {
             bulk_load(st + L::SFW_OFF, sfw_src + static_cast<size_t>(ks) * A * 512, A * 512, &full[s]);
-          } else {
+          } else if constexpr (WSRC == WSRC_VQ_SVQ) {
             bulk_load(st + L::SIDX_OFF, sidx_src + static_cast<size_t>(ks) * (128 * L::kG), 128 * L::kG,
                       &full[s]);
-          }
+          }                                        // PostScale-QB: the decoders write the atoms
         }
       }
       __syncwarp();
@@ -428,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int a = 0; a < A; ++a)
             tc_cp_32x128b_warpx4(tmem + L::COL_SFX + (XG == 2 ? 8 * a + 4 * g : 4 * a),
                                  sdesc_sf_atom(sfx_s + (g * A + a) * 512));
-        if constexpr (!L::kSVQ) {
+        if constexpr (!L::kSfwDec) {
 #pragma unroll
           for (int a = 0; a < A; ++a)
             tc_cp_32x128b_warpx4(tmem + L::COL_SFW + 4 * a, sdesc_sf_atom(sfw_s + a * 512));
@@ -440,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
       }
       if (elect_one()) {
-        if constexpr (L::kSVQ) {
+        if constexpr (L::kSfwDec) {
 #pragma unroll
           for (int a = 0; a < A; ++a)
             tc_cp_32x128b_warpx4(tmem + L::COL_SFW + 4 * a, sdesc_sf_atom(sfw_s + a * 512));
@@ -486,6 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr int kBufs = 2 / G;                   // copy buffers per group
       const int grp = dt / GT, gt = dt - grp * GT;
       const int bar_id = 2 + grp;
+      const int qbn_w = static_cast<int>((static_cast<int64_t>(n_tile) * 128) / qn);   // QBlock row
       uint8_t* lut = smem + L::LUT_OFF + grp * kBufs * kBuf;
       const uint32_t lut_s = smem_u32(lut);
       ItemMap<GT> cm;
@@ -505,6 +523,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* st = stages + s * L::BYTES;
         decode_w_tile<GT>(st + L::IDX_OFF, lut_s + b * kBuf, st + L::W_OFF, cm);
         if constexpr (L::kSVQ) decode_sf_tile<L::kG, GT>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, gt);
+        if constexpr (L::kQBS) {
+          const int ks = ks_begin + i;
+          const uint8_t* qb = w_sf + static_cast<size_t>(qbn_w) * (K / qk);
+          const int qbk = cb_split ? 2 * ks : (ks * kStageK) / qk;
+          fill_sf_qbs<A, GT>(st + L::SFW_OFF, __ldg(qb + qbk), __ldg(qb + qbk + (cb_split ? 1 : 0)), gt);
+        }
         fence_proxy_async_smem();                    // each thread's tile writes -> async proxy
         __syncwarp();
         if (lane == 0) mbar_arrive(&dec[s]);         // one arrival per decoder warp of the group
@@ -635,7 +659,7 @@ __global__ void __launch_bounds__(160)
   const size_t tile_id = static_cast<size_t>(n_tile) * KS + ks;
   const size_t wsf = (static_cast<size_t>(n_tile) * KB4 + static_cast<size_t>(ks) * A) * 512;
   if (threadIdx.x == 0) {
-    const uint32_t tx = 8192 + (cb_split ? 1024 : 512) + (L::kSVQ ? 128 * L::kG : A * 512);
+    const uint32_t tx = 8192 + (cb_split ? 1024 : 512) + (L::kSVQ ? 128 * L::kG : L::kQBS ? 0 : A * 512);
     mbar_arrive_expect_tx(bar, tx);
     bulk_load(st + L::IDX_OFF, w.idx + tile_id * 8192, 8192, bar);
     const int qbn = static_cast<int>((static_cast<int64_t>(n_tile) * 128) / qn);
@@ -644,7 +668,7 @@ __global__ void __launch_bounds__(160)
               bar);
     if constexpr (L::kSVQ) {
       bulk_load(st + L::SIDX_OFF, w.sidx + tile_id * (128 * L::kG), 128 * L::kG, bar);
-    } else {
+    } else if constexpr (!L::kQBS) {
       bulk_load(st + L::SFW_OFF, w.sf + wsf, A * 512, bar);
     }
   }
@@ -657,6 +681,11 @@ __global__ void __launch_bounds__(160)
     cm.init(dt, cb_split);
     decode_w_tile<128>(st + L::IDX_OFF, smem_u32(lut), st + L::W_OFF, cm);
     if constexpr (L::kSVQ) decode_sf_tile<L::kG, 128>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, dt);
+    if constexpr (L::kQBS) {
+      const uint8_t* qb = w.sf + static_cast<size_t>((static_cast<int64_t>(n_tile) * 128) / qn) * (K / qk);
+      const int qbk = cb_split ? 2 * ks : (ks * kStageK) / qk;
+      fill_sf_qbs<A, 128>(st + L::SFW_OFF, __ldg(qb + qbk), __ldg(qb + qbk + cb_split), dt);
+    }
   }
   __syncthreads();
   if (threadIdx.x >= 32 && ok) {

@@ -41,6 +41,11 @@ mxc_status resolve_qblock(int64_t N, int64_t K, int64_t qn_in, int64_t qk_in, in
   return MXC_OK;
 }
 
+// Where a VQ weight's block scales come from, for the kernels.
+int wsrc_of(mxc_strategy st) {
+  return st == MXC_PRESCALE_PLUS ? WSRC_VQ_SVQ : st == MXC_POSTSCALE_QB ? WSRC_VQ_QBS : WSRC_VQ_DIRECT;
+}
+
 mxc_status check_shape(int64_t N, int64_t K) {
   if (N <= 0 || K <= 0) return MXC_ERR_INVALID_ARG;
   if (N % kTileN || K % kStageK) return MXC_ERR_ALIGNMENT;
@@ -52,7 +57,8 @@ mxc_status check_weight_common(mxc_strategy strategy, mxc_format fmt, int64_t N,
                                int64_t* rqn, int64_t* rqk) {
   mxc_status s = check_format(fmt);
   if (s != MXC_OK) return s;
-  if (strategy != MXC_POSTSCALE && strategy != MXC_PRESCALE && strategy != MXC_PRESCALE_PLUS)
+  if (strategy != MXC_POSTSCALE && strategy != MXC_PRESCALE && strategy != MXC_PRESCALE_PLUS &&
+      strategy != MXC_POSTSCALE_QB)
     return MXC_ERR_INVALID_ARG;
   if ((s = check_shape(N, K)) != MXC_OK) return s;
   return resolve_qblock(N, K, qn, qk, rqn, rqk);
@@ -141,6 +147,10 @@ mxc_status mxc_packed_weight_sizes(const mxc_weight_host* w, mxc_packed_sizes* o
     out->scales = 0;
     out->sidx = static_cast<size_t>(w->N) * (w->K / (8 * B));
     out->scb = 256 * 8;
+  } else if (w->strategy == MXC_POSTSCALE_QB) {
+    out->scales = static_cast<size_t>(w->N / qn) * static_cast<size_t>(w->K / qk);
+    out->sidx = 0;
+    out->scb = 0;
   } else {
     out->scales = sf_bytes(w->N, w->K, w->fmt);
     out->sidx = 0;
@@ -173,6 +183,9 @@ mxc_status mxc_pack_weight(const mxc_weight_host* w, uint8_t* idx_out, uint8_t* 
           for (int64_t r = 0; r < kTileN; ++r)
             std::memcpy(sidx_out + ((nt * KS + ks) * kTileN + r) * G, w->sidx + (nt * kTileN + r) * row + ks * G, G);
     }
+  } else if (scales_out && w->strategy == MXC_POSTSCALE_QB) {
+    if (!w->scales) return MXC_ERR_INVALID_ARG;
+    std::memcpy(scales_out, w->scales, sz.scales);   // [N/qn][K/qk]: already the packed layout
   } else if (scales_out) {
     if (!w->scales) return MXC_ERR_INVALID_ARG;
     const int64_t KB = K / B;
@@ -281,7 +294,7 @@ mxc_status mxc_linear(const mxc_mx_tensor* a, const mxc_weight* w, void* y, int6
   if ((s = check_device()) != MXC_OK) return s;
   LinearArgs L{};
   fill_activation(L, a);
-  L.wsrc = w->strategy == MXC_PRESCALE_PLUS ? WSRC_VQ_SVQ : WSRC_VQ_DIRECT;
+  L.wsrc = wsrc_of(w->strategy);
   L.N = w->N;
   L.qn = qn;
   L.qk = qk;
@@ -351,7 +364,7 @@ mxc_status mxc_moe_linear(const mxc_mx_tensor* a, const int32_t* d_offsets, cons
   if ((s = check_device()) != MXC_OK) return s;
   MoeArgs m{};
   fill_activation(m.base, a);
-  m.base.wsrc = w0.strategy == MXC_PRESCALE_PLUS ? WSRC_VQ_SVQ : WSRC_VQ_DIRECT;
+  m.base.wsrc = wsrc_of(w0.strategy);
   m.base.N = w0.N;
   m.base.qn = qn;
   m.base.qk = qk;
@@ -420,7 +433,7 @@ mxc_status mxc_decode_weight(const mxc_weight* w, uint8_t* q_out, int64_t ldq, u
   if (ldq < w->K / 2 || ldq % 16 || !aligned16(q_out) || !aligned16(sf_out)) return MXC_ERR_ALIGNMENT;
   if ((s = check_device()) != MXC_OK) return s;
   DecodeArgs d{};
-  d.wsrc = w->strategy == MXC_PRESCALE_PLUS ? WSRC_VQ_SVQ : WSRC_VQ_DIRECT;
+  d.wsrc = wsrc_of(w->strategy);
   d.fmt = w->fmt == MXC_FMT_E8M0_B32 ? FMT_E8M0 : FMT_E4M3;
   d.N = w->N;
   d.K = w->K;

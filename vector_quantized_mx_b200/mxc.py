@@ -19,7 +19,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmxc.so"
 
 FMT = {"e8m0_b32": 0, "e4m3_b16": 1, "ue5m3_b16": 2}
 BLOCK = {"e8m0_b32": 32, "e4m3_b16": 16}
-STRATEGY = {"postscale": 0, "prescale": 1, "prescale_plus": 2}
+STRATEGY = {"postscale": 0, "prescale": 1, "prescale_plus": 2, "postscale_qb": 3}
 OUT = {torch.float32: 0, torch.bfloat16: 1}
 
 STATUS = {0: "MXC_OK", 1: "MXC_ERR_INVALID_ARG", 2: "MXC_ERR_UNSUPPORTED", 3: "MXC_ERR_ALIGNMENT",
@@ -213,6 +213,8 @@ class PackedWeight:
         n = self.idx.numel() + self.cb.numel() * 2
         if self.strategy == "prescale_plus":
             return n + self.sidx.numel() + self.scb.numel()
+        if self.strategy == "postscale_qb":
+            return n + self.scales.numel()              # one scale per QBlock
         return n + self.N * self.K // BLOCK[self.fmt]
 
 
