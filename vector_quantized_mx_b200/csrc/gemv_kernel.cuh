@@ -277,11 +277,17 @@ __global__ void __maxnreg__(64)
       // PostScale-QB: the weight scale atoms of the slice, each 512 bytes of its
       // QBlock's scale (atoms in the second half of a stage use the second QBlock
       // when the QBlock is 128 wide along K); then the MMA warp copies them to TMEM.
+      // Lane i loads atom i's byte (at most 32 atoms), so all loads are in flight at
+      // once; each atom then takes its byte from that lane.
       const uint8_t* qb = p.w.sf + static_cast<size_t>((static_cast<int64_t>(n_tile) * 128) / p.qn) * (K / p.qk);
-      for (int i = 0; i < nks * A; ++i) {
-        const int ks = ks_begin + i / A, a = i % A;
+      uint32_t mine = 0;
+      if (lane < nks * A) {
+        const int ks = ks_begin + lane / A, a = lane % A;
         const int qbk = H == 2 ? 2 * ks + (a >= A / 2 ? 1 : 0) : (ks * kStageK) / p.qk;
-        const uint32_t v = static_cast<uint32_t>(__ldg(qb + qbk)) * 0x01010101u;
+        mine = __ldg(qb + qbk);
+      }
+      for (int i = 0; i < nks * A; ++i) {
+        const uint32_t v = __shfl_sync(0xffffffffu, mine, i) * 0x01010101u;
         reinterpret_cast<uint4*>(smem + L::SFW_OFF + i * 512)[lane] = make_uint4(v, v, v, v);
       }
       fence_proxy_async_smem();                      // generic writes -> tcgen05.cp reads

@@ -521,14 +521,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = grp; i < nks && ok; i += G) {
         const int s = i % STAGES;
         uint8_t* st = stages + s * L::BYTES;
-        decode_w_tile<GT>(st + L::IDX_OFF, lut_s + b * kBuf, st + L::W_OFF, cm);
-        if constexpr (L::kSVQ) decode_sf_tile<L::kG, GT>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, gt);
-        if constexpr (L::kQBS) {
+        uint32_t qs0 = 0, qs1 = 0;                   // PostScale-QB: the stage's QBlock scale(s),
+        if constexpr (L::kQBS) {                     // loaded before the decode hides their latency
           const int ks = ks_begin + i;
           const uint8_t* qb = w_sf + static_cast<size_t>(qbn_w) * (K / qk);
           const int qbk = cb_split ? 2 * ks : (ks * kStageK) / qk;
-          fill_sf_qbs<A, GT>(st + L::SFW_OFF, __ldg(qb + qbk), __ldg(qb + qbk + (cb_split ? 1 : 0)), gt);
+          qs0 = __ldg(qb + qbk);
+          qs1 = __ldg(qb + qbk + (cb_split ? 1 : 0));
         }
+        decode_w_tile<GT>(st + L::IDX_OFF, lut_s + b * kBuf, st + L::W_OFF, cm);
+        if constexpr (L::kSVQ) decode_sf_tile<L::kG, GT>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, gt);
+        if constexpr (L::kQBS) fill_sf_qbs<A, GT>(st + L::SFW_OFF, qs0, qs1, gt);
         fence_proxy_async_smem();                    // each thread's tile writes -> async proxy
         __syncwarp();
         if (lane == 0) mbar_arrive(&dec[s]);         // one arrival per decoder warp of the group
