@@ -1,0 +1,75 @@
+"""Host replay of the grouped-expert (MoE) tile scheduler.
+
+Device side (act_quant.cuh group_prologue_kernel, mma_kernel.cuh gemm_kernel<MOE>):
+the prologue turns expert offsets into tile_prefix[g] = sum over g' < g of
+ceil(rows_g' / 128); the launch has ceil(M/128) + E row tiles; row tile t with
+t < tile_prefix[E] belongs to the last expert e whose tile_prefix[e] <= t (binary
+search) and covers rows [offsets[e] + 128 (t - tile_prefix[e]), offsets[e+1]) clipped
+to 128 rows; later row tiles exit.  Its scale rows are group t of the grouped
+quantizer's padded SF layout.  This replay checks, for many offset patterns (empty
+experts, single rows, multiples of 128, one huge expert), that the launch has
+enough row tiles and that every expert row is computed exactly once, by a tile of
+its own expert, and no tile reaches into another expert.
+"""
+import numpy as np
+import pytest
+
+
+def tile_prefix(offsets):
+    counts = np.diff(offsets)
+    tiles = np.where(counts > 0, (counts + 127) // 128, 0)
+    return np.concatenate([[0], np.cumsum(tiles)])
+
+
+def owner(prefix, E, t):
+    lo, hi = 0, E - 1
+    while lo < hi:                       # last expert whose first tile <= t
+        mid = (lo + hi + 1) >> 1
+        if prefix[mid] <= t:
+            lo = mid
+        else:
+            hi = mid - 1
+    return lo
+
+
+def replay(offsets):
+    E = len(offsets) - 1
+    M = int(offsets[-1])
+    prefix = tile_prefix(offsets)
+    grid_tiles = (M + 127) // 128 + E
+    assert grid_tiles >= prefix[E]
+    cover = np.zeros(M, dtype=np.int64)
+    for t in range(grid_tiles):
+        if t >= prefix[E]:
+            continue                     # the CTA exits
+        e = owner(prefix, E, t)
+        m0 = offsets[e] + (t - prefix[e]) * 128
+        m1 = min(m0 + 128, offsets[e + 1])
+        assert offsets[e] <= m0 < m1 <= offsets[e + 1], (t, e, m0, m1)
+        cover[m0:m1] += 1
+    assert np.all(cover == 1)
+
+
+def patterns():
+    yield [0, 0]
+    yield [0, 1]
+    yield [0, 128]
+    yield [0, 129]
+    yield [0, 0, 0, 5, 5, 300, 300]                        # empty experts first, between, last
+    yield [0, 256, 256, 257, 1000, 1000]
+    rng = np.random.default_rng(0)
+    for E in (1, 2, 7, 128):
+        for _ in range(20):
+            counts = rng.choice([0, 0, 1, 16, 127, 128, 129, 255, 256, 1841], size=E)
+            yield np.concatenate([[0], np.cumsum(counts)]).tolist()
+
+
+@pytest.mark.parametrize("offsets", list(patterns()))
+def test_every_row_once(offsets):
+    replay(np.asarray(offsets, dtype=np.int64))
+
+
+def test_zipf_routing_of_the_moe_workload():
+    from vector_quantized_mx_b200 import synth
+    _, off = synth.config4_routing()
+    replay(np.asarray(off, dtype=np.int64))
