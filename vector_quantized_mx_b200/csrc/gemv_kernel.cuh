@@ -1,6 +1,6 @@
 // gemv_kernel.cuh -- the decode-shaped MXCode W4A4 linear layer (M <= 16 tokens).
 //
-// "MXCode: Vector Quantization for MX-Native Inference at Scale", Sec. 5 (decode
+// "MXCode: Vector Quantization for MX-Native Inference at Scale", Table 3 (decode
 // TPOT): at decode batch sizes the layer streams its weights once, so the time goes
 // to bringing the compressed weights in and turning them into tensor-core operands.
 // Each CTA owns 128 output channels x a slice of at most 8 stages of 256 input
@@ -9,8 +9,8 @@
 //
 //   * the loader copies the slice's index bytes with one 4-D tensor copy per
 //     K-quarter (quarter c of every stage: the packed layout stores each 128 x 256
-//     tile as four slabs of 64 input channels), quarter 0 first, and all token
-//     tiles with one 3-D tensor copy;
+//     tile as four slabs of 64 input channels), quarter 0 first; the MMA warp
+//     fetches all token tiles with one 3-D tensor copy;
 //   * decoder lane l decodes stage l mod 8, so the 32 per-lane codebook copies in
 //     shared memory hold, in bank l, the codebook of lane l's stage: the codebooks
 //     of the whole slice are laid out once (one entry per 32-bit word, 32 KB) and
@@ -22,7 +22,8 @@
 //     both give bit-identical results on the same operands;
 //   * the index slabs pass through two quarter buffers (quarters 2 and 3 reuse
 //     the buffers of quarters 0 and 1 once those are decoded); the weight scale
-//     atoms come in by one bulk copy and the MMA warp moves them to TMEM with
+//     atoms come in by one bulk copy (PostScale-QB: the loader warp builds them
+//     from one byte per QBlock) and the MMA warp moves them to TMEM with
 //     tcgen05.cp;
 //   * token scales: with at most 16 tokens only the first 16 of the 128 rows of
 //     an activation scale atom carry scales (the rest is zero padding), so four
@@ -31,11 +32,11 @@
 //     make of the whole atom -- instead of 144 CTAs copying 16 KB each;
 //   * split-K, two ranks, FP32 output: rank 0 zeroes its output tile after the
 //     dependency wait (token-scale warps) and both ranks add their scaled partials
-//     with red.global.add
-//     (two addends onto zero: the result does not depend on their order); more
-//     ranks or BF16 output: the partial tiles go to rank 0 as one 8 KB bulk copy
-//     between shared memories (completion on an mbarrier there, an acknowledgement
-//     back before the sender may exit) and rank 0 adds them in rank order.
+//     with red.global.add (two addends onto zero: the result does not depend on
+//     their order); more ranks or BF16 output: the partial tiles go to rank 0 as
+//     one 8 KB bulk copy between shared memories (completion on an mbarrier there,
+//     an acknowledgement back before the sender may exit) and rank 0 adds the
+//     scaled partials in rank order (for two ranks the same FP32 value).
 //
 // Programmatic dependent launch: only the token tiles, the token scales and the
 // activation tensor scale come from the previous kernel (typically the activation
