@@ -10,25 +10,28 @@
 //               copies of its scale atoms, the stage's packed index tile (8 KB),
 //               its QBlock codebook(s) (512 B each) and the weight scales (direct
 //               atoms, or scale-VQ indices).  Native FP4 weights come by TMA.
-//   warps 2..5  decoders: the stage's codebook is replicated once per lane (so
-//               the random gathers are free of bank conflicts), then every index
-//               becomes a 16-bit codebook entry (4 E2M1 codes) and 16-byte chunks
-//               of FP4 are written straight into the swizzled K-major operand
-//               tile the tensor core reads.  PreScale+ scale indices become scale
-//               bytes in the tcgen05 scale-factor atom layout.  Then epilogue.
+//   warps 2..17 decoders (two groups of 8 warps on alternate stages for T <= 128,
+//               all 16 on every stage for T = 256): the stage's codebook is
+//               replicated once per lane (so the random gathers are free of bank
+//               conflicts), then every index becomes a 16-bit codebook entry (4
+//               E2M1 codes) and 16-byte chunks of FP4 are written straight into
+//               the swizzled K-major operand tile the tensor core reads.  PreScale+
+//               scale indices become scale bytes in the tcgen05 scale-factor atom
+//               layout; PostScale-QB atoms are filled with the QBlock's scale byte.
+//               Then epilogue.
 //   warp 1      one thread issues tcgen05.cp (scale atoms -> TMEM) and four
 //               tcgen05.mma block-scaled FP4 MMAs (K = 64 each) per stage into a
 //               128 x T FP32 accumulator in TMEM, and frees the stage with
 //               tcgen05.commit.
-//   epilogue    warps 2..5 read the accumulator with tcgen05.ld, apply the FP32
+//   epilogue    warps 2..17 read the accumulator with tcgen05.ld, apply the FP32
 //               tensor scales and store FP32/BF16 rows of Y.  For split-K (decode)
 //               the CTAs of one output tile form a thread-block cluster: ranks
 //               1.. write their partial tiles into rank 0's shared memory and
 //               rank 0 adds them in rank order (deterministic, no workspace).
 //
 // The weight tile is the MMA's A operand (M = 128 rows of W), the token tile is
-// the B operand (N = T tokens), so one kernel serves decode (T = 16) and
-// prefill (T = 128) without a transpose.
+// the B operand (N = T tokens), so one kernel serves the decode shapes the decode
+// GEMV does not take (T = 16) and prefill (T = 128 or 256) without a transpose.
 #pragma once
 
 #include "mxc_device.cuh"
