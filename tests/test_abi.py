@@ -161,3 +161,14 @@ def test_gpu_calls_reject_bad_arguments_synchronously(L):
     assert L.mxc_quantize_act(16, 4, 500, 512, 0, None, 16, 256, 16, None, 16, 256, None) == 3
     # quantize: E4M3 needs a tensor-scale output
     assert L.mxc_quantize_act(16, 4, 512, 512, 1, None, 16, 256, 16, None, 16, 256, None) == 1
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path, monkeypatch):
+    """No CPU or library fallback: without libmxc.so every call raises."""
+    monkeypatch.setattr(mxc, "_lib", None)
+    monkeypatch.setattr(mxc, "_LIB_PATH", str(tmp_path / "libmxc.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        mxc.lib()
+    w = synth.make_weight(1, "e8m0_b32", "prescale", 256, 512, 0, 0)
+    with pytest.raises(RuntimeError, match="missing"):
+        mxc.pack_weight_host(w)
