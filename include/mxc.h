@@ -84,8 +84,8 @@ typedef enum mxc_format {
 } mxc_format;
 
 /* MXCode strategies (abstract).  PostScale and PreScale share one decode path
- * (the pages' "shared Pre/PostScale FP4 projection backend", Figure 4 and
- * Table 3 captions); the strategy only selects where block scales come from. */
+ * (the Figure 4 and Table 3 captions describe a single FP4 projection backend
+ * serving both); the strategy only selects where block scales come from. */
 typedef enum mxc_strategy {
   MXC_POSTSCALE = 0,     /* direct block scales                                */
   MXC_PRESCALE = 1,      /* direct block scales                                */
@@ -226,10 +226,10 @@ mxc_status mxc_quantize_act_grouped(const void* x_bf16, int64_t M, int64_t K, in
                                     size_t ws_bytes, mxc_stream_t stream);
 
 /* MXCode W4A4 linear layer: y[M, N] = A[M, K] . W[N, K]^T, where A is the
- * MX-quantized activation and W the VQ weight reconstructed on the fly
- * (abstract: "reconstruct MX-native W4A4 operands without materializing
- * intermediate high-precision weights").  Accumulation is FP32 on the tensor
- * cores; y = acc * w_tscale * a_tscale, written as FP32 or BF16 (RNE).
+ * MX-quantized activation and W the VQ weight reconstructed on the fly (the
+ * abstract's point: the VQ storage becomes MX-native FP4 operands directly, with
+ * no high-precision copy of the weight in between).  Accumulation is FP32 on the
+ * tensor cores; y = acc * w_tscale * a_tscale, written as FP32 or BF16 (RNE).
  * a         activation, a->fmt must equal w->fmt; a->rows = M; a->sf in SF layout
  * w         packed VQ weight (device pointers inside)
  * y         device, [M, ldy] elements of y_dtype (ldy >= N)

@@ -1,8 +1,8 @@
 // mma_kernel.cuh -- the MXCode W4A4 linear layer on sm_100a tensor cores.
 //
-// "MXCode: Vector Quantization for MX-Native Inference at Scale" (abstract):
-// MX-native W4A4 operands are reconstructed from VQ storage "without
-// materializing intermediate high-precision weights".  Here every CTA owns a
+// "MXCode: Vector Quantization for MX-Native Inference at Scale" (abstract): the
+// VQ storage is turned directly into MX-native W4A4 operands, and no
+// high-precision copy of the weight is ever formed.  Here every CTA owns a
 // 128 (output channels) x T (tokens) tile of Y^T and runs a pipeline over K in
 // stages of 256 input channels:
 //
