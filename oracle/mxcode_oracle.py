@@ -27,7 +27,9 @@ What it computes, and where the method defines it
 * Storage accounting (Table 2 "Weight (BPE)" row; Figure 3 caption): indices +
   FP4 codebooks + scales (+ scale-VQ metadata), tensor scale excluded.
 
-Readings of points the pages leave open are listed in DESIGN.md ("Readings").
+Where the pages leave a point open (the activation recipe, nibble order, scale-VQ
+grouping, QBlock tiling, the PostScale storage), the function that decides it
+states the reading it takes in its docstring.
 Everything is FP64 except the FP32 steps of the E4M3 scale recipe, which are
 done in FP32 on purpose because the recipe is defined in FP32.
 
