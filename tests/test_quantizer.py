@@ -86,3 +86,9 @@ def test_quantized_weight_runs_through_the_gpu_path():
         assert mxc.get_device_error() == 0
         ref, sabs = O.w4a4_linear(x, w)
         assert np.all(np.abs(y - ref) <= 1e-4 * sabs)
+
+
+def test_command_line_report(capsys):
+    Q.main(["--n", "128", "--k", "256", "--qb", "128", "--iters", "2", "--strategy", "postscale_qb"])
+    out = capsys.readouterr().out
+    assert out.startswith("postscale_qb e4m3_b16 QBlock 128: SQNR") and "bits/weight" in out
