@@ -41,12 +41,26 @@ N_COPIES = 12
 
 
 def peaks():
+    """(HBM GB/s, its kind) from MEASURED_PEAKS.json, else the machine's fallback figure."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def fp4_peak(sustained: bool = False):
+    """Dense block-scaled FP4 tensor peak in TFLOP/s and how it was obtained: the
+    measured cuBLAS bf16 peak (burst, or sustained for a kernel timed inside a long
+    step) times 4, the nominal FP4 / BF16 dense ratio (9 / 2.25 PFLOP/s)."""
+    key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return 4.0 * float(p[key]), f"measured {key} x 4 (nominal FP4/BF16 ratio)"
+    except Exception:
+        return 4.0 * (1400.0 if sustained else 1590.0), "fallback bf16 x 4 (nominal FP4/BF16 ratio)"
 
 
 # ---------------------------------------------------------------------------
@@ -111,12 +125,46 @@ class ClockSampler:
 def oracle_sample(w, x, rows: slice):
     """The oracle on a slice of output channels: (seconds, weight bytes consumed, Y, sum |a w|)."""
     from oracle import mxcode_oracle as O
+    from vector_quantized_mx_b200 import synth
     t0 = time.perf_counter()
-    sub = type(w)(w.fmt, w.strategy, rows.stop - rows.start, w.K, w.qn, w.qk, w.idx[rows],
-                  w.cb[rows.start // w.qn:rows.stop // w.qn], w.scales[rows], None, None, w.w_tscale)
+    sub = synth.weight_rows(w, rows.start, rows.stop)
     ref, sabs = O.w4a4_linear(x, sub)
     dt = time.perf_counter() - t0
     return dt, O.storage_bytes(sub), ref, sabs
+
+
+def oracle_tile(w, x_rows, cols: slice, tscale=None):
+    """The oracle on a tile: the given activation rows (quantized with the tensor
+    scale of the whole activation, `tscale`) times the weight rows `cols`.
+    Returns (seconds, Y tile, sum |a w| tile)."""
+    from oracle import mxcode_oracle as O
+    from vector_quantized_mx_b200 import synth
+    t0 = time.perf_counter()
+    codes, sf, s = O.quantize_act(x_rows, w.fmt, tscale)
+    a_hat = O.dequant_act(codes, sf, w.fmt, s)
+    w_hat = O.dequant_weight(synth.weight_rows(w, cols.start, cols.stop))
+    ref, sabs = O.linear(a_hat, w_hat), O.abs_linear(a_hat, w_hat)
+    return time.perf_counter() - t0, ref, sabs
+
+
+def tile_baseline(w, x, tiles, y_gpu, budget_s, tscale=None):
+    """Times the oracle on (row-slice, column-slice) tiles of a layer until budget_s
+    seconds of CPU work; each tile is also compared with the GPU output (a NumPy
+    array, FP32 or BF16 as float): |gpu - oracle| <= 1e-4 * sum |a w| (+ BF16
+    rounding when y_gpu came from a BF16 output).  Returns (TFLOP/s, tiles, seconds)."""
+    t_tot, flops, n = 0.0, 0.0, 0
+    for r, c, bf16 in tiles:
+        dt, ref, sabs = oracle_tile(w, x[r], c, tscale)
+        got = np.asarray(y_gpu[r, c], dtype=np.float64)
+        bound = 1e-4 * sabs + (np.abs(ref) * 2.0 ** -8 if bf16 else 0.0)
+        if not np.all(np.abs(got - ref) <= bound):
+            raise SystemExit(f"bench: GPU tile rows {r} cols {c} does not match the oracle")
+        t_tot += dt
+        flops += 2.0 * (r.stop - r.start) * (c.stop - c.start) * w.K
+        n += 1
+        if t_tot >= budget_s:
+            break
+    return flops / t_tot / 1e12, n, t_tot
 
 
 def blas_threads():
@@ -333,6 +381,12 @@ def run_gpu(args, rank, world, dist):
         torch.cuda.synchronize()
     ms_e2e = max_over_ranks(s0.elapsed_time(s1) / steps, dist, dev)
 
+    extra = {}
+    with_cpu = not args.no_cpu_baseline and world == 1 and rank == 0
+    if "prefill" in args.legs:
+        extra["prefill"] = prefill_leg(dev, stream, capture, time_graph, steps, world, with_cpu)
+    if "moe" in args.legs:
+        extra["moe"] = moe_leg(dev, stream, capture, time_graph, steps, world, with_cpu)
     if rank != 0:
         return
     # our kernels per step: the activation quantizer (one launch up to 16 x 8192
@@ -369,7 +423,185 @@ def run_gpu(args, rank, world, dist):
     }
     if not args.no_cpu_baseline and world == 1:       # the oracle on the host: rank 0 at N=1 only
         out["cpu_baseline"] = cpu_baseline(w, x, y_ref.cpu().numpy())
+    if extra is not None:
+        out.update(extra)
     print(json.dumps(out), flush=True)
+
+
+def rotated(pw0, n):
+    """n packed copies of one weight (the same values in distinct buffers)."""
+    from vector_quantized_mx_b200 import mxc
+    cl = lambda t: None if t is None else t.clone()
+    return [pw0] + [mxc.PackedWeight(pw0.fmt, pw0.strategy, pw0.N, pw0.K, pw0.qn, pw0.qk, pw0.idx.clone(),
+                                     pw0.cb.clone(), cl(pw0.scales), cl(pw0.sidx), cl(pw0.scb), pw0.w_tscale)
+                    for _ in range(n - 1)]
+
+
+def prefill_leg(dev, stream, capture, time_graph, steps, world, with_cpu):
+    """Config 3: prefill GEMM, PreScale E8M0-B32, M=8192, K=4096, N=9216, 256x256
+    QBlocks, BF16 output.  One step = activation quantization + MXCode linear (decode
+    once into the workspace, then the native block-scaled GEMM).  The dominant kernel
+    is the GEMM; its duration is taken from the native linear on the decoded weight,
+    which launches exactly that kernel on the same operands."""
+    import torch
+    from vector_quantized_mx_b200 import mxc, synth
+    w, x = synth.config3()
+    M, N, K = x.shape[0], w.N, w.K
+    copies = rotated(mxc.pack_weight(w, device=dev), N_COPIES)
+    x_dev = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+    act = mxc.empty_act(M, K, w.fmt, dev)
+    qws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    lws = mxc.linear_workspace(M, N, K, w.fmt, dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.stream(stream):
+        nat0 = mxc.decode_weight(copies[0], stream=stream)
+        nats = [nat0] + [mxc.MXTensor(nat0.q.clone(), nat0.sf.clone(), nat0.tscale.clone(), N, K, w.fmt)
+                         for _ in range(N_COPIES - 1)]
+        mxc.quantize_act(x_dev, w.fmt, out=act, ws=qws, stream=stream)
+        mxc.linear(act, copies[0], y=y, ws=lws, stream=stream)
+        yn = mxc.native_linear(act, nats[0], out_dtype=torch.bfloat16, ws=lws, stream=stream)
+    stream.synchronize()
+    if mxc.get_device_error(stream) != 0:
+        raise SystemExit("bench: the prefill step failed")
+    same = bool(torch.equal(y, yn))
+
+    def step(i):
+        mxc.quantize_act(x_dev, w.fmt, out=act, ws=qws, stream=stream)
+        mxc.linear(act, copies[i % N_COPIES], y=y, ws=lws, stream=stream)
+
+    def lin(i):
+        mxc.linear(act, copies[i % N_COPIES], y=y, ws=lws, stream=stream)
+
+    def nat_lin(i):
+        mxc.native_linear(act, nats[i % N_COPIES], y=yn, ws=lws, stream=stream)
+
+    def nat_step(i):
+        mxc.quantize_act(x_dev, w.fmt, out=act, ws=qws, stream=stream)
+        mxc.native_linear(act, nats[i % N_COPIES], y=yn, ws=lws, stream=stream)
+    n = max(10, steps // 4)
+    ms = {name: time_graph(capture(n, fn)) / n for name, fn in
+          (("step", step), ("linear", lin), ("native_linear", nat_lin), ("native_step", nat_step))}
+    flops = 2.0 * M * N * K
+    peak, peak_kind = fp4_peak()
+    wbytes = copies[0].storage_bytes()
+    out = {"workload": "prefill GEMM: PreScale E8M0-B32-FP4, M=8192, K=4096, N=9216, 256x256 QBlocks, BF16 out",
+           "ms_per_step": ms["step"], "ms_linear": ms["linear"],
+           "tflops": world * flops / (ms["linear"] * 1e-3) / 1e12,
+           "tflops_step": world * flops / (ms["step"] * 1e-3) / 1e12,
+           "weight_GBps": world * wbytes / (ms["linear"] * 1e-3) / 1e9,
+           "roofline": {"bound": "tensor", "unit": "TFLOP/s", "peak": peak, "peak_kind": peak_kind,
+                        "kernel": "gemm_kernel<E8M0, native, T=256> (the GEMM of the decode-once path)",
+                        "ms_per_launch": ms["native_linear"], "flops_per_launch": flops,
+                        "achieved": flops / (ms["native_linear"] * 1e-3) / 1e12,
+                        "frac": flops / (ms["native_linear"] * 1e-3) / 1e12 / peak,
+                        "layer_frac": flops / (ms["linear"] * 1e-3) / 1e12 / peak, "traffic": None},
+           "native_fp4": {"ms_linear": ms["native_linear"], "ms_per_step": ms["native_step"],
+                          "mxcode_speedup": ms["native_linear"] / ms["linear"],
+                          "mxcode_step_speedup": ms["native_step"] / ms["step"],
+                          "bitwise_equal_outputs": same},
+           "gpu_launches_per_step": 3, "l2": f"rotating {N_COPIES} weight copies; 151 MB BF16 output per step"}
+    if with_cpu:
+        yh = y.float().cpu().numpy()
+        rng = np.random.default_rng(3)
+        tiles = []
+        for _ in range(8):
+            r0, c0 = int(rng.integers(0, M // 256)) * 256, int(rng.integers(0, N // 256)) * 256
+            tiles.append((slice(r0, r0 + 256), slice(c0, c0 + 256), True))
+        v, nt, t = tile_baseline(w, x, tiles, yh, budget_s=8.0)
+        out["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                               "sample": f"{nt} seeded 256x256 output tiles (K=4096) of the prefill layer, "
+                                         f"each compared with the GPU output, {t:.1f} s"}
+    return out
+
+
+def moe_leg(dev, stream, capture, time_graph, steps, world, with_cpu):
+    """Config 4: MoE, PreScale+ E4M3-B16, 128 experts with gate/up [3072, 4096] and
+    down [4096, 1536], 2048 tokens routed top-8 by Zipf(1.1) = 16384 expert-sorted
+    rows, BF16 outputs.  One step = grouped quantization + MXCode grouped linear,
+    for gate/up and then for down (whose input is synthetic: the SwiGLU between the
+    two is not part of the layer).  Roofline per projection: the aggregate bound
+    max(compressed weight bytes / HBM, flops / FP4 peak)."""
+    import torch
+    from vector_quantized_mx_b200 import mxc, synth
+    row_tok, off = synth.config4_routing()
+    E = synth.MOE_EXPERTS
+    offd = torch.from_numpy(off.astype(np.int32)).to(dev)
+    M = int(off[-1])
+    proj = {}
+    for name in ("gate_up", "down"):
+        x = synth.config4_activations(name, row_tok)
+        ws = [synth.config4_expert(e, name) for e in range(E)]
+        packed = [mxc.pack_weight(w, device=dev) for w in ws]
+        K, N = ws[0].K, ws[0].N
+        proj[name] = {"x": x, "w": ws, "packed": packed, "K": K, "N": N,
+                      "x_dev": torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev),
+                      "act": mxc.empty_act_grouped(M, K, E, "e4m3_b16", dev),
+                      "qws": torch.zeros(256 + 4 * (E + 1), dtype=torch.uint8, device=dev),
+                      "mws": torch.zeros(max(16, mxc.lib().mxc_moe_workspace_bytes(M, E, N, K, 1)),
+                                         dtype=torch.uint8, device=dev),
+                      "y": torch.empty((M, N), dtype=torch.bfloat16, device=dev),
+                      "bytes": sum(p.storage_bytes() for p in packed), "flops": 2.0 * M * N * K}
+
+    def quant(p):
+        mxc.quantize_act_grouped(p["x_dev"], "e4m3_b16", offd, out=p["act"], ws=p["qws"], stream=stream)
+
+    def moe(p):
+        mxc.moe_linear(p["act"], offd, p["packed"], y=p["y"], ws=p["mws"], stream=stream)
+
+    with torch.cuda.stream(stream):
+        for p in proj.values():
+            quant(p)
+            moe(p)
+    stream.synchronize()
+    if mxc.get_device_error(stream) != 0:
+        raise SystemExit("bench: the MoE step failed")
+
+    def step(i):
+        for p in proj.values():
+            quant(p)
+            moe(p)
+    n = max(5, steps // 8)
+    ms_step = time_graph(capture(n, step)) / n
+    hbm, hbm_kind = peaks()
+    peak, peak_kind = fp4_peak()
+    out = {"workload": "MoE: PreScale+ E4M3-B16-FP4, 128 experts (gate/up 3072x4096, down 4096x1536), "
+                       "2048 tokens top-8 Zipf(1.1) = 16384 rows, 256x256 QBlocks, BF16 out",
+           "ms_per_step": ms_step, "rows": M, "gpu_launches_per_step": 4 * 2}
+    for name, p in proj.items():
+        n_l = max(5, steps // 8)
+        ms_lin = time_graph(capture(n_l, lambda i, p=p: moe(p))) / n_l
+        t_bw = p["bytes"] / (hbm * 1e9) * 1e3
+        t_fl = p["flops"] / (peak * 1e12) * 1e3
+        out[name] = {"ms_linear": ms_lin, "tflops": world * p["flops"] / (ms_lin * 1e-3) / 1e12,
+                     "weight_GBps": world * p["bytes"] / (ms_lin * 1e-3) / 1e9, "weight_bytes": p["bytes"],
+                     "roofline": {"bound": "hbm" if t_bw >= t_fl else "tensor",
+                                  "kernel": "gemm_kernel<E4M3, VQ scale-VQ, T=128, MoE> + group prologue",
+                                  "target_ms": max(t_bw, t_fl), "frac": max(t_bw, t_fl) / ms_lin,
+                                  "hbm_peak_GBps": hbm, "hbm_kind": hbm_kind,
+                                  "fp4_peak_TFLOPs": peak, "fp4_kind": peak_kind, "traffic": None}}
+    if with_cpu:
+        from oracle import mxcode_oracle as O
+        counts = np.diff(off)
+        p = proj["gate_up"]
+        yh = p["y"].float().cpu().numpy()
+        s = O.tensor_scale_e4m3(p["x"])
+        t_tot, flops, nt = 0.0, 0.0, 0
+        for e in [int(counts.argmax()), 0, 17, 64, 127]:
+            r0, r1 = int(off[e]), min(int(off[e + 1]), int(off[e]) + 128)
+            if r1 <= r0:
+                continue
+            dt, ref, sabs = oracle_tile(p["w"][e], p["x"][r0:r1], slice(1024, 1280), s)
+            got = yh[r0:r1, 1024:1280]
+            if not np.all(np.abs(got - ref) <= 1e-4 * sabs + np.abs(ref) * 2.0 ** -8):
+                raise SystemExit(f"bench: MoE expert {e} does not match the oracle")
+            t_tot += dt
+            flops += 2.0 * (r1 - r0) * 256 * p["K"]
+            nt += 1
+        out["cpu_baseline"] = {"value": flops / t_tot / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+                               "kind": "oracle",
+                               "sample": f"{nt} expert tiles (<=128 rows x 256 columns, K=4096) of gate/up, "
+                                         f"each compared with the GPU output, {t_tot:.1f} s"}
+    return out
 
 
 def main():
@@ -380,6 +612,8 @@ def main():
     ap.add_argument("--impl", default="mxcode", choices=["mxcode", "reference"])
     ap.add_argument("--m", type=int, default=16, choices=[1, 4, 16])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--legs", default="prefill,moe",
+                    help="extra workloads timed after the decode line: prefill (config 3), moe (config 4)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))

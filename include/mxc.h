@@ -249,13 +249,21 @@ mxc_status mxc_native_linear(const mxc_mx_tensor* a, const mxc_mx_tensor* w, voi
                              mxc_dtype y_dtype, void* ws, size_t ws_bytes, mxc_stream_t stream);
 
 /* Grouped-expert (MoE) MXCode linear: rows of `a` are sorted by expert, expert e
- * owning rows [d_offsets[e], d_offsets[e+1]); y[r, :] = A[r, :] . W_e^T.
+ * owning rows [d_offsets[e], d_offsets[e+1]); y[r, :] = A[r, :] . W_e^T.  The
+ * weights are MoE expert tensors, as in the paper's evaluation (Table 4 caption:
+ * the VQ-coded tensors are the experts of Qwen3's MoE layers); every expert is a
+ * VQ weight of the same shape and coding.
  * a         quantized with mxc_quantize_act_grouped (grouped SF layout)
  * d_offsets device int32 [E+1] (validated on the device)
  * experts   host array of E packed weights that share strategy, format, N, K,
- *           qn, qk (their device pointers may differ); E <= 256
+ *           qn, qk (their device pointers may differ); E <= 256, larger E
+ *           returns MXC_ERR_UNSUPPORTED
  * y         device, [M, ldy]
- * ws        device workspace of mxc_moe_workspace_bytes() bytes */
+ * ws        device workspace of mxc_moe_workspace_bytes() bytes
+ * Checks, in this order: the activation (INVALID_ARG / ALIGNMENT / UNSUPPORTED),
+ * null pointers and E <= 0 (INVALID_ARG), E > 256 (UNSUPPORTED), each expert
+ * weight, consistency with the activation, the output, then the device
+ * (NO_DEVICE) and the workspace (WORKSPACE). */
 mxc_status mxc_moe_linear(const mxc_mx_tensor* a, const int32_t* d_offsets, const mxc_weight* experts,
                           int32_t E, void* y, int64_t ldy, mxc_dtype y_dtype, void* ws,
                           size_t ws_bytes, mxc_stream_t stream);
@@ -265,11 +273,13 @@ mxc_status mxc_moe_linear(const mxc_mx_tensor* a, const int32_t* d_offsets, cons
  * that forbid allocator calls, or C callers with no device allocator at hand.
  * The paper has no counterpart to this entry point; it exists for the calling
  * environment only.  It takes the same arguments as mxc_moe_linear minus the
- * workspace, and runs the same kernels.
+ * workspace, checks them in the same order with the same statuses, and runs
+ * the same kernels, so its output is bit-identical to mxc_moe_linear's.
  * Scratch: the per-call expert tile table lives in a fixed module-global array
- * in device memory, held by every GPU that loads the library until the process
- * exits.  Limit: E <= 256 experts; larger E returns MXC_ERR_UNSUPPORTED and
- * enqueues nothing.
+ * of 1280 bytes in device memory (room for the largest table, E = 256 experts),
+ * held by every GPU that loads the library until the process exits.  Limit:
+ * E <= 256 experts, as for mxc_moe_linear; larger E returns MXC_ERR_UNSUPPORTED
+ * and enqueues nothing.
  * The first call on each device looks up that array's device address (no
  * allocation); make the first call on a device before any stream capture that
  * includes this entry point.  Every call rewrites the table before reading it,
@@ -287,6 +297,16 @@ mxc_status mxc_moe_linear_noalloc(const mxc_mx_tensor* a, const int32_t* d_offse
  * hold exactly the same values. */
 mxc_status mxc_decode_weight(const mxc_weight* w, uint8_t* q_out, int64_t ldq, uint8_t* sf_out,
                              mxc_stream_t stream);
+
+/* Self-test of the device timeout path (test infrastructure; the paper has no
+ * counterpart).  Enqueues one tiny kernel whose single bounded pipeline wait --
+ * the same wait every kernel of this library uses -- is on a barrier that nothing
+ * completes, with a limit of limit_cycles SM clocks (1 .. 2e9) instead of the
+ * pipelines' two billion.  The wait runs out, the kernel records MXC_ERR_TIMEOUT
+ * in the device error word and returns normally: no fault, no hang, nothing left
+ * in flight, the context stays usable.  mxc_get_device_error() then returns
+ * MXC_ERR_TIMEOUT.  Returns MXC_ERR_INVALID_ARG for a limit out of range. */
+mxc_status mxc_selftest_wait_timeout(int64_t limit_cycles, mxc_stream_t stream);
 
 /* Waits for the stream, then reads and clears the device error word of the
  * current device: MXC_OK, MXC_ERR_DEVICE_INVALID or MXC_ERR_TIMEOUT. */

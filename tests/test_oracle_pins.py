@@ -315,6 +315,107 @@ def test_w4a4_linear_exact_rationals_tiny():
             assert abs(Fraction(float(y[m, n])) - exact) <= Fraction(2) ** -45 * max(1, abs(exact))
 
 
+# ---------------------------------------------------------------------------
+# The FP32 tensor scale of E4M3-B16 (Table 1: E4M3 block scales per 16 elements
+# with an FP32 tensor scale): it multiplies every reconstructed activation and
+# weight exactly once.  Each check below is computed without the oracle's
+# dequant_* functions, from codes, scale bytes and tensor scales; a mutant of the
+# oracle that drops, inverts or squares the factor must fail them.
+# ---------------------------------------------------------------------------
+
+_E4M3_ONE = 0x38                     # E4M3 byte of 1.0 (exponent 7 = bias, mantissa 0)
+_TWICE_E2M1 = np.array([0, 1, 2, 3, 4, 6, 8, 12], dtype=np.int64)   # 2 x E2M1 magnitude
+
+
+def _twice(codes):
+    c = np.asarray(codes).astype(np.int64)
+    return np.where(c & 8, -_TWICE_E2M1[c & 7], _TWICE_E2M1[c & 7])
+
+
+def _e4m3_tscale_case(seed, M=12, N=24, K=256):
+    """E4M3-B16 weight and activation codes, random positive block scales."""
+    rng = np.random.default_rng(seed)
+    ca = rng.integers(0, 16, size=(M, K), dtype=np.uint8)
+    cw = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    sa = rng.integers(0x20, 0x50, size=(M, K // 16), dtype=np.uint8)
+    sw = rng.integers(0x20, 0x50, size=(N, K // 16), dtype=np.uint8)
+    idx, cb = _encode_vq(cw, 8, 64)
+    return ca, cw, sa, sw, idx, cb
+
+
+def _tensor_scale_pins_hold(O_mod) -> bool:
+    """True when O_mod's reconstruction applies both FP32 tensor scales exactly once."""
+    M, N, K = 12, 24, 256
+    # (1) unit block scales, power-of-two tensor scales 2^-3 (weight), 2^-5 (activation):
+    #     2a and 2w are integers, so 4 * 2^8 * Y equals an exact int64 matmul
+    ca, cw, _, _, idx, cb = _e4m3_tscale_case(21, M, N, K)
+    one_a = np.full((M, K // 16), _E4M3_ONE, np.uint8)
+    one_w = np.full((N, K // 16), _E4M3_ONE, np.uint8)
+    w = synth.VQWeight("e4m3_b16", "prescale", N, K, 8, 64, idx, cb, one_w, None, None, 2.0 ** -3)
+    y = O_mod.linear(O_mod.dequant_act(ca, one_a, "e4m3_b16", 2.0 ** -5), O_mod.dequant_weight(w))
+    exact = _twice(ca) @ _twice(cw).T
+    if not np.array_equal(4.0 * 2.0 ** 8 * y, exact.astype(np.float64)):
+        return False
+    # (2) random E4M3 block scales and non-power-of-two FP32 tensor scales: Y equals the
+    #     exact rational sum of code x block scale x tensor scale products (block scales
+    #     decoded by torch's float8_e4m3fn cast, not by the oracle)
+    ca, cw, sa, sw, idx, cb = _e4m3_tscale_case(22, M, N, K)
+    ts_w = float(np.float32(1.0) / np.float32(2688.0))
+    ts_a = float(np.float32(0.0123))
+    w = synth.VQWeight("e4m3_b16", "prescale", N, K, 8, 64, idx, cb, sw, None, None, ts_w)
+    y = O_mod.linear(O_mod.dequant_act(ca, sa, "e4m3_b16", ts_a), O_mod.dequant_weight(w))
+    dec = lambda b: torch.from_numpy(np.ascontiguousarray(b)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    va, vw = dec(sa), dec(sw)
+    ia, iw = _twice(ca), _twice(cw)
+    fa, fw = Fraction(ts_a), Fraction(ts_w)
+    rng = np.random.default_rng(23)
+    for _ in range(40):
+        m, n = int(rng.integers(M)), int(rng.integers(N))
+        ex = sum(Fraction(int(ia[m, k])) / 2 * Fraction(float(va[m, k // 16])) * fa *
+                 Fraction(int(iw[n, k])) / 2 * Fraction(float(vw[n, k // 16])) * fw for k in range(K))
+        if abs(Fraction(float(y[m, n])) - ex) > Fraction(2) ** -44 * max(abs(ex), Fraction(2) ** -200):
+            return False
+    return True
+
+
+def test_tensor_scales_enter_exactly_once():
+    assert _tensor_scale_pins_hold(O)
+
+
+@pytest.mark.parametrize("mutant", ["drop", "invert", "square", "drop_weight"])
+def test_tensor_scale_pins_catch_mutants(mutant):
+    """The same pins on a copy of the oracle with a planted mistake in the tensor
+    scale (on the CPU, in the oracle only): each mutant must fail them."""
+    import types
+
+    def dequant_act(codes, sf, fmt, tscale):
+        B = O.BLOCK[fmt]
+        S = np.repeat(O.scale_value(sf, fmt), B, axis=1)
+        t = {"drop": 1.0, "invert": 1.0 / float(tscale), "square": float(tscale) ** 2,
+             "drop_weight": float(tscale)}[mutant]
+        return O.e2m1_value(codes) * S * t
+
+    def dequant_weight(w):
+        ts = 1.0 if mutant == "drop_weight" else w.w_tscale
+        return dequant_act(O.weight_codes(w), O.weight_scale_bytes(w), w.fmt, ts)
+
+    M_ = types.SimpleNamespace(linear=O.linear, dequant_act=dequant_act, dequant_weight=dequant_weight)
+    assert not _tensor_scale_pins_hold(M_)
+
+
+def test_w4a4_linear_scales_with_the_activation_tensor_scale():
+    """E4M3-B16 end to end: multiplying the activation by 2^j multiplies its FP32
+    tensor scale amax/2688 by 2^j and leaves every block scale byte and code alone,
+    so the layer's output must scale by exactly 2^j (once, not squared or inverted)."""
+    rng = np.random.default_rng(31)
+    x = rng.normal(size=(6, 128))
+    w = synth.make_weight(124, "e4m3_b16", "prescale", 16, 128, 0, 0)
+    y0, _ = O.w4a4_linear(bf16_bits(x), w)
+    for j in (-3, 5):
+        yj, _ = O.w4a4_linear(bf16_bits(x * 2.0 ** j), w)
+        assert np.array_equal(yj, y0 * 2.0 ** j)
+
+
 def test_checksums_linearity():
     rng = np.random.default_rng(2)
     a = rng.normal(size=(33, 70))

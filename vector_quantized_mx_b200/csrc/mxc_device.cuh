@@ -73,20 +73,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity to complete.  Returns false
-// (and records MXC_ERR_TIMEOUT) if it does not complete within kWaitLimitCycles.
+// (and records MXC_ERR_TIMEOUT) if it does not complete within `limit` SM clocks.
 // Between polls the thread backs off briefly, so that many waiting threads do not
 // keep the shared-memory pipe busy with barrier polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     __nanosleep(32);
     if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       set_device_error(MXC_ERR_TIMEOUT);
       return false;
     }
   }
+}
+
+// The pipelines' wait: bounded by kWaitLimitCycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_limit(bar, parity, kWaitLimitCycles);
 }
 
 // ------------------------------------------------------------------------------------

@@ -109,6 +109,18 @@ inline size_t sf_off_host(int64_t r, int64_t kb, int64_t kb_per_row) {
          (kb % 4);
 }
 
+// Runs the pipelines' bounded mbarrier wait on a barrier that nothing arrives
+// at: the wait gives up after `limit` clocks, records MXC_ERR_TIMEOUT and the
+// kernel returns (nothing is in flight).
+__global__ void wait_timeout_probe_kernel(long long limit) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait_limit(&bar, 0, limit);
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -341,8 +353,9 @@ mxc_status mxc_native_linear(const mxc_mx_tensor* a, const mxc_mx_tensor* w, voi
   return run_linear(L, reinterpret_cast<cudaStream_t>(stream));
 }
 
-mxc_status mxc_moe_linear(const mxc_mx_tensor* a, const int32_t* d_offsets, const mxc_weight* experts, int32_t E,
-                          void* y, int64_t ldy, mxc_dtype y_dtype, void* ws, size_t ws_bytes, mxc_stream_t stream) {
+// Argument checks shared by both grouped entry points, in one order of precedence.
+static mxc_status moe_prepare(const mxc_mx_tensor* a, const int32_t* d_offsets, const mxc_weight* experts, int32_t E,
+                              void* y, int64_t ldy, mxc_dtype y_dtype, MoeArgs* m) {
   mxc_status s = check_mx_tensor(a);
   if (s != MXC_OK) return s;
   if (!d_offsets || !experts || E <= 0) return MXC_ERR_INVALID_ARG;
@@ -360,22 +373,30 @@ mxc_status mxc_moe_linear(const mxc_mx_tensor* a, const int32_t* d_offsets, cons
   const mxc_weight& w0 = experts[0];
   if (a->fmt != w0.fmt || a->K != w0.K) return MXC_ERR_INVALID_ARG;
   if ((s = check_output(y, ldy, w0.N, y_dtype)) != MXC_OK) return s;
+  *m = MoeArgs{};
+  fill_activation(m->base, a);
+  m->base.wsrc = wsrc_of(w0.strategy);
+  m->base.N = w0.N;
+  m->base.qn = qn;
+  m->base.qk = qk;
+  m->base.y = y;
+  m->base.ldy = ldy;
+  m->base.out_bf16 = y_dtype == MXC_OUT_BF16;
+  m->offsets = d_offsets;
+  m->E = E;
+  m->experts = experts;
+  return MXC_OK;
+}
+
+mxc_status mxc_moe_linear(const mxc_mx_tensor* a, const int32_t* d_offsets, const mxc_weight* experts, int32_t E,
+                          void* y, int64_t ldy, mxc_dtype y_dtype, void* ws, size_t ws_bytes, mxc_stream_t stream) {
+  MoeArgs m;
+  mxc_status s = moe_prepare(a, d_offsets, experts, E, y, ldy, y_dtype, &m);
+  if (s != MXC_OK) return s;
   if (a->rows == 0) return MXC_OK;
   if ((s = check_device()) != MXC_OK) return s;
-  MoeArgs m{};
-  fill_activation(m.base, a);
-  m.base.wsrc = wsrc_of(w0.strategy);
-  m.base.N = w0.N;
-  m.base.qn = qn;
-  m.base.qk = qk;
-  m.base.y = y;
-  m.base.ldy = ldy;
-  m.base.out_bf16 = y_dtype == MXC_OUT_BF16;
   m.base.ws = ws;
   m.base.ws_bytes = ws_bytes;
-  m.offsets = d_offsets;
-  m.E = E;
-  m.experts = experts;
   return run_moe_linear(m, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -387,8 +408,10 @@ mxc_status mxc_moe_linear(const mxc_mx_tensor* a, const int32_t* d_offsets, cons
 // ------------------------------------------------------------------------------------
 namespace {
 
-constexpr int kNoallocScratchInts = kMaxGroups + 1;   // largest table: 256 experts
-static __device__ __align__(256) int32_t g_moe_noalloc_scratch[kNoallocScratchInts];
+// The largest table the grouped kernels use (256 experts), in whole 256-byte units,
+// exactly the workspace size mxc_moe_workspace_bytes reports for 256 experts.
+constexpr size_t kNoallocScratchBytes = (static_cast<size_t>(kMaxGroups + 1) * sizeof(int32_t) + 255) / 256 * 256;
+static __device__ __align__(256) int32_t g_moe_noalloc_scratch[kNoallocScratchBytes / sizeof(int32_t)];
 
 constexpr int kMaxDevices = 64;
 std::atomic<int32_t*> g_noalloc_ptr[kMaxDevices];
@@ -415,14 +438,18 @@ extern "C" {
 
 mxc_status mxc_moe_linear_noalloc(const mxc_mx_tensor* a, const int32_t* d_offsets, const mxc_weight* experts,
                                   int32_t E, void* y, int64_t ldy, mxc_dtype y_dtype, mxc_stream_t stream) {
-  if (E > kNoallocScratchInts - 1) return MXC_ERR_UNSUPPORTED;
-  if (!a || !d_offsets || !experts || E <= 0) return MXC_ERR_INVALID_ARG;
-  mxc_status s = check_device();
+  MoeArgs m;
+  mxc_status s = moe_prepare(a, d_offsets, experts, E, y, ldy, y_dtype, &m);
   if (s != MXC_OK) return s;
+  if (a->rows == 0) return MXC_OK;
+  if ((s = check_device()) != MXC_OK) return s;
+  const size_t need = mxc_moe_workspace_bytes(a->rows, E, m.base.N, m.base.K, a->fmt);
+  if (need > kNoallocScratchBytes) return MXC_ERR_UNSUPPORTED;   // cannot happen for E <= 256
   int32_t* scratch = nullptr;
   if ((s = noalloc_scratch(&scratch)) != MXC_OK) return s;
-  return mxc_moe_linear(a, d_offsets, experts, E, y, ldy, y_dtype, scratch,
-                        sizeof(int32_t) * kNoallocScratchInts, stream);
+  m.base.ws = scratch;
+  m.base.ws_bytes = kNoallocScratchBytes;
+  return run_moe_linear(m, reinterpret_cast<cudaStream_t>(stream));
 }
 
 mxc_status mxc_decode_weight(const mxc_weight* w, uint8_t* q_out, int64_t ldq, uint8_t* sf_out, mxc_stream_t stream) {
@@ -448,6 +475,14 @@ mxc_status mxc_decode_weight(const mxc_weight* w, uint8_t* q_out, int64_t ldq, u
   d.ldq = ldq;
   d.sf_out = sf_out;
   return run_decode_weight(d, reinterpret_cast<cudaStream_t>(stream));
+}
+
+mxc_status mxc_selftest_wait_timeout(int64_t limit_cycles, mxc_stream_t stream) {
+  if (limit_cycles < 1 || limit_cycles > kWaitLimitCycles) return MXC_ERR_INVALID_ARG;
+  mxc_status s = check_device();
+  if (s != MXC_OK) return s;
+  wait_timeout_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_cycles);
+  return cudaGetLastError() == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
 }
 
 mxc_status mxc_get_device_error(mxc_stream_t stream) {

@@ -31,6 +31,7 @@ EXPORTED = (
     "mxc_quantize_act_workspace_bytes", "mxc_linear_workspace_bytes", "mxc_moe_workspace_bytes",
     "mxc_grouped_sf_rows_bound", "mxc_quantize_act", "mxc_quantize_act_grouped", "mxc_linear",
     "mxc_native_linear", "mxc_moe_linear", "mxc_moe_linear_noalloc", "mxc_decode_weight", "mxc_get_device_error",
+    "mxc_selftest_wait_timeout",
 )
 
 
@@ -95,6 +96,7 @@ def lib() -> ctypes.CDLL:
                                                       vp, i64, ctypes.c_int, vp]),
             "mxc_decode_weight": (ctypes.c_int, [ctypes.POINTER(_Weight), vp, i64, vp, vp]),
             "mxc_get_device_error": (ctypes.c_int, [vp]),
+            "mxc_selftest_wait_timeout": (ctypes.c_int, [i64, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -165,23 +167,32 @@ def quantize_act(x: torch.Tensor, fmt: str, tscale_in: Optional[torch.Tensor] = 
     return out
 
 
-def quantize_act_grouped(x: torch.Tensor, fmt: str, offsets: torch.Tensor, tscale_in=None, stream=None) -> MXTensor:
+def empty_act_grouped(M: int, K: int, E: int, fmt: str, device) -> MXTensor:
+    """Output buffers for quantize_act_grouped (grouped SF layout, padding zeroed)."""
+    rows_sf = lib().mxc_grouped_sf_rows_bound(M, E)
+    q = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+    sf = torch.zeros((max(1, sf_bytes(rows_sf, K, fmt)),), dtype=torch.uint8, device=device)
+    ts = torch.empty((1,), dtype=torch.float32, device=device) if fmt == "e4m3_b16" else None
+    return MXTensor(q, sf, ts, M, K, fmt)
+
+
+def quantize_act_grouped(x: torch.Tensor, fmt: str, offsets: torch.Tensor, tscale_in=None,
+                         out: Optional[MXTensor] = None, ws: Optional[torch.Tensor] = None,
+                         stream=None) -> MXTensor:
     """mxc_quantize_act_grouped: rows sorted by group, offsets int32 [E+1] on the device."""
     assert x.dtype == torch.bfloat16 and offsets.dtype == torch.int32
     M, K = x.shape
     E = offsets.numel() - 1
     dev = x.device
-    rows_sf = lib().mxc_grouped_sf_rows_bound(M, E)
-    q = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
-    sf = torch.zeros((max(1, sf_bytes(rows_sf, K, fmt)),), dtype=torch.uint8, device=dev)
-    ts = torch.empty((1,), dtype=torch.float32, device=dev) if fmt == "e4m3_b16" else None
-    ws = torch.empty((lib().mxc_quantize_act_workspace_bytes(M, K, FMT[fmt]) + 4 * (E + 1),), dtype=torch.uint8,
-                     device=dev)
+    out = empty_act_grouped(M, K, E, fmt, dev) if out is None else out
+    if ws is None:
+        ws = torch.empty((lib().mxc_quantize_act_workspace_bytes(M, K, FMT[fmt]) + 4 * (E + 1),),
+                         dtype=torch.uint8, device=dev)
     _check(lib().mxc_quantize_act_grouped(x.data_ptr(), M, K, x.stride(0), FMT[fmt], offsets.data_ptr(), E,
-                                          _ptr(tscale_in), q.data_ptr(), K // 2, sf.data_ptr(), _ptr(ts),
-                                          ws.data_ptr(), ws.numel(), _stream(stream)),
+                                          _ptr(tscale_in), out.q.data_ptr(), out.q.stride(0), out.sf.data_ptr(),
+                                          _ptr(out.tscale), ws.data_ptr(), ws.numel(), _stream(stream)),
            "mxc_quantize_act_grouped")
-    return MXTensor(q, sf, ts, M, K, fmt)
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -336,6 +347,11 @@ def decode_weight(w: PackedWeight, stream=None) -> MXTensor:
            "mxc_decode_weight")
     ts = torch.tensor([w.w_tscale], dtype=torch.float32, device=dev)
     return MXTensor(q, sf, ts, w.N, w.K, w.fmt)
+
+
+def selftest_wait_timeout(limit_cycles: int, stream=None) -> None:
+    """mxc_selftest_wait_timeout: a bounded device wait that is made to run out."""
+    _check(lib().mxc_selftest_wait_timeout(limit_cycles, _stream(stream)), "mxc_selftest_wait_timeout")
 
 
 def get_device_error(stream=None) -> int:

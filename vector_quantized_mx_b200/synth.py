@@ -150,6 +150,23 @@ class VQWeight:
         return BLOCK[self.fmt]
 
 
+def weight_rows(w: "VQWeight", r0: int, r1: int) -> "VQWeight":
+    """Rows [r0, r1) of a logical VQ weight as a weight of their own (array slicing
+    only).  Either r0 is a multiple of qn or the range lies inside one QBlock row,
+    so QBlock row (r0 + i) // qn of the whole weight is row i // qn of the slice."""
+    assert r0 % w.qn == 0 or r0 // w.qn == (r1 - 1) // w.qn
+    q0, q1 = r0 // w.qn, (r1 - 1) // w.qn + 1
+    scales = sidx = None
+    if w.strategy == POSTSCALE_QB:
+        scales = w.scales[q0:q1]
+    elif w.strategy == PRESCALE_PLUS:
+        sidx = w.sidx[r0:r1]
+    else:
+        scales = w.scales[r0:r1]
+    return VQWeight(w.fmt, w.strategy, r1 - r0, w.K, w.qn, w.qk, w.idx[r0:r1], w.cb[q0:q1], scales, sidx, w.scb,
+                    w.w_tscale)
+
+
 TSCALE_E4M3 = float(np.float32(1.0) / np.float32(2688.0))
 
 
