@@ -198,20 +198,38 @@ __global__ void __maxnreg__(64)
     prefetch_tensormap(&tmap_x);
     if constexpr (WSRC == WSRC_NATIVE) prefetch_tensormap(&tmap_wq);
     if constexpr (L::kVQ) prefetch_tensormap(&tmap_idx);
-    // this CTA's weight stream into L2: codebooks and scales first, then the bulk
+    // The weight stream, requested at once and in the order it is consumed (nothing
+    // here waits for the rest of the CTA or the cluster: the copies land in this CTA's
+    // own shared memory on barriers initialised above).  Codebooks, index quarter 0 of
+    // every stage, the weight scales and quarter 1 go straight to shared memory;
+    // quarters 2 and 3, whose buffers free up only as quarters 0 and 1 are decoded,
+    // go to L2 now and are copied in later.  (A plain L2 prefetch of the slice in
+    // address order would complete quarter 0 -- spread over all stages -- only when
+    // nearly the whole slice had arrived, and the decode could not overlap it.)
     if constexpr (L::kVQ) {
-      l2_prefetch_bulk(w_cb + static_cast<size_t>(qb0) * 256, static_cast<uint32_t>(qb1 - qb0 + 1) * 512);
+      const uint32_t cb_bytes = static_cast<uint32_t>(qb1 - qb0 + 1) * 512;
+      mbar_arrive_expect_tx(bar_cb, cb_bytes);
+      bulk_load(smem + L::CB_OFF, w_cb + static_cast<size_t>(qb0) * 256, cb_bytes, bar_cb);
+      // quarter j of stages [ks_begin, ks_begin + ks_per_split): box {2048 B, 1, stages, 1};
+      // stages past K (last split) arrive zero-filled and are not used
+      mbar_arrive_expect_tx(&full[0], p.ks_per_split * 2048);
+      tma_load_4d(smem + L::IDX_OFF, &tmap_idx, 0, 0, ks_begin, n_tile, &full[0]);
     }
-    if constexpr (L::kSVQ) {
-      l2_prefetch_bulk(w_sidx, static_cast<uint32_t>(nks) * 128 * L::kG);
-    } else if constexpr (!L::kQBS) {
-      l2_prefetch_bulk(w_sf, static_cast<uint32_t>(nks) * A * 512);
+    if constexpr (!L::kSVQ && !L::kQBS) {
+      mbar_arrive_expect_tx(bar_sfw, nks * A * 512);
+      bulk_load(smem + L::SFW_OFF, w_sf, nks * A * 512, bar_sfw);
     }
     if constexpr (L::kVQ) {
-      l2_prefetch_bulk(w_idx, static_cast<uint32_t>(nks) * 8192);
+      mbar_arrive_expect_tx(&full[1], p.ks_per_split * 2048);
+      tma_load_4d(smem + L::IDX_OFF + L::IDX_BUF, &tmap_idx, 0, 1, ks_begin, n_tile, &full[1]);
+      for (int s = 0; s < nks; ++s) l2_prefetch_bulk(w_idx + static_cast<size_t>(s) * 8192 + 4096, 4096);
     } else {
-      for (int s = 0; s < nks; ++s) l2_prefetch_tile_2d(&tmap_wq, (ks_begin + s) * 128, n_tile * 128);
+      for (int s = 0; s < nks; ++s) {
+        mbar_arrive_expect_tx(&full[s], 16384);
+        tma_load_2d(smem + L::W_OFF + s * 16384, &tmap_wq, (ks_begin + s) * 128, n_tile * 128, &full[s]);
+      }
     }
+    if constexpr (L::kSVQ) l2_prefetch_bulk(w_sidx, static_cast<uint32_t>(nks) * 128 * L::kG);
   }
   if (warp == 1) {
     __syncwarp();                                    // tcgen05.alloc is warp-aligned
@@ -251,28 +269,9 @@ __global__ void __maxnreg__(64)
 
   if (warp == 0) {
     // =============================== loader ===============================
-    __syncwarp();
-    if (elect_one()) {
-      // weights only, in the order they are needed: codebooks, index quarter 0, weight
-      // scales, quarters 1..3 (the MMA warp fetches the token operands after the wait)
-      if constexpr (L::kVQ) {
-        const uint32_t cb_bytes = static_cast<uint32_t>(qb1 - qb0 + 1) * 512;
-        mbar_arrive_expect_tx(bar_cb, cb_bytes);
-        bulk_load(smem + L::CB_OFF, w_cb + static_cast<size_t>(qb0) * 256, cb_bytes, bar_cb);
-        // quarter j of stages [ks_begin, ks_begin + ks_per_split): box {2048 B, 1, stages, 1};
-        // stages past K (last split) arrive zero-filled and are not used
-        mbar_arrive_expect_tx(&full[0], p.ks_per_split * 2048);
-        tma_load_4d(smem + L::IDX_OFF, &tmap_idx, 0, 0, ks_begin, n_tile, &full[0]);
-      }
-      if constexpr (!L::kSVQ && !L::kQBS) {
-        mbar_arrive_expect_tx(bar_sfw, nks * A * 512);
-        bulk_load(smem + L::SFW_OFF, w_sf, nks * A * 512, bar_sfw);
-      }
-      if constexpr (L::kVQ) {                        // K-quarter 1 of every stage
-        mbar_arrive_expect_tx(&full[1], p.ks_per_split * 2048);
-        tma_load_4d(smem + L::IDX_OFF + L::IDX_BUF, &tmap_idx, 0, 1, ks_begin, n_tile, &full[1]);
-      }
-    }
+    // (codebooks, index quarters 0 and 1, the weight scales or native weight tiles
+    // were requested during setup; the MMA warp fetches the token operands after the
+    // dependency wait)
     __syncwarp();
     if constexpr (L::kQBS) {
       // PostScale-QB: the weight scale atoms of the slice, each 512 bytes of its
@@ -295,17 +294,12 @@ __global__ void __maxnreg__(64)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_sfw);
     }
-    if (elect_one()) {
-      if constexpr (L::kVQ) {
-        for (int j = 2; j < 4; ++j) {                // K-quarter j of every stage
+    if constexpr (L::kVQ) {
+      if (elect_one()) {
+        for (int j = 2; j < 4; ++j) {                // K-quarter j of every stage (from L2 by now)
           if (!mbar_wait(&dec_ph[j - 2], 0)) break;  // its buffer has been decoded
           mbar_arrive_expect_tx(&full[j], p.ks_per_split * 2048);
           tma_load_4d(smem + L::IDX_OFF + (j % 2) * L::IDX_BUF, &tmap_idx, 0, j, ks_begin, n_tile, &full[j]);
-        }
-      } else {
-        for (int s = 0; s < nks; ++s) {
-          mbar_arrive_expect_tx(&full[s], 16384);
-          tma_load_2d(smem + L::W_OFF + s * 16384, &tmap_wq, (ks_begin + s) * 128, n_tile * 128, &full[s]);
         }
       }
     }

@@ -28,10 +28,55 @@ inline EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
+// Encoded tensor maps are cached per thread, keyed by everything that goes into the
+// encoding (kind, base address, extents, strides, box): a decode step calls the
+// same layers with the same buffers over and over, and encoding costs about a
+// microsecond of host time per map.  A hit returns the identical 128-byte map.
+struct MapKey {
+  int kind;
+  const void* base;
+  int64_t a, b, c, d;
+  bool operator==(const MapKey& o) const {
+    return kind == o.kind && base == o.base && a == o.a && b == o.b && c == o.c && d == o.d;
+  }
+};
+constexpr int kMapCacheSize = 64;
+struct MapCache {
+  MapKey key[kMapCacheSize];
+  CUtensorMap map[kMapCacheSize];
+  int n = 0, next = 0;
+  const CUtensorMap* find(const MapKey& k) const {
+    for (int i = 0; i < n; ++i)
+      if (key[i] == k) return &map[i];
+    return nullptr;
+  }
+  void put(const MapKey& k, const CUtensorMap& m) {
+    const int i = n < kMapCacheSize ? n++ : next;
+    next = (i + 1) % kMapCacheSize;
+    key[i] = k;
+    map[i] = m;
+  }
+};
+inline MapCache& map_cache() {
+  static thread_local MapCache c;
+  return c;
+}
+template <typename F>
+inline bool cached_map(CUtensorMap* map, const MapKey& k, F encode) {
+  MapCache& c = map_cache();
+  if (const CUtensorMap* m = c.find(k)) {
+    *map = *m;
+    return true;
+  }
+  if (!encode(map)) return false;
+  c.put(k, *map);
+  return true;
+}
+
 // 2-D map over an FP4 matrix [rows, K/2 bytes] (row stride ld bytes); box = 128
 // bytes (256 FP4 values) x box_rows rows, 128-byte swizzle, zero fill outside.
-inline bool make_fp4_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int64_t ld,
-                         int box_rows) {
+inline bool encode_fp4_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int64_t ld,
+                           int box_rows) {
   EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return false;
   std::memset(map, 0, sizeof(*map));
@@ -43,12 +88,16 @@ inline bool make_fp4_map(CUtensorMap* map, const void* base, int64_t rows, int64
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+inline bool make_fp4_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int64_t ld, int box_rows) {
+  return cached_map(map, MapKey{1, base, rows, K, ld, box_rows},
+                    [&](CUtensorMap* m) { return encode_fp4_map(m, base, rows, K, ld, box_rows); });
+}
 
 // 3-D map over the same FP4 matrix seen as [K/256 stages][rows][128 bytes] (stage
 // stride 128 bytes): one box = box_rows rows x box_stages consecutive 256-column
 // stages, each stage a [box_rows][128 B] tile in the 128-byte swizzle.
-inline bool make_fp4_stage_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int64_t ld,
-                               int box_rows, int box_stages) {
+inline bool encode_fp4_stage_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int64_t ld,
+                                 int box_rows, int box_stages) {
   EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return false;
   std::memset(map, 0, sizeof(*map));
@@ -60,11 +109,16 @@ inline bool make_fp4_stage_map(CUtensorMap* map, const void* base, int64_t rows,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+inline bool make_fp4_stage_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int64_t ld,
+                               int box_rows, int box_stages) {
+  return cached_map(map, MapKey{2, base, rows, K, ld, (static_cast<int64_t>(box_stages) << 32) | box_rows},
+                    [&](CUtensorMap* m) { return encode_fp4_stage_map(m, base, rows, K, ld, box_rows, box_stages); });
+}
 
 // 4-D map over packed weight indices [N/128][K/256][4][128][16] seen as 8-byte
 // elements: dims {256 (one 2 KB K-quarter slab), 4 quarters, K/256 stages, N/128
 // bands}; one box = quarter q of box_stages consecutive stages of one band.
-inline bool make_idx_map(CUtensorMap* map, const void* base, int64_t N, int64_t K, int box_stages) {
+inline bool encode_idx_map(CUtensorMap* map, const void* base, int64_t N, int64_t K, int box_stages) {
   EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return false;
   std::memset(map, 0, sizeof(*map));
@@ -76,6 +130,24 @@ inline bool make_idx_map(CUtensorMap* map, const void* base, int64_t N, int64_t 
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 4, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+inline bool make_idx_map(CUtensorMap* map, const void* base, int64_t N, int64_t K, int box_stages) {
+  return cached_map(map, MapKey{3, base, N, K, box_stages, 0},
+                    [&](CUtensorMap* m) { return encode_idx_map(m, base, N, K, box_stages); });
+}
+
+// The dynamic shared-memory opt-in of a kernel, set once per device (the attribute
+// belongs to the function on the device that is current when it is set).
+template <typename Kern>
+inline cudaError_t ensure_smem_attr(Kern kern, int bytes, uint64_t* done_mask) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit && (__atomic_load_n(done_mask, __ATOMIC_ACQUIRE) & bit)) return cudaSuccess;
+  err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err == cudaSuccess && bit) __atomic_fetch_or(done_mask, bit, __ATOMIC_RELEASE);
+  return err;
 }
 
 // ------------------------------------------------------------------------------------
@@ -136,7 +208,8 @@ cudaError_t launch_gemm_ncb(const CUtensorMap& tx, const CUtensorMap& tw,
                             const GemmParams<MOE ? kMaxGroups : 1>& p, dim3 grid, cudaStream_t stream) {
   using L = StageLayout<FMT, WSRC, T, NCB>;
   auto kern = gemm_kernel<FMT, WSRC, T, MOE, NCB>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+  static uint64_t attr_set = 0;
+  cudaError_t err = ensure_smem_attr(kern, L::SMEM, &attr_set);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -189,7 +262,8 @@ cudaError_t launch_gemv(const CUtensorMap& tx, const CUtensorMap& tw, const CUte
                         dim3 grid, cudaStream_t stream) {
   using L = GemvLayout<FMT, WSRC>;
   auto kern = gemv_kernel<FMT, WSRC>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+  static uint64_t attr_set = 0;
+  cudaError_t err = ensure_smem_attr(kern, L::SMEM, &attr_set);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -393,7 +467,8 @@ template <int FMT, int WSRC>
 cudaError_t launch_decode_dump(const DecodeArgs& a, cudaStream_t stream) {
   constexpr int smem = DumpLayout<FMT, WSRC>::SMEM;
   auto kern = decode_dump_kernel<FMT, WSRC>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static uint64_t attr_set = 0;
+  cudaError_t err = ensure_smem_attr(kern, smem, &attr_set);
   if (err != cudaSuccess) return err;
   ExpertPtrs w{};
   w.idx = a.w_idx;

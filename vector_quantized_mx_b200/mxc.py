@@ -139,8 +139,14 @@ class MXTensor:
     fmt: str
 
     def _c(self) -> _MxTensor:
-        return _MxTensor(self.q.data_ptr(), self.sf.data_ptr(), _ptr(self.tscale), self.rows, self.K,
-                         self.q.stride(0), FMT[self.fmt])
+        # the C struct is rebuilt only when a field it holds has changed
+        key = (self.q.data_ptr(), self.sf.data_ptr(), _ptr(self.tscale), self.rows, self.K, self.q.stride(0),
+               self.fmt)
+        c = self.__dict__.get("_cstruct")
+        if c is None or c[0] != key:
+            c = (key, _MxTensor(key[0], key[1], key[2], self.rows, self.K, key[5], FMT[self.fmt]))
+            self.__dict__["_cstruct"] = c
+        return c[1]
 
 
 def empty_act(M: int, K: int, fmt: str, device) -> MXTensor:
@@ -216,9 +222,13 @@ class PackedWeight:
     w_tscale: float
 
     def _c(self) -> _Weight:
-        return _Weight(STRATEGY[self.strategy], FMT[self.fmt], self.N, self.K, self.qn, self.qk,
-                       self.idx.data_ptr(), self.cb.data_ptr(), _ptr(self.scales), _ptr(self.sidx),
-                       _ptr(self.scb), self.w_tscale)
+        key = (self.strategy, self.fmt, self.N, self.K, self.qn, self.qk, self.idx.data_ptr(), self.cb.data_ptr(),
+               _ptr(self.scales), _ptr(self.sidx), _ptr(self.scb), self.w_tscale)
+        c = self.__dict__.get("_cstruct")
+        if c is None or c[0] != key:
+            c = (key, _Weight(STRATEGY[self.strategy], FMT[self.fmt], *key[2:]))
+            self.__dict__["_cstruct"] = c
+        return c[1]
 
     def storage_bytes(self) -> int:
         n = self.idx.numel() + self.cb.numel() * 2
