@@ -387,6 +387,8 @@ def run_gpu(args, rank, world, dist):
         extra["prefill"] = prefill_leg(dev, stream, capture, time_graph, steps, world, with_cpu)
     if "moe" in args.legs:
         extra["moe"] = moe_leg(dev, stream, capture, time_graph, steps, world, with_cpu)
+    if "sweep" in args.legs:
+        extra["sweep"] = sweep_leg(dev, stream, capture, time_graph, steps, world)
     if rank != 0:
         return
     # our kernels per step: the activation quantizer (one launch up to 16 x 8192
@@ -604,6 +606,76 @@ def moe_leg(dev, stream, capture, time_graph, steps, world, with_cpu):
     return out
 
 
+def sweep_leg(dev, stream, capture, time_graph, steps, world):
+    """Config 5: K = N = 8192; M in {1, 16, 128, 1024, 16384} x QBlock in {full tensor,
+    1024^2, 256^2, 128^2} x {PostScale, PreScale, PreScale+} x {E8M0-B32, E4M3-B16}
+    (120 MXCode points), plus native FP4 (4.25 / 4.50 bits per weight) on the same
+    decoded values of the PreScale 256^2 weights for each format and M (10 points).
+    Each point times the linear layer alone, over 6 rotating weight copies (>= 100 MB,
+    so M <= 128 streams its weights from HBM).  Bound: HBM for M <= 16, FP4 tensor
+    for M >= 1024, both reported at M = 128; frac is against the bound's peak."""
+    import torch
+    from vector_quantized_mx_b200 import mxc, synth
+    K = N = 8192
+    n_copies = 6
+    hbm, hbm_kind = peaks()
+    fp4, fp4_kind = fp4_peak()
+    acts = {}
+    for M in synth.SWEEP_M:
+        x = torch.from_numpy(synth.config5_activations(M).view(np.int16)).view(torch.bfloat16).to(dev)
+        for fmt in synth.FORMATS:
+            with torch.cuda.stream(stream):
+                acts[(M, fmt)] = mxc.quantize_act(x, fmt, stream=stream)
+        del x
+    stream.synchronize()
+    ws = {M: mxc.linear_workspace(M, N, K, "e4m3_b16", dev) for M in synth.SWEEP_M}
+    ys = {M: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for M in synth.SWEEP_M}
+    cols = ["M", "qblock", "strategy", "format", "ms", "tflops", "weight_GBps", "bound", "frac", "x_native"]
+    rows, native = [], {}
+
+    def timed(fn):
+        n = max(5, steps // 4)
+        return time_graph(capture(n, fn)) / n
+
+    for fmt in synth.FORMATS:
+        for strat in synth.STRATEGIES:
+            for qb in synth.SWEEP_QB:
+                w = synth.config5_weight(qb, strat, fmt)
+                copies = rotated(mxc.pack_weight(w, device=dev), n_copies)
+                wbytes = copies[0].storage_bytes()
+                nats = None
+                if strat == "prescale" and qb == 256:
+                    with torch.cuda.stream(stream):
+                        nat0 = mxc.decode_weight(copies[0], stream=stream)
+                    nats = [nat0] + [mxc.MXTensor(nat0.q.clone(), nat0.sf.clone(), nat0.tscale.clone(), N, K, fmt)
+                                     for _ in range(n_copies - 1)]
+                for M in synth.SWEEP_M:
+                    a, y, wk = acts[(M, fmt)], ys[M], ws[M]
+                    ms = timed(lambda i: mxc.linear(a, copies[i % n_copies], y=y, ws=wk, stream=stream))
+                    if nats is not None:
+                        native[(fmt, M)] = timed(lambda i: mxc.native_linear(a, nats[i % n_copies], y=y, ws=wk,
+                                                                             stream=stream))
+                    flops = 2.0 * M * N * K
+                    io = wbytes + M * K // 2 + M * K // (32 if fmt == "e8m0_b32" else 16) + M * N * 2
+                    f_hbm = io / (ms * 1e-3) / 1e9 / hbm
+                    f_fp4 = flops / (ms * 1e-3) / 1e12 / fp4
+                    bound = "hbm" if M <= 16 else "tensor" if M >= 1024 else "both"
+                    frac = f_hbm if M <= 16 else f_fp4 if M >= 1024 else [f_hbm, f_fp4]
+                    rows.append([M, qb or "full", strat, fmt, ms, world * flops / (ms * 1e-3) / 1e12,
+                                 world * wbytes / (ms * 1e-3) / 1e9, bound, frac, None])
+                del copies, nats
+    if mxc.get_device_error(stream) != 0:
+        raise SystemExit("bench: a sweep point failed")
+    for r in rows:
+        r[9] = native[(r[3], r[0])] / r[4]
+    nat_rows = [[M, fmt, native[(fmt, M)], world * 2.0 * M * N * K / (native[(fmt, M)] * 1e-3) / 1e12]
+                for fmt in synth.FORMATS for M in synth.SWEEP_M]
+    return {"workload": "K=N=8192 sweep: M x QBlock x strategy x format, BF16 out", "columns": cols,
+            "points": rows, "native_columns": ["M", "format", "ms", "tflops"], "native": nat_rows,
+            "peaks": {"hbm_GBps": hbm, "hbm_kind": hbm_kind, "fp4_TFLOPs": fp4, "fp4_kind": fp4_kind},
+            "l2": f"{n_copies} rotating weight copies per point"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -612,8 +684,9 @@ def main():
     ap.add_argument("--impl", default="mxcode", choices=["mxcode", "reference"])
     ap.add_argument("--m", type=int, default=16, choices=[1, 4, 16])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--legs", default="prefill,moe",
-                    help="extra workloads timed after the decode line: prefill (config 3), moe (config 4)")
+    ap.add_argument("--legs", default="prefill,moe,sweep",
+                    help="extra workloads timed after the decode line: prefill (config 3), moe (config 4), "
+                         "sweep (config 5)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -354,3 +354,103 @@ def storage_bytes(w) -> int:
     else:
         n += w.scales.size
     return int(n)
+
+
+# ---------------------------------------------------------------------------
+# SwiGLU between the MoE gate/up and down projections, and the MX quantization
+# of its FP32 output (the down projection's W4A4 activation).  The pages name
+# the MoE expert tensors (Table 4 caption: Qwen3's experts, whose FFN is
+# h = SiLU(gate) * up); they give no arithmetic for it, so these are readings:
+#
+# * gate/up weight [2F, K]: rows [0, F) are the gate projection, rows [F, 2F)
+#   the up projection; g and u are the layer's FP32 outputs (accumulator times
+#   the FP32 tensor scales, as the linear layer returns them);
+# * h = SiLU(g) * u with SiLU(g) = g / (1 + exp(-g)), every step one FP32
+#   operation, so that the codes that h's quantization decides are decided in
+#   the precision the kernel computes them in;
+# * exp is a fixed FP32 function E, written out below (Cody and Waite's
+#   two-constant reduction x = n ln2 + r, then the Taylor polynomial of e^r to
+#   degree 7 by Horner's rule, then the exact scaling by 2^n); E(x) = +inf for
+#   x > 88 and 0 for x < -86, where the FP32 result would be near overflow or
+#   subnormal;
+# * h is quantized by the activation rule above (blocks along h's channels),
+#   applied to FP32 values instead of BF16 ones; for E4M3-B16 with a given FP32
+#   tensor scale (a calibrated scale: h's global maximum is not known while the
+#   gate/up tiles are still being produced).
+# ---------------------------------------------------------------------------
+
+_F32 = np.float32
+_EXP_LOG2E = _F32(1.44269504088896341)
+_EXP_C1 = _F32(0.693359375)                         # ln 2 rounded to 9 bits: n * C1 is exact
+_EXP_C2 = _F32(0.6931471805599453 - 0.693359375)    # the rest of ln 2
+_EXP_TAYLOR = [_F32(1.0 / math.factorial(i)) for i in range(7, -1, -1)]   # 1/7!, ..., 1/1!, 1/0!
+
+
+def exp_fp32(x) -> np.ndarray:
+    """E(x): e^x in FP32 by a fixed sequence of FP32 operations (no fused multiply-add).
+
+    n = rint(x * log2 e); r = (x - n*C1) - n*C2 with C1 + C2 = ln 2; p = Taylor
+    polynomial of e^r to degree 7 (Horner, one multiply and one add per step);
+    E = p * 2^n.  +inf above 88, 0 below -86.
+    """
+    x = np.asarray(x, dtype=_F32)
+    with np.errstate(over="ignore", invalid="ignore"):
+        n = np.rint(x * _EXP_LOG2E).astype(_F32)
+        r = (x - n * _EXP_C1) - n * _EXP_C2
+        p = np.full_like(x, _EXP_TAYLOR[0])
+        for c in _EXP_TAYLOR[1:]:
+            p = p * r + c
+        ni = np.clip(n, -126, 127).astype(np.int32)
+        scale = ((ni + 127).astype(np.uint32) << 23).view(_F32)     # 2^n, exact
+        e = p * scale
+    e = np.where(x > _F32(88.0), _F32(np.inf), e)
+    return np.where(x < _F32(-86.0), _F32(0.0), e).astype(_F32)
+
+
+def swiglu_fp32(g, u) -> np.ndarray:
+    """h = SiLU(g) * u = (g / (1 + E(-g))) * u, each operation in FP32."""
+    g = np.asarray(g, dtype=_F32)
+    u = np.asarray(u, dtype=_F32)
+    with np.errstate(over="ignore", invalid="ignore", divide="ignore"):
+        d = _F32(1.0) + exp_fp32(-g)
+        return ((g / d) * u).astype(_F32)
+
+
+def quantize_values_e8m0(x):
+    """E8M0-B32 MX quantization of FP32 values [rows, F] (the rule of quantize_act_e8m0)."""
+    x = np.asarray(x, dtype=_F32).astype(np.float64)
+    M, F = x.shape
+    xb = x.reshape(M, F // 32, 32)
+    amax = np.abs(xb).max(axis=2)
+    _, ex = np.frexp(amax)
+    e = np.clip(ex.astype(np.int64) - 1 - 2, -127, 127)
+    e = np.where(amax == 0, -127, e)
+    codes = _signed_codes(xb, xb / np.ldexp(1.0, e)[:, :, None])
+    return codes.reshape(M, F), (e + 127).astype(np.uint8)
+
+
+def quantize_values_e4m3(x, tscale: float):
+    """E4M3-B16 MX quantization of FP32 values [rows, F] with a given FP32 tensor
+    scale s (the rule of quantize_act_e4m3)."""
+    s = _F32(tscale)
+    x = np.asarray(x, dtype=_F32).astype(np.float64)
+    M, F = x.shape
+    xb = x.reshape(M, F // 16, 16)
+    amax = np.abs(xb).max(axis=2).astype(_F32)
+    t = ((amax / _F32(6.0)).astype(_F32) / s).astype(_F32)
+    sb = e4m3_encode_rne_satfinite(np.where(np.isfinite(t), t, np.float64(448.0)))
+    denom = (e4m3_value(sb).astype(_F32) * s).astype(_F32).astype(np.float64)
+    safe = np.where(denom == 0, 1.0, denom)
+    q = np.where((sb == 0)[:, :, None], 0.0, xb / safe[:, :, None])
+    return _signed_codes(xb, q).reshape(M, F), sb.astype(np.uint8)
+
+
+def swiglu_quantize(y_gate_up, fmt: str, tscale: Optional[float] = None):
+    """The down projection's activation from the FP32 gate/up output [rows, 2F]:
+    h = swiglu_fp32(gate, up), then MX codes [rows, F] and block scales [rows, F/B]."""
+    y = np.asarray(y_gate_up, dtype=_F32)
+    F = y.shape[1] // 2
+    h = swiglu_fp32(y[:, :F], y[:, F:])
+    if fmt == E8M0_B32:
+        return quantize_values_e8m0(h)
+    return quantize_values_e4m3(h, tscale)

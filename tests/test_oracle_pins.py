@@ -512,3 +512,94 @@ def test_zipf_routing_first_choice_matches_closed_form():
     p1 = 1 / H
     assert abs(H - 4.431) < 5e-3
     assert abs(np.mean(first == 0) - p1) < 4 * math.sqrt(p1 * (1 - p1) / T)
+
+
+# ---------------------------------------------------------------------------
+# SwiGLU and the FP32-value quantization of the down projection's activation
+# (MoE expert tensors, Table 4 caption): pinned to FP64 mathematics, to special
+# values, and to the BF16 quantizers above on values both can take.
+# ---------------------------------------------------------------------------
+
+def test_exp_fp32_matches_the_exponential():
+    x = np.linspace(-86.0, 88.0, 400001).astype(np.float32)
+    x = np.concatenate([x, np.float32([0.0, -0.0, 1.0, -1.0, 0.5, 1e-30, -1e-30])])
+    e = O.exp_fp32(x).astype(np.float64)
+    ref = np.exp(x.astype(np.float64))
+    assert np.all(np.abs(e - ref) <= 2 * 2.0 ** -24 * ref)          # within 2 ulp
+    assert O.exp_fp32(np.float32(0.0)) == 1.0
+    assert np.all(O.exp_fp32(np.float32([88.5, 100.0, 1e30])) == np.inf)
+    assert np.all(O.exp_fp32(np.float32([-86.5, -100.0, -1e30])) == 0.0)
+    # FP32 in, FP32 out, a fixed function of its input
+    assert O.exp_fp32(x).dtype == np.float32
+    assert np.array_equal(O.exp_fp32(x), O.exp_fp32(x.copy()))
+
+
+def test_swiglu_fp32_matches_fp64_silu_times_up():
+    rng = np.random.default_rng(41)
+    g = np.concatenate([np.linspace(-40, 40, 200001), rng.normal(0, 4, 100000)]).astype(np.float32)
+    u = rng.normal(0, 2, g.size).astype(np.float32)
+    h = O.swiglu_fp32(g, u).astype(np.float64)
+    gd, ud = g.astype(np.float64), u.astype(np.float64)
+    ref = gd / (1.0 + np.exp(-gd)) * ud
+    ok = np.abs(ref) > 1e-35
+    assert np.all(np.abs(h - ref)[ok] <= 6 * 2.0 ** -24 * np.abs(ref[ok]))   # a few FP32 roundings
+    # special values: SiLU(0) = 0, SiLU(g) = g for large g, -0 for very negative g
+    sp = O.swiglu_fp32(np.float32([0.0, 100.0, -100.0, 3e38]), np.float32([5.0, 2.0, 7.0, 1.0]))
+    assert sp[0] == 0.0 and sp[1] == 200.0 and sp[2] == 0.0 and np.signbit(sp[2]) and sp[3] == np.float32(3e38)
+
+
+def test_fp32_value_quantizers_equal_the_bf16_ones_on_bf16_values():
+    rng = np.random.default_rng(43)
+    bits = bf16_bits(rng.normal(size=(6, 256)) * np.exp(rng.uniform(-10, 10, (6, 1))))
+    vals = O.bf16_value(bits).astype(np.float32)
+    c1, s1 = O.quantize_act_e8m0(bits)
+    c2, s2 = O.quantize_values_e8m0(vals)
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
+    ts = np.float32(0.0371)
+    c1, s1, _ = O.quantize_act_e4m3(bits, ts)
+    c2, s2 = O.quantize_values_e4m3(vals, ts)
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
+
+
+def test_fp32_value_quantizers_exact_decisions():
+    """Random FP32 values (24-bit mantissas, not BF16): the E8M0 exponent by the
+    |v| / 2^e in [4, 8) characterisation, the E4M3 scale by torch's FP32 arithmetic
+    and float8 cast, every code by exact rational rounding."""
+    rng = np.random.default_rng(47)
+    v = (rng.normal(size=(4, 64)) * np.exp(rng.uniform(-6, 6, (4, 1)))).astype(np.float32)
+    codes, sf = O.quantize_values_e8m0(v)
+    for r in range(4):
+        for b in range(2):
+            blk = [Fraction(float(t)) for t in v[r, 32 * b:32 * b + 32]]
+            amax = max(abs(t) for t in blk)
+            e = 0
+            while amax / Fraction(2) ** e >= 8:
+                e += 1
+            while amax / Fraction(2) ** e < 4:
+                e -= 1
+            assert int(sf[r, b]) == e + 127
+            for j, t in enumerate(blk):
+                assert int(codes[r, 32 * b + j]) == _rne_e2m1_fraction(t / Fraction(2) ** e) | (8 if t < 0 else 0)
+    s = np.float32(0.0123)
+    codes, sb = O.quantize_values_e4m3(v, s)
+    vt = torch.from_numpy(v).reshape(4, 4, 16)
+    t = (vt.abs().amax(dim=2) / 6.0) / torch.tensor(s)
+    assert np.array_equal(sb, t.clamp(max=448.0).to(torch.float8_e4m3fn).view(torch.uint8).numpy())
+    denom = (torch.from_numpy(sb).view(torch.float8_e4m3fn).float() * torch.tensor(s)).numpy()
+    for r in range(4):
+        for k in range(64):
+            d = Fraction(float(denom[r, k // 16]))
+            val = Fraction(float(v[r, k]))
+            mag = 0 if d == 0 else _rne_e2m1_fraction(val / d)
+            assert int(codes[r, k]) == mag | (8 if val < 0 else 0)
+
+
+def test_swiglu_quantize_splits_gate_and_up():
+    rng = np.random.default_rng(53)
+    y = rng.normal(0, 3, (5, 2 * 64)).astype(np.float32)
+    c, s = O.swiglu_quantize(y, "e8m0_b32")
+    c2, s2 = O.quantize_values_e8m0(O.swiglu_fp32(y[:, :64], y[:, 64:]))
+    assert np.array_equal(c, c2) and np.array_equal(s, s2)
+    c, s = O.swiglu_quantize(y, "e4m3_b16", 0.01)
+    c2, s2 = O.quantize_values_e4m3(O.swiglu_fp32(y[:, :64], y[:, 64:]), 0.01)
+    assert np.array_equal(c, c2) and np.array_equal(s, s2)
