@@ -581,6 +581,34 @@ def moe_leg(dev, stream, capture, time_graph, steps, world, with_cpu):
                                   "target_ms": max(t_bw, t_fl), "frac": max(t_bw, t_fl) / ms_lin,
                                   "hbm_peak_GBps": hbm, "hbm_kind": hbm_kind,
                                   "fp4_peak_TFLOPs": peak, "fp4_kind": peak_kind, "traffic": None}}
+    # The MoE FFN with SwiGLU fused into the gate/up epilogue, which writes the down
+    # projection's FP4 activation directly: grouped quantization -> gate/up + SwiGLU
+    # -> down.  h's E4M3 tensor scale is calibrated once from a torch evaluation of
+    # SwiGLU on the gate/up output (plumbing, outside the timed region).
+    pg, pd = proj["gate_up"], proj["down"]
+    F = pg["N"] // 2
+    with torch.cuda.stream(stream):
+        ygu = mxc.moe_linear(pg["act"], offd, pg["packed"], stream=stream)
+        hcal = torch.nn.functional.silu(ygu[:, :F]) * ygu[:, F:]
+        h_ts = (hcal.abs().max() / 2688.0).reshape(1).to(torch.float32)
+        h_act = mxc.moe_gate_up_swiglu(pg["act"], offd, pg["packed"], h_tscale=h_ts, ws=pg["mws"], stream=stream)
+    stream.synchronize()
+    del ygu, hcal
+
+    def ffn(i):
+        quant(pg)
+        mxc.moe_gate_up_swiglu(pg["act"], offd, pg["packed"], h_tscale=h_ts, out=h_act, ws=pg["mws"], stream=stream)
+        mxc.moe_linear(h_act, offd, pd["packed"], y=pd["y"], ws=pd["mws"], stream=stream)
+    n_f = max(5, steps // 8)
+    ms_ffn = time_graph(capture(n_f, ffn)) / n_f
+    ms_gus = time_graph(capture(n_f, lambda i: mxc.moe_gate_up_swiglu(
+        pg["act"], offd, pg["packed"], h_tscale=h_ts, out=h_act, ws=pg["mws"], stream=stream))) / n_f
+    if mxc.get_device_error(stream) != 0:
+        raise SystemExit("bench: the fused MoE FFN failed")
+    out["ffn_swiglu_fused"] = {"ms_per_step": ms_ffn, "ms_gate_up_swiglu": ms_gus,
+                               "tflops": world * (pg["flops"] + pd["flops"]) / (ms_ffn * 1e-3) / 1e12,
+                               "steps": "grouped quantization, gate/up + SwiGLU + FP4 quantization of h, down",
+                               "gpu_launches_per_step": 2 + 2 + 2}
     if with_cpu:
         from oracle import mxcode_oracle as O
         counts = np.diff(off)

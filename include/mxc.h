@@ -268,6 +268,38 @@ mxc_status mxc_moe_linear(const mxc_mx_tensor* a, const int32_t* d_offsets, cons
                           int32_t E, void* y, int64_t ldy, mxc_dtype y_dtype, void* ws,
                           size_t ws_bytes, mxc_stream_t stream);
 
+/* The gate/up projection of a MoE layer fused with SwiGLU and with the MX
+ * quantization of its result, which is the down projection's W4A4 activation
+ * (the experts are Qwen3's MoE FFN tensors: Table 4 caption).  Each expert's
+ * gate/up weight is [2F, K]: rows [0, F) are the gate projection, rows [F, 2F)
+ * the up projection.  For every row r of expert e, with g and u the FP32 outputs
+ * of the two projections (accumulator times the FP32 tensor scales, as
+ * mxc_moe_linear returns them):
+ *   h = SiLU(g) * u = (g / (1 + exp(-g))) * u,
+ * evaluated one IEEE FP32 operation at a time, with exp(x) computed as
+ * 2^n * P(r), x = n ln2 + r (Cody-Waite reduction, ln2 split into a 9-bit head
+ * and the rest), P the degree-7 Taylor polynomial of e^r by Horner's rule, no
+ * fused multiply-add; exp(x) = +inf above 88 and 0 below -86.  h is then
+ * quantized exactly as mxc_quantize_act quantizes BF16 input (blocks of B
+ * consecutive channels of h), in the activation's format:
+ *   E8M0-B32: no tensor scale;
+ *   E4M3-B16: with the given FP32 tensor scale *h_tscale_in (a calibrated scale:
+ *             h's global maximum is unknown while its tiles are produced).
+ * h is never written in a wider type.
+ * a, d_offsets, experts, E, ws, ws_bytes: as for mxc_moe_linear (N = 2F, F a
+ *           multiple of 128)
+ * h_tscale_in device FP32, required for E4M3-B16, ignored for E8M0-B32
+ * h_q       device, FP4 matrix [M, ldh] (ldh >= F/2, a multiple of 16)
+ * h_sf      device, grouped SF layout of h's [rows, F/B] scales (the layout of
+ *           mxc_quantize_act_grouped over the same offsets: each expert's rows
+ *           start at the next multiple of 128 rows; mxc_grouped_sf_rows_bound(M, E)
+ *           rows are enough); the padding rows of every expert tile get zero
+ *           scales.  (h_q, h_sf, h_tscale_in) is the activation of the down
+ *           projection's mxc_moe_linear over the same d_offsets. */
+mxc_status mxc_moe_gate_up_swiglu(const mxc_mx_tensor* a, const int32_t* d_offsets, const mxc_weight* experts,
+                                  int32_t E, const float* h_tscale_in, uint8_t* h_q, int64_t ldh, uint8_t* h_sf,
+                                  void* ws, size_t ws_bytes, mxc_stream_t stream);
+
 /* mxc_moe_linear for callers that cannot allocate device memory: code that
  * runs inside a CUDA stream capture, plugin hosts and real-time serving loops
  * that forbid allocator calls, or C callers with no device allocator at hand.

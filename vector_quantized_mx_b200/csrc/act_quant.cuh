@@ -10,6 +10,8 @@
 // block amax, scale byte, 32/16 E2M1 codes decided by the sign of an exact
 // fused multiply-add against each rounding midpoint, one vector store of FP4.
 // The work is HBM-bound (read 2 bytes/element, write ~0.53).
+#pragma once
+
 #include <cstdint>
 
 #include "mxc_device.cuh"
@@ -64,6 +66,70 @@ __device__ __forceinline__ uint32_t e2m1_code(float x, float d) {
   const bool lo = __fmaf_rn(mu, d, -a) < 0.0f;                     // a > mu d
   const uint32_t c = (hi ? 4u : 0u) + (mid ? 2u : 0u) + (lo ? 1u : 0u);
   return c | ((__float_as_uint(x) >> 28) & 8u);
+}
+
+// ------------------------------------------------------------------------------------
+// SwiGLU of the MoE projections, one FP32 operation per step (so that the codes of
+// its quantization are decided in exactly this arithmetic).  E(x) = e^x by Cody and
+// Waite's reduction x = n ln2 + r (ln2 split into a 9-bit head, so n * head is
+// exact, and the rest), the degree-7 Taylor polynomial of e^r by Horner's rule and
+// the exact scaling by 2^n; +inf above 88 and 0 below -86.  No fused multiply-add.
+// ------------------------------------------------------------------------------------
+__device__ __forceinline__ float exp_fp32(float x) {
+  const float n = rintf(__fmul_rn(x, 1.44269504088896341f));
+  const float r = __fsub_rn(__fsub_rn(x, __fmul_rn(n, 0.693359375f)),
+                            __fmul_rn(n, static_cast<float>(0.6931471805599453 - 0.693359375)));
+  float q = static_cast<float>(1.0 / 5040.0);
+  q = __fadd_rn(__fmul_rn(q, r), static_cast<float>(1.0 / 720.0));
+  q = __fadd_rn(__fmul_rn(q, r), static_cast<float>(1.0 / 120.0));
+  q = __fadd_rn(__fmul_rn(q, r), static_cast<float>(1.0 / 24.0));
+  q = __fadd_rn(__fmul_rn(q, r), static_cast<float>(1.0 / 6.0));
+  q = __fadd_rn(__fmul_rn(q, r), 0.5f);
+  q = __fadd_rn(__fmul_rn(q, r), 1.0f);
+  q = __fadd_rn(__fmul_rn(q, r), 1.0f);
+  const int ni = min(127, max(-126, static_cast<int>(n)));
+  const float e = __fmul_rn(q, __int_as_float((ni + 127) << 23));
+  return x > 88.0f ? __int_as_float(0x7F800000) : x < -86.0f ? 0.0f : e;
+}
+
+// h = (g / (1 + E(-g))) * u
+__device__ __forceinline__ float swiglu_fp32(float g, float u) {
+  return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, exp_fp32(-g))), u);
+}
+
+// MX quantization of one block of B FP32 values (B = 32: E8M0 scale; B = 16: E4M3
+// scale over the given tensor scale s), the rule of quantize_block applied to FP32
+// instead of BF16 input: q receives the B/8 words of packed E2M1 codes (element 2i
+// in the low nibble of byte i), sfb the scale byte.
+template <int B>
+__device__ __forceinline__ void quantize_block_f32(const float (&v)[B], bool e4m3, float s, uint32_t (&q)[B / 8],
+                                                   uint32_t& sfb) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < B; ++i) a = fmaxf(a, fabsf(v[i]));
+  float d = 0.0f;
+  if (!e4m3) {
+    const uint32_t u = __float_as_uint(a);
+    if (a == 0.0f) {
+      sfb = 0;
+    } else {
+      const uint32_t E = (u >> 23) & 0xFF;
+      const int flog = E ? static_cast<int>(E) - 127 : (31 - __clz(u & 0x7FFFFF)) - 149;
+      const int e = min(127, max(-127, flog - 2));
+      sfb = static_cast<uint32_t>(e + 127);
+      d = exp2_int(e);
+    }
+  } else {
+    sfb = e4m3_encode_satfinite(__fdiv_rn(__fdiv_rn(a, 6.0f), s));
+    d = sfb ? __fmul_rn(e4m3_decode(sfb), s) : 0.0f;
+  }
+#pragma unroll
+  for (int i = 0; i < B / 8; ++i) q[i] = 0;
+#pragma unroll
+  for (int i = 0; i < B; ++i) {
+    const uint32_t c = d == 0.0f ? ((__float_as_uint(v[i]) >> 28) & 8u) : e2m1_code(v[i], d);
+    q[i / 8] |= c << (4 * (i % 8));
+  }
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -203,11 +203,11 @@ size_t moe_workspace_bytes(int64_t /*M*/, int32_t E, int64_t /*N*/, int64_t /*K*
 // ------------------------------------------------------------------------------------
 // Launch
 // ------------------------------------------------------------------------------------
-template <int FMT, int WSRC, int T, bool MOE, int NCB>
+template <int FMT, int WSRC, int T, bool MOE, int NCB, bool SWI = false>
 cudaError_t launch_gemm_ncb(const CUtensorMap& tx, const CUtensorMap& tw,
                             const GemmParams<MOE ? kMaxGroups : 1>& p, dim3 grid, cudaStream_t stream) {
-  using L = StageLayout<FMT, WSRC, T, NCB>;
-  auto kern = gemm_kernel<FMT, WSRC, T, MOE, NCB>;
+  using L = StageLayout<FMT, WSRC, T, NCB, SWI ? 2 : 1>;
+  auto kern = gemm_kernel<FMT, WSRC, T, MOE, NCB, SWI>;
   static uint64_t attr_set = 0;
   cudaError_t err = ensure_smem_attr(kern, L::SMEM, &attr_set);
   if (err != cudaSuccess) return err;
@@ -231,13 +231,13 @@ cudaError_t launch_gemm_ncb(const CUtensorMap& tx, const CUtensorMap& tw,
 }
 
 // Two codebooks per stage only for VQ weights whose QBlock is 128 wide along K.
-template <int FMT, int WSRC, int T, bool MOE>
+template <int FMT, int WSRC, int T, bool MOE, bool SWI = false>
 cudaError_t launch_gemm(const CUtensorMap& tx, const CUtensorMap& tw,
                         const GemmParams<MOE ? kMaxGroups : 1>& p, dim3 grid, cudaStream_t stream) {
   if constexpr (WSRC != WSRC_NATIVE) {
-    if (p.qk == 128) return launch_gemm_ncb<FMT, WSRC, T, MOE, 2>(tx, tw, p, grid, stream);
+    if (p.qk == 128) return launch_gemm_ncb<FMT, WSRC, T, MOE, 2, SWI>(tx, tw, p, grid, stream);
   }
-  return launch_gemm_ncb<FMT, WSRC, T, MOE, 1>(tx, tw, p, grid, stream);
+  return launch_gemm_ncb<FMT, WSRC, T, MOE, 1, SWI>(tx, tw, p, grid, stream);
 }
 
 template <int FMT, int WSRC, int T>
@@ -449,8 +449,27 @@ mxc_status run_moe_linear(const MoeArgs& m, cudaStream_t stream) {
     p.w[e].scb = w.scb;
     p.w[e].w_tscale = w.w_tscale;
   }
-  const dim3 grid(static_cast<unsigned>(a.N / kTileN), static_cast<unsigned>((a.M + 127) / 128 + m.E), 1);
   cudaError_t err;
+  if (m.swiglu) {
+    // SwiGLU: each CTA owns 128 channels of h (gate rows and the matching up rows)
+    p.F = static_cast<int>(a.N / 2);
+    p.h_q = m.h_q;
+    p.ldh = m.ldh;
+    p.h_sf = m.h_sf;
+    p.h_tscale = m.h_tscale;
+    const dim3 grid(static_cast<unsigned>(a.N / 2 / kTileN), static_cast<unsigned>((a.M + 127) / 128 + m.E), 1);
+    if (a.fmt == FMT_E8M0) {
+      if (a.wsrc == WSRC_VQ_DIRECT) err = launch_gemm<FMT_E8M0, WSRC_VQ_DIRECT, 128, true, true>(tx, tx, p, grid, stream);
+      else if (a.wsrc == WSRC_VQ_SVQ) err = launch_gemm<FMT_E8M0, WSRC_VQ_SVQ, 128, true, true>(tx, tx, p, grid, stream);
+      else err = launch_gemm<FMT_E8M0, WSRC_VQ_QBS, 128, true, true>(tx, tx, p, grid, stream);
+    } else {
+      if (a.wsrc == WSRC_VQ_DIRECT) err = launch_gemm<FMT_E4M3, WSRC_VQ_DIRECT, 128, true, true>(tx, tx, p, grid, stream);
+      else if (a.wsrc == WSRC_VQ_SVQ) err = launch_gemm<FMT_E4M3, WSRC_VQ_SVQ, 128, true, true>(tx, tx, p, grid, stream);
+      else err = launch_gemm<FMT_E4M3, WSRC_VQ_QBS, 128, true, true>(tx, tx, p, grid, stream);
+    }
+    return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
+  }
+  const dim3 grid(static_cast<unsigned>(a.N / kTileN), static_cast<unsigned>((a.M + 127) / 128 + m.E), 1);
   if (a.fmt == FMT_E8M0) {
     if (a.wsrc == WSRC_VQ_DIRECT) err = launch_gemm<FMT_E8M0, WSRC_VQ_DIRECT, 128, true>(tx, tx, p, grid, stream);
     else if (a.wsrc == WSRC_VQ_SVQ) err = launch_gemm<FMT_E8M0, WSRC_VQ_SVQ, 128, true>(tx, tx, p, grid, stream);

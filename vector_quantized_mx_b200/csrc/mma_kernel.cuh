@@ -34,6 +34,7 @@
 // GEMV does not take (T = 16) and prefill (T = 128 or 256) without a transpose.
 #pragma once
 
+#include "act_quant.cuh"
 #include "mxc_device.cuh"
 #include "mxc_internal.h"
 
@@ -71,12 +72,20 @@ struct GemmParams {
   int E;                     // MoE
   const int32_t* offsets;
   const int32_t* tile_prefix;
+  // MoE gate/up with SwiGLU: h = SiLU(gate) * up is quantized straight into the
+  // down projection's activation (F = N / 2 channels)
+  int F;
+  uint8_t* h_q;              // FP4 [M, ldh]
+  int64_t ldh;
+  uint8_t* h_sf;             // grouped SF layout of [rows, F / B]
+  const float* h_tscale;     // E4M3-B16: the given FP32 tensor scale of h
   ExpertPtrs w[NEXP];
 };
 
 // Shared-memory layout of one pipeline stage and of the whole CTA.  NCB = codebooks
-// per 256-channel stage: 2 when the QBlock is 128 wide along K, else 1.
-template <int FMT, int WSRC, int T, int NCB = 1>
+// per 256-channel stage: 2 when the QBlock is 128 wide along K, else 1.  NACC =
+// accumulators in TMEM (2 for the SwiGLU gate/up pair).
+template <int FMT, int WSRC, int T, int NCB = 1, int NACC = 1>
 struct StageLayout {
   static constexpr bool kVQ = WSRC != WSRC_NATIVE;
   static constexpr bool kSVQ = WSRC == WSRC_VQ_SVQ;
@@ -103,10 +112,11 @@ struct StageLayout {
   static constexpr int LUT_OFF = CTRL + STAGES * BYTES;
   static constexpr int RED_OFF = LUT_OFF + LUT;
   static constexpr int SMEM = 1024 + RED_OFF + RED;
-  // TMEM columns: accumulator [0,T), weight scales [T,T+16), token scales after.
-  static constexpr int COL_SFW = T;
-  static constexpr int COL_SFX = T + 16;
-  static constexpr int COLS_USED = T + 16 + 16 * kXG;
+  // TMEM columns: accumulators [0, NACC*T), weight scales [NACC*T, NACC*T+16), token
+  // scales after.
+  static constexpr int COL_SFW = NACC * T;
+  static constexpr int COL_SFX = NACC * T + 16;
+  static constexpr int COLS_USED = NACC * T + 16 + 16 * kXG;
   static constexpr int TMEM_COLS = COLS_USED <= 32 ? 32 : COLS_USED <= 64 ? 64 : COLS_USED <= 128 ? 128
                                    : COLS_USED <= 256 ? 256 : 512;
   static_assert(STAGES >= 2, "stage does not fit");
@@ -263,11 +273,12 @@ __device__ __forceinline__ void store_out(void* y, int64_t ldy, int out_bf16, in
 // ------------------------------------------------------------------------------------
 // The kernel
 // ------------------------------------------------------------------------------------
-template <int FMT, int WSRC, int T, bool MOE, int NCB>
+template <int FMT, int WSRC, int T, bool MOE, int NCB, bool SWI = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_wq,
                 const __grid_constant__ GemmParams<MOE ? kMaxGroups : 1> p) {
-  using L = StageLayout<FMT, WSRC, T, NCB>;
+  static_assert(!SWI || (MOE && T == 128), "SwiGLU runs on MoE gate/up tiles of 128 tokens");
+  using L = StageLayout<FMT, WSRC, T, NCB, SWI ? 2 : 1>;
   constexpr int STAGES = L::STAGES;
   constexpr int A = L::kAtoms;
   constexpr int XG = L::kXG;
@@ -315,6 +326,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     ks_end = min(KS, ks_begin + p.ks_per_split);
   }
   const int nks = ks_end - ks_begin;
+  // SwiGLU: the CTA runs the gate tile (weight rows of band n_tile) and then the up
+  // tile (band n_tile + F/128) over the same tokens: 2 * nks pipeline stages, the
+  // second pass into the second accumulator.
+  const int nst = SWI ? 2 * nks : nks;
+  const int up_band = SWI ? p.F / 128 : 0;
   // Loop invariants in registers (the asm statements below clobber "memory").
   const uint8_t* const w_idx = wp->idx;
   const uint16_t* const w_cb = wp->cb;
@@ -363,7 +379,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // =============================== loader ===============================
-    const int qbn = static_cast<int>((static_cast<int64_t>(n_tile) * 128) / qn);
     const int cb_per_row = K / qk;
     constexpr bool cb_split = NCB == 2;
     // Token scale groups that exist: the SF buffer holds ceil(M/128) groups of 128
@@ -389,18 +404,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (WSRC == WSRC_VQ_SVQ) tx += 8192 + (cb_split ? 1024 : 512) + 128 * L::kG;
     if constexpr (WSRC == WSRC_VQ_QBS) tx += 8192 + (cb_split ? 1024 : 512);
     const uint8_t* sfx_src = a_sf + static_cast<size_t>(sf_group0) * KB4 * 512;
-    const uint8_t* sfw_src = w_sf + static_cast<size_t>(n_tile) * KB4 * 512;
-    const uint8_t* idx_src = w_idx + static_cast<size_t>(n_tile) * KS * 8192;
-    const uint8_t* sidx_src = w_sidx + static_cast<size_t>(n_tile) * KS * (128 * L::kG);
-    const uint16_t* cb_src = w_cb + static_cast<size_t>(qbn) * cb_per_row * 256;
     const int y0 = static_cast<int>(m0);
     int issued = 0;
-    for (int i = 0; i < nks; ++i) {
+    for (int i = 0; i < nst; ++i) {
       const int s = i % STAGES;
       const uint32_t ph = (i / STAGES) & 1;
       if (i >= STAGES && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1))) break;
       if (elect_one()) {
-        const int ks = ks_begin + i;
+        const bool up = SWI && i >= nks;             // SwiGLU: second pass, the up tile
+        const int ks = ks_begin + (up ? i - nks : i);
+        const int band = n_tile + (up ? up_band : 0);
+        const int qbn = static_cast<int>((static_cast<int64_t>(band) * 128) / qn);
+        const uint8_t* sfw_src = w_sf + static_cast<size_t>(band) * KB4 * 512;
+        const uint8_t* idx_src = w_idx + static_cast<size_t>(band) * KS * 8192;
+        const uint8_t* sidx_src = w_sidx + static_cast<size_t>(band) * KS * (128 * L::kG);
+        const uint16_t* cb_src = w_cb + static_cast<size_t>(qbn) * cb_per_row * 256;
         uint8_t* st = stages + s * L::BYTES;
         mbar_arrive_expect_tx(&full[s], tx);
         for (int q = 0; q < x_boxes; ++q)
@@ -433,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&full[i % STAGES], (i / STAGES) & 1);
   } else if (warp == 1) {
     // ============================ MMA issuer ==============================
-    for (int i = 0; i < nks; ++i) {
+    for (int i = 0; i < nst; ++i) {
       const int s = i % STAGES;
       const uint32_t ph = (i / STAGES) & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) break;
@@ -466,20 +484,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_cp_32x128b_warpx4(tmem + L::COL_SFW + 4 * a, sdesc_sf_atom(sfw_s + a * 512));
         }
         const uint32_t w_s = smem_u32(st + L::W_OFF), x_s = smem_u32(st + L::X_OFF);
+        const bool up = SWI && i >= nks;             // SwiGLU: the up tile accumulates apart
+        const int il = up ? i - nks : i;
+        const uint32_t d_t = tmem + (up ? static_cast<uint32_t>(T) : 0u);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const uint64_t adesc = sdesc_kmajor_sw128(w_s + 32 * j);
           const uint64_t bdesc = sdesc_kmajor_sw128(x_s + 32 * j);
-          const uint32_t acc = (i > 0 || j > 0) ? 1u : 0u;
+          const uint32_t acc = (il > 0 || j > 0) ? 1u : 0u;
           if constexpr (FMT == FMT_E4M3) {
             constexpr uint32_t idesc = idesc_mxf4(T, 0, 0, 0);
-            tc_mma_mxf4nvf4_block16(tmem, adesc, bdesc, idesc, tmem + L::COL_SFW + 4 * j,
+            tc_mma_mxf4nvf4_block16(d_t, adesc, bdesc, idesc, tmem + L::COL_SFW + 4 * j,
                                     tmem + L::COL_SFX + (XG == 2 ? 8 * j : 4 * j), acc);
           } else {
             const int a = j >> 1;
             const uint32_t id = static_cast<uint32_t>(j & 1) * 2;
             const uint32_t idesc = idesc_mxf4(T, 1, static_cast<int>(id), static_cast<int>(id));
-            tc_mma_mxf4_block32(tmem, adesc, bdesc, idesc, (tmem + L::COL_SFW + 4 * a) | (id << 30),
+            tc_mma_mxf4_block32(d_t, adesc, bdesc, idesc, (tmem + L::COL_SFW + 4 * a) | (id << 30),
                                 (tmem + L::COL_SFX + (XG == 2 ? 8 * a : 4 * a)) | (id << 30), acc);
           }
         }
@@ -506,7 +527,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr int kBufs = 2 / G;                   // copy buffers per group
       const int grp = dt / GT, gt = dt - grp * GT;
       const int bar_id = 2 + grp;
-      const int qbn_w = static_cast<int>((static_cast<int64_t>(n_tile) * 128) / qn);   // QBlock row
       uint8_t* lut = smem + L::LUT_OFF + grp * kBufs * kBuf;
       const uint32_t lut_s = smem_u32(lut);
       ItemMap<GT> cm;
@@ -516,17 +536,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       bool ok = true;
       int b = 0;
-      if (grp < nks) {
+      if (grp < nst) {
         const bool got = mbar_wait(&full[grp % STAGES], (grp / STAGES) & 1);
         if (got) build_lut<GT>(stage_cb(grp), 1 + cb_split, reinterpret_cast<uint32_t*>(lut), gt);
         ok = named_bar_and(bar_id, GT, got);         // one decision for the group
       }
-      for (int i = grp; i < nks && ok; i += G) {
+      for (int i = grp; i < nst && ok; i += G) {
         const int s = i % STAGES;
         uint8_t* st = stages + s * L::BYTES;
         uint32_t qs0 = 0, qs1 = 0;                   // PostScale-QB: the stage's QBlock scale(s),
         if constexpr (L::kQBS) {                     // loaded before the decode hides their latency
-          const int ks = ks_begin + i;
+          const bool up = SWI && i >= nks;
+          const int ks = ks_begin + (up ? i - nks : i);
+          const int qbn_w = static_cast<int>((static_cast<int64_t>(n_tile + (up ? up_band : 0)) * 128) / qn);
           const uint8_t* qb = w_sf + static_cast<size_t>(qbn_w) * (K / qk);
           const int qbk = cb_split ? 2 * ks : (ks * kStageK) / qk;
           qs0 = __ldg(qb + qbk);
@@ -539,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&dec[s]);         // one arrival per decoder warp of the group
         const int in = i + G;
-        if (in < nks) {                              // this group's next stage
+        if (in < nst) {                              // this group's next stage
           if (kBufs == 1) named_bar_sync(bar_id, GT);   // lookups of stage i done before the rebuild
           const int nb = kBufs == 2 ? (b ^ 1) : 0;
           const bool got = mbar_wait(&full[in % STAGES], (in / STAGES) & 1);
@@ -560,7 +582,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t ldy = p.ldy;
     const int out_bf16 = p.out_bf16;
     const uint32_t taddr = tmem + (static_cast<uint32_t>(qd * 32) << 16) + chalf * TCOL;
-    if constexpr (T <= 32) {
+    if constexpr (SWI) {
+      // Gate accumulator at columns [0, T), up at [T, 2T): this thread holds channel
+      // `row` (a TMEM lane) of both for this warp's TCOL tokens.  Phase 1: h = SiLU(g) * u
+      // in FP32 into a [128 tokens][HS] staging table over the pipeline stages (all
+      // copies, decodes and MMAs are done by now).  Phase 2: each thread quantizes
+      // whole blocks (one token, B consecutive channels) for the down projection:
+      // FP4 codes into h_q, block scales into the grouped SF layout (padding rows of
+      // the expert's tile get zero scales).
+      constexpr int HS = 132;                          // padded rows: conflict-free 16-byte reads
+      static_assert(128 * HS * 4 <= STAGES * L::BYTES, "h staging fits in the pipeline stages");
+      float* const hst = reinterpret_cast<float*>(stages);
+      const bool wok = __all_sync(0xffffffffu, ep_ok);
+#pragma unroll 1
+      for (int c0 = 0; c0 < TCOL; c0 += 16) {
+        uint32_t vg[16], vu[16];
+        __syncwarp();                                  // tcgen05.ld is warp-aligned
+        tmem_ld_32x32b_x16(taddr + c0, vg);
+        tmem_ld_32x32b_x16(taddr + T + c0, vu);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          hst[(chalf * TCOL + c0 + c) * HS + row] =
+              swiglu_fp32(__fmul_rn(__uint_as_float(vg[c]), scale), __fmul_rn(__uint_as_float(vu[c]), scale));
+      }
+      named_bar_sync(4, kDecThreads);                  // the staging table is complete
+      if (wok) {
+        constexpr int B = L::kB, NB = 128 / B;         // blocks of one token in this tile
+        const float hs = FMT == FMT_E4M3 ? *p.h_tscale : 1.0f;
+        const int kbr = p.F / B;                       // h blocks per row
+        for (int u = threadIdx.x - 64; u < 128 * NB; u += kDecThreads) {
+          const int t = u & 127, b = u >> 7;
+          const int64_t m = m0 + t;
+          const float4* src = reinterpret_cast<const float4*>(hst + t * HS + b * B);
+          float v[B];
+#pragma unroll
+          for (int i = 0; i < B / 4; ++i) {
+            const float4 f = src[i];
+            v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
+          }
+          uint32_t q[B / 8], sfb;
+          quantize_block_f32<B>(v, FMT == FMT_E4M3, hs, q, sfb);
+          const int kb = n_tile * NB + b;              // block index along h's channels
+          if (m < m_end) {
+            uint8_t* dst = p.h_q + m * p.ldh + kb * (B / 2);
+            if constexpr (B == 32) *reinterpret_cast<uint4*>(dst) = make_uint4(q[0], q[1], q[2], q[3]);
+            else *reinterpret_cast<uint2*>(dst) = make_uint2(q[0], q[1]);
+          }
+          p.h_sf[sf_offset(static_cast<int64_t>(sf_group0) * 128 + t, kb, kbr)] =
+              static_cast<uint8_t>(m < m_end ? sfb : 0u);
+        }
+      }
+    } else if constexpr (T <= 32) {
       // this warp's accumulator columns in registers: one TMEM round trip
       __syncwarp();                                  // tcgen05.ld is warp-aligned: converge after the waits
       if constexpr (TCOL == 4) tmem_ld_32x32b_x4(taddr, acc_regs);

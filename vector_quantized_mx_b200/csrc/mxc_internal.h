@@ -67,6 +67,13 @@ struct MoeArgs {
   const int32_t* offsets;
   int32_t E;
   const mxc_weight* experts;    // host array
+  // gate/up with SwiGLU: h = SiLU(gate) * up quantized into the down projection's
+  // activation instead of writing y
+  int swiglu;
+  uint8_t* h_q;
+  int64_t ldh;
+  uint8_t* h_sf;
+  const float* h_tscale;
 };
 
 struct DecodeArgs {

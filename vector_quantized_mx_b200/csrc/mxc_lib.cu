@@ -353,9 +353,11 @@ mxc_status mxc_native_linear(const mxc_mx_tensor* a, const mxc_mx_tensor* w, voi
   return run_linear(L, reinterpret_cast<cudaStream_t>(stream));
 }
 
-// Argument checks shared by both grouped entry points, in one order of precedence.
-static mxc_status moe_prepare(const mxc_mx_tensor* a, const int32_t* d_offsets, const mxc_weight* experts, int32_t E,
-                              void* y, int64_t ldy, mxc_dtype y_dtype, MoeArgs* m) {
+// Argument checks shared by the grouped entry points, in one order of precedence
+// (activation, offsets and expert table, each expert, consistency); the output is
+// checked by the caller.
+static mxc_status moe_prepare_inputs(const mxc_mx_tensor* a, const int32_t* d_offsets, const mxc_weight* experts,
+                                     int32_t E, MoeArgs* m) {
   mxc_status s = check_mx_tensor(a);
   if (s != MXC_OK) return s;
   if (!d_offsets || !experts || E <= 0) return MXC_ERR_INVALID_ARG;
@@ -372,19 +374,26 @@ static mxc_status moe_prepare(const mxc_mx_tensor* a, const int32_t* d_offsets, 
   }
   const mxc_weight& w0 = experts[0];
   if (a->fmt != w0.fmt || a->K != w0.K) return MXC_ERR_INVALID_ARG;
-  if ((s = check_output(y, ldy, w0.N, y_dtype)) != MXC_OK) return s;
   *m = MoeArgs{};
   fill_activation(m->base, a);
   m->base.wsrc = wsrc_of(w0.strategy);
   m->base.N = w0.N;
   m->base.qn = qn;
   m->base.qk = qk;
-  m->base.y = y;
-  m->base.ldy = ldy;
-  m->base.out_bf16 = y_dtype == MXC_OUT_BF16;
   m->offsets = d_offsets;
   m->E = E;
   m->experts = experts;
+  return MXC_OK;
+}
+
+static mxc_status moe_prepare(const mxc_mx_tensor* a, const int32_t* d_offsets, const mxc_weight* experts, int32_t E,
+                              void* y, int64_t ldy, mxc_dtype y_dtype, MoeArgs* m) {
+  mxc_status s = moe_prepare_inputs(a, d_offsets, experts, E, m);
+  if (s != MXC_OK) return s;
+  if ((s = check_output(y, ldy, m->base.N, y_dtype)) != MXC_OK) return s;
+  m->base.y = y;
+  m->base.ldy = ldy;
+  m->base.out_bf16 = y_dtype == MXC_OUT_BF16;
   return MXC_OK;
 }
 
@@ -397,6 +406,29 @@ mxc_status mxc_moe_linear(const mxc_mx_tensor* a, const int32_t* d_offsets, cons
   if ((s = check_device()) != MXC_OK) return s;
   m.base.ws = ws;
   m.base.ws_bytes = ws_bytes;
+  return run_moe_linear(m, reinterpret_cast<cudaStream_t>(stream));
+}
+
+mxc_status mxc_moe_gate_up_swiglu(const mxc_mx_tensor* a, const int32_t* d_offsets, const mxc_weight* experts,
+                                  int32_t E, const float* h_tscale_in, uint8_t* h_q, int64_t ldh, uint8_t* h_sf,
+                                  void* ws, size_t ws_bytes, mxc_stream_t stream) {
+  MoeArgs m;
+  mxc_status s = moe_prepare_inputs(a, d_offsets, experts, E, &m);
+  if (s != MXC_OK) return s;
+  const int64_t F = m.base.N / 2;
+  if (m.base.N % 2 || F % kTileN) return MXC_ERR_ALIGNMENT;
+  if (!h_q || !h_sf) return MXC_ERR_INVALID_ARG;
+  if (ldh < F / 2 || ldh % 16 || !aligned16(h_q) || !aligned16(h_sf)) return MXC_ERR_ALIGNMENT;
+  if (a->fmt == MXC_FMT_E4M3_B16 && !h_tscale_in) return MXC_ERR_INVALID_ARG;
+  if (a->rows == 0) return MXC_OK;
+  if ((s = check_device()) != MXC_OK) return s;
+  m.base.ws = ws;
+  m.base.ws_bytes = ws_bytes;
+  m.swiglu = 1;
+  m.h_q = h_q;
+  m.ldh = ldh;
+  m.h_sf = h_sf;
+  m.h_tscale = h_tscale_in;
   return run_moe_linear(m, reinterpret_cast<cudaStream_t>(stream));
 }
 

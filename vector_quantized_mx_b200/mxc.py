@@ -31,7 +31,7 @@ EXPORTED = (
     "mxc_quantize_act_workspace_bytes", "mxc_linear_workspace_bytes", "mxc_moe_workspace_bytes",
     "mxc_grouped_sf_rows_bound", "mxc_quantize_act", "mxc_quantize_act_grouped", "mxc_linear",
     "mxc_native_linear", "mxc_moe_linear", "mxc_moe_linear_noalloc", "mxc_decode_weight", "mxc_get_device_error",
-    "mxc_selftest_wait_timeout",
+    "mxc_selftest_wait_timeout", "mxc_moe_gate_up_swiglu",
 )
 
 
@@ -97,6 +97,8 @@ def lib() -> ctypes.CDLL:
             "mxc_decode_weight": (ctypes.c_int, [ctypes.POINTER(_Weight), vp, i64, vp, vp]),
             "mxc_get_device_error": (ctypes.c_int, [vp]),
             "mxc_selftest_wait_timeout": (ctypes.c_int, [i64, vp]),
+            "mxc_moe_gate_up_swiglu": (ctypes.c_int, [ctypes.POINTER(_MxTensor), vp, ctypes.POINTER(_Weight), i32, vp,
+                                                      vp, i64, vp, vp, sz, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -332,6 +334,31 @@ def moe_linear(a: MXTensor, offsets: torch.Tensor, experts: Sequence[PackedWeigh
     _check(lib().mxc_moe_linear(ctypes.byref(at), offsets.data_ptr(), table, E, y.data_ptr(), y.stride(0),
                                 OUT[y.dtype], ws.data_ptr(), ws.numel(), _stream(stream)), "mxc_moe_linear")
     return y
+
+
+def moe_gate_up_swiglu(a: MXTensor, offsets: torch.Tensor, experts: Sequence[PackedWeight],
+                       h_tscale: Optional[torch.Tensor] = None, out: Optional[MXTensor] = None,
+                       ws: Optional[torch.Tensor] = None, stream=None) -> MXTensor:
+    """mxc_moe_gate_up_swiglu: gate/up projection, SwiGLU and the down projection's MX
+    quantization in one kernel.  Returns h as a grouped MXTensor (F = N/2 channels)
+    that moe_linear takes over the same offsets.  h_tscale (float32 [1], device) is
+    required for e4m3_b16."""
+    E = len(experts)
+    dev = a.q.device
+    F = experts[0].N // 2
+    if out is None:
+        out = empty_act_grouped(a.rows, F, E, a.fmt, dev)
+        if a.fmt == "e4m3_b16":
+            out.tscale = h_tscale
+    if ws is None:
+        ws = torch.empty((max(16, lib().mxc_moe_workspace_bytes(a.rows, E, experts[0].N, a.K, FMT[a.fmt])),),
+                         dtype=torch.uint8, device=dev)
+    table = (_Weight * E)(*[w._c() for w in experts])
+    at = a._c()
+    _check(lib().mxc_moe_gate_up_swiglu(ctypes.byref(at), offsets.data_ptr(), table, E, _ptr(h_tscale),
+                                        out.q.data_ptr(), out.q.stride(0), out.sf.data_ptr(), ws.data_ptr(),
+                                        ws.numel(), _stream(stream)), "mxc_moe_gate_up_swiglu")
+    return out
 
 
 def moe_linear_noalloc(a: MXTensor, offsets: torch.Tensor, experts: Sequence[PackedWeight],
