@@ -435,7 +435,7 @@ def rotated(pw0, n):
     from vector_quantized_mx_b200 import mxc
     cl = lambda t: None if t is None else t.clone()
     return [pw0] + [mxc.PackedWeight(pw0.fmt, pw0.strategy, pw0.N, pw0.K, pw0.qn, pw0.qk, pw0.idx.clone(),
-                                     pw0.cb.clone(), cl(pw0.scales), cl(pw0.sidx), cl(pw0.scb), pw0.w_tscale)
+                                     pw0.cb.clone(), cl(pw0.scales), cl(pw0.sidx), cl(pw0.scb), pw0.w_tscale, pw0.ds)
                     for _ in range(n - 1)]
 
 

@@ -118,12 +118,22 @@ typedef struct mxc_mx_tensor {
  *           (k mod 4) in bits 4t..4t+3.  512 bytes per QBlock.
  *   scales  device (PostScale/PreScale), SF layout of the [N, K/B] scale bytes;
  *           (MXC_POSTSCALE_QB) [N/qn][K/qk] bytes, one scale per QBlock.
- *   sidx    device (PreScale+), [N/128][K/256][128][256/(8B)] bytes: scale-codebook
- *           index of each group of 8 consecutive scales along K.
- *   scb     device (PreScale+), [256][8] scale bytes.
- *   qn, qk  QBlock size; 0 means the whole dimension.  qn must be a multiple
- *           of 128 (or N); qk must be 128 or a multiple of 256 (or K).
- *   w_tscale  FP32 tensor scale (E4M3-B16); use 1.0 for E8M0-B32. */
+ *   sidx    device (PreScale+), [N/128][U][128][G] bytes: the scale-codebook index
+ *           of each group of ds consecutive block scales along K (ds = scale_group).
+ *           With ds*B <= 256 a unit is one 256-channel stage holding G = 256/(ds*B)
+ *           groups of each row (U = K/256); with ds*B > 256 a unit is one group
+ *           (G = 1, U = K/(ds*B)).  Either way U*G = K/(ds*B).
+ *   scb     device (PreScale+), [256][ds] scale bytes.
+ *   qn, qk  QBlock size; 0 means the whole dimension.  qn must be 64 or a
+ *           multiple of 128 (or N); qk must be 64, 128 or a multiple of 256 (or K).
+ *           QBlocks of 64 rows or 64 input channels (down to 64 x 64, the fine end
+ *           of Figure 3's sweep) are decoded once per call into the workspace and
+ *           run on the native GEMM at every M (see mxc_linear_workspace_bytes_for);
+ *           the grouped (MoE) calls do not take them.
+ *   w_tscale  FP32 tensor scale (E4M3-B16); use 1.0 for E8M0-B32.
+ *   scale_group  PreScale+: ds, the block scales one scale index covers (Table 4
+ *           caption: 8; 16 and 32 are Figure 3's higher scale-compression ratios);
+ *           0 means 8.  K must be a multiple of ds*B.  Ignored by other strategies. */
 typedef struct mxc_weight {
   mxc_strategy strategy;
   mxc_format fmt;
@@ -134,12 +144,13 @@ typedef struct mxc_weight {
   const uint8_t* sidx;
   const uint8_t* scb;
   float w_tscale;
+  int32_t scale_group;
 } mxc_weight;
 
 /* The same weight in its logical host layout, as produced by a quantizer:
  *   idx [N, K/4] uint8, cb [N/qn, K/qk, 256] uint16, scales [N, K/B] uint8
- *   (direct), [N/qn, K/qk] uint8 (PostScale-QB), or sidx [N, K/(8B)] uint8 +
- *   scb [256, 8] uint8 (PreScale+). */
+ *   (direct), [N/qn, K/qk] uint8 (PostScale-QB), or sidx [N, K/(ds*B)] uint8 +
+ *   scb [256, ds] uint8 (PreScale+, ds = scale_group). */
 typedef struct mxc_weight_host {
   mxc_strategy strategy;
   mxc_format fmt;
@@ -150,6 +161,7 @@ typedef struct mxc_weight_host {
   const uint8_t* sidx;
   const uint8_t* scb;
   float w_tscale;
+  int32_t scale_group;
 } mxc_weight_host;
 
 /* Byte sizes of the packed buffers (host-side arithmetic only). */
@@ -187,6 +199,11 @@ mxc_status mxc_pack_weight(const mxc_weight_host* w, uint8_t* idx_out, uint8_t* 
 size_t mxc_quantize_act_workspace_bytes(int64_t M, int64_t K, mxc_format fmt);
 size_t mxc_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, mxc_format fmt);
 size_t mxc_moe_workspace_bytes(int64_t M, int32_t E, int64_t N, int64_t K, mxc_format fmt);
+/* The workspace mxc_linear needs for this weight at M rows: mxc_linear_workspace_bytes,
+ * except for QBlocks of 64 rows or 64 input channels, which need the decoded weight's
+ * room (N*K/2 rounded up to 1 KiB, plus N*K/B) at every M -- without it mxc_linear
+ * returns MXC_ERR_WORKSPACE for them.  0 for an invalid weight. */
+size_t mxc_linear_workspace_bytes_for(const mxc_weight* w, int64_t M);
 
 /* Rows of the SF layout that mxc_quantize_act_grouped writes:
  * sum over groups of ceil(rows_g / 128) * 128, bounded by M + 128*E. */

@@ -243,7 +243,9 @@ def weight_codes(w) -> np.ndarray:
 
 
 def weight_scale_bytes(w) -> np.ndarray:
-    """Block-scale bytes [N, K/B]: stored directly, scb[sidx[n, kb//8], kb % 8] (PreScale+),
+    """Block-scale bytes [N, K/B]: stored directly, scb[sidx[n, kb//ds], kb % ds] (PreScale+,
+    groups of ds consecutive scales along K; ds = 8 in Table 4's caption, larger ds are the
+    higher scale-compression ratios of Figure 3 (b, c); the weight's `ds`, 8 if it has none),
     or the QBlock's scale scales[n//qn, (kb*B)//qk] (PostScale-QB)."""
     if w.strategy == "postscale_qb":
         B = BLOCK[w.fmt]
@@ -254,7 +256,8 @@ def weight_scale_bytes(w) -> np.ndarray:
         KB = w.K // BLOCK[w.fmt]
         kb = np.arange(KB)[None, :]
         n = np.arange(w.N)[:, None]
-        return w.scb[w.sidx[n, kb // 8], kb % 8].astype(np.uint8)
+        ds = getattr(w, "ds", 8)
+        return w.scb[w.sidx[n, kb // ds], kb % ds].astype(np.uint8)
     return np.asarray(w.scales, dtype=np.uint8)
 
 

@@ -79,6 +79,34 @@ def test_pack_layouts(L, fmt, strategy):
         assert np.array_equal(mxc.sf_to_rows(h["scales"], N, K, fmt), w.scales)
 
 
+@pytest.mark.parametrize("fmt", ["e8m0_b32", "e4m3_b16"])
+@pytest.mark.parametrize("ds", [16, 32])
+def test_pack_scale_index_units(L, fmt, ds):
+    """PreScale+ with larger scale groups: the packed indices come in units of one
+    256-channel stage (G = 256/(ds*B) groups per row) or of one group spanning
+    ds*B/256 stages (G = 1); either way [N/128][U][128][G] with U*G = K/(ds*B)."""
+    B = synth.BLOCK[fmt]
+    N, K = 256, max(1024, 2 * ds * B)
+    w = synth.make_weight(8, fmt, "prescale_plus", N, K, 128, 256, ds=ds)
+    h = _pack(w)
+    row = K // (ds * B)
+    G = 256 // (ds * B) if ds * B <= 256 else 1
+    U = row // G
+    st = h["sidx"].reshape(N // 128, U, 128, G)
+    for nt in range(N // 128):
+        for u in range(U):
+            assert np.array_equal(st[nt, u], w.sidx[nt * 128:(nt + 1) * 128, u * G:(u + 1) * G])
+    assert h["scb"].size == 256 * ds
+    keep = []
+    hw = mxc._host_struct(w, keep)
+    sizes = mxc._PackedSizes()
+    assert L.mxc_packed_weight_sizes(ctypes.byref(hw), ctypes.byref(sizes)) == 0
+    assert sizes.sidx == N * row and sizes.scb == 256 * ds
+    for bad, status in ((12, 1), (64, 1)):              # only 8, 16 or 32
+        hw.scale_group = bad
+        assert L.mxc_packed_weight_sizes(ctypes.byref(hw), ctypes.byref(sizes)) == status
+
+
 def test_sf_layout_word_holds_one_row(L):
     """Each 32-bit word of the SF layout holds four consecutive scales of one row."""
     N, K = 128, 512
@@ -101,8 +129,11 @@ def test_packed_sizes_rejects_bad_shapes(L):
     hw.K = 500
     assert L.mxc_packed_weight_sizes(ctypes.byref(hw), ctypes.byref(sizes)) == 3   # alignment
     hw.K = 512
-    hw.qk = 64
-    assert L.mxc_packed_weight_sizes(ctypes.byref(hw), ctypes.byref(sizes)) == 3
+    for qn, qk, status in ((0, 32, 3), (0, 192, 3), (32, 0, 3), (192, 0, 3),   # QBlock sides the kernels refuse
+                           (64, 64, 0), (64, 0, 0), (0, 64, 0), (0, 128, 0), (128, 256, 0)):
+        hw.qn, hw.qk = qn, qk
+        assert L.mxc_packed_weight_sizes(ctypes.byref(hw), ctypes.byref(sizes)) == status, (qn, qk)
+    hw.qn = 0
     hw.qk = 0
     hw.fmt = 2
     assert L.mxc_packed_weight_sizes(ctypes.byref(hw), ctypes.byref(sizes)) == 2   # UE5M3 unsupported

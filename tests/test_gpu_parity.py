@@ -411,3 +411,97 @@ def test_decode_gemv_bf16_output(M):
     assert torch.equal(y16, yn)
     ref, sabs = O.w4a4_linear(x, w)
     assert_close(y16.float().cpu().numpy(), ref, sabs + np.abs(ref) * 2.0 ** -8 / TOL, what=f"bf16 M={M}")
+
+
+# ---------------------------------------------------------------------------
+# PreScale+ with larger scale groups (ds = 16, 32: Figure 3's higher scale
+# compression ratios), through every kernel path
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", ["e8m0_b32", "e4m3_b16"])
+@pytest.mark.parametrize("ds", [16, 32])
+@pytest.mark.parametrize("M", [16, 130, 1024])
+def test_prescale_plus_scale_groups(fmt, ds, M):
+    """Decoded weight bit-exact; decode GEMV (M=16), fused GEMM (M=130) and decode-once
+    (M=1024) within the oracle bound and equal to native FP4 on the decoded weight."""
+    N, K = 512, 2048
+    w = synth.make_weight(101, fmt, "prescale_plus", N, K, 256, 256, ds=ds)
+    pw, d = check_decode(w)
+    x = synth.make_activations(101, M, K, outliers=True)
+    a = mxc.quantize_act(dev_bf16(x), fmt)
+    y = mxc.linear(a, pw)
+    yn = mxc.native_linear(a, d)
+    assert mxc.get_device_error() == 0
+    assert torch.equal(y, yn)
+    rows = np.arange(M) if M <= 130 else np.arange(0, M, 7)
+    codes, sf, s = O.quantize_act(x, fmt)
+    a_hat = O.dequant_act(codes, sf, fmt, s)[rows]
+    w_hat = O.dequant_weight(w)
+    assert_close(y.cpu().numpy()[rows], O.linear(a_hat, w_hat), O.abs_linear(a_hat, w_hat),
+                 what=f"ds={ds} {fmt} M={M}")
+
+
+@pytest.mark.parametrize("ds", [16, 32])
+def test_moe_prescale_plus_scale_groups(ds):
+    E, N, K = 4, 256, 1024
+    counts = [3, 0, 140, 20]
+    offsets = np.concatenate([[0], np.cumsum(counts)])
+    ws = [synth.make_weight(102, "e8m0_b32", "prescale_plus", N, K, 256, 256, sub=e, ds=ds) for e in range(E)]
+    x = synth.make_activations(102, int(offsets[-1]), K, outliers=False)
+    off_d = torch.from_numpy(offsets.astype(np.int32)).cuda()
+    a = mxc.quantize_act_grouped(dev_bf16(x), "e8m0_b32", off_d)
+    y = mxc.moe_linear(a, off_d, [mxc.pack_weight(w) for w in ws]).cpu().numpy()
+    assert mxc.get_device_error() == 0
+    codes, sf, s = O.quantize_act(x, "e8m0_b32")
+    a_hat = O.dequant_act(codes, sf, "e8m0_b32", s)
+    for e in range(E):
+        r0, r1 = offsets[e], offsets[e + 1]
+        if r1 > r0:
+            w_hat = O.dequant_weight(ws[e])
+            assert_close(y[r0:r1], O.linear(a_hat[r0:r1], w_hat), O.abs_linear(a_hat[r0:r1], w_hat),
+                         what=f"moe ds={ds} expert {e}")
+
+
+# ---------------------------------------------------------------------------
+# QBlocks of 64 rows or 64 input channels (down to 64 x 64: Figure 3's sweep),
+# decoded once per call by the direct-lookup decode kernel
+# ---------------------------------------------------------------------------
+
+SMALL_QB = [("e8m0_b32", "prescale", 64, 64), ("e4m3_b16", "postscale", 64, 64),
+            ("e4m3_b16", "prescale_plus", 64, 256), ("e8m0_b32", "postscale_qb", 64, 64),
+            ("e4m3_b16", "postscale_qb", 128, 64), ("e8m0_b32", "prescale_plus", 128, 64),
+            ("e4m3_b16", "prescale", 64, 128)]
+
+
+@pytest.mark.parametrize("case", SMALL_QB, ids=lambda c: "-".join(map(str, c)))
+def test_small_qblock_decode_bitexact(case):
+    fmt, strat, qn, qk = case
+    check_decode(synth.make_weight(111, fmt, strat, 384, 1024, qn, qk))
+
+
+@pytest.mark.parametrize("case", SMALL_QB[:4], ids=lambda c: "-".join(map(str, c)))
+@pytest.mark.parametrize("M", [1, 16, 130])
+def test_small_qblock_linear(case, M):
+    fmt, strat, qn, qk = case
+    w = synth.make_weight(112, fmt, strat, 512, 1024, qn, qk)
+    x = synth.make_activations(112, M, 1024, outliers=True)
+    y, pw, a = run_mxcode(w, x)
+    ref, sabs = O.w4a4_linear(x, w)
+    assert_close(y.cpu().numpy(), ref, sabs, what=f"{case} M={M}")
+    assert torch.equal(y, mxc.native_linear(a, mxc.decode_weight(pw)))
+    # without the decode workspace the call refuses, and enqueues nothing
+    yy = torch.full_like(y, 3.0)
+    with pytest.raises(mxc.MxcError) as e:
+        mxc.linear(a, pw, y=yy, ws=torch.empty((16,), dtype=torch.uint8, device="cuda"))
+    assert e.value.status == 4                       # MXC_ERR_WORKSPACE
+    assert torch.all(yy == 3.0)
+
+
+def test_small_qblock_moe_is_refused():
+    w = mxc.pack_weight(synth.make_weight(113, "e8m0_b32", "prescale", 256, 512, 64, 64))
+    x = synth.make_activations(113, 8, 512, outliers=False)
+    off = torch.tensor([0, 8], dtype=torch.int32, device="cuda")
+    a = mxc.quantize_act_grouped(dev_bf16(x), "e8m0_b32", off)
+    with pytest.raises(mxc.MxcError) as e:
+        mxc.moe_linear(a, off, [w])
+    assert e.value.status == 2                       # MXC_ERR_UNSUPPORTED

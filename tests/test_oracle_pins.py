@@ -260,20 +260,28 @@ def test_weight_codes_round_trip(qn, qk):
 
 
 @pytest.mark.parametrize("fmt", ["e8m0_b32", "e4m3_b16"])
-def test_scale_vq_round_trip(fmt):
-    rng = np.random.default_rng(11)
+@pytest.mark.parametrize("ds", [8, 16, 32])
+def test_scale_vq_round_trip(fmt, ds):
+    """Scale VQ with groups of ds consecutive scales along K (Table 4 caption: ds = 8;
+    Figure 3 b, c: higher scale-compression ratios): block scales drawn from a palette
+    of ds-byte groups, encoded by an exact table written here, must come back."""
+    rng = np.random.default_rng(11 + ds)
     B = O.BLOCK[fmt]
-    N, K = 48, 8 * B * 6
-    palette = rng.integers(100, 140, size=(256, 8), dtype=np.uint8)
-    groups = rng.integers(0, 256, size=(N, K // (8 * B)))
+    N, K = 48, ds * B * 6
+    palette = rng.integers(100, 140, size=(256, ds), dtype=np.uint8)
+    groups = rng.integers(0, 256, size=(N, K // (ds * B)))
     target = palette[groups].reshape(N, K // B)
-    table, inv = np.unique(target.reshape(-1, 8), axis=0, return_inverse=True)
-    scb = np.zeros((256, 8), dtype=np.uint8)
+    table, inv = np.unique(target.reshape(-1, ds), axis=0, return_inverse=True)
+    scb = np.zeros((256, ds), dtype=np.uint8)
     scb[:len(table)] = table
-    sidx = inv.reshape(N, K // (8 * B)).astype(np.uint8)
+    sidx = inv.reshape(N, K // (ds * B)).astype(np.uint8)
     w = synth.VQWeight(fmt, "prescale_plus", N, K, N, K, np.zeros((N, K // 4), np.uint8),
-                       np.zeros((1, 1, 256), np.uint16), None, sidx, scb, 1.0)
+                       np.zeros((1, 1, 256), np.uint16), None, sidx, scb, 1.0, ds)
     assert np.array_equal(O.weight_scale_bytes(w), target)
+    # storage: one index byte per ds*B weights, plus the 256 x ds byte table
+    assert O.bits_per_weight(fmt, "prescale_plus", N, K, N, K, scale_group=ds) == pytest.approx(
+        8 / 4 + 4 * 4 * 256 / (N * K) + 8 / (ds * B) + 256 * ds * 8 / (N * K))
+    assert O.storage_bytes(w) == N * K // 4 + 512 + N * K // (ds * B) + 256 * ds
 
 
 # ---------------------------------------------------------------------------

@@ -79,7 +79,6 @@ struct GemvLayout {
   static constexpr bool kQBS = WSRC == WSRC_VQ_QBS;   // atoms built from one byte per QBlock
   static constexpr int kB = FMT == FMT_E8M0 ? 32 : 16;
   static constexpr int kAtoms = kStageK / kB / 4;      // scale atoms per 128 rows per stage
-  static constexpr int kG = kStageK / (8 * kB);        // PreScale+ scale groups per row per stage
   static constexpr int S = kGemvMaxStages;
   static constexpr int W_OFF = 0;                      // S x [128][128 B] FP4, 128-byte swizzle
   static constexpr int X_OFF = W_OFF + S * 16384;      // S x [16][128 B] FP4 token tiles
@@ -175,7 +174,7 @@ __global__ void __maxnreg__(64)
   const uint16_t* const w_cb = p.w.cb + static_cast<size_t>(qbn) * cb_per_row * 256;
   // direct scales: this slice's atoms in the SF layout (PostScale-QB indexes p.w.sf by QBlock)
   const uint8_t* const w_sf = p.w.sf + (static_cast<size_t>(n_tile) * KB4 + static_cast<size_t>(ks_begin) * A) * 512;
-  const uint8_t* const w_sidx = p.w.sidx + (static_cast<size_t>(n_tile) * KS + ks_begin) * (128 * L::kG);
+  const SvqGeom sv(p.w.ds, L::kB, KS);                // PreScale+ index units of this band
   const uint8_t* const a_sf =
       p.a_sf + (static_cast<size_t>(sf_group0) * KB4 + static_cast<size_t>(ks_begin) * A) * 512;
   const int red_off = L::IDX_OFF;                               // rank 0's receive area
@@ -229,7 +228,10 @@ __global__ void __maxnreg__(64)
         tma_load_2d(smem + L::W_OFF + s * 16384, &tmap_wq, (ks_begin + s) * 128, n_tile * 128, &full[s]);
       }
     }
-    if constexpr (L::kSVQ) l2_prefetch_bulk(w_sidx, static_cast<uint32_t>(nks) * 128 * L::kG);
+    if constexpr (L::kSVQ) {
+      const int u0 = ks_begin / sv.spu, u1 = (ks_end - 1) / sv.spu;
+      l2_prefetch_bulk(sv.unit(p.w.sidx, n_tile, ks_begin), static_cast<uint32_t>(u1 - u0 + 1) * 128 * sv.G);
+    }
   }
   if (warp == 1) {
     __syncwarp();                                    // tcgen05.alloc is warp-aligned
@@ -446,19 +448,21 @@ __global__ void __maxnreg__(64)
     auto svq_scales_to_tmem = [&]() {
       if constexpr (L::kSVQ) {
         __syncwarp();                                // tcgen05.st is warp-aligned
-        // PreScale+ (Table 4 caption: Ks = 256, ds = 8): row `lane` of atom (s, a)
-        // holds, for rows 32 g + lane (g = 0..3), scales 4a..4a+3 of stage s, i.e.
-        // word a mod 2 of the 8-byte scale-codebook entry of scale group a/2.
+        // PreScale+ (Table 4 caption: Ks = 256, ds = 8; larger ds compress further):
+        // row `lane` of atom (s, a) holds, for rows 32 g + lane (g = 0..3), block
+        // scales 4a..4a+3 of stage s: one word of the scale-codebook entry.
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(qd * 32) << 16);
         const uint32_t* scb32 = reinterpret_cast<const uint32_t*>(p.w.scb);
         for (int i = cg; i < nks * A; i += 4) {
           const int s = i / A, a = i % A;
-          const uint8_t* si = w_sidx + static_cast<size_t>(s) * 128 * L::kG + (a >> 1);
+          const int ks = ks_begin + s;
+          const uint8_t* un = sv.unit(p.w.sidx, n_tile, ks);
+          const int kb = sv.kb_base(ks, L::kB) + 4 * a;
           uint4 v;
-          v.x = __ldg(scb32 + 2 * __ldg(si + (0 * 32 + lane) * L::kG) + (a & 1));
-          v.y = __ldg(scb32 + 2 * __ldg(si + (1 * 32 + lane) * L::kG) + (a & 1));
-          v.z = __ldg(scb32 + 2 * __ldg(si + (2 * 32 + lane) * L::kG) + (a & 1));
-          v.w = __ldg(scb32 + 2 * __ldg(si + (3 * 32 + lane) * L::kG) + (a & 1));
+          v.x = svq_word(un + (0 * 32 + lane) * sv.G, scb32, sv.ds, kb);
+          v.y = svq_word(un + (1 * 32 + lane) * sv.G, scb32, sv.ds, kb);
+          v.z = svq_word(un + (2 * 32 + lane) * sv.G, scb32, sv.ds, kb);
+          v.w = svq_word(un + (3 * 32 + lane) * sv.G, scb32, sv.ds, kb);
           tmem_st_32x32b_x4(lane_base + L::COL_SFW + 4 * i, v);
         }
         tmem_st_wait();

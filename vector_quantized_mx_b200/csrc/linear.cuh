@@ -196,6 +196,15 @@ size_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt) {
   return M >= kDecodeOnceMinM ? decoded_weight_bytes(N, K, fmt) : 0;
 }
 
+// QBlocks of 64 rows or 64 input channels: a 128 x 256 tile-stage draws on up to 8
+// codebooks, more than the fused decoders' per-lane copies hold, so such weights are
+// always decoded once (by the direct-lookup decode kernel) and run on the native GEMM.
+inline bool small_qblock(int64_t qn, int64_t qk) { return qn < kTileN || qk < 128; }
+
+size_t linear_workspace_bytes_for(int64_t M, int64_t N, int64_t K, int fmt, int64_t qn, int64_t qk) {
+  return small_qblock(qn, qk) ? decoded_weight_bytes(N, K, fmt) : linear_workspace_bytes(M, N, K, fmt);
+}
+
 size_t moe_workspace_bytes(int64_t /*M*/, int32_t E, int64_t /*N*/, int64_t /*K*/, int /*fmt*/) {
   return align_up(static_cast<size_t>(E + 1) * sizeof(int32_t), 256);
 }
@@ -306,14 +315,18 @@ inline ExpertPtrs expert_ptrs(const LinearArgs& a) {
   e.sidx = a.w_sidx;
   e.scb = a.w_scb;
   e.w_tscale = a.w_tscale;
+  e.ds = a.w_ds;
   return e;
 }
 
 mxc_status run_decode_weight(const DecodeArgs& a, cudaStream_t stream);
 
 mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
-  if (a.wsrc != WSRC_NATIVE && a.M >= kDecodeOnceMinM && a.ws &&
-      a.ws_bytes >= decoded_weight_bytes(a.N, a.K, a.fmt) && reinterpret_cast<uintptr_t>(a.ws) % 16 == 0) {
+  const bool small = a.wsrc != WSRC_NATIVE && small_qblock(a.qn, a.qk);
+  const bool ws_ok = a.ws && a.ws_bytes >= decoded_weight_bytes(a.N, a.K, a.fmt) &&
+                     reinterpret_cast<uintptr_t>(a.ws) % 16 == 0;
+  if (small && !ws_ok) return MXC_ERR_WORKSPACE;
+  if (a.wsrc != WSRC_NATIVE && (small || a.M >= kDecodeOnceMinM) && ws_ok) {
     // decode once into the workspace, then the native GEMM on the decoded operands
     DecodeArgs d{};
     d.wsrc = a.wsrc;
@@ -327,6 +340,7 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
     d.w_sf = a.w_sf;
     d.w_sidx = a.w_sidx;
     d.w_scb = a.w_scb;
+    d.ds = a.w_ds;
     d.q_out = static_cast<uint8_t*>(a.ws);
     d.ldq = a.K / 2;
     d.sf_out = static_cast<uint8_t*>(a.ws) + decoded_codes_bytes(a.N, a.K);
@@ -448,6 +462,7 @@ mxc_status run_moe_linear(const MoeArgs& m, cudaStream_t stream) {
     p.w[e].sidx = w.sidx;
     p.w[e].scb = w.scb;
     p.w[e].w_tscale = w.w_tscale;
+    p.w[e].ds = w.scale_group ? w.scale_group : 8;
   }
   cudaError_t err;
   if (m.swiglu) {
@@ -495,14 +510,43 @@ cudaError_t launch_decode_dump(const DecodeArgs& a, cudaStream_t stream) {
   w.sf = a.w_sf;
   w.sidx = a.w_sidx;
   w.scb = a.w_scb;
+  w.ds = a.ds;
   const dim3 grid(static_cast<unsigned>(a.N / kTileN), static_cast<unsigned>(a.K / kStageK));
   kern<<<grid, 160, smem, stream>>>(w, static_cast<int>(a.N), static_cast<int>(a.K), static_cast<int>(a.qn),
                                     static_cast<int>(a.qk), a.q_out, a.ldq, a.sf_out);
   return cudaGetLastError();
 }
 
+template <int FMT, int WSRC>
+cudaError_t launch_decode_dump_small(const DecodeArgs& a, cudaStream_t stream) {
+  ExpertPtrs w{};
+  w.idx = a.w_idx;
+  w.cb = a.w_cb;
+  w.sf = a.w_sf;
+  w.sidx = a.w_sidx;
+  w.scb = a.w_scb;
+  w.ds = a.ds;
+  const dim3 grid(static_cast<unsigned>(a.N / kTileN), static_cast<unsigned>(a.K / kStageK));
+  decode_dump_small_kernel<FMT, WSRC><<<grid, 128, 0, stream>>>(w, static_cast<int>(a.N), static_cast<int>(a.K),
+                                                                static_cast<int>(a.qn), static_cast<int>(a.qk),
+                                                                a.q_out, a.ldq, a.sf_out);
+  return cudaGetLastError();
+}
+
 mxc_status run_decode_weight(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t err;
+  if (small_qblock(a.qn, a.qk)) {
+    if (a.fmt == FMT_E8M0) {
+      err = a.wsrc == WSRC_VQ_SVQ   ? launch_decode_dump_small<FMT_E8M0, WSRC_VQ_SVQ>(a, stream)
+            : a.wsrc == WSRC_VQ_QBS ? launch_decode_dump_small<FMT_E8M0, WSRC_VQ_QBS>(a, stream)
+                                    : launch_decode_dump_small<FMT_E8M0, WSRC_VQ_DIRECT>(a, stream);
+    } else {
+      err = a.wsrc == WSRC_VQ_SVQ   ? launch_decode_dump_small<FMT_E4M3, WSRC_VQ_SVQ>(a, stream)
+            : a.wsrc == WSRC_VQ_QBS ? launch_decode_dump_small<FMT_E4M3, WSRC_VQ_QBS>(a, stream)
+                                    : launch_decode_dump_small<FMT_E4M3, WSRC_VQ_DIRECT>(a, stream);
+    }
+    return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
+  }
   if (a.fmt == FMT_E8M0) {
     err = a.wsrc == WSRC_VQ_SVQ   ? launch_decode_dump<FMT_E8M0, WSRC_VQ_SVQ>(a, stream)
           : a.wsrc == WSRC_VQ_QBS ? launch_decode_dump<FMT_E8M0, WSRC_VQ_QBS>(a, stream)

@@ -55,7 +55,7 @@ struct ExpertPtrs {
   const uint8_t* sidx;   // PreScale+ scale indices (packed tiles)
   const uint8_t* scb;    // PreScale+ scale codebook [256][8]
   float w_tscale;
-  int pad_;
+  int ds;                // PreScale+ scale group (block scales per scale index)
 };
 
 template <int NEXP>
@@ -94,7 +94,7 @@ struct StageLayout {
   static constexpr int kB = FMT == FMT_E8M0 ? 32 : 16;
   static constexpr int kAtoms = kStageK / kB / 4;     // scale atoms per 128 rows per stage
   static constexpr int kXG = (T + 127) / 128;         // 128-row scale groups in the token tile
-  static constexpr int kG = kStageK / (8 * kB);       // PreScale+ scale groups per row per stage
+  static constexpr int kG = kStageK / (8 * kB);       // PreScale+ index bytes per row per stage, at most
   static constexpr int W_OFF = 0;
   static constexpr int X_OFF = 16384;
   static constexpr int SFW_OFF = X_OFF + T * 128;
@@ -212,20 +212,44 @@ __device__ __forceinline__ void decode_w_tile(const uint8_t* __restrict__ idx, u
   }
 }
 
-// PreScale+ (Table 4 caption: Ks = 256, ds = 8): each scale-codebook index
-// selects 8 scale bytes, i.e. two 32-bit words of the scale-factor atoms (kb
-// 8g..8g+3 -> atom 2g, kb 8g+4..8g+7 -> atom 2g+1).  128 rows x G groups.
-template <int G, int NT>
-__device__ __forceinline__ void decode_sf_tile(const uint8_t* __restrict__ sidx,
-                                               const uint8_t* __restrict__ scb, uint8_t* __restrict__ sfw,
-                                               int dt) {
-  for (int u = dt; u < 128 * G; u += NT) {   // consecutive threads: consecutive atom words
-    const int word = u & 127, g = u >> 7;
+// PreScale+ (Table 4 caption: Ks = 256 entries, ds = 8; Figure 3 b, c: larger ds
+// compress the scales further): one scale-codebook index per group of ds
+// consecutive block scales of a row.  The packed indices of a 128-row band come in
+// units: one 256-channel stage with G = 256/(ds*B) groups per row when ds*B <= 256,
+// else one group (G = 1) spanning spu = ds*B/256 stages.
+struct SvqGeom {
+  int ds, G, spu, U;
+  __device__ __forceinline__ SvqGeom(int ds_, int B, int KS) {   // ds_ <= 0 (no scale VQ): the default 8
+    ds = ds_ > 0 ? ds_ : 8;
+    G = max(1, kStageK / (ds * B));
+    spu = max(1, ds * B / kStageK);
+    U = KS / spu;
+  }
+  // the unit of the band's indices that holds stage ks: [128][G] bytes
+  __device__ __forceinline__ const uint8_t* unit(const uint8_t* sidx, int band, int ks) const {
+    return sidx + (static_cast<size_t>(band) * U + ks / spu) * 128 * G;
+  }
+  // first block of stage ks within its unit
+  __device__ __forceinline__ int kb_base(int ks, int B) const { return (ks % spu) * (kStageK / B); }
+};
+
+// The 32-bit word of block scales kb..kb+3 (kb a multiple of 4, counted from the
+// unit's first block) of one row: word (kb mod ds)/4 of the entry that the row's
+// index for group kb/ds selects.  Generic loads: the indices and the table may sit
+// in shared or global memory.
+__device__ __forceinline__ uint32_t svq_word(const uint8_t* row_idx, const uint32_t* scb32, int ds, int kb) {
+  return scb32[static_cast<uint32_t>(row_idx[kb / ds]) * (ds / 4) + (kb % ds) / 4];
+}
+
+// A stage's weight scale atoms (A atoms of 128 rows x 4 blocks, the tcgen05 scale
+// layout) from the unit's indices; kb0 = the stage's first block within the unit.
+template <int A, int NT>
+__device__ __forceinline__ void decode_sf_tile(const uint8_t* sidx, int G, const uint32_t* scb32, int ds, int kb0,
+                                               uint8_t* __restrict__ sfw, int dt) {
+  for (int u = dt; u < 128 * A; u += NT) {   // consecutive threads: consecutive atom words
+    const int word = u & 127, a = u >> 7;
     const int r = (word >> 2) + 32 * (word & 3);
-    const uint32_t si = sidx[r * G + g];
-    const uint2 s8 = *reinterpret_cast<const uint2*>(scb + si * 8);
-    reinterpret_cast<uint32_t*>(sfw + (2 * g) * 512)[word] = s8.x;
-    reinterpret_cast<uint32_t*>(sfw + (2 * g + 1) * 512)[word] = s8.y;
+    reinterpret_cast<uint32_t*>(sfw + a * 512)[word] = svq_word(sidx + r * G, scb32, ds, kb0 + 4 * a);
   }
 }
 
@@ -358,9 +382,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, L::TMEM_COLS);
     tmem_relinquish();
   }
+  // PreScale+: the scale codebook (256 x ds bytes) in shared memory when it is the
+  // 2 KB of ds = 8, else read in place (through L1)
+  const SvqGeom sv(wp->ds, L::kB, KS);
+  const int sv_ds = sv.ds;
+  const uint32_t* const scb32 = sv_ds == 8 ? reinterpret_cast<const uint32_t*>(scb_smem)
+                                           : reinterpret_cast<const uint32_t*>(w_scb);
   if constexpr (L::kSVQ) {
-    for (int i = threadIdx.x; i < 512; i += kThreads)
-      reinterpret_cast<uint32_t*>(scb_smem)[i] = __ldg(reinterpret_cast<const uint32_t*>(w_scb) + i);
+    if (sv_ds == 8)
+      for (int i = threadIdx.x; i < 512; i += kThreads)
+        reinterpret_cast<uint32_t*>(scb_smem)[i] = __ldg(reinterpret_cast<const uint32_t*>(w_scb) + i);
   }
   tc_fence_before();
   __syncthreads();
@@ -401,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t tx = x_boxes * x_box_bytes + xg_valid * A * 512;
     if constexpr (WSRC == WSRC_NATIVE) tx += 16384 + A * 512;
     if constexpr (WSRC == WSRC_VQ_DIRECT) tx += 8192 + (cb_split ? 1024 : 512) + A * 512;
-    if constexpr (WSRC == WSRC_VQ_SVQ) tx += 8192 + (cb_split ? 1024 : 512) + 128 * L::kG;
+    if constexpr (WSRC == WSRC_VQ_SVQ) tx += 8192 + (cb_split ? 1024 : 512) + 128 * sv.G;
     if constexpr (WSRC == WSRC_VQ_QBS) tx += 8192 + (cb_split ? 1024 : 512);
     const uint8_t* sfx_src = a_sf + static_cast<size_t>(sf_group0) * KB4 * 512;
     const int y0 = static_cast<int>(m0);
@@ -417,7 +448,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qbn = static_cast<int>((static_cast<int64_t>(band) * 128) / qn);
         const uint8_t* sfw_src = w_sf + static_cast<size_t>(band) * KB4 * 512;
         const uint8_t* idx_src = w_idx + static_cast<size_t>(band) * KS * 8192;
-        const uint8_t* sidx_src = w_sidx + static_cast<size_t>(band) * KS * (128 * L::kG);
         const uint16_t* cb_src = w_cb + static_cast<size_t>(qbn) * cb_per_row * 256;
         uint8_t* st = stages + s * L::BYTES;
         mbar_arrive_expect_tx(&full[s], tx);
@@ -438,8 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (WSRC == WSRC_VQ_DIRECT) {
             bulk_load(st + L::SFW_OFF, sfw_src + static_cast<size_t>(ks) * A * 512, A * 512, &full[s]);
           } else if constexpr (WSRC == WSRC_VQ_SVQ) {
-            bulk_load(st + L::SIDX_OFF, sidx_src + static_cast<size_t>(ks) * (128 * L::kG), 128 * L::kG,
-                      &full[s]);
+            bulk_load(st + L::SIDX_OFF, sv.unit(w_sidx, band, ks), 128 * sv.G, &full[s]);
           }                                        // PostScale-QB: the decoders write the atoms
         }
       }
@@ -555,7 +584,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           qs1 = __ldg(qb + qbk + (cb_split ? 1 : 0));
         }
         decode_w_tile<GT>(st + L::IDX_OFF, lut_s + b * kBuf, st + L::W_OFF, cm);
-        if constexpr (L::kSVQ) decode_sf_tile<L::kG, GT>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, gt);
+        if constexpr (L::kSVQ) {
+          const int ks = ks_begin + (SWI && i >= nks ? i - nks : i);
+          decode_sf_tile<A, GT>(st + L::SIDX_OFF, sv.G, scb32, sv_ds, sv.kb_base(ks, L::kB), st + L::SFW_OFF, gt);
+        }
         if constexpr (L::kQBS) fill_sf_qbs<A, GT>(st + L::SFW_OFF, qs0, qs1, gt);
         fence_proxy_async_smem();                    // each thread's tile writes -> async proxy
         __syncwarp();
@@ -730,15 +762,19 @@ __global__ void __launch_bounds__(160)
     mbar_init(bar, 1);
     fence_mbar_init();
   }
+  const SvqGeom sv(w.ds, L::kB, KS);
+  const uint32_t* const scb32 = sv.ds == 8 ? reinterpret_cast<const uint32_t*>(scb_smem)
+                                           : reinterpret_cast<const uint32_t*>(w.scb);
   if constexpr (L::kSVQ) {
-    for (int i = threadIdx.x; i < 512; i += 160)
-      reinterpret_cast<uint32_t*>(scb_smem)[i] = __ldg(reinterpret_cast<const uint32_t*>(w.scb) + i);
+    if (sv.ds == 8)
+      for (int i = threadIdx.x; i < 512; i += 160)
+        reinterpret_cast<uint32_t*>(scb_smem)[i] = __ldg(reinterpret_cast<const uint32_t*>(w.scb) + i);
   }
   __syncthreads();
   const size_t tile_id = static_cast<size_t>(n_tile) * KS + ks;
   const size_t wsf = (static_cast<size_t>(n_tile) * KB4 + static_cast<size_t>(ks) * A) * 512;
   if (threadIdx.x == 0) {
-    const uint32_t tx = 8192 + (cb_split ? 1024 : 512) + (L::kSVQ ? 128 * L::kG : L::kQBS ? 0 : A * 512);
+    const uint32_t tx = 8192 + (cb_split ? 1024 : 512) + (L::kSVQ ? 128 * sv.G : L::kQBS ? 0 : A * 512);
     mbar_arrive_expect_tx(bar, tx);
     bulk_load(st + L::IDX_OFF, w.idx + tile_id * 8192, 8192, bar);
     const int qbn = static_cast<int>((static_cast<int64_t>(n_tile) * 128) / qn);
@@ -746,7 +782,7 @@ __global__ void __launch_bounds__(160)
     bulk_load(st + L::CB_OFF, w.cb + (static_cast<size_t>(qbn) * (K / qk) + qbk) * 256, cb_split ? 1024 : 512,
               bar);
     if constexpr (L::kSVQ) {
-      bulk_load(st + L::SIDX_OFF, w.sidx + tile_id * (128 * L::kG), 128 * L::kG, bar);
+      bulk_load(st + L::SIDX_OFF, sv.unit(w.sidx, n_tile, ks), 128 * sv.G, bar);
     } else if constexpr (!L::kQBS) {
       bulk_load(st + L::SFW_OFF, w.sf + wsf, A * 512, bar);
     }
@@ -759,7 +795,8 @@ __global__ void __launch_bounds__(160)
     ItemMap<128> cm;
     cm.init(dt, cb_split);
     decode_w_tile<128>(st + L::IDX_OFF, smem_u32(lut), st + L::W_OFF, cm);
-    if constexpr (L::kSVQ) decode_sf_tile<L::kG, 128>(st + L::SIDX_OFF, scb_smem, st + L::SFW_OFF, dt);
+    if constexpr (L::kSVQ)
+      decode_sf_tile<A, 128>(st + L::SIDX_OFF, sv.G, scb32, sv.ds, sv.kb_base(ks, L::kB), st + L::SFW_OFF, dt);
     if constexpr (L::kQBS) {
       const uint8_t* qb = w.sf + static_cast<size_t>((static_cast<int64_t>(n_tile) * 128) / qn) * (K / qk);
       const int qbk = cb_split ? 2 * ks : (ks * kStageK) / qk;
@@ -776,6 +813,78 @@ __global__ void __launch_bounds__(160)
     }
     for (int i = dt; i < A * 32; i += 128)
       reinterpret_cast<uint4*>(sf_out + wsf)[i] = reinterpret_cast<const uint4*>(st + L::SFW_OFF)[i];
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// Decode dump for small QBlocks (64 rows or 64 input channels, down to 64 x 64: the fine
+// end of Figure 3's QBlock sweep).  A 128 x 256 tile-stage then draws on up to 8
+// codebooks ([2 row halves][4 K-quarters]), too many for per-lane codebook copies, so
+// the stage's codebooks sit once in shared memory and every index is looked up
+// directly (bank conflicts allowed).  Writes the same plain layouts as
+// decode_dump_kernel: FP4 codes [N, ldq], SF-layout scales.  Grid (N/128, K/256).
+// ------------------------------------------------------------------------------------
+template <int FMT, int WSRC>
+__global__ void __launch_bounds__(128)
+    decode_dump_small_kernel(const ExpertPtrs w, int N, int K, int qn, int qk, uint8_t* __restrict__ q_out,
+                             int64_t ldq, uint8_t* __restrict__ sf_out) {
+  constexpr int B = FMT == FMT_E8M0 ? 32 : 16;
+  constexpr int A = kStageK / B / 4;                   // scale atoms per 128 rows per stage
+  __shared__ uint16_t cbs[8 * 256];
+  const int n_tile = blockIdx.x, ks = blockIdx.y, KS = K / kStageK;
+  const int rows_cb = qn < kTileN ? kTileN / qn : 1;   // codebook rows in the 128-row tile
+  const int qke = qk < kStageK ? qk : kStageK;
+  const int nkq = kStageK / qke;                       // codebooks along K in the stage
+  const int qbn0 = static_cast<int>((static_cast<int64_t>(n_tile) * kTileN) / qn);
+  const int qbk0 = static_cast<int>((static_cast<int64_t>(ks) * kStageK) / qk);
+  // the stage's codebooks, [rows_cb][nkq][256] entries (at most 8 x 512 bytes)
+  for (int i = threadIdx.x; i < rows_cb * nkq * 128; i += 128) {
+    const int c = i >> 7, wd = i & 127, rh = c / nkq, kq = c % nkq;
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(
+        w.cb + (static_cast<size_t>(qbn0 + rh) * (K / qk) + qbk0 + kq) * 256);
+    reinterpret_cast<uint32_t*>(cbs)[i] = __ldg(src + wd);
+  }
+  __syncthreads();
+  // item (r, q): the 16 indices of row r in K-quarter q -> 32 bytes of FP4 codes
+  const uint8_t* tile = w.idx + (static_cast<size_t>(n_tile) * KS + ks) * 8192;
+  for (int it = threadIdx.x; it < 512; it += 128) {
+    const int r = it & 127, q = it >> 7;
+    const uint16_t* cb = cbs + ((r / (kTileN / rows_cb)) * nkq + (q * 64) / qke) * 256;
+    const uint4 iv = ldg_nc_v4(tile + q * 2048 + r * 16);
+    const uint32_t x[4] = {iv.x, iv.y, iv.z, iv.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t b = x[j >> 1] >> (16 * (j & 1));
+      o[j] = static_cast<uint32_t>(cb[b & 0xFF]) | (static_cast<uint32_t>(cb[(b >> 8) & 0xFF]) << 16);
+    }
+    uint8_t* dst = q_out + (static_cast<int64_t>(n_tile) * kTileN + r) * ldq + static_cast<int64_t>(ks) * 128 + q * 32;
+    *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(dst + 16) = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+  // the tile-stage's scale atoms in the SF layout
+  const size_t wsf = (static_cast<size_t>(n_tile) * (K / B / 4) + static_cast<size_t>(ks) * A) * 512;
+  if constexpr (WSRC == WSRC_VQ_DIRECT) {
+    for (int i = threadIdx.x; i < A * 32; i += 128)
+      reinterpret_cast<uint4*>(sf_out + wsf)[i] = ldg_nc_v4(w.sf + wsf + static_cast<size_t>(i) * 16);
+  } else if constexpr (WSRC == WSRC_VQ_SVQ) {
+    const SvqGeom sv(w.ds, B, KS);
+    decode_sf_tile<A, 128>(sv.unit(w.sidx, n_tile, ks), sv.G, reinterpret_cast<const uint32_t*>(w.scb), sv.ds,
+                           sv.kb_base(ks, B), sf_out + wsf, threadIdx.x);
+  } else {
+    // PostScale-QB: word (r % 32) * 4 + g of atom a holds the scales of rows 32 g + r % 32
+    // (one QBlock row: qn >= 64) for blocks 4a..4a+3, each from its QBlock
+    for (int i = threadIdx.x; i < A * 128; i += 128) {
+      const int a = i >> 7, g = i & 3;
+      const int qbn = static_cast<int>((static_cast<int64_t>(n_tile) * kTileN + 32 * g) / qn);
+      uint32_t v = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int64_t c = static_cast<int64_t>(ks) * kStageK + static_cast<int64_t>(4 * a + b) * B;
+        v |= static_cast<uint32_t>(__ldg(w.sf + static_cast<size_t>(qbn) * (K / qk) + c / qk)) << (8 * b);
+      }
+      reinterpret_cast<uint32_t*>(sf_out + wsf)[i] = v;
+    }
   }
 }
 

@@ -52,6 +52,7 @@ struct LinearArgs {
   const uint8_t* w_q;           // native
   int64_t w_ldq;                // native
   float w_tscale;
+  int w_ds;                     // PreScale+ scale group
   const float* w_tscale_dev;    // native (device) or null
   // output
   void* y;
@@ -84,6 +85,7 @@ struct DecodeArgs {
   const uint8_t* w_sf;
   const uint8_t* w_sidx;
   const uint8_t* w_scb;
+  int ds;                       // PreScale+ scale group
   uint8_t* q_out;
   int64_t ldq;
   uint8_t* sf_out;
@@ -94,6 +96,7 @@ mxc_status run_moe_linear(const MoeArgs& a, cudaStream_t stream);
 mxc_status run_decode_weight(const DecodeArgs& a, cudaStream_t stream);
 
 size_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt);
+size_t linear_workspace_bytes_for(int64_t M, int64_t N, int64_t K, int fmt, int64_t qn, int64_t qk);
 size_t moe_workspace_bytes(int64_t M, int32_t E, int64_t N, int64_t K, int fmt);
 
 }  // namespace mxc

@@ -36,8 +36,10 @@ mxc_status resolve_qblock(int64_t N, int64_t K, int64_t qn_in, int64_t qk_in, in
   *qn = qn_in ? qn_in : N;
   *qk = qk_in ? qk_in : K;
   if (*qn <= 0 || *qk <= 0) return MXC_ERR_INVALID_ARG;
-  if (*qn % kTileN || N % *qn) return MXC_ERR_ALIGNMENT;
-  if (!(*qk == 128 || *qk % kStageK == 0) || K % *qk) return MXC_ERR_ALIGNMENT;
+  // 64 rows or 64 input channels (down to 64 x 64), 128 input channels, or multiples
+  // of the 128-row tile and the 256-channel stage
+  if ((*qn != 64 && *qn % kTileN) || N % *qn) return MXC_ERR_ALIGNMENT;
+  if (!(*qk == 64 || *qk == 128 || *qk % kStageK == 0) || K % *qk) return MXC_ERR_ALIGNMENT;
   return MXC_OK;
 }
 
@@ -53,20 +55,32 @@ mxc_status check_shape(int64_t N, int64_t K) {
   return MXC_OK;
 }
 
+// PreScale+ scale group: 0 means 8 (Table 4 caption); 16 and 32 are the higher
+// scale-compression ratios of Figure 3; K must hold whole groups.
+mxc_status resolve_scale_group(mxc_strategy strategy, mxc_format fmt, int64_t K, int32_t sg, int* ds) {
+  *ds = 8;
+  if (strategy != MXC_PRESCALE_PLUS) return MXC_OK;
+  *ds = sg ? sg : 8;
+  if (*ds != 8 && *ds != 16 && *ds != 32) return MXC_ERR_INVALID_ARG;
+  if (K % (static_cast<int64_t>(*ds) * block_of(fmt))) return MXC_ERR_ALIGNMENT;
+  return MXC_OK;
+}
+
 mxc_status check_weight_common(mxc_strategy strategy, mxc_format fmt, int64_t N, int64_t K, int64_t qn, int64_t qk,
-                               int64_t* rqn, int64_t* rqk) {
+                               int32_t sg, int64_t* rqn, int64_t* rqk, int* ds) {
   mxc_status s = check_format(fmt);
   if (s != MXC_OK) return s;
   if (strategy != MXC_POSTSCALE && strategy != MXC_PRESCALE && strategy != MXC_PRESCALE_PLUS &&
       strategy != MXC_POSTSCALE_QB)
     return MXC_ERR_INVALID_ARG;
   if ((s = check_shape(N, K)) != MXC_OK) return s;
+  if ((s = resolve_scale_group(strategy, fmt, K, sg, ds)) != MXC_OK) return s;
   return resolve_qblock(N, K, qn, qk, rqn, rqk);
 }
 
-mxc_status check_device_weight(const mxc_weight* w, int64_t* qn, int64_t* qk) {
+mxc_status check_device_weight(const mxc_weight* w, int64_t* qn, int64_t* qk, int* ds) {
   if (!w) return MXC_ERR_INVALID_ARG;
-  mxc_status s = check_weight_common(w->strategy, w->fmt, w->N, w->K, w->qn, w->qk, qn, qk);
+  mxc_status s = check_weight_common(w->strategy, w->fmt, w->N, w->K, w->qn, w->qk, w->scale_group, qn, qk, ds);
   if (s != MXC_OK) return s;
   if (!w->idx || !w->cb) return MXC_ERR_INVALID_ARG;
   if (!aligned16(w->idx) || !aligned16(w->cb)) return MXC_ERR_ALIGNMENT;
@@ -150,15 +164,16 @@ size_t mxc_sf_bytes(int64_t rows, int64_t K, mxc_format fmt) {
 mxc_status mxc_packed_weight_sizes(const mxc_weight_host* w, mxc_packed_sizes* out) {
   if (!w || !out) return MXC_ERR_INVALID_ARG;
   int64_t qn, qk;
-  mxc_status s = check_weight_common(w->strategy, w->fmt, w->N, w->K, w->qn, w->qk, &qn, &qk);
+  int ds;
+  mxc_status s = check_weight_common(w->strategy, w->fmt, w->N, w->K, w->qn, w->qk, w->scale_group, &qn, &qk, &ds);
   if (s != MXC_OK) return s;
   const int B = block_of(w->fmt);
   out->idx = static_cast<size_t>(w->N) * (w->K / 4);
   out->cb = static_cast<size_t>(w->N / qn) * (w->K / qk) * 256 * sizeof(uint16_t);
   if (w->strategy == MXC_PRESCALE_PLUS) {
     out->scales = 0;
-    out->sidx = static_cast<size_t>(w->N) * (w->K / (8 * B));
-    out->scb = 256 * 8;
+    out->sidx = static_cast<size_t>(w->N) * (w->K / (static_cast<int64_t>(ds) * B));
+    out->scb = 256 * static_cast<size_t>(ds);
   } else if (w->strategy == MXC_POSTSCALE_QB) {
     out->scales = static_cast<size_t>(w->N / qn) * static_cast<size_t>(w->K / qk);
     out->sidx = 0;
@@ -189,11 +204,15 @@ mxc_status mxc_pack_weight(const mxc_weight_host* w, uint8_t* idx_out, uint8_t* 
   if (w->strategy == MXC_PRESCALE_PLUS) {
     if (sidx_out) {
       if (!w->sidx) return MXC_ERR_INVALID_ARG;
-      const int64_t G = kStageK / (8 * B), row = K / (8 * B);
+      // units of the band's indices: a 256-channel stage holding G = 256/(ds*B)
+      // groups of each row when ds*B <= 256, else one group (G = 1)
+      const int ds = w->scale_group ? w->scale_group : 8;
+      const int64_t row = K / (static_cast<int64_t>(ds) * B);
+      const int64_t G = ds * B <= kStageK ? kStageK / (ds * B) : 1, U = row / G;
       for (int64_t nt = 0; nt < N / kTileN; ++nt)
-        for (int64_t ks = 0; ks < KS; ++ks)
+        for (int64_t u = 0; u < U; ++u)
           for (int64_t r = 0; r < kTileN; ++r)
-            std::memcpy(sidx_out + ((nt * KS + ks) * kTileN + r) * G, w->sidx + (nt * kTileN + r) * row + ks * G, G);
+            std::memcpy(sidx_out + ((nt * U + u) * kTileN + r) * G, w->sidx + (nt * kTileN + r) * row + u * G, G);
     }
   } else if (scales_out && w->strategy == MXC_POSTSCALE_QB) {
     if (!w->scales) return MXC_ERR_INVALID_ARG;
@@ -213,6 +232,15 @@ size_t mxc_quantize_act_workspace_bytes(int64_t /*M*/, int64_t /*K*/, mxc_format
 size_t mxc_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, mxc_format fmt) {
   if (check_format(fmt) != MXC_OK || check_shape(N, K) != MXC_OK || M < 0) return 0;
   return linear_workspace_bytes(M, N, K, fmt);
+}
+
+size_t mxc_linear_workspace_bytes_for(const mxc_weight* w, int64_t M) {
+  int64_t qn, qk;
+  int ds;
+  if (!w || M < 0 || check_weight_common(w->strategy, w->fmt, w->N, w->K, w->qn, w->qk, w->scale_group, &qn, &qk,
+                                         &ds) != MXC_OK)
+    return 0;
+  return linear_workspace_bytes_for(M, w->N, w->K, w->fmt == MXC_FMT_E8M0_B32 ? FMT_E8M0 : FMT_E4M3, qn, qk);
 }
 
 size_t mxc_moe_workspace_bytes(int64_t M, int32_t E, int64_t N, int64_t K, mxc_format fmt) {
@@ -299,7 +327,8 @@ mxc_status mxc_linear(const mxc_mx_tensor* a, const mxc_weight* w, void* y, int6
   mxc_status s = check_mx_tensor(a);
   if (s != MXC_OK) return s;
   int64_t qn, qk;
-  if ((s = check_device_weight(w, &qn, &qk)) != MXC_OK) return s;
+  int ds;
+  if ((s = check_device_weight(w, &qn, &qk, &ds)) != MXC_OK) return s;
   if (a->fmt != w->fmt || a->K != w->K) return MXC_ERR_INVALID_ARG;
   if ((s = check_output(y, ldy, w->N, y_dtype)) != MXC_OK) return s;
   if (a->rows == 0) return MXC_OK;
@@ -316,6 +345,7 @@ mxc_status mxc_linear(const mxc_mx_tensor* a, const mxc_weight* w, void* y, int6
   L.w_sidx = w->sidx;
   L.w_scb = w->scb;
   L.w_tscale = w->w_tscale;
+  L.w_ds = ds;
   L.y = y;
   L.ldy = ldy;
   L.out_bf16 = y_dtype == MXC_OUT_BF16;
@@ -363,17 +393,20 @@ static mxc_status moe_prepare_inputs(const mxc_mx_tensor* a, const int32_t* d_of
   if (!d_offsets || !experts || E <= 0) return MXC_ERR_INVALID_ARG;
   if (E > kMaxGroups) return MXC_ERR_UNSUPPORTED;
   int64_t qn, qk;
-  if ((s = check_device_weight(&experts[0], &qn, &qk)) != MXC_OK) return s;
+  int ds;
+  if ((s = check_device_weight(&experts[0], &qn, &qk, &ds)) != MXC_OK) return s;
   for (int32_t e = 1; e < E; ++e) {
     const mxc_weight& w = experts[e];
     int64_t qn2, qk2;
-    if ((s = check_device_weight(&w, &qn2, &qk2)) != MXC_OK) return s;
+    int ds2;
+    if ((s = check_device_weight(&w, &qn2, &qk2, &ds2)) != MXC_OK) return s;
     if (w.strategy != experts[0].strategy || w.fmt != experts[0].fmt || w.N != experts[0].N ||
-        w.K != experts[0].K || qn2 != qn || qk2 != qk)
+        w.K != experts[0].K || qn2 != qn || qk2 != qk || ds2 != ds)
       return MXC_ERR_INVALID_ARG;
   }
   const mxc_weight& w0 = experts[0];
   if (a->fmt != w0.fmt || a->K != w0.K) return MXC_ERR_INVALID_ARG;
+  if (small_qblock(qn, qk)) return MXC_ERR_UNSUPPORTED;   // grouped kernels decode in the GEMM
   *m = MoeArgs{};
   fill_activation(m->base, a);
   m->base.wsrc = wsrc_of(w0.strategy);
@@ -486,7 +519,8 @@ mxc_status mxc_moe_linear_noalloc(const mxc_mx_tensor* a, const int32_t* d_offse
 
 mxc_status mxc_decode_weight(const mxc_weight* w, uint8_t* q_out, int64_t ldq, uint8_t* sf_out, mxc_stream_t stream) {
   int64_t qn, qk;
-  mxc_status s = check_device_weight(w, &qn, &qk);
+  int ds;
+  mxc_status s = check_device_weight(w, &qn, &qk, &ds);
   if (s != MXC_OK) return s;
   if (!q_out || !sf_out) return MXC_ERR_INVALID_ARG;
   if (ldq < w->K / 2 || ldq % 16 || !aligned16(q_out) || !aligned16(sf_out)) return MXC_ERR_ALIGNMENT;
@@ -503,6 +537,7 @@ mxc_status mxc_decode_weight(const mxc_weight* w, uint8_t* q_out, int64_t ldq, u
   d.w_sf = w->scales;
   d.w_sidx = w->sidx;
   d.w_scb = w->scb;
+  d.ds = ds;
   d.q_out = q_out;
   d.ldq = ldq;
   d.sf_out = sf_out;

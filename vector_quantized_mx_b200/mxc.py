@@ -31,7 +31,7 @@ EXPORTED = (
     "mxc_quantize_act_workspace_bytes", "mxc_linear_workspace_bytes", "mxc_moe_workspace_bytes",
     "mxc_grouped_sf_rows_bound", "mxc_quantize_act", "mxc_quantize_act_grouped", "mxc_linear",
     "mxc_native_linear", "mxc_moe_linear", "mxc_moe_linear_noalloc", "mxc_decode_weight", "mxc_get_device_error",
-    "mxc_selftest_wait_timeout", "mxc_moe_gate_up_swiglu",
+    "mxc_selftest_wait_timeout", "mxc_moe_gate_up_swiglu", "mxc_linear_workspace_bytes_for",
 )
 
 
@@ -51,7 +51,8 @@ class _Weight(ctypes.Structure):
     _fields_ = [("strategy", ctypes.c_int), ("fmt", ctypes.c_int), ("N", ctypes.c_int64),
                 ("K", ctypes.c_int64), ("qn", ctypes.c_int64), ("qk", ctypes.c_int64),
                 ("idx", ctypes.c_void_p), ("cb", ctypes.c_void_p), ("scales", ctypes.c_void_p),
-                ("sidx", ctypes.c_void_p), ("scb", ctypes.c_void_p), ("w_tscale", ctypes.c_float)]
+                ("sidx", ctypes.c_void_p), ("scb", ctypes.c_void_p), ("w_tscale", ctypes.c_float),
+                ("scale_group", ctypes.c_int32)]
 
 
 _WeightHost = _Weight  # identical field layout (mxc_weight_host)
@@ -82,6 +83,7 @@ def lib() -> ctypes.CDLL:
             "mxc_quantize_act_workspace_bytes": (sz, [i64, i64, ctypes.c_int]),
             "mxc_linear_workspace_bytes": (sz, [i64, i64, i64, ctypes.c_int]),
             "mxc_moe_workspace_bytes": (sz, [i64, i32, i64, i64, ctypes.c_int]),
+            "mxc_linear_workspace_bytes_for": (sz, [ctypes.POINTER(_Weight), i64]),
             "mxc_grouped_sf_rows_bound": (i64, [i64, i32]),
             "mxc_quantize_act": (ctypes.c_int, [vp, i64, i64, i64, ctypes.c_int, vp, vp, i64, vp, vp, vp, sz, vp]),
             "mxc_quantize_act_grouped": (ctypes.c_int, [vp, i64, i64, i64, ctypes.c_int, vp, i32, vp, vp, i64, vp,
@@ -222,10 +224,11 @@ class PackedWeight:
     sidx: Optional[torch.Tensor]
     scb: Optional[torch.Tensor]
     w_tscale: float
+    ds: int = 8                 # PreScale+ scale group
 
     def _c(self) -> _Weight:
         key = (self.strategy, self.fmt, self.N, self.K, self.qn, self.qk, self.idx.data_ptr(), self.cb.data_ptr(),
-               _ptr(self.scales), _ptr(self.sidx), _ptr(self.scb), self.w_tscale)
+               _ptr(self.scales), _ptr(self.sidx), _ptr(self.scb), self.w_tscale, self.ds)
         c = self.__dict__.get("_cstruct")
         if c is None or c[0] != key:
             c = (key, _Weight(STRATEGY[self.strategy], FMT[self.fmt], *key[2:]))
@@ -250,7 +253,7 @@ def _host_struct(w, keep: list) -> _WeightHost:
         return a.ctypes.data
     return _WeightHost(STRATEGY[w.strategy], FMT[w.fmt], w.N, w.K, w.qn, w.qk, arr(w.idx, np.uint8),
                        arr(w.cb, np.uint16), arr(w.scales, np.uint8), arr(w.sidx, np.uint8), arr(w.scb, np.uint8),
-                       float(w.w_tscale))
+                       float(w.w_tscale), int(getattr(w, "ds", 8)))
 
 
 def pack_weight_host(w) -> dict:
@@ -279,7 +282,7 @@ def pack_weight(w, device="cuda") -> PackedWeight:
         return None if a is None else torch.from_numpy(a).to(device)
     cb = torch.from_numpy(h["cb"].view(np.int16)).to(device)
     return PackedWeight(w.fmt, w.strategy, w.N, w.K, w.qn, w.qk, up(h["idx"]), cb, up(h["scales"]),
-                        up(h["sidx"]), up(h["scb"]), float(w.w_tscale))
+                        up(h["sidx"]), up(h["scb"]), float(w.w_tscale), int(getattr(w, "ds", 8)))
 
 
 # ---------------------------------------------------------------------------
@@ -300,8 +303,10 @@ def linear(a: MXTensor, w: PackedWeight, out_dtype=torch.float32, y: Optional[to
     """mxc_linear: y[M, N] = A . W^T with W decoded on the fly."""
     dev = a.q.device
     y = _out(a.rows, w.N, out_dtype, dev) if y is None else y
-    ws = linear_workspace(a.rows, w.N, w.K, w.fmt, dev) if ws is None else ws
     at, wt = a._c(), w._c()
+    if ws is None:
+        n = lib().mxc_linear_workspace_bytes_for(ctypes.byref(wt), a.rows)
+        ws = torch.empty((max(n, 16),), dtype=torch.uint8, device=dev)
     _check(lib().mxc_linear(ctypes.byref(at), ctypes.byref(wt), y.data_ptr(), y.stride(0), OUT[y.dtype],
                             ws.data_ptr(), ws.numel(), _stream(stream)), "mxc_linear")
     return y

@@ -129,8 +129,9 @@ class VQWeight:
     cb[a, b, c]    uint16, centroid c of QBlock (a, b) = (n // qn, k // qk)
     scales[n, kb]  uint8 block-scale byte (PostScale / PreScale), kb = k // B
     sidx[n, g]     uint8 scale-codebook index of scale group g = kb // 8 (PreScale+)
-    scb[c, t]      uint8 scale codebook: 256 entries of 8 scale bytes (PreScale+)
+    scb[c, t]      uint8 scale codebook: 256 entries of ds scale bytes (PreScale+)
     w_tscale       FP32 tensor scale (1.0 for E8M0-B32)
+    ds             PreScale+ scale group: ds consecutive block scales along K per index
     """
     fmt: str
     strategy: str
@@ -144,6 +145,7 @@ class VQWeight:
     sidx: Optional[np.ndarray]
     scb: Optional[np.ndarray]
     w_tscale: float
+    ds: int = 8
 
     @property
     def block(self) -> int:
@@ -164,15 +166,16 @@ def weight_rows(w: "VQWeight", r0: int, r1: int) -> "VQWeight":
     else:
         scales = w.scales[r0:r1]
     return VQWeight(w.fmt, w.strategy, r1 - r0, w.K, w.qn, w.qk, w.idx[r0:r1], w.cb[q0:q1], scales, sidx, w.scb,
-                    w.w_tscale)
+                    w.w_tscale, w.ds)
 
 
 TSCALE_E4M3 = float(np.float32(1.0) / np.float32(2688.0))
 
 
 def make_weight(seed: int, fmt: str, strategy: str, N: int, K: int, qn: int, qk: int,
-                e8m0_exp=(-8, 1), sub: int = 0) -> VQWeight:
-    """Draw one VQ weight; qn/qk = 0 means the QBlock spans the whole dimension."""
+                e8m0_exp=(-8, 1), sub: int = 0, ds: int = 8) -> VQWeight:
+    """Draw one VQ weight; qn/qk = 0 means the QBlock spans the whole dimension; ds is the
+    PreScale+ scale group (consecutive block scales per scale index)."""
     qn = N if qn in (0, None) else qn
     qk = K if qk in (0, None) else qk
     B = BLOCK[fmt]
@@ -180,11 +183,11 @@ def make_weight(seed: int, fmt: str, strategy: str, N: int, K: int, qn: int, qk:
     cb = draw_codebooks(stream(seed, "cb", sub), N // qn, K // qk)
     scales = sidx = scb = None
     if strategy == PRESCALE_PLUS:
-        sidx = stream(seed, "sidx", sub).integers(0, 256, size=(N, K // (8 * B)), dtype=np.uint8)
+        sidx = stream(seed, "sidx", sub).integers(0, 256, size=(N, K // (ds * B)), dtype=np.uint8)
         if fmt == FMT_E8M0_B32:
-            scb = draw_e8m0_bytes(stream(seed, "scb", sub), (256, 8), *e8m0_exp)
+            scb = draw_e8m0_bytes(stream(seed, "scb", sub), (256, ds), *e8m0_exp)
         else:
-            scb = draw_e4m3_bytes(stream(seed, "scb", sub), (256, 8))
+            scb = draw_e4m3_bytes(stream(seed, "scb", sub), (256, ds))
     else:
         shape = (N // qn, K // qk) if strategy == POSTSCALE_QB else (N, K // B)   # per QBlock or per block
         if fmt == FMT_E8M0_B32:
@@ -192,7 +195,7 @@ def make_weight(seed: int, fmt: str, strategy: str, N: int, K: int, qn: int, qk:
         else:
             scales = draw_e4m3_bytes(stream(seed, "scale", sub), shape)
     w_tscale = 1.0 if fmt == FMT_E8M0_B32 else TSCALE_E4M3
-    return VQWeight(fmt, strategy, N, K, qn, qk, idx, cb, scales, sidx, scb, w_tscale)
+    return VQWeight(fmt, strategy, N, K, qn, qk, idx, cb, scales, sidx, scb, w_tscale, ds)
 
 
 def make_activations(seed: int, M: int, K: int, outliers: bool, sub: int = 0) -> np.ndarray:
