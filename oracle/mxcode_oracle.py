@@ -26,12 +26,15 @@ What it computes, and where the method defines it
   +-6) and, for E4M3-B16, an FP32 tensor scale amax/(6*448).
 * Storage accounting (Table 2 "Weight (BPE)" row; Figure 3 caption): indices +
   FP4 codebooks + scales (+ scale-VQ metadata), tensor scale excluded.
+* The MoE FFN step between the gate/up and down projections (Table 4 caption:
+  Qwen3's MoE expert tensors): h = SiLU(gate) * up in FP32 with a fixed FP32 exp,
+  and the MX quantization of FP32 values (end of this file).
 
 Where the pages leave a point open (the activation recipe, nibble order, scale-VQ
 grouping, QBlock tiling, the PostScale storage), the function that decides it
 states the reading it takes in its docstring.
-Everything is FP64 except the FP32 steps of the E4M3 scale recipe, which are
-done in FP32 on purpose because the recipe is defined in FP32.
+Everything is FP64 except the FP32 steps of the E4M3 scale recipe and of SwiGLU,
+which are done in FP32 on purpose because they are defined in FP32.
 
 Parity pins: every function here is pinned by tests/test_oracle_pins.py to
 something other than itself (closed forms, library routines, brute force,

@@ -296,14 +296,30 @@ __global__ void __maxnreg__(64)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_sfw);
     }
+    int issued_q = 2;                                // index quarters requested so far
     if constexpr (L::kVQ) {
       if (elect_one()) {
         for (int j = 2; j < 4; ++j) {                // K-quarter j of every stage (from L2 by now)
           if (!mbar_wait(&dec_ph[j - 2], 0)) break;  // its buffer has been decoded
           mbar_arrive_expect_tx(&full[j], p.ks_per_split * 2048);
           tma_load_4d(smem + L::IDX_OFF + (j % 2) * L::IDX_BUF, &tmap_idx, 0, j, ks_begin, n_tile, &full[j]);
+          issued_q = j + 1;
         }
       }
+      issued_q = static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<unsigned>(issued_q)));   // the elected lane's count
+    }
+    __syncwarp();
+    // Every copy this CTA requested lands before the CTA can retire, even when a
+    // consumer gave up waiting (timeout path): codebooks, index quarters, weight
+    // scales or native tiles.  On the normal path these have all completed already.
+    if (lane == 0) {
+      if constexpr (L::kVQ) {
+        mbar_wait(bar_cb, 0);
+        for (int j = 0; j < issued_q; ++j) mbar_wait(&full[j], 0);
+      } else {
+        for (int s = 0; s < nks; ++s) mbar_wait(&full[s], 0);
+      }
+      if constexpr (!L::kSVQ && !L::kQBS) mbar_wait(bar_sfw, 0);
     }
     __syncwarp();
     if (splits > 1 && rank == 0 && !red_atomic) {
