@@ -195,7 +195,9 @@ mxc_status mxc_pack_weight(const mxc_weight_host* w, uint8_t* idx_out, uint8_t* 
  * mxc_linear: 0 below 1024 rows; from 1024 rows the room for the weight decoded
  * once per call (N*K/2 bytes of FP4 codes rounded up to 1 KiB, then N*K/B bytes
  * of SF-layout scales).  A smaller workspace is not an error there: the call
- * then runs the fused decode-in-GEMM kernel, which is slower at that size. */
+ * then runs the fused decode-in-GEMM kernel, which is slower at that size.
+ * mxc_moe_linear and mxc_moe_gate_up_swiglu: the expert tile and chunk tables,
+ * 2 (E+1) int32 rounded up to whole 256-byte units. */
 size_t mxc_quantize_act_workspace_bytes(int64_t M, int64_t K, mxc_format fmt);
 size_t mxc_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, mxc_format fmt);
 size_t mxc_moe_workspace_bytes(int64_t M, int32_t E, int64_t N, int64_t K, mxc_format fmt);
@@ -324,14 +326,15 @@ mxc_status mxc_moe_gate_up_swiglu(const mxc_mx_tensor* a, const int32_t* d_offse
  * environment only.  It takes the same arguments as mxc_moe_linear minus the
  * workspace, checks them in the same order with the same statuses, and runs
  * the same kernels, so its output is bit-identical to mxc_moe_linear's.
- * Scratch: the per-call expert tile table lives in a fixed module-global array
- * of 1280 bytes in device memory (room for the largest table, E = 256 experts),
+ * Scratch: the per-call expert tile and chunk tables live in a fixed
+ * module-global array of 2304 bytes in device memory (room for the largest
+ * tables, E = 256 experts),
  * held by every GPU that loads the library until the process exits.  Limit:
  * E <= 256 experts, as for mxc_moe_linear; larger E returns MXC_ERR_UNSUPPORTED
  * and enqueues nothing.
  * The first call on each device looks up that array's device address (no
  * allocation); make the first call on a device before any stream capture that
- * includes this entry point.  Every call rewrites the table before reading it,
+ * includes this entry point.  Every call rewrites the tables before reading them,
  * so nothing needs clearing between calls, but all calls on a device share the
  * array: calls whose executions overlap on the GPU (e.g. on two streams without
  * ordering between them) race.  The function calls no cudaMalloc, cudaFree or

@@ -237,11 +237,11 @@ def test_bf16_output():
 # Grouped experts (MoE)
 # ---------------------------------------------------------------------------
 
-def run_moe(fmt, strat, E, N, K, counts, seed):
+def run_moe(fmt, strat, E, N, K, counts, seed, qn=256, qk=256):
     offsets = np.zeros(E + 1, dtype=np.int64)
     offsets[1:] = np.cumsum(counts)
     M = int(offsets[-1])
-    ws = [synth.make_weight(seed, fmt, strat, N, K, 256, 256, sub=e) for e in range(E)]
+    ws = [synth.make_weight(seed, fmt, strat, N, K, qn, qk, sub=e) for e in range(E)]
     x = synth.make_activations(seed, M, K, outliers=False)
     off_d = torch.from_numpy(offsets.astype(np.int32)).cuda()
     a = mxc.quantize_act_grouped(dev_bf16(x), fmt, off_d)
@@ -267,6 +267,19 @@ def run_moe(fmt, strat, E, N, K, counts, seed):
 @pytest.mark.parametrize("strat", ["prescale", "prescale_plus", "postscale_qb"])
 def test_moe_small(fmt, strat):
     run_moe(fmt, strat, 6, 256, 512, [0, 5, 130, 1, 257, 0], seed=61)
+
+
+@pytest.mark.parametrize("fmt,strat,qn,qk", [("e4m3_b16", "prescale_plus", 128, 128),
+                                              ("e8m0_b32", "postscale_qb", 256, 128),
+                                              ("e4m3_b16", "prescale", 256, 512),
+                                              ("e8m0_b32", "prescale_plus", 0, 0),
+                                              ("e4m3_b16", "postscale", 512, 256)])
+def test_moe_rounds(fmt, strat, qn, qk):
+    """K = 1536: a full round of four 256-channel stages and a ragged one of two;
+    QBlocks 128 wide along K (two codebooks a stage), 512 wide (one codebook for two
+    stages) and the whole tensor; experts of 1 to 3 token tiles (a chunk of two
+    tiles, a chunk of one, a ragged tile)."""
+    run_moe(fmt, strat, 6, 512, 1536, [300, 0, 17, 129, 256, 1], seed=63, qn=qn, qk=qk)
 
 
 def test_moe_bad_offsets_sets_device_error():

@@ -1,4 +1,4 @@
-"""Host replay of the grouped-expert (MoE) tile scheduler.
+"""Host replay of the grouped-expert (MoE) tile and chunk schedulers.
 
 Device side (act_quant.cuh group_prologue_kernel, mma_kernel.cuh gemm_kernel<MOE>):
 the prologue turns expert offsets into tile_prefix[g] = sum over g' < g of
@@ -64,12 +64,52 @@ def patterns():
             yield np.concatenate([[0], np.cumsum(counts)]).tolist()
 
 
+def chunk_prefix(offsets):
+    tiles = np.diff(tile_prefix(offsets))
+    return np.concatenate([[0], np.cumsum((tiles + 1) // 2)])
+
+
+def replay_chunks(offsets):
+    """round_kernel.cuh moe_round_kernel: chunk c of the launch's ceil(M/256) + E
+    belongs to the last expert e with chunk_prefix[e] <= c; it runs the expert's
+    128-row tiles 2 (c - chunk_prefix[e]) and the next one if the expert has it,
+    scale groups tile_prefix[e] + those tile numbers."""
+    E = len(offsets) - 1
+    M = int(offsets[-1])
+    tp, cp = tile_prefix(offsets), chunk_prefix(offsets)
+    grid_chunks = (M + 255) // 256 + E
+    assert grid_chunks >= cp[E]
+    cover = np.zeros(M, dtype=np.int64)
+    groups = np.zeros(tp[E], dtype=np.int64)
+    for c in range(grid_chunks):
+        if c >= cp[E]:
+            continue
+        e = owner(cp, E, c)
+        k = c - cp[e]
+        nt = min(2, tp[e + 1] - tp[e] - 2 * k)
+        assert nt >= 1, (c, e)
+        for t in range(nt):
+            m0 = offsets[e] + (2 * k + t) * 128
+            m1 = min(m0 + 128, offsets[e + 1])
+            assert offsets[e] <= m0 < m1 <= offsets[e + 1], (c, e, t, m0, m1)
+            cover[m0:m1] += 1
+            groups[tp[e] + 2 * k + t] += 1
+    assert np.all(cover == 1)
+    assert np.all(groups == 1)           # every scale group read by exactly one tile
+
+
 @pytest.mark.parametrize("offsets", list(patterns()))
 def test_every_row_once(offsets):
     replay(np.asarray(offsets, dtype=np.int64))
+
+
+@pytest.mark.parametrize("offsets", list(patterns()))
+def test_every_row_once_in_chunks(offsets):
+    replay_chunks(np.asarray(offsets, dtype=np.int64))
 
 
 def test_zipf_routing_of_the_moe_workload():
     from vector_quantized_mx_b200 import synth
     _, off = synth.config4_routing()
     replay(np.asarray(off, dtype=np.int64))
+    replay_chunks(np.asarray(off, dtype=np.int64))

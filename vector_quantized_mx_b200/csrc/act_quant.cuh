@@ -380,11 +380,13 @@ __global__ void __launch_bounds__(kSmallQuantThreadsAll / CTAS) quantize_small_k
 
 // ------------------------------------------------------------------------------------
 // Group prologue: validates offsets and writes tile_prefix[g] = sum over g' < g of
-// ceil(rows_g' / 128), g = 0..E.  Malformed offsets set MXC_ERR_DEVICE_INVALID and
-// an all-zero prefix, so that the kernels that follow do no work.
+// ceil(rows_g' / 128), g = 0..E, and (when chunk_prefix is given) chunk_prefix[g] =
+// sum over g' < g of ceil(tiles_g' / 2): the 256-row chunks the grouped kernel runs.
+// Malformed offsets set MXC_ERR_DEVICE_INVALID and all-zero prefixes, so that the
+// kernels that follow do no work.
 // ------------------------------------------------------------------------------------
 __global__ void group_prologue_kernel(const int32_t* __restrict__ offsets, int32_t E, int64_t M,
-                                      int32_t* __restrict__ tile_prefix) {
+                                      int32_t* __restrict__ tile_prefix, int32_t* __restrict__ chunk_prefix) {
   __shared__ int bad;
   __shared__ int32_t tiles[kMaxGroups + 1];
   if (threadIdx.x == 0) bad = (offsets[0] != 0 || offsets[E] != M);
@@ -396,12 +398,15 @@ __global__ void group_prologue_kernel(const int32_t* __restrict__ offsets, int32
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    int32_t acc = 0;
+    int32_t acc = 0, acc2 = 0;
     for (int g = 0; g < E; ++g) {
       tile_prefix[g] = bad ? 0 : acc;
+      if (chunk_prefix) chunk_prefix[g] = bad ? 0 : acc2;
       acc += tiles[g];
+      acc2 += (tiles[g] + 1) / 2;
     }
     tile_prefix[E] = bad ? 0 : acc;
+    if (chunk_prefix) chunk_prefix[E] = bad ? 0 : acc2;
     if (bad) set_device_error(MXC_ERR_DEVICE_INVALID);
   }
 }
@@ -410,8 +415,8 @@ __global__ void group_prologue_kernel(const int32_t* __restrict__ offsets, int32
 // Host launchers
 // ------------------------------------------------------------------------------------
 cudaError_t launch_group_prologue(const int32_t* offsets, int32_t E, int64_t M, int32_t* tile_prefix,
-                                  cudaStream_t stream) {
-  group_prologue_kernel<<<1, 256, 0, stream>>>(offsets, E, M, tile_prefix);
+                                  cudaStream_t stream, int32_t* chunk_prefix) {
+  group_prologue_kernel<<<1, 256, 0, stream>>>(offsets, E, M, tile_prefix, chunk_prefix);
   return cudaGetLastError();
 }
 

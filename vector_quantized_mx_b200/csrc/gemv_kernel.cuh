@@ -229,7 +229,7 @@ __global__ void __maxnreg__(64)
       }
     }
     if constexpr (L::kSVQ) {
-      const int u0 = ks_begin / sv.spu, u1 = (ks_end - 1) / sv.spu;
+      const int u0 = ks_begin >> sv.lspu, u1 = (ks_end - 1) >> sv.lspu;
       l2_prefetch_bulk(sv.unit(p.w.sidx, n_tile, ks_begin), static_cast<uint32_t>(u1 - u0 + 1) * 128 * sv.G);
     }
   }
@@ -475,10 +475,10 @@ __global__ void __maxnreg__(64)
           const uint8_t* un = sv.unit(p.w.sidx, n_tile, ks);
           const int kb = sv.kb_base(ks, L::kB) + 4 * a;
           uint4 v;
-          v.x = svq_word(un + (0 * 32 + lane) * sv.G, scb32, sv.ds, kb);
-          v.y = svq_word(un + (1 * 32 + lane) * sv.G, scb32, sv.ds, kb);
-          v.z = svq_word(un + (2 * 32 + lane) * sv.G, scb32, sv.ds, kb);
-          v.w = svq_word(un + (3 * 32 + lane) * sv.G, scb32, sv.ds, kb);
+          v.x = svq_word(un + (0 * 32 + lane) * sv.G, scb32, sv.lds, kb);
+          v.y = svq_word(un + (1 * 32 + lane) * sv.G, scb32, sv.lds, kb);
+          v.z = svq_word(un + (2 * 32 + lane) * sv.G, scb32, sv.lds, kb);
+          v.w = svq_word(un + (3 * 32 + lane) * sv.G, scb32, sv.lds, kb);
           tmem_st_32x32b_x4(lane_base + L::COL_SFW + 4 * i, v);
         }
         tmem_st_wait();

@@ -2,9 +2,10 @@
 // split-K policy, workspace layout, template dispatch.
 #pragma once
 
+#include <atomic>
 #include <cstring>
 
-#include "gemv_kernel.cuh"
+#include "round_kernel.cuh"
 
 namespace mxc {
 
@@ -205,8 +206,9 @@ size_t linear_workspace_bytes_for(int64_t M, int64_t N, int64_t K, int fmt, int6
   return small_qblock(qn, qk) ? decoded_weight_bytes(N, K, fmt) : linear_workspace_bytes(M, N, K, fmt);
 }
 
+// The expert tile prefix and chunk prefix, (E + 1) int32 each.
 size_t moe_workspace_bytes(int64_t /*M*/, int32_t E, int64_t /*N*/, int64_t /*K*/, int /*fmt*/) {
-  return align_up(static_cast<size_t>(E + 1) * sizeof(int32_t), 256);
+  return align_up(2 * static_cast<size_t>(E + 1) * sizeof(int32_t), 256);
 }
 
 // ------------------------------------------------------------------------------------
@@ -428,14 +430,85 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
   return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
 }
 
+template <int FMT, int WSRC>
+cudaError_t launch_round(const CUtensorMap& tx, const MoeRoundParams& p, dim3 grid, cudaStream_t stream) {
+  using L = RoundLayout<FMT, WSRC>;
+  auto kern = moe_round_kernel<FMT, WSRC>;
+  static uint64_t attr_set = 0;
+  cudaError_t err = ensure_smem_attr(kern, L::SMEM, &attr_set);
+  if (err != cudaSuccess) return err;
+  kern<<<grid, kRoundThreads, L::SMEM, stream>>>(tx, p);
+  return cudaGetLastError();
+}
+
+// SMs of the current device (looked up once per device).
+inline int device_sms() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kSMs;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = kSMs;
+  cached[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// Grouped experts without the fused SwiGLU: the round kernel, persistent, one CTA per
+// SM walking the (128-row weight band, chunk of up to 256 rows of one expert) items.
+mxc_status launch_moe_round(const MoeArgs& m, const CUtensorMap& tx, const int32_t* tile_prefix,
+                            const int32_t* chunk_prefix, cudaStream_t stream) {
+  const LinearArgs& a = m.base;
+  static thread_local MoeRoundParams p;           // about 12 KB with the expert table
+  std::memset(&p, 0, sizeof(p));
+  p.M = static_cast<int>(a.M);
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.qn = static_cast<int>(a.qn);
+  p.qk = static_cast<int>(a.qk);
+  p.a_sf = a.a_sf;
+  p.a_tscale = a.a_tscale;
+  p.y = a.y;
+  p.ldy = a.ldy;
+  p.out_bf16 = a.out_bf16;
+  p.E = m.E;
+  p.offsets = m.offsets;
+  p.tile_prefix = tile_prefix;
+  p.chunk_prefix = chunk_prefix;
+  for (int e = 0; e < m.E; ++e) {
+    const mxc_weight& w = m.experts[e];
+    p.w[e].idx = w.idx;
+    p.w[e].cb = w.cb;
+    p.w[e].sf = w.scales;
+    p.w[e].sidx = w.sidx;
+    p.w[e].scb = w.scb;
+    p.w[e].w_tscale = w.w_tscale;
+    p.w[e].ds = w.scale_group ? w.scale_group : 8;
+  }
+  const dim3 grid(static_cast<unsigned>(device_sms()), 1, 1);
+  cudaError_t err;
+  if (a.fmt == FMT_E8M0) {
+    if (a.wsrc == WSRC_VQ_DIRECT) err = launch_round<FMT_E8M0, WSRC_VQ_DIRECT>(tx, p, grid, stream);
+    else if (a.wsrc == WSRC_VQ_SVQ) err = launch_round<FMT_E8M0, WSRC_VQ_SVQ>(tx, p, grid, stream);
+    else err = launch_round<FMT_E8M0, WSRC_VQ_QBS>(tx, p, grid, stream);
+  } else {
+    if (a.wsrc == WSRC_VQ_DIRECT) err = launch_round<FMT_E4M3, WSRC_VQ_DIRECT>(tx, p, grid, stream);
+    else if (a.wsrc == WSRC_VQ_SVQ) err = launch_round<FMT_E4M3, WSRC_VQ_SVQ>(tx, p, grid, stream);
+    else err = launch_round<FMT_E4M3, WSRC_VQ_QBS>(tx, p, grid, stream);
+  }
+  return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
+}
+
 mxc_status run_moe_linear(const MoeArgs& m, cudaStream_t stream) {
   const LinearArgs& a = m.base;
   const size_t need = moe_workspace_bytes(a.M, m.E, a.N, a.K, a.fmt);
   if (!a.ws || a.ws_bytes < need) return MXC_ERR_WORKSPACE;
   int32_t* tile_prefix = reinterpret_cast<int32_t*>(a.ws);
-  if (launch_group_prologue(m.offsets, m.E, a.M, tile_prefix, stream) != cudaSuccess) return MXC_ERR_CUDA;
+  int32_t* chunk_prefix = tile_prefix + (m.E + 1);
+  if (launch_group_prologue(m.offsets, m.E, a.M, tile_prefix, stream, chunk_prefix) != cudaSuccess)
+    return MXC_ERR_CUDA;
   CUtensorMap tx;
   if (!make_fp4_map(&tx, a.a_q, a.M, a.K, a.ldq, kMoeXBox)) return MXC_ERR_CUDA;   // 32-row boxes
+  if (!m.swiglu) return launch_moe_round(m, tx, tile_prefix, chunk_prefix, stream);
   // GemmParams with the expert table (about 12 KB of kernel parameters).
   static thread_local GemmParams<kMaxGroups> p;
   std::memset(&p, 0, sizeof(p));
@@ -484,17 +557,7 @@ mxc_status run_moe_linear(const MoeArgs& m, cudaStream_t stream) {
     }
     return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
   }
-  const dim3 grid(static_cast<unsigned>(a.N / kTileN), static_cast<unsigned>((a.M + 127) / 128 + m.E), 1);
-  if (a.fmt == FMT_E8M0) {
-    if (a.wsrc == WSRC_VQ_DIRECT) err = launch_gemm<FMT_E8M0, WSRC_VQ_DIRECT, 128, true>(tx, tx, p, grid, stream);
-    else if (a.wsrc == WSRC_VQ_SVQ) err = launch_gemm<FMT_E8M0, WSRC_VQ_SVQ, 128, true>(tx, tx, p, grid, stream);
-    else err = launch_gemm<FMT_E8M0, WSRC_VQ_QBS, 128, true>(tx, tx, p, grid, stream);
-  } else {
-    if (a.wsrc == WSRC_VQ_DIRECT) err = launch_gemm<FMT_E4M3, WSRC_VQ_DIRECT, 128, true>(tx, tx, p, grid, stream);
-    else if (a.wsrc == WSRC_VQ_SVQ) err = launch_gemm<FMT_E4M3, WSRC_VQ_SVQ, 128, true>(tx, tx, p, grid, stream);
-    else err = launch_gemm<FMT_E4M3, WSRC_VQ_QBS, 128, true>(tx, tx, p, grid, stream);
-  }
-  return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
+  return MXC_ERR_UNSUPPORTED;
 }
 
 template <int FMT, int WSRC>

@@ -218,38 +218,42 @@ __device__ __forceinline__ void decode_w_tile(const uint8_t* __restrict__ idx, u
 // units: one 256-channel stage with G = 256/(ds*B) groups per row when ds*B <= 256,
 // else one group (G = 1) spanning spu = ds*B/256 stages.
 struct SvqGeom {
-  int ds, G, spu, U;
+  // ds in {8, 16, 32}, B in {16, 32}: every quantity below is a power of two, kept
+  // with its base-2 logarithm so that the scale decode divides by shifting
+  int ds, G, spu, U, lds, lspu;
   __device__ __forceinline__ SvqGeom(int ds_, int B, int KS) {   // ds_ <= 0 (no scale VQ): the default 8
     ds = ds_ > 0 ? ds_ : 8;
     G = max(1, kStageK / (ds * B));
     spu = max(1, ds * B / kStageK);
-    U = KS / spu;
+    lds = 31 - __clz(ds);
+    lspu = 31 - __clz(spu);
+    U = KS >> lspu;
   }
   // the unit of the band's indices that holds stage ks: [128][G] bytes
   __device__ __forceinline__ const uint8_t* unit(const uint8_t* sidx, int band, int ks) const {
-    return sidx + (static_cast<size_t>(band) * U + ks / spu) * 128 * G;
+    return sidx + (static_cast<size_t>(band) * U + (ks >> lspu)) * 128 * G;
   }
   // first block of stage ks within its unit
-  __device__ __forceinline__ int kb_base(int ks, int B) const { return (ks % spu) * (kStageK / B); }
+  __device__ __forceinline__ int kb_base(int ks, int B) const { return (ks & (spu - 1)) * (kStageK / B); }
 };
 
 // The 32-bit word of block scales kb..kb+3 (kb a multiple of 4, counted from the
 // unit's first block) of one row: word (kb mod ds)/4 of the entry that the row's
-// index for group kb/ds selects.  Generic loads: the indices and the table may sit
-// in shared or global memory.
-__device__ __forceinline__ uint32_t svq_word(const uint8_t* row_idx, const uint32_t* scb32, int ds, int kb) {
-  return scb32[static_cast<uint32_t>(row_idx[kb / ds]) * (ds / 4) + (kb % ds) / 4];
+// index for group kb/ds selects (lds = log2 ds).  Generic loads: the indices and the
+// table may sit in shared or global memory.
+__device__ __forceinline__ uint32_t svq_word(const uint8_t* row_idx, const uint32_t* scb32, int lds, int kb) {
+  return scb32[(static_cast<uint32_t>(row_idx[kb >> lds]) << (lds - 2)) + ((kb & ((1 << lds) - 1)) >> 2)];
 }
 
 // A stage's weight scale atoms (A atoms of 128 rows x 4 blocks, the tcgen05 scale
 // layout) from the unit's indices; kb0 = the stage's first block within the unit.
 template <int A, int NT>
-__device__ __forceinline__ void decode_sf_tile(const uint8_t* sidx, int G, const uint32_t* scb32, int ds, int kb0,
+__device__ __forceinline__ void decode_sf_tile(const uint8_t* sidx, int G, const uint32_t* scb32, int lds, int kb0,
                                                uint8_t* __restrict__ sfw, int dt) {
   for (int u = dt; u < 128 * A; u += NT) {   // consecutive threads: consecutive atom words
     const int word = u & 127, a = u >> 7;
     const int r = (word >> 2) + 32 * (word & 3);
-    reinterpret_cast<uint32_t*>(sfw + a * 512)[word] = svq_word(sidx + r * G, scb32, ds, kb0 + 4 * a);
+    reinterpret_cast<uint32_t*>(sfw + a * 512)[word] = svq_word(sidx + r * G, scb32, lds, kb0 + 4 * a);
   }
 }
 
@@ -385,11 +389,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // PreScale+: the scale codebook (256 x ds bytes) in shared memory when it is the
   // 2 KB of ds = 8, else read in place (through L1)
   const SvqGeom sv(wp->ds, L::kB, KS);
-  const int sv_ds = sv.ds;
-  const uint32_t* const scb32 = sv_ds == 8 ? reinterpret_cast<const uint32_t*>(scb_smem)
+  const int sv_lds = sv.lds;
+  const uint32_t* const scb32 = sv.ds == 8 ? reinterpret_cast<const uint32_t*>(scb_smem)
                                            : reinterpret_cast<const uint32_t*>(w_scb);
   if constexpr (L::kSVQ) {
-    if (sv_ds == 8)
+    if (sv.ds == 8)
       for (int i = threadIdx.x; i < 512; i += kThreads)
         reinterpret_cast<uint32_t*>(scb_smem)[i] = __ldg(reinterpret_cast<const uint32_t*>(w_scb) + i);
   }
@@ -586,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         decode_w_tile<GT>(st + L::IDX_OFF, lut_s + b * kBuf, st + L::W_OFF, cm);
         if constexpr (L::kSVQ) {
           const int ks = ks_begin + (SWI && i >= nks ? i - nks : i);
-          decode_sf_tile<A, GT>(st + L::SIDX_OFF, sv.G, scb32, sv_ds, sv.kb_base(ks, L::kB), st + L::SFW_OFF, gt);
+          decode_sf_tile<A, GT>(st + L::SIDX_OFF, sv.G, scb32, sv_lds, sv.kb_base(ks, L::kB), st + L::SFW_OFF, gt);
         }
         if constexpr (L::kQBS) fill_sf_qbs<A, GT>(st + L::SFW_OFF, qs0, qs1, gt);
         fence_proxy_async_smem();                    // each thread's tile writes -> async proxy
@@ -796,7 +800,7 @@ __global__ void __launch_bounds__(160)
     cm.init(dt, cb_split);
     decode_w_tile<128>(st + L::IDX_OFF, smem_u32(lut), st + L::W_OFF, cm);
     if constexpr (L::kSVQ)
-      decode_sf_tile<A, 128>(st + L::SIDX_OFF, sv.G, scb32, sv.ds, sv.kb_base(ks, L::kB), st + L::SFW_OFF, dt);
+      decode_sf_tile<A, 128>(st + L::SIDX_OFF, sv.G, scb32, sv.lds, sv.kb_base(ks, L::kB), st + L::SFW_OFF, dt);
     if constexpr (L::kQBS) {
       const uint8_t* qb = w.sf + static_cast<size_t>((static_cast<int64_t>(n_tile) * 128) / qn) * (K / qk);
       const int qbk = cb_split ? 2 * ks : (ks * kStageK) / qk;
@@ -869,7 +873,7 @@ __global__ void __launch_bounds__(128)
       reinterpret_cast<uint4*>(sf_out + wsf)[i] = ldg_nc_v4(w.sf + wsf + static_cast<size_t>(i) * 16);
   } else if constexpr (WSRC == WSRC_VQ_SVQ) {
     const SvqGeom sv(w.ds, B, KS);
-    decode_sf_tile<A, 128>(sv.unit(w.sidx, n_tile, ks), sv.G, reinterpret_cast<const uint32_t*>(w.scb), sv.ds,
+    decode_sf_tile<A, 128>(sv.unit(w.sidx, n_tile, ks), sv.G, reinterpret_cast<const uint32_t*>(w.scb), sv.lds,
                            sv.kb_base(ks, B), sf_out + wsf, threadIdx.x);
   } else {
     // PostScale-QB: word (r % 32) * 4 + g of atom a holds the scales of rows 32 g + r % 32

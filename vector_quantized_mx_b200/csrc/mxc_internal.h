@@ -31,7 +31,7 @@ struct QuantizeArgs {
 
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream);
 cudaError_t launch_group_prologue(const int32_t* offsets, int32_t E, int64_t M, int32_t* tile_prefix,
-                                  cudaStream_t stream);
+                                  cudaStream_t stream, int32_t* chunk_prefix = nullptr);
 
 // Linear-layer launch descriptions (filled by the host API after validation).
 struct LinearArgs {

@@ -468,14 +468,14 @@ mxc_status mxc_moe_gate_up_swiglu(const mxc_mx_tensor* a, const int32_t* d_offse
 }  // extern "C"
 
 // ------------------------------------------------------------------------------------
-// Allocation-free MoE entry point: the expert tile table (E+1 int32) lives in a
-// fixed module-global array instead of a caller workspace.
+// Allocation-free MoE entry point: the expert tile and chunk tables (E+1 int32 each)
+// live in a fixed module-global array instead of a caller workspace.
 // ------------------------------------------------------------------------------------
 namespace {
 
-// The largest table the grouped kernels use (256 experts), in whole 256-byte units,
+// The largest tables the grouped kernels use (256 experts), in whole 256-byte units,
 // exactly the workspace size mxc_moe_workspace_bytes reports for 256 experts.
-constexpr size_t kNoallocScratchBytes = (static_cast<size_t>(kMaxGroups + 1) * sizeof(int32_t) + 255) / 256 * 256;
+constexpr size_t kNoallocScratchBytes = (2 * static_cast<size_t>(kMaxGroups + 1) * sizeof(int32_t) + 255) / 256 * 256;
 static __device__ __align__(256) int32_t g_moe_noalloc_scratch[kNoallocScratchBytes / sizeof(int32_t)];
 
 constexpr int kMaxDevices = 64;
