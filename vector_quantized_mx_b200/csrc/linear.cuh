@@ -430,15 +430,28 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
   return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
 }
 
-template <int FMT, int WSRC>
+template <int FMT, int WSRC, bool SWI>
 cudaError_t launch_round(const CUtensorMap& tx, const MoeRoundParams& p, dim3 grid, cudaStream_t stream) {
   using L = RoundLayout<FMT, WSRC>;
-  auto kern = moe_round_kernel<FMT, WSRC>;
+  auto kern = moe_round_kernel<FMT, WSRC, SWI>;
   static uint64_t attr_set = 0;
   cudaError_t err = ensure_smem_attr(kern, L::SMEM, &attr_set);
   if (err != cudaSuccess) return err;
   kern<<<grid, kRoundThreads, L::SMEM, stream>>>(tx, p);
   return cudaGetLastError();
+}
+
+template <bool SWI>
+cudaError_t dispatch_round(int fmt, int wsrc, const CUtensorMap& tx, const MoeRoundParams& p, dim3 grid,
+                           cudaStream_t stream) {
+  if (fmt == FMT_E8M0) {
+    if (wsrc == WSRC_VQ_DIRECT) return launch_round<FMT_E8M0, WSRC_VQ_DIRECT, SWI>(tx, p, grid, stream);
+    if (wsrc == WSRC_VQ_SVQ) return launch_round<FMT_E8M0, WSRC_VQ_SVQ, SWI>(tx, p, grid, stream);
+    return launch_round<FMT_E8M0, WSRC_VQ_QBS, SWI>(tx, p, grid, stream);
+  }
+  if (wsrc == WSRC_VQ_DIRECT) return launch_round<FMT_E4M3, WSRC_VQ_DIRECT, SWI>(tx, p, grid, stream);
+  if (wsrc == WSRC_VQ_SVQ) return launch_round<FMT_E4M3, WSRC_VQ_SVQ, SWI>(tx, p, grid, stream);
+  return launch_round<FMT_E4M3, WSRC_VQ_QBS, SWI>(tx, p, grid, stream);
 }
 
 // SMs of the current device (looked up once per device).
@@ -453,11 +466,19 @@ inline int device_sms() {
   return n;
 }
 
-// Grouped experts without the fused SwiGLU: the round kernel, persistent, one CTA per
-// SM walking the (128-row weight band, chunk of up to 256 rows of one expert) items.
-mxc_status launch_moe_round(const MoeArgs& m, const CUtensorMap& tx, const int32_t* tile_prefix,
-                            const int32_t* chunk_prefix, cudaStream_t stream) {
+// Grouped experts: the round kernel, persistent, one CTA per SM walking the (128-row
+// weight band, unit of one expert's rows) items -- units of up to 256 rows, or with
+// the fused SwiGLU (gate and up accumulators of one tile) of up to 128.
+mxc_status run_moe_linear(const MoeArgs& m, cudaStream_t stream) {
   const LinearArgs& a = m.base;
+  const size_t need = moe_workspace_bytes(a.M, m.E, a.N, a.K, a.fmt);
+  if (!a.ws || a.ws_bytes < need) return MXC_ERR_WORKSPACE;
+  int32_t* tile_prefix = reinterpret_cast<int32_t*>(a.ws);
+  int32_t* chunk_prefix = tile_prefix + (m.E + 1);
+  if (launch_group_prologue(m.offsets, m.E, a.M, tile_prefix, stream, chunk_prefix) != cudaSuccess)
+    return MXC_ERR_CUDA;
+  CUtensorMap tx;
+  if (!make_fp4_map(&tx, a.a_q, a.M, a.K, a.ldq, kMoeXBox)) return MXC_ERR_CUDA;   // 32-row boxes
   static thread_local MoeRoundParams p;           // about 12 KB with the expert table
   std::memset(&p, 0, sizeof(p));
   p.M = static_cast<int>(a.M);
@@ -486,78 +507,18 @@ mxc_status launch_moe_round(const MoeArgs& m, const CUtensorMap& tx, const int32
   }
   const dim3 grid(static_cast<unsigned>(device_sms()), 1, 1);
   cudaError_t err;
-  if (a.fmt == FMT_E8M0) {
-    if (a.wsrc == WSRC_VQ_DIRECT) err = launch_round<FMT_E8M0, WSRC_VQ_DIRECT>(tx, p, grid, stream);
-    else if (a.wsrc == WSRC_VQ_SVQ) err = launch_round<FMT_E8M0, WSRC_VQ_SVQ>(tx, p, grid, stream);
-    else err = launch_round<FMT_E8M0, WSRC_VQ_QBS>(tx, p, grid, stream);
-  } else {
-    if (a.wsrc == WSRC_VQ_DIRECT) err = launch_round<FMT_E4M3, WSRC_VQ_DIRECT>(tx, p, grid, stream);
-    else if (a.wsrc == WSRC_VQ_SVQ) err = launch_round<FMT_E4M3, WSRC_VQ_SVQ>(tx, p, grid, stream);
-    else err = launch_round<FMT_E4M3, WSRC_VQ_QBS>(tx, p, grid, stream);
-  }
-  return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
-}
-
-mxc_status run_moe_linear(const MoeArgs& m, cudaStream_t stream) {
-  const LinearArgs& a = m.base;
-  const size_t need = moe_workspace_bytes(a.M, m.E, a.N, a.K, a.fmt);
-  if (!a.ws || a.ws_bytes < need) return MXC_ERR_WORKSPACE;
-  int32_t* tile_prefix = reinterpret_cast<int32_t*>(a.ws);
-  int32_t* chunk_prefix = tile_prefix + (m.E + 1);
-  if (launch_group_prologue(m.offsets, m.E, a.M, tile_prefix, stream, chunk_prefix) != cudaSuccess)
-    return MXC_ERR_CUDA;
-  CUtensorMap tx;
-  if (!make_fp4_map(&tx, a.a_q, a.M, a.K, a.ldq, kMoeXBox)) return MXC_ERR_CUDA;   // 32-row boxes
-  if (!m.swiglu) return launch_moe_round(m, tx, tile_prefix, chunk_prefix, stream);
-  // GemmParams with the expert table (about 12 KB of kernel parameters).
-  static thread_local GemmParams<kMaxGroups> p;
-  std::memset(&p, 0, sizeof(p));
-  p.M = static_cast<int>(a.M);
-  p.N = static_cast<int>(a.N);
-  p.K = static_cast<int>(a.K);
-  p.qn = static_cast<int>(a.qn);
-  p.qk = static_cast<int>(a.qk);
-  p.a_sf = a.a_sf;
-  p.a_tscale = a.a_tscale;
-  p.y = a.y;
-  p.ldy = a.ldy;
-  p.out_bf16 = a.out_bf16;
-  p.splits = 1;
-  p.ks_per_split = static_cast<int>(a.K / kStageK);
-  p.E = m.E;
-  p.offsets = m.offsets;
-  p.tile_prefix = tile_prefix;
-  for (int e = 0; e < m.E; ++e) {
-    const mxc_weight& w = m.experts[e];
-    p.w[e].idx = w.idx;
-    p.w[e].cb = w.cb;
-    p.w[e].sf = w.scales;
-    p.w[e].sidx = w.sidx;
-    p.w[e].scb = w.scb;
-    p.w[e].w_tscale = w.w_tscale;
-    p.w[e].ds = w.scale_group ? w.scale_group : 8;
-  }
-  cudaError_t err;
   if (m.swiglu) {
-    // SwiGLU: each CTA owns 128 channels of h (gate rows and the matching up rows)
+    // each item owns 128 channels of h: gate rows and the matching up rows
     p.F = static_cast<int>(a.N / 2);
     p.h_q = m.h_q;
     p.ldh = m.ldh;
     p.h_sf = m.h_sf;
     p.h_tscale = m.h_tscale;
-    const dim3 grid(static_cast<unsigned>(a.N / 2 / kTileN), static_cast<unsigned>((a.M + 127) / 128 + m.E), 1);
-    if (a.fmt == FMT_E8M0) {
-      if (a.wsrc == WSRC_VQ_DIRECT) err = launch_gemm<FMT_E8M0, WSRC_VQ_DIRECT, 128, true, true>(tx, tx, p, grid, stream);
-      else if (a.wsrc == WSRC_VQ_SVQ) err = launch_gemm<FMT_E8M0, WSRC_VQ_SVQ, 128, true, true>(tx, tx, p, grid, stream);
-      else err = launch_gemm<FMT_E8M0, WSRC_VQ_QBS, 128, true, true>(tx, tx, p, grid, stream);
-    } else {
-      if (a.wsrc == WSRC_VQ_DIRECT) err = launch_gemm<FMT_E4M3, WSRC_VQ_DIRECT, 128, true, true>(tx, tx, p, grid, stream);
-      else if (a.wsrc == WSRC_VQ_SVQ) err = launch_gemm<FMT_E4M3, WSRC_VQ_SVQ, 128, true, true>(tx, tx, p, grid, stream);
-      else err = launch_gemm<FMT_E4M3, WSRC_VQ_QBS, 128, true, true>(tx, tx, p, grid, stream);
-    }
-    return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
+    err = dispatch_round<true>(a.fmt, a.wsrc, tx, p, grid, stream);
+  } else {
+    err = dispatch_round<false>(a.fmt, a.wsrc, tx, p, grid, stream);
   }
-  return MXC_ERR_UNSUPPORTED;
+  return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
 }
 
 template <int FMT, int WSRC>

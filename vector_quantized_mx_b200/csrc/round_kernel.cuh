@@ -51,6 +51,13 @@ struct MoeRoundParams {
   const int32_t* offsets;
   const int32_t* tile_prefix;         // [E+1] 128-row tiles before each expert
   const int32_t* chunk_prefix;        // [E+1] 256-row chunks before each expert
+  // fused SwiGLU (gate/up weights [2F, K]): h = SiLU(g) u, quantized for the down
+  // projection into h_q [M, ldh] and the grouped SF layout h_sf
+  int F;
+  uint8_t* h_q;
+  int64_t ldh;
+  uint8_t* h_sf;
+  const float* h_tscale;              // E4M3-B16: the given FP32 tensor scale of h
   ExpertPtrs w[kMaxGroups];
 };
 
@@ -89,40 +96,46 @@ struct RoundLayout {
   static_assert(SMEM <= 232448, "shared memory");
 };
 
-// One work item: 128 weight rows (n_tile) of expert e against one chunk of up to two
-// 128-token tiles of its rows.
+// One work item: 128 weight rows (band n_tile) of expert e against one unit of its
+// rows: a chunk of up to two 128-token tiles, or (fused SwiGLU, whose gate and up
+// accumulators take the TMEM of two tiles) one tile.
 struct RoundItem {
   int e, n_tile, nt, tile0;           // tile0: SF group of the first tile
   int64_t m0, m_end;                  // rows [m0, min(m0 + 128 nt, m_end))
 };
 
-// Item k of the launch: chunk k / n_tiles, band k mod n_tiles (consecutive CTAs take
-// the bands of one chunk, which then share its token tiles in L2).  The tables are
-// the shared-memory copies of the tile and chunk prefixes.
-__device__ __forceinline__ RoundItem round_item(int k, int n_tiles, int E, const int32_t* t_tile,
+// Item k of the launch: unit k / n_bands, band k mod n_bands (consecutive CTAs take
+// the bands of one unit, which then share its token tiles in L2).  The tables are the
+// shared-memory copies of the tile and chunk prefixes; UT = tiles per unit (1 or 2).
+template <int UT>
+__device__ __forceinline__ RoundItem round_item(int k, int n_bands, int E, const int32_t* t_tile,
                                                 const int32_t* t_chunk, const int32_t* offsets, bool rows) {
+  const int32_t* t_unit = UT == 1 ? t_tile : t_chunk;
   RoundItem it;
-  const int chunk = k / n_tiles;
-  it.n_tile = k - chunk * n_tiles;
+  const int unit = k / n_bands;
+  it.n_tile = k - unit * n_bands;
   int lo = 0, hi = E - 1;
-  while (lo < hi) {                                  // last expert whose first chunk <= chunk
+  while (lo < hi) {                                  // last expert whose first unit <= unit
     const int mid = (lo + hi + 1) >> 1;
-    if (t_chunk[mid] <= chunk) lo = mid; else hi = mid - 1;
+    if (t_unit[mid] <= unit) lo = mid; else hi = mid - 1;
   }
   it.e = lo;
-  const int c = chunk - t_chunk[lo];
-  it.nt = min(kChunkTiles, t_tile[lo + 1] - t_tile[lo] - 2 * c);
-  it.tile0 = t_tile[lo] + 2 * c;
+  const int c = unit - t_unit[lo];
+  it.nt = min(UT, t_tile[lo + 1] - t_tile[lo] - UT * c);
+  it.tile0 = t_tile[lo] + UT * c;
   it.m0 = 0;
   it.m_end = 0;
   if (rows) {
-    it.m0 = __ldg(offsets + lo) + static_cast<int64_t>(2 * c) * 128;
+    it.m0 = __ldg(offsets + lo) + static_cast<int64_t>(UT * c) * 128;
     it.m_end = __ldg(offsets + lo + 1);
   }
   return it;
 }
 
-template <int FMT, int WSRC>
+// SWI: fused SwiGLU.  An item then runs its K rounds twice, on the gate band n_tile
+// (accumulator columns [0, 128)) and on the matching up band n_tile + F/128 (columns
+// [128, 256)): virtual rounds 0 .. 2 nr - 1, the second nr on the up band.
+template <int FMT, int WSRC, bool SWI>
 __global__ void __launch_bounds__(kRoundThreads, 1)
     moe_round_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ MoeRoundParams p) {
   using L = RoundLayout<FMT, WSRC>;
@@ -130,11 +143,14 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
   static_assert(kDecWarps == 16, "decode map assumes 16 decoder warps");
 
   const int K = p.K, KS = K / kStageK, KB4 = K / L::kB / 4;
-  const int n_tiles = p.N / kTileN;
+  const int n_bands = (SWI ? p.N / 2 : p.N) / kTileN;
   const int qn = p.qn, qk = p.qk;
   const int H = qk == 128 ? 2 : 1;                   // codebooks per stage along K
   const int cb_per_row = K / qk;
-  const int nr = (KS + RS - 1) / RS;                 // rounds per item
+  const int nr = (KS + RS - 1) / RS;                 // K rounds
+  const int nrv = SWI ? 2 * nr : nr;                 // rounds per item
+  auto kr = [&](int v) { return SWI && v >= nr ? v - nr : v; };                     // K round of round v
+  auto wband = [&](const RoundItem& it, int v) { return it.n_tile + (SWI && v >= nr ? n_bands : 0); };
   auto qb_first = [&](int ks) { return H == 2 ? 2 * ks : (ks * kStageK) / qk; };
   auto qb_last = [&](int ks) { return H == 2 ? 2 * ks + 1 : (ks * kStageK) / qk; };
   auto qbn_of = [&](int n_tile) { return static_cast<int>((static_cast<int64_t>(n_tile) * 128) / qn); };
@@ -149,10 +165,12 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
   for (int i = static_cast<int>(threadIdx.x); i < 2 * (E + 1); i += kRoundThreads)
     t_tile[i] = i <= E ? p.tile_prefix[i] : p.chunk_prefix[i - (E + 1)];
   __syncthreads();
-  const int n_items = n_tiles * t_chunk[E];
+  const int n_items = n_bands * (SWI ? t_tile[E] : t_chunk[E]);
   const int k_first = blockIdx.x, k_step = gridDim.x;
   if (k_first >= n_items) return;                    // nothing for this CTA
-  auto item = [&](int k, bool rows) { return round_item(k, n_tiles, E, t_tile, t_chunk, p.offsets, rows); };
+  auto item = [&](int k, bool rows) {
+    return round_item<SWI ? 1 : kChunkTiles>(k, n_bands, E, t_tile, t_chunk, p.offsets, rows);
+  };
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::CTRL_OFF);
   // A round's weight data comes in two parts: "lo" = its codebooks, scale indices and
@@ -165,17 +183,19 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
   uint64_t* dec_ph = bars + 4;      // [2] half h (K-quarters 2h, 2h+1) of the round decoded; half 0 also
                                     //     means the round's weight scales are in TMEM
   uint64_t* xfree = bars + 8;       // MMAs of one (round, tile) done: the token buffer is free
-  uint64_t* w_free = bars + 9;      // MMAs of one round done: the operand tiles are free
+  uint64_t* w_free = bars + 9;      // MMAs of one round's half 0 done: its quarters 0-1 of the operand
+                                    //     tiles are free (w_free + 4: half 1, quarters 2-3)
   uint64_t* accum = bars + 10;      // all MMAs of an item done
-  uint64_t* acc_free = bars + 11;   // the epilogue has read an item's accumulators
+  uint64_t* acc_free = bars + 11;   // the epilogue (fused SwiGLU: the decoders) has read an item's accumulators
   uint64_t* mma_done = bars + 12;   // every MMA this CTA issued is complete (once, at the end)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
-  constexpr int kBars = 13;
+  uint64_t* w_free1 = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  constexpr int kBars = 14;
 
   // ---- setup ----
   if (warp == 0) {
     if (lane < kBars)
-      mbar_init(bars + lane, lane >= 4 && lane < 6 ? kDecWarps : lane == 11 ? kRoundEpiWarps : 1);
+      mbar_init(bars + lane, lane >= 4 && lane < 6 ? kDecWarps : lane == 11 ? (SWI ? kDecWarps : kRoundEpiWarps) : 1);
     __syncwarp();
     if (lane == 0) {
       fence_mbar_init();
@@ -194,38 +214,40 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
 
   if (warp == 0) {
     // =============================== loader ===============================
-    auto issue_lo = [&](const RoundItem& it, int r) {
+    auto issue_lo = [&](const RoundItem& it, int v) {    // round v of item it
+      const int r = kr(v), band = wband(it, v);
       const int ks0 = r * RS, rs = min(RS, KS - ks0);
       const int qb0 = qb_first(ks0), qb1 = qb_last(ks0 + rs - 1);
       const uint8_t* const w_idx = p.w[it.e].idx;
       const uint16_t* const w_cb = p.w[it.e].cb;
-      const int qbn = qbn_of(it.n_tile);
+      const int qbn = qbn_of(band);
       uint32_t tx = rs * 4096 + (qb1 - qb0 + 1) * 512;
       [[maybe_unused]] int nu = 0;
       [[maybe_unused]] const SvqGeom sv(p.w[it.e].ds, L::kB, KS);
       if constexpr (L::kSVQ) {
         nu = ((ks0 + rs - 1) >> sv.lspu) - (ks0 >> sv.lspu) + 1;
         tx += nu * 128 * sv.G;
-        if (r == 0) tx += 256 * sv.ds;
+        if (v == 0) tx += 256 * sv.ds;
       }
-      if (r == 0) {                                  // the item's later rounds on their way into L2
+      if (r == 0) {                                  // the band's later rounds on their way into L2
         for (int ks = RS; ks < KS; ks += 4)          // 32 KB a request
-          l2_prefetch_bulk(w_idx + (static_cast<size_t>(it.n_tile) * KS + ks) * 8192,
+          l2_prefetch_bulk(w_idx + (static_cast<size_t>(band) * KS + ks) * 8192,
                            static_cast<uint32_t>(min(4, KS - ks)) * 8192);
         l2_prefetch_bulk(w_cb + static_cast<size_t>(qbn) * cb_per_row * 256, static_cast<uint32_t>(cb_per_row) * 512);
       }
       mbar_arrive_expect_tx(bar_lo, tx);
       for (int s = 0; s < rs; ++s)
-        bulk_load(smem + L::IDX_OFF + s * 8192, w_idx + (static_cast<size_t>(it.n_tile) * KS + ks0 + s) * 8192, 4096,
+        bulk_load(smem + L::IDX_OFF + s * 8192, w_idx + (static_cast<size_t>(band) * KS + ks0 + s) * 8192, 4096,
                   bar_lo);
       bulk_load(smem + L::CB_OFF, w_cb + (static_cast<size_t>(qbn) * cb_per_row + qb0) * 256, (qb1 - qb0 + 1) * 512,
                 bar_lo);
       if constexpr (L::kSVQ) {
-        bulk_load(smem + L::SIDX_OFF, sv.unit(p.w[it.e].sidx, it.n_tile, ks0), nu * 128 * sv.G, bar_lo);
-        if (r == 0) bulk_load(smem + L::AUX_OFF, p.w[it.e].scb, 256 * sv.ds, bar_lo);
+        bulk_load(smem + L::SIDX_OFF, sv.unit(p.w[it.e].sidx, band, ks0), nu * 128 * sv.G, bar_lo);
+        if (v == 0) bulk_load(smem + L::AUX_OFF, p.w[it.e].scb, 256 * sv.ds, bar_lo);
       }
     };
-    auto issue_hi = [&](const RoundItem& it, int r, int g) {   // g: the global round number
+    auto issue_hi = [&](const RoundItem& it, int v, int g) {   // g: the global round number
+      const int r = kr(v), band = wband(it, v);
       const int ks0 = r * RS, rs = min(RS, KS - ks0);
       uint64_t* bar = bar_hi + (g & 1);
       const uint8_t* const w_idx = p.w[it.e].idx;
@@ -234,14 +256,14 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
       mbar_arrive_expect_tx(bar, tx);
       for (int s = 0; s < rs; ++s)
         bulk_load(smem + L::IDX_OFF + s * 8192 + 4096,
-                  w_idx + (static_cast<size_t>(it.n_tile) * KS + ks0 + s) * 8192 + 4096, 4096, bar);
+                  w_idx + (static_cast<size_t>(band) * KS + ks0 + s) * 8192 + 4096, 4096, bar);
       if constexpr (WSRC == WSRC_VQ_DIRECT)
         bulk_load(smem + L::AUX_OFF + (g & 1) * RS * A * 512,
-                  p.w[it.e].sf + (static_cast<size_t>(it.n_tile) * KB4 + static_cast<size_t>(ks0) * A) * 512,
+                  p.w[it.e].sf + (static_cast<size_t>(band) * KB4 + static_cast<size_t>(ks0) * A) * 512,
                   rs * A * 512, bar);
     };
-    auto issue_x = [&](const RoundItem& it, int r, int t) {    // tile t's tokens and their scales, round r
-      const int ks0 = r * RS, rs = min(RS, KS - ks0);
+    auto issue_x = [&](const RoundItem& it, int v, int t) {    // tile t's tokens and their scales, round v
+      const int ks0 = kr(v) * RS, rs = min(RS, KS - ks0);
       const int64_t tm0 = it.m0 + static_cast<int64_t>(t) * 128;
       const int64_t rows = it.m_end - tm0 < 128 ? it.m_end - tm0 : 128;
       const int boxes = static_cast<int>((rows + kMoeXBox - 1) / kMoeXBox);
@@ -253,6 +275,25 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
       bulk_load(smem + L::SFX_OFF,
                 p.a_sf + (static_cast<size_t>(it.tile0 + t) * KB4 + static_cast<size_t>(ks0) * A) * 512, rs * A * 512,
                 bar_x);
+    };
+    // The first round of an item into L2 while the item before it runs: its index
+    // tiles, codebooks, scale indices and scale codebook, and its first token tile.
+    auto prefetch_first_round = [&](const RoundItem& it) {
+      const int rs = min(RS, KS);
+      l2_prefetch_bulk(p.w[it.e].idx + static_cast<size_t>(it.n_tile) * KS * 8192, static_cast<uint32_t>(rs) * 8192);
+      const int qb1 = qb_last(rs - 1);
+      l2_prefetch_bulk(p.w[it.e].cb + static_cast<size_t>(qbn_of(it.n_tile)) * cb_per_row * 256,
+                       static_cast<uint32_t>(qb1 + 1) * 512);
+      if constexpr (L::kSVQ) {
+        const SvqGeom sv(p.w[it.e].ds, L::kB, KS);
+        l2_prefetch_bulk(sv.unit(p.w[it.e].sidx, it.n_tile, 0), static_cast<uint32_t>(sv.U) * 128 * sv.G);
+        l2_prefetch_bulk(p.w[it.e].scb, 256 * sv.ds);
+      }
+      const int64_t rows = it.m_end - it.m0 < 128 ? it.m_end - it.m0 : 128;
+      const int boxes = static_cast<int>((rows + kMoeXBox - 1) / kMoeXBox);
+      for (int s = 0; s < rs; ++s)
+        for (int q = 0; q < boxes; ++q)
+          l2_prefetch_tile_2d(&tmap_x, s * 128, static_cast<int>(it.m0) + q * kMoeXBox);
     };
     RoundItem cur = item(k_first, true);
     __syncwarp();
@@ -268,11 +309,14 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
     for (int k = k_first; k < n_items && ok; k += k_step) {
       const bool has_next = k + k_step < n_items;
       RoundItem nxt = cur;
-      if (has_next) nxt = item(k + k_step, true);    // loads in flight while this item runs
-      for (int r = 0; r < nr && ok; ++r, ++g) {
-        const bool next_round = r + 1 < nr || has_next;
-        const RoundItem& ni = r + 1 < nr ? cur : nxt;
-        const int nrr = r + 1 < nr ? r + 1 : 0;
+      if (has_next) {
+        nxt = item(k + k_step, true);                // loads in flight while this item runs
+        if (lane == 0) prefetch_first_round(nxt);
+      }
+      for (int r = 0; r < nrv && ok; ++r, ++g) {
+        const bool next_round = r + 1 < nrv || has_next;
+        const RoundItem& ni = r + 1 < nrv ? cur : nxt;
+        const int nrr = r + 1 < nrv ? r + 1 : 0;
         if (next_round) {
           // the decoders are done with this round's codebooks, scale indices and index
           // quarters 0-1: the next round's may come in
@@ -320,7 +364,8 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
     int g = 0, kx = 0, i = 0;
     for (int k = k_first; k < n_items && ok; k += k_step, ++i) {
       const RoundItem it = item(k, false);
-      for (int r = 0; r < nr && ok; ++r, ++g) {
+      for (int v = 0; v < nrv && ok; ++v, ++g) {
+        const int r = kr(v);
         const int ks0 = r * RS, rs = min(RS, KS - ks0);
         const uint32_t sfw_c = tmem + L::COL_SFW + (g & 1) * L::SF_COLS;
         if constexpr (!L::kSfwDec) {
@@ -343,13 +388,14 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
             for (int a = 0; a < rs * A; ++a) tc_cp_32x128b_warpx4(sfx_c + 4 * a, sdesc_sf_atom(s0 + a * 512));
           }
           __syncwarp();
-          if (i > 0 && r == 0 && t == 0) {           // the last item's accumulators have been read
+          if (i > 0 && v == 0 && t == 0) {           // the last item's accumulators have been read
             ok = __all_sync(0xffffffffu, mbar_wait(acc_free, (i - 1) & 1));
             if (!ok) break;
             tc_fence_after();
           }
           const uint32_t w_s0 = smem_u32(smem + L::W_OFF), x_s0 = smem_u32(smem + L::X_OFF);
-          const uint32_t d_t = tmem + static_cast<uint32_t>(t) * 128;
+          // tile t's accumulator; fused SwiGLU: the gate's, then (second pass) the up's
+          const uint32_t d_t = tmem + static_cast<uint32_t>(SWI ? (v >= nr ? 1 : 0) : t) * 128;
           // D[token][channel]: the tokens are the MMA's A operand (M = 128 TMEM lanes),
           // the decoded weight rows its B operand (N = 128 columns), so that each
           // epilogue thread holds one token's row of outputs
@@ -378,11 +424,15 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
               }
             }
             __syncwarp();
+            if (j == 1 && t == it.nt - 1) {          // quarters 0-1 of the operand tiles may be rewritten
+              if (elect_one()) tc_commit(w_free);
+              __syncwarp();
+            }
           }
           if (!ok) break;
           if (elect_one()) {
             tc_commit(xfree);                        // this tile's token buffer may be refilled
-            if (t == it.nt - 1) tc_commit(w_free);   // this round's operand tiles may be rewritten
+            if (t == it.nt - 1) tc_commit(w_free1);  // and quarters 2-3 of the operand tiles
           }
           __syncwarp();
         }
@@ -430,12 +480,12 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
         lut[(2 * i + 1) * 32] = wv[i] >> 16;
       }
     };
-    int g = 0;
-    for (int k = k_first; k < n_items; k += k_step) {
-      const RoundItem it = item(k, false);
+    int g = 0, di = 0;
+    for (int k = k_first; k < n_items; k += k_step, ++di) {
+      const RoundItem it = item(k, SWI);
       const SvqGeom sv(p.w[it.e].ds, L::kB, KS);
-      const uint8_t* const qbs_row = p.w[it.e].sf + static_cast<size_t>(qbn_of(it.n_tile)) * cb_per_row;
-      for (int r = 0; r < nr; ++r, ++g) {
+      for (int v = 0; v < nrv; ++v, ++g) {
+        const int r = kr(v);
         const int ks0 = r * RS, rs = min(RS, KS - ks0);
         const bool act = s_l < rs;
         const bool sf_act = sf_s < rs;
@@ -443,6 +493,7 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
         // PostScale-QB: the QBlock bytes of this warp's stage, blocks 4a.. (byte a, a < A)
         uint32_t qbs = 0u;
         if constexpr (L::kQBS) {
+          const uint8_t* const qbs_row = p.w[it.e].sf + static_cast<size_t>(qbn_of(wband(it, v))) * cb_per_row;
           if (sf_act) {
 #pragma unroll
             for (int a = 0; a < A; ++a) {
@@ -460,7 +511,8 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
         if (g > 0) named_bar_sync(2, kDecThreads);  // every lane is done with the last round's copies
         lay_out(act && landed, c0, c1);
         named_bar_sync(2, kDecThreads);              // this round's copies are complete
-        if (g > 0) mbar_wait(w_free, (g - 1) & 1);   // the last round's MMAs are done with the tiles
+        // quarters 0-1 of the operand tiles: the last round's MMAs of them are done
+        if (g > 0) mbar_wait(w_free, (g - 1) & 1);
         // Weight scale atom a of this warp's stage into TMEM (PreScale+ from the scale
         // codebook, PostScale-QB the QBlock's byte); row `lane` of the atom, column q,
         // holds block scales 4a..4a+3 of weight row 32 q + lane.
@@ -506,6 +558,7 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
           bool have = landed;
           if (h == 1) {                              // quarters 2-3 of the round's index tiles
             have = mbar_wait(bar_hi + (g & 1), (g >> 1) & 1) && landed;
+            if (g > 0) mbar_wait(w_free1, (g - 1) & 1);   // and of the operand tiles, once free
             if (H == 2) {                            // and the stage's second codebook
               named_bar_sync(2, kDecThreads);
               lay_out(act && landed, d0, d1);
@@ -537,6 +590,59 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
           if (lane == 0) mbar_arrive(&dec_ph[h]);
         }
       }
+      if constexpr (SWI) {
+        // The item's h = SiLU(g) u (gate accumulator columns [0, 128), up [128, 256))
+        // for this warp's 32 tokens (its TMEM lane quadrant) and 32 channels, column
+        // group dw/4: channels n_tile*128 + 32 (dw/4) .. + 31 of h, in blocks of B.
+        // Each block is quantized for the down projection (FP4 codes into h_q, the
+        // scale byte into the grouped SF layout); the tile's rows past the expert's
+        // get zero scales.
+        constexpr int B = L::kB;
+        const float scale = p.w[it.e].w_tscale * (p.a_tscale ? *p.a_tscale : 1.0f);
+        const float hs = FMT == FMT_E4M3 ? *p.h_tscale : 1.0f;
+        const int kbr = p.F / B;
+        const int cg = dw >> 2;
+        const int64_t q0 = it.m0 + qd * 32;
+        const bool live = q0 < it.m_end;             // warp-uniform: some token of the expert here
+        const int64_t m = q0 + lane;
+        const int64_t srow = static_cast<int64_t>(it.tile0) * 128 + qd * 32 + lane;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+        const bool ep_ok = mbar_wait(accum, di & 1);
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = cg * 32; c0 < cg * 32 + 32; c0 += B) {
+          float h[B];
+          if (live) {
+#pragma unroll
+            for (int part = 0; part < B / 8; ++part) {   // 8 columns at a time: few live registers
+              uint32_t vg[8], vu[8];
+              __syncwarp();                          // tcgen05.ld is warp-aligned
+              const uint32_t ta = lane_base + c0 + 8 * part;
+              tmem_ld_32x32b_x8(ta, vg);
+              tmem_ld_32x32b_x8(ta + 128, vu);
+              tmem_ld_wait();
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                h[8 * part + c] = swiglu_fp32(__fmul_rn(__uint_as_float(vg[c]), scale),
+                                              __fmul_rn(__uint_as_float(vu[c]), scale));
+            }
+          }
+          if (!ep_ok) continue;
+          const int kbh = (it.n_tile * 128 + c0) / B;   // block index along h's channels
+          uint32_t sfb = 0u;
+          if (live && m < it.m_end) {
+            uint32_t q[B / 8];
+            quantize_block_f32<B>(h, FMT == FMT_E4M3, hs, q, sfb);
+            uint8_t* dst = p.h_q + m * p.ldh + kbh * (B / 2);
+            if constexpr (B == 32) *reinterpret_cast<uint4*>(dst) = make_uint4(q[0], q[1], q[2], q[3]);
+            else *reinterpret_cast<uint2*>(dst) = make_uint2(q[0], q[1]);
+          }
+          p.h_sf[sf_offset(srow, kbh, kbr)] = static_cast<uint8_t>(sfb);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_free);        // the next item's MMAs may overwrite
+      }
     }
   } else {
     // ============================== epilogue ==============================
@@ -549,7 +655,8 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
     // 16-byte row stores where Y's rows allow them
     const bool vec = (reinterpret_cast<uintptr_t>(p.y) & 15u) == 0 && (ldy % (out_bf16 ? 8 : 4)) == 0;
     int i = 0;
-    for (int k = k_first; k < n_items; k += k_step, ++i) {
+    // (the fused SwiGLU's output is written by the decoder warps)
+    for (int k = k_first; k < (SWI ? 0 : n_items); k += k_step, ++i) {
       const RoundItem it = item(k, true);
       const float scale = p.w[it.e].w_tscale * a_ts;
       const bool ep_ok = mbar_wait(accum, i & 1);
