@@ -1,15 +1,17 @@
-"""Host replay of the grouped-expert (MoE) tile and chunk schedulers.
+"""Host replay of the grouped-expert (MoE) schedule.
 
-Device side (act_quant.cuh group_prologue_kernel, mma_kernel.cuh gemm_kernel<MOE>):
+Device side (act_quant.cuh group_prologue_kernel, round_kernel.cuh moe_round_kernel):
 the prologue turns expert offsets into tile_prefix[g] = sum over g' < g of
-ceil(rows_g' / 128); the launch has ceil(M/128) + E row tiles; row tile t with
-t < tile_prefix[E] belongs to the last expert e whose tile_prefix[e] <= t (binary
-search) and covers rows [offsets[e] + 128 (t - tile_prefix[e]), offsets[e+1]) clipped
-to 128 rows; later row tiles exit.  Its scale rows are group t of the grouped
-quantizer's padded SF layout.  This replay checks, for many offset patterns (empty
-experts, single rows, multiples of 128, one huge expert), that the launch has
-enough row tiles and that every expert row is computed exactly once, by a tile of
-its own expert, and no tile reaches into another expert.
+ceil(rows_g' / 128) and chunk_prefix[g] = sum over g' < g of ceil(tiles_g' / 2).
+The persistent kernel's work items are (unit, 128-row weight band) pairs; a unit is a
+chunk of up to two 128-row tiles of one expert (plain linear) or one tile (fused
+SwiGLU).  Unit u belongs to the last expert e whose prefix entry is <= u (binary
+search) and covers rows [offsets[e] + 128 t, offsets[e+1]) clipped to its tiles; its
+scale rows are groups tile_prefix[e] + t of the grouped quantizer's padded SF layout.
+These replays check, for many offset patterns (empty experts, single rows, multiples
+of 128, one huge expert), that every expert row is computed exactly once, by a unit
+of its own expert, that no unit reaches into another expert, and that every scale
+group is read by exactly one tile.
 """
 import numpy as np
 import pytest
@@ -33,15 +35,13 @@ def owner(prefix, E, t):
 
 
 def replay(offsets):
+    """Single-tile units (fused SwiGLU items)."""
     E = len(offsets) - 1
     M = int(offsets[-1])
     prefix = tile_prefix(offsets)
-    grid_tiles = (M + 127) // 128 + E
-    assert grid_tiles >= prefix[E]
+    assert prefix[E] <= (M + 127) // 128 + E
     cover = np.zeros(M, dtype=np.int64)
-    for t in range(grid_tiles):
-        if t >= prefix[E]:
-            continue                     # the CTA exits
+    for t in range(prefix[E]):
         e = owner(prefix, E, t)
         m0 = offsets[e] + (t - prefix[e]) * 128
         m1 = min(m0 + 128, offsets[e + 1])
@@ -70,20 +70,16 @@ def chunk_prefix(offsets):
 
 
 def replay_chunks(offsets):
-    """round_kernel.cuh moe_round_kernel: chunk c of the launch's ceil(M/256) + E
-    belongs to the last expert e with chunk_prefix[e] <= c; it runs the expert's
-    128-row tiles 2 (c - chunk_prefix[e]) and the next one if the expert has it,
-    scale groups tile_prefix[e] + those tile numbers."""
+    """Units of up to two tiles (plain linear items): unit c belongs to the last expert e
+    with chunk_prefix[e] <= c and runs the expert's tiles 2 (c - chunk_prefix[e]) and the
+    next one if the expert has it, scale groups tile_prefix[e] + those tile numbers."""
     E = len(offsets) - 1
     M = int(offsets[-1])
     tp, cp = tile_prefix(offsets), chunk_prefix(offsets)
-    grid_chunks = (M + 255) // 256 + E
-    assert grid_chunks >= cp[E]
+    assert cp[E] <= (M + 255) // 256 + E
     cover = np.zeros(M, dtype=np.int64)
     groups = np.zeros(tp[E], dtype=np.int64)
-    for c in range(grid_chunks):
-        if c >= cp[E]:
-            continue
+    for c in range(cp[E]):
         e = owner(cp, E, c)
         k = c - cp[e]
         nt = min(2, tp[e + 1] - tp[e] - 2 * k)

@@ -214,11 +214,11 @@ size_t moe_workspace_bytes(int64_t /*M*/, int32_t E, int64_t /*N*/, int64_t /*K*
 // ------------------------------------------------------------------------------------
 // Launch
 // ------------------------------------------------------------------------------------
-template <int FMT, int WSRC, int T, bool MOE, int NCB, bool SWI = false>
-cudaError_t launch_gemm_ncb(const CUtensorMap& tx, const CUtensorMap& tw,
-                            const GemmParams<MOE ? kMaxGroups : 1>& p, dim3 grid, cudaStream_t stream) {
-  using L = StageLayout<FMT, WSRC, T, NCB, SWI ? 2 : 1>;
-  auto kern = gemm_kernel<FMT, WSRC, T, MOE, NCB, SWI>;
+template <int FMT, int WSRC, int T, int NCB>
+cudaError_t launch_gemm_ncb(const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams<1>& p, dim3 grid,
+                            cudaStream_t stream) {
+  using L = StageLayout<FMT, WSRC, T, NCB>;
+  auto kern = gemm_kernel<FMT, WSRC, T, NCB>;
   static uint64_t attr_set = 0;
   cudaError_t err = ensure_smem_attr(kern, L::SMEM, &attr_set);
   if (err != cudaSuccess) return err;
@@ -242,19 +242,19 @@ cudaError_t launch_gemm_ncb(const CUtensorMap& tx, const CUtensorMap& tw,
 }
 
 // Two codebooks per stage only for VQ weights whose QBlock is 128 wide along K.
-template <int FMT, int WSRC, int T, bool MOE, bool SWI = false>
-cudaError_t launch_gemm(const CUtensorMap& tx, const CUtensorMap& tw,
-                        const GemmParams<MOE ? kMaxGroups : 1>& p, dim3 grid, cudaStream_t stream) {
+template <int FMT, int WSRC, int T>
+cudaError_t launch_gemm(const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams<1>& p, dim3 grid,
+                        cudaStream_t stream) {
   if constexpr (WSRC != WSRC_NATIVE) {
-    if (p.qk == 128) return launch_gemm_ncb<FMT, WSRC, T, MOE, 2, SWI>(tx, tw, p, grid, stream);
+    if (p.qk == 128) return launch_gemm_ncb<FMT, WSRC, T, 2>(tx, tw, p, grid, stream);
   }
-  return launch_gemm_ncb<FMT, WSRC, T, MOE, 1, SWI>(tx, tw, p, grid, stream);
+  return launch_gemm_ncb<FMT, WSRC, T, 1>(tx, tw, p, grid, stream);
 }
 
 template <int FMT, int WSRC, int T>
 cudaError_t dispatch_dense(const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams<1>& p, dim3 grid,
                            cudaStream_t stream) {
-  return launch_gemm<FMT, WSRC, T, false>(tx, tw, p, grid, stream);
+  return launch_gemm<FMT, WSRC, T>(tx, tw, p, grid, stream);
 }
 
 template <int FMT, int WSRC>

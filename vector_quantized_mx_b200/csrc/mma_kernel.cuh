@@ -69,23 +69,12 @@ struct GemmParams {
   int64_t ldy;
   int out_bf16;
   int splits, ks_per_split;  // split-K over a cluster of `splits` CTAs (1 = off)
-  int E;                     // MoE
-  const int32_t* offsets;
-  const int32_t* tile_prefix;
-  // MoE gate/up with SwiGLU: h = SiLU(gate) * up is quantized straight into the
-  // down projection's activation (F = N / 2 channels)
-  int F;
-  uint8_t* h_q;              // FP4 [M, ldh]
-  int64_t ldh;
-  uint8_t* h_sf;             // grouped SF layout of [rows, F / B]
-  const float* h_tscale;     // E4M3-B16: the given FP32 tensor scale of h
   ExpertPtrs w[NEXP];
 };
 
 // Shared-memory layout of one pipeline stage and of the whole CTA.  NCB = codebooks
-// per 256-channel stage: 2 when the QBlock is 128 wide along K, else 1.  NACC =
-// accumulators in TMEM (2 for the SwiGLU gate/up pair).
-template <int FMT, int WSRC, int T, int NCB = 1, int NACC = 1>
+// per 256-channel stage: 2 when the QBlock is 128 wide along K, else 1.
+template <int FMT, int WSRC, int T, int NCB = 1>
 struct StageLayout {
   static constexpr bool kVQ = WSRC != WSRC_NATIVE;
   static constexpr bool kSVQ = WSRC == WSRC_VQ_SVQ;
@@ -112,11 +101,10 @@ struct StageLayout {
   static constexpr int LUT_OFF = CTRL + STAGES * BYTES;
   static constexpr int RED_OFF = LUT_OFF + LUT;
   static constexpr int SMEM = 1024 + RED_OFF + RED;
-  // TMEM columns: accumulators [0, NACC*T), weight scales [NACC*T, NACC*T+16), token
-  // scales after.
-  static constexpr int COL_SFW = NACC * T;
-  static constexpr int COL_SFX = NACC * T + 16;
-  static constexpr int COLS_USED = NACC * T + 16 + 16 * kXG;
+  // TMEM columns: accumulator [0, T), weight scales [T, T+16), token scales after.
+  static constexpr int COL_SFW = T;
+  static constexpr int COL_SFX = T + 16;
+  static constexpr int COLS_USED = T + 16 + 16 * kXG;
   static constexpr int TMEM_COLS = COLS_USED <= 32 ? 32 : COLS_USED <= 64 ? 64 : COLS_USED <= 128 ? 128
                                    : COLS_USED <= 256 ? 256 : 512;
   static_assert(STAGES >= 2, "stage does not fit");
@@ -301,12 +289,11 @@ __device__ __forceinline__ void store_out(void* y, int64_t ldy, int out_bf16, in
 // ------------------------------------------------------------------------------------
 // The kernel
 // ------------------------------------------------------------------------------------
-template <int FMT, int WSRC, int T, bool MOE, int NCB, bool SWI = false>
+template <int FMT, int WSRC, int T, int NCB>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_wq,
-                const __grid_constant__ GemmParams<MOE ? kMaxGroups : 1> p) {
-  static_assert(!SWI || (MOE && T == 128), "SwiGLU runs on MoE gate/up tiles of 128 tokens");
-  using L = StageLayout<FMT, WSRC, T, NCB, SWI ? 2 : 1>;
+                const __grid_constant__ GemmParams<1> p) {
+  using L = StageLayout<FMT, WSRC, T, NCB>;
   constexpr int STAGES = L::STAGES;
   constexpr int A = L::kAtoms;
   constexpr int XG = L::kXG;
@@ -330,35 +317,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- which tile this CTA owns ----
   const int n_tile = blockIdx.x;
-  int64_t m0, m_end;
-  int sf_group0, ks_begin = 0, ks_end = KS, split = 0;
   const ExpertPtrs* wp = &p.w[0];
-  if constexpr (MOE) {
-    const int tile = blockIdx.y;
-    if (tile >= p.tile_prefix[p.E]) return;          // beyond this call's tile count
-    int lo = 0, hi = p.E - 1;
-    while (lo < hi) {                                // last expert whose first tile <= tile
-      const int mid = (lo + hi + 1) >> 1;
-      if (p.tile_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
-    }
-    m0 = p.offsets[lo] + static_cast<int64_t>(tile - p.tile_prefix[lo]) * 128;
-    m_end = p.offsets[lo + 1];
-    sf_group0 = tile;
-    wp = &p.w[lo];
-  } else {
-    m0 = static_cast<int64_t>(blockIdx.y) * T;
-    m_end = p.M;
-    sf_group0 = static_cast<int>(m0 / 128);
-    split = blockIdx.z;
-    ks_begin = split * p.ks_per_split;
-    ks_end = min(KS, ks_begin + p.ks_per_split);
-  }
+  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * T;
+  const int64_t m_end = p.M;
+  const int sf_group0 = static_cast<int>(m0 / 128);
+  const int split = blockIdx.z;
+  const int ks_begin = split * p.ks_per_split;
+  const int ks_end = min(KS, ks_begin + p.ks_per_split);
   const int nks = ks_end - ks_begin;
-  // SwiGLU: the CTA runs the gate tile (weight rows of band n_tile) and then the up
-  // tile (band n_tile + F/128) over the same tokens: 2 * nks pipeline stages, the
-  // second pass into the second accumulator.
-  const int nst = SWI ? 2 * nks : nks;
-  const int up_band = SWI ? p.F / 128 : 0;
+  const int nst = nks;
   // Loop invariants in registers (the asm statements below clobber "memory").
   const uint8_t* const w_idx = wp->idx;
   const uint16_t* const w_cb = wp->cb;
@@ -418,22 +385,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr bool cb_split = NCB == 2;
     // Token scale groups that exist: the SF buffer holds ceil(M/128) groups of 128
     // rows (dense) -- a 256-token tile at the end of M may cover only one.
-    int xg_valid = XG;
-    if constexpr (!MOE) {
-      const int groups = static_cast<int>((static_cast<int64_t>(p.M) + 127) / 128);
-      xg_valid = groups - sf_group0 < XG ? groups - sf_group0 : XG;
-    }
-    // Expert tiles load only the 32-row boxes that hold the expert's rows (most
-    // experts own far fewer than 128): the rows of the neighbouring experts would
-    // be wasted ingest.  Columns past the expert's rows are computed on stale
-    // (finite: E2M1 has no NaN) shared memory and never stored.
-    int x_boxes = 1, x_box_bytes = T * 128;
-    if constexpr (MOE) {
-      const int64_t rows = m_end - m0 < T ? m_end - m0 : T;
-      x_boxes = static_cast<int>((rows + kMoeXBox - 1) / kMoeXBox);
-      x_box_bytes = kMoeXBox * 128;
-    }
-    uint32_t tx = x_boxes * x_box_bytes + xg_valid * A * 512;
+    const int groups = static_cast<int>((static_cast<int64_t>(p.M) + 127) / 128);
+    const int xg_valid = groups - sf_group0 < XG ? groups - sf_group0 : XG;
+    uint32_t tx = T * 128 + xg_valid * A * 512;
     if constexpr (WSRC == WSRC_NATIVE) tx += 16384 + A * 512;
     if constexpr (WSRC == WSRC_VQ_DIRECT) tx += 8192 + (cb_split ? 1024 : 512) + A * 512;
     if constexpr (WSRC == WSRC_VQ_SVQ) tx += 8192 + (cb_split ? 1024 : 512) + 128 * sv.G;
@@ -446,17 +400,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ph = (i / STAGES) & 1;
       if (i >= STAGES && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1))) break;
       if (elect_one()) {
-        const bool up = SWI && i >= nks;             // SwiGLU: second pass, the up tile
-        const int ks = ks_begin + (up ? i - nks : i);
-        const int band = n_tile + (up ? up_band : 0);
+        const int ks = ks_begin + i;
+        const int band = n_tile;
         const int qbn = static_cast<int>((static_cast<int64_t>(band) * 128) / qn);
         const uint8_t* sfw_src = w_sf + static_cast<size_t>(band) * KB4 * 512;
         const uint8_t* idx_src = w_idx + static_cast<size_t>(band) * KS * 8192;
         const uint16_t* cb_src = w_cb + static_cast<size_t>(qbn) * cb_per_row * 256;
         uint8_t* st = stages + s * L::BYTES;
         mbar_arrive_expect_tx(&full[s], tx);
-        for (int q = 0; q < x_boxes; ++q)
-          tma_load_2d(st + L::X_OFF + q * x_box_bytes, &tmap_x, ks * 128, y0 + q * kMoeXBox, &full[s]);
+        tma_load_2d(st + L::X_OFF, &tmap_x, ks * 128, y0, &full[s]);
 #pragma unroll
         for (int g = 0; g < XG; ++g)
           if (g < xg_valid)                          // a missing group's rows are past M: never stored
@@ -517,9 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_cp_32x128b_warpx4(tmem + L::COL_SFW + 4 * a, sdesc_sf_atom(sfw_s + a * 512));
         }
         const uint32_t w_s = smem_u32(st + L::W_OFF), x_s = smem_u32(st + L::X_OFF);
-        const bool up = SWI && i >= nks;             // SwiGLU: the up tile accumulates apart
-        const int il = up ? i - nks : i;
-        const uint32_t d_t = tmem + (up ? static_cast<uint32_t>(T) : 0u);
+        const int il = i;
+        const uint32_t d_t = tmem;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const uint64_t adesc = sdesc_kmajor_sw128(w_s + 32 * j);
@@ -579,9 +530,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* st = stages + s * L::BYTES;
         uint32_t qs0 = 0, qs1 = 0;                   // PostScale-QB: the stage's QBlock scale(s),
         if constexpr (L::kQBS) {                     // loaded before the decode hides their latency
-          const bool up = SWI && i >= nks;
-          const int ks = ks_begin + (up ? i - nks : i);
-          const int qbn_w = static_cast<int>((static_cast<int64_t>(n_tile + (up ? up_band : 0)) * 128) / qn);
+          const int ks = ks_begin + i;
+          const int qbn_w = static_cast<int>((static_cast<int64_t>(n_tile) * 128) / qn);
           const uint8_t* qb = w_sf + static_cast<size_t>(qbn_w) * (K / qk);
           const int qbk = cb_split ? 2 * ks : (ks * kStageK) / qk;
           qs0 = __ldg(qb + qbk);
@@ -589,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         decode_w_tile<GT>(st + L::IDX_OFF, lut_s + b * kBuf, st + L::W_OFF, cm);
         if constexpr (L::kSVQ) {
-          const int ks = ks_begin + (SWI && i >= nks ? i - nks : i);
+          const int ks = ks_begin + i;
           decode_sf_tile<A, GT>(st + L::SIDX_OFF, sv.G, scb32, sv_lds, sv.kb_base(ks, L::kB), st + L::SFW_OFF, gt);
         }
         if constexpr (L::kQBS) fill_sf_qbs<A, GT>(st + L::SFW_OFF, qs0, qs1, gt);
@@ -618,58 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t ldy = p.ldy;
     const int out_bf16 = p.out_bf16;
     const uint32_t taddr = tmem + (static_cast<uint32_t>(qd * 32) << 16) + chalf * TCOL;
-    if constexpr (SWI) {
-      // Gate accumulator at columns [0, T), up at [T, 2T): this thread holds channel
-      // `row` (a TMEM lane) of both for this warp's TCOL tokens.  Phase 1: h = SiLU(g) * u
-      // in FP32 into a [128 tokens][HS] staging table over the pipeline stages (all
-      // copies, decodes and MMAs are done by now).  Phase 2: each thread quantizes
-      // whole blocks (one token, B consecutive channels) for the down projection:
-      // FP4 codes into h_q, block scales into the grouped SF layout (padding rows of
-      // the expert's tile get zero scales).
-      constexpr int HS = 132;                          // padded rows: conflict-free 16-byte reads
-      static_assert(128 * HS * 4 <= STAGES * L::BYTES, "h staging fits in the pipeline stages");
-      float* const hst = reinterpret_cast<float*>(stages);
-      const bool wok = __all_sync(0xffffffffu, ep_ok);
-#pragma unroll 1
-      for (int c0 = 0; c0 < TCOL; c0 += 16) {
-        uint32_t vg[16], vu[16];
-        __syncwarp();                                  // tcgen05.ld is warp-aligned
-        tmem_ld_32x32b_x16(taddr + c0, vg);
-        tmem_ld_32x32b_x16(taddr + T + c0, vu);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          hst[(chalf * TCOL + c0 + c) * HS + row] =
-              swiglu_fp32(__fmul_rn(__uint_as_float(vg[c]), scale), __fmul_rn(__uint_as_float(vu[c]), scale));
-      }
-      named_bar_sync(4, kDecThreads);                  // the staging table is complete
-      if (wok) {
-        constexpr int B = L::kB, NB = 128 / B;         // blocks of one token in this tile
-        const float hs = FMT == FMT_E4M3 ? *p.h_tscale : 1.0f;
-        const int kbr = p.F / B;                       // h blocks per row
-        for (int u = threadIdx.x - 64; u < 128 * NB; u += kDecThreads) {
-          const int t = u & 127, b = u >> 7;
-          const int64_t m = m0 + t;
-          const float4* src = reinterpret_cast<const float4*>(hst + t * HS + b * B);
-          float v[B];
-#pragma unroll
-          for (int i = 0; i < B / 4; ++i) {
-            const float4 f = src[i];
-            v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
-          }
-          uint32_t q[B / 8], sfb;
-          quantize_block_f32<B>(v, FMT == FMT_E4M3, hs, q, sfb);
-          const int kb = n_tile * NB + b;              // block index along h's channels
-          if (m < m_end) {
-            uint8_t* dst = p.h_q + m * p.ldh + kb * (B / 2);
-            if constexpr (B == 32) *reinterpret_cast<uint4*>(dst) = make_uint4(q[0], q[1], q[2], q[3]);
-            else *reinterpret_cast<uint2*>(dst) = make_uint2(q[0], q[1]);
-          }
-          p.h_sf[sf_offset(static_cast<int64_t>(sf_group0) * 128 + t, kb, kbr)] =
-              static_cast<uint8_t>(m < m_end ? sfb : 0u);
-        }
-      }
-    } else if constexpr (T <= 32) {
+    if constexpr (T <= 32) {
       // this warp's accumulator columns in registers: one TMEM round trip
       __syncwarp();                                  // tcgen05.ld is warp-aligned: converge after the waits
       if constexpr (TCOL == 4) tmem_ld_32x32b_x4(taddr, acc_regs);
@@ -718,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);
   }
-  if constexpr (T <= 32 && !MOE) {
+  if constexpr (T <= 32) {
     if (splits > 1) {
       // All partial tiles have landed in rank 0's shared memory after this barrier.
       __syncwarp();
