@@ -7,6 +7,7 @@ decode_native   mxc_native_linear on the same decoded weights
 prefill         mxc_linear, PreScale E8M0-B32, M=2048, K=4096, N=9216 (BF16 out)
 prefill_native  mxc_native_linear on the same decoded weights
 moe             mxc_moe_linear, PreScale+ E4M3-B16, gate/up 3072x4096, 128 experts, Zipf(1.1) top-8
+swiglu          mxc_moe_gate_up_swiglu on the same gate/up weights and rows
 quant           mxc_quantize_act, E8M0-B32, 8192 x 4096 BF16
 Each case checks the device error word after its launches.
 """
@@ -26,7 +27,7 @@ def _dev_bf16(bits, dev):
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["decode", "decode_native", "prefill", "prefill_native", "moe", "quant"])
+    ap.add_argument("case", choices=["decode", "decode_native", "prefill", "prefill_native", "moe", "swiglu", "quant"])
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args(argv)
     build.build()
@@ -48,14 +49,18 @@ def main(argv=None):
                 mxc.linear(a, pw, torch.bfloat16)
             else:
                 mxc.native_linear(a, nat, torch.bfloat16)
-    elif args.case == "moe":
+    elif args.case in ("moe", "swiglu"):
         row_tok, off = synth.config4_routing()
         xg = synth.config4_activations("gate_up", row_tok)
         experts = [mxc.pack_weight(synth.config4_expert(e, "gate_up"), dev) for e in range(synth.MOE_EXPERTS)]
         offd = torch.from_numpy(off.astype(np.int32)).to(dev)
         a = mxc.quantize_act_grouped(_dev_bf16(xg, dev), "e4m3_b16", offd)
+        h_ts = torch.tensor([0.01], dtype=torch.float32, device=dev)
         for _ in range(args.reps):
-            mxc.moe_linear(a, offd, experts, torch.bfloat16)
+            if args.case == "moe":
+                mxc.moe_linear(a, offd, experts, torch.bfloat16)
+            else:
+                mxc.moe_gate_up_swiglu(a, offd, experts, h_tscale=h_ts)
     else:
         x = synth.make_activations(3, 8192, 4096, outliers=True)
         xd = _dev_bf16(x, dev)
