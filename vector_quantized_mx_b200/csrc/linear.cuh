@@ -5,6 +5,7 @@
 #include <atomic>
 #include <cstring>
 
+#include "pair_kernel.cuh"
 #include "round_kernel.cuh"
 
 namespace mxc {
@@ -132,6 +133,25 @@ inline bool encode_idx_map(CUtensorMap* map, const void* base, int64_t N, int64_
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// 2-D map over an SF-layout scale buffer seen as rows of one 512-byte atom (64
+// eight-byte elements): dims {64, atoms}; one box = box_atoms consecutive atoms.
+inline bool encode_sf_map(CUtensorMap* map, const void* base, int64_t atoms, int box_atoms) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return false;
+  std::memset(map, 0, sizeof(*map));
+  const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(atoms)};
+  const cuuint64_t strides[1] = {512};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_atoms)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+inline bool make_sf_map(CUtensorMap* map, const void* base, int64_t atoms, int box_atoms) {
+  return cached_map(map, MapKey{4, base, atoms, box_atoms, 0, 0},
+                    [&](CUtensorMap* m) { return encode_sf_map(m, base, atoms, box_atoms); });
+}
+
 inline bool make_idx_map(CUtensorMap* map, const void* base, int64_t N, int64_t K, int box_stages) {
   return cached_map(map, MapKey{3, base, N, K, box_stages, 0},
                     [&](CUtensorMap* m) { return encode_idx_map(m, base, N, K, box_stages); });
@@ -323,6 +343,52 @@ inline ExpertPtrs expert_ptrs(const LinearArgs& a) {
 
 mxc_status run_decode_weight(const DecodeArgs& a, cudaStream_t stream);
 
+// SMs of the current device (looked up once per device).
+inline int device_sms() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kSMs;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = kSMs;
+  cached[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// Native weights, 256-token tiles, N a multiple of 256: CTA pairs (tcgen05 cta_group::2)
+// of 256 weight rows x 256 tokens.
+template <int FMT>
+cudaError_t launch_pair(const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams<1>& p, cudaStream_t stream) {
+  using L = PairLayout<FMT>;
+  const int64_t KB4 = p.K / L::kB / 4;
+  CUtensorMap tsx, tsw;
+  if (!make_sf_map(&tsx, p.a_sf, (static_cast<int64_t>(p.M) + 127) / 128 * KB4, L::A) ||
+      !make_sf_map(&tsw, p.w[0].sf, static_cast<int64_t>(p.N) / 128 * KB4, L::A))
+    return cudaErrorInvalidValue;
+  auto kern = gemm_pair_kernel<FMT>;
+  static uint64_t attr_set = 0;
+  cudaError_t err = ensure_smem_attr(kern, L::SMEM, &attr_set);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  const int64_t tiles = static_cast<int64_t>(p.N / 256) * ((p.M + 255) / 256);
+  const int64_t pairs = std::min<int64_t>(device_sms() / 2, tiles);
+  if (pairs <= 0) return cudaSuccess;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = L::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, kern, tx, tw, tsx, tsw, p);
+  if (err != cudaSuccess) return err;
+  return cudaGetLastError();
+}
+
 mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
   const bool small = a.wsrc != WSRC_NATIVE && small_qblock(a.qn, a.qk);
   const bool ws_ok = a.ws && a.ws_bytes >= decoded_weight_bytes(a.N, a.K, a.fmt) &&
@@ -359,8 +425,9 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
     return run_linear(b, stream);
   }
   const int T = token_tile(a.M);
+  const bool pair = a.wsrc == WSRC_NATIVE && T == 256 && a.N % 256 == 0;
   CUtensorMap tx, tw;
-  if (!make_fp4_map(&tx, a.a_q, a.M, a.K, a.ldq, T)) return MXC_ERR_CUDA;
+  if (!make_fp4_map(&tx, a.a_q, a.M, a.K, a.ldq, pair ? 128 : T)) return MXC_ERR_CUDA;
   if (a.wsrc == WSRC_NATIVE) {
     if (!make_fp4_map(&tw, a.w_q, a.N, a.K, a.w_ldq, 128)) return MXC_ERR_CUDA;
   } else {
@@ -382,6 +449,11 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
   p.ks_per_split = static_cast<int>(a.K / kStageK);
   p.w[0] = expert_ptrs(a);
   if (a.wsrc == WSRC_NATIVE) p.w[0].sf = a.w_sf;
+  if (pair) {
+    const cudaError_t err = a.fmt == FMT_E8M0 ? launch_pair<FMT_E8M0>(tx, tw, p, stream)
+                                              : launch_pair<FMT_E4M3>(tx, tw, p, stream);
+    return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
+  }
   const int n_tiles = static_cast<int>(a.N / kTileN);
   const int m_tiles = static_cast<int>((a.M + T - 1) / T);
   if (T == 16) {
@@ -454,17 +526,6 @@ cudaError_t dispatch_round(int fmt, int wsrc, const CUtensorMap& tx, const MoeRo
   return launch_round<FMT_E4M3, WSRC_VQ_QBS, SWI>(tx, p, grid, stream);
 }
 
-// SMs of the current device (looked up once per device).
-inline int device_sms() {
-  static std::atomic<int> cached[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kSMs;
-  int n = cached[dev].load(std::memory_order_relaxed);
-  if (n > 0) return n;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = kSMs;
-  cached[dev].store(n, std::memory_order_relaxed);
-  return n;
-}
 
 // Grouped experts: the round kernel, persistent, one CTA per SM walking the (128-row
 // weight band, unit of one expert's rows) items -- units of up to 256 rows, or with
