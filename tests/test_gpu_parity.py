@@ -221,6 +221,34 @@ def test_mxcode_equals_native_on_decoded_weights(fmt, M, strat):
     assert torch.equal(y, yn)
 
 
+@pytest.mark.parametrize("fmt", ["e8m0_b32", "e4m3_b16"])
+@pytest.mark.parametrize("M,K", [(129, 256), (300, 1536), (700, 1024), (1000, 4096)])
+@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
+def test_pair_gemm_equals_one_cta(fmt, M, K, out):
+    """Native weights with 256-token tiles and N a multiple of 256 run on CTA pairs
+    (cta_group::2, persistent); with N = 384 the one-CTA kernel runs.  On the same
+    decoded operands the first 384 output channels must agree bit for bit, ragged
+    token tiles included (a pair's second half past M), one stage (K = 256) included,
+    and lie within the oracle's bound."""
+    w = synth.make_weight(61, fmt, "prescale", 512, K, 256, 256)
+    x = synth.make_activations(61, M, K, outliers=True)
+    pw = mxc.pack_weight(w)
+    wn = mxc.decode_weight(pw)
+    a = mxc.quantize_act(dev_bf16(x), fmt)
+    y = mxc.native_linear(a, wn, out)                              # N = 512: CTA pairs
+    B = 32 if fmt == "e8m0_b32" else 16
+    rows = 384                                                      # 128-row scale blocks are contiguous
+    w384 = mxc.MXTensor(wn.q[:rows].contiguous(), wn.sf.view(-1)[: rows * K // B].contiguous(), wn.tscale,
+                        rows, K, fmt)
+    y384 = mxc.native_linear(a, w384, out)                          # N = 384: one CTA per tile
+    assert mxc.get_device_error() == 0
+    assert torch.equal(y[:, :rows], y384)
+    ref, sabs = O.w4a4_linear(x, w)
+    yy = y.float().cpu().numpy()
+    bound = sabs if out == torch.float32 else sabs + np.abs(ref) * 2.0 ** -8 / TOL
+    assert_close(yy, ref, bound, what=f"pair {fmt} M={M} K={K}")
+
+
 def test_bf16_output():
     w = synth.make_weight(51, "e4m3_b16", "prescale", 256, 1024, 256, 256)
     x = synth.make_activations(51, 40, 1024, outliers=True)

@@ -152,6 +152,25 @@ inline bool make_sf_map(CUtensorMap* map, const void* base, int64_t atoms, int b
                     [&](CUtensorMap* m) { return encode_sf_map(m, base, atoms, box_atoms); });
 }
 
+// 2-D map over a BF16 output [rows, ld] (cols used): box 64 x 128 rows, 128-byte
+// swizzle (the layout of the GEMM's output staging).
+inline bool encode_bf16_out_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return false;
+  std::memset(map, 0, sizeof(*map));
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+inline bool make_bf16_out_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld) {
+  return cached_map(map, MapKey{5, base, rows, cols, ld, 0},
+                    [&](CUtensorMap* m) { return encode_bf16_out_map(m, base, rows, cols, ld); });
+}
+
 inline bool make_idx_map(CUtensorMap* map, const void* base, int64_t N, int64_t K, int box_stages) {
   return cached_map(map, MapKey{3, base, N, K, box_stages, 0},
                     [&](CUtensorMap* m) { return encode_idx_map(m, base, N, K, box_stages); });
@@ -365,6 +384,13 @@ cudaError_t launch_pair(const CUtensorMap& tx, const CUtensorMap& tw, const Gemm
   if (!make_sf_map(&tsx, p.a_sf, (static_cast<int64_t>(p.M) + 127) / 128 * KB4, L::A) ||
       !make_sf_map(&tsw, p.w[0].sf, static_cast<int64_t>(p.N) / 128 * KB4, L::A))
     return cudaErrorInvalidValue;
+  // BF16 output with 16-byte aligned rows: staged tiles written by tensor stores
+  CUtensorMap ty = tx;
+  int y_tma = 0;
+  if (p.out_bf16 && (reinterpret_cast<uintptr_t>(p.y) & 15u) == 0 && p.ldy % 8 == 0) {
+    if (!make_bf16_out_map(&ty, p.y, p.M, p.N, p.ldy)) return cudaErrorInvalidValue;
+    y_tma = 1;
+  }
   auto kern = gemm_pair_kernel<FMT>;
   static uint64_t attr_set = 0;
   cudaError_t err = ensure_smem_attr(kern, L::SMEM, &attr_set);
@@ -384,7 +410,7 @@ cudaError_t launch_pair(const CUtensorMap& tx, const CUtensorMap& tw, const Gemm
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  err = cudaLaunchKernelEx(&cfg, kern, tx, tw, tsx, tsw, p);
+  err = cudaLaunchKernelEx(&cfg, kern, tx, tw, tsx, tsw, ty, y_tma, p);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }

@@ -34,14 +34,18 @@ struct PairLayout {
   static constexpr int SFW_OFF = SFX_OFF + A * 512;          // 2 x A atoms: the pair's 256 weight rows
   static constexpr int BYTES = ((SFW_OFF + 2 * A * 512) + 1023) / 1024 * 1024;
   static constexpr int CTRL = 1024;                          // barriers and the TMEM slot
-  static constexpr int STAGES_FIT = (227 * 1024 - 1024 - CTRL) / BYTES;
+  // BF16 output staging: four [128 tokens][64 weight rows] sub-tiles of 128-byte rows
+  // in the 128-byte swizzle, written out by tensor stores
+  static constexpr int OUT_BYTES = 4 * 16384;
+  static constexpr int STAGES_FIT = (227 * 1024 - 1024 - CTRL - OUT_BYTES) / BYTES;
   // TMEM: accumulator [0, 256) (lanes = this CTA's tokens, columns = the pair's 256
   // weight rows); per stage slot 12 A columns of scales (tokens: 4 A, weights: 8 A,
   // the two 128-row groups interleaved)
   static constexpr int SF_COLS = 12 * A;
   static constexpr int STAGES_TMEM = (512 - 256) / SF_COLS;
   static constexpr int STAGES = STAGES_FIT < STAGES_TMEM ? STAGES_FIT : STAGES_TMEM;
-  static constexpr int SMEM = 1024 + CTRL + STAGES * BYTES;
+  static constexpr int OUT_OFF = CTRL + STAGES * BYTES;      // from the aligned base
+  static constexpr int SMEM = 1024 + OUT_OFF + OUT_BYTES;
   static_assert(STAGES >= 3, "pipeline depth");
   static_assert(SMEM <= 232448, "shared memory");
 };
@@ -105,6 +109,29 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
       : "memory");
 }
+// Two FP32 values rounded to nearest-even BF16 (the hardware conversion), lo in the
+// low half.
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Tensor store of a shared-memory box (bulk async group of this thread).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, const void* src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(smem_u32(src))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// This thread's committed bulk groups have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// ... and are complete.
+__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void tc_cp_pair_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
@@ -118,6 +145,7 @@ template <int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                      const __grid_constant__ CUtensorMap tmap_sfx, const __grid_constant__ CUtensorMap tmap_sfw,
+                     const __grid_constant__ CUtensorMap tmap_y, const int y_tma,
                      const __grid_constant__ GemmParams<1> p) {
   using L = PairLayout<FMT>;
   constexpr int STAGES = L::STAGES;
@@ -129,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);   // [STAGES] rank 0: both CTAs' copies of a stage landed
   uint64_t* empty = full + STAGES;                      // [STAGES] the pair's MMAs of a stage are done
   uint64_t* accum = empty + STAGES;                     // a tile's MMAs are done
-  uint64_t* acc_free = accum + 1;                       // rank 0: both CTAs' epilogues have read the tile
+  uint64_t* acc_free = accum + 1;                       // rank 0: both CTAs' epilogue warps have read the tile
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_free + 1);
   uint8_t* stages = smem + L::CTRL;
 
@@ -149,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(accum, 1);
-    mbar_init(acc_free, 2);                             // one arrival from each CTA's epilogue
+    mbar_init(acc_free, 2 * kDecWarps);                 // every epilogue warp of both CTAs
     fence_mbar_init();
     prefetch_tensormap(&tmap_x);
     prefetch_tensormap(&tmap_w);
@@ -275,12 +303,59 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t ldy = p.ldy;
     const bool vec = (reinterpret_cast<uintptr_t>(p.y) & 15u) == 0 && (ldy % (out_bf16 ? 8 : 4)) == 0;
     const uint32_t acc_free0 = mapa_shared(smem_u32(acc_free), 0);
+    uint8_t* const out_stage = smem + L::OUT_OFF;
     int j = 0;
     for (int t = pair; t < n_tiles; t += pairs, ++j) {
       const int n0p = (t % n_pn) * 256;
       const int64_t q0 = static_cast<int64_t>(t / n_pn) * 256 + 128 * rank + qd * 32;
       const bool ep_ok = mbar_wait(accum, j & 1);
       tc_fence_after();
+      if (y_tma) {
+        // BF16 rows through the staging sub-tiles and tensor stores: warp (qd, cg) writes
+        // rows 32 qd .. + 31 of sub-tile cg (weight rows n0p + 64 cg .. + 63), 16-byte
+        // chunk c of row r at chunk c ^ (r mod 8) -- the 128-byte swizzle of the store map.
+        if (threadIdx.x == 64) bulk_wait_group_read0();   // the last tile's stores have read the staging
+        named_bar_sync(1, kDecThreads);
+        const bool live = q0 < p.M;                     // warp-uniform: some token of this quadrant exists
+        // the warp's 64 columns into registers, release the accumulator, then the BF16
+        // staging stores
+        uint32_t v[64];
+        if (live) {
+          __syncwarp();                                 // tcgen05.ld is warp-aligned
+          const uint32_t ta = tmem + (static_cast<uint32_t>(qd * 32) << 16) + cg * 64;
+          tmem_ld_32x32b_x32(ta, v);
+          tmem_ld_32x32b_x32(ta + 32, v + 32);
+          tmem_ld_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {                                // the next tile's MMAs may start
+          if (rank == 0) mbar_arrive(acc_free);
+          else mbar_remote_arrive(acc_free0);
+        }
+        if (live) {
+          const int r = qd * 32 + lane;
+          uint8_t* const row = out_stage + cg * 16384 + r * 128;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {                 // 16-byte chunk k of the row
+            uint32_t h2[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              h2[c] = bf16x2_rn(__uint_as_float(v[8 * k + 2 * c]) * scale, __uint_as_float(v[8 * k + 2 * c + 1]) * scale);
+            *reinterpret_cast<uint4*>(row + ((k ^ (r & 7)) << 4)) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
+          }
+        }
+        fence_proxy_async_smem();                       // staging writes -> the tensor stores' reads
+        named_bar_sync(1, kDecThreads);                 // staging complete
+        if (threadIdx.x == 64) {
+          const int y0 = static_cast<int>(t / n_pn) * 256 + 128 * static_cast<int>(rank);
+          if (ep_ok && y0 < p.M) {                      // rows past M are clipped by the map
+            for (int g = 0; g < 4; ++g) tma_store_2d(&tmap_y, n0p + 64 * g, y0, out_stage + g * 16384);
+            bulk_commit_group();
+          }
+        }
+        continue;
+      }
       if (q0 < p.M) {                                   // warp-uniform: some token of this quadrant exists
         const int64_t m = q0 + lane;
         const bool row_ok = ep_ok && m < p.M;
@@ -326,14 +401,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      named_bar_sync(1, kDecThreads);                   // all 16 warps are done with the accumulator
-      if (threadIdx.x == 64) {
+      __syncwarp();
+      if (lane == 0) {                                  // this warp is done with the accumulator
         if (rank == 0) mbar_arrive(acc_free);
         else mbar_remote_arrive(acc_free0);
       }
     }
   }
 
+  if (threadIdx.x == 64) bulk_wait_group0();           // the output stores are done
   __syncwarp();
   tc_fence_before();
   __syncthreads();
