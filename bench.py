@@ -492,7 +492,7 @@ def prefill_leg(dev, stream, capture, time_graph, steps, world, with_cpu):
            "tflops_step": world * flops / (ms["step"] * 1e-3) / 1e12,
            "weight_GBps": world * wbytes / (ms["linear"] * 1e-3) / 1e9,
            "roofline": {"bound": "tensor", "unit": "TFLOP/s", "peak": peak, "peak_kind": peak_kind,
-                        "kernel": "gemm_kernel<E8M0, native, T=256> (the GEMM of the decode-once path)",
+                        "kernel": "gemm_pair_kernel<E8M0> (persistent CTA-pair native GEMM of the decode-once path)",
                         "ms_per_launch": ms["native_linear"], "flops_per_launch": flops,
                         "achieved": flops / (ms["native_linear"] * 1e-3) / 1e12,
                         "frac": flops / (ms["native_linear"] * 1e-3) / 1e12 / peak,
@@ -577,7 +577,7 @@ def moe_leg(dev, stream, capture, time_graph, steps, world, with_cpu):
         out[name] = {"ms_linear": ms_lin, "tflops": world * p["flops"] / (ms_lin * 1e-3) / 1e12,
                      "weight_GBps": world * p["bytes"] / (ms_lin * 1e-3) / 1e9, "weight_bytes": p["bytes"],
                      "roofline": {"bound": "hbm" if t_bw >= t_fl else "tensor",
-                                  "kernel": "gemm_kernel<E4M3, VQ scale-VQ, T=128, MoE> + group prologue",
+                                  "kernel": "moe_round_kernel<E4M3, VQ scale-VQ> (persistent) + group prologue",
                                   "target_ms": max(t_bw, t_fl), "frac": max(t_bw, t_fl) / ms_lin,
                                   "hbm_peak_GBps": hbm, "hbm_kind": hbm_kind,
                                   "fp4_peak_TFLOPs": peak, "fp4_kind": peak_kind, "traffic": None}}

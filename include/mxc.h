@@ -192,10 +192,11 @@ mxc_status mxc_pack_weight(const mxc_weight_host* w, uint8_t* idx_out, uint8_t* 
 
 /* Workspace bytes each GPU call needs (0 if none).  M = activation rows;
  * for mxc_moe_linear M is the total number of (token, expert) rows.
- * mxc_linear: 0 below 1024 rows; from 1024 rows the room for the weight decoded
- * once per call (N*K/2 bytes of FP4 codes rounded up to 1 KiB, then N*K/B bytes
- * of SF-layout scales).  A smaller workspace is not an error there: the call
- * then runs the fused decode-in-GEMM kernel, which is slower at that size.
+ * mxc_linear: 0 up to 128 rows; above 128 rows when N is a multiple of 256 (else
+ * from 1024 rows) the room for the weight decoded once per call (N*K/2 bytes of
+ * FP4 codes rounded up to 1 KiB, then N*K/B bytes of SF-layout scales).  A smaller
+ * workspace is not an error there: the call then runs the fused decode-in-GEMM
+ * kernel, which is slower at those sizes.
  * mxc_moe_linear and mxc_moe_gate_up_swiglu: the expert tile and chunk tables,
  * 2 (E+1) int32 rounded up to whole 256-byte units. */
 size_t mxc_quantize_act_workspace_bytes(int64_t M, int64_t K, mxc_format fmt);
@@ -254,10 +255,11 @@ mxc_status mxc_quantize_act_grouped(const void* x_bf16, int64_t M, int64_t K, in
  * y         device, [M, ldy] elements of y_dtype (ldy >= N)
  * ws        device workspace of mxc_linear_workspace_bytes() bytes (16-byte aligned)
  * M <= 16 takes the split-K decode path; larger M the tiled prefill path, which
- * decodes each weight tile inside the GEMM.  From 1024 rows, with the workspace
- * given, the call instead decodes the weight once into it (MX-native FP4 codes
- * and scales, the output of mxc_decode_weight) and runs the native block-scaled
- * GEMM on that: the same operands in the same K order, so the same result bits. */
+ * decodes each weight tile inside the GEMM.  Above 128 rows when N is a multiple
+ * of 256 (else from 1024 rows), with the workspace given, the call instead decodes
+ * the weight once into it (MX-native FP4 codes and scales, the output of
+ * mxc_decode_weight) and runs the native block-scaled GEMM on that: the same
+ * operands in the same K order, so the same result bits. */
 mxc_status mxc_linear(const mxc_mx_tensor* a, const mxc_weight* w, void* y, int64_t ldy,
                       mxc_dtype y_dtype, void* ws, size_t ws_bytes, mxc_stream_t stream);
 

@@ -142,10 +142,14 @@ def test_packed_sizes_rejects_bad_shapes(L):
 
 
 def test_workspace_sizes(L):
-    # from 1024 tokens: the decoded weight (FP4 codes, then the SF-layout scales)
+    # decode once: the decoded weight (FP4 codes, then the SF-layout scales), above 128
+    # tokens when N is a multiple of 256 (the CTA-pair GEMM), else from 1024 tokens
     assert L.mxc_linear_workspace_bytes(4096, 9216, 4096, 1) == 9216 * 4096 // 2 + 9216 * 4096 // 16
     assert L.mxc_linear_workspace_bytes(1024, 9216, 4096, 0) == 9216 * 4096 // 2 + 9216 * 4096 // 32
-    assert L.mxc_linear_workspace_bytes(1023, 9216, 4096, 1) == 0          # fused tiles: none
+    assert L.mxc_linear_workspace_bytes(129, 9216, 4096, 1) == 9216 * 4096 // 2 + 9216 * 4096 // 16
+    assert L.mxc_linear_workspace_bytes(128, 9216, 4096, 1) == 0           # fused tiles: none
+    assert L.mxc_linear_workspace_bytes(1023, 9344, 4096, 1) == 0          # N % 256 != 0: fused below 1024
+    assert L.mxc_linear_workspace_bytes(1024, 9344, 4096, 1) == 9344 * 4096 // 2 + 9344 * 4096 // 16
     assert L.mxc_linear_workspace_bytes(16, 9216, 4096, 1) == 0            # decode: split-K in cluster SMEM
     assert L.mxc_moe_workspace_bytes(16384, 128, 3072, 4096, 1) >= 129 * 4
     assert L.mxc_grouped_sf_rows_bound(16384, 128) == 16384 + 128 * 128

@@ -216,14 +216,16 @@ inline void decode_splits(int64_t N, int64_t K, int* splits, int* ks_per_split) 
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// From this many tokens on, the layer decodes its weight once per call into the
-// workspace (native FP4 codes + SF-layout scales: MX-native operands, never a
-// high-precision weight) and runs the native block-scaled GEMM on it: a token tile
-// of the fused kernel decodes the weight tiles it needs again, which costs more
-// than one decode pass once the tokens fill several tiles per weight tile
-// (measured on B200: fused faster below 1024 tokens, decode-once 1.1x faster at
-// 1024 and 1.4x at 8192 for K = 4096, N = 9216).
+// Decode once: the layer decodes its weight once per call into the workspace (native
+// FP4 codes + SF-layout scales: MX-native operands, never a high-precision weight)
+// and runs the native block-scaled GEMM on it, instead of the fused kernel in which
+// every token tile decodes again the weight tiles it multiplies.  With 256-token
+// tiles and N a multiple of 256 the native GEMM runs on CTA pairs, and decoding
+// once wins from the first 256-token tile on (measured on B200, K = 4096, N = 9216:
+// equal at 130 tokens, 28 vs 43 us at 768; K = N = 8192: 37 vs 42 us at 130);
+// otherwise the one-CTA native GEMM makes it pay from 1024 tokens on.
 constexpr int64_t kDecodeOnceMinM = 1024;
+inline bool decode_once(int64_t M, int64_t N) { return M >= kDecodeOnceMinM || (M > 128 && N % 256 == 0); }
 
 inline size_t decoded_codes_bytes(int64_t N, int64_t K) { return align_up(static_cast<size_t>(N * K / 2), 1024); }
 inline size_t decoded_weight_bytes(int64_t N, int64_t K, int fmt) {
@@ -231,9 +233,9 @@ inline size_t decoded_weight_bytes(int64_t N, int64_t K, int fmt) {
 }
 
 // Small M: split-K partial sums stay in cluster shared memory, no workspace.
-// M >= kDecodeOnceMinM: room for the decoded weight (without it the fused kernel runs).
+// Decode once (above): room for the decoded weight (without it the fused kernel runs).
 size_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt) {
-  return M >= kDecodeOnceMinM ? decoded_weight_bytes(N, K, fmt) : 0;
+  return decode_once(M, N) ? decoded_weight_bytes(N, K, fmt) : 0;
 }
 
 // QBlocks of 64 rows or 64 input channels: a 128 x 256 tile-stage draws on up to 8
@@ -420,7 +422,7 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
   const bool ws_ok = a.ws && a.ws_bytes >= decoded_weight_bytes(a.N, a.K, a.fmt) &&
                      reinterpret_cast<uintptr_t>(a.ws) % 16 == 0;
   if (small && !ws_ok) return MXC_ERR_WORKSPACE;
-  if (a.wsrc != WSRC_NATIVE && (small || a.M >= kDecodeOnceMinM) && ws_ok) {
+  if (a.wsrc != WSRC_NATIVE && (small || decode_once(a.M, a.N)) && ws_ok) {
     // decode once into the workspace, then the native GEMM on the decoded operands
     DecodeArgs d{};
     d.wsrc = a.wsrc;
