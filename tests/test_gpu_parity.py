@@ -391,8 +391,8 @@ def test_config3_full_size_prefill():
 @pytest.mark.parametrize("M", [16, 1024])
 def test_config5_full_size_point(M):
     """K = N = 8192, PreScale E4M3-B16 with 256 x 256 QBlocks: M=16 (decode, pipelined
-    fallback: 16 stages per split) and M=1024 (decode-once); oracle tile + checksums,
-    and equality with native FP4 on the decoded weight."""
+    kernel: 16 stages per split) and M=1024 (decode-once); oracle tile + checksums, and
+    equality with native FP4 on the decoded weight."""
     w = synth.config5_weight(256, "prescale", "e4m3_b16")
     x = synth.config5_activations(M)
     pw = mxc.pack_weight(w)
@@ -546,3 +546,56 @@ def test_small_qblock_moe_is_refused():
     with pytest.raises(mxc.MxcError) as e:
         mxc.moe_linear(a, off, [w])
     assert e.value.status == 2                       # MXC_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------------------
+# Decode GEMV with split-K through the workspace (more than two ranks, or slices
+# past 8 stages): no cluster, the last rank to arrive sums the partials in rank order
+# ---------------------------------------------------------------------------
+
+def _splitk_ws_layout(N, K, M=16):
+    n = mxc.lib().mxc_linear_workspace_bytes(M, N, K, 1)
+    ctr = (N // 128 * 4 + 255) // 256 * 256
+    return n, ctr
+
+
+@pytest.mark.parametrize("fmt,strat,N,K,M", [
+    ("e4m3_b16", "postscale", 512, 4096, 16),      # 4 ranks of 4 stages (cluster path: same split)
+    ("e8m0_b32", "prescale", 256, 8192, 1),        # 4 ranks of 8 stages (cluster path: same split)
+    ("e4m3_b16", "prescale_plus", 256, 9216, 16),  # 5 ranks, the last one 4 stages (cluster path: none)
+    ("e8m0_b32", "postscale_qb", 256, 12288, 7),   # 6 ranks of 8 stages
+    ("e4m3_b16", "native", 512, 2048, 16),         # native FP4 weights, 4 ranks of 2 stages
+])
+def test_gemv_splitk_through_workspace(fmt, strat, N, K, M):
+    native = strat == "native"
+    w = synth.make_weight(131, fmt, "prescale" if native else strat, N, K, 256, 256)
+    x = synth.make_activations(131, M, K, outliers=True)
+    a = mxc.quantize_act(dev_bf16(x), fmt)
+    pw = mxc.pack_weight(w)
+    wt = mxc.decode_weight(pw) if native else pw
+    call = mxc.native_linear if native else mxc.linear
+    n, ctr = _splitk_ws_layout(N, K, M)
+    assert n > ctr
+    ws = mxc.linear_workspace(M, N, K, fmt, "cuda")
+    y = call(a, wt, ws=ws)
+    assert mxc.get_device_error() == 0
+    assert torch.count_nonzero(ws[:ctr]).item() == 0          # every counter back at zero
+    ref, sabs = O.w4a4_linear(x, w)
+    assert_close(y.cpu().numpy(), ref, sabs, what=f"{fmt} {strat} N={N} K={K} M={M}")
+    # deterministic: the same bits again, and BF16 output is the rounding of FP32
+    y2 = call(a, wt, ws=ws)
+    yb = call(a, wt, out_dtype=torch.bfloat16, ws=ws)
+    assert mxc.get_device_error() == 0
+    assert torch.equal(y, y2)
+    assert torch.equal(yb, y.to(torch.bfloat16))
+    assert torch.count_nonzero(ws[:ctr]).item() == 0
+    if not native:
+        assert torch.equal(y, mxc.native_linear(a, mxc.decode_weight(pw)))
+    # without the workspace the split-K cluster path runs; where it splits K the same
+    # way (at most 4 ranks of at most 8 stages) it gives the same bits
+    yc = call(a, wt, ws=torch.zeros((16,), dtype=torch.uint8, device="cuda"))
+    assert mxc.get_device_error() == 0
+    if K // 256 <= 32 and (K // 256) % 4 == 0:
+        assert torch.equal(y, yc)
+    else:
+        assert_close(yc.cpu().numpy(), ref, sabs, what=f"{fmt} {strat} N={N} K={K} M={M} (no workspace)")

@@ -36,7 +36,14 @@
 //     their order); more ranks or BF16 output: the partial tiles go to rank 0 as
 //     one 8 KB bulk copy between shared memories (completion on an mbarrier there,
 //     an acknowledgement back before the sender may exit) and rank 0 adds the
-//     scaled partials in rank order (for two ranks the same FP32 value).
+//     scaled partials in rank order (for two ranks the same FP32 value);
+//   * split-K through the workspace (more than two ranks, or slices of K past one
+//     CTA's 8 resident stages, when the caller gives the room): no cluster -- a
+//     cluster of four one-CTA-per-SM CTAs cannot be placed in one wave -- each
+//     rank writes its scaled partial tile to the workspace and takes a ticket from
+//     the tile's arrival counter (atomicInc wrapping at splits - 1, so the counter
+//     is back at zero after every call); the rank that arrives last adds the
+//     partials in rank order, the same FP32 value as the paths above.
 //
 // Programmatic dependent launch: only the token tiles, the token scales and the
 // activation tensor scale come from the previous kernel (typically the activation
@@ -70,6 +77,8 @@ struct GemvParams {
   int out_bf16;
   int splits, ks_per_split;
   ExpertPtrs w;
+  float* red_part;            // workspace split-K: [tile][rank][128][16] scaled partials, or null
+  unsigned int* red_ctr;      // workspace split-K: one arrival counter per output tile (zero on entry)
 };
 
 template <int FMT, int WSRC>
@@ -165,7 +174,9 @@ __global__ void __maxnreg__(64)
   const int ks_begin = blockIdx.z * p.ks_per_split;
   const int ks_end = min(KS, ks_begin + p.ks_per_split);
   const int nks = ks_end - ks_begin;
-  const uint32_t rank = splits > 1 ? cluster_ctarank() : 0u;
+  const bool red_ws = p.red_part != nullptr;                     // split-K through the workspace
+  const bool clustered = splits > 1 && !red_ws;                 // the split CTAs of a tile are a cluster
+  const uint32_t rank = red_ws ? blockIdx.z : clustered ? cluster_ctarank() : 0u;
   const int H = (L::kVQ && p.qk == 128) ? 2 : 1;     // codebooks per stage along K
   const int qbn = L::kVQ ? static_cast<int>((static_cast<int64_t>(n_tile) * 128) / p.qn) : 0;
   const int cb_per_row = L::kVQ ? K / p.qk : 0;
@@ -178,7 +189,7 @@ __global__ void __maxnreg__(64)
   const uint8_t* const a_sf =
       p.a_sf + (static_cast<size_t>(sf_group0) * KB4 + static_cast<size_t>(ks_begin) * A) * 512;
   const int red_off = L::IDX_OFF;                               // rank 0's receive area
-  const bool red_atomic = splits == 2 && !p.out_bf16;           // split-K by global reductions
+  const bool red_atomic = clustered && splits == 2 && !p.out_bf16;   // split-K by global reductions
   // codebooks used by the slice: a contiguous range [qb0, qb1] of the band's row
   const int qb0 = !L::kVQ ? 0 : H == 2 ? 2 * ks_begin : (ks_begin * kStageK) / p.qk;
   const int qb1 = !L::kVQ ? 0 : H == 2 ? 2 * ks_end - 1 : ((ks_end - 1) * kStageK) / p.qk;
@@ -192,7 +203,7 @@ __global__ void __maxnreg__(64)
   }
   if (warp == 0 && lane == 0) {
     // rank 0 expects every other rank's partial tile; armed before it lets them send
-    if (splits > 1 && rank == 0) mbar_arrive_expect_tx(red_full, (splits - 1) * 128 * kGemvT * 4);
+    if (clustered && rank == 0) mbar_arrive_expect_tx(red_full, (splits - 1) * 128 * kGemvT * 4);
     fence_mbar_init();
     prefetch_tensormap(&tmap_x);
     if constexpr (WSRC == WSRC_NATIVE) prefetch_tensormap(&tmap_wq);
@@ -242,12 +253,12 @@ __global__ void __maxnreg__(64)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (splits > 1) {
+  if (clustered) {
     __syncwarp();
     cluster_arrive_relaxed();                        // barriers above are initialised (fenced)
   }
   griddep_launch_dependents();
-  if (splits > 1) {
+  if (clustered) {
     __syncwarp();
     cluster_wait_acquire();                          // every CTA of the cluster is set up
   }
@@ -322,7 +333,7 @@ __global__ void __maxnreg__(64)
       if constexpr (!L::kSVQ && !L::kQBS) mbar_wait(bar_sfw, 0);
     }
     __syncwarp();
-    if (splits > 1 && rank == 0 && !red_atomic) {
+    if (clustered && rank == 0 && !red_atomic) {
       // Let the other ranks send their partials once the receive area (the index
       // buffers) is free: after the last decode phase.  Sent even after a failed
       // wait, so that no rank waits for the signal in vain.
@@ -570,6 +581,42 @@ __global__ void __maxnreg__(64)
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           if (mbase + c < p.M) atomicAdd(y + (mbase + c) * p.ldy + n, __fmul_rn(v[c], scale));
+      }
+    } else if (red_ws) {
+      // the scaled partial into this rank's slot; the last rank to arrive at the
+      // tile's counter adds all partials in rank order (products and sums rounded
+      // separately, no fused multiply-add: the value of the other split-K paths)
+      store = false;
+      const size_t tile = static_cast<size_t>(blockIdx.y) * gridDim.x + n_tile;
+      float* const part = p.red_part + tile * splits * (128 * kGemvT);
+      const int off = row * kGemvT + cg * 4;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) v[c] = __fmul_rn(v[c], scale);
+      const float4 own = make_float4(v[0], v[1], v[2], v[3]);
+      __stcg(reinterpret_cast<float4*>(part + static_cast<size_t>(rank) * (128 * kGemvT) + off), own);
+      __threadfence();                               // the partial is visible before the ticket
+      named_bar_sync(2, kDecThreads);
+      uint32_t* const last = reinterpret_cast<uint32_t*>(bars + 25);
+      if (threadIdx.x == 64)                         // every CTA arrives once, also after a failed wait
+        *last = atomicInc(p.red_ctr + tile, static_cast<unsigned>(splits - 1)) == static_cast<unsigned>(splits - 1);
+      named_bar_sync(2, kDecThreads);
+      if (*last) {
+        __threadfence();                             // the other ranks' partials are visible
+        float4 a = rank == 0 ? own : __ldcg(reinterpret_cast<const float4*>(part + off));
+        for (int r = 1; r < splits; ++r) {
+          const float4 o = r == static_cast<int>(rank)
+                               ? own
+                               : __ldcg(reinterpret_cast<const float4*>(part + static_cast<size_t>(r) * (128 * kGemvT) + off));
+          a.x = __fadd_rn(a.x, o.x);
+          a.y = __fadd_rn(a.y, o.y);
+          a.z = __fadd_rn(a.z, o.z);
+          a.w = __fadd_rn(a.w, o.w);
+        }
+        v[0] = a.x;
+        v[1] = a.y;
+        v[2] = a.z;
+        v[3] = a.w;
+        store = ep_ok;
       }
     } else if (splits > 1) {
       if (rank != 0) {

@@ -216,6 +216,37 @@ inline void decode_splits(int64_t N, int64_t K, int* splits, int* ks_per_split) 
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Split-K of the decode path through the workspace: when a tile would need more than
+// two cluster ranks, or slices longer than the GEMV's 8 resident stages, its ranks run
+// without a cluster (a cluster of four one-CTA-per-SM CTAs does not fit one wave) and
+// reduce through the workspace: one arrival counter per output tile (zero on entry,
+// zero again at exit), then [tile][rank][128][16] FP32 scaled partials.  Ranks: the
+// fewest that give slices of at most 8 stages, and no fewer than the cluster split;
+// only while all CTAs fit one wave (N = 4608, K = 8192: 9.8 us against 14.9 us on
+// clusters of four; past one wave the pipelined kernel is faster: K = N = 8192 16.3
+// against 16.7 us, N = 18432, K = 4096 15.1 against 17.1 us).
+constexpr int kGemvWsMaxSplits = 16;
+inline bool gemv_ws_split(int64_t N, int64_t K, int* splits, int* ks_per_split) {
+  int s, per;
+  decode_splits(N, K, &s, &per);
+  if (s <= 2 && per <= kGemvMaxStages) return false;   // the two-rank cluster path
+  const int KS = static_cast<int>(K / kStageK);
+  int n = (KS + kGemvMaxStages - 1) / kGemvMaxStages;
+  n = n < s ? s : n;
+  per = (KS + n - 1) / n;
+  n = (KS + per - 1) / per;
+  if (n > kGemvWsMaxSplits || (N / kTileN) * n > kSMs) return false;
+  *splits = n;
+  *ks_per_split = per;
+  return true;
+}
+inline size_t splitk_ctr_bytes(int64_t N) { return align_up(static_cast<size_t>(N / kTileN) * 4, 256); }
+inline size_t splitk_ws_bytes(int64_t M, int64_t N, int64_t K) {
+  int s, per;
+  if (M > kDecodeMaxM || !gemv_ws_split(N, K, &s, &per)) return 0;
+  return splitk_ctr_bytes(N) + static_cast<size_t>(N / kTileN) * s * 128 * kGemvT * 4;
+}
+
 // Decode once: the layer decodes its weight once per call into the workspace (native
 // FP4 codes + SF-layout scales: MX-native operands, never a high-precision weight)
 // and runs the native block-scaled GEMM on it, instead of the fused kernel in which
@@ -232,10 +263,11 @@ inline size_t decoded_weight_bytes(int64_t N, int64_t K, int fmt) {
   return decoded_codes_bytes(N, K) + static_cast<size_t>(N * K / (fmt == FMT_E8M0 ? 32 : 16));
 }
 
-// Small M: split-K partial sums stay in cluster shared memory, no workspace.
+// Small M: the split-K area when the shape reduces through the workspace (else the
+// partial sums stay in cluster shared memory and no workspace is needed).
 // Decode once (above): room for the decoded weight (without it the fused kernel runs).
 size_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt) {
-  return decode_once(M, N) ? decoded_weight_bytes(N, K, fmt) : 0;
+  return decode_once(M, N) ? decoded_weight_bytes(N, K, fmt) : splitk_ws_bytes(M, N, K);
 }
 
 // QBlocks of 64 rows or 64 input channels: a 128 x 256 tile-stage draws on up to 8
@@ -244,7 +276,8 @@ size_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt) {
 inline bool small_qblock(int64_t qn, int64_t qk) { return qn < kTileN || qk < 128; }
 
 size_t linear_workspace_bytes_for(int64_t M, int64_t N, int64_t K, int fmt, int64_t qn, int64_t qk) {
-  return small_qblock(qn, qk) ? decoded_weight_bytes(N, K, fmt) : linear_workspace_bytes(M, N, K, fmt);
+  return small_qblock(qn, qk) ? decoded_weight_bytes(N, K, fmt) + splitk_ws_bytes(M, N, K)
+                               : linear_workspace_bytes(M, N, K, fmt);
 }
 
 // The expert tile prefix and chunk prefix, (E + 1) int32 each.
@@ -327,7 +360,7 @@ cudaError_t launch_gemv(const CUtensorMap& tx, const CUtensorMap& tw, const CUte
   attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[na].val.programmaticStreamSerializationAllowed = 1;
   ++na;
-  if (p.splits > 1) {
+  if (p.splits > 1 && p.red_part == nullptr) {
     attr[na].id = cudaLaunchAttributeClusterDimension;
     attr[na].val.clusterDim.x = 1;
     attr[na].val.clusterDim.y = 1;
@@ -448,8 +481,9 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
     b.w_ldq = d.ldq;
     b.w_sf = d.sf_out;
     b.w_tscale_dev = nullptr;                      // the weight tensor scale stays b.w_tscale
-    b.ws = nullptr;
-    b.ws_bytes = 0;
+    const size_t used = decoded_weight_bytes(a.N, a.K, a.fmt);   // the rest may hold the split-K area
+    b.ws = a.ws_bytes > used ? static_cast<uint8_t*>(a.ws) + used : nullptr;
+    b.ws_bytes = a.ws_bytes > used ? a.ws_bytes - used : 0;
     return run_linear(b, stream);
   }
   const int T = token_tile(a.M);
@@ -487,9 +521,19 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
   if (T == 16) {
     int splits, per;
     decode_splits(a.N, a.K, &splits, &per);
+    float* red_part = nullptr;
+    unsigned int* red_ctr = nullptr;
+    int ws_splits, ws_per;
+    if (a.M <= kDecodeMaxM && gemv_ws_split(a.N, a.K, &ws_splits, &ws_per) && a.ws &&
+        a.ws_bytes >= splitk_ws_bytes(a.M, a.N, a.K) && reinterpret_cast<uintptr_t>(a.ws) % 16 == 0) {
+      splits = ws_splits;
+      per = ws_per;
+      red_ctr = static_cast<unsigned int*>(a.ws);
+      red_part = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) + splitk_ctr_bytes(a.N));
+    }
     p.splits = splits;
     p.ks_per_split = per;
-    if (per <= kGemvMaxStages && splits <= kGemvMaxSplits) {
+    if (per <= kGemvMaxStages && (splits <= kGemvMaxSplits || red_part)) {
       CUtensorMap tx3, ti = tw;
       if (!make_fp4_stage_map(&tx3, a.a_q, a.M, a.K, a.ldq, kGemvT, per)) return MXC_ERR_CUDA;
       if (a.wsrc != WSRC_NATIVE && !make_idx_map(&ti, a.w_idx, a.N, a.K, per)) return MXC_ERR_CUDA;
@@ -508,6 +552,8 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
       g.splits = splits;
       g.ks_per_split = per;
       g.w = p.w[0];
+      g.red_part = red_part;
+      g.red_ctr = red_ctr;
       const dim3 grid(n_tiles, m_tiles, splits);
       const cudaError_t err = a.fmt == FMT_E8M0 ? dispatch_gemv<FMT_E8M0>(a.wsrc, tx3, tw, ti, g, grid, stream)
                                                 : dispatch_gemv<FMT_E4M3>(a.wsrc, tx3, tw, ti, g, grid, stream);

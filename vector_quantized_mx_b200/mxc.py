@@ -294,8 +294,10 @@ def _out(M: int, N: int, dtype, dev) -> torch.Tensor:
 
 
 def linear_workspace(M: int, N: int, K: int, fmt: str, device) -> torch.Tensor:
+    """Workspace of mxc_linear / mxc_native_linear, zero-filled (its split-K arrival
+    counters must be zero when a call starts; every call leaves them zero)."""
     n = lib().mxc_linear_workspace_bytes(M, N, K, FMT[fmt])
-    return torch.empty((max(n, 16),), dtype=torch.uint8, device=device)
+    return torch.zeros((max(n, 16),), dtype=torch.uint8, device=device)
 
 
 def linear(a: MXTensor, w: PackedWeight, out_dtype=torch.float32, y: Optional[torch.Tensor] = None,
@@ -306,7 +308,7 @@ def linear(a: MXTensor, w: PackedWeight, out_dtype=torch.float32, y: Optional[to
     at, wt = a._c(), w._c()
     if ws is None:
         n = lib().mxc_linear_workspace_bytes_for(ctypes.byref(wt), a.rows)
-        ws = torch.empty((max(n, 16),), dtype=torch.uint8, device=dev)
+        ws = torch.zeros((max(n, 16),), dtype=torch.uint8, device=dev)
     _check(lib().mxc_linear(ctypes.byref(at), ctypes.byref(wt), y.data_ptr(), y.stride(0), OUT[y.dtype],
                             ws.data_ptr(), ws.numel(), _stream(stream)), "mxc_linear")
     return y
