@@ -599,3 +599,38 @@ def test_gemv_splitk_through_workspace(fmt, strat, N, K, M):
         assert torch.equal(y, yc)
     else:
         assert_close(yc.cpu().numpy(), ref, sabs, what=f"{fmt} {strat} N={N} K={K} M={M} (no workspace)")
+
+
+# ---------------------------------------------------------------------------
+# Decode GEMV slices of 9 to 16 stages: two rounds of 8 resident stages per CTA
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt,strat,N,K,qk,M,out,ws", [
+    ("e4m3_b16", "postscale", 6400, 4608, 256, 16, torch.float32, True),       # 2 ranks of 9: red.global.add
+    ("e8m0_b32", "prescale", 4864, 7680, 128, 5, torch.bfloat16, True),        # 3 ranks of 10: cluster sum, 2 codebooks a stage
+    ("e4m3_b16", "prescale_plus", 256, 10240, 256, 16, torch.float32, False),  # 4 ranks of 10 (no workspace)
+    ("e8m0_b32", "postscale_qb", 256, 9216, 256, 1, torch.float32, False),     # 4 ranks of 9, one stage in round 1
+    ("e4m3_b16", "native", 6400, 4608, 256, 16, torch.bfloat16, True),         # native FP4 weights
+])
+def test_gemv_two_rounds(fmt, strat, N, K, qk, M, out, ws):
+    native = strat == "native"
+    w = synth.make_weight(141, fmt, "prescale" if native else strat, N, K, 256, qk)
+    x = synth.make_activations(141, M, K, outliers=True)
+    a = mxc.quantize_act(dev_bf16(x), fmt)
+    pw = mxc.pack_weight(w)
+    nat = mxc.decode_weight(pw)
+    wsb = mxc.linear_workspace(M, N, K, fmt, "cuda") if ws else torch.zeros((16,), dtype=torch.uint8, device="cuda")
+    y = (mxc.native_linear(a, nat, out, ws=wsb) if native else mxc.linear(a, pw, out, ws=wsb))
+    assert mxc.get_device_error() == 0
+    ref, sabs = O.w4a4_linear(x, w)
+    if out == torch.float32:
+        assert_close(y.cpu().numpy(), ref, sabs, what=f"{fmt} {strat} N={N} K={K} M={M}")
+    else:
+        # BF16 output: one more rounding of at most half an ulp of the FP32 value
+        y32 = (mxc.native_linear(a, nat, ws=wsb) if native else mxc.linear(a, pw, ws=wsb))
+        assert torch.equal(y, y32.to(torch.bfloat16))
+        assert_close(y32.cpu().numpy(), ref, sabs, what=f"{fmt} {strat} N={N} K={K} M={M}")
+    if not native:                                   # the same MMAs on the decoded weight
+        assert torch.equal(y, mxc.native_linear(a, nat, out, ws=wsb))
+    assert torch.equal(y, (mxc.native_linear(a, nat, out, ws=wsb) if native else mxc.linear(a, pw, out, ws=wsb)))
+    assert mxc.get_device_error() == 0

@@ -3,9 +3,11 @@
 // "MXCode: Vector Quantization for MX-Native Inference at Scale", Table 3 (decode
 // TPOT): at decode batch sizes the layer streams its weights once, so the time goes
 // to bringing the compressed weights in and turning them into tensor-core operands.
-// Each CTA owns 128 output channels x a slice of at most 8 stages of 256 input
-// channels (split-K over the CTAs of a thread-block cluster) and keeps the slice on
-// chip:
+// Each CTA owns 128 output channels x a slice of 256-channel stages (split-K over
+// the CTAs of a thread-block cluster) and keeps up to 8 stages of it on chip; a
+// slice of up to 16 stages runs as two rounds of 8 through the same buffers (the
+// second round's stream is requested once the first round's MMAs have completed,
+// and goes to L2 while the first round decodes):
 //
 //   * the loader copies the slice's index bytes with one 4-D tensor copy per
 //     K-quarter (quarter c of every stage: the packed layout stores each 128 x 256
@@ -60,7 +62,7 @@
 namespace mxc {
 
 constexpr int kGemvT = 16;          // token tile = MMA N
-constexpr int kGemvMaxStages = 8;   // 256-channel stages per CTA, all resident
+constexpr int kGemvMaxStages = 8;   // 256-channel stages resident per CTA (one round)
 constexpr int kGemvMaxSplits = 4;   // cluster size
 constexpr int kGemvSfxWarps = 4;    // token-scale warps, one per TMEM lane quadrant
 constexpr int kGemvThreads = kThreads + 32 * kGemvSfxWarps;
@@ -162,6 +164,7 @@ __global__ void __maxnreg__(64)
   uint64_t* bar_sfw = bars + 17;    // weight scale atoms (bulk copy)
   uint64_t* bar_cb = bars + 18;     // codebooks of the slice (bulk copy)
   uint64_t* sfx_ready = bars + 20; // token scale atoms in TMEM (one arrival per token-scale warp)
+  uint64_t* round_free = bars + 21; // a round's MMAs are done: its buffers and scale columns may be reused
   uint64_t* red_ack = bars + 22;    // rank > 0: rank 0 has received this rank's partial tile
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
 
@@ -190,14 +193,67 @@ __global__ void __maxnreg__(64)
       p.a_sf + (static_cast<size_t>(sf_group0) * KB4 + static_cast<size_t>(ks_begin) * A) * 512;
   const int red_off = L::IDX_OFF;                               // rank 0's receive area
   const bool red_atomic = clustered && splits == 2 && !p.out_bf16;   // split-K by global reductions
-  // codebooks used by the slice: a contiguous range [qb0, qb1] of the band's row
-  const int qb0 = !L::kVQ ? 0 : H == 2 ? 2 * ks_begin : (ks_begin * kStageK) / p.qk;
-  const int qb1 = !L::kVQ ? 0 : H == 2 ? 2 * ks_end - 1 : ((ks_end - 1) * kStageK) / p.qk;
+  // Slices longer than the 8 resident stages run in rounds of 8: round r covers the
+  // stages [ks_begin + 8 r, + rcount(r)).  A round's buffers, TMEM scale columns and
+  // token tiles are reused once the MMAs of the round before have completed
+  // (round_free); the accumulator runs on across rounds, so the MMAs keep the order
+  // round by round, quarter-major within a round.
+  const int rounds = (nks + L::S - 1) / L::S;
+  const int rbox = min(p.ks_per_split, L::S);         // stages per tensor copy (the maps' box)
+  auto rcount = [&](int r) { return min(L::S, nks - L::S * r); };
+  // codebooks used by round r: a contiguous range [qb_first, qb_last] of the band's row
+  auto qb_first = [&](int r) {
+    const int b = ks_begin + L::S * r;
+    return !L::kVQ ? 0 : H == 2 ? 2 * b : (b * kStageK) / p.qk;
+  };
+  auto qb_last = [&](int r) {
+    const int e = ks_begin + L::S * r + rcount(r);   // one past the round's last stage
+    return !L::kVQ ? 0 : H == 2 ? 2 * e - 1 : ((e - 1) * kStageK) / p.qk;
+  };
+  // The weight stream of round r, requested at once and in the order it is consumed
+  // (nothing here waits for the rest of the CTA or the cluster: the copies land in
+  // this CTA's own shared memory on its own barriers).  Codebooks, index quarter 0 of
+  // every stage, the weight scales and quarter 1 go straight to shared memory;
+  // quarters 2 and 3, whose buffers free up only as quarters 0 and 1 are decoded, go
+  // to L2 now and are copied in later.  (A plain L2 prefetch of the slice in address
+  // order would complete quarter 0 -- spread over all stages -- only when nearly the
+  // whole slice had arrived, and the decode could not overlap it.)
+  auto issue_round = [&](int r) {
+    const int rb = ks_begin + L::S * r, rn = rcount(r);
+    if constexpr (L::kVQ) {
+      const int qa = qb_first(r);
+      const uint32_t cb_bytes = static_cast<uint32_t>(qb_last(r) - qa + 1) * 512;
+      mbar_arrive_expect_tx(bar_cb, cb_bytes);
+      bulk_load(smem + L::CB_OFF, w_cb + static_cast<size_t>(qa) * 256, cb_bytes, bar_cb);
+      // quarter j of the round's stages: box {2048 B, 1, rbox stages, 1}; stages past
+      // the round (and past K) arrive too, zero-filled past K, and are not used
+      mbar_arrive_expect_tx(&full[0], rbox * 2048);
+      tma_load_4d(smem + L::IDX_OFF, &tmap_idx, 0, 0, rb, n_tile, &full[0]);
+    }
+    if constexpr (!L::kSVQ && !L::kQBS) {
+      mbar_arrive_expect_tx(bar_sfw, rn * A * 512);
+      bulk_load(smem + L::SFW_OFF, w_sf + static_cast<size_t>(L::S * r) * A * 512, rn * A * 512, bar_sfw);
+    }
+    if constexpr (L::kVQ) {
+      mbar_arrive_expect_tx(&full[1], rbox * 2048);
+      tma_load_4d(smem + L::IDX_OFF + L::IDX_BUF, &tmap_idx, 0, 1, rb, n_tile, &full[1]);
+      for (int s = 0; s < rn; ++s) l2_prefetch_bulk(w_idx + static_cast<size_t>(L::S * r + s) * 8192 + 4096, 4096);
+    } else {
+      for (int s = 0; s < rn; ++s) {
+        mbar_arrive_expect_tx(&full[s], 16384);
+        tma_load_2d(smem + L::W_OFF + s * 16384, &tmap_wq, (rb + s) * 128, n_tile * 128, &full[s]);
+      }
+    }
+    if constexpr (L::kSVQ) {
+      const int u0 = rb >> sv.lspu, u1 = (rb + rn - 1) >> sv.lspu;
+      l2_prefetch_bulk(sv.unit(p.w.sidx, n_tile, rb), static_cast<uint32_t>(u1 - u0 + 1) * 128 * sv.G);
+    }
+  };
 
   // ---- setup (nothing here depends on earlier kernels) ----
   if (warp == 0) {
     // full[0..7], bar_x, dec_ph[0..3], sf_ready, accum, red_full, red_ready, bar_sfw, bar_cb,
-    // (unused), sfx_ready, (unused), red_ack
+    // (unused), sfx_ready, round_free, red_ack
     if (lane < 23) mbar_init(bars + lane, (lane >= 9 && lane < 14) ? kDecWarps : lane == 20 ? kGemvSfxWarps : 1);
     __syncwarp();
   }
@@ -208,41 +264,7 @@ __global__ void __maxnreg__(64)
     prefetch_tensormap(&tmap_x);
     if constexpr (WSRC == WSRC_NATIVE) prefetch_tensormap(&tmap_wq);
     if constexpr (L::kVQ) prefetch_tensormap(&tmap_idx);
-    // The weight stream, requested at once and in the order it is consumed (nothing
-    // here waits for the rest of the CTA or the cluster: the copies land in this CTA's
-    // own shared memory on barriers initialised above).  Codebooks, index quarter 0 of
-    // every stage, the weight scales and quarter 1 go straight to shared memory;
-    // quarters 2 and 3, whose buffers free up only as quarters 0 and 1 are decoded,
-    // go to L2 now and are copied in later.  (A plain L2 prefetch of the slice in
-    // address order would complete quarter 0 -- spread over all stages -- only when
-    // nearly the whole slice had arrived, and the decode could not overlap it.)
-    if constexpr (L::kVQ) {
-      const uint32_t cb_bytes = static_cast<uint32_t>(qb1 - qb0 + 1) * 512;
-      mbar_arrive_expect_tx(bar_cb, cb_bytes);
-      bulk_load(smem + L::CB_OFF, w_cb + static_cast<size_t>(qb0) * 256, cb_bytes, bar_cb);
-      // quarter j of stages [ks_begin, ks_begin + ks_per_split): box {2048 B, 1, stages, 1};
-      // stages past K (last split) arrive zero-filled and are not used
-      mbar_arrive_expect_tx(&full[0], p.ks_per_split * 2048);
-      tma_load_4d(smem + L::IDX_OFF, &tmap_idx, 0, 0, ks_begin, n_tile, &full[0]);
-    }
-    if constexpr (!L::kSVQ && !L::kQBS) {
-      mbar_arrive_expect_tx(bar_sfw, nks * A * 512);
-      bulk_load(smem + L::SFW_OFF, w_sf, nks * A * 512, bar_sfw);
-    }
-    if constexpr (L::kVQ) {
-      mbar_arrive_expect_tx(&full[1], p.ks_per_split * 2048);
-      tma_load_4d(smem + L::IDX_OFF + L::IDX_BUF, &tmap_idx, 0, 1, ks_begin, n_tile, &full[1]);
-      for (int s = 0; s < nks; ++s) l2_prefetch_bulk(w_idx + static_cast<size_t>(s) * 8192 + 4096, 4096);
-    } else {
-      for (int s = 0; s < nks; ++s) {
-        mbar_arrive_expect_tx(&full[s], 16384);
-        tma_load_2d(smem + L::W_OFF + s * 16384, &tmap_wq, (ks_begin + s) * 128, n_tile * 128, &full[s]);
-      }
-    }
-    if constexpr (L::kSVQ) {
-      const int u0 = ks_begin >> sv.lspu, u1 = (ks_end - 1) >> sv.lspu;
-      l2_prefetch_bulk(sv.unit(p.w.sidx, n_tile, ks_begin), static_cast<uint32_t>(u1 - u0 + 1) * 128 * sv.G);
-    }
+    issue_round(0);                                  // the first round's weight stream
   }
   if (warp == 1) {
     __syncwarp();                                    // tcgen05.alloc is warp-aligned
@@ -282,120 +304,151 @@ __global__ void __maxnreg__(64)
 
   if (warp == 0) {
     // =============================== loader ===============================
-    // (codebooks, index quarters 0 and 1, the weight scales or native weight tiles
-    // were requested during setup; the MMA warp fetches the token operands after the
-    // dependency wait)
+    // (round 0's codebooks, index quarters 0 and 1, weight scales or native weight
+    // tiles were requested during setup; the MMA warp fetches the token operands
+    // after the dependency wait)
     __syncwarp();
-    if constexpr (L::kQBS) {
-      // PostScale-QB: the weight scale atoms of the slice, each 512 bytes of its
-      // QBlock's scale (atoms in the second half of a stage use the second QBlock
-      // when the QBlock is 128 wide along K); then the MMA warp copies them to TMEM.
-      // Lane i loads atom i's byte (at most 32 atoms), so all loads are in flight at
-      // once; each atom then takes its byte from that lane.
-      const uint8_t* qb = p.w.sf + static_cast<size_t>((static_cast<int64_t>(n_tile) * 128) / p.qn) * (K / p.qk);
-      uint32_t mine = 0;
-      if (lane < nks * A) {
-        const int ks = ks_begin + lane / A, a = lane % A;
-        const int qbk = H == 2 ? 2 * ks + (a >= A / 2 ? 1 : 0) : (ks * kStageK) / p.qk;
-        mine = __ldg(qb + qbk);
+    int last_r = 0;                                  // the last round whose stream was requested
+    int issued_q = 2;                                // its index quarters requested so far
+    for (int r = 0; r < rounds; ++r) {
+      const int rb = ks_begin + L::S * r, rn = rcount(r);
+      const uint32_t ph = static_cast<uint32_t>(r & 1);
+      if (r > 0) {
+        // the round before is multiplied: its buffers take this round's stream
+        if (!__all_sync(0xffffffffu, mbar_wait(round_free, (r - 1) & 1))) break;
+        if (lane == 0) issue_round(r);
+        last_r = r;
+        issued_q = 2;
       }
-      for (int i = 0; i < nks * A; ++i) {
-        const uint32_t v = __shfl_sync(0xffffffffu, mine, i) * 0x01010101u;
-        reinterpret_cast<uint4*>(smem + L::SFW_OFF + i * 512)[lane] = make_uint4(v, v, v, v);
-      }
-      fence_proxy_async_smem();                      // generic writes -> tcgen05.cp reads
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_sfw);
-    }
-    int issued_q = 2;                                // index quarters requested so far
-    if constexpr (L::kVQ) {
-      if (elect_one()) {
-        for (int j = 2; j < 4; ++j) {                // K-quarter j of every stage (from L2 by now)
-          if (!mbar_wait(&dec_ph[j - 2], 0)) break;  // its buffer has been decoded
-          mbar_arrive_expect_tx(&full[j], p.ks_per_split * 2048);
-          tma_load_4d(smem + L::IDX_OFF + (j % 2) * L::IDX_BUF, &tmap_idx, 0, j, ks_begin, n_tile, &full[j]);
-          issued_q = j + 1;
+      if constexpr (L::kQBS) {
+        // PostScale-QB: the weight scale atoms of the round, each 512 bytes of its
+        // QBlock's scale (atoms in the second half of a stage use the second QBlock
+        // when the QBlock is 128 wide along K); then the MMA warp copies them to TMEM.
+        // Lane i loads atom i's byte (at most 32 atoms), so all loads are in flight at
+        // once; each atom then takes its byte from that lane.
+        const uint8_t* qb = p.w.sf + static_cast<size_t>((static_cast<int64_t>(n_tile) * 128) / p.qn) * (K / p.qk);
+        uint32_t mine = 0;
+        if (lane < rn * A) {
+          const int ks = rb + lane / A, a = lane % A;
+          const int qbk = H == 2 ? 2 * ks + (a >= A / 2 ? 1 : 0) : (ks * kStageK) / p.qk;
+          mine = __ldg(qb + qbk);
         }
+        for (int i = 0; i < rn * A; ++i) {
+          const uint32_t v = __shfl_sync(0xffffffffu, mine, i) * 0x01010101u;
+          reinterpret_cast<uint4*>(smem + L::SFW_OFF + i * 512)[lane] = make_uint4(v, v, v, v);
+        }
+        fence_proxy_async_smem();                    // generic writes -> tcgen05.cp reads
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_sfw);
       }
-      issued_q = static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<unsigned>(issued_q)));   // the elected lane's count
+      if constexpr (L::kVQ) {
+        if (elect_one()) {
+          for (int j = 2; j < 4; ++j) {              // K-quarter j of every stage (from L2 by now)
+            if (!mbar_wait(&dec_ph[j - 2], ph)) break;   // its buffer has been decoded
+            mbar_arrive_expect_tx(&full[j], rbox * 2048);
+            tma_load_4d(smem + L::IDX_OFF + (j % 2) * L::IDX_BUF, &tmap_idx, 0, j, rb, n_tile, &full[j]);
+            issued_q = j + 1;
+          }
+          if (issued_q == 4 && r + 1 < rounds) {     // the next round's stream into L2 meanwhile
+            const int nb = L::S * (r + 1), nn = rcount(r + 1);
+            l2_prefetch_bulk(w_idx + static_cast<size_t>(nb) * 8192, static_cast<uint32_t>(nn) * 8192);
+            if constexpr (!L::kSVQ && !L::kQBS)
+              l2_prefetch_bulk(w_sf + static_cast<size_t>(nb) * A * 512, static_cast<uint32_t>(nn) * A * 512);
+          }
+        }
+        issued_q = static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<unsigned>(issued_q)));   // the elected lane's count
+      }
+      __syncwarp();
     }
-    __syncwarp();
     // Every copy this CTA requested lands before the CTA can retire, even when a
     // consumer gave up waiting (timeout path): codebooks, index quarters, weight
-    // scales or native tiles.  On the normal path these have all completed already.
+    // scales or native tiles.  The copies of earlier rounds completed before their
+    // round's MMAs did; on the normal path the last round's have completed too.
     if (lane == 0) {
+      const uint32_t ph = static_cast<uint32_t>(last_r & 1);
       if constexpr (L::kVQ) {
-        mbar_wait(bar_cb, 0);
-        for (int j = 0; j < issued_q; ++j) mbar_wait(&full[j], 0);
+        mbar_wait(bar_cb, ph);
+        for (int j = 0; j < issued_q; ++j) mbar_wait(&full[j], ph);
       } else {
-        for (int s = 0; s < nks; ++s) mbar_wait(&full[s], 0);
+        for (int s = 0; s < rcount(last_r); ++s) mbar_wait(&full[s], ph);
       }
-      if constexpr (!L::kSVQ && !L::kQBS) mbar_wait(bar_sfw, 0);
+      if constexpr (!L::kSVQ && !L::kQBS) mbar_wait(bar_sfw, ph);
     }
     __syncwarp();
     if (clustered && rank == 0 && !red_atomic) {
       // Let the other ranks send their partials once the receive area (the index
       // buffers) is free: after the last decode phase.  Sent even after a failed
       // wait, so that no rank waits for the signal in vain.
-      if constexpr (L::kVQ) mbar_wait(&dec_ph[3], 0);
+      if constexpr (L::kVQ) mbar_wait(&dec_ph[3], static_cast<uint32_t>((rounds - 1) & 1));
       if (lane > 0 && lane < splits) mbar_remote_arrive(mapa_shared(smem_u32(red_ready), lane));
     }
   } else if (warp == 1) {
     // ============================ MMA issuer ==============================
     const uint32_t w_s0 = smem_u32(smem + L::W_OFF), x_s0 = smem_u32(smem + L::X_OFF);
     bool ok = true;
-    if constexpr (!L::kSVQ) {
-      // weight scale atoms -> TMEM; copies and MMAs issue in order from this thread
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_sfw, 0));
-      if (ok && elect_one()) {
-        const uint32_t sfw_s0 = smem_u32(smem + L::SFW_OFF);
-        for (int i = 0; i < nks * A; ++i)
-          tc_cp_32x128b_warpx4(tmem + L::COL_SFW + 4 * i, sdesc_sf_atom(sfw_s0 + i * 512));
-      }
-      __syncwarp();
-    }
-    griddep_wait();                                  // the token operands are written
-    __syncwarp();
-    if (elect_one()) {
-      // token tiles of all stages: box {128 B, 16 rows, ks_per_split stages}; stages
-      // past K (last split) arrive zero-filled and are not used
-      mbar_arrive_expect_tx(bar_x, p.ks_per_split * kGemvT * 128);
-      tma_load_3d(smem + L::X_OFF, &tmap_x, 0, static_cast<int>(m0), ks_begin, bar_x);
-    }
-    __syncwarp();
-    ok = __all_sync(0xffffffffu, mbar_wait(sfx_ready, 0)) && ok;
-    ok = __all_sync(0xffffffffu, mbar_wait(bar_x, 0)) && ok;
-    if constexpr (L::kSVQ) ok = __all_sync(0xffffffffu, mbar_wait(sf_ready, 0)) && ok;
-    if constexpr (!L::kVQ) {
-      for (int s = 0; s < nks && ok; ++s) ok = __all_sync(0xffffffffu, mbar_wait(&full[s], 0));
-    }
-    tc_fence_after();
-    for (int j = 0; j < 4 && ok; ++j) {
-      if constexpr (L::kVQ) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&dec_ph[j], 0))) {
-          ok = false;
-          break;
-        }
+    for (int r = 0; r < rounds && ok; ++r) {
+      const int rb = ks_begin + L::S * r, rn = rcount(r);
+      const uint32_t ph = static_cast<uint32_t>(r & 1);
+      if (r > 0) {                                   // the round before has been multiplied
+        ok = __all_sync(0xffffffffu, mbar_wait(round_free, (r - 1) & 1));
+        if (!ok) break;
         tc_fence_after();
       }
+      if constexpr (!L::kSVQ) {
+        // weight scale atoms -> TMEM; copies and MMAs issue in order from this thread
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_sfw, ph));
+        if (ok && elect_one()) {
+          const uint32_t sfw_s0 = smem_u32(smem + L::SFW_OFF);
+          for (int i = 0; i < rn * A; ++i)
+            tc_cp_32x128b_warpx4(tmem + L::COL_SFW + 4 * i, sdesc_sf_atom(sfw_s0 + i * 512));
+        }
+        __syncwarp();
+      }
+      if (r == 0) griddep_wait();                    // the token operands are written
+      __syncwarp();
       if (elect_one()) {
-        for (int s = 0; s < nks; ++s) {
-          const uint64_t adesc = sdesc_kmajor_sw128(w_s0 + s * 16384 + 32 * j);
-          const uint64_t bdesc = sdesc_kmajor_sw128(x_s0 + s * kGemvT * 128 + 32 * j);
-          const uint32_t acc = (s > 0 || j > 0) ? 1u : 0u;
-          const uint32_t sfw_t = tmem + L::COL_SFW + 4 * s * A, sfx_t = tmem + L::COL_SFX + 4 * s * A;
-          if constexpr (FMT == FMT_E4M3) {
-            constexpr uint32_t idesc = idesc_mxf4(kGemvT, 0, 0, 0);
-            tc_mma_mxf4nvf4_block16(tmem, adesc, bdesc, idesc, sfw_t + 4 * j, sfx_t + 4 * j, acc);
-          } else {
-            const int a = j >> 1;
-            const uint32_t id = static_cast<uint32_t>(j & 1) * 2;
-            const uint32_t idesc = idesc_mxf4(kGemvT, 1, static_cast<int>(id), static_cast<int>(id));
-            tc_mma_mxf4_block32(tmem, adesc, bdesc, idesc, (sfw_t + 4 * a) | (id << 30), (sfx_t + 4 * a) | (id << 30),
-                                acc);
+        // token tiles of the round's stages: box {128 B, 16 rows, rbox stages}; stages
+        // past the round (and past K) arrive too, zero-filled past K, and are not used
+        mbar_arrive_expect_tx(bar_x, rbox * kGemvT * 128);
+        tma_load_3d(smem + L::X_OFF, &tmap_x, 0, static_cast<int>(m0), rb, bar_x);
+      }
+      __syncwarp();
+      ok = __all_sync(0xffffffffu, mbar_wait(sfx_ready, ph)) && ok;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_x, ph)) && ok;
+      if constexpr (L::kSVQ) ok = __all_sync(0xffffffffu, mbar_wait(sf_ready, ph)) && ok;
+      if constexpr (!L::kVQ) {
+        for (int s = 0; s < rn && ok; ++s) ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph));
+      }
+      tc_fence_after();
+      for (int j = 0; j < 4 && ok; ++j) {
+        if constexpr (L::kVQ) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&dec_ph[j], ph))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        if (elect_one()) {
+          for (int s = 0; s < rn; ++s) {
+            const uint64_t adesc = sdesc_kmajor_sw128(w_s0 + s * 16384 + 32 * j);
+            const uint64_t bdesc = sdesc_kmajor_sw128(x_s0 + s * kGemvT * 128 + 32 * j);
+            const uint32_t acc = (r > 0 || s > 0 || j > 0) ? 1u : 0u;
+            const uint32_t sfw_t = tmem + L::COL_SFW + 4 * s * A, sfx_t = tmem + L::COL_SFX + 4 * s * A;
+            if constexpr (FMT == FMT_E4M3) {
+              constexpr uint32_t idesc = idesc_mxf4(kGemvT, 0, 0, 0);
+              tc_mma_mxf4nvf4_block16(tmem, adesc, bdesc, idesc, sfw_t + 4 * j, sfx_t + 4 * j, acc);
+            } else {
+              const int a = j >> 1;
+              const uint32_t id = static_cast<uint32_t>(j & 1) * 2;
+              const uint32_t idesc = idesc_mxf4(kGemvT, 1, static_cast<int>(id), static_cast<int>(id));
+              tc_mma_mxf4_block32(tmem, adesc, bdesc, idesc, (sfw_t + 4 * a) | (id << 30),
+                                  (sfx_t + 4 * a) | (id << 30), acc);
+            }
           }
         }
+        __syncwarp();
       }
+      if (ok && r + 1 < rounds && elect_one()) tc_commit(round_free);   // the round's buffers may be refilled
       __syncwarp();
     }
     if (elect_one()) tc_commit(accum);
@@ -411,30 +464,38 @@ __global__ void __maxnreg__(64)
     // loads in flight at once); the upper half reaches lanes 0..15 by a shuffle.
     const uint32_t taddr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + L::COL_SFX;
     const int r16 = lane & 15, half = lane >> 4;
-    uint32_t v[16];
-#pragma unroll
-    for (int a = 0; a < 16; ++a) {
-      const int atom = 16 * half + a;
-      v[a] = atom < nks * A
-                 ? __ldg(reinterpret_cast<const uint32_t*>(a_sf + static_cast<size_t>(atom) * 512 + r16 * 16))
-                 : 0u;
-    }
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {                    // 8 atoms = 32 columns per store
-      if (8 * c >= nks * A) break;                   // uniform over the warp
-      uint32_t w[8];
-#pragma unroll
-      for (int a = 0; a < 8; ++a) {
-        const uint32_t x = c < 2 ? v[8 * c + a] : __shfl_down_sync(0xffffffffu, v[8 * (c - 2) + a], 16);
-        w[a] = half == 0 ? x : 0u;                   // lanes 16..31: padding rows
+    for (int r = 0; r < rounds; ++r) {
+      const int na = rcount(r) * A;                  // the round's atoms
+      const uint8_t* const a_sf_r = a_sf + static_cast<size_t>(L::S * r) * A * 512;
+      if (r > 0) {                                   // the round before has been multiplied
+        if (!__all_sync(0xffffffffu, mbar_wait(round_free, (r - 1) & 1))) break;
+        tc_fence_after();
       }
-      __syncwarp();                                  // tcgen05.st is warp-aligned
-      tmem_st_sfx8(taddr + 32 * c, w);
+      uint32_t v[16];
+#pragma unroll
+      for (int a = 0; a < 16; ++a) {
+        const int atom = 16 * half + a;
+        v[a] = atom < na
+                   ? __ldg(reinterpret_cast<const uint32_t*>(a_sf_r + static_cast<size_t>(atom) * 512 + r16 * 16))
+                   : 0u;
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {                  // 8 atoms = 32 columns per store
+        if (8 * c >= na) break;                      // uniform over the warp
+        uint32_t w[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+          const uint32_t x = c < 2 ? v[8 * c + a] : __shfl_down_sync(0xffffffffu, v[8 * (c - 2) + a], 16);
+          w[a] = half == 0 ? x : 0u;                 // lanes 16..31: padding rows
+        }
+        __syncwarp();                                // tcgen05.st is warp-aligned
+        tmem_st_sfx8(taddr + 32 * c, w);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sfx_ready);
     }
-    tmem_st_wait();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(sfx_ready);
     if (red_atomic) {
       if (rank == 0) {                               // zero this tile of Y, rows < M
         const int st = threadIdx.x - (2 + kDecWarps) * 32;
@@ -452,7 +513,6 @@ __global__ void __maxnreg__(64)
     // --- the stage codebook words this lane lays out (loads issued first) ---
     const int s_l = lane & 7;                        // this lane's stage
     const int q = dw * 4 + (lane >> 3);              // 64 threads per stage
-    const bool active = L::kVQ && s_l < nks;
     // Entries [16 kb, 16 kb + 16) of the codebook of this lane's stage (first or,
     // QBlock 128 wide along K, second half of the stage), kb = (dw + s_l/2) mod 16:
     // over the 16 warps each lane still covers all 256 entries, and the 8 lanes of a
@@ -460,10 +520,10 @@ __global__ void __maxnreg__(64)
     // the two 16-byte halves are read in an order that alternates with the stage.
     const int kb = (dw + (s_l >> 1)) & 15;
     const int h0 = s_l & 1;
-    auto cb_words = [&](int epoch, uint4* c0, uint4* c1) {
-      const int ks = ks_begin + s_l;
+    auto cb_words = [&](int r, int epoch, uint4* c0, uint4* c1) {
+      const int ks = ks_begin + L::S * r + s_l;
       const int qbk = H == 2 ? 2 * ks + epoch : (ks * kStageK) / p.qk;
-      const uint8_t* cp = smem + L::CB_OFF + (qbk - qb0) * 512 + 32 * kb;
+      const uint8_t* cp = smem + L::CB_OFF + (qbk - qb_first(r)) * 512 + 32 * kb;
       const uint4 first = *reinterpret_cast<const uint4*>(cp + 16 * h0);
       const uint4 second = *reinterpret_cast<const uint4*>(cp + 16 * (1 - h0));
       *c0 = h0 ? second : first;                      // entries 16 kb .. 16 kb + 7
@@ -472,7 +532,7 @@ __global__ void __maxnreg__(64)
 
     // --- PreScale+ weight scale atoms -> TMEM lanes of this warp's quadrant
     //     (atoms i = cg mod 4), after decode phase 0 ---
-    auto svq_scales_to_tmem = [&]() {
+    auto svq_scales_to_tmem = [&](int r) {
       if constexpr (L::kSVQ) {
         __syncwarp();                                // tcgen05.st is warp-aligned
         // PreScale+ (Table 4 caption: Ks = 256, ds = 8; larger ds compress further):
@@ -480,9 +540,9 @@ __global__ void __maxnreg__(64)
         // scales 4a..4a+3 of stage s: one word of the scale-codebook entry.
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(qd * 32) << 16);
         const uint32_t* scb32 = reinterpret_cast<const uint32_t*>(p.w.scb);
-        for (int i = cg; i < nks * A; i += 4) {
+        for (int i = cg; i < rcount(r) * A; i += 4) {
           const int s = i / A, a = i % A;
-          const int ks = ks_begin + s;
+          const int ks = ks_begin + L::S * r + s;
           const uint8_t* un = sv.unit(p.w.sidx, n_tile, ks);
           const int kb = sv.kb_base(ks, L::kB) + 4 * a;
           uint4 v;
@@ -500,55 +560,61 @@ __global__ void __maxnreg__(64)
     };
 
     if constexpr (L::kVQ) {
-      // both codebooks into registers now: the staging area is overwritten by the
-      // decoded tiles of the last stage
-      uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0, d0 = c0, d1 = c0;
-      const bool cb_ok = mbar_wait(bar_cb, 0);
-      if (active && cb_ok) {
-        cb_words(0, &c0, &c1);
-        if (H == 2) cb_words(1, &d0, &d1);
-      }
-      // --- codebook copies: lane l's copy (bank l) = codebook of stage l mod 8,
-      //     entry e in the low half of word e*32 + l ---
       uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L::LUT_OFF) + (16 * kb) * 32 + lane;
-      auto lay_out = [&](const uint4& a, const uint4& b) {
-        if (!active) return;
-        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          lut[(2 * i) * 32] = w[i] & 0xFFFFu;
-          lut[(2 * i + 1) * 32] = w[i] >> 16;
-        }
-      };
-      lay_out(c0, c1);
-      named_bar_sync(2, kDecThreads);                // all copies written
       const uint32_t lut_lane = smem_u32(smem + L::LUT_OFF) + lane * 4;
       const uint8_t* idx_l = smem + L::IDX_OFF + s_l * 2048;
       uint8_t* wt = smem + L::W_OFF + s_l * 16384;
-      for (int j = 0; j < 4; ++j) {
-        if (H == 2 && j == 2) {                      // second half of each stage: its own codebook
-          named_bar_sync(2, kDecThreads);            // everyone is done with the first codebooks
-          lay_out(d0, d1);
-          named_bar_sync(2, kDecThreads);
+      for (int r = 0; r < rounds; ++r) {
+        const uint32_t ph = static_cast<uint32_t>(r & 1);
+        const bool active = s_l < rcount(r);
+        // both codebooks into registers now: the staging area is overwritten by the
+        // decoded tiles of the last stage.  (Every decoder is done with the copies of
+        // the round before: its MMAs, which waited for all decode phases, completed
+        // before this round's codebooks were requested.)
+        uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0, d0 = c0, d1 = c0;
+        const bool cb_ok = mbar_wait(bar_cb, ph);
+        if (active && cb_ok) {
+          cb_words(r, 0, &c0, &c1);
+          if (H == 2) cb_words(r, 1, &d0, &d1);
         }
-        const bool landed = mbar_wait(&full[j], 0);
-        if (active && landed) {
+        // --- codebook copies: lane l's copy (bank l) = codebook of stage l mod 8,
+        //     entry e in the low half of word e*32 + l ---
+        auto lay_out = [&](const uint4& a, const uint4& b) {
+          if (!active) return;
+          const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int r = (q + 64 * i + s_l) & 127;  // offset by the stage: conflict-free stores
-            const uint4 iv = *reinterpret_cast<const uint4*>(idx_l + (j % 2) * L::IDX_BUF + r * 16);
-            const uint4 o0 = make_uint4(lut32_pair(lut_lane, iv.x, 0), lut32_pair(lut_lane, iv.x, 2),
-                                        lut32_pair(lut_lane, iv.y, 0), lut32_pair(lut_lane, iv.y, 2));
-            const uint4 o1 = make_uint4(lut32_pair(lut_lane, iv.z, 0), lut32_pair(lut_lane, iv.z, 2),
-                                        lut32_pair(lut_lane, iv.w, 0), lut32_pair(lut_lane, iv.w, 2));
-            *reinterpret_cast<uint4*>(wt + r * 128 + (((2 * j) ^ (r & 7)) << 4)) = o0;
-            *reinterpret_cast<uint4*>(wt + r * 128 + (((2 * j + 1) ^ (r & 7)) << 4)) = o1;
+          for (int i = 0; i < 8; ++i) {
+            lut[(2 * i) * 32] = w[i] & 0xFFFFu;
+            lut[(2 * i + 1) * 32] = w[i] >> 16;
           }
+        };
+        lay_out(c0, c1);
+        named_bar_sync(2, kDecThreads);              // all copies written
+        for (int j = 0; j < 4; ++j) {
+          if (H == 2 && j == 2) {                    // second half of each stage: its own codebook
+            named_bar_sync(2, kDecThreads);          // everyone is done with the first codebooks
+            lay_out(d0, d1);
+            named_bar_sync(2, kDecThreads);
+          }
+          const bool landed = mbar_wait(&full[j], ph);
+          if (active && landed) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int rw = (q + 64 * i + s_l) & 127;   // offset by the stage: conflict-free stores
+              const uint4 iv = *reinterpret_cast<const uint4*>(idx_l + (j % 2) * L::IDX_BUF + rw * 16);
+              const uint4 o0 = make_uint4(lut32_pair(lut_lane, iv.x, 0), lut32_pair(lut_lane, iv.x, 2),
+                                          lut32_pair(lut_lane, iv.y, 0), lut32_pair(lut_lane, iv.y, 2));
+              const uint4 o1 = make_uint4(lut32_pair(lut_lane, iv.z, 0), lut32_pair(lut_lane, iv.z, 2),
+                                          lut32_pair(lut_lane, iv.w, 0), lut32_pair(lut_lane, iv.w, 2));
+              *reinterpret_cast<uint4*>(wt + rw * 128 + (((2 * j) ^ (rw & 7)) << 4)) = o0;
+              *reinterpret_cast<uint4*>(wt + rw * 128 + (((2 * j + 1) ^ (rw & 7)) << 4)) = o1;
+            }
+          }
+          fence_proxy_async_smem();                  // tile writes -> tensor-core operand reads
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&dec_ph[j]);
+          if (j == 0) svq_scales_to_tmem(r);         // needed with quarter 0's MMAs
         }
-        fence_proxy_async_smem();                    // tile writes -> tensor-core operand reads
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&dec_ph[j]);
-        if (j == 0) svq_scales_to_tmem();            // needed with quarter 0's MMAs
       }
     }
     // ------------------------------ epilogue ------------------------------

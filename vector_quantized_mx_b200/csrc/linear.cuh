@@ -533,10 +533,12 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
     }
     p.splits = splits;
     p.ks_per_split = per;
-    if (per <= kGemvMaxStages && (splits <= kGemvMaxSplits || red_part)) {
+    // slices of up to two rounds of 8 resident stages
+    if (per <= 2 * kGemvMaxStages && (splits <= kGemvMaxSplits || red_part)) {
+      const int box = per < kGemvMaxStages ? per : kGemvMaxStages;   // stages per tensor copy: one round
       CUtensorMap tx3, ti = tw;
-      if (!make_fp4_stage_map(&tx3, a.a_q, a.M, a.K, a.ldq, kGemvT, per)) return MXC_ERR_CUDA;
-      if (a.wsrc != WSRC_NATIVE && !make_idx_map(&ti, a.w_idx, a.N, a.K, per)) return MXC_ERR_CUDA;
+      if (!make_fp4_stage_map(&tx3, a.a_q, a.M, a.K, a.ldq, kGemvT, box)) return MXC_ERR_CUDA;
+      if (a.wsrc != WSRC_NATIVE && !make_idx_map(&ti, a.w_idx, a.N, a.K, box)) return MXC_ERR_CUDA;
       GemvParams g{};
       g.M = p.M;
       g.N = p.N;
