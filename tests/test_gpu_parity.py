@@ -602,7 +602,7 @@ def test_gemv_splitk_through_workspace(fmt, strat, N, K, M):
 
 
 # ---------------------------------------------------------------------------
-# Decode GEMV slices of 9 to 16 stages: two rounds of 8 resident stages per CTA
+# Decode GEMV slices of 9 to 32 stages: rounds of 8 resident stages per CTA
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("fmt,strat,N,K,qk,M,out,ws", [
@@ -611,8 +611,10 @@ def test_gemv_splitk_through_workspace(fmt, strat, N, K, M):
     ("e4m3_b16", "prescale_plus", 256, 10240, 256, 16, torch.float32, False),  # 4 ranks of 10 (no workspace)
     ("e8m0_b32", "postscale_qb", 256, 9216, 256, 1, torch.float32, False),     # 4 ranks of 9, one stage in round 1
     ("e4m3_b16", "native", 6400, 4608, 256, 16, torch.bfloat16, True),         # native FP4 weights
+    ("e4m3_b16", "postscale", 6400, 12288, 256, 16, torch.float32, True),      # 2 ranks of 24: three rounds
+    ("e8m0_b32", "prescale_plus", 256, 32768, 256, 3, torch.bfloat16, False),  # 4 ranks of 32: four rounds
 ])
-def test_gemv_two_rounds(fmt, strat, N, K, qk, M, out, ws):
+def test_gemv_rounds(fmt, strat, N, K, qk, M, out, ws):
     native = strat == "native"
     w = synth.make_weight(141, fmt, "prescale" if native else strat, N, K, 256, qk)
     x = synth.make_activations(141, M, K, outliers=True)

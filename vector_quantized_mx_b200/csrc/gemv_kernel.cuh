@@ -5,9 +5,9 @@
 // to bringing the compressed weights in and turning them into tensor-core operands.
 // Each CTA owns 128 output channels x a slice of 256-channel stages (split-K over
 // the CTAs of a thread-block cluster) and keeps up to 8 stages of it on chip; a
-// slice of up to 16 stages runs as two rounds of 8 through the same buffers (the
-// second round's stream is requested once the first round's MMAs have completed,
-// and goes to L2 while the first round decodes):
+// longer slice (up to 32 stages) runs as rounds of 8 through the same buffers (a
+// round's stream is requested once the round before has been multiplied, and goes
+// to L2 while that round decodes):
 //
 //   * the loader copies the slice's index bytes with one 4-D tensor copy per
 //     K-quarter (quarter c of every stage: the packed layout stores each 128 x 256
@@ -63,6 +63,7 @@ namespace mxc {
 
 constexpr int kGemvT = 16;          // token tile = MMA N
 constexpr int kGemvMaxStages = 8;   // 256-channel stages resident per CTA (one round)
+constexpr int kGemvMaxRounds = 4;   // rounds per slice: slices of up to 32 stages
 constexpr int kGemvMaxSplits = 4;   // cluster size
 constexpr int kGemvSfxWarps = 4;    // token-scale warps, one per TMEM lane quadrant
 constexpr int kGemvThreads = kThreads + 32 * kGemvSfxWarps;

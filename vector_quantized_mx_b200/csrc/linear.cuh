@@ -533,8 +533,8 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
     }
     p.splits = splits;
     p.ks_per_split = per;
-    // slices of up to two rounds of 8 resident stages
-    if (per <= 2 * kGemvMaxStages && (splits <= kGemvMaxSplits || red_part)) {
+    // slices of up to kGemvMaxRounds rounds of 8 resident stages
+    if (per <= kGemvMaxRounds * kGemvMaxStages && (splits <= kGemvMaxSplits || red_part)) {
       const int box = per < kGemvMaxStages ? per : kGemvMaxStages;   // stages per tensor copy: one round
       CUtensorMap tx3, ti = tw;
       if (!make_fp4_stage_map(&tx3, a.a_q, a.M, a.K, a.ldq, kGemvT, box)) return MXC_ERR_CUDA;
