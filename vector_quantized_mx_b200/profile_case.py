@@ -27,12 +27,21 @@ def _dev_bf16(bits, dev):
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["decode", "decode_native", "prefill", "prefill_native", "moe", "swiglu", "quant"])
+    ap.add_argument("case", choices=["decode", "decode_native", "decode_long", "prefill", "prefill_native", "moe",
+                                     "swiglu", "quant"])
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args(argv)
     build.build()
     dev = torch.device("cuda", 0)
-    if args.case.startswith("decode"):
+    if args.case == "decode_long":
+        # K = N = 8192 at M = 16 (PostScale E4M3-B16, 256 x 256 QBlocks): two rounds a CTA
+        w = synth.config5_weight(256, "postscale", "e4m3_b16")
+        x = synth.config5_activations(16)
+        pw = mxc.pack_weight(w, dev)
+        a = mxc.quantize_act(_dev_bf16(x, dev), w.fmt)
+        for _ in range(args.reps):
+            mxc.linear(a, pw)
+    elif args.case.startswith("decode"):
         w, x = synth.config2(16)
         pw = mxc.pack_weight(w, dev)
         a = mxc.quantize_act(_dev_bf16(x, dev), w.fmt)
