@@ -141,6 +141,26 @@ __device__ __forceinline__ uint32_t lut32_pair(uint32_t lut_lane, uint32_t x, in
   return __byte_perm(wa, wb, 0x5410u);
 }
 
+// A decoder thread's share of K-quarter j of its lane's stage s_l: two of the stage's
+// 128 rows (q and q + 64, offset by the stage so that the 8 stages' stores meet
+// different banks), 16 index bytes each from the quarter's slab idx_q, decoded through
+// the lane's codebook copy into 32 bytes of row r of the stage tile wt (128-byte
+// swizzle: 16-byte chunk c of row r at chunk c ^ (r mod 8)).
+__device__ __forceinline__ void decode_quarter_rows(uint32_t lut_lane, const uint8_t* idx_q, uint8_t* wt, int q,
+                                                    int s_l, int j) {
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int rw = (q + 64 * i + s_l) & 127;
+    const uint4 iv = *reinterpret_cast<const uint4*>(idx_q + rw * 16);
+    const uint4 o0 = make_uint4(lut32_pair(lut_lane, iv.x, 0), lut32_pair(lut_lane, iv.x, 2),
+                                lut32_pair(lut_lane, iv.y, 0), lut32_pair(lut_lane, iv.y, 2));
+    const uint4 o1 = make_uint4(lut32_pair(lut_lane, iv.z, 0), lut32_pair(lut_lane, iv.z, 2),
+                                lut32_pair(lut_lane, iv.w, 0), lut32_pair(lut_lane, iv.w, 2));
+    *reinterpret_cast<uint4*>(wt + rw * 128 + (((2 * j) ^ (rw & 7)) << 4)) = o0;
+    *reinterpret_cast<uint4*>(wt + rw * 128 + (((2 * j + 1) ^ (rw & 7)) << 4)) = o1;
+  }
+}
+
 // At most 64 registers a thread (704 x 64 = 45,056 of the SM's 65,536), so that the
 // kernel launched next to it (the activation quantizer of the next layer, a
 // 16-CTA cluster of 256-thread CTAs) still finds room on the same SMs.
@@ -598,19 +618,7 @@ __global__ void __maxnreg__(64)
             named_bar_sync(2, kDecThreads);
           }
           const bool landed = mbar_wait(&full[j], ph);
-          if (active && landed) {
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-              const int rw = (q + 64 * i + s_l) & 127;   // offset by the stage: conflict-free stores
-              const uint4 iv = *reinterpret_cast<const uint4*>(idx_l + (j % 2) * L::IDX_BUF + rw * 16);
-              const uint4 o0 = make_uint4(lut32_pair(lut_lane, iv.x, 0), lut32_pair(lut_lane, iv.x, 2),
-                                          lut32_pair(lut_lane, iv.y, 0), lut32_pair(lut_lane, iv.y, 2));
-              const uint4 o1 = make_uint4(lut32_pair(lut_lane, iv.z, 0), lut32_pair(lut_lane, iv.z, 2),
-                                          lut32_pair(lut_lane, iv.w, 0), lut32_pair(lut_lane, iv.w, 2));
-              *reinterpret_cast<uint4*>(wt + rw * 128 + (((2 * j) ^ (rw & 7)) << 4)) = o0;
-              *reinterpret_cast<uint4*>(wt + rw * 128 + (((2 * j + 1) ^ (rw & 7)) << 4)) = o1;
-            }
-          }
+          if (active && landed) decode_quarter_rows(lut_lane, idx_l + (j % 2) * L::IDX_BUF, wt, q, s_l, j);
           fence_proxy_async_smem();                  // tile writes -> tensor-core operand reads
           __syncwarp();
           if (lane == 0) mbar_arrive(&dec_ph[j]);

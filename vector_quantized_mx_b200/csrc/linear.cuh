@@ -5,6 +5,7 @@
 #include <atomic>
 #include <cstring>
 
+#include "decode_pass.cuh"
 #include "pair_kernel.cuh"
 #include "round_kernel.cuh"
 
@@ -658,13 +659,20 @@ mxc_status run_moe_linear(const MoeArgs& m, cudaStream_t stream) {
   return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
 }
 
+// Decode pass: one CTA per 128 rows x 8 stages; q_out is written by tensor stores
+// (16-byte aligned base, ldq a multiple of 16: checked by the callers).
 template <int FMT, int WSRC>
-cudaError_t launch_decode_dump(const DecodeArgs& a, cudaStream_t stream) {
-  constexpr int smem = DumpLayout<FMT, WSRC>::SMEM;
-  auto kern = decode_dump_kernel<FMT, WSRC>;
+cudaError_t launch_decode_pass(const DecodeArgs& a, cudaStream_t stream) {
+  using L = PassLayout<FMT, WSRC>;
+  auto kern = decode_pass_kernel<FMT, WSRC>;
   static uint64_t attr_set = 0;
-  cudaError_t err = ensure_smem_attr(kern, smem, &attr_set);
+  cudaError_t err = ensure_smem_attr(kern, L::SMEM, &attr_set);
   if (err != cudaSuccess) return err;
+  const int KS = static_cast<int>(a.K / kStageK);
+  const int box = KS < kGemvMaxStages ? KS : kGemvMaxStages;   // stages per tensor copy
+  CUtensorMap ti, tq;
+  if (!make_idx_map(&ti, a.w_idx, a.N, a.K, box) || !make_fp4_stage_map(&tq, a.q_out, a.N, a.K, a.ldq, 128, box))
+    return cudaErrorInvalidValue;
   ExpertPtrs w{};
   w.idx = a.w_idx;
   w.cb = a.w_cb;
@@ -672,9 +680,9 @@ cudaError_t launch_decode_dump(const DecodeArgs& a, cudaStream_t stream) {
   w.sidx = a.w_sidx;
   w.scb = a.w_scb;
   w.ds = a.ds;
-  const dim3 grid(static_cast<unsigned>(a.N / kTileN), static_cast<unsigned>(a.K / kStageK));
-  kern<<<grid, 160, smem, stream>>>(w, static_cast<int>(a.N), static_cast<int>(a.K), static_cast<int>(a.qn),
-                                    static_cast<int>(a.qk), a.q_out, a.ldq, a.sf_out);
+  const dim3 grid(static_cast<unsigned>(a.N / kTileN), static_cast<unsigned>((KS + kGemvMaxStages - 1) / kGemvMaxStages));
+  kern<<<grid, kPassThreads, L::SMEM, stream>>>(ti, tq, w, static_cast<int>(a.N), static_cast<int>(a.K),
+                                                static_cast<int>(a.qn), static_cast<int>(a.qk), box, a.sf_out);
   return cudaGetLastError();
 }
 
@@ -709,13 +717,13 @@ mxc_status run_decode_weight(const DecodeArgs& a, cudaStream_t stream) {
     return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
   }
   if (a.fmt == FMT_E8M0) {
-    err = a.wsrc == WSRC_VQ_SVQ   ? launch_decode_dump<FMT_E8M0, WSRC_VQ_SVQ>(a, stream)
-          : a.wsrc == WSRC_VQ_QBS ? launch_decode_dump<FMT_E8M0, WSRC_VQ_QBS>(a, stream)
-                                  : launch_decode_dump<FMT_E8M0, WSRC_VQ_DIRECT>(a, stream);
+    err = a.wsrc == WSRC_VQ_SVQ   ? launch_decode_pass<FMT_E8M0, WSRC_VQ_SVQ>(a, stream)
+          : a.wsrc == WSRC_VQ_QBS ? launch_decode_pass<FMT_E8M0, WSRC_VQ_QBS>(a, stream)
+                                  : launch_decode_pass<FMT_E8M0, WSRC_VQ_DIRECT>(a, stream);
   } else {
-    err = a.wsrc == WSRC_VQ_SVQ   ? launch_decode_dump<FMT_E4M3, WSRC_VQ_SVQ>(a, stream)
-          : a.wsrc == WSRC_VQ_QBS ? launch_decode_dump<FMT_E4M3, WSRC_VQ_QBS>(a, stream)
-                                  : launch_decode_dump<FMT_E4M3, WSRC_VQ_DIRECT>(a, stream);
+    err = a.wsrc == WSRC_VQ_SVQ   ? launch_decode_pass<FMT_E4M3, WSRC_VQ_SVQ>(a, stream)
+          : a.wsrc == WSRC_VQ_QBS ? launch_decode_pass<FMT_E4M3, WSRC_VQ_QBS>(a, stream)
+                                  : launch_decode_pass<FMT_E4M3, WSRC_VQ_DIRECT>(a, stream);
   }
   return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
 }

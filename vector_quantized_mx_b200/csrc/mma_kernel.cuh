@@ -636,96 +636,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------------------------
-// Decode dump: the decoders of gemm_kernel, with the stage written back to global
-// memory in plain layouts (FP4 matrix, SF layout).  Grid (N/128, K/256), 160 threads.
-// ------------------------------------------------------------------------------------
-template <int FMT, int WSRC>
-struct DumpLayout {
-  using L = StageLayout<FMT, WSRC, 16>;
-  static constexpr int LUT_OFF = L::CTRL + L::BYTES;
-  static constexpr int SMEM = 1024 + LUT_OFF + 2 * kLutBytes;
-};
-
-template <int FMT, int WSRC>
-__global__ void __launch_bounds__(160)
-    decode_dump_kernel(const ExpertPtrs w, int N, int K, int qn, int qk, uint8_t* __restrict__ q_out,
-                       int64_t ldq, uint8_t* __restrict__ sf_out) {
-  using L = StageLayout<FMT, WSRC, 16>;
-  constexpr int A = L::kAtoms;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
-  uint8_t* scb_smem = smem + 2048;
-  uint8_t* st = smem + L::CTRL;
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + DumpLayout<FMT, WSRC>::LUT_OFF);
-  const int n_tile = blockIdx.x, ks = blockIdx.y;
-  const int KS = K / kStageK, KB4 = K / L::kB / 4;
-  const int cb_split = qk == 128;
-  if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
-    fence_mbar_init();
-  }
-  const SvqGeom sv(w.ds, L::kB, KS);
-  const uint32_t* const scb32 = sv.ds == 8 ? reinterpret_cast<const uint32_t*>(scb_smem)
-                                           : reinterpret_cast<const uint32_t*>(w.scb);
-  if constexpr (L::kSVQ) {
-    if (sv.ds == 8)
-      for (int i = threadIdx.x; i < 512; i += 160)
-        reinterpret_cast<uint32_t*>(scb_smem)[i] = __ldg(reinterpret_cast<const uint32_t*>(w.scb) + i);
-  }
-  __syncthreads();
-  const size_t tile_id = static_cast<size_t>(n_tile) * KS + ks;
-  const size_t wsf = (static_cast<size_t>(n_tile) * KB4 + static_cast<size_t>(ks) * A) * 512;
-  if (threadIdx.x == 0) {
-    const uint32_t tx = 8192 + (cb_split ? 1024 : 512) + (L::kSVQ ? 128 * sv.G : L::kQBS ? 0 : A * 512);
-    mbar_arrive_expect_tx(bar, tx);
-    bulk_load(st + L::IDX_OFF, w.idx + tile_id * 8192, 8192, bar);
-    const int qbn = static_cast<int>((static_cast<int64_t>(n_tile) * 128) / qn);
-    const int qbk = cb_split ? 2 * ks : (ks * kStageK) / qk;
-    bulk_load(st + L::CB_OFF, w.cb + (static_cast<size_t>(qbn) * (K / qk) + qbk) * 256, cb_split ? 1024 : 512,
-              bar);
-    if constexpr (L::kSVQ) {
-      bulk_load(st + L::SIDX_OFF, sv.unit(w.sidx, n_tile, ks), 128 * sv.G, bar);
-    } else if constexpr (!L::kQBS) {
-      bulk_load(st + L::SFW_OFF, w.sf + wsf, A * 512, bar);
-    }
-  }
-  const bool ok = mbar_wait(bar, 0);
-  const int dt = threadIdx.x - 32;
-  if (threadIdx.x >= 32 && ok) build_lut<128>(reinterpret_cast<const uint16_t*>(st + L::CB_OFF), 1 + cb_split, lut, dt);
-  __syncthreads();
-  if (threadIdx.x >= 32 && ok) {
-    ItemMap<128> cm;
-    cm.init(dt, cb_split);
-    decode_w_tile<128>(st + L::IDX_OFF, smem_u32(lut), st + L::W_OFF, cm);
-    if constexpr (L::kSVQ)
-      decode_sf_tile<A, 128>(st + L::SIDX_OFF, sv.G, scb32, sv.lds, sv.kb_base(ks, L::kB), st + L::SFW_OFF, dt);
-    if constexpr (L::kQBS) {
-      const uint8_t* qb = w.sf + static_cast<size_t>((static_cast<int64_t>(n_tile) * 128) / qn) * (K / qk);
-      const int qbk = cb_split ? 2 * ks : (ks * kStageK) / qk;
-      fill_sf_qbs<A, 128>(st + L::SFW_OFF, __ldg(qb + qbk), __ldg(qb + qbk + cb_split), dt);
-    }
-  }
-  __syncthreads();
-  if (threadIdx.x >= 32 && ok) {
-    for (int it = 0; it < 8; ++it) {
-      const int c = it * 128 + dt;
-      const int r = c >> 3, j = c & 7;
-      const uint4 v = *reinterpret_cast<const uint4*>(st + L::W_OFF + r * 128 + ((j ^ (r & 7)) << 4));
-      *reinterpret_cast<uint4*>(q_out + (static_cast<int64_t>(n_tile) * 128 + r) * ldq + ks * 128 + j * 16) = v;
-    }
-    for (int i = dt; i < A * 32; i += 128)
-      reinterpret_cast<uint4*>(sf_out + wsf)[i] = reinterpret_cast<const uint4*>(st + L::SFW_OFF)[i];
-  }
-}
-
-// ------------------------------------------------------------------------------------
 // Decode dump for small QBlocks (64 rows or 64 input channels, down to 64 x 64: the fine
 // end of Figure 3's QBlock sweep).  A 128 x 256 tile-stage then draws on up to 8
 // codebooks ([2 row halves][4 K-quarters]), too many for per-lane codebook copies, so
 // the stage's codebooks sit once in shared memory and every index is looked up
-// directly (bank conflicts allowed).  Writes the same plain layouts as
-// decode_dump_kernel: FP4 codes [N, ldq], SF-layout scales.  Grid (N/128, K/256).
+// directly (bank conflicts allowed).  Writes the same plain layouts as the decode
+// pass: FP4 codes [N, ldq], SF-layout scales.  Grid (N/128, K/256).
 // ------------------------------------------------------------------------------------
 template <int FMT, int WSRC>
 __global__ void __launch_bounds__(128)
