@@ -192,17 +192,18 @@ mxc_status mxc_pack_weight(const mxc_weight_host* w, uint8_t* idx_out, uint8_t* 
 
 /* Workspace bytes each GPU call needs (0 if none).  M = activation rows;
  * for mxc_moe_linear M is the total number of (token, expert) rows.
- * mxc_linear: up to 16 rows, the split-K area when the 128-row output tiles are
+ * mxc_linear: a workspace it uses starts with 4 KiB of split-K arrival counters,
+ * which only the split-K below touches and which every call leaves zero: zero a
+ * workspace once after allocating it, and it stays valid whichever mxc_linear /
+ * mxc_native_linear calls use it.  Up to 16 rows, when the 128-row output tiles are
  * split along K into more than two ranks (ranks s = min(4, 148 / (N/128)), at
- * least 1) or into slices longer than 2048 input channels: N/128 uint32 arrival
- * counters rounded up to 256 bytes, then N/128 x R x 8 KiB of FP32 partial tiles,
- * R = the fewest ranks (at least s, at most 16) whose slices are at most 2048
- * input channels long, provided N/128 x R <= 148 (one CTA per SM); else 0.  The counters must be zero when a call starts and every
- * call leaves them zero: zero the workspace once after allocating it (and again
- * after another call has used it for other data).  Without the area, or with a
- * smaller workspace, the call runs on split-K clusters (slower for those shapes),
- * not an error.  17 to 128 rows: 0.  Above 128 rows when N is a multiple of 256
- * (else from 1024 rows) the room for the weight decoded once per call (N*K/2
+ * least 1) or into slices longer than 2048 input channels: the counters, then
+ * N/128 x R x 8 KiB of FP32 partial tiles, R = the fewest ranks (at least s, at
+ * most 16) whose slices are at most 2048 input channels long, provided
+ * N/128 x R <= 148 (one CTA per SM) and N/128 <= 1024; else 0.  Without that room
+ * the call runs on split-K clusters (slower for those shapes), not an error.  17
+ * to 128 rows: 0.  Above 128 rows when N is a multiple of 256 (else from 1024
+ * rows): the counters, then the room for the weight decoded once per call (N*K/2
  * bytes of FP4 codes rounded up to 1 KiB, then N*K/B bytes of SF-layout scales).
  * A smaller workspace is not an error there: the call then runs the fused
  * decode-in-GEMM kernel, which is slower at those sizes.
@@ -213,9 +214,9 @@ size_t mxc_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, mxc_format fm
 size_t mxc_moe_workspace_bytes(int64_t M, int32_t E, int64_t N, int64_t K, mxc_format fmt);
 /* The workspace mxc_linear needs for this weight at M rows: mxc_linear_workspace_bytes,
  * except for QBlocks of 64 rows or 64 input channels, which need the decoded weight's
- * room (N*K/2 rounded up to 1 KiB, plus N*K/B) at every M -- without it mxc_linear
- * returns MXC_ERR_WORKSPACE for them -- followed, up to 16 rows, by the split-K area
- * described above (same zero rule).  0 for an invalid weight. */
+ * room (N*K/2 rounded up to 1 KiB, plus N*K/B) after the counter area at every M --
+ * without it mxc_linear returns MXC_ERR_WORKSPACE for them -- followed, up to 16
+ * rows, by the split-K partial tiles described above.  0 for an invalid weight. */
 size_t mxc_linear_workspace_bytes_for(const mxc_weight* w, int64_t M);
 
 /* Rows of the SF layout that mxc_quantize_act_grouped writes:

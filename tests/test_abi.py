@@ -142,24 +142,24 @@ def test_packed_sizes_rejects_bad_shapes(L):
 
 
 def test_workspace_sizes(L):
-    # decode once: the decoded weight (FP4 codes, then the SF-layout scales), above 128
-    # tokens when N is a multiple of 256 (the CTA-pair GEMM), else from 1024 tokens
-    assert L.mxc_linear_workspace_bytes(4096, 9216, 4096, 1) == 9216 * 4096 // 2 + 9216 * 4096 // 16
-    assert L.mxc_linear_workspace_bytes(1024, 9216, 4096, 0) == 9216 * 4096 // 2 + 9216 * 4096 // 32
-    assert L.mxc_linear_workspace_bytes(129, 9216, 4096, 1) == 9216 * 4096 // 2 + 9216 * 4096 // 16
+    # every linear-layer workspace starts with a 4 KiB area of split-K arrival counters
+    C = 4096
+    # decode once: the counters, then the decoded weight (FP4 codes, then the SF-layout
+    # scales), above 128 tokens when N is a multiple of 256 (the CTA-pair GEMM), else
+    # from 1024 tokens
+    assert L.mxc_linear_workspace_bytes(4096, 9216, 4096, 1) == C + 9216 * 4096 // 2 + 9216 * 4096 // 16
+    assert L.mxc_linear_workspace_bytes(1024, 9216, 4096, 0) == C + 9216 * 4096 // 2 + 9216 * 4096 // 32
+    assert L.mxc_linear_workspace_bytes(129, 9216, 4096, 1) == C + 9216 * 4096 // 2 + 9216 * 4096 // 16
     assert L.mxc_linear_workspace_bytes(128, 9216, 4096, 1) == 0           # fused tiles: none
     assert L.mxc_linear_workspace_bytes(1023, 9344, 4096, 1) == 0          # N % 256 != 0: fused below 1024
-    assert L.mxc_linear_workspace_bytes(1024, 9344, 4096, 1) == 9344 * 4096 // 2 + 9344 * 4096 // 16
+    assert L.mxc_linear_workspace_bytes(1024, 9344, 4096, 1) == C + 9344 * 4096 // 2 + 9344 * 4096 // 16
     assert L.mxc_linear_workspace_bytes(16, 9216, 4096, 1) == 0            # decode: split-K in cluster SMEM
-    # decode with more than two split-K ranks or slices past 2048 channels: counters
-    # (N/128 uint32, rounded up to 256 B), then N/128 x ranks x 8 KiB of partial tiles
     # decode with more than two split-K ranks or slices past 2048 channels, all CTAs in
-    # one wave of 148: counters (N/128 uint32, rounded up to 256 B), then N/128 x ranks
-    # x 8 KiB of partial tiles
-    assert L.mxc_linear_workspace_bytes(16, 4608, 8192, 1) == 256 + 36 * 4 * 8192      # 4 ranks of 2048
-    assert L.mxc_linear_workspace_bytes(16, 4096, 4096, 1) == 256 + 32 * 4 * 4 * 2048  # 4 ranks of 1024
-    assert L.mxc_linear_workspace_bytes(1, 256, 9216, 0) == 256 + 2 * 5 * 8192         # 5 ranks, last short
-    assert L.mxc_linear_workspace_bytes(16, 128, 32768, 1) == 256 + 1 * 16 * 8192      # 16 ranks
+    # one wave of 148: the counters, then N/128 x ranks x 8 KiB of partial tiles
+    assert L.mxc_linear_workspace_bytes(16, 4608, 8192, 1) == C + 36 * 4 * 8192       # 4 ranks of 2048
+    assert L.mxc_linear_workspace_bytes(16, 4096, 4096, 1) == C + 32 * 4 * 4 * 2048   # 4 ranks of 1024
+    assert L.mxc_linear_workspace_bytes(1, 256, 9216, 0) == C + 2 * 5 * 8192          # 5 ranks, last short
+    assert L.mxc_linear_workspace_bytes(16, 128, 32768, 1) == C + 1 * 16 * 8192       # 16 ranks
     assert L.mxc_linear_workspace_bytes(16, 8192, 8192, 1) == 0            # 64 x 4 CTAs: two waves
     assert L.mxc_linear_workspace_bytes(16, 18432, 4096, 1) == 0           # 144 x 2 CTAs: two waves
     assert L.mxc_linear_workspace_bytes(17, 4608, 8192, 1) == 0            # tiled path: none

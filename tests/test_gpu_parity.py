@@ -555,8 +555,7 @@ def test_small_qblock_moe_is_refused():
 
 def _splitk_ws_layout(N, K, M=16):
     n = mxc.lib().mxc_linear_workspace_bytes(M, N, K, 1)
-    ctr = (N // 128 * 4 + 255) // 256 * 256
-    return n, ctr
+    return n, 4096                                   # the counter area leads every linear workspace
 
 
 @pytest.mark.parametrize("fmt,strat,N,K,M", [
@@ -636,3 +635,27 @@ def test_gemv_rounds(fmt, strat, N, K, qk, M, out, ws):
         assert torch.equal(y, mxc.native_linear(a, nat, out, ws=wsb))
     assert torch.equal(y, (mxc.native_linear(a, nat, out, ws=wsb) if native else mxc.linear(a, pw, out, ws=wsb)))
     assert mxc.get_device_error() == 0
+
+
+def test_linear_workspace_shared_by_decode_once_and_split_k():
+    """One workspace, zeroed once, serves a decode call that reduces through its arrival
+    counters, a decode-once call (which writes the decoded weight past the counter area)
+    and the decode call again: the counters stay valid and the results do not change."""
+    fmt, N, K = "e4m3_b16", 512, 4096                # 4 output tiles: 4 split-K ranks at M <= 16
+    w = synth.make_weight(151, fmt, "postscale", N, K, 256, 256)
+    pw = mxc.pack_weight(w)
+    x = synth.make_activations(151, 256, K, outliers=True)
+    a16 = mxc.quantize_act(dev_bf16(x[:16]), fmt)
+    a256 = mxc.quantize_act(dev_bf16(x), fmt)
+    ws = mxc.linear_workspace(256, N, K, fmt, "cuda")
+    assert ws.numel() >= mxc.lib().mxc_linear_workspace_bytes(16, N, K, 1) > 4096
+    y1 = mxc.linear(a16, pw, ws=ws)
+    y256 = mxc.linear(a256, pw, ws=ws)               # decode once into the same workspace
+    y2 = mxc.linear(a16, pw, ws=ws)
+    assert mxc.get_device_error() == 0
+    assert torch.count_nonzero(ws[:4096]).item() == 0
+    assert torch.equal(y1, y2)
+    ref, sabs = O.w4a4_linear(x[:16], w)
+    assert_close(y2.cpu().numpy(), ref, sabs, what="decode after decode once")
+    ref256, sabs256 = O.w4a4_linear(x, w)
+    assert_close(y256.cpu().numpy(), ref256, sabs256, what="decode once")

@@ -217,11 +217,17 @@ inline void decode_splits(int64_t N, int64_t K, int* splits, int* ks_per_split) 
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// The linear layer's workspace starts with a fixed area of split-K arrival counters
+// (one per 128-row output tile, at most 1024), which only the workspace split-K below
+// touches and which it leaves zero: a workspace zeroed once keeps valid counters
+// whichever calls (decode once, other shapes) used the rest of it.
+constexpr size_t kSplitkCtrBytes = 4096;
+
 // Split-K of the decode path through the workspace: when a tile would need more than
 // two cluster ranks, or slices longer than the GEMV's 8 resident stages, its ranks run
 // without a cluster (a cluster of four one-CTA-per-SM CTAs does not fit one wave) and
-// reduce through the workspace: one arrival counter per output tile (zero on entry,
-// zero again at exit), then [tile][rank][128][16] FP32 scaled partials.  Ranks: the
+// reduce through the workspace: the tile's arrival counter (zero on entry, zero again
+// at exit), and [tile][rank][128][16] FP32 scaled partials after the counter area.  Ranks: the
 // fewest that give slices of at most 8 stages, and no fewer than the cluster split;
 // only while all CTAs fit one wave (N = 4608, K = 8192: 9.8 us against 14.9 us on
 // clusters of four; past one wave the pipelined kernel is faster: K = N = 8192 16.3
@@ -236,16 +242,17 @@ inline bool gemv_ws_split(int64_t N, int64_t K, int* splits, int* ks_per_split) 
   n = n < s ? s : n;
   per = (KS + n - 1) / n;
   n = (KS + per - 1) / per;
-  if (n > kGemvWsMaxSplits || (N / kTileN) * n > kSMs) return false;
+  if (n > kGemvWsMaxSplits || (N / kTileN) * n > kSMs || N / kTileN > static_cast<int64_t>(kSplitkCtrBytes / 4))
+    return false;
   *splits = n;
   *ks_per_split = per;
   return true;
 }
-inline size_t splitk_ctr_bytes(int64_t N) { return align_up(static_cast<size_t>(N / kTileN) * 4, 256); }
-inline size_t splitk_ws_bytes(int64_t M, int64_t N, int64_t K) {
+// the partial tiles' bytes (0 when the shape does not reduce through the workspace)
+inline size_t splitk_part_bytes(int64_t M, int64_t N, int64_t K) {
   int s, per;
   if (M > kDecodeMaxM || !gemv_ws_split(N, K, &s, &per)) return 0;
-  return splitk_ctr_bytes(N) + static_cast<size_t>(N / kTileN) * s * 128 * kGemvT * 4;
+  return static_cast<size_t>(N / kTileN) * s * 128 * kGemvT * 4;
 }
 
 // Decode once: the layer decodes its weight once per call into the workspace (native
@@ -264,11 +271,14 @@ inline size_t decoded_weight_bytes(int64_t N, int64_t K, int fmt) {
   return decoded_codes_bytes(N, K) + static_cast<size_t>(N * K / (fmt == FMT_E8M0 ? 32 : 16));
 }
 
-// Small M: the split-K area when the shape reduces through the workspace (else the
-// partial sums stay in cluster shared memory and no workspace is needed).
-// Decode once (above): room for the decoded weight (without it the fused kernel runs).
+// Small M: the counters and the partial tiles when the shape reduces through the
+// workspace (else the partial sums stay in cluster shared memory and no workspace is
+// needed).  Decode once (above): the counter area, then room for the decoded weight
+// (without it the fused kernel runs).
 size_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt) {
-  return decode_once(M, N) ? decoded_weight_bytes(N, K, fmt) : splitk_ws_bytes(M, N, K);
+  if (decode_once(M, N)) return kSplitkCtrBytes + decoded_weight_bytes(N, K, fmt);
+  const size_t part = splitk_part_bytes(M, N, K);
+  return part ? kSplitkCtrBytes + part : 0;
 }
 
 // QBlocks of 64 rows or 64 input channels: a 128 x 256 tile-stage draws on up to 8
@@ -277,7 +287,7 @@ size_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt) {
 inline bool small_qblock(int64_t qn, int64_t qk) { return qn < kTileN || qk < 128; }
 
 size_t linear_workspace_bytes_for(int64_t M, int64_t N, int64_t K, int fmt, int64_t qn, int64_t qk) {
-  return small_qblock(qn, qk) ? decoded_weight_bytes(N, K, fmt) + splitk_ws_bytes(M, N, K)
+  return small_qblock(qn, qk) ? kSplitkCtrBytes + decoded_weight_bytes(N, K, fmt) + splitk_part_bytes(M, N, K)
                                : linear_workspace_bytes(M, N, K, fmt);
 }
 
@@ -453,7 +463,7 @@ cudaError_t launch_pair(const CUtensorMap& tx, const CUtensorMap& tw, const Gemm
 
 mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
   const bool small = a.wsrc != WSRC_NATIVE && small_qblock(a.qn, a.qk);
-  const bool ws_ok = a.ws && a.ws_bytes >= decoded_weight_bytes(a.N, a.K, a.fmt) &&
+  const bool ws_ok = a.ws && a.ws_bytes >= kSplitkCtrBytes + decoded_weight_bytes(a.N, a.K, a.fmt) &&
                      reinterpret_cast<uintptr_t>(a.ws) % 16 == 0;
   if (small && !ws_ok) return MXC_ERR_WORKSPACE;
   if (a.wsrc != WSRC_NATIVE && (small || decode_once(a.M, a.N)) && ws_ok) {
@@ -471,9 +481,9 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
     d.w_sidx = a.w_sidx;
     d.w_scb = a.w_scb;
     d.ds = a.w_ds;
-    d.q_out = static_cast<uint8_t*>(a.ws);
+    d.q_out = static_cast<uint8_t*>(a.ws) + kSplitkCtrBytes;
     d.ldq = a.K / 2;
-    d.sf_out = static_cast<uint8_t*>(a.ws) + decoded_codes_bytes(a.N, a.K);
+    d.sf_out = d.q_out + decoded_codes_bytes(a.N, a.K);
     const mxc_status s = run_decode_weight(d, stream);
     if (s != MXC_OK) return s;
     LinearArgs b = a;
@@ -482,9 +492,7 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
     b.w_ldq = d.ldq;
     b.w_sf = d.sf_out;
     b.w_tscale_dev = nullptr;                      // the weight tensor scale stays b.w_tscale
-    const size_t used = decoded_weight_bytes(a.N, a.K, a.fmt);   // the rest may hold the split-K area
-    b.ws = a.ws_bytes > used ? static_cast<uint8_t*>(a.ws) + used : nullptr;
-    b.ws_bytes = a.ws_bytes > used ? a.ws_bytes - used : 0;
+    b.ws_used = decoded_weight_bytes(a.N, a.K, a.fmt);   // the split-K partial tiles may follow it
     return run_linear(b, stream);
   }
   const int T = token_tile(a.M);
@@ -526,11 +534,12 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
     unsigned int* red_ctr = nullptr;
     int ws_splits, ws_per;
     if (a.M <= kDecodeMaxM && gemv_ws_split(a.N, a.K, &ws_splits, &ws_per) && a.ws &&
-        a.ws_bytes >= splitk_ws_bytes(a.M, a.N, a.K) && reinterpret_cast<uintptr_t>(a.ws) % 16 == 0) {
+        a.ws_bytes >= kSplitkCtrBytes + a.ws_used + splitk_part_bytes(a.M, a.N, a.K) &&
+        reinterpret_cast<uintptr_t>(a.ws) % 16 == 0) {
       splits = ws_splits;
       per = ws_per;
       red_ctr = static_cast<unsigned int*>(a.ws);
-      red_part = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) + splitk_ctr_bytes(a.N));
+      red_part = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) + kSplitkCtrBytes + a.ws_used);
     }
     p.splits = splits;
     p.ks_per_split = per;

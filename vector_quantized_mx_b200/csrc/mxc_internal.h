@@ -58,9 +58,11 @@ struct LinearArgs {
   void* y;
   int64_t ldy;
   int out_bf16;
-  // workspace
+  // workspace: [split-K arrival counters, kSplitkCtrBytes][the decoded weight, decode once]
+  // [split-K partial tiles]; ws_used = bytes past the counter area already taken
   void* ws;
   size_t ws_bytes;
+  size_t ws_used;
 };
 
 struct MoeArgs {
