@@ -100,8 +100,12 @@ struct GemvLayout {
   // once rank 0 has decoded; never used by native weights).
   static constexpr int IDX_OFF = X_OFF + S * kGemvT * 128;
   static constexpr int IDX_BUF = S * 2048;
-  static constexpr int SFW_OFF = IDX_OFF + 2 * IDX_BUF;           // weight scale atoms (direct, native)
-  static constexpr int LUT_OFF = SFW_OFF + (kSVQ ? 0 : S * kAtoms * 512);   // 256 words x 32 lanes
+  // weight scale atoms (direct, native, PostScale-QB); PreScale+: the scale codebook
+  // ([256][ds], at most 8 KB) and the round's scale-index units (at most 2 KB)
+  static constexpr int SFW_OFF = IDX_OFF + 2 * IDX_BUF;
+  static constexpr int SCB_OFF = SFW_OFF;
+  static constexpr int SIDX_OFF = SFW_OFF + 8192;
+  static constexpr int LUT_OFF = SFW_OFF + (kSVQ ? 16384 : S * kAtoms * 512);   // 256 words x 32 lanes
   static constexpr int CTRL_OFF = LUT_OFF + (kVQ ? kGemvLutBytes : 0);
   // The slice's codebooks (at most 16 x 512 B) land in the second half of the last
   // stage's FP4 tile, which is not written before the codebook copies are laid out.
@@ -182,7 +186,7 @@ __global__ void __maxnreg__(64)
   uint64_t* accum = bars + 14;
   uint64_t* red_full = bars + 15;   // rank 0: partial tiles received
   uint64_t* red_ready = bars + 16;  // rank > 0: rank 0 may receive
-  uint64_t* bar_sfw = bars + 17;    // weight scale atoms (bulk copy)
+  uint64_t* bar_sfw = bars + 17;    // weight scale atoms, or PreScale+ scale indices (+ codebook), by bulk copy
   uint64_t* bar_cb = bars + 18;     // codebooks of the slice (bulk copy)
   uint64_t* sfx_ready = bars + 20; // token scale atoms in TMEM (one arrival per token-scale warp)
   uint64_t* round_free = bars + 21; // a round's MMAs are done: its buffers and scale columns may be reused
@@ -265,9 +269,13 @@ __global__ void __maxnreg__(64)
         tma_load_2d(smem + L::W_OFF + s * 16384, &tmap_wq, (rb + s) * 128, n_tile * 128, &full[s]);
       }
     }
-    if constexpr (L::kSVQ) {
+    if constexpr (L::kSVQ) {                         // the round's scale indices (+ the scale codebook)
       const int u0 = rb >> sv.lspu, u1 = (rb + rn - 1) >> sv.lspu;
-      l2_prefetch_bulk(sv.unit(p.w.sidx, n_tile, rb), static_cast<uint32_t>(u1 - u0 + 1) * 128 * sv.G);
+      const uint32_t sidx_bytes = static_cast<uint32_t>(u1 - u0 + 1) * 128 * sv.G;
+      const uint32_t scb_bytes = r == 0 ? 256u * static_cast<uint32_t>(sv.ds) : 0u;
+      mbar_arrive_expect_tx(bar_sfw, sidx_bytes + scb_bytes);
+      bulk_load(smem + L::SIDX_OFF, sv.unit(p.w.sidx, n_tile, rb), sidx_bytes, bar_sfw);
+      if (r == 0) bulk_load(smem + L::SCB_OFF, p.w.scb, scb_bytes, bar_sfw);
     }
   };
 
@@ -375,6 +383,11 @@ __global__ void __maxnreg__(64)
             l2_prefetch_bulk(w_idx + static_cast<size_t>(nb) * 8192, static_cast<uint32_t>(nn) * 8192);
             if constexpr (!L::kSVQ && !L::kQBS)
               l2_prefetch_bulk(w_sf + static_cast<size_t>(nb) * A * 512, static_cast<uint32_t>(nn) * A * 512);
+            if constexpr (L::kSVQ) {
+              const int nbs = ks_begin + nb;
+              const int u0 = nbs >> sv.lspu, u1 = (nbs + nn - 1) >> sv.lspu;
+              l2_prefetch_bulk(sv.unit(p.w.sidx, n_tile, nbs), static_cast<uint32_t>(u1 - u0 + 1) * 128 * sv.G);
+            }
           }
         }
         issued_q = static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<unsigned>(issued_q)));   // the elected lane's count
@@ -393,7 +406,7 @@ __global__ void __maxnreg__(64)
       } else {
         for (int s = 0; s < rcount(last_r); ++s) mbar_wait(&full[s], ph);
       }
-      if constexpr (!L::kSVQ && !L::kQBS) mbar_wait(bar_sfw, ph);
+      if constexpr (!L::kQBS) mbar_wait(bar_sfw, ph);
     }
     __syncwarp();
     if (clustered && rank == 0 && !red_atomic) {
@@ -558,19 +571,24 @@ __global__ void __maxnreg__(64)
         __syncwarp();                                // tcgen05.st is warp-aligned
         // PreScale+ (Table 4 caption: Ks = 256, ds = 8; larger ds compress further):
         // row `lane` of atom (s, a) holds, for rows 32 g + lane (g = 0..3), block
-        // scales 4a..4a+3 of stage s: one word of the scale-codebook entry.
+        // scales 4a..4a+3 of stage s: one word of the scale-codebook entry.  The
+        // round's scale indices and the scale codebook are in shared memory.
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(qd * 32) << 16);
-        const uint32_t* scb32 = reinterpret_cast<const uint32_t*>(p.w.scb);
+        const bool have = mbar_wait(bar_sfw, static_cast<uint32_t>(r & 1));
+        const uint32_t* scb32 = reinterpret_cast<const uint32_t*>(smem + L::SCB_OFF);
+        const int u0 = (ks_begin + L::S * r) >> sv.lspu;
         for (int i = cg; i < rcount(r) * A; i += 4) {
           const int s = i / A, a = i % A;
           const int ks = ks_begin + L::S * r + s;
-          const uint8_t* un = sv.unit(p.w.sidx, n_tile, ks);
+          const uint8_t* un = smem + L::SIDX_OFF + ((ks >> sv.lspu) - u0) * 128 * sv.G;
           const int kb = sv.kb_base(ks, L::kB) + 4 * a;
-          uint4 v;
-          v.x = svq_word(un + (0 * 32 + lane) * sv.G, scb32, sv.lds, kb);
-          v.y = svq_word(un + (1 * 32 + lane) * sv.G, scb32, sv.lds, kb);
-          v.z = svq_word(un + (2 * 32 + lane) * sv.G, scb32, sv.lds, kb);
-          v.w = svq_word(un + (3 * 32 + lane) * sv.G, scb32, sv.lds, kb);
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (have) {
+            v.x = svq_word(un + (0 * 32 + lane) * sv.G, scb32, sv.lds, kb);
+            v.y = svq_word(un + (1 * 32 + lane) * sv.G, scb32, sv.lds, kb);
+            v.z = svq_word(un + (2 * 32 + lane) * sv.G, scb32, sv.lds, kb);
+            v.w = svq_word(un + (3 * 32 + lane) * sv.G, scb32, sv.lds, kb);
+          }
           tmem_st_32x32b_x4(lane_base + L::COL_SFW + 4 * i, v);
         }
         tmem_st_wait();
