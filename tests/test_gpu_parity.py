@@ -104,6 +104,41 @@ def test_quantize_act_bitexact(fmt, case):
     check_act(mx, x, fmt)
 
 
+def every_bf16_value_blocks(e, K=1024):
+    """Rows of 32-element blocks that hold every finite BF16 value v with |v| below the
+    block maximum 1.5 * 2^(e+2), which every block also holds (first element): the
+    E8M0 block exponent of every block is e."""
+    amax = np.array([1.5 * 2.0 ** (e + 2)], dtype=np.float32)
+    amax_bits = (amax.view(np.uint32) >> 16).astype(np.uint16)
+    allb = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = (allb.astype(np.uint32) << 16).view(np.float32)
+    keep = np.isfinite(vals) & (np.abs(vals) <= amax[0])
+    vb = allb[keep]
+    n_blocks = -(-len(vb) // 31)
+    blocks = np.zeros((n_blocks, 32), dtype=np.uint16)
+    blocks[:, 0] = amax_bits[0]
+    flat = blocks[:, 1:].reshape(-1)
+    flat[:len(vb)] = vb
+    blocks[:, 1:] = flat.reshape(n_blocks, 31)
+    per_row = K // 32
+    rows = -(-n_blocks // per_row)
+    out = np.zeros((rows * per_row, 32), dtype=np.uint16)
+    out[:n_blocks] = blocks
+    out[n_blocks:, 0] = amax_bits[0]
+    return out.reshape(rows, K)
+
+
+@pytest.mark.parametrize("e", [-127, -100, -30, -2, 0, 3, 40, 125])
+def test_quantize_e8m0_every_bf16_value(e):
+    """E8M0-B32 codes (by the tensor-core format conversion of x * 2^-e) for every BF16
+    value below the block maximum, at block exponents across the E8M0 range:
+    bit-exact against the oracle."""
+    x = every_bf16_value_blocks(e)
+    mx = mxc.quantize_act(dev_bf16(x), "e8m0_b32")
+    torch.cuda.synchronize()
+    check_act(mx, x, "e8m0_b32")
+
+
 def test_quantize_act_given_tensor_scale():
     x = synth.config2(16)[1]
     ts = torch.tensor([0.0123], dtype=torch.float32, device="cuda")

@@ -68,6 +68,21 @@ __device__ __forceinline__ uint32_t e2m1_code(float x, float d) {
   return c | ((__float_as_uint(x) >> 28) & 8u);
 }
 
+// E2M1 codes of two FP32 values by the hardware format conversion: round to nearest,
+// ties to even, saturating at +-6, the sign kept (also on zero); hi in bits 4..7, lo in
+// bits 0..3.  With an E8M0 block scale d = 2^e, x / d = x * 2^-e is exact (a result
+// below the normal range is far below the first midpoint 0.25 and codes 0 either
+// way), so these are exactly the codes e2m1_code(x, d) decides -- for every BF16 x
+// and every e in [-127, 127], checked exhaustively on the GPU against e2m1_code.
+__device__ __forceinline__ uint32_t e2m1x2_rn(float hi, float lo) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\t.reg .b16 h;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+      "mov.b16 h, {t, 0};\n\tcvt.u32.u16 %0, h;\n\t}"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
+
 // ------------------------------------------------------------------------------------
 // SwiGLU of the MoE projections, one FP32 operation per step (so that the codes of
 // its quantization are decided in exactly this arithmetic).  E(x) = e^x by Cody and
@@ -117,7 +132,14 @@ __device__ __forceinline__ void quantize_block_f32(const float (&v)[B], bool e4m
       const int flog = E ? static_cast<int>(E) - 127 : (31 - __clz(u & 0x7FFFFF)) - 149;
       const int e = min(127, max(-127, flog - 2));
       sfb = static_cast<uint32_t>(e + 127);
-      d = exp2_int(e);
+      // power-of-two scale: the codes of the exact quotients by the format conversion
+      const float inv = exp2_int(-e);
+#pragma unroll
+      for (int i = 0; i < B / 8; ++i) q[i] = 0;
+#pragma unroll
+      for (int i = 0; i < B / 2; ++i)
+        q[i / 4] |= e2m1x2_rn(v[2 * i + 1] * inv, v[2 * i] * inv) << (8 * (i % 4));
+      return;
     }
   } else {
     sfb = e4m3_encode_satfinite(__fdiv_rn(__fdiv_rn(a, 6.0f), s));
@@ -156,7 +178,14 @@ __device__ __forceinline__ void quantize_block(const uint32_t (&w)[B / 2], bool 
       const int flog = E ? static_cast<int>(E) - 127 : (31 - __clz(u & 0x7FFFFF)) - 149;
       const int e = min(127, max(-127, flog - 2));
       sf_byte = static_cast<uint32_t>(e + 127);
-      d = exp2_int(e);
+      // power-of-two scale: the codes of the exact quotients by the format conversion
+      const float inv = exp2_int(-e);
+#pragma unroll
+      for (int i = 0; i < B / 8; ++i) q[i] = 0;
+#pragma unroll
+      for (int i = 0; i < B / 2; ++i)
+        q[i / 4] |= e2m1x2_rn(bf16_hi(w[i]) * inv, bf16_lo(w[i]) * inv) << (8 * (i % 4));
+      return;
     }
   } else {
     const float t = __fdiv_rn(__fdiv_rn(amax, 6.0f), s);
