@@ -12,7 +12,7 @@
 //   * the loader copies the slice's index bytes with one 4-D tensor copy per
 //     K-quarter (quarter c of every stage: the packed layout stores each 128 x 256
 //     tile as four slabs of 64 input channels), quarter 0 first; the MMA warp
-//     fetches all token tiles with one 3-D tensor copy;
+//     fetches the round's token tiles with one 3-D tensor copy;
 //   * decoder lane l decodes stage l mod 8, so the 32 per-lane codebook copies in
 //     shared memory hold, in bank l, the codebook of lane l's stage: the codebooks
 //     of the whole slice are laid out once (one entry per 32-bit word, 32 KB) and
@@ -26,7 +26,9 @@
 //     the buffers of quarters 0 and 1 once those are decoded); the weight scale
 //     atoms come in by one bulk copy (PostScale-QB: the loader warp builds them
 //     from one byte per QBlock) and the MMA warp moves them to TMEM with
-//     tcgen05.cp;
+//     tcgen05.cp; PreScale+: the loader bulk-copies the round's scale indices
+//     (and once the scale codebook) into that staging area and the decoder warps
+//     build the atoms from shared memory and write them with tcgen05.st;
 //   * token scales: with at most 16 tokens only the first 16 of the 128 rows of
 //     an activation scale atom carry scales (the rest is zero padding), so four
 //     extra warps, one per TMEM lane quadrant, load those 16 words per atom and
@@ -39,9 +41,10 @@
 //     one 8 KB bulk copy between shared memories (completion on an mbarrier there,
 //     an acknowledgement back before the sender may exit) and rank 0 adds the
 //     scaled partials in rank order (for two ranks the same FP32 value);
-//   * split-K through the workspace (more than two ranks, or slices of K past one
-//     CTA's 8 resident stages, when the caller gives the room): no cluster -- a
-//     cluster of four one-CTA-per-SM CTAs cannot be placed in one wave -- each
+//   * split-K through the workspace (more than two ranks, or slices past 8
+//     stages, while all CTAs fit one wave and the caller gives the room): no
+//     cluster -- a cluster of four one-CTA-per-SM CTAs cannot be placed in one
+//     wave -- each
 //     rank writes its scaled partial tile to the workspace and takes a ticket from
 //     the tile's arrival counter (atomicInc wrapping at splits - 1, so the counter
 //     is back at zero after every call); the rank that arrives last adds the
