@@ -234,7 +234,8 @@ __global__ void amax_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K
 }
 
 // One (scale row, block) unit: dense mode maps scale row = data row (rows past M
-// only get zero scales); grouped mode maps padded scale rows back to data rows.
+// only get zero scales); grouped mode maps padded scale rows back to data rows
+// (offsets and tile_prefix: the CTA's shared-memory copies).
 template <int B>
 __device__ __forceinline__ void quantize_unit(const uint16_t* __restrict__ x, int64_t M, int64_t K, int64_t ldx,
                                               int e4m3, float s, uint8_t* __restrict__ q, int64_t ldq,
@@ -290,6 +291,18 @@ __global__ void __launch_bounds__(256) quantize_kernel(
     uint8_t* __restrict__ q, int64_t ldq, uint8_t* __restrict__ sf, float* __restrict__ tscale_out,
     int64_t sf_rows, const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_prefix,
     int32_t n_groups) {
+  // grouped mode: the group offsets and tile prefix once per CTA into shared memory,
+  // so that each unit's group search costs shared-memory loads, not L2 round trips
+  __shared__ int32_t off_s[kMaxGroups + 1], tp_s[kMaxGroups + 1];
+  if (tile_prefix) {
+    for (int g = threadIdx.x; g <= n_groups; g += blockDim.x) {
+      off_s[g] = offsets[g];
+      tp_s[g] = tile_prefix[g];
+    }
+    __syncthreads();
+    offsets = off_s;
+    tile_prefix = tp_s;
+  }
   const int kb_per_row = static_cast<int>(K / B);
   float s = 1.0f;
   if (e4m3) {
