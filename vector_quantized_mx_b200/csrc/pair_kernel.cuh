@@ -314,11 +314,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // BF16 rows through the staging sub-tiles and tensor stores: warp (qd, cg) writes
         // rows 32 qd .. + 31 of sub-tile cg (weight rows n0p + 64 cg .. + 63), 16-byte
         // chunk c of row r at chunk c ^ (r mod 8) -- the 128-byte swizzle of the store map.
-        if (threadIdx.x == 64) bulk_wait_group_read0();   // the last tile's stores have read the staging
-        named_bar_sync(1, kDecThreads);
         const bool live = q0 < p.M;                     // warp-uniform: some token of this quadrant exists
-        // the warp's 64 columns into registers, release the accumulator, then the BF16
-        // staging stores
+        // the warp's 64 columns into registers and the accumulator released at once
+        // (no CTA-wide barrier on the way: the next tile's MMAs wait for this), then,
+        // once the last tile's stores have read the staging, the BF16 staging stores
         uint32_t v[64];
         if (live) {
           __syncwarp();                                 // tcgen05.ld is warp-aligned
@@ -333,6 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (rank == 0) mbar_arrive(acc_free);
           else mbar_remote_arrive(acc_free0);
         }
+        if (threadIdx.x == 64) bulk_wait_group_read0();   // the last tile's stores have read the staging
+        named_bar_sync(1, kDecThreads);
         if (live) {
           const int r = qd * 32 + lane;
           uint8_t* const row = out_stage + cg * 16384 + r * 128;
