@@ -643,7 +643,7 @@ def test_gemv_splitk_through_workspace(fmt, strat, N, K, M):
     ("e4m3_b16", "postscale", 6400, 4608, 256, 16, torch.float32, True),       # 2 ranks of 9: red.global.add
     ("e8m0_b32", "prescale", 4864, 7680, 128, 5, torch.bfloat16, True),        # 3 ranks of 10: cluster sum, 2 codebooks a stage
     ("e4m3_b16", "prescale_plus", 256, 10240, 256, 16, torch.float32, False),  # 4 ranks of 10 (no workspace)
-    ("e8m0_b32", "postscale_qb", 256, 9216, 256, 1, torch.float32, False),     # 4 ranks of 9, one stage in round 1
+    ("e8m0_b32", "postscale_qb", 256, 9216, 256, 1, torch.float32, False),     # 4 ranks of 9, one stage in the second round of 8
     ("e4m3_b16", "native", 6400, 4608, 256, 16, torch.bfloat16, True),         # native FP4 weights
     ("e4m3_b16", "postscale", 6400, 12288, 256, 16, torch.float32, True),      # 2 ranks of 24: three rounds
     ("e8m0_b32", "prescale_plus", 256, 32768, 256, 3, torch.bfloat16, False),  # 4 ranks of 32: four rounds
