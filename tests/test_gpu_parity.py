@@ -647,6 +647,8 @@ def test_gemv_splitk_through_workspace(fmt, strat, N, K, M):
     ("e4m3_b16", "native", 6400, 4608, 256, 16, torch.bfloat16, True),         # native FP4 weights
     ("e4m3_b16", "postscale", 6400, 12288, 256, 16, torch.float32, True),      # 2 ranks of 24: three rounds
     ("e8m0_b32", "prescale_plus", 256, 32768, 256, 3, torch.bfloat16, False),  # 4 ranks of 32: four rounds
+    ("e4m3_b16", "prescale_plus", 256, 10240, 128, 16, torch.float32, False),  # two codebooks a stage, scale VQ
+    ("e8m0_b32", "postscale_qb", 512, 8704, 128, 9, torch.float32, False),     # two codebooks a stage, QBlock scales
 ])
 def test_gemv_rounds(fmt, strat, N, K, qk, M, out, ws):
     native = strat == "native"
