@@ -269,6 +269,15 @@ __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, uint32_t src,
 __device__ __forceinline__ void mbar_remote_arrive(uint32_t remote_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
+// Arrive on an mbarrier of another CTA of the cluster with the instruction's default
+// semantics (release at CTA scope), for a signal that publishes no memory: "this
+// thread's tensor-memory loads are complete" after tcgen05.wait::ld and
+// tcgen05.fence::before_thread_sync.  A cluster-scope release waits for the thread's
+// memory traffic to reach cluster scope first (about 900 cycles in the pair GEMM's
+// epilogue, on the path between one tile's last MMA and the next tile's first).
+__device__ __forceinline__ void mbar_remote_arrive_signal(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
 
 // ------------------------------------------------------------------------------------
 // Programmatic dependent launch and L2 prefetch

@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) {                                // the next tile's MMAs may start
           if (rank == 0) mbar_arrive(acc_free);
-          else mbar_remote_arrive(acc_free0);
+          else mbar_remote_arrive_signal(acc_free0);
         }
         if (threadIdx.x == 64) bulk_wait_group_read0();   // the last tile's stores have read the staging
         named_bar_sync(1, kDecThreads);
@@ -405,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) {                                  // this warp is done with the accumulator
         if (rank == 0) mbar_arrive(acc_free);
-        else mbar_remote_arrive(acc_free0);
+        else mbar_remote_arrive_signal(acc_free0);
       }
     }
   }
