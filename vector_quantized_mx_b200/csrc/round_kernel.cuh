@@ -14,15 +14,19 @@
 //   * the decoders lay out the 32 per-lane codebook copies once per round (decoder
 //     lane l decodes stage l mod 4, so lane l's copy holds that stage's codebook:
 //     conflict-free lookups, as in the decode GEMV) and decode the four stages K-quarter
-//     by K-quarter straight into the swizzled FP4 operand tiles; PreScale+ and
-//     PostScale-QB weight scales they write to TMEM themselves, from shared memory;
+//     by K-quarter straight into the swizzled FP4 operand tiles; PreScale+ weight
+//     scale atoms they build once per round in shared memory from the scale indices
+//     and the scale codebook (the MMA warp moves them to TMEM with tcgen05.cp), the
+//     PostScale-QB ones they write to TMEM themselves from the QBlock's byte;
 //   * the MMA warp runs the first token tile's block-scaled MMAs (M = 128 weight rows,
 //     N = 128 tokens, K = 64) quarter by quarter behind the decode, then the second
 //     tile's on the same decoded weights: each weight tile is decoded once per 256
 //     tokens of its expert instead of once per 128;
 //   * the token operands of one tile and round (four stages, only the 32-row boxes
 //     that hold the expert's rows) and its scale atoms stream through one buffer,
-//     reloaded for the next tile once the MMAs that read it are done.
+//     reloaded for the next tile once the MMAs that read it are done -- by a warp of
+//     their own, so that the weight loader never waits for a token buffer before
+//     requesting the next round's weight data.
 //
 // Two TMEM accumulators hold the chunk's two tiles across all rounds; the epilogue
 // scales them and writes FP32 or BF16 rows of Y.  Within a tile the K order of the
@@ -37,7 +41,8 @@ namespace mxc {
 constexpr int kRoundStages = 4;       // 256-channel stages decoded together
 constexpr int kChunkTiles = 2;        // 128-token tiles per work item
 constexpr int kRoundEpiWarps = 4;     // epilogue warps, one per TMEM lane quadrant
-constexpr int kRoundThreads = kThreads + 32 * kRoundEpiWarps;
+constexpr int kRoundTokWarp = 2 + kDecWarps + kRoundEpiWarps;   // the token-tile loader
+constexpr int kRoundThreads = 32 * (kRoundTokWarp + 1);
 
 struct MoeRoundParams {
   int M, N, K;
@@ -61,11 +66,20 @@ struct MoeRoundParams {
   ExpertPtrs w[kMaxGroups];
 };
 
+// The expert data of a work item, copied once per item from the kernel parameters
+// into shared memory (by the loader, ahead of the item): a parameter read indexed by
+// the expert costs a constant-cache round trip of the order of a thousand SM clocks,
+// which the loader would otherwise pay before every round's copies and the decoders
+// before their first use of the scale-VQ geometry.
+struct ItemSlot {
+  ExpertPtrs w;
+  int qbn[2];                         // codebook row of the item's band (fused SwiGLU: and of its up band)
+};
+
 template <int FMT, int WSRC>
 struct RoundLayout {
   static constexpr bool kSVQ = WSRC == WSRC_VQ_SVQ;
   static constexpr bool kQBS = WSRC == WSRC_VQ_QBS;
-  static constexpr bool kSfwDec = kSVQ || kQBS;             // weight scales written to TMEM by the decoders
   static constexpr int kB = FMT == FMT_E8M0 ? 32 : 16;
   static constexpr int A = kStageK / kB / 4;                 // scale atoms per 128 rows per stage
   static constexpr int RS = kRoundStages;
@@ -75,14 +89,16 @@ struct RoundLayout {
   static constexpr int LUT_OFF = IDX_OFF + RS * 8192;        // 32 per-lane copies x 256 words
   static constexpr int CB_OFF = LUT_OFF + kGemvLutBytes;      // the round's codebooks (<= 2 per stage)
   // Weight scale data: the direct scale atoms of two rounds (by round parity); or
-  // the expert's scale codebook [256][ds] (<= 8 KB) and the round's scale indices
-  // (<= 1 KB).
+  // the expert's scale codebook [256][ds] (<= 8 KB), the round's scale indices
+  // (<= 1 KB) and the round's scale atoms built from them (SFS_OFF, for tcgen05.cp).
   static constexpr int AUX_OFF = CB_OFF + 2 * RS * 512;
-  static constexpr int AUX_BYTES = 16384;
   static constexpr int SIDX_OFF = AUX_OFF + 8192;
+  static constexpr int SFS_OFF = AUX_OFF + 10240;
+  static constexpr int AUX_BYTES = kSVQ ? 10240 + RS * A * 512 : 16384;
   static constexpr int SFX_OFF = AUX_OFF + AUX_BYTES;        // token scale atoms of one (round, tile)
   static constexpr int TAB_OFF = SFX_OFF + RS * A * 512;     // tile and chunk prefixes, 2 (E+1) int32
   static constexpr int CTRL_OFF = TAB_OFF + 2 * (kMaxGroups + 1) * 4 + 8;
+  static constexpr int EXP_OFF = CTRL_OFF + 128;             // two ItemSlots, by item parity
   static constexpr int SMEM = 1024 + CTRL_OFF + 256;
   // TMEM: accumulators of the item's two tiles [0, 256), then two buffers each of
   // weight scales (by round parity) and token scales (by (round, tile) parity), so
@@ -93,6 +109,8 @@ struct RoundLayout {
   static constexpr int TMEM_COLS = 512;
   static_assert(COL_SFX + 2 * SF_COLS <= TMEM_COLS, "tensor memory");
   static_assert(2 * RS * A * 512 <= AUX_BYTES, "direct scale staging");
+  static_assert(SFS_OFF % 1024 == 0, "scale atom staging");
+  static_assert(CTRL_OFF % 8 == 0 && 128 + 2 * sizeof(ItemSlot) <= 256, "control area");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
@@ -181,7 +199,7 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
   uint64_t* bar_hi = bars + 1;      // [2], by round parity
   uint64_t* bar_x = bars + 3;       // a tile's token operands and scales landed
   uint64_t* dec_ph = bars + 4;      // [2] half h (K-quarters 2h, 2h+1) of the round decoded; half 0 also
-                                    //     means the round's weight scales are in TMEM
+                                    //     means (PostScale-QB) the round's weight scales are in TMEM
   uint64_t* xfree = bars + 8;       // MMAs of one (round, tile) done: the token buffer is free
   uint64_t* w_free = bars + 9;      // MMAs of one round's half 0 done: its quarters 0-1 of the operand
                                     //     tiles are free (w_free + 4: half 1, quarters 2-3)
@@ -189,13 +207,17 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
   uint64_t* acc_free = bars + 11;   // the epilogue (fused SwiGLU: the decoders) has read an item's accumulators
   uint64_t* mma_done = bars + 12;   // every MMA this CTA issued is complete (once, at the end)
   uint64_t* w_free1 = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
-  constexpr int kBars = 14;
+  uint64_t* sf_ready = bars + 14;   // PreScale+: the round's weight scale atoms are in shared memory
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  constexpr int kBars = 15;
+  static_assert(8 * kBars + 4 <= 128, "barriers below the item slots");
+  ItemSlot* const slots = reinterpret_cast<ItemSlot*>(smem + L::EXP_OFF);
 
   // ---- setup ----
   if (warp == 0) {
     if (lane < kBars)
-      mbar_init(bars + lane, lane >= 4 && lane < 6 ? kDecWarps : lane == 11 ? (SWI ? kDecWarps : kRoundEpiWarps) : 1);
+      mbar_init(bars + lane, (lane >= 4 && lane < 6) || lane == 14 ? kDecWarps
+                                                                  : lane == 11 ? (SWI ? kDecWarps : kRoundEpiWarps) : 1);
     __syncwarp();
     if (lane == 0) {
       fence_mbar_init();
@@ -214,80 +236,107 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
 
   if (warp == 0) {
     // =============================== loader ===============================
-    auto issue_lo = [&](const RoundItem& it, int v) {    // round v of item it
+    // the item's expert data into its slot (its first round's copies read it from there)
+    auto fill_slot = [&](ItemSlot* sl, const RoundItem& it) {
+      sl->w = p.w[it.e];
+      sl->qbn[0] = qbn_of(it.n_tile);
+      sl->qbn[1] = SWI ? qbn_of(it.n_tile + n_bands) : 0;
+    };
+    // Each copy is prepared (addresses and byte counts in registers) before the wait
+    // that releases it and fired right after: with the decoders keeping the shared
+    // memory pipe busy, the loader's own shared-memory reads and address arithmetic
+    // take of the order of a thousand SM clocks, which would otherwise sit between
+    // the decoders finishing a half and the next round's data being requested.
+    struct LoCopy {                                  // a round's first part
+      const uint8_t* idx;                            // its index tiles (quarters 0-1 of each stage)
+      const uint16_t* cb;                            // its codebooks
+      const uint8_t* sidx;                           // PreScale+: its scale-index units
+      const uint8_t* scb;                            // PreScale+: the scale codebook (an item's first round)
+      uint32_t tx, cb_bytes, sidx_bytes, scb_bytes;
+      int rs;
+    };
+    struct HiCopy {                                  // a round's second part
+      const uint8_t* idx;                            // quarters 2-3 of each stage
+      const uint8_t* sf;                             // direct scales: the round's scale atoms
+      uint32_t tx;
+      int rs;
+    };
+    auto prepare_lo = [&](const RoundItem& it, int v, const ItemSlot& sl) {    // round v of item it
       const int r = kr(v), band = wband(it, v);
       const int ks0 = r * RS, rs = min(RS, KS - ks0);
       const int qb0 = qb_first(ks0), qb1 = qb_last(ks0 + rs - 1);
-      const uint8_t* const w_idx = p.w[it.e].idx;
-      const uint16_t* const w_cb = p.w[it.e].cb;
-      const int qbn = qbn_of(band);
-      uint32_t tx = rs * 4096 + (qb1 - qb0 + 1) * 512;
-      [[maybe_unused]] int nu = 0;
-      [[maybe_unused]] const SvqGeom sv(p.w[it.e].ds, L::kB, KS);
+      const int qbn = sl.qbn[SWI && v >= nr ? 1 : 0];
+      LoCopy c;
+      c.rs = rs;
+      c.idx = sl.w.idx + (static_cast<size_t>(band) * KS + ks0) * 8192;
+      c.cb = sl.w.cb + (static_cast<size_t>(qbn) * cb_per_row + qb0) * 256;
+      c.cb_bytes = static_cast<uint32_t>(qb1 - qb0 + 1) * 512;
+      c.tx = rs * 4096 + c.cb_bytes;
+      c.sidx = nullptr;
+      c.scb = nullptr;
+      c.sidx_bytes = 0;
+      c.scb_bytes = 0;
       if constexpr (L::kSVQ) {
-        nu = ((ks0 + rs - 1) >> sv.lspu) - (ks0 >> sv.lspu) + 1;
-        tx += nu * 128 * sv.G;
-        if (v == 0) tx += 256 * sv.ds;
+        const SvqGeom sv(sl.w.ds, L::kB, KS);
+        c.sidx = sv.unit(sl.w.sidx, band, ks0);
+        c.sidx_bytes = static_cast<uint32_t>(((ks0 + rs - 1) >> sv.lspu) - (ks0 >> sv.lspu) + 1) * 128 * sv.G;
+        if (v == 0) {
+          c.scb = sl.w.scb;
+          c.scb_bytes = 256 * sv.ds;
+        }
+        c.tx += c.sidx_bytes + c.scb_bytes;
       }
-      if (r == 0) {                                  // the band's later rounds on their way into L2
+      if (r == 0 && lane == 0) {                     // the band's later rounds on their way into L2
         for (int ks = RS; ks < KS; ks += 4)          // 32 KB a request
-          l2_prefetch_bulk(w_idx + (static_cast<size_t>(band) * KS + ks) * 8192,
+          l2_prefetch_bulk(sl.w.idx + (static_cast<size_t>(band) * KS + ks) * 8192,
                            static_cast<uint32_t>(min(4, KS - ks)) * 8192);
-        l2_prefetch_bulk(w_cb + static_cast<size_t>(qbn) * cb_per_row * 256, static_cast<uint32_t>(cb_per_row) * 512);
+        l2_prefetch_bulk(sl.w.cb + static_cast<size_t>(qbn) * cb_per_row * 256,
+                         static_cast<uint32_t>(cb_per_row) * 512);
       }
-      mbar_arrive_expect_tx(bar_lo, tx);
-      for (int s = 0; s < rs; ++s)
-        bulk_load(smem + L::IDX_OFF + s * 8192, w_idx + (static_cast<size_t>(band) * KS + ks0 + s) * 8192, 4096,
-                  bar_lo);
-      bulk_load(smem + L::CB_OFF, w_cb + (static_cast<size_t>(qbn) * cb_per_row + qb0) * 256, (qb1 - qb0 + 1) * 512,
-                bar_lo);
+      return c;
+    };
+    auto fire_lo = [&](const LoCopy& c) {
+      mbar_arrive_expect_tx(bar_lo, c.tx);
+      for (int s = 0; s < c.rs; ++s) bulk_load(smem + L::IDX_OFF + s * 8192, c.idx + s * 8192, 4096, bar_lo);
+      bulk_load(smem + L::CB_OFF, c.cb, c.cb_bytes, bar_lo);
       if constexpr (L::kSVQ) {
-        bulk_load(smem + L::SIDX_OFF, sv.unit(p.w[it.e].sidx, band, ks0), nu * 128 * sv.G, bar_lo);
-        if (v == 0) bulk_load(smem + L::AUX_OFF, p.w[it.e].scb, 256 * sv.ds, bar_lo);
+        bulk_load(smem + L::SIDX_OFF, c.sidx, c.sidx_bytes, bar_lo);
+        if (c.scb_bytes) bulk_load(smem + L::AUX_OFF, c.scb, c.scb_bytes, bar_lo);
       }
     };
-    auto issue_hi = [&](const RoundItem& it, int v, int g) {   // g: the global round number
+    auto prepare_hi = [&](const RoundItem& it, int v, const ItemSlot& sl) {
       const int r = kr(v), band = wband(it, v);
       const int ks0 = r * RS, rs = min(RS, KS - ks0);
-      uint64_t* bar = bar_hi + (g & 1);
-      const uint8_t* const w_idx = p.w[it.e].idx;
-      uint32_t tx = rs * 4096;
-      if constexpr (WSRC == WSRC_VQ_DIRECT) tx += rs * A * 512;
-      mbar_arrive_expect_tx(bar, tx);
-      for (int s = 0; s < rs; ++s)
-        bulk_load(smem + L::IDX_OFF + s * 8192 + 4096,
-                  w_idx + (static_cast<size_t>(band) * KS + ks0 + s) * 8192 + 4096, 4096, bar);
-      if constexpr (WSRC == WSRC_VQ_DIRECT)
-        bulk_load(smem + L::AUX_OFF + (g & 1) * RS * A * 512,
-                  p.w[it.e].sf + (static_cast<size_t>(band) * KB4 + static_cast<size_t>(ks0) * A) * 512,
-                  rs * A * 512, bar);
+      HiCopy c;
+      c.rs = rs;
+      c.idx = sl.w.idx + (static_cast<size_t>(band) * KS + ks0) * 8192 + 4096;
+      c.sf = nullptr;
+      c.tx = rs * 4096;
+      if constexpr (WSRC == WSRC_VQ_DIRECT) {
+        c.sf = sl.w.sf + (static_cast<size_t>(band) * KB4 + static_cast<size_t>(ks0) * A) * 512;
+        c.tx += rs * A * 512;
+      }
+      return c;
     };
-    auto issue_x = [&](const RoundItem& it, int v, int t) {    // tile t's tokens and their scales, round v
-      const int ks0 = kr(v) * RS, rs = min(RS, KS - ks0);
-      const int64_t tm0 = it.m0 + static_cast<int64_t>(t) * 128;
-      const int64_t rows = it.m_end - tm0 < 128 ? it.m_end - tm0 : 128;
-      const int boxes = static_cast<int>((rows + kMoeXBox - 1) / kMoeXBox);
-      mbar_arrive_expect_tx(bar_x, rs * boxes * kMoeXBox * 128 + rs * A * 512);
-      for (int s = 0; s < rs; ++s)
-        for (int q = 0; q < boxes; ++q)
-          tma_load_2d(smem + L::X_OFF + s * 16384 + q * kMoeXBox * 128, &tmap_x, (ks0 + s) * 128,
-                      static_cast<int>(tm0) + q * kMoeXBox, bar_x);
-      bulk_load(smem + L::SFX_OFF,
-                p.a_sf + (static_cast<size_t>(it.tile0 + t) * KB4 + static_cast<size_t>(ks0) * A) * 512, rs * A * 512,
-                bar_x);
+    auto fire_hi = [&](const HiCopy& c, int g) {     // g: the global round number
+      uint64_t* bar = bar_hi + (g & 1);
+      mbar_arrive_expect_tx(bar, c.tx);
+      for (int s = 0; s < c.rs; ++s) bulk_load(smem + L::IDX_OFF + s * 8192 + 4096, c.idx + s * 8192, 4096, bar);
+      if constexpr (WSRC == WSRC_VQ_DIRECT)
+        bulk_load(smem + L::AUX_OFF + (g & 1) * RS * A * 512, c.sf, c.rs * A * 512, bar);
     };
     // The first round of an item into L2 while the item before it runs: its index
     // tiles, codebooks, scale indices and scale codebook, and its first token tile.
-    auto prefetch_first_round = [&](const RoundItem& it) {
+    auto prefetch_first_round = [&](const RoundItem& it, const ItemSlot& sl) {
       const int rs = min(RS, KS);
-      l2_prefetch_bulk(p.w[it.e].idx + static_cast<size_t>(it.n_tile) * KS * 8192, static_cast<uint32_t>(rs) * 8192);
+      l2_prefetch_bulk(sl.w.idx + static_cast<size_t>(it.n_tile) * KS * 8192, static_cast<uint32_t>(rs) * 8192);
       const int qb1 = qb_last(rs - 1);
-      l2_prefetch_bulk(p.w[it.e].cb + static_cast<size_t>(qbn_of(it.n_tile)) * cb_per_row * 256,
+      l2_prefetch_bulk(sl.w.cb + static_cast<size_t>(sl.qbn[0]) * cb_per_row * 256,
                        static_cast<uint32_t>(qb1 + 1) * 512);
       if constexpr (L::kSVQ) {
-        const SvqGeom sv(p.w[it.e].ds, L::kB, KS);
-        l2_prefetch_bulk(sv.unit(p.w[it.e].sidx, it.n_tile, 0), static_cast<uint32_t>(sv.U) * 128 * sv.G);
-        l2_prefetch_bulk(p.w[it.e].scb, 256 * sv.ds);
+        const SvqGeom sv(sl.w.ds, L::kB, KS);
+        l2_prefetch_bulk(sv.unit(sl.w.sidx, it.n_tile, 0), static_cast<uint32_t>(sv.U) * 128 * sv.G);
+        l2_prefetch_bulk(sl.w.scb, 256 * sv.ds);
       }
       const int64_t rows = it.m_end - it.m0 < 128 ? it.m_end - it.m0 : 128;
       const int boxes = static_cast<int>((rows + kMoeXBox - 1) / kMoeXBox);
@@ -295,34 +344,52 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
         for (int q = 0; q < boxes; ++q)
           l2_prefetch_tile_2d(&tmap_x, s * 128, static_cast<int>(it.m0) + q * kMoeXBox);
     };
+    // Item li's expert data sits in slots[li & 1]: the slot of item li + 1 is filled
+    // when item li starts (the decoders read a slot only in the first round of its
+    // item, after that round's first part has landed, which the loader requests after
+    // filling the slot; by then every reader of the slot's previous item is past it).
     RoundItem cur = item(k_first, true);
     __syncwarp();
-    if (elect_one()) {
-      issue_lo(cur, 0);
-      issue_hi(cur, 0, 0);
-      issue_x(cur, 0, 0);
-    }
+    if (elect_one()) fill_slot(&slots[0], cur);
     __syncwarp();
-    int nlo = 1, nhi = 1, nx = 1;                    // copies issued so far
-    int g = 0, kx = 0;                               // global round, (round, tile) counters
+    {
+      const LoCopy lo = prepare_lo(cur, 0, slots[0]);
+      const HiCopy hi = prepare_hi(cur, 0, slots[0]);
+      if (elect_one()) {
+        fire_lo(lo);
+        fire_hi(hi, 0);
+      }
+      __syncwarp();
+    }
+    int nlo = 1, nhi = 1;                            // copies issued so far
+    int g = 0;                                       // global round
     bool ok = true;
-    for (int k = k_first; k < n_items && ok; k += k_step) {
+    for (int k = k_first, li = 0; k < n_items && ok; k += k_step, ++li) {
       const bool has_next = k + k_step < n_items;
       RoundItem nxt = cur;
+      ItemSlot& sc = slots[li & 1];
+      ItemSlot& sn = slots[(li + 1) & 1];
       if (has_next) {
         nxt = item(k + k_step, true);                // loads in flight while this item runs
-        if (lane == 0) prefetch_first_round(nxt);
+        if (elect_one()) {
+          fill_slot(&sn, nxt);
+          prefetch_first_round(nxt, sn);
+        }
+        __syncwarp();
       }
       for (int r = 0; r < nrv && ok; ++r, ++g) {
         const bool next_round = r + 1 < nrv || has_next;
         const RoundItem& ni = r + 1 < nrv ? cur : nxt;
+        const ItemSlot& ns = r + 1 < nrv ? sc : sn;
         const int nrr = r + 1 < nrv ? r + 1 : 0;
         if (next_round) {
+          const LoCopy lo = prepare_lo(ni, nrr, ns);
+          const HiCopy hi = prepare_hi(ni, nrr, ns);
           // the decoders are done with this round's codebooks, scale indices and index
           // quarters 0-1: the next round's may come in
           ok = __all_sync(0xffffffffu, mbar_wait(&dec_ph[0], g & 1));
           if (!ok) break;
-          if (elect_one()) issue_lo(ni, nrr);
+          if (elect_one()) fire_lo(lo);
           __syncwarp();
           ++nlo;
           // and with quarters 2-3; the direct scale atoms go to the other staging
@@ -330,22 +397,9 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
           // decode began (the decoders waited for round g-1's MMAs)
           ok = __all_sync(0xffffffffu, mbar_wait(&dec_ph[1], g & 1));
           if (!ok) break;
-          if (elect_one()) issue_hi(ni, nrr, g + 1);
+          if (elect_one()) fire_hi(hi, g + 1);
           __syncwarp();
           ++nhi;
-        }
-        for (int t = 0; t < cur.nt && ok; ++t, ++kx) {
-          ok = __all_sync(0xffffffffu, mbar_wait(xfree, kx & 1));   // its MMAs are done with the buffer
-          if (!ok) break;
-          const bool more = t + 1 < cur.nt || next_round;
-          if (more) {
-            if (elect_one()) {
-              if (t + 1 < cur.nt) issue_x(cur, r, t + 1);
-              else issue_x(ni, nrr, 0);
-            }
-            __syncwarp();
-            ++nx;
-          }
         }
       }
       cur = nxt;
@@ -355,7 +409,6 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
     if (lane == 0) {
       mbar_wait(bar_lo, (nlo - 1) & 1);
       mbar_wait(bar_hi + ((nhi - 1) & 1), ((nhi - 1) >> 1) & 1);
-      mbar_wait(bar_x, (nx - 1) & 1);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -368,12 +421,15 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
         const int r = kr(v);
         const int ks0 = r * RS, rs = min(RS, KS - ks0);
         const uint32_t sfw_c = tmem + L::COL_SFW + (g & 1) * L::SF_COLS;
-        if constexpr (!L::kSfwDec) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar_hi + (g & 1), (g >> 1) & 1));
+        if constexpr (!L::kQBS) {
+          // the round's weight scale atoms: direct ones as loaded (by round parity),
+          // PreScale+ ones once the decoders have built them from the scale indices
+          if constexpr (L::kSVQ) ok = __all_sync(0xffffffffu, mbar_wait(sf_ready, g & 1));
+          else ok = __all_sync(0xffffffffu, mbar_wait(bar_hi + (g & 1), (g >> 1) & 1));
           if (!ok) break;
           tc_fence_after();
           if (elect_one()) {
-            const uint32_t s0 = smem_u32(smem + L::AUX_OFF + (g & 1) * RS * A * 512);
+            const uint32_t s0 = smem_u32(smem + (L::kSVQ ? L::SFS_OFF : L::AUX_OFF + (g & 1) * RS * A * 512));
             for (int a = 0; a < rs * A; ++a) tc_cp_32x128b_warpx4(sfw_c + 4 * a, sdesc_sf_atom(s0 + a * 512));
           }
           __syncwarp();
@@ -483,7 +539,8 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
     int g = 0, di = 0;
     for (int k = k_first; k < n_items; k += k_step, ++di) {
       const RoundItem it = item(k, SWI);
-      const SvqGeom sv(p.w[it.e].ds, L::kB, KS);
+      SvqGeom sv(8, L::kB, KS);                      // the item's, once its first round has landed
+      [[maybe_unused]] float w_ts = 1.0f;            // the expert's weight tensor scale
       for (int v = 0; v < nrv; ++v, ++g) {
         const int r = kr(v);
         const int ks0 = r * RS, rs = min(RS, KS - ks0);
@@ -503,6 +560,11 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
           }
         }
         const bool landed = __all_sync(0xffffffffu, mbar_wait(bar_lo, g & 1));
+        if (v == 0) {                                // the item's slot (filled before this copy was requested)
+          const ItemSlot& sl = slots[di & 1];
+          sv = SvqGeom(sl.w.ds, L::kB, KS);
+          w_ts = sl.w.w_tscale;
+        }
         uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0, d0 = c0, d1 = c0;
         if (act && landed) {
           cb_words(ks0 + s_l, 0, qb0, &c0, &c1);
@@ -512,31 +574,36 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
         lay_out(act && landed, c0, c1);
         named_bar_sync(2, kDecThreads);              // this round's copies are complete
         // quarters 0-1 of the operand tiles: the last round's MMAs of them are done
+        // (and with them the tcgen05.cp of the last round's PreScale+ scale atoms)
         if (g > 0) mbar_wait(w_free, (g - 1) & 1);
-        // Weight scale atom a of this warp's stage into TMEM (PreScale+ from the scale
-        // codebook, PostScale-QB the QBlock's byte); row `lane` of the atom, column q,
-        // holds block scales 4a..4a+3 of weight row 32 q + lane.
-        auto sf_atom = [&](int a) {
-          if constexpr (L::kSfwDec) {
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if constexpr (L::kSVQ) {
-              if (landed) {
-                const int ks = ks0 + sf_s;
-                const uint8_t* un = smem + L::SIDX_OFF + ((ks >> sv.lspu) - (ks0 >> sv.lspu)) * 128 * sv.G;
-                const uint32_t* scb32 = reinterpret_cast<const uint32_t*>(smem + L::AUX_OFF);
-                const int kbk = sv.kb_base(ks, L::kB) + 4 * a;
-                v.x = svq_word(un + (0 * 32 + lane) * sv.G, scb32, sv.lds, kbk);
-                v.y = svq_word(un + (1 * 32 + lane) * sv.G, scb32, sv.lds, kbk);
-                v.z = svq_word(un + (2 * 32 + lane) * sv.G, scb32, sv.lds, kbk);
-                v.w = svq_word(un + (3 * 32 + lane) * sv.G, scb32, sv.lds, kbk);
-              }
-            } else {
-              const uint32_t b = ((qbs >> (8 * a)) & 0xFFu) * 0x01010101u;
-              v = make_uint4(b, b, b, b);
+        if constexpr (L::kSVQ) {
+          // PreScale+ (Table 4 caption: Ks = 256, ds = 8): the round's weight scale atoms
+          // in shared memory, each 128-row atom word looked up once from the scale
+          // indices and the scale codebook (one word per decoder thread and stage with
+          // E4M3-B16); the MMA warp copies them to TMEM with tcgen05.cp
+          if (landed) {
+            const uint32_t* scb32 = reinterpret_cast<const uint32_t*>(smem + L::AUX_OFF);
+            const int dt = dw * 32 + lane;
+            for (int s = 0; s < rs; ++s) {
+              const int ks = ks0 + s;
+              decode_sf_tile<A, kDecThreads>(smem + L::SIDX_OFF + ((ks >> sv.lspu) - (ks0 >> sv.lspu)) * 128 * sv.G,
+                                             sv.G, scb32, sv.lds, sv.kb_base(ks, L::kB), smem + L::SFS_OFF + s * A * 512,
+                                             dt);
             }
+          }
+          fence_proxy_async_smem();                  // atom writes -> tcgen05.cp reads
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sf_ready);
+        }
+        // PostScale-QB: weight scale atom a of this warp's stage into TMEM, the QBlock's
+        // byte; row `lane` of the atom, column q, holds block scales 4a..4a+3 of weight
+        // row 32 q + lane.
+        auto sf_atom = [&](int a) {
+          if constexpr (L::kQBS) {
+            const uint32_t b = ((qbs >> (8 * a)) & 0xFFu) * 0x01010101u;
             tmem_st_32x32b_x4(tmem + (static_cast<uint32_t>(qd * 32) << 16) + L::COL_SFW + (g & 1) * L::SF_COLS +
                                   4 * (sf_s * A + a),
-                              v);
+                              make_uint4(b, b, b, b));
           }
         };
         const uint8_t* idx_l = smem + L::IDX_OFF + s_l * 8192 + row_i * 16;
@@ -565,7 +632,7 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
               named_bar_sync(2, kDecThreads);
             }
           }
-          if constexpr (L::kSfwDec) {
+          if constexpr (L::kQBS) {
             if (h == 0) {
               __syncwarp();                          // tcgen05.st is warp-aligned
               if (sf_act) {
@@ -578,7 +645,7 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
             decode_quarter(2 * h);
             decode_quarter(2 * h + 1);
           }
-          if constexpr (L::kSfwDec) {
+          if constexpr (L::kQBS) {
             if (h == 0) {
               __syncwarp();
               tmem_st_wait();
@@ -598,7 +665,7 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
         // scale byte into the grouped SF layout); the tile's rows past the expert's
         // get zero scales.
         constexpr int B = L::kB;
-        const float scale = p.w[it.e].w_tscale * (p.a_tscale ? *p.a_tscale : 1.0f);
+        const float scale = w_ts * (p.a_tscale ? *p.a_tscale : 1.0f);
         const float hs = FMT == FMT_E4M3 ? *p.h_tscale : 1.0f;
         const int kbr = p.F / B;
         const int cg = dw >> 2;
@@ -644,7 +711,7 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
         if (lane == 0) mbar_arrive(acc_free);        // the next item's MMAs may overwrite
       }
     }
-  } else {
+  } else if (warp < kRoundTokWarp) {
     // ============================== epilogue ==============================
     // Warp 18 + q reads TMEM lane quadrant (18 + q) mod 4: tokens 32 ((18 + q) mod 4)
     // .. + 31 of each tile, each thread one token's 128 output channels of the band.
@@ -711,6 +778,53 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_free);          // the next item's MMAs may overwrite
     }
+  } else {
+    // ========================== token-tile loader ==========================
+    // The token operands and scales of each (round, tile) of this CTA's items, in the
+    // order the MMA warp consumes them, each once the MMAs that read the buffer's
+    // previous contents have completed.
+    struct XCopy {                                   // one tile's tokens and their scales for one round
+      const uint8_t* sf;
+      uint32_t tx;
+      int ks0, rs, tm0, boxes;
+    };
+    auto prepare_x = [&](const RoundItem& it, int v, int t) {    // tile t of round v
+      XCopy c;
+      c.ks0 = kr(v) * RS;
+      c.rs = min(RS, KS - c.ks0);
+      const int64_t tm0 = it.m0 + static_cast<int64_t>(t) * 128;
+      const int64_t rows = it.m_end - tm0 < 128 ? it.m_end - tm0 : 128;
+      c.tm0 = static_cast<int>(tm0);
+      c.boxes = static_cast<int>((rows + kMoeXBox - 1) / kMoeXBox);
+      c.sf = p.a_sf + (static_cast<size_t>(it.tile0 + t) * KB4 + static_cast<size_t>(c.ks0) * A) * 512;
+      c.tx = c.rs * c.boxes * kMoeXBox * 128 + c.rs * A * 512;
+      return c;
+    };
+    auto fire_x = [&](const XCopy& c) {
+      mbar_arrive_expect_tx(bar_x, c.tx);
+      for (int s = 0; s < c.rs; ++s)
+        for (int q = 0; q < c.boxes; ++q)
+          tma_load_2d(smem + L::X_OFF + s * 16384 + q * kMoeXBox * 128, &tmap_x, (c.ks0 + s) * 128,
+                      c.tm0 + q * kMoeXBox, bar_x);
+      bulk_load(smem + L::SFX_OFF, c.sf, c.rs * A * 512, bar_x);
+    };
+    int kx = 0;                                      // (round, tile) copies issued
+    bool ok = true;
+    for (int k = k_first; k < n_items && ok; k += k_step) {
+      const RoundItem it = item(k, true);
+      for (int v = 0; v < nrv && ok; ++v) {
+        for (int t = 0; t < it.nt && ok; ++t, ++kx) {
+          const XCopy xc = prepare_x(it, v, t);
+          if (kx > 0) ok = __all_sync(0xffffffffu, mbar_wait(xfree, (kx - 1) & 1));   // the buffer is free
+          if (!ok) break;
+          if (elect_one()) fire_x(xc);
+          __syncwarp();
+        }
+      }
+    }
+    // every copy requested lands before the CTA can retire
+    if (lane == 0 && kx > 0) mbar_wait(bar_x, (kx - 1) & 1);
+    __syncwarp();
   }
 
   __syncwarp();
