@@ -246,30 +246,36 @@ __global__ void __maxnreg__(64)
   // to L2 now and are copied in later.  (A plain L2 prefetch of the slice in address
   // order would complete quarter 0 -- spread over all stages -- only when nearly the
   // whole slice had arrived, and the decode could not overlap it.)
+  // Every weight byte is read once per launch: its copies are marked evict-first in
+  // L2 (wpol), so that the stream does not evict what each launch reuses -- the kernel
+  // code and parameters (whose first reads otherwise go to memory at every launch,
+  // ahead of the first copy), the activations and the output.
+  const uint64_t wpol = l2_policy_evict_first();
   auto issue_round = [&](int r) {
     const int rb = ks_begin + L::S * r, rn = rcount(r);
     if constexpr (L::kVQ) {
       const int qa = qb_first(r);
       const uint32_t cb_bytes = static_cast<uint32_t>(qb_last(r) - qa + 1) * 512;
       mbar_arrive_expect_tx(bar_cb, cb_bytes);
-      bulk_load(smem + L::CB_OFF, w_cb + static_cast<size_t>(qa) * 256, cb_bytes, bar_cb);
+      bulk_load_hint(smem + L::CB_OFF, w_cb + static_cast<size_t>(qa) * 256, cb_bytes, bar_cb, wpol);
       // quarter j of the round's stages: box {2048 B, 1, rbox stages, 1}; stages past
       // the round (and past K) arrive too, zero-filled past K, and are not used
       mbar_arrive_expect_tx(&full[0], rbox * 2048);
-      tma_load_4d(smem + L::IDX_OFF, &tmap_idx, 0, 0, rb, n_tile, &full[0]);
+      tma_load_4d_hint(smem + L::IDX_OFF, &tmap_idx, 0, 0, rb, n_tile, &full[0], wpol);
     }
     if constexpr (!L::kSVQ && !L::kQBS) {
       mbar_arrive_expect_tx(bar_sfw, rn * A * 512);
-      bulk_load(smem + L::SFW_OFF, w_sf + static_cast<size_t>(L::S * r) * A * 512, rn * A * 512, bar_sfw);
+      bulk_load_hint(smem + L::SFW_OFF, w_sf + static_cast<size_t>(L::S * r) * A * 512, rn * A * 512, bar_sfw, wpol);
     }
     if constexpr (L::kVQ) {
       mbar_arrive_expect_tx(&full[1], rbox * 2048);
-      tma_load_4d(smem + L::IDX_OFF + L::IDX_BUF, &tmap_idx, 0, 1, rb, n_tile, &full[1]);
-      for (int s = 0; s < rn; ++s) l2_prefetch_bulk(w_idx + static_cast<size_t>(L::S * r + s) * 8192 + 4096, 4096);
+      tma_load_4d_hint(smem + L::IDX_OFF + L::IDX_BUF, &tmap_idx, 0, 1, rb, n_tile, &full[1], wpol);
+      for (int s = 0; s < rn; ++s)
+        l2_prefetch_bulk_hint(w_idx + static_cast<size_t>(L::S * r + s) * 8192 + 4096, 4096, wpol);
     } else {
       for (int s = 0; s < rn; ++s) {
         mbar_arrive_expect_tx(&full[s], 16384);
-        tma_load_2d(smem + L::W_OFF + s * 16384, &tmap_wq, (rb + s) * 128, n_tile * 128, &full[s]);
+        tma_load_2d_hint(smem + L::W_OFF + s * 16384, &tmap_wq, (rb + s) * 128, n_tile * 128, &full[s], wpol);
       }
     }
     if constexpr (L::kSVQ) {                         // the round's scale indices (+ the scale codebook)
@@ -277,7 +283,7 @@ __global__ void __maxnreg__(64)
       const uint32_t sidx_bytes = static_cast<uint32_t>(u1 - u0 + 1) * 128 * sv.G;
       const uint32_t scb_bytes = r == 0 ? 256u * static_cast<uint32_t>(sv.ds) : 0u;
       mbar_arrive_expect_tx(bar_sfw, sidx_bytes + scb_bytes);
-      bulk_load(smem + L::SIDX_OFF, sv.unit(p.w.sidx, n_tile, rb), sidx_bytes, bar_sfw);
+      bulk_load_hint(smem + L::SIDX_OFF, sv.unit(p.w.sidx, n_tile, rb), sidx_bytes, bar_sfw, wpol);
       if (r == 0) bulk_load(smem + L::SCB_OFF, p.w.scb, scb_bytes, bar_sfw);
     }
   };
@@ -378,14 +384,15 @@ __global__ void __maxnreg__(64)
           for (int j = 2; j < 4; ++j) {              // K-quarter j of every stage (from L2 by now)
             if (!mbar_wait(&dec_ph[j - 2], ph)) break;   // its buffer has been decoded
             mbar_arrive_expect_tx(&full[j], rbox * 2048);
-            tma_load_4d(smem + L::IDX_OFF + (j % 2) * L::IDX_BUF, &tmap_idx, 0, j, rb, n_tile, &full[j]);
+            tma_load_4d_hint(smem + L::IDX_OFF + (j % 2) * L::IDX_BUF, &tmap_idx, 0, j, rb, n_tile, &full[j], wpol);
             issued_q = j + 1;
           }
           if (issued_q == 4 && r + 1 < rounds) {     // the next round's stream into L2 meanwhile
             const int nb = L::S * (r + 1), nn = rcount(r + 1);
-            l2_prefetch_bulk(w_idx + static_cast<size_t>(nb) * 8192, static_cast<uint32_t>(nn) * 8192);
+            l2_prefetch_bulk_hint(w_idx + static_cast<size_t>(nb) * 8192, static_cast<uint32_t>(nn) * 8192, wpol);
             if constexpr (!L::kSVQ && !L::kQBS)
-              l2_prefetch_bulk(w_sf + static_cast<size_t>(nb) * A * 512, static_cast<uint32_t>(nn) * A * 512);
+              l2_prefetch_bulk_hint(w_sf + static_cast<size_t>(nb) * A * 512, static_cast<uint32_t>(nn) * A * 512,
+                                    wpol);
             if constexpr (L::kSVQ) {
               const int nbs = ks_begin + nb;
               const int u0 = nbs >> sv.lspu, u1 = (nbs + nn - 1) >> sv.lspu;

@@ -261,6 +261,9 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
       uint32_t tx;
       int rs;
     };
+    // The expert weights are read once per (band, chunk) item: evict-first in L2, so
+    // that they do not push out the token tiles, which the bands of a chunk share.
+    const uint64_t wpol = l2_policy_evict_first();
     auto prepare_lo = [&](const RoundItem& it, int v, const ItemSlot& sl) {    // round v of item it
       const int r = kr(v), band = wband(it, v);
       const int ks0 = r * RS, rs = min(RS, KS - ks0);
@@ -288,8 +291,8 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
       }
       if (r == 0 && lane == 0) {                     // the band's later rounds on their way into L2
         for (int ks = RS; ks < KS; ks += 4)          // 32 KB a request
-          l2_prefetch_bulk(sl.w.idx + (static_cast<size_t>(band) * KS + ks) * 8192,
-                           static_cast<uint32_t>(min(4, KS - ks)) * 8192);
+          l2_prefetch_bulk_hint(sl.w.idx + (static_cast<size_t>(band) * KS + ks) * 8192,
+                                static_cast<uint32_t>(min(4, KS - ks)) * 8192, wpol);
         l2_prefetch_bulk(sl.w.cb + static_cast<size_t>(qbn) * cb_per_row * 256,
                          static_cast<uint32_t>(cb_per_row) * 512);
       }
@@ -297,7 +300,8 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
     };
     auto fire_lo = [&](const LoCopy& c) {
       mbar_arrive_expect_tx(bar_lo, c.tx);
-      for (int s = 0; s < c.rs; ++s) bulk_load(smem + L::IDX_OFF + s * 8192, c.idx + s * 8192, 4096, bar_lo);
+      for (int s = 0; s < c.rs; ++s)
+        bulk_load_hint(smem + L::IDX_OFF + s * 8192, c.idx + s * 8192, 4096, bar_lo, wpol);
       bulk_load(smem + L::CB_OFF, c.cb, c.cb_bytes, bar_lo);
       if constexpr (L::kSVQ) {
         bulk_load(smem + L::SIDX_OFF, c.sidx, c.sidx_bytes, bar_lo);
@@ -321,7 +325,8 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
     auto fire_hi = [&](const HiCopy& c, int g) {     // g: the global round number
       uint64_t* bar = bar_hi + (g & 1);
       mbar_arrive_expect_tx(bar, c.tx);
-      for (int s = 0; s < c.rs; ++s) bulk_load(smem + L::IDX_OFF + s * 8192 + 4096, c.idx + s * 8192, 4096, bar);
+      for (int s = 0; s < c.rs; ++s)
+        bulk_load_hint(smem + L::IDX_OFF + s * 8192 + 4096, c.idx + s * 8192, 4096, bar, wpol);
       if constexpr (WSRC == WSRC_VQ_DIRECT)
         bulk_load(smem + L::AUX_OFF + (g & 1) * RS * A * 512, c.sf, c.rs * A * 512, bar);
     };
@@ -329,7 +334,8 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
     // tiles, codebooks, scale indices and scale codebook, and its first token tile.
     auto prefetch_first_round = [&](const RoundItem& it, const ItemSlot& sl) {
       const int rs = min(RS, KS);
-      l2_prefetch_bulk(sl.w.idx + static_cast<size_t>(it.n_tile) * KS * 8192, static_cast<uint32_t>(rs) * 8192);
+      l2_prefetch_bulk_hint(sl.w.idx + static_cast<size_t>(it.n_tile) * KS * 8192, static_cast<uint32_t>(rs) * 8192,
+                            wpol);
       const int qb1 = qb_last(rs - 1);
       l2_prefetch_bulk(sl.w.cb + static_cast<size_t>(sl.qbn[0]) * cb_per_row * 256,
                        static_cast<uint32_t>(qb1 + 1) * 512);
