@@ -228,6 +228,18 @@ def run_reference(args, rank, world):
 # Multi-rank arithmetic (host side; covered by CPU tests over gloo)
 # ---------------------------------------------------------------------------
 
+def measured_traffic(key: str):
+    """dram__bytes_read.sum + dram__bytes_write.sum of one launch of a kernel, from the
+    ncu capture recorded in profiles/traffic.txt under `key`, or None."""
+    prof = os.path.join(ROOT, "profiles", "traffic.txt")
+    if os.path.exists(prof):
+        for line in open(prof):
+            parts = line.split()
+            if len(parts) == 2 and parts[0] == key:
+                return int(parts[1])
+    return None
+
+
 def max_over_ranks(x: float, dist=None, device="cpu") -> float:
     """The largest value over all ranks of the process group (the slowest rank's
     time); x itself without one.  Every rank must call it at the same point."""
@@ -452,13 +464,7 @@ def run_gpu(args, rank, world, dist):
     # our kernels per step: the activation quantizer (one launch up to 16 x 8192
     # elements, else tensor amax + quantize) and the linear layer
     launches_per_step = (1 if M * w.K <= 16 * 8192 else 2) + 1
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "traffic.txt")   # ncu dram read+write of one launch
-    if os.path.exists(prof):
-        for line in open(prof):
-            parts = line.split()
-            if len(parts) == 2 and parts[0] == "decode_gemv_m16_bytes_per_launch":
-                traffic = int(parts[1])
+    traffic = measured_traffic("decode_gemv_m16_bytes_per_launch")
     out = {
         "metric": "MXCode W4A4 effective weight bandwidth (compressed bytes/s)",
         "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": warmup,
@@ -643,7 +649,8 @@ def moe_leg(dev, stream, capture, time_graph, steps, world, with_cpu):
                                   "kernel": "moe_round_kernel<E4M3, VQ scale-VQ> (persistent) + group prologue",
                                   "target_ms": max(t_bw, t_fl), "frac": max(t_bw, t_fl) / ms_lin,
                                   "hbm_peak_GBps": hbm, "hbm_kind": hbm_kind,
-                                  "fp4_peak_TFLOPs": peak, "fp4_kind": peak_kind, "traffic": None}}
+                                  "fp4_peak_TFLOPs": peak, "fp4_kind": peak_kind,
+                                  "traffic": measured_traffic(f"moe_{name}_bytes_per_launch")}}
     # The MoE FFN with SwiGLU fused into the gate/up epilogue, which writes the down
     # projection's FP4 activation directly: grouped quantization -> gate/up + SwiGLU
     # -> down.  h's E4M3 tensor scale is calibrated once from a torch evaluation of
