@@ -202,7 +202,13 @@ mxc_status mxc_pack_weight(const mxc_weight_host* w, uint8_t* idx_out, uint8_t* 
  * most 16) whose slices are at most 2048 input channels long, provided
  * N/128 x R <= 148 (one CTA per SM) and N/128 <= 1024; else 0.  Without that room
  * the call runs on split-K clusters (slower for those shapes), not an error.  17
- * to 128 rows: 0.  Above 128 rows when N is a multiple of 256 (else from 1024
+ * to 128 rows (128-token tiles of the fused kernel), when N/128 <= 1024 and the
+ * 128-row output tiles can be split along K into R = min(4, 148 / (N/128), K/256)
+ * >= 2 ranks (R recomputed as the number of slices of ceil(K/256 / R) stages): the
+ * counters, then N/128 x R x 64 KiB of FP32 partial tiles; else 0.  Without that
+ * room the call runs one CTA per output tile (slower), not an error.  The
+ * partials are added in rank order, so a result depends on the room given, not on
+ * timing.  Above 128 rows when N is a multiple of 256 (else from 1024
  * rows): the counters, then the room for the weight decoded once per call (N*K/2
  * bytes of FP4 codes rounded up to 1 KiB, then N*K/B bytes of SF-layout scales).
  * A smaller workspace is not an error there: the call then runs the fused
@@ -266,7 +272,8 @@ mxc_status mxc_quantize_act_grouped(const void* x_bf16, int64_t M, int64_t K, in
  * y         device, [M, ldy] elements of y_dtype (ldy >= N)
  * ws        device workspace of mxc_linear_workspace_bytes() bytes (16-byte aligned)
  * M <= 16 takes the split-K decode path; larger M the tiled prefill path, which
- * decodes each weight tile inside the GEMM.  Above 128 rows when N is a multiple
+ * decodes each weight tile inside the GEMM (17 to 128 rows: split along K through
+ * the workspace when it has the room, see mxc_linear_workspace_bytes).  Above 128 rows when N is a multiple
  * of 256 (else from 1024 rows), with the workspace given, the call instead decodes
  * the weight once into it (MX-native FP4 codes and scales, the output of
  * mxc_decode_weight) and runs the native block-scaled GEMM on that: the same

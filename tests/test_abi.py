@@ -150,7 +150,8 @@ def test_workspace_sizes(L):
     assert L.mxc_linear_workspace_bytes(4096, 9216, 4096, 1) == C + 9216 * 4096 // 2 + 9216 * 4096 // 16
     assert L.mxc_linear_workspace_bytes(1024, 9216, 4096, 0) == C + 9216 * 4096 // 2 + 9216 * 4096 // 32
     assert L.mxc_linear_workspace_bytes(129, 9216, 4096, 1) == C + 9216 * 4096 // 2 + 9216 * 4096 // 16
-    assert L.mxc_linear_workspace_bytes(128, 9216, 4096, 1) == 0           # fused tiles: none
+    # 17..128 tokens (fused 128-token tiles): split-K partials [tile][rank][128][128] FP32
+    assert L.mxc_linear_workspace_bytes(128, 9216, 4096, 1) == C + 72 * 2 * 128 * 128 * 4   # 72 tiles x 2 ranks
     assert L.mxc_linear_workspace_bytes(1023, 9344, 4096, 1) == 0          # N % 256 != 0: fused below 1024
     assert L.mxc_linear_workspace_bytes(1024, 9344, 4096, 1) == C + 9344 * 4096 // 2 + 9344 * 4096 // 16
     assert L.mxc_linear_workspace_bytes(16, 9216, 4096, 1) == 0            # decode: split-K in cluster SMEM
@@ -162,7 +163,7 @@ def test_workspace_sizes(L):
     assert L.mxc_linear_workspace_bytes(16, 128, 32768, 1) == C + 1 * 16 * 8192       # 16 ranks
     assert L.mxc_linear_workspace_bytes(16, 8192, 8192, 1) == 0            # 64 x 4 CTAs: two waves
     assert L.mxc_linear_workspace_bytes(16, 18432, 4096, 1) == 0           # 144 x 2 CTAs: two waves
-    assert L.mxc_linear_workspace_bytes(17, 4608, 8192, 1) == 0            # tiled path: none
+    assert L.mxc_linear_workspace_bytes(17, 4608, 8192, 1) == C + 36 * 4 * 128 * 128 * 4   # 36 tiles x 4 ranks
     assert L.mxc_linear_workspace_bytes(16, 128, 65536, 1) == 0            # 32 ranks: past the limit
     assert L.mxc_moe_workspace_bytes(16384, 128, 3072, 4096, 1) >= 129 * 4
     assert L.mxc_grouped_sf_rows_bound(16384, 128) == 16384 + 128 * 128

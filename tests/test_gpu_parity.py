@@ -257,6 +257,31 @@ def test_mxcode_equals_native_on_decoded_weights(fmt, M, strat):
 
 
 @pytest.mark.parametrize("fmt", ["e8m0_b32", "e4m3_b16"])
+@pytest.mark.parametrize("M", [17, 77, 128])
+@pytest.mark.parametrize("strat", ["prescale_plus", "postscale"])
+def test_mid_m_split_k_through_the_workspace(fmt, M, strat):
+    """17..128 tokens run the fused kernel on 128-token tiles; with the workspace given,
+    each tile's K is split over CTAs (N = 512: 4 tiles x 4 ranks of 2 stages) whose
+    scaled partials the last rank adds in rank order.  Checked against the oracle with
+    FP32 and BF16 output, ragged token tiles included; MXCode and native FP4 on the same
+    decoded operands take the same split and agree bit for bit; without a workspace the
+    one-CTA-per-tile path runs and agrees within the bound."""
+    w = synth.make_weight(71, fmt, strat, 512, 2048, 256, 256)
+    x = synth.make_activations(71, M, 2048, outliers=True)
+    assert mxc.lib().mxc_linear_workspace_bytes(M, 512, 2048, 1) == 4096 + 4 * 4 * 128 * 128 * 4
+    y, pw, a = run_mxcode(w, x)
+    ref, sabs = O.w4a4_linear(x, w)
+    assert_close(y.cpu().numpy(), ref, sabs, what=f"split {strat} {fmt} M={M}")
+    yb = mxc.linear(a, pw, torch.bfloat16)
+    assert torch.equal(yb, y.to(torch.bfloat16))                  # BF16 = RNE of the same FP32 sum
+    wn = mxc.decode_weight(pw)
+    assert torch.equal(mxc.native_linear(a, wn), y)
+    y1 = mxc.linear(a, pw, ws=torch.zeros(16, dtype=torch.uint8, device="cuda"))   # no room: no split
+    assert mxc.get_device_error() == 0
+    assert_close(y1.cpu().numpy(), ref, sabs, what=f"no split {strat} {fmt} M={M}")
+
+
+@pytest.mark.parametrize("fmt", ["e8m0_b32", "e4m3_b16"])
 @pytest.mark.parametrize("M,K", [(129, 256), (300, 1536), (700, 1024), (1000, 4096)])
 @pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
 def test_pair_gemm_equals_one_cta(fmt, M, K, out):

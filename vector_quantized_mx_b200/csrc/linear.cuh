@@ -248,11 +248,33 @@ inline bool gemv_ws_split(int64_t N, int64_t K, int* splits, int* ks_per_split) 
   *ks_per_split = per;
   return true;
 }
+// Split-K of the fused kernel's 128-token tiles (17 to 128 tokens) through the
+// workspace: with one CTA per 128-row output tile the grid would leave most SMs idle
+// (K = N = 8192: 64 of 148), so each tile's K runs in `splits` slices on separate
+// CTAs (as many as fill one wave, at most 4); each writes its scaled partial tile,
+// [tile][rank][128 tokens][128] FP32 after the counter area, and the tile's last rank
+// to arrive adds them in rank order.
+constexpr int kMidMaxSplits = 4;
+inline bool mid_split(int64_t M, int64_t N, int64_t K, int* splits, int* ks_per_split) {
+  if (M <= kDecodeMaxM || M > 128) return false;
+  const int n_tiles = static_cast<int>(N / kTileN);
+  const int KS = static_cast<int>(K / kStageK);
+  if (n_tiles <= 0 || n_tiles > static_cast<int>(kSplitkCtrBytes / 4)) return false;
+  int s = kSMs / n_tiles;
+  s = s > kMidMaxSplits ? kMidMaxSplits : s;
+  s = s > KS ? KS : s;
+  if (s < 2) return false;
+  const int per = (KS + s - 1) / s;
+  *splits = (KS + per - 1) / per;
+  *ks_per_split = per;
+  return *splits >= 2;
+}
 // the partial tiles' bytes (0 when the shape does not reduce through the workspace)
 inline size_t splitk_part_bytes(int64_t M, int64_t N, int64_t K) {
   int s, per;
-  if (M > kDecodeMaxM || !gemv_ws_split(N, K, &s, &per)) return 0;
-  return static_cast<size_t>(N / kTileN) * s * 128 * kGemvT * 4;
+  if (M <= kDecodeMaxM)
+    return gemv_ws_split(N, K, &s, &per) ? static_cast<size_t>(N / kTileN) * s * 128 * kGemvT * 4 : 0;
+  return mid_split(M, N, K, &s, &per) ? static_cast<size_t>(N / kTileN) * s * 128 * 128 * 4 : 0;
 }
 
 // Decode once: the layer decodes its weight once per call into the workspace (native
@@ -313,7 +335,7 @@ cudaError_t launch_gemm_ncb(const CUtensorMap& tx, const CUtensorMap& tw, const 
   cfg.dynamicSmemBytes = L::SMEM;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  if (p.splits > 1) {                       // the split CTAs of a tile are one cluster
+  if (p.splits > 1 && p.red_part == nullptr) {   // the split CTAs of a tile are one cluster
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 1;
     attr[0].val.clusterDim.y = 1;
@@ -570,6 +592,17 @@ mxc_status run_linear(const LinearArgs& a, cudaStream_t stream) {
       const cudaError_t err = a.fmt == FMT_E8M0 ? dispatch_gemv<FMT_E8M0>(a.wsrc, tx3, tw, ti, g, grid, stream)
                                                 : dispatch_gemv<FMT_E4M3>(a.wsrc, tx3, tw, ti, g, grid, stream);
       return err == cudaSuccess ? MXC_OK : MXC_ERR_CUDA;
+    }
+  }
+  if (T == 128) {
+    int splits, per;
+    if (mid_split(a.M, a.N, a.K, &splits, &per) && a.ws &&
+        a.ws_bytes >= kSplitkCtrBytes + a.ws_used + splitk_part_bytes(a.M, a.N, a.K) &&
+        reinterpret_cast<uintptr_t>(a.ws) % 16 == 0) {
+      p.splits = splits;
+      p.ks_per_split = per;
+      p.red_ctr = static_cast<unsigned int*>(a.ws);
+      p.red_part = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) + kSplitkCtrBytes + a.ws_used);
     }
   }
   const dim3 grid(n_tiles, m_tiles, p.splits);

@@ -68,7 +68,10 @@ struct GemmParams {
   void* y;
   int64_t ldy;
   int out_bf16;
-  int splits, ks_per_split;  // split-K over a cluster of `splits` CTAs (1 = off)
+  int splits, ks_per_split;  // split-K over a cluster of `splits` CTAs (1 = off), or through the workspace
+  float* red_part;           // 128-token tiles, split-K through the workspace: [tile][rank][T][128] scaled
+                             // partials, or null
+  unsigned int* red_ctr;     // and one arrival counter per output tile (zero on entry, zero again at exit)
   ExpertPtrs w[NEXP];
 };
 
@@ -592,6 +595,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     } else {
+      // Split-K of a 128-token tile through the workspace: this rank's scaled partial,
+      // token-major [T][128] FP32 (a warp's stores are coalesced); the rank of the tile
+      // that arrives last at its counter adds the partials in rank order (products and
+      // sums rounded separately).
+      const size_t tile = static_cast<size_t>(blockIdx.y) * gridDim.x + n_tile;
+      float* const part = p.red_part ? p.red_part + tile * splits * (static_cast<size_t>(T) * 128) : nullptr;
 #pragma unroll 1
       for (int c0 = 0; c0 < TCOL; c0 += 32) {
         uint32_t v[32];
@@ -599,12 +608,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_32x32b_x32(taddr + c0, v);
         tmem_ld_wait();
         if (!ep_ok) continue;
+        if (part) {
+          float* const dst =
+              part + static_cast<size_t>(split) * (T * 128) + static_cast<size_t>(chalf * TCOL + c0) * 128 + row;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) __stcg(dst + c * 128, __fmul_rn(__uint_as_float(v[c]), scale));
+          continue;
+        }
         const int64_t rem = m_end - (mbase + c0);
         if (rem <= 0) continue;
         const int cmax = rem < 32 ? static_cast<int>(rem) : 32;
 #pragma unroll
         for (int c = 0; c < 32; ++c)
           if (c < cmax) store_out(y, ldy, out_bf16, mbase + c0 + c, n, __uint_as_float(v[c]) * scale);
+      }
+      if (part) {
+        __threadfence();                             // the partial is visible before the ticket
+        named_bar_sync(4, kDecThreads);
+        uint32_t* const last = tmem_slot + 1;
+        if (threadIdx.x == 64)                       // every rank arrives once, also after a failed wait
+          *last = atomicInc(p.red_ctr + tile, static_cast<unsigned>(splits - 1)) == static_cast<unsigned>(splits - 1);
+        named_bar_sync(4, kDecThreads);
+        if (*last) {
+          __threadfence();                           // the other ranks' partials are visible
+          const float* const src = part + static_cast<size_t>(chalf * TCOL) * 128 + row;
+#pragma unroll 1
+          for (int c0 = 0; c0 < TCOL; c0 += 32) {
+            // one rank's 32 values at a time, all loads in flight together
+            float sum[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) sum[c] = __ldcg(src + (c0 + c) * 128);
+            for (int r = 1; r < splits; ++r) {
+              float t[32];
+#pragma unroll
+              for (int c = 0; c < 32; ++c) t[c] = __ldcg(src + static_cast<size_t>(r) * (T * 128) + (c0 + c) * 128);
+#pragma unroll
+              for (int c = 0; c < 32; ++c) sum[c] = __fadd_rn(sum[c], t[c]);
+            }
+            if (!ep_ok) continue;
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (mbase + c0 + c < m_end) store_out(y, ldy, out_bf16, mbase + c0 + c, n, sum[c]);
+          }
+        }
       }
     }
   }
