@@ -565,7 +565,8 @@ def prefill_leg(dev, stream, capture, time_graph, steps, world, with_cpu):
                         "ms_per_launch": ms["native_linear"], "flops_per_launch": flops,
                         "achieved": flops / (ms["native_linear"] * 1e-3) / 1e12,
                         "frac": flops / (ms["native_linear"] * 1e-3) / 1e12 / peak,
-                        "layer_frac": flops / (ms["linear"] * 1e-3) / 1e12 / peak, "traffic": None},
+                        "layer_frac": flops / (ms["linear"] * 1e-3) / 1e12 / peak,
+                        "traffic": measured_traffic("prefill_pair_gemm_bytes_per_launch")},
            "native_fp4": {"ms_linear": ms["native_linear"], "ms_per_step": ms["native_step"],
                           "mxcode_speedup": ms["native_linear"] / ms["linear"],
                           "mxcode_step_speedup": ms["native_step"] / ms["step"],

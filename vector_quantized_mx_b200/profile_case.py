@@ -4,7 +4,7 @@
 
 decode          mxc_linear, PostScale E4M3-B16, M=16, K=4096, N=9216 (split-K decode path)
 decode_native   mxc_native_linear on the same decoded weights
-prefill         mxc_linear, PreScale E8M0-B32, M=2048, K=4096, N=9216 (BF16 out)
+prefill         mxc_linear, PreScale E8M0-B32, M=2048 (--rows), K=4096, N=9216 (BF16 out)
 prefill_native  mxc_native_linear on the same decoded weights
 moe             mxc_moe_linear, PreScale+ E4M3-B16, gate/up 3072x4096, 128 experts, Zipf(1.1) top-8
 swiglu          mxc_moe_gate_up_swiglu on the same gate/up weights and rows
@@ -30,6 +30,7 @@ def main(argv=None):
     ap.add_argument("case", choices=["decode", "decode_native", "decode_long", "prefill", "prefill_native", "moe",
                                      "swiglu", "quant"])
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--rows", type=int, default=2048, help="prefill cases: activation rows (at most 8192)")
     args = ap.parse_args(argv)
     build.build()
     dev = torch.device("cuda", 0)
@@ -51,7 +52,7 @@ def main(argv=None):
     elif args.case.startswith("prefill"):
         w, x = synth.config3()
         pw = mxc.pack_weight(w, dev)
-        a = mxc.quantize_act(_dev_bf16(x[:2048], dev), w.fmt)
+        a = mxc.quantize_act(_dev_bf16(x[:args.rows], dev), w.fmt)
         nat = mxc.decode_weight(pw) if args.case == "prefill_native" else None
         for _ in range(args.reps):
             if nat is None:
