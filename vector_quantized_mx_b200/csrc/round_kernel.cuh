@@ -587,15 +587,27 @@ __global__ void __launch_bounds__(kRoundThreads, 1)
           // in shared memory, each 128-row atom word looked up once from the scale
           // indices and the scale codebook (one word per decoder thread and stage with
           // E4M3-B16); the MMA warp copies them to TMEM with tcgen05.cp
-          if (landed) {
+          // Thread dt owns word dt of the A atoms of every stage (atom dt / 128, word
+          // dt mod 128 = row (w / 4) + 32 (w mod 4): the SF atom layout); the lookups of
+          // all stages are issued before any is stored, so that their shared-memory
+          // latencies overlap (one stage after the other they took ~1,500 SM clocks).
+          static_assert(128 * A <= kDecThreads, "one atom word per decoder thread and stage");
+          const int dt = dw * 32 + lane;
+          if (landed && dt < 128 * A) {
             const uint32_t* scb32 = reinterpret_cast<const uint32_t*>(smem + L::AUX_OFF);
-            const int dt = dw * 32 + lane;
-            for (int s = 0; s < rs; ++s) {
+            const int word = dt & 127, a = dt >> 7;
+            const int r = (word >> 2) + 32 * (word & 3);
+            uint32_t wv[RS];
+#pragma unroll
+            for (int s = 0; s < RS; ++s) {
               const int ks = ks0 + s;
-              decode_sf_tile<A, kDecThreads>(smem + L::SIDX_OFF + ((ks >> sv.lspu) - (ks0 >> sv.lspu)) * 128 * sv.G,
-                                             sv.G, scb32, sv.lds, sv.kb_base(ks, L::kB), smem + L::SFS_OFF + s * A * 512,
-                                             dt);
+              if (s < rs)
+                wv[s] = svq_word(smem + L::SIDX_OFF + ((ks >> sv.lspu) - (ks0 >> sv.lspu)) * 128 * sv.G + r * sv.G, scb32,
+                                 sv.lds, sv.kb_base(ks, L::kB) + 4 * a);
             }
+#pragma unroll
+            for (int s = 0; s < RS; ++s)
+              if (s < rs) reinterpret_cast<uint32_t*>(smem + L::SFS_OFF + (s * A + a) * 512)[word] = wv[s];
           }
           fence_proxy_async_smem();                  // atom writes -> tcgen05.cp reads
           __syncwarp();
