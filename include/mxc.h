@@ -339,9 +339,10 @@ mxc_status mxc_moe_gate_up_swiglu(const mxc_mx_tensor* a, const int32_t* d_offse
                                   int32_t E, const float* h_tscale_in, uint8_t* h_q, int64_t ldh, uint8_t* h_sf,
                                   void* ws, size_t ws_bytes, mxc_stream_t stream);
 
-/* mxc_moe_linear for callers that cannot allocate device memory: code that
- * runs inside a CUDA stream capture, plugin hosts and real-time serving loops
- * that forbid allocator calls, or C callers with no device allocator at hand.
+/* mxc_moe_linear for callers that cannot allocate device memory: plugins whose
+ * host owns all device memory and hands out none, real-time serving loops that
+ * forbid allocator calls (an allocation may block or synchronize the device
+ * mid-step), or C callers with no device allocator at hand.
  * The paper has no counterpart to this entry point; it exists for the calling
  * environment only.  It takes the same arguments as mxc_moe_linear minus the
  * workspace, checks them in the same order with the same statuses, and runs

@@ -1,6 +1,7 @@
 """mxc_moe_linear_noalloc: the grouped-expert layer for callers that cannot allocate
-device memory (stream-capture regions, plugin hosts and serving loops that forbid
-allocator calls).  It must give the same result as mxc_moe_linear, which takes a
+device memory (plugins whose host owns all device memory, real-time serving loops
+that forbid allocator calls because an allocation may block or synchronize mid-step,
+C callers without a device allocator).  It must give the same result as mxc_moe_linear, which takes a
 caller workspace, on consecutive calls that reuse the library's fixed scratch
 array.  This file runs last so that a failure here never hides the others.
 """
