@@ -581,7 +581,7 @@ def test_small_qblock_decode_bitexact(case):
 
 
 @pytest.mark.parametrize("case", SMALL_QB[:4], ids=lambda c: "-".join(map(str, c)))
-@pytest.mark.parametrize("M", [1, 16, 130])
+@pytest.mark.parametrize("M", [1, 16, 77, 130])
 def test_small_qblock_linear(case, M):
     fmt, strat, qn, qk = case
     w = synth.make_weight(112, fmt, strat, 512, 1024, qn, qk)
